@@ -1,0 +1,118 @@
+"""CPU oracle for the 2-D convolution forward pass -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The CUDA library and its Python binding
+never import it; the two share no code.
+
+The arithmetic lives in ``conv2d_oracle.c`` (fp64, six nested loops with
+bounds-checked zero padding, after the "手撕 Conv2D" page (lpnh.cn/news/2493075)
+§1.1-§2.1).  This module compiles that file with gcc (no -ffast-math, so IEEE
+double arithmetic is kept) and exposes it through ctypes.  Inputs are widened
+to float64 before the call; widening bf16- or fp32-valued data is exact.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+SOURCE = os.path.join(_HERE, "conv2d_oracle.c")
+LIBRARY = os.path.join(_HERE, "liboracle.so")
+
+_lib = None
+
+
+def build(source: str = SOURCE, output: str = LIBRARY, extra_flags=()) -> str:
+    """Compile ``source`` into the shared library ``output`` and return its path."""
+    cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", *extra_flags,
+           "-o", output, source]
+    subprocess.run(cmd, check=True)
+    return output
+
+
+def load(path: str | None = None):
+    """Load (building first if needed) the oracle library; returns a ctypes handle."""
+    global _lib
+    if path is not None:
+        return _bind(ctypes.CDLL(path))
+    if _lib is None:
+        if (not os.path.exists(LIBRARY)
+                or os.path.getmtime(LIBRARY) < os.path.getmtime(SOURCE)):
+            build()
+        _lib = _bind(ctypes.CDLL(LIBRARY))
+    return _lib
+
+
+def _bind(lib):
+    L = ctypes.c_long
+    P = ctypes.c_void_p
+    lib.oracle_conv2d_out_size.argtypes = [L, L, L, L, L, ctypes.POINTER(L)]
+    lib.oracle_conv2d_out_size.restype = ctypes.c_int
+    lib.oracle_conv2d_nchw.argtypes = [P, P, P, P] + [L] * 11
+    lib.oracle_conv2d_nchw.restype = ctypes.c_int
+    lib.oracle_conv2d_points.argtypes = [P, P, P] + [L] * 11 + [P, L, P]
+    lib.oracle_conv2d_points.restype = ctypes.c_int
+    lib.oracle_num_threads.argtypes = []
+    lib.oracle_num_threads.restype = ctypes.c_int
+    return lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _f64(a):
+    return None if a is None else np.ascontiguousarray(a, dtype=np.float64)
+
+
+def out_size(size, k, stride=1, pad=0, dilation=1, lib=None):
+    """Output extent along one dimension; raises ValueError when it is below 1."""
+    lib = lib or load()
+    out = ctypes.c_long(0)
+    if lib.oracle_conv2d_out_size(size, k, stride, pad, dilation, ctypes.byref(out)) != 0:
+        raise ValueError(f"no valid output for in={size} k={k} s={stride} p={pad} d={dilation}")
+    return out.value
+
+
+def conv2d(x, w, bias=None, stride=1, pad=0, dilation=1, groups=1, lib=None):
+    """y = conv2d(x, w, bias) in float64; x NCHW, w OIHW (C_out, C_in/groups, Kh, Kw)."""
+    lib = lib or load()
+    x, w, bias = _f64(x), _f64(w), _f64(bias)
+    N, C_in, H, W = x.shape
+    C_out, cin_g, Kh, Kw = w.shape
+    if cin_g * groups != C_in:
+        raise ValueError("weight shape does not match C_in / groups")
+    if bias is not None and bias.shape != (C_out,):
+        raise ValueError("bias must have shape (C_out,)")
+    Ho = out_size(H, Kh, stride, pad, dilation, lib)
+    Wo = out_size(W, Kw, stride, pad, dilation, lib)
+    y = np.empty((N, C_out, Ho, Wo), dtype=np.float64)
+    rc = lib.oracle_conv2d_nchw(_ptr(x), _ptr(w), _ptr(bias), _ptr(y), N, C_in, H, W,
+                                C_out, Kh, Kw, stride, pad, dilation, groups)
+    if rc != 0:
+        raise ValueError("oracle rejected the shape")
+    return y
+
+
+def conv2d_points(x, w, bias, idx, stride=1, pad=0, dilation=1, groups=1, lib=None):
+    """Selected outputs y[n, oc, oh, ow] for the rows (n, oc, oh, ow) of ``idx``."""
+    lib = lib or load()
+    x, w, bias = _f64(x), _f64(w), _f64(bias)
+    idx = np.ascontiguousarray(idx, dtype=np.int64).reshape(-1, 4)
+    N, C_in, H, W = x.shape
+    C_out, _, Kh, Kw = w.shape
+    out = np.empty(idx.shape[0], dtype=np.float64)
+    rc = lib.oracle_conv2d_points(_ptr(x), _ptr(w), _ptr(bias), N, C_in, H, W, C_out,
+                                  Kh, Kw, stride, pad, dilation, groups, _ptr(idx),
+                                  idx.shape[0], _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle rejected the shape or an index")
+    return out
+
+
+def num_threads(lib=None) -> int:
+    """OpenMP threads the oracle's loops use."""
+    return int((lib or load()).oracle_num_threads())
