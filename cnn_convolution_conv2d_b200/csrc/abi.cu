@@ -1,0 +1,582 @@
+// abi.cu -- the C ABI declared in include/conv2d_b200.h: argument validation, the
+// per-problem plan (tile shapes, pipeline depth, split of the reduction, scratch
+// layout), tensor-map encoding and kernel dispatch.  Host code only; every step of
+// the convolution itself runs in the kernels of igemm.cu and layout.cu.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <atomic>
+#include <mutex>
+#include <string>
+
+#include "common.cuh"
+#include "conv2d_b200.h"
+
+namespace conv2d_b200 {
+namespace {
+
+// ------------------------------------------------------------ error state ---
+thread_local std::string t_last_error;
+
+int fail(int status, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    t_last_error = buf;
+    return status;
+}
+
+int ok() {
+    t_last_error.clear();
+    return CONV_OK;
+}
+
+// Watchdog status word written by device code when a bounded wait runs out.
+__device__ int g_device_status;
+
+constexpr int kMaxDevices = 64;
+constexpr size_t kSmemBudget = 227 * 1024;
+constexpr long long kDefaultTimeoutNs = 2000000000LL;
+
+struct DeviceInfo {
+    bool ready = false;
+    int sms = 0;
+    int *status = nullptr;
+};
+DeviceInfo g_devices[kMaxDevices];
+std::mutex g_mutex;
+long long g_timeout_ns = kDefaultTimeoutNs;
+int g_starve = 0;
+cudaEvent_t g_main_start = nullptr, g_main_stop = nullptr;
+std::atomic<unsigned long long> g_launches{0};
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+using EncodeIm2colFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                    const cuuint64_t *, const cuuint64_t *, const int *,
+                                    const int *, cuuint32_t, cuuint32_t, const cuuint32_t *,
+                                    CUtensorMapInterleave, CUtensorMapSwizzle,
+                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode_tiled = nullptr;
+EncodeIm2colFn g_encode_im2col = nullptr;
+
+// Looks up the current device's SM count and status word, and the driver's
+// tensor-map encoders, once.
+int device_info(DeviceInfo **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(CONV_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= kMaxDevices) return fail(CONV_ERR_UNSUPPORTED, "device index %d", dev);
+    std::lock_guard<std::mutex> lock(g_mutex);
+    DeviceInfo &d = g_devices[dev];
+    if (!d.ready) {
+        int major = 0, minor = 0;
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+        if (major != 10 || minor != 0)
+            return fail(CONV_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a",
+                        dev, major, minor);
+        e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return fail(CONV_ERR_CUDA, "SM count: %s", cudaGetErrorString(e));
+        e = cudaGetSymbolAddress(reinterpret_cast<void **>(&d.status), g_device_status);
+        if (e != cudaSuccess)
+            return fail(CONV_ERR_CUDA, "status word address: %s", cudaGetErrorString(e));
+        if (!g_encode_tiled || !g_encode_im2col) {
+            cudaDriverEntryPointQueryResult q1, q2;
+            void *f1 = nullptr, *f2 = nullptr;
+            e = cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f1, 12000,
+                                                 cudaEnableDefault, &q1);
+            if (e != cudaSuccess || q1 != cudaDriverEntryPointSuccess || !f1)
+                return fail(CONV_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+            e = cudaGetDriverEntryPointByVersion("cuTensorMapEncodeIm2col", &f2, 12000,
+                                                 cudaEnableDefault, &q2);
+            if (e != cudaSuccess || q2 != cudaDriverEntryPointSuccess || !f2)
+                return fail(CONV_ERR_CUDA, "cuTensorMapEncodeIm2col entry point unavailable");
+            g_encode_tiled = reinterpret_cast<EncodeTiledFn>(f1);
+            g_encode_im2col = reinterpret_cast<EncodeIm2colFn>(f2);
+        }
+        d.ready = true;
+    }
+    *out = &d;
+    return CONV_OK;
+}
+
+// ------------------------------------------------------------------- plan ---
+struct Plan {
+    int N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups;
+    bool f32;
+    int elt;
+    conv_layout_t layout;
+    int Ho, Wo;
+    long long M;
+    int Cin_g, Cout_g, Cpg;
+    bool xcopy;     // x goes through the channels-last padding kernel first
+    int cb;         // bytes of channels per plane row (16, 32, 64 or 128)
+    int BN, taps, nCB, planes, kstages, Kp;
+    int n_mtiles, n_ntiles, splits, units, stages;
+    size_t smem;
+    size_t off_xcopy, off_partial, off_xcol, ws_total;
+};
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+int round_up(int v, int a) { return (v + a - 1) / a * a; }
+
+int out_size(int in, int k, int s, int p, int d, int *out) {
+    const long long numer = static_cast<long long>(in) + 2LL * p - static_cast<long long>(d) * (k - 1) - 1;
+    if (numer < 0) return -1;
+    *out = static_cast<int>(numer / s + 1);
+    return 0;
+}
+
+// Validates a problem and fills the plan.  `explicit_im2col` adds the X_col
+// buffer to the scratch layout.  `sms` = 0 plans without split (size queries
+// made before a device is known use the device's count when one is current).
+int make_plan(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stride, int pad,
+              int dilation, int groups, conv_dtype_t dtype, conv_layout_t layout,
+              bool explicit_im2col, int sms, Plan *P) {
+    if (N < 1 || C_in < 1 || H < 1 || W < 1 || C_out < 1 || Kh < 1 || Kw < 1)
+        return fail(CONV_ERR_INVALID_ARG, "sizes must be >= 1 (N=%d C_in=%d H=%d W=%d C_out=%d Kh=%d Kw=%d)",
+                    N, C_in, H, W, C_out, Kh, Kw);
+    if (stride < 1 || dilation < 1 || pad < 0 || groups < 1)
+        return fail(CONV_ERR_INVALID_ARG, "need stride >= 1, dilation >= 1, pad >= 0, groups >= 1");
+    if (C_in % groups != 0 || C_out % groups != 0)
+        return fail(CONV_ERR_INVALID_ARG, "C_in (%d) and C_out (%d) must be divisible by groups (%d)",
+                    C_in, C_out, groups);
+    if (dtype != CONV_F32 && dtype != CONV_BF16)
+        return fail(CONV_ERR_INVALID_ARG, "unknown dtype %d", static_cast<int>(dtype));
+    if (layout != CONV_NHWC && layout != CONV_NCHW)
+        return fail(CONV_ERR_INVALID_ARG, "unknown layout %d", static_cast<int>(layout));
+    Plan p{};
+    p.N = N; p.C_in = C_in; p.H = H; p.W = W; p.C_out = C_out; p.Kh = Kh; p.Kw = Kw;
+    p.stride = stride; p.pad = pad; p.dilation = dilation; p.groups = groups;
+    p.f32 = dtype == CONV_F32;
+    p.elt = p.f32 ? 4 : 2;
+    p.layout = layout;
+    if (out_size(H, Kh, stride, pad, dilation, &p.Ho) || out_size(W, Kw, stride, pad, dilation, &p.Wo))
+        return fail(CONV_ERR_INVALID_ARG, "empty output: the dilated kernel is larger than the padded input");
+    p.M = static_cast<long long>(N) * p.Ho * p.Wo;
+    // Limits of the hardware im2col addressing (traversal stride <= 8, bounding-box
+    // corners in [-128, 127] for a 4-D tensor) and of 32-bit indexing.
+    if (stride > 8) return fail(CONV_ERR_UNSUPPORTED, "stride %d > 8", stride);
+    if (pad > 127) return fail(CONV_ERR_UNSUPPORTED, "pad %d > 127", pad);
+    const long long up_h = pad - static_cast<long long>(Kh - 1) * dilation;
+    const long long up_w = pad - static_cast<long long>(Kw - 1) * dilation;
+    if (up_h < -128 || up_w < -128)
+        return fail(CONV_ERR_UNSUPPORTED, "dilation*(K-1) - pad exceeds 128");
+    if (p.M >= (1LL << 31) - 256) return fail(CONV_ERR_UNSUPPORTED, "N*Ho*Wo too large");
+    if (static_cast<long long>(N) * H * W * C_in >= (1LL << 40))
+        return fail(CONV_ERR_UNSUPPORTED, "input too large");
+
+    p.Cin_g = C_in / groups;
+    p.Cout_g = C_out / groups;
+    const int align = 16 / p.elt;
+    p.Cpg = round_up(p.Cin_g, align);
+    p.xcopy = layout == CONV_NCHW || p.Cpg != p.Cin_g;
+    const int row_bytes = p.Cpg * p.elt;
+    p.cb = row_bytes % 128 == 0 ? 128 : row_bytes % 64 == 0 ? 64 : row_bytes % 32 == 0 ? 32 : 16;
+    const int cap = p.f32 ? 128 : 256;
+    const int nt = (p.Cout_g + cap - 1) / cap;
+    p.BN = round_up((p.Cout_g + nt - 1) / nt, 16);
+    p.n_ntiles = (p.Cout_g + p.BN - 1) / p.BN;
+    p.taps = Kh * Kw;
+    p.nCB = row_bytes / p.cb;
+    p.planes = p.taps * p.nCB;
+    const int np = 128 / p.cb;
+    p.kstages = (p.planes + np - 1) / np;
+    p.Kp = p.taps * p.Cpg;
+    p.n_mtiles = static_cast<int>((p.M + 127) / 128);
+    const long long base = static_cast<long long>(p.n_mtiles) * p.n_ntiles * groups;
+    if (base >= (1LL << 31)) return fail(CONV_ERR_UNSUPPORTED, "too many tiles");
+    p.splits = 1;
+    if (sms > 0 && base < sms) {
+        int s = static_cast<int>(sms / base);
+        s = s < p.kstages / 4 ? s : p.kstages / 4;
+        s = s < 16 ? s : 16;
+        if (s >= 2) p.splits = s;
+    }
+    p.units = static_cast<int>(base * p.splits);
+    const size_t stage = static_cast<size_t>(128 + p.BN) * 128 * (p.f32 ? 2 : 1);
+    int stages = static_cast<int>((kSmemBudget - 2048) / stage);
+    p.stages = stages > 8 ? 8 : stages;
+    if (p.stages < 2) return fail(CONV_ERR_UNSUPPORTED, "tile does not fit in shared memory");
+    p.smem = igemm_smem_bytes(p.f32, p.BN, p.stages);
+
+    size_t off = 0;
+    p.off_xcopy = off;
+    if (p.xcopy) off = align_up(off + static_cast<size_t>(N) * H * W * groups * p.Cpg * p.elt, 256);
+    p.off_partial = off;
+    if (p.splits > 1) off = align_up(off + static_cast<size_t>(p.splits) * p.M * C_out * 4, 256);
+    p.off_xcol = off;
+    if (explicit_im2col) off = align_up(off + static_cast<size_t>(p.M) * groups * p.Kp * p.elt, 256);
+    p.ws_total = off;
+    *P = p;
+    return CONV_OK;
+}
+
+bool aligned16(const void *ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+
+CUtensorMapSwizzle swizzle_for(int cb) {
+    switch (cb) {
+        case 128: return CU_TENSOR_MAP_SWIZZLE_128B;
+        case 64: return CU_TENSOR_MAP_SWIZZLE_64B;
+        case 32: return CU_TENSOR_MAP_SWIZZLE_32B;
+        default: return CU_TENSOR_MAP_SWIZZLE_NONE;
+    }
+}
+
+CUtensorMapDataType tma_type(const Plan &p) {
+    return p.f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+}
+
+// A operand, implicit: im2col view of the channels-last input.
+int encode_a_im2col(const Plan &p, const void *x_nhwc, CUtensorMap *map) {
+    const cuuint64_t ctot = static_cast<cuuint64_t>(p.groups) * p.Cpg;
+    cuuint64_t dims[4] = {ctot, static_cast<cuuint64_t>(p.W), static_cast<cuuint64_t>(p.H),
+                          static_cast<cuuint64_t>(p.N)};
+    cuuint64_t strides[3] = {ctot * p.elt, ctot * p.elt * p.W, ctot * p.elt * p.W * p.H};
+    int lower[2] = {-p.pad, -p.pad};  // (w, h)
+    int upper[2] = {p.pad - (p.Kw - 1) * p.dilation, p.pad - (p.Kh - 1) * p.dilation};
+    cuuint32_t estr[4] = {1, static_cast<cuuint32_t>(p.stride), static_cast<cuuint32_t>(p.stride), 1};
+    CUresult r = g_encode_im2col(map, tma_type(p), 4, const_cast<void *>(x_nhwc), dims, strides, lower,
+                                 upper, static_cast<cuuint32_t>(p.cb / p.elt), 128, estr,
+                                 CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_for(p.cb),
+                                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(CONV_ERR_CUDA, "cuTensorMapEncodeIm2col failed (%d)", static_cast<int>(r));
+    return CONV_OK;
+}
+
+// A operand, explicit: the X_col matrix (M rows of groups*Kp elements).
+int encode_a_xcol(const Plan &p, const void *xcol, CUtensorMap *map) {
+    const cuuint64_t cols = static_cast<cuuint64_t>(p.groups) * p.Kp;
+    cuuint64_t dims[2] = {cols, static_cast<cuuint64_t>(p.M)};
+    cuuint64_t strides[1] = {cols * p.elt};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(p.cb / p.elt), 128};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode_tiled(map, tma_type(p), 2, const_cast<void *>(xcol), dims, strides, box, estr,
+                                CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_for(p.cb),
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(CONV_ERR_CUDA, "cuTensorMapEncodeTiled (X_col) failed (%d)", static_cast<int>(r));
+    return CONV_OK;
+}
+
+// B operand: packed weights viewed as {Kp, Cout_g, groups}.
+int encode_b(const Plan &p, const void *w_packed, CUtensorMap *map) {
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(p.Kp), static_cast<cuuint64_t>(p.Cout_g),
+                          static_cast<cuuint64_t>(p.groups)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(p.Kp) * p.elt,
+                             static_cast<cuuint64_t>(p.Kp) * p.elt * p.Cout_g};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(p.cb / p.elt), static_cast<cuuint32_t>(p.BN), 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode_tiled(map, tma_type(p), 3, const_cast<void *>(w_packed), dims, strides, box,
+                                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_for(p.cb),
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(CONV_ERR_CUDA, "cuTensorMapEncodeTiled (weights) failed (%d)", static_cast<int>(r));
+    return CONV_OK;
+}
+
+int check_launch(cudaError_t e, const char *what) {
+    if (e != cudaSuccess) return fail(CONV_ERR_CUDA, "%s launch: %s", what, cudaGetErrorString(e));
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return CONV_OK;
+}
+
+// Shared body of conv2d_forward and conv2d_forward_im2col_gemm.
+int forward_impl(bool explicit_im2col, const void *x, const void *w_packed, const void *bias, void *y,
+                 int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stride, int pad,
+                 int dilation, int groups, conv_dtype_t dtype, conv_layout_t layout, void *workspace,
+                 size_t workspace_bytes, cudaStream_t stream) {
+    DeviceInfo *dev = nullptr;
+    Plan p;
+    int st = make_plan(N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype, layout,
+                       explicit_im2col, 0, &p);
+    if (st != CONV_OK) return st;
+    if (!x || !w_packed || !y) return fail(CONV_ERR_INVALID_ARG, "x, w_packed and y must not be NULL");
+    st = device_info(&dev);
+    if (st != CONV_OK) return st;
+    st = make_plan(N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype, layout,
+                   explicit_im2col, dev->sms, &p);
+    if (st != CONV_OK) return st;
+    if (p.ws_total > 0 && (!workspace || workspace_bytes < p.ws_total))
+        return fail(CONV_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", p.ws_total,
+                    workspace ? workspace_bytes : static_cast<size_t>(0));
+    if (!aligned16(x) || !aligned16(w_packed) || !aligned16(y) || (bias && !aligned16(bias)) ||
+        (workspace && !aligned16(workspace)))
+        return fail(CONV_ERR_UNSUPPORTED, "device pointers must be 16-byte aligned");
+
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    const void *x_nhwc = p.xcopy ? static_cast<const void *>(ws + p.off_xcopy) : x;
+    void *xcol = explicit_im2col ? static_cast<void *>(ws + p.off_xcol) : nullptr;
+
+    IgemmParams kp;
+    std::memset(&kp, 0, sizeof(kp));
+    st = explicit_im2col ? encode_a_xcol(p, xcol, &kp.tmap_a) : encode_a_im2col(p, x_nhwc, &kp.tmap_a);
+    if (st != CONV_OK) return st;
+    st = encode_b(p, w_packed, &kp.tmap_b);
+    if (st != CONV_OK) return st;
+    kp.M = static_cast<int>(p.M);
+    kp.HoWo = p.Ho * p.Wo;
+    kp.Wo = p.Wo;
+    kp.stride = stride;
+    kp.pad = pad;
+    kp.dilation = dilation;
+    kp.Kw = Kw;
+    kp.taps = p.taps;
+    kp.Cpg = p.Cpg;
+    kp.nCB = p.nCB;
+    kp.planes = p.planes;
+    kp.kstages = p.kstages;
+    kp.Kp = p.Kp;
+    kp.groups = groups;
+    kp.Cout_g = p.Cout_g;
+    kp.Cout = C_out;
+    kp.BN = p.BN;
+    kp.n_mtiles = p.n_mtiles;
+    kp.n_ntiles = p.n_ntiles;
+    kp.splits = p.splits;
+    kp.units = p.units;
+    kp.stages = p.stages;
+    uint32_t cols = 32;
+    while (cols < static_cast<uint32_t>(2 * p.BN)) cols <<= 1;
+    kp.tmem_cols = cols;
+    kp.bias = bias;
+    if (p.splits > 1) {
+        kp.y = ws + p.off_partial;
+        kp.out_mode = kOutPartial;
+        kp.vec_ok = (C_out % 4 == 0 && p.Cout_g % 4 == 0) ? 1 : 0;
+    } else {
+        kp.y = y;
+        kp.out_mode = layout == CONV_NCHW ? kOutNCHW : kOutNHWC;
+        const int per16 = 16 / p.elt;
+        kp.vec_ok = (C_out % per16 == 0 && p.Cout_g % per16 == 0) ? 1 : 0;
+    }
+    kp.status = dev->status;
+    kp.timeout_ns = g_timeout_ns;
+    kp.starve = g_starve;
+
+    if (p.xcopy) {
+        cudaError_t e = layout == CONV_NCHW
+                            ? launch_nchw_to_nhwc(x, ws + p.off_xcopy, N, C_in, H, W, groups, p.Cpg, p.elt, stream)
+                            : launch_nhwc_pad(x, ws + p.off_xcopy, N, C_in, H, W, groups, p.Cpg, p.elt, stream);
+        if ((st = check_launch(e, "channels-last copy")) != CONV_OK) return st;
+    }
+    if (explicit_im2col) {
+        cudaError_t e = launch_im2col(x_nhwc, xcol, N, H, W, groups, p.Cpg, p.Ho, p.Wo, Kh, Kw,
+                                      stride, pad, dilation, p.elt, stream);
+        if ((st = check_launch(e, "im2col")) != CONV_OK) return st;
+    }
+    const int grid = p.units < dev->sms ? p.units : dev->sms;
+    cudaEvent_t ev_start = g_main_start, ev_stop = g_main_stop;
+    if (ev_start && ev_stop) cudaEventRecord(ev_start, stream);
+    cudaError_t e = launch_igemm(kp, p.f32, p.cb, !explicit_im2col, grid, p.smem, stream);
+    if ((st = check_launch(e, "tensor-core product")) != CONV_OK) return st;
+    if (ev_start && ev_stop) cudaEventRecord(ev_stop, stream);
+    if (p.splits > 1) {
+        e = launch_splitk_reduce(reinterpret_cast<const float *>(ws + p.off_partial), bias, y,
+                                 static_cast<int>(p.M), C_out, p.Ho * p.Wo, p.splits,
+                                 layout == CONV_NCHW ? kOutNCHW : kOutNHWC, p.f32, stream);
+        if ((st = check_launch(e, "split reduction")) != CONV_OK) return st;
+    }
+    return ok();
+}
+
+int workspace_impl(bool explicit_im2col, int N, int C_in, int H, int W, int C_out, int Kh, int Kw,
+                   int stride, int pad, int dilation, int groups, conv_dtype_t dtype,
+                   conv_layout_t layout, size_t *bytes) {
+    if (!bytes) return fail(CONV_ERR_INVALID_ARG, "bytes must not be NULL");
+    Plan p;
+    int st = make_plan(N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype, layout,
+                       explicit_im2col, 0, &p);
+    if (st != CONV_OK) return st;
+    DeviceInfo *dev = nullptr;
+    int sms = 0;
+    int ndev = 0;
+    if (cudaGetDeviceCount(&ndev) == cudaSuccess && ndev > 0 && device_info(&dev) == CONV_OK)
+        sms = dev->sms;
+    else
+        cudaGetLastError();  // no usable device: size without a split
+    st = make_plan(N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype, layout,
+                   explicit_im2col, sms, &p);
+    if (st != CONV_OK) return st;
+    *bytes = p.ws_total;
+    return ok();
+}
+
+int elt_of(conv_dtype_t dtype) { return dtype == CONV_F32 ? 4 : dtype == CONV_BF16 ? 2 : 0; }
+
+}  // namespace
+}  // namespace conv2d_b200
+
+using namespace conv2d_b200;
+
+#pragma GCC visibility push(default)
+extern "C" {
+
+int conv2d_output_size(int in, int k, int stride, int pad, int dilation, int *out) {
+    if (!out || in < 1 || k < 1 || stride < 1 || pad < 0 || dilation < 1)
+        return fail(CONV_ERR_INVALID_ARG, "output size: invalid argument");
+    int v = 0;
+    if (out_size(in, k, stride, pad, dilation, &v) != 0)
+        return fail(CONV_ERR_INVALID_ARG, "output size: the dilated kernel is larger than the padded input");
+    *out = v;
+    return ok();
+}
+
+int conv2d_packed_weight_size(int C_out, int C_in, int Kh, int Kw, int groups, conv_dtype_t dtype,
+                              size_t *bytes) {
+    const int elt = elt_of(dtype);
+    if (!bytes || elt == 0 || C_out < 1 || C_in < 1 || Kh < 1 || Kw < 1 || groups < 1 ||
+        C_in % groups || C_out % groups)
+        return fail(CONV_ERR_INVALID_ARG, "packed weight size: invalid argument");
+    const int cpg = round_up(C_in / groups, 16 / elt);
+    *bytes = static_cast<size_t>(C_out) * Kh * Kw * cpg * elt;
+    return ok();
+}
+
+int conv2d_pack_weight(const void *w_oihw, void *w_packed, int C_out, int C_in, int Kh, int Kw,
+                       int groups, conv_dtype_t dtype, conv_stream_t stream) {
+    size_t bytes = 0;
+    int st = conv2d_packed_weight_size(C_out, C_in, Kh, Kw, groups, dtype, &bytes);
+    if (st != CONV_OK) return st;
+    if (!w_oihw || !w_packed) return fail(CONV_ERR_INVALID_ARG, "weight pointers must not be NULL");
+    const int elt = elt_of(dtype);
+    const int cpg = round_up(C_in / groups, 16 / elt);
+    return check_launch(launch_pack_weight(w_oihw, w_packed, C_out, C_in / groups, Kh, Kw, cpg, elt,
+                                           reinterpret_cast<cudaStream_t>(stream)),
+                        "weight pack") == CONV_OK
+               ? ok()
+               : CONV_ERR_CUDA;
+}
+
+int conv2d_workspace_size(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stride,
+                          int pad, int dilation, int groups, conv_dtype_t dtype,
+                          conv_layout_t layout, size_t *bytes) {
+    return workspace_impl(false, N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype,
+                          layout, bytes);
+}
+
+int conv2d_im2col_workspace_size(int N, int C_in, int H, int W, int C_out, int Kh, int Kw,
+                                 int stride, int pad, int dilation, int groups,
+                                 conv_dtype_t dtype, conv_layout_t layout, size_t *bytes) {
+    return workspace_impl(true, N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype,
+                          layout, bytes);
+}
+
+int conv2d_forward(const void *x, const void *w_packed, const void *bias, void *y, int N, int C_in,
+                   int H, int W, int C_out, int Kh, int Kw, int stride, int pad, int dilation,
+                   int groups, conv_dtype_t dtype, conv_layout_t layout, void *workspace,
+                   size_t workspace_bytes, conv_stream_t stream) {
+    return forward_impl(false, x, w_packed, bias, y, N, C_in, H, W, C_out, Kh, Kw, stride, pad,
+                        dilation, groups, dtype, layout, workspace, workspace_bytes,
+                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+int conv2d_forward_im2col_gemm(const void *x, const void *w_packed, const void *bias, void *y,
+                               int N, int C_in, int H, int W, int C_out, int Kh, int Kw,
+                               int stride, int pad, int dilation, int groups, conv_dtype_t dtype,
+                               conv_layout_t layout, void *workspace, size_t workspace_bytes,
+                               conv_stream_t stream) {
+    return forward_impl(true, x, w_packed, bias, y, N, C_in, H, W, C_out, Kh, Kw, stride, pad,
+                        dilation, groups, dtype, layout, workspace, workspace_bytes,
+                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+int conv2d_forward_hostio(const void *x_host, void *y_host, void *x_dev, void *y_dev,
+                          const void *w_packed, const void *bias, int N, int C_in, int H, int W,
+                          int C_out, int Kh, int Kw, int stride, int pad, int dilation, int groups,
+                          conv_dtype_t dtype, conv_layout_t layout, void *workspace,
+                          size_t workspace_bytes, conv_stream_t stream) {
+    Plan p;
+    int st = make_plan(N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype, layout,
+                       false, 0, &p);
+    if (st != CONV_OK) return st;
+    if (!x_host || !y_host || !x_dev || !y_dev)
+        return fail(CONV_ERR_INVALID_ARG, "host and device activation buffers must not be NULL");
+    const size_t xb = static_cast<size_t>(N) * C_in * H * W * p.elt;
+    const size_t yb = static_cast<size_t>(p.M) * C_out * p.elt;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(x_dev, x_host, xb, cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return fail(CONV_ERR_CUDA, "input copy: %s", cudaGetErrorString(e));
+    st = forward_impl(false, x_dev, w_packed, bias, y_dev, N, C_in, H, W, C_out, Kh, Kw, stride,
+                      pad, dilation, groups, dtype, layout, workspace, workspace_bytes, s);
+    if (st != CONV_OK) return st;
+    e = cudaMemcpyAsync(y_host, y_dev, yb, cudaMemcpyDeviceToHost, s);
+    if (e != cudaSuccess) return fail(CONV_ERR_CUDA, "output copy: %s", cudaGetErrorString(e));
+    return ok();
+}
+
+int conv2d_nchw_to_nhwc(const void *src, void *dst, int N, int C, int H, int W, int groups,
+                        int Cpg, conv_dtype_t dtype, conv_stream_t stream) {
+    const int elt = elt_of(dtype);
+    if (!src || !dst || elt == 0 || N < 1 || C < 1 || H < 1 || W < 1 || groups < 1 ||
+        C % groups || Cpg < C / groups)
+        return fail(CONV_ERR_INVALID_ARG, "nchw_to_nhwc: invalid argument");
+    if (!aligned16(src) || !aligned16(dst))
+        return fail(CONV_ERR_UNSUPPORTED, "device pointers must be 16-byte aligned");
+    return check_launch(launch_nchw_to_nhwc(src, dst, N, C, H, W, groups, Cpg, elt,
+                                            reinterpret_cast<cudaStream_t>(stream)),
+                        "nchw_to_nhwc") == CONV_OK
+               ? ok()
+               : CONV_ERR_CUDA;
+}
+
+int conv2d_nhwc_to_nchw(const void *src, void *dst, int N, int C, int H, int W,
+                        conv_dtype_t dtype, conv_stream_t stream) {
+    const int elt = elt_of(dtype);
+    if (!src || !dst || elt == 0 || N < 1 || C < 1 || H < 1 || W < 1)
+        return fail(CONV_ERR_INVALID_ARG, "nhwc_to_nchw: invalid argument");
+    return check_launch(launch_nhwc_to_nchw(src, dst, N, C, H, W, elt,
+                                            reinterpret_cast<cudaStream_t>(stream)),
+                        "nhwc_to_nchw") == CONV_OK
+               ? ok()
+               : CONV_ERR_CUDA;
+}
+
+int conv2d_sync_status(conv_stream_t stream) {
+    cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(CONV_ERR_CUDA, "stream: %s", cudaGetErrorString(e));
+    DeviceInfo *dev = nullptr;
+    int st = device_info(&dev);
+    if (st != CONV_OK) return st;
+    int v = 0;
+    e = cudaMemcpy(&v, dev->status, sizeof(int), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return fail(CONV_ERR_CUDA, "status read: %s", cudaGetErrorString(e));
+    if (v != 0) {
+        const int zero = 0;
+        cudaMemcpy(dev->status, &zero, sizeof(int), cudaMemcpyHostToDevice);
+        return fail(CONV_ERR_TIMEOUT, "device watchdog fired (code %d)", v);
+    }
+    return ok();
+}
+
+const char *conv2d_last_error(void) { return t_last_error.c_str(); }
+
+int conv2d_set_main_kernel_events(void *start, void *stop) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (start && stop) {
+        g_main_start = static_cast<cudaEvent_t>(start);
+        g_main_stop = static_cast<cudaEvent_t>(stop);
+    } else {
+        g_main_start = g_main_stop = nullptr;
+    }
+    return ok();
+}
+
+int conv2d_kernel_launch_count(unsigned long long *count) {
+    if (!count) return fail(CONV_ERR_INVALID_ARG, "count must not be NULL");
+    *count = g_launches.load(std::memory_order_relaxed);
+    return ok();
+}
+
+int conv2d_debug_set_watchdog(long long timeout_ns, int starve_loads) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    g_timeout_ns = timeout_ns > 0 ? timeout_ns : kDefaultTimeoutNs;
+    g_starve = starve_loads ? 1 : 0;
+    return ok();
+}
+
+}  // extern "C"
+#pragma GCC visibility pop

@@ -1,0 +1,525 @@
+// igemm.cu -- the convolution forward pass as an implicit matrix product on the
+// sm_100a tensor cores (tcgen05), never forming the im2col matrix in memory.
+//
+// The product is the one of the im2col/GEMM tutorial (zskr.cn/news/1820658) §2.3,
+// Y = W_row @ X_col, computed transposed: rows are output pixels
+// m = (n*Ho + oh)*Wo + ow (tcgen05 M = 128 per tile), columns are the output channels
+// of one group (tcgen05 N = BN), and the reduction runs over the filter taps
+// (kh, kw) and the input channels of the group -- the "expand per tile, multiply,
+// discard" scheme the "手撕 Conv2D" page (lpnh.cn/news/2493075) §4.1 mentions, with
+// the expansion done by the tensor memory accelerator's im2col mode.
+//
+// One persistent CTA per SM, warp-specialised:
+//   warp 0      : TMA producer -- per stage, one im2col load of 128 output pixels x
+//                 CB bytes of channels per plane (filter-tap offsets kw*d, kh*d; reads
+//                 outside the image return zero, which is the zero padding) and one
+//                 tiled load of BN weight rows x CB bytes per plane;
+//   warp 1      : allocates tensor memory and issues tcgen05.mma from one thread,
+//                 releasing each stage with tcgen05.commit;
+//   warps 2..5  : epilogue -- tcgen05.ld of the fp32 accumulator, + bias, round, store;
+//   warps 6..9  : (fp32 only) split every staged fp32 value v into tf32 parts
+//                 hi = tf32(v), lo = tf32(v - hi) for the three-product scheme.
+// Two accumulators in tensor memory let the epilogue of one tile overlap the
+// main loop of the next.  Every wait is bounded (see ptx.cuh).
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace conv2d_b200 {
+namespace {
+
+using namespace ptx;
+
+constexpr int kBM = 128;                  // output pixels per tile
+constexpr int kStageRowBytes = 128;       // reduction bytes per operand row per stage
+constexpr int kAStageBytes = kBM * kStageRowBytes;
+constexpr int kMaxStages = 8;
+constexpr int kBarrierBlock = 1024;       // barriers + flags, ahead of the stage ring
+
+constexpr int kProducerWarp = 0;
+constexpr int kMmaWarp = 1;
+constexpr int kEpiWarp0 = 2;
+constexpr int kCvtWarp0 = 6;
+
+template <bool kF32>
+constexpr int threads_for() { return kF32 ? 320 : 192; }
+
+__host__ __device__ inline uint32_t stage_bytes(bool f32, int BN) {
+    return static_cast<uint32_t>((kAStageBytes + BN * kStageRowBytes) * (f32 ? 2 : 1));
+}
+
+struct SharedBlock {  // lives at the start of the 1024-aligned dynamic shared memory
+    uint64_t full[kMaxStages];
+    uint64_t empty[kMaxStages];
+    uint64_t converted[kMaxStages];
+    uint64_t acc_full[2];
+    uint64_t acc_empty[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+};
+static_assert(sizeof(SharedBlock) <= kBarrierBlock, "barrier block too small");
+
+struct Unit {
+    int mtile, g, ntile, split, k0, k1;
+};
+
+__device__ __forceinline__ Unit decode_unit(const IgemmParams &p, int u) {
+    Unit t;
+    t.split = u % p.splits;
+    int r = u / p.splits;
+    t.ntile = r % p.n_ntiles;
+    r /= p.n_ntiles;
+    t.g = r % p.groups;
+    t.mtile = r / p.groups;
+    t.k0 = static_cast<int>((static_cast<long long>(t.split) * p.kstages) / p.splits);
+    t.k1 = static_cast<int>((static_cast<long long>(t.split + 1) * p.kstages) / p.splits);
+    return t;
+}
+
+__device__ __forceinline__ float tf32_round(float v) {
+    // round to the nearest value with 10 explicit mantissa bits (ties away from zero)
+    return __uint_as_float((__float_as_uint(v) + 0x1000u) & 0xFFFFE000u);
+}
+
+// Bounded wait that ignores the abort flag: used only while tearing down after an
+// abort, to let copies already in flight land before the CTA exits.
+__device__ __forceinline__ void wait_quiet(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
+    const uint64_t start = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer_ns() - start > limit_ns) return;
+    }
+}
+
+// --------------------------------------------------------------- epilogue ---
+template <bool kF32>
+__device__ __forceinline__ void store_chunk16(const IgemmParams &p, int m, int g, int col0,
+                                              int split, const uint32_t (&r)[16]) {
+    if (m >= p.M) return;
+    const int nvalid = min(16, p.Cout_g - col0);
+    if (nvalid <= 0) return;
+    const int oc0 = g * p.Cout_g + col0;
+    float v[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+
+    if (p.out_mode == kOutPartial) {
+        float *dst = static_cast<float *>(p.y) +
+                     (static_cast<size_t>(split) * p.M + m) * p.Cout + oc0;
+        if (nvalid == 16 && p.vec_ok) {
+            float4 *d4 = reinterpret_cast<float4 *>(dst);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                d4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                if (i < nvalid) dst[i] = v[i];
+        }
+        return;
+    }
+    if (p.bias) {
+        if constexpr (kF32) {
+            const float *b = static_cast<const float *>(p.bias) + oc0;
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                if (i < nvalid) v[i] += __ldg(b + i);
+        } else {
+            const __nv_bfloat16 *b = static_cast<const __nv_bfloat16 *>(p.bias) + oc0;
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                if (i < nvalid) v[i] += __bfloat162float(b[i]);
+        }
+    }
+    if (p.out_mode == kOutNHWC) {
+        if constexpr (kF32) {
+            float *dst = static_cast<float *>(p.y) + static_cast<size_t>(m) * p.Cout + oc0;
+            if (nvalid == 16 && p.vec_ok) {
+                float4 *d4 = reinterpret_cast<float4 *>(dst);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    d4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    if (i < nvalid) dst[i] = v[i];
+            }
+        } else {
+            __nv_bfloat16 *dst =
+                static_cast<__nv_bfloat16 *>(p.y) + static_cast<size_t>(m) * p.Cout + oc0;
+            if (nvalid == 16 && p.vec_ok) {
+                uint32_t packed[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+                    packed[i] = *reinterpret_cast<uint32_t *>(&h);
+                }
+                uint4 *d4 = reinterpret_cast<uint4 *>(dst);
+                d4[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+                d4[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    if (i < nvalid) dst[i] = __float2bfloat16_rn(v[i]);
+            }
+        }
+    } else {  // kOutNCHW: lanes hold consecutive pixels, so each column is a coalesced row
+        const int n = m / p.HoWo;
+        const int pix = m - n * p.HoWo;
+        const size_t base = (static_cast<size_t>(n) * p.Cout + oc0) * p.HoWo + pix;
+        if constexpr (kF32) {
+            float *dst = static_cast<float *>(p.y) + base;
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                if (i < nvalid) dst[static_cast<size_t>(i) * p.HoWo] = v[i];
+        } else {
+            __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.y) + base;
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                if (i < nvalid) dst[static_cast<size_t>(i) * p.HoWo] = __float2bfloat16_rn(v[i]);
+        }
+    }
+}
+
+// ------------------------------------------------------------------ MMAs ---
+// Issues the tensor-core instructions for one staged block of the reduction
+// (128 bytes per operand row: kNP planes of kCB bytes).
+template <bool kF32, int kCB>
+__device__ __forceinline__ void issue_stage(uint32_t a, uint32_t b, uint32_t alo, uint32_t blo,
+                                            int BN, uint32_t d_tmem, uint32_t idesc,
+                                            bool first) {
+    constexpr int kNP = kStageRowBytes / kCB;
+    const uint32_t a_plane = kBM * kCB;
+    const uint32_t b_plane = static_cast<uint32_t>(BN) * kCB;
+    if constexpr (kCB >= 32) {
+        constexpr uint32_t kSw = kCB == 128 ? kSw128 : (kCB == 64 ? kSw64 : kSw32);
+        constexpr uint32_t kSbo = 8 * kCB;  // eight rows of one swizzle atom
+#pragma unroll
+        for (int j = 0; j < kNP; ++j) {
+#pragma unroll
+            for (int kk = 0; kk < kCB / 32; ++kk) {
+                const uint32_t ao = j * a_plane + kk * 32;
+                const uint32_t bo = j * b_plane + kk * 32;
+                const uint32_t acc = (first && j == 0 && kk == 0) ? 0u : 1u;
+                if constexpr (kF32) {
+                    mma_tf32(d_tmem, smem_desc(alo + ao, 16, kSbo, kSw),
+                             smem_desc(b + bo, 16, kSbo, kSw), idesc, acc);
+                    mma_tf32(d_tmem, smem_desc(a + ao, 16, kSbo, kSw),
+                             smem_desc(blo + bo, 16, kSbo, kSw), idesc, 1u);
+                    mma_tf32(d_tmem, smem_desc(a + ao, 16, kSbo, kSw),
+                             smem_desc(b + bo, 16, kSbo, kSw), idesc, 1u);
+                } else {
+                    mma_bf16(d_tmem, smem_desc(a + ao, 16, kSbo, kSw),
+                             smem_desc(b + bo, 16, kSbo, kSw), idesc, acc);
+                }
+            }
+        }
+    } else {
+        // 16-byte planes, no swizzle: core matrices of 8 rows x 16 bytes stacked every
+        // 128 bytes (SBO); one instruction's 32-byte K slice spans two planes (LBO).
+#pragma unroll
+        for (int j = 0; j < kNP; j += 2) {
+            const uint32_t acc = (first && j == 0) ? 0u : 1u;
+            const uint32_t ao = j * a_plane, bo = j * b_plane;
+            if constexpr (kF32) {
+                mma_tf32(d_tmem, smem_desc(alo + ao, a_plane, 128, kSwNone),
+                         smem_desc(b + bo, b_plane, 128, kSwNone), idesc, acc);
+                mma_tf32(d_tmem, smem_desc(a + ao, a_plane, 128, kSwNone),
+                         smem_desc(blo + bo, b_plane, 128, kSwNone), idesc, 1u);
+                mma_tf32(d_tmem, smem_desc(a + ao, a_plane, 128, kSwNone),
+                         smem_desc(b + bo, b_plane, 128, kSwNone), idesc, 1u);
+            } else {
+                mma_bf16(d_tmem, smem_desc(a + ao, a_plane, 128, kSwNone),
+                         smem_desc(b + bo, b_plane, 128, kSwNone), idesc, acc);
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------- kernel ---
+template <bool kF32, int kCB, bool kIm2col>
+__global__ void __launch_bounds__(threads_for<kF32>(), 1)
+    igemm_kernel(const __grid_constant__ IgemmParams p) {
+    constexpr int kElt = kF32 ? 4 : 2;
+    constexpr int kCBe = kCB / kElt;              // channels (elements) per plane row
+    constexpr int kNP = kStageRowBytes / kCB;     // planes per stage
+
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_addr = smem_addr(smem_raw);
+    uint8_t *base = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+    SharedBlock &sb = *reinterpret_cast<SharedBlock *>(base);
+    uint8_t *ring = base + kBarrierBlock;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int BN = p.BN;
+    const uint32_t sbytes = stage_bytes(kF32, BN);
+    const uint32_t b_off = kAStageBytes;
+    const uint32_t alo_off = kAStageBytes + BN * kStageRowBytes;
+    const uint32_t blo_off = alo_off + kAStageBytes;
+    const uint32_t tx_bytes = kAStageBytes + BN * kStageRowBytes;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < p.stages; ++s) {
+            mbar_init(&sb.full[s], 1);
+            mbar_init(&sb.empty[s], 1);
+            mbar_init(&sb.converted[s], 128);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sb.acc_full[i], 1);
+            mbar_init(&sb.acc_empty[i], 4);
+        }
+        mbar_init(&sb.drain, 1);
+        sb.abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == kMmaWarp) {
+        tmem_alloc(&sb.tmem_base, p.tmem_cols);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem_base = sb.tmem_base;
+
+    Watchdog wd;
+    wd.abort = &sb.abort;
+    wd.status = p.status;
+    wd.timeout_ns = static_cast<uint64_t>(p.timeout_ns);
+
+    if (warp == kProducerWarp) {
+        // ------------------------------------------------------ TMA producer ---
+        if (lane == 0) {
+            prefetch_tensormap(&p.tmap_a);
+            prefetch_tensormap(&p.tmap_b);
+            int stage = 0;
+            uint32_t phase = 0;
+            long long loads_issued = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
+                const Unit t = decode_unit(p, u);
+                const int m0 = t.mtile * kBM;
+                int img = 0, h0 = 0, w0 = 0;
+                if constexpr (kIm2col) {
+                    img = m0 / p.HoWo;
+                    const int rem = m0 - img * p.HoWo;
+                    const int oh = rem / p.Wo;
+                    const int ow = rem - oh * p.Wo;
+                    h0 = oh * p.stride - p.pad;
+                    w0 = ow * p.stride - p.pad;
+                }
+                for (int ks = t.k0; ks < t.k1; ++ks) {
+                    if (!mbar_wait(&sb.empty[stage], phase ^ 1u, wd, kDevTimeoutEmpty)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *st = ring + static_cast<size_t>(stage) * sbytes;
+                    if (!p.starve) {
+                        mbar_arrive_expect_tx(&sb.full[stage], tx_bytes);
+#pragma unroll
+                        for (int j = 0; j < kNP; ++j) {
+                            const int plane = ks * kNP + j;
+                            const int kelem = plane * kCBe;  // offset in the group's reduction
+                            if constexpr (kIm2col) {
+                                const int tap = min(plane / p.nCB, p.taps - 1);
+                                const int cblk = plane - (plane / p.nCB) * p.nCB;
+                                const int kh = tap / p.Kw;
+                                const int kw = tap - kh * p.Kw;
+                                const int c = t.g * p.Cpg + cblk * kCBe;
+                                tma_load_im2col_4d(st + j * (kBM * kCB), &p.tmap_a, &sb.full[stage],
+                                                   c, w0, h0, img,
+                                                   static_cast<uint16_t>(kw * p.dilation),
+                                                   static_cast<uint16_t>(kh * p.dilation));
+                            } else {
+                                tma_load_2d(st + j * (kBM * kCB), &p.tmap_a, &sb.full[stage],
+                                            t.g * p.Kp + kelem, m0);
+                            }
+                            tma_load_3d(st + b_off + j * (BN * kCB), &p.tmap_b, &sb.full[stage],
+                                        kelem, t.ntile * BN, t.g);
+                        }
+                        ++loads_issued;
+                    }
+                    if (++stage == p.stages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (*wd.abort && loads_issued > 0) {
+                // Let the copies still in flight land before the CTA goes away.
+                const long long first = loads_issued > p.stages ? loads_issued - p.stages : 0;
+                for (long long i = first; i < loads_issued; ++i)
+                    wait_quiet(&sb.full[i % p.stages], static_cast<uint32_t>((i / p.stages) & 1),
+                               wd.timeout_ns);
+            }
+        }
+    } else if (warp == kMmaWarp) {
+        // --------------------------------------------------- tensor-core issue ---
+        if (lane == 0) {
+            const uint32_t idesc = instr_desc(kF32 ? 2u : 1u, kBM, static_cast<uint32_t>(BN));
+            int stage = 0;
+            uint32_t phase = 0;
+            int abuf = 0;
+            uint32_t aphase = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
+                const Unit t = decode_unit(p, u);
+                if (!mbar_wait(&sb.acc_empty[abuf], aphase ^ 1u, wd, kDevTimeoutAccEmpty)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after_sync();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(abuf * BN);
+                for (int ks = t.k0; ks < t.k1; ++ks) {
+                    uint64_t *ready = kF32 ? &sb.converted[stage] : &sb.full[stage];
+                    if (!mbar_wait(ready, phase, wd, kF32 ? kDevTimeoutConvert : kDevTimeoutFull)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    const uint32_t st = smem_addr(ring + static_cast<size_t>(stage) * sbytes);
+                    issue_stage<kF32, kCB>(st, st + b_off, st + alo_off, st + blo_off, BN, d_tmem,
+                                           idesc, ks == t.k0);
+                    mma_commit(&sb.empty[stage]);
+                    if (++stage == p.stages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                mma_commit(&sb.acc_full[abuf]);
+                abuf ^= 1;
+                if (abuf == 0) aphase ^= 1u;
+            }
+            if (!ok || *wd.abort) {
+                mma_commit(&sb.drain);
+                wait_quiet(&sb.drain, 0, wd.timeout_ns);
+            }
+        }
+        __syncwarp();
+    } else if (warp < kEpiWarp0 + 4) {
+        // ------------------------------------------------------------ epilogue ---
+        const int quarter = warp & 3;  // tensor-memory lanes [32*quarter, 32*quarter + 32)
+        const int row = quarter * 32 + lane;
+        int abuf = 0;
+        uint32_t aphase = 0;
+        for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
+            const Unit t = decode_unit(p, u);
+            const bool ok = mbar_wait(&sb.acc_full[abuf], aphase, wd, kDevTimeoutAccFull);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            tc_fence_after_sync();
+            const int m = t.mtile * kBM + row;
+            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                                   static_cast<uint32_t>(abuf * BN);
+            for (int c = 0; c < BN; c += 16) {
+                uint32_t r[16];
+                tmem_ld_x16(taddr + static_cast<uint32_t>(c), r);
+                tmem_ld_wait();
+                store_chunk16<kF32>(p, m, t.g, t.ntile * BN + c, t.split, r);
+            }
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sb.acc_empty[abuf]);
+            abuf ^= 1;
+            if (abuf == 0) aphase ^= 1u;
+        }
+    } else if constexpr (kF32) {
+        // ------------------------------------------- fp32 -> tf32 hi/lo split ---
+        const int tid = (warp - kCvtWarp0) * 32 + lane;  // 0..127
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
+            const Unit t = decode_unit(p, u);
+            for (int ks = t.k0; ks < t.k1; ++ks) {
+                if (!mbar_wait(&sb.full[stage], phase, wd, kDevTimeoutFull)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t *st = ring + static_cast<size_t>(stage) * sbytes;
+                float4 *a = reinterpret_cast<float4 *>(st);
+                float4 *alo = reinterpret_cast<float4 *>(st + alo_off);
+                for (int i = tid; i < kAStageBytes / 16; i += 128) {
+                    const float4 v = a[i];
+                    float4 h, l;
+                    h.x = tf32_round(v.x); l.x = tf32_round(v.x - h.x);
+                    h.y = tf32_round(v.y); l.y = tf32_round(v.y - h.y);
+                    h.z = tf32_round(v.z); l.z = tf32_round(v.z - h.z);
+                    h.w = tf32_round(v.w); l.w = tf32_round(v.w - h.w);
+                    a[i] = h;
+                    alo[i] = l;
+                }
+                float4 *b = reinterpret_cast<float4 *>(st + b_off);
+                float4 *blo = reinterpret_cast<float4 *>(st + blo_off);
+                const int nb = BN * kStageRowBytes / 16;
+                for (int i = tid; i < nb; i += 128) {
+                    const float4 v = b[i];
+                    float4 h, l;
+                    h.x = tf32_round(v.x); l.x = tf32_round(v.x - h.x);
+                    h.y = tf32_round(v.y); l.y = tf32_round(v.y - h.y);
+                    h.z = tf32_round(v.z); l.z = tf32_round(v.z - h.z);
+                    h.w = tf32_round(v.w); l.w = tf32_round(v.w - h.w);
+                    b[i] = h;
+                    blo[i] = l;
+                }
+                fence_proxy_async_smem();
+                mbar_arrive(&sb.converted[stage]);
+                if (++stage == p.stages) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+    }
+
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem_base, p.tmem_cols);
+    }
+}
+
+template <bool kF32, int kCB, bool kIm2col>
+cudaError_t launch_one(const IgemmParams &p, int grid, size_t smem, cudaStream_t stream) {
+    auto kern = igemm_kernel<kF32, kCB, kIm2col>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    kern<<<grid, threads_for<kF32>(), smem, stream>>>(p);
+    return cudaGetLastError();
+}
+
+template <bool kF32, bool kIm2col>
+cudaError_t launch_cb(const IgemmParams &p, int cb, int grid, size_t smem, cudaStream_t s) {
+    switch (cb) {
+        case 128: return launch_one<kF32, 128, kIm2col>(p, grid, smem, s);
+        case 64: return launch_one<kF32, 64, kIm2col>(p, grid, smem, s);
+        case 32: return launch_one<kF32, 32, kIm2col>(p, grid, smem, s);
+        case 16: return launch_one<kF32, 16, kIm2col>(p, grid, smem, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace
+
+size_t igemm_smem_bytes(bool f32, int BN, int stages) {
+    return 1024 /* alignment slack */ + kBarrierBlock +
+           static_cast<size_t>(stages) * stage_bytes(f32, BN);
+}
+
+int igemm_threads(bool f32) { return f32 ? threads_for<true>() : threads_for<false>(); }
+
+cudaError_t launch_igemm(const IgemmParams &p, bool f32, int cb_bytes, bool im2col, int grid,
+                         size_t smem_bytes, cudaStream_t stream) {
+    if (p.stages < 2 || p.stages > kMaxStages) return cudaErrorInvalidValue;
+    if (f32) {
+        return im2col ? launch_cb<true, true>(p, cb_bytes, grid, smem_bytes, stream)
+                      : launch_cb<true, false>(p, cb_bytes, grid, smem_bytes, stream);
+    }
+    return im2col ? launch_cb<false, true>(p, cb_bytes, grid, smem_bytes, stream)
+                  : launch_cb<false, false>(p, cb_bytes, grid, smem_bytes, stream);
+}
+
+}  // namespace conv2d_b200

@@ -1,0 +1,304 @@
+// layout.cu -- bandwidth-bound helper kernels around the tensor-core product:
+//   * NCHW -> channels-last with per-group zero channel padding ("layout in");
+//   * channels-last -> NCHW ("layout out", zskr §3.2 step 5);
+//   * weight packing OIHW -> (oc, kh, kw, c) with zero channel padding;
+//   * explicit im2col (the pages' X_col, one row per output pixel);
+//   * the fp32 reduction of split partial sums, + bias, in the output layout.
+// All are plain coalesced CUDA-core kernels with grid-stride loops; none reads or
+// writes outside the extents passed in.
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+
+namespace conv2d_b200 {
+namespace {
+
+constexpr int kThreads = 256;
+
+inline int grid_for(long long work, int per_block = kThreads) {
+    long long g = (work + per_block - 1) / per_block;
+    if (g < 1) g = 1;
+    if (g > 148LL * 64) g = 148LL * 64;  // grid-stride loops cover the rest
+    return static_cast<int>(g);
+}
+
+template <int kElt> struct Word;
+template <> struct Word<2> { using T = uint16_t; };
+template <> struct Word<4> { using T = uint32_t; };
+
+// --- NCHW -> channels-last, small padded channel counts (Ctot * elt <= 64 bytes):
+// one thread per pixel; reads are coalesced across the warp (consecutive pixels of
+// one channel plane), each pixel's Ctot channels are written as 16-byte words.
+template <int kElt>
+__global__ void nchw_to_nhwc_small(const void *__restrict__ src, void *__restrict__ dst, int N,
+                                   int C, int HW, int groups, int Cpg) {
+    using T = typename Word<kElt>::T;
+    const T *s = static_cast<const T *>(src);
+    T *d = static_cast<T *>(dst);
+    const int Cg = C / groups;
+    const int Ctot = groups * Cpg;
+    const long long total = static_cast<long long>(N) * HW;
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const long long n = i / HW;
+        const long long pix = i - n * HW;
+        alignas(16) T vals[64 / kElt];
+        for (int cc = 0; cc < Ctot; ++cc) {
+            const int g = cc / Cpg, c = cc - g * Cpg;
+            vals[cc] = c < Cg ? s[(n * C + g * Cg + c) * HW + pix] : T(0);
+        }
+        uint4 *d4 = reinterpret_cast<uint4 *>(d + i * Ctot);
+        const uint4 *v4 = reinterpret_cast<const uint4 *>(vals);
+        for (int k = 0; k < Ctot * kElt / 16; ++k) d4[k] = v4[k];
+    }
+}
+
+// --- NCHW -> channels-last, general: 32 x 32 tiles through shared memory.
+// Block (32, 8); tile = 32 destination channels x 32 pixels of one image.
+template <int kElt>
+__global__ void nchw_to_nhwc_tiled(const void *__restrict__ src, void *__restrict__ dst, int N,
+                                   int C, int HW, int groups, int Cpg) {
+    using T = typename Word<kElt>::T;
+    __shared__ T tile[32][33];
+    const T *s = static_cast<const T *>(src);
+    T *d = static_cast<T *>(dst);
+    const int Cg = C / groups;
+    const int Ctot = groups * Cpg;
+    const int tiles_c = (Ctot + 31) / 32, tiles_p = (HW + 31) / 32;
+    const long long ntiles = static_cast<long long>(N) * tiles_c * tiles_p;
+    for (long long t = blockIdx.x; t < ntiles; t += gridDim.x) {
+        const long long n = t / (static_cast<long long>(tiles_c) * tiles_p);
+        const int r = static_cast<int>(t - n * tiles_c * tiles_p);
+        const int c0 = (r / tiles_p) * 32, p0 = (r % tiles_p) * 32;
+        for (int k = threadIdx.y; k < 32; k += 8) {  // read: channel rows, pixel columns
+            const int cc = c0 + k, pix = p0 + threadIdx.x;
+            T v = T(0);
+            if (cc < Ctot && pix < HW) {
+                const int g = cc / Cpg, c = cc - g * Cpg;
+                if (c < Cg) v = s[(n * C + g * Cg + c) * HW + pix];
+            }
+            tile[k][threadIdx.x] = v;
+        }
+        __syncthreads();
+        for (int k = threadIdx.y; k < 32; k += 8) {  // write: pixel rows, channel columns
+            const int pix = p0 + k, cc = c0 + threadIdx.x;
+            if (pix < HW && cc < Ctot) d[(n * HW + pix) * Ctot + cc] = tile[threadIdx.x][k];
+        }
+        __syncthreads();
+    }
+}
+
+// --- channels-last C -> channels-last groups*Cpg (zero channels appended per group).
+template <int kElt>
+__global__ void nhwc_pad_kernel(const void *__restrict__ src, void *__restrict__ dst,
+                                long long pixels, int C, int groups, int Cpg) {
+    using T = typename Word<kElt>::T;
+    const T *s = static_cast<const T *>(src);
+    T *d = static_cast<T *>(dst);
+    const int Cg = C / groups;
+    const int Ctot = groups * Cpg;
+    const long long total = pixels * Ctot;
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const long long pix = i / Ctot;
+        const int cc = static_cast<int>(i - pix * Ctot);
+        const int g = cc / Cpg, c = cc - g * Cpg;
+        d[i] = c < Cg ? s[pix * C + g * Cg + c] : T(0);
+    }
+}
+
+// --- channels-last -> NCHW: 32 x 32 tiles through shared memory.
+template <int kElt>
+__global__ void nhwc_to_nchw_tiled(const void *__restrict__ src, void *__restrict__ dst, int N,
+                                   int C, int HW) {
+    using T = typename Word<kElt>::T;
+    __shared__ T tile[32][33];
+    const T *s = static_cast<const T *>(src);
+    T *d = static_cast<T *>(dst);
+    const int tiles_c = (C + 31) / 32, tiles_p = (HW + 31) / 32;
+    const long long ntiles = static_cast<long long>(N) * tiles_c * tiles_p;
+    for (long long t = blockIdx.x; t < ntiles; t += gridDim.x) {
+        const long long n = t / (static_cast<long long>(tiles_c) * tiles_p);
+        const int r = static_cast<int>(t - n * tiles_c * tiles_p);
+        const int c0 = (r / tiles_p) * 32, p0 = (r % tiles_p) * 32;
+        for (int k = threadIdx.y; k < 32; k += 8) {  // read: pixel rows, channel columns
+            const int pix = p0 + k, c = c0 + threadIdx.x;
+            tile[k][threadIdx.x] = (pix < HW && c < C) ? s[(n * HW + pix) * C + c] : T(0);
+        }
+        __syncthreads();
+        for (int k = threadIdx.y; k < 32; k += 8) {  // write: channel rows, pixel columns
+            const int c = c0 + k, pix = p0 + threadIdx.x;
+            if (c < C && pix < HW) d[(n * C + c) * HW + pix] = tile[threadIdx.x][k];
+        }
+        __syncthreads();
+    }
+}
+
+// --- weights OIHW (Cout, Cin_g, Kh, Kw) -> (Cout, Kh, Kw, Cpg), zero for c >= Cin_g.
+template <int kElt>
+__global__ void pack_weight_kernel(const void *__restrict__ w, void *__restrict__ wp, int Cout,
+                                   int Cin_g, int Kh, int Kw, int Cpg) {
+    using T = typename Word<kElt>::T;
+    const T *s = static_cast<const T *>(w);
+    T *d = static_cast<T *>(wp);
+    const long long total = static_cast<long long>(Cout) * Kh * Kw * Cpg;
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const int c = static_cast<int>(i % Cpg);
+        long long r = i / Cpg;
+        const int kw = static_cast<int>(r % Kw);
+        r /= Kw;
+        const int kh = static_cast<int>(r % Kh);
+        const long long oc = r / Kh;
+        d[i] = c < Cin_g ? s[((oc * Cin_g + c) * Kh + kh) * Kw + kw] : T(0);
+    }
+}
+
+// --- explicit im2col: xcol[m][g*Kp + (kh*Kw + kw)*Cpg + c] = x[n][ih][iw][g*Cpg + c]
+// (0 outside the image), m = (n*Ho + oh)*Wo + ow.  One thread per 16-byte chunk; a
+// chunk never straddles two taps because Cpg*elt is a multiple of 16.
+template <int kElt>
+__global__ void im2col_kernel(const void *__restrict__ x, void *__restrict__ xcol, int N, int H,
+                              int W, int groups, int Cpg, int Ho, int Wo, int Kh, int Kw,
+                              int stride, int pad, int dilation) {
+    constexpr int kPer = 16 / kElt;  // elements per chunk
+    const int Kp = Kh * Kw * Cpg;
+    const int row_chunks = groups * Kp / kPer;
+    const int Ctot = groups * Cpg;
+    const long long total = static_cast<long long>(N) * Ho * Wo * row_chunks;
+    const uint4 *xs = static_cast<const uint4 *>(x);
+    uint4 *d = static_cast<uint4 *>(xcol);
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const long long m = i / row_chunks;
+        const int k = static_cast<int>(i - m * row_chunks) * kPer;  // element column
+        const int g = k / Kp;
+        const int kr = k - g * Kp;
+        const int tap = kr / Cpg, c = kr - tap * Cpg;
+        const int kh = tap / Kw, kw = tap - kh * Kw;
+        const int n = static_cast<int>(m / (static_cast<long long>(Ho) * Wo));
+        const int rem = static_cast<int>(m - static_cast<long long>(n) * Ho * Wo);
+        const int oh = rem / Wo, ow = rem - (rem / Wo) * Wo;
+        const int ih = oh * stride + kh * dilation - pad;
+        const int iw = ow * stride + kw * dilation - pad;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (ih >= 0 && ih < H && iw >= 0 && iw < W)
+            v = xs[((static_cast<long long>(n) * H + ih) * W + iw) * Ctot / kPer + (g * Cpg + c) / kPer];
+        d[i] = v;
+    }
+}
+
+// --- split reduction: y = bias + sum_s ws[s][m][oc], in the output layout.
+template <bool kF32>
+__global__ void splitk_reduce_kernel(const float *__restrict__ ws, const void *__restrict__ bias,
+                                     void *__restrict__ y, int M, int Cout, int HoWo, int splits,
+                                     int nchw) {
+    const long long total = static_cast<long long>(M) * Cout;
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        long long m, oc;
+        if (nchw) {  // consecutive threads walk pixels of one channel: coalesced writes
+            const long long plane = static_cast<long long>(HoWo);
+            const long long n = i / (plane * Cout);
+            const long long r = i - n * plane * Cout;
+            oc = r / plane;
+            m = n * plane + (r - oc * plane);
+        } else {
+            m = i / Cout;
+            oc = i - m * Cout;
+        }
+        float acc = 0.f;
+        if (bias)
+            acc = kF32 ? static_cast<const float *>(bias)[oc]
+                       : __bfloat162float(static_cast<const __nv_bfloat16 *>(bias)[oc]);
+        for (int s = 0; s < splits; ++s) acc += ws[(static_cast<long long>(s) * M + m) * Cout + oc];
+        if (kF32)
+            static_cast<float *>(y)[i] = acc;
+        else
+            static_cast<__nv_bfloat16 *>(y)[i] = __float2bfloat16_rn(acc);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_nchw_to_nhwc(const void *src, void *dst, int N, int C, int H, int W,
+                                int groups, int Cpg, int elt, cudaStream_t s) {
+    const int HW = H * W;
+    const int Ctot = groups * Cpg;
+    const long long pixels = static_cast<long long>(N) * HW;
+    if (Ctot * elt <= 64 && (Ctot * elt) % 16 == 0) {
+        if (elt == 2)
+            nchw_to_nhwc_small<2><<<grid_for(pixels), kThreads, 0, s>>>(src, dst, N, C, HW, groups, Cpg);
+        else
+            nchw_to_nhwc_small<4><<<grid_for(pixels), kThreads, 0, s>>>(src, dst, N, C, HW, groups, Cpg);
+    } else {
+        const long long tiles = static_cast<long long>(N) * ((Ctot + 31) / 32) * ((HW + 31) / 32);
+        const int grid = static_cast<int>(tiles < 148LL * 32 ? tiles : 148LL * 32);
+        if (elt == 2)
+            nchw_to_nhwc_tiled<2><<<grid, dim3(32, 8), 0, s>>>(src, dst, N, C, HW, groups, Cpg);
+        else
+            nchw_to_nhwc_tiled<4><<<grid, dim3(32, 8), 0, s>>>(src, dst, N, C, HW, groups, Cpg);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_nhwc_pad(const void *src, void *dst, int N, int C, int H, int W, int groups,
+                            int Cpg, int elt, cudaStream_t s) {
+    const long long pixels = static_cast<long long>(N) * H * W;
+    const long long total = pixels * groups * Cpg;
+    if (elt == 2)
+        nhwc_pad_kernel<2><<<grid_for(total), kThreads, 0, s>>>(src, dst, pixels, C, groups, Cpg);
+    else
+        nhwc_pad_kernel<4><<<grid_for(total), kThreads, 0, s>>>(src, dst, pixels, C, groups, Cpg);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_nhwc_to_nchw(const void *src, void *dst, int N, int C, int H, int W, int elt,
+                                cudaStream_t s) {
+    const int HW = H * W;
+    const long long tiles = static_cast<long long>(N) * ((C + 31) / 32) * ((HW + 31) / 32);
+    const int grid = static_cast<int>(tiles < 148LL * 32 ? tiles : 148LL * 32);
+    if (elt == 2)
+        nhwc_to_nchw_tiled<2><<<grid, dim3(32, 8), 0, s>>>(src, dst, N, C, HW);
+    else
+        nhwc_to_nchw_tiled<4><<<grid, dim3(32, 8), 0, s>>>(src, dst, N, C, HW);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_pack_weight(const void *w, void *wp, int Cout, int Cin_g, int Kh, int Kw,
+                               int Cpg, int elt, cudaStream_t s) {
+    const long long total = static_cast<long long>(Cout) * Kh * Kw * Cpg;
+    if (elt == 2)
+        pack_weight_kernel<2><<<grid_for(total), kThreads, 0, s>>>(w, wp, Cout, Cin_g, Kh, Kw, Cpg);
+    else
+        pack_weight_kernel<4><<<grid_for(total), kThreads, 0, s>>>(w, wp, Cout, Cin_g, Kh, Kw, Cpg);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_im2col(const void *x_nhwc, void *xcol, int N, int H, int W, int groups,
+                          int Cpg, int Ho, int Wo, int Kh, int Kw, int stride, int pad,
+                          int dilation, int elt, cudaStream_t s) {
+    const long long chunks = static_cast<long long>(N) * Ho * Wo * groups * Kh * Kw * Cpg * elt / 16;
+    if (elt == 2)
+        im2col_kernel<2><<<grid_for(chunks), kThreads, 0, s>>>(x_nhwc, xcol, N, H, W, groups, Cpg,
+                                                              Ho, Wo, Kh, Kw, stride, pad, dilation);
+    else
+        im2col_kernel<4><<<grid_for(chunks), kThreads, 0, s>>>(x_nhwc, xcol, N, H, W, groups, Cpg,
+                                                              Ho, Wo, Kh, Kw, stride, pad, dilation);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_splitk_reduce(const float *ws, const void *bias, void *y, int M, int Cout,
+                                 int HoWo, int splits, int out_mode, bool f32, cudaStream_t s) {
+    const long long total = static_cast<long long>(M) * Cout;
+    const int nchw = out_mode == kOutNCHW ? 1 : 0;
+    if (f32)
+        splitk_reduce_kernel<true><<<grid_for(total), kThreads, 0, s>>>(ws, bias, y, M, Cout, HoWo,
+                                                                        splits, nchw);
+    else
+        splitk_reduce_kernel<false><<<grid_for(total), kThreads, 0, s>>>(ws, bias, y, M, Cout, HoWo,
+                                                                         splits, nchw);
+    return cudaGetLastError();
+}
+
+}  // namespace conv2d_b200

@@ -1,0 +1,206 @@
+/*
+ * conv2d_b200.h -- C ABI of the B200 (sm_100a) 2-D convolution forward library.
+ *
+ * The operation is the 2-D convolution forward pass
+ *     y[n][oc][oh][ow] = bias[oc] + sum_{c < C_in/groups, kh < Kh, kw < Kw}
+ *         x[n][g*C_in/groups + c][oh*stride + kh*dilation - pad]
+ *                                [ow*stride + kw*dilation - pad] * w[oc][c][kh][kw]
+ * with g = oc / (C_out/groups) and terms whose input row or column falls outside
+ * the image dropped (zero padding).  Definition: "手撕 Conv2D" interview page
+ * (lpnh.cn/news/2493075) §1.1 (index map) and §2.1 (bounds-checked padding, bias
+ * added once per output); dilation per the same page §7; groups and shapes per
+ * "PyTorch高维张量乘法与conv2d/conv3d维度语义解析" (pwwt.cn/news/6111401) §4.1 and
+ * §4.3; output size per the same page §4.2.  The im2col + matrix-product view
+ * Y = W_row @ X_col is the one the im2col/GEMM tutorial (zskr.cn/news/1820658)
+ * §2.2-§2.3 gives; conv2d_forward computes that product without forming X_col.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Pointers named x, y, w_*, bias, workspace are DEVICE pointers owned by the
+ *   caller (cudaMalloc or any allocator of device memory); the library never
+ *   frees or keeps them.  Pointers named *_host are host pointers (pinned memory
+ *   gives asynchronous copies).  Every device pointer must be 16-byte aligned.
+ * - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every call
+ *   that takes a stream only enqueues work on it and returns; results are ready
+ *   once the stream reaches that point.  Device-side watchdog failures are
+ *   reported by conv2d_sync_status().
+ * - dtype CONV_BF16: x, w, bias and y hold bfloat16; products are accumulated
+ *   in fp32 and bias is added in fp32 before one round-to-nearest-even to bf16.
+ *   dtype CONV_F32: all tensors are fp32; the products run on tensor cores with
+ *   the three-term TF32 split (a*b ~ a_hi*b_hi + a_hi*b_lo + a_lo*b_hi) and
+ *   fp32 accumulation.
+ * - layout CONV_NCHW: x is (N, C_in, H, W) and y is (N, C_out, Ho, Wo).
+ *   layout CONV_NHWC: x is (N, H, W, C_in) and y is (N, Ho, Wo, C_out).
+ * - Stride, pad and dilation apply to both spatial dimensions; padding is zero
+ *   padding on both sides.
+ * - Every function returns a conv_status_t.  On any status other than CONV_OK
+ *   nothing has been enqueued and no output byte has been written;
+ *   conv2d_last_error() then returns a message for the calling thread.
+ */
+#ifndef CONV2D_B200_H
+#define CONV2D_B200_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t; declared here so that this header needs no CUDA header. */
+typedef struct CUstream_st *conv_stream_t;
+
+typedef enum {
+    CONV_OK = 0,
+    CONV_ERR_INVALID_ARG = 1, /* a shape, size or pointer argument is invalid   */
+    CONV_ERR_UNSUPPORTED = 2, /* valid, but outside what the kernels cover      */
+    CONV_ERR_CUDA = 3,        /* a CUDA runtime or driver call failed           */
+    CONV_ERR_TIMEOUT = 4,     /* a device-side wait ran out (see sync_status)   */
+    CONV_ERR_WORKSPACE = 5    /* the workspace passed in is too small           */
+} conv_status_t;
+
+typedef enum { CONV_F32 = 0, CONV_BF16 = 1 } conv_dtype_t;
+typedef enum { CONV_NHWC = 0, CONV_NCHW = 1 } conv_layout_t;
+
+/* Output extent along one spatial dimension,
+ *     *out = floor((in + 2*pad - dilation*(k - 1) - 1) / stride) + 1,
+ * the formula of "PyTorch高维张量乘法与conv2d/conv3d维度语义解析" §4.2 (and of the
+ * Conv2d documentation walk-through, dpshk.com/news/5792599, §3.2).
+ * CONV_ERR_INVALID_ARG if in, k, stride or dilation < 1, pad < 0, out is NULL,
+ * or the result would be below 1 (a negative numerator is rejected, not floored). */
+int conv2d_output_size(int in, int k, int stride, int pad, int dilation, int *out);
+
+/* Bytes of the packed weight buffer that conv2d_pack_weight writes:
+ * C_out * Kh * Kw * Cpg elements of dtype, where Cpg is C_in/groups rounded up
+ * to a multiple of 8 (bf16) or 4 (fp32). */
+int conv2d_packed_weight_size(int C_out, int C_in, int Kh, int Kw, int groups,
+                              conv_dtype_t dtype, size_t *bytes);
+
+/* Packs w_oihw (C_out, C_in/groups, Kh, Kw) -- the pages' weight layout
+ * ("PyTorch高维张量乘法..." §4.1) -- into the layout the kernels read: for each
+ * output channel the taps in (kh, kw) order, each tap's input channels
+ * contiguous and zero-padded to Cpg (the OHWI order the Conv2d documentation
+ * walk-through, dpshk.com/news/5792599, §5.2 describes for channels-last
+ * frameworks).  Done once per weight, outside the timed path.
+ * w_packed must hold conv2d_packed_weight_size() bytes; the two buffers must
+ * not overlap. */
+int conv2d_pack_weight(const void *w_oihw, void *w_packed, int C_out, int C_in,
+                       int Kh, int Kw, int groups, conv_dtype_t dtype,
+                       conv_stream_t stream);
+
+/* Device scratch bytes conv2d_forward needs for this problem (0 when none).
+ * Scratch holds a channels-last, channel-padded copy of x when layout is
+ * CONV_NCHW or C_in/groups is not a multiple of 8 (bf16) / 4 (fp32), and fp32
+ * partial sums when the reduction over C_in*Kh*Kw is split across SMs to fill
+ * the machine.  Arguments are validated as in conv2d_forward. */
+int conv2d_workspace_size(int N, int C_in, int H, int W, int C_out, int Kh, int Kw,
+                          int stride, int pad, int dilation, int groups,
+                          conv_dtype_t dtype, conv_layout_t layout, size_t *bytes);
+
+/* The convolution forward pass as an implicit matrix product that never forms
+ * the im2col matrix: rows are output pixels (N*Ho*Wo), columns output channels
+ * of a group, and the reduction runs over (kh, kw, c).  Input patches are staged
+ * tile by tile into shared memory by the tensor memory accelerator's im2col mode
+ * (out-of-image reads return zero: the zero padding), weights by tiled loads,
+ * tcgen05 tensor-core instructions accumulate in tensor memory, and the epilogue
+ * adds bias and stores y in `layout`.
+ *   x         : input, layout as above, dtype elements
+ *   w_packed  : weights from conv2d_pack_weight (same C_out, C_in, Kh, Kw, groups, dtype)
+ *   bias      : (C_out,) dtype elements, or NULL for no bias
+ *   y         : output, layout as above; must not overlap any input
+ *   workspace : at least conv2d_workspace_size() bytes (may be NULL when that is 0)
+ * Errors: CONV_ERR_INVALID_ARG for a non-positive size, stride < 1, dilation < 1,
+ * pad < 0, C_in or C_out not divisible by groups (pwwt §4.3), an empty output,
+ * or a NULL x / w_packed / y; CONV_ERR_WORKSPACE when workspace_bytes is too
+ * small; CONV_ERR_UNSUPPORTED for a misaligned pointer, stride > 8,
+ * pad > 127, dilation*(K-1) - pad outside [-128, 127] (limits of the hardware
+ * im2col addressing), or C_in/groups not a multiple of 8 (bf16) / 4 (fp32)
+ * when groups > 1; CONV_ERR_CUDA if the launch fails. */
+int conv2d_forward(const void *x, const void *w_packed, const void *bias, void *y,
+                   int N, int C_in, int H, int W, int C_out, int Kh, int Kw,
+                   int stride, int pad, int dilation, int groups,
+                   conv_dtype_t dtype, conv_layout_t layout,
+                   void *workspace, size_t workspace_bytes, conv_stream_t stream);
+
+/* Device scratch bytes conv2d_forward_im2col_gemm needs: the explicit im2col
+ * matrix (N*Ho*Wo rows of groups*Kh*Kw*Cpg elements) plus what conv2d_forward
+ * would need. */
+int conv2d_im2col_workspace_size(int N, int C_in, int H, int W, int C_out, int Kh,
+                                 int Kw, int stride, int pad, int dilation,
+                                 int groups, conv_dtype_t dtype, conv_layout_t layout,
+                                 size_t *bytes);
+
+/* The pages' own formulation, kept as a comparison point: an im2col kernel
+ * writes X_col (one row per output pixel, (kh, kw, c) along the row -- the
+ * transpose of zskr §2.2's column matrix) into the workspace, then the same
+ * tensor-core matrix product Y = X_col * W_row^T + bias runs over it (zskr
+ * §2.3, lpnh §4.2).  Arguments and errors as conv2d_forward; the workspace must
+ * hold conv2d_im2col_workspace_size() bytes. */
+int conv2d_forward_im2col_gemm(const void *x, const void *w_packed, const void *bias,
+                               void *y, int N, int C_in, int H, int W, int C_out,
+                               int Kh, int Kw, int stride, int pad, int dilation,
+                               int groups, conv_dtype_t dtype, conv_layout_t layout,
+                               void *workspace, size_t workspace_bytes,
+                               conv_stream_t stream);
+
+/* End-to-end call for host-resident activations: enqueues on `stream` the copy
+ * of x_host into x_dev, conv2d_forward(x_dev, ...) into y_dev, and the copy of
+ * y_dev back into y_host.  x_host/y_host are host buffers of the x and y sizes
+ * (pinned for asynchronous copies); x_dev/y_dev are caller-owned device buffers
+ * of the same sizes.  Weights and bias stay resident on the device.  Returns
+ * after enqueuing; y_host is valid once the stream is synchronised.  Errors as
+ * conv2d_forward. */
+int conv2d_forward_hostio(const void *x_host, void *y_host, void *x_dev, void *y_dev,
+                          const void *w_packed, const void *bias,
+                          int N, int C_in, int H, int W, int C_out, int Kh, int Kw,
+                          int stride, int pad, int dilation, int groups,
+                          conv_dtype_t dtype, conv_layout_t layout,
+                          void *workspace, size_t workspace_bytes,
+                          conv_stream_t stream);
+
+/* Layout change NCHW -> channels-last: dst[n][h][w][g*Cpg + c] = src[n][g*Cg + c][h][w]
+ * for c < Cg = C/groups and zero for Cg <= c < Cpg (Cpg >= Cg).  This is the
+ * "layout in" step for NCHW callers (pwwt §6.3 on channels_last; zero channels
+ * make every pixel row a multiple of 16 bytes).  dst holds N*H*W*groups*Cpg
+ * elements. */
+int conv2d_nchw_to_nhwc(const void *src, void *dst, int N, int C, int H, int W,
+                        int groups, int Cpg, conv_dtype_t dtype, conv_stream_t stream);
+
+/* Layout change channels-last -> NCHW: dst[n][c][h][w] = src[n][h][w][c]
+ * (the final transpose of zskr §3.2 step 5). */
+int conv2d_nhwc_to_nchw(const void *src, void *dst, int N, int C, int H, int W,
+                        conv_dtype_t dtype, conv_stream_t stream);
+
+/* Waits for `stream`, then reports and clears the device watchdog status:
+ * CONV_ERR_TIMEOUT if a kernel of this library gave up on a wait since the
+ * last call (its output is then incomplete), CONV_ERR_CUDA if the stream
+ * reported an error, else CONV_OK. */
+int conv2d_sync_status(conv_stream_t stream);
+
+/* Message describing the last non-OK status returned on the calling thread
+ * (empty string if none).  The pointer stays valid until the thread's next call. */
+const char *conv2d_last_error(void);
+
+/* Measurement aid: when `start` and `stop` (cudaEvent_t handles the caller created
+ * with timing enabled) are both non-NULL, every later forward call records `start`
+ * on its stream immediately before launching its tensor-core kernel and `stop`
+ * immediately after it, so that the caller can time that kernel alone inside a
+ * longer sequence of work.  Passing NULL, NULL turns this off.  The setting is
+ * per process; events are only recorded, never waited on. */
+int conv2d_set_main_kernel_events(void *start, void *stop);
+
+/* Total number of kernels this library has launched (or, under stream capture,
+ * added to a graph) in this process, written to *count. */
+int conv2d_kernel_launch_count(unsigned long long *count);
+
+/* Test hook for the watchdog: every later launch uses `timeout_ns` as the limit
+ * of each device-side wait (<= 0 restores the default of 2 s) and, if
+ * `starve_loads` is non-zero, issues no input loads, so the waits for them run
+ * out.  Used only by the tests that check that a kernel returns an error status
+ * instead of hanging. */
+int conv2d_debug_set_watchdog(long long timeout_ns, int starve_loads);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CONV2D_B200_H */

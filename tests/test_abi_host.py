@@ -1,0 +1,118 @@
+"""The C-ABI library on the host, without a GPU: it loads, exports every function the
+header declares, and rejects invalid arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import cnn_convolution_conv2d_b200 as cb
+import oracle_pins
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "conv2d_b200.h")
+
+
+def declared_functions():
+    text = open(HEADER, encoding="utf-8").read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(conv2d_\w+)\s*\(", text, flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from cnn_convolution_conv2d_b200 import build
+    build.build()
+    return cb.load()
+
+
+def test_header_declares_the_abi():
+    names = declared_functions()
+    assert "conv2d_forward" in names and "conv2d_sync_status" in names
+    assert set(names) == set(cb.SIGNATURES), set(names) ^ set(cb.SIGNATURES)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_output_size_matches_the_pages(lib):
+    for size, k, s, p, d, expected, src in oracle_pins.read_output_size_cases():
+        out = ctypes.c_int(-7)
+        st = lib.conv2d_output_size(size, k, s, p, d, ctypes.byref(out))
+        if expected < 0:
+            assert st == cb.CONV_ERR_INVALID_ARG, src
+        else:
+            assert st == cb.CONV_OK and out.value == expected, (src, st, out.value)
+
+
+@pytest.mark.parametrize("args", [
+    (0, 3, 1, 0, 1), (5, 0, 1, 0, 1), (5, 3, 0, 0, 1), (5, 3, 1, -1, 1), (5, 3, 1, 0, 0),
+    (2, 5, 1, 0, 1),  # kernel larger than the input
+])
+def test_output_size_rejects(lib, args):
+    out = ctypes.c_int(0)
+    assert lib.conv2d_output_size(*args, ctypes.byref(out)) == cb.CONV_ERR_INVALID_ARG
+    assert cb.conv2d_last_error()
+
+
+def test_packed_weight_size(lib):
+    assert cb.conv2d_packed_weight_size(64, 3, 7, 7, 1, cb.CONV_BF16) == 64 * 49 * 8 * 2
+    assert cb.conv2d_packed_weight_size(4, 3, 3, 3, 1, cb.CONV_F32) == 4 * 9 * 4 * 4
+    assert cb.conv2d_packed_weight_size(512, 512, 3, 3, 32, cb.CONV_BF16) == 512 * 9 * 16 * 2
+    with pytest.raises(cb.Conv2dError):
+        cb.conv2d_packed_weight_size(6, 4, 3, 3, 4, cb.CONV_BF16)   # C_out % groups
+
+
+GOOD = dict(N=2, C_in=8, H=9, W=9, C_out=16, Kh=3, Kw=3, stride=1, pad=1, dilation=1, groups=1)
+BAD = [
+    dict(N=0), dict(C_in=0), dict(H=0), dict(W=-1), dict(C_out=0), dict(Kh=0), dict(Kw=0),
+    dict(stride=0), dict(pad=-1), dict(dilation=0), dict(groups=0), dict(groups=3),
+    dict(C_out=12, groups=8),  # C_out % groups
+    dict(Kh=12),               # empty output
+    dict(H=2, W=2, pad=0),     # kernel larger than the image
+]
+
+
+def _call_forward(lib, shape, x=16, w=16, y=16, dtype=cb.CONV_BF16, layout=cb.CONV_NHWC):
+    s = dict(GOOD, **shape)
+    return lib.conv2d_forward(x, w, None, y, s["N"], s["C_in"], s["H"], s["W"], s["C_out"], s["Kh"],
+                              s["Kw"], s["stride"], s["pad"], s["dilation"], s["groups"], dtype,
+                              layout, None, 0, None)
+
+
+@pytest.mark.parametrize("shape", BAD, ids=lambda d: ",".join(f"{k}={v}" for k, v in d.items()))
+def test_forward_rejects_invalid_shapes(lib, shape):
+    assert _call_forward(lib, shape) == cb.CONV_ERR_INVALID_ARG
+    assert cb.conv2d_last_error()
+
+
+def test_forward_rejects_null_pointers_and_bad_enums(lib):
+    assert _call_forward(lib, {}, x=None) == cb.CONV_ERR_INVALID_ARG
+    assert _call_forward(lib, {}, w=None) == cb.CONV_ERR_INVALID_ARG
+    assert _call_forward(lib, {}, y=None) == cb.CONV_ERR_INVALID_ARG
+    assert _call_forward(lib, {}, dtype=7) == cb.CONV_ERR_INVALID_ARG
+    assert _call_forward(lib, {}, layout=5) == cb.CONV_ERR_INVALID_ARG
+
+
+def test_forward_reports_unsupported_limits(lib):
+    assert _call_forward(lib, dict(stride=9, H=40, W=40)) == cb.CONV_ERR_UNSUPPORTED
+    assert _call_forward(lib, dict(pad=128, H=4, W=4)) == cb.CONV_ERR_UNSUPPORTED
+
+
+def test_workspace_size_without_device(lib):
+    # channels-last input with C_in a multiple of 8: no scratch at all
+    assert cb.conv2d_workspace_size(2, 8, 9, 9, 16, 3, 3, 1, 1, 1, 1, cb.CONV_BF16, "nhwc") == 0
+    # NCHW input: a channels-last copy padded to 8 channels
+    assert cb.conv2d_workspace_size(2, 3, 9, 9, 16, 3, 3, 1, 1, 1, 1, cb.CONV_BF16, "nchw") >= 2 * 9 * 9 * 8 * 2
+    # explicit im2col adds X_col: M rows of Kh*Kw*Cpg elements
+    xcol = 2 * 9 * 9 * 9 * 8 * 2
+    assert cb.conv2d_im2col_workspace_size(2, 8, 9, 9, 16, 3, 3, 1, 1, 1, 1, cb.CONV_BF16, "nhwc") >= xcol
+    with pytest.raises(cb.Conv2dError):
+        cb.conv2d_workspace_size(2, 8, 9, 9, 16, 3, 3, 1, 1, 1, 3, cb.CONV_BF16, "nhwc")
+
+
+def test_watchdog_hook_accepts_settings(lib):
+    cb.conv2d_debug_set_watchdog(1000, False)
+    cb.conv2d_debug_set_watchdog(0, False)   # back to the default

@@ -1,0 +1,214 @@
+"""CUDA path vs the fp64 oracle, element by element, through the C ABI (needs a B200).
+
+Small cases span several 128-row tiles with a ragged last tile and finish in the
+oracle within seconds; full-size cases run in the launch configuration the
+benchmark times and are checked on sampled outputs plus every corner."""
+import numpy as np
+import pytest
+
+import cnn_convolution_conv2d_b200 as cb
+from cnn_convolution_conv2d_b200 import workloads
+import oracle
+import parity
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def cuda_ready():
+    import torch
+    assert torch.cuda.is_available(), "these tests need a CUDA device (run with -m 'not gpu' on CPU)"
+    from cnn_convolution_conv2d_b200 import build
+    build.build()
+    cb.load()
+    cb.conv2d_debug_set_watchdog(0, False)
+    yield
+    cb.conv2d_sync_status()
+
+
+SMALL = {  # oracle-sized versions of every workload (same seeds and distributions)
+    "tiny_f32_nchw": {},
+    "stem_bf16": dict(N=2, H=62, W=62),                        # M = 1922: 16 tiles, 2 rows in the last
+    "resnet3x3_bf16_nhwc": dict(N=2, H=20, W=20),              # M = 800
+    "pointwise1x1_bf16": dict(N=2, H=20, W=20),                # 4 column tiles of 256
+    "grouped_dilated_bf16": dict(N=2),                         # 32 groups x 16 channels, s2 p2 d2
+    "grouped_dilated_f32": dict(N=2),
+    "k7_17x17_bf16": dict(N=1, C_in=128, C_out=128),           # split reduction across SMs
+    "k7_17x17_f32": dict(N=1, C_in=128, C_out=128),
+}
+
+
+@pytest.mark.parametrize("name", sorted(SMALL))
+def test_small_workloads(name):
+    cfg = parity.config(name, **SMALL[name])
+    inp = workloads.make_inputs(cfg)
+    ref = parity.run_oracle(cfg, inp)
+    got = parity.run_gpu(cfg, inp)
+    parity.assert_close(cfg, got, ref, name)
+
+
+@pytest.mark.parametrize("name", sorted(SMALL))
+def test_small_workloads_other_layout(name):
+    base = parity.config(name, **SMALL[name])
+    cfg = base.scaled(layout="nhwc" if base.layout == "nchw" else "nchw")
+    inp = workloads.make_inputs(cfg)
+    parity.assert_close(cfg, parity.run_gpu(cfg, inp), parity.run_oracle(cfg, inp), name)
+
+
+@pytest.mark.parametrize("name", ["tiny_f32_nchw", "stem_bf16", "resnet3x3_bf16_nhwc",
+                                  "grouped_dilated_bf16", "k7_17x17_f32"])
+def test_explicit_im2col_gemm(name):
+    cfg = parity.config(name, **SMALL[name])
+    inp = workloads.make_inputs(cfg)
+    ref = parity.run_oracle(cfg, inp)
+    got = parity.run_gpu(cfg, inp, explicit_im2col=True)
+    parity.assert_close(cfg, got, ref, name + " (explicit im2col)")
+
+
+EDGE = [  # N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups
+    (1, 8, 1, 1, 16, 1, 1, 1, 0, 1, 1),      # a single pixel
+    (1, 3, 1, 1, 4, 3, 3, 2, 1, 1, 1),       # single pixel, only the centre tap in the image
+    (3, 5, 13, 11, 40, 3, 3, 1, 1, 1, 1),    # odd C_in, C_out not a multiple of 16
+    (2, 12, 10, 14, 24, 3, 5, 2, 2, 1, 1),   # non-square kernel, stride 2
+    (2, 16, 15, 15, 32, 3, 3, 3, 4, 3, 1),   # stride 3, dilation 3, large pad
+    (2, 64, 9, 9, 48, 1, 1, 2, 0, 1, 1),     # 1x1 with stride 2
+    (1, 24, 12, 12, 36, 3, 3, 1, 1, 1, 4),   # groups with 6 input / 9 output channels each
+    (2, 64, 8, 8, 64, 3, 3, 1, 1, 2, 8),     # 8 channels per group, dilation 2
+    (1, 32, 30, 30, 8, 5, 5, 1, 0, 1, 1),    # C_out 8 < one 16-wide column tile
+    (1, 96, 7, 9, 200, 2, 2, 1, 0, 1, 1),    # even kernel, C_out not a multiple of the tile
+    (1, 16, 40, 3, 16, 7, 1, 8, 3, 1, 1),    # stride 8 (the largest supported), thin image
+    (5, 8, 6, 6, 16, 3, 3, 1, 1, 1, 1),      # several images inside one 128-row tile
+]
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("layout", ["nhwc", "nchw"])
+@pytest.mark.parametrize("shape", EDGE, ids=lambda s: "x".join(map(str, s)))
+def test_edge_shapes(shape, layout, dtype):
+    N, C_in, H, W, C_out, Kh, Kw, s, p, d, g = shape
+    cfg = workloads.ConvConfig("edge", N, C_in, H, W, C_out, Kh, Kw, s, p, d, g, True, dtype, layout,
+                               seed=sum(shape))
+    inp = workloads.make_inputs(cfg)
+    parity.assert_close(cfg, parity.run_gpu(cfg, inp), parity.run_oracle(cfg, inp), str(shape))
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("explicit", [False, True])
+@pytest.mark.parametrize("shape", [(2, 3, 9, 11, 4, 3, 3, 2, 1, 1, 1), (2, 16, 12, 12, 32, 3, 3, 1, 1, 1, 1),
+                                   (1, 32, 10, 10, 64, 3, 3, 1, 1, 2, 4)],
+                         ids=lambda s: "x".join(map(str, s)))
+def test_small_integers_bit_exact(shape, explicit, dtype):
+    """Integer inputs in [-2, 2]: every partial sum is exact, so outputs match exactly."""
+    N, C_in, H, W, C_out, Kh, Kw, s, p, d, g = shape
+    cfg = workloads.ConvConfig("ints", N, C_in, H, W, C_out, Kh, Kw, s, p, d, g, True, dtype, "nhwc",
+                               ("integers", -2, 2), ("integers", -2, 2), ("integers", -2, 2), seed=7)
+    inp = workloads.make_inputs(cfg)
+    ref = parity.run_oracle(cfg, inp)
+    assert np.abs(ref).max() <= 256  # exactly representable in bf16 as well
+    got = parity.run_gpu(cfg, inp, explicit_im2col=explicit)
+    assert np.array_equal(got, ref)
+
+
+FULL = ["stem_bf16", "resnet3x3_bf16_nhwc", "pointwise1x1_bf16", "grouped_dilated_bf16",
+        "grouped_dilated_f32", "k7_17x17_bf16", "k7_17x17_f32", "tiny_f32_nchw"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_sampled(name):
+    import torch
+    cfg = workloads.CONFIGS[name]
+    inp = workloads.make_inputs(cfg)
+    layer = parity.make_layer(cfg, inp)
+    y = layer(parity.to_device_x(cfg, inp["x"]))
+    cb.conv2d_sync_status()
+    shape = (cfg.N, cfg.C_out, cfg.Ho, cfg.Wo)
+    assert tuple(y.shape) == (shape if cfg.layout == "nchw" else (cfg.N, cfg.Ho, cfg.Wo, cfg.C_out))
+    assert bool(torch.isfinite(y).all())
+    idx = parity.sample_indices(shape, 512, seed=99)
+    n, oc, oh, ow = (torch.from_numpy(idx[:, i]).cuda() for i in range(4))
+    got = (y[n, oc, oh, ow] if cfg.layout == "nchw" else y[n, oh, ow, oc]).float().cpu().numpy()
+    ref = oracle.conv2d_points(inp["x"], inp["w"], inp["b"], idx, cfg.stride, cfg.pad, cfg.dilation,
+                               cfg.groups)
+    if cfg.dtype == "f32":
+        err = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+        assert err <= parity.F32_NORMWISE, err
+    else:
+        assert np.abs(got - ref).max() <= parity.BF16_MAXABS * np.abs(ref).max()
+
+
+def test_layout_kernels_round_trip():
+    import torch
+    x = torch.randn(3, 5, 7, 9, dtype=torch.float32).to(torch.bfloat16).cuda()
+    nhwc = torch.empty(3, 7, 9, 8, dtype=torch.bfloat16, device="cuda")
+    cb.conv2d_nchw_to_nhwc(x, nhwc, 3, 5, 7, 9, 1, 8, cb.CONV_BF16)
+    back = torch.empty_like(x)
+    cb.conv2d_nhwc_to_nchw(nhwc[..., :5].contiguous(), back, 3, 5, 7, 9, cb.CONV_BF16)
+    cb.conv2d_sync_status()
+    assert torch.equal(back, x)
+    assert torch.equal(nhwc[..., :5], x.permute(0, 2, 3, 1))
+    assert bool((nhwc[..., 5:] == 0).all())
+    # wide channel counts take the shared-memory tiled path
+    x2 = torch.randn(2, 70, 33, 31, dtype=torch.float32).cuda()
+    y2 = torch.empty(2, 33, 31, 70, dtype=torch.float32, device="cuda")
+    cb.conv2d_nchw_to_nhwc(x2, y2, 2, 70, 33, 31, 1, 70, cb.CONV_F32)
+    b2 = torch.empty_like(x2)
+    cb.conv2d_nhwc_to_nchw(y2, b2, 2, 70, 33, 31, cb.CONV_F32)
+    cb.conv2d_sync_status()
+    assert torch.equal(y2, x2.permute(0, 2, 3, 1)) and torch.equal(b2, x2)
+
+
+def test_pack_weight_layout():
+    import torch
+    w = torch.randn(6, 3, 2, 5, dtype=torch.float32).cuda()
+    wp = cb.conv2d_pack_weight(w, groups=1)
+    cb.conv2d_sync_status()
+    ref = torch.zeros(6, 2, 5, 4, device="cuda")
+    ref[..., :3] = w.permute(0, 2, 3, 1)
+    assert torch.equal(wp.view(6, 2, 5, 4), ref)
+
+
+def test_hostio_matches_device_call():
+    import torch
+    cfg = parity.config("stem_bf16", N=2, H=62, W=62)
+    inp = workloads.make_inputs(cfg)
+    layer = parity.make_layer(cfg, inp)
+    x_dev = parity.to_device_x(cfg, inp["x"])
+    y_dev_ref = layer(x_dev)
+    x_host = x_dev.cpu().pin_memory()
+    y_host = torch.empty(y_dev_ref.shape, dtype=y_dev_ref.dtype).pin_memory()
+    x2 = torch.empty_like(x_dev)
+    y2 = torch.empty_like(y_dev_ref)
+    layer.forward_hostio(x_host, y_host, x2, y2)
+    cb.conv2d_sync_status()
+    assert torch.equal(y_host, y_dev_ref.cpu())
+
+
+def test_repeated_calls_are_identical():
+    import torch
+    cfg = parity.config("k7_17x17_bf16", N=1, C_in=128, C_out=128)
+    inp = workloads.make_inputs(cfg)
+    layer = parity.make_layer(cfg, inp)
+    x = parity.to_device_x(cfg, inp["x"])
+    a = layer(x)
+    b = layer(x)
+    cb.conv2d_sync_status()
+    assert torch.equal(a, b)
+
+
+def test_watchdog_returns_timeout_instead_of_hanging():
+    """With loads withheld, every wait in the kernel runs out after 1 ms; the kernel
+    exits, the status reads TIMEOUT, and the next normal call works."""
+    cfg = parity.config("resnet3x3_bf16_nhwc", N=1, H=12, W=12)
+    inp = workloads.make_inputs(cfg)
+    layer = parity.make_layer(cfg, inp)
+    x = parity.to_device_x(cfg, inp["x"])
+    try:
+        cb.conv2d_debug_set_watchdog(1_000_000, True)
+        layer(x)
+        with pytest.raises(cb.Conv2dError) as err:
+            cb.conv2d_sync_status()
+        assert err.value.status == cb.CONV_ERR_TIMEOUT
+    finally:
+        cb.conv2d_debug_set_watchdog(0, False)
+    cb.conv2d_sync_status()  # status was cleared
+    parity.assert_close(cfg, parity.run_gpu(cfg, inp, layer=layer), parity.run_oracle(cfg, inp), "after timeout")
