@@ -1,0 +1,503 @@
+#!/usr/bin/env python
+"""Throughput of the conv2d forward hot path on B200 -- prints ONE JSON line (rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the whole forward path over one batch of the workload:
+output-size computation, the layout-in copy (NCHW -> channels-last, channels padded),
+the implicit-GEMM tensor-core kernel (patch gather, weight tiles, product, bias
+epilogue) and the NCHW output store -- one call of the C ABI's conv2d_forward.
+The default workload is the first-layer ("stem") convolution, 32x3x224x224 ->
+64 channels, 7x7, stride 2, pad 3, bf16.
+
+Timing: W untimed warm-up steps, then exactly K steps, captured as CUDA graphs
+of G steps each and replayed, bracketed by a barrier and a device synchronise on
+both sides and timed with CUDA events on the launching stream (max over ranks).
+Consecutive steps rotate over several input/output sets whose total size is more
+than twice the 126 MB L2, so no step finds its input in L2.  The tensor-core
+kernel is timed separately by events recorded around each of its launches.
+SM clocks and throttle reasons are sampled through NVML during the timed region.
+
+Multi-GPU (torchrun): every rank runs its own batch (different seed), nothing is
+exchanged on the data path; `value` is the work of all ranks over the slowest
+rank's time (weak scaling).
+
+--impl reference times the CPU oracle (fp64, OpenMP) on bounded samples of the
+same workload, as the comparison arm; on torchrun only rank 0 runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+DEFAULT_WORKLOAD = "stem_bf16"
+L2_BYTES = 126 * 1000 * 1000
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ["igemm.cu", "ptx.cuh", "common.cuh"]
+
+
+# ------------------------------------------------------------ arithmetic ---
+def flops(cfg) -> float:
+    """Algorithmic FLOPs of one forward pass: 2*N*C_out*Ho*Wo*(C_in/groups)*Kh*Kw
+    ("PyTorch高维张量乘法与conv2d/conv3d维度语义解析" §3.3); padding taps included,
+    channel padding and split-K partial sums not."""
+    return 2.0 * cfg.N * cfg.C_out * cfg.Ho * cfg.Wo * (cfg.C_in // cfg.groups) * cfg.Kh * cfg.Kw
+
+
+def elt_bytes(cfg) -> int:
+    return 2 if cfg.dtype == "bf16" else 4
+
+
+def step_bytes(cfg) -> float:
+    """Minimum bytes a whole step must move: x, w, bias read once, y written once."""
+    e = elt_bytes(cfg)
+    return e * (cfg.N * cfg.C_in * cfg.H * cfg.W + cfg.C_out * (cfg.C_in // cfg.groups) * cfg.Kh * cfg.Kw
+                + (cfg.C_out if cfg.bias else 0) + cfg.N * cfg.C_out * cfg.Ho * cfg.Wo)
+
+
+def padded_channels(cfg) -> int:
+    align = 16 // elt_bytes(cfg)
+    cg = cfg.C_in // cfg.groups
+    return (cg + align - 1) // align * align
+
+
+def uses_gather(cfg) -> bool:
+    """Mirrors the library's choice of the software-gather kernel: one group, fewer
+    than 32 bytes of input channels per pixel, a reduction that fits its tables."""
+    e = elt_bytes(cfg)
+    per16 = 16 // e
+    vec = cfg.layout == "nchw" and cfg.dilation == 1 and (cfg.W * e) % 16 == 0 and cfg.Kw <= per16
+    kc = cfg.C_in * cfg.Kh * (per16 if vec else cfg.Kw)
+    kpad = -(-kc // (32 // e)) * (32 // e)
+    return cfg.groups == 1 and cfg.C_in * e < 32 and kpad <= 256 and cfg.C_out <= (256 if e == 2 else 128)
+
+
+def main_kernel_bytes(cfg) -> float:
+    """Minimum bytes the tensor-core kernel itself moves per launch: its input (x
+    itself for the gather kernel, else the channels-last input or its channel-padded
+    copy when the step makes one), the packed weights, the bias, and the output."""
+    e = elt_bytes(cfg)
+    cpg = padded_channels(cfg)
+    copy = (cfg.layout == "nchw" or cpg != cfg.C_in // cfg.groups) and not uses_gather(cfg)
+    x_in = cfg.N * cfg.H * cfg.W * (cfg.groups * cpg if copy else cfg.C_in)
+    w = cfg.C_out * cfg.Kh * cfg.Kw * cpg
+    return e * (x_in + w + (cfg.C_out if cfg.bias else 0) + cfg.N * cfg.C_out * cfg.Ho * cfg.Wo)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except (OSError, ValueError, KeyError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "cnn_convolution_conv2d_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(workload: str):
+    """DRAM bytes per launch of the tensor-core kernel from the committed ncu summary,
+    or None when there is none or the kernel source changed since it was taken."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            d = json.load(f).get(workload)
+    except (OSError, ValueError):
+        return None
+    if not d or d.get("kernel_hash") != kernel_source_hash():
+        return None
+    return float(d["dram_bytes_per_launch"])
+
+
+def roofline(cfg, kernel_ms: float, peaks, peak_kind: str, workload: str) -> dict:
+    f = flops(cfg)
+    b = main_kernel_bytes(cfg)
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if f / b >= ridge and cfg.dtype == "bf16":
+        achieved = f / (kernel_ms * 1e-3) / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        out = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+               "peak_source": f"{peak_kind} bf16 sustained (kernel timed inside a long run)"}
+    else:
+        achieved = b / (kernel_ms * 1e-3) / 1e9
+        peak = peaks["hbm_gbs"]
+        out = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+               "peak_source": f"{peak_kind} HBM copy bandwidth"}
+    out["frac"] = achieved / peak
+    out["kernel"] = ("gather_kernel (software-gathered im2col rows, tcgen05)" if uses_gather(cfg)
+                     else "igemm_kernel (hardware im2col TMA, tcgen05)")
+    out["kernel_ms"] = kernel_ms
+    out["algorithmic_bytes_per_launch"] = b
+    out["algorithmic_flops_per_launch"] = f
+    out["traffic"] = committed_traffic(workload)
+    return out
+
+
+# ---------------------------------------------------------------- clocks ---
+class ClockSampler:
+    """Polls SM clock and throttle reasons through NVML (what nvidia-smi reads)."""
+
+    REASONS = {  # NVML clocks-event reason bits
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index: int, interval_s: float = 0.005):
+        self.samples = []
+        self.interval = interval_s
+        self.error = None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            import torch
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+            self.handle = pynvml.nvmlDeviceGetHandleByUUID(uuid.encode())
+            self.nvml = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+        except Exception as exc:  # no NVML: report why instead of numbers
+            self.error = f"NVML unavailable: {exc}"
+            self.handle = None
+        self._thread = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        nv = self.nvml
+        while not self._stop.is_set():
+            try:
+                t = time.perf_counter()
+                mhz = nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)
+                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                self.samples.append((t, mhz, reasons))
+            except Exception as exc:
+                self.error = str(exc)
+                return
+            time.sleep(self.interval)
+
+    def start(self):
+        if self.handle is not None:
+            self._thread.start()
+
+    def stop(self):
+        self._stop.set()
+        if self._thread.is_alive():
+            self._thread.join()
+
+    def summary(self, t0: float, t1: float) -> dict:
+        if self.handle is None:
+            return {"error": self.error}
+        window = [s for s in self.samples if t0 <= s[0] <= t1]
+        if not window:  # region shorter than one polling interval: nearest sample
+            window = sorted(self.samples, key=lambda s: abs(s[0] - (t0 + t1) / 2))[:1]
+        if not window:
+            return {"error": self.error or "no samples"}
+        mask = 0
+        for s in window:
+            mask |= s[2]
+        reasons = [name for bit, name in self.REASONS.items() if mask & bit and name != "gpu_idle"]
+        return {"sm_mhz": statistics.median(s[1] for s in window), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(window)}
+
+
+# ----------------------------------------------------------- distributed ---
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def max_over_ranks(value: float, world: int, device) -> float:
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------ CPU oracle ---
+def oracle_rate_sample(cfg, inp, seconds: float, seed: int = 1234, max_points=None):
+    """Times the fp64 oracle on random output points of the workload for about
+    `seconds`; returns (flop_per_s, points, wall_s, threads)."""
+    import numpy as np
+    import oracle
+    rng = np.random.default_rng(seed)
+    shape = (cfg.N, cfg.C_out, cfg.Ho, cfg.Wo)
+    per_point = 2.0 * (cfg.C_in // cfg.groups) * cfg.Kh * cfg.Kw
+    x64 = inp["x"].astype(np.float64)
+    w64 = inp["w"].astype(np.float64)
+    b64 = None if inp["b"] is None else inp["b"].astype(np.float64)
+
+    def run(points):
+        idx = np.stack([rng.integers(0, n, points) for n in shape], axis=1)
+        t = time.perf_counter()
+        oracle.conv2d_points(x64, w64, b64, idx, cfg.stride, cfg.pad, cfg.dilation, cfg.groups)
+        return time.perf_counter() - t
+
+    probe = 2000
+    dt = max(run(probe), 1e-4)
+    points = int(probe * seconds / dt)
+    total = cfg.N * cfg.C_out * cfg.Ho * cfg.Wo
+    points = max(1, min(points, total, max_points or total))
+    wall = run(points)
+    return points * per_point / wall, points, wall, oracle.num_threads()
+
+
+def run_reference(args, cfg):
+    """The comparison arm: the oracle as it stands on this machine's host cores."""
+    import numpy as np
+    from cnn_convolution_conv2d_b200 import workloads
+    inp = workloads.make_inputs(cfg)
+    per_point = 2.0 * (cfg.C_in // cfg.groups) * cfg.Kh * cfg.Kw
+    budget = 90.0 / max(1, args.steps + args.warmup)  # whole run: about a minute and a half
+    rate, _, _, threads = oracle_rate_sample(cfg, inp, min(budget, 2.0))
+    points = max(64, int(budget * rate / per_point))
+    import oracle
+    rng = np.random.default_rng(7)
+    shape = (cfg.N, cfg.C_out, cfg.Ho, cfg.Wo)
+    x64, w64 = inp["x"].astype(np.float64), inp["w"].astype(np.float64)
+    b64 = None if inp["b"] is None else inp["b"].astype(np.float64)
+    idx = [np.stack([rng.integers(0, n, points) for n in shape], axis=1)
+           for _ in range(args.steps + args.warmup)]
+    for i in range(args.warmup):
+        oracle.conv2d_points(x64, w64, b64, idx[i], cfg.stride, cfg.pad, cfg.dilation, cfg.groups)
+    t = time.perf_counter()
+    for i in range(args.warmup, args.warmup + args.steps):
+        oracle.conv2d_points(x64, w64, b64, idx[i], cfg.stride, cfg.pad, cfg.dilation, cfg.groups)
+    wall = time.perf_counter() - t
+    value = args.steps * points * per_point / wall / 1e12
+    sample = (f"{points} random output points per step of {cfg.name} "
+              f"({points / (cfg.N * cfg.C_out * cfg.Ho * cfg.Wo):.2e} of one forward pass)")
+    line = {
+        "impl": "reference", "metric": metric_name(cfg), "value": value, "unit": "TFLOP/s",
+        "n_gpus": 0, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": wall / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(cfg, args, world=1),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------- our path ---
+def metric_name(cfg) -> str:
+    return "conv2d fwd TFLOP/s on 1 B200 and % of dense tensor (or HBM) roofline"
+
+
+def workload_config(cfg, args, world: int) -> dict:
+    desc = (f"{cfg.name}: N={cfg.N} C_in={cfg.C_in} {cfg.H}x{cfg.W} -> C_out={cfg.C_out}, "
+            f"{cfg.Kh}x{cfg.Kw} s{cfg.stride} p{cfg.pad} d{cfg.dilation} g{cfg.groups}, "
+            f"{'bias' if cfg.bias else 'no bias'}, {cfg.dtype}, {cfg.layout.upper()} in/out")
+    return {"workload": desc, "global_batch": cfg.N * world, "per_gpu_batch": cfg.N,
+            "flop_per_step_per_gpu": flops(cfg),
+            "parallelism": f"replicas x{world} (batch shards, no collective on the data path)"}
+
+
+def run_ours(args, cfg):
+    import numpy as np
+    import torch
+
+    import cnn_convolution_conv2d_b200 as cb
+    from cnn_convolution_conv2d_b200 import build, workloads
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=device)
+    if rank == 0:
+        build.build()
+    barrier(world)
+    cb.load()
+
+    inp = workloads.make_inputs(cfg, seed=cfg.seed + 1000 * rank)
+    dt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+    x_host = torch.from_numpy(inp["x"]).to(dt)
+    if cfg.layout == "nhwc":
+        x_host = x_host.permute(0, 2, 3, 1).contiguous()
+    w = torch.from_numpy(inp["w"]).to(dt).to(device)
+    b = None if inp["b"] is None else torch.from_numpy(inp["b"]).to(dt).to(device)
+    layer = cb.Conv2dB200(w, b, cfg.stride, cfg.pad, cfg.dilation, cfg.groups, cfg.layout)
+    y_shape = layer.out_shape(cfg.N, cfg.H, cfg.W)
+    set_bytes = (x_host.numel() + math.prod(y_shape)) * x_host.element_size()
+    nsets = max(2, min(16, math.ceil(2 * L2_BYTES / set_bytes) + 1))
+    xs = [x_host.to(device) for _ in range(nsets)]
+    ys = [torch.empty(y_shape, dtype=dt, device=device) for _ in range(nsets)]
+    layer.workspace(cfg.N, cfg.H, cfg.W)
+    stream = torch.cuda.current_stream()
+
+    for i in range(max(args.warmup, 3)):
+        layer(xs[i % nsets], ys[i % nsets])
+    cb.conv2d_sync_status()
+
+    # Steps per captured graph: a divisor of K, at most 512.
+    G = 1
+    for g in range(min(args.steps, 512), 0, -1):
+        if args.steps % g == 0:
+            G = g
+            break
+    reps = args.steps // G
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(G)]
+    for a, c in kev:  # create the underlying events before capture
+        a.record()
+        c.record()
+    torch.cuda.synchronize()
+    launches0 = cb.conv2d_kernel_launch_count()
+    if args.graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for i in range(G):
+                cb.conv2d_set_main_kernel_events(*kev[i])
+                layer(xs[i % nsets], ys[i % nsets])
+        cb.conv2d_set_main_kernel_events(None, None)
+        launches_per_rep = cb.conv2d_kernel_launch_count() - launches0
+        graph.replay()  # one untimed replay: graph upload
+        torch.cuda.synchronize()
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.05)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    launches_before = cb.conv2d_kernel_launch_count()
+    t0 = time.perf_counter()
+    ev0.record(stream)
+    if args.graph:
+        for _ in range(reps):
+            graph.replay()
+    else:
+        for r in range(reps):
+            for i in range(G):
+                cb.conv2d_set_main_kernel_events(*kev[i])
+                layer(xs[i % nsets], ys[i % nsets])
+        cb.conv2d_set_main_kernel_events(None, None)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    t1 = time.perf_counter()
+    barrier(world)
+    clocks.stop()
+    cb.conv2d_sync_status()
+    launches = (launches_per_rep * reps if args.graph
+                else cb.conv2d_kernel_launch_count() - launches_before)
+    elapsed_ms = max_over_ranks(ev0.elapsed_time(ev1), world, device)
+    kernel_ms = statistics.fmean(a.elapsed_time(c) for a, c in kev)
+    kernel_ms = max_over_ranks(kernel_ms, world, device)
+    ms_per_step = elapsed_ms / args.steps
+    value = world * flops(cfg) * args.steps / (elapsed_ms * 1e-3) / 1e12
+
+    # End to end through the host-buffer entry point: H2D of x, forward, D2H of y.
+    x_pin = x_host.pin_memory()
+    y_pin = torch.empty(y_shape, dtype=dt).pin_memory()
+    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    for _ in range(3):
+        layer.forward_hostio(x_pin, y_pin, xs[0], ys[0])
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        layer.forward_hostio(x_pin, y_pin, xs[0], ys[0])
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    cb.conv2d_sync_status()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, device) / e2e_steps
+    e2e_value = world * flops(cfg) / (e2e_ms * 1e-3) / 1e12
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, points, wall, threads = oracle_rate_sample(cfg, inp, args.cpu_seconds)
+        cpu = {"value": rate / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+               "sample": f"{points} random output points of one {cfg.name} forward pass "
+                         f"({wall:.1f} s of fp64 CPU work)"}
+
+    if rank == 0:
+        peaks, peak_kind = load_peaks()
+        cfgd = workload_config(cfg, args, world)
+        cfgd["l2"] = (f"not resident: steps rotate over {nsets} input/output sets "
+                      f"({nsets * set_bytes / 1e6:.0f} MB > 2x the 126 MB L2)")
+        cfgd["launch"] = f"CUDA graphs of {G} steps x {reps} replays" if args.graph else "eager"
+        line = {
+            "metric": metric_name(cfg), "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": cfg.dtype, "data": "synthetic (seeded; x ~ N(0,1), He-scaled weights)",
+            "config": cfgd,
+            "roofline": roofline(cfg, kernel_ms, peaks, peak_kind, cfg.name),
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
+                    "d2h_bytes_per_step": math.prod(y_shape) * x_host.element_size(),
+                    "ms_per_step": e2e_ms, "steps": e2e_steps,
+                    "api": "conv2d_forward_hostio (pinned host x -> device, forward, device y -> pinned host)"},
+            "gpu_launches": launches,
+            "clocks": clocks.summary(t0, t1),
+        }
+        print(json.dumps(line), flush=True)
+    if args.graph:
+        del graph
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-graph", dest="graph", action="store_false")
+    ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    from cnn_convolution_conv2d_b200 import workloads
+    cfg = workloads.CONFIGS[args.workload]
+    rank, world, _ = dist_env()
+    if world != args.gpus:
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args, cfg)
+        return
+    run_ours(args, cfg)
+
+
+if __name__ == "__main__":
+    main()

@@ -114,6 +114,11 @@ struct Plan {
     int Ho, Wo;
     long long M;
     int Cin_g, Cout_g, Cpg;
+    bool gather;    // few input channels: the software-gather kernel reads x directly
+    bool vec_rows;  // ... with 16-byte row loads (NCHW, aligned rows, unit dilation)
+    bool halo;      // ... from input rows staged in shared memory by TMA
+    int R, BW, ME;  // halo rows per tile, staged row width, left zero margin (elements)
+    int Kc, Kpad;   // its compact reduction length and padded length
     bool xcopy;     // x goes through the channels-last padding kernel first
     int cb;         // bytes of channels per plane row (16, 32, 64 or 128)
     int BN, taps, nCB, planes, kstages, Kp;
@@ -175,6 +180,62 @@ int make_plan(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stri
     p.Cout_g = C_out / groups;
     const int align = 16 / p.elt;
     p.Cpg = round_up(p.Cin_g, align);
+    // Fewer than 32 bytes of channels per pixel: hardware im2col rows would be too
+    // narrow, so the gather kernel builds the rows from x in place (groups = 1, the
+    // whole C_out x K weight matrix resident in shared memory).
+    // Row-vector order when x is NCHW with 16-byte-aligned rows and the column taps
+    // are contiguous (unit dilation) and fit one 16-byte word.
+    const int per16 = 16 / p.elt;
+    p.vec_rows = layout == CONV_NCHW && dilation == 1 && (W * p.elt) % 16 == 0 && Kw <= per16;
+    p.Kc = p.vec_rows ? C_in * Kh * per16 : C_in * Kh * Kw;
+    p.Kpad = round_up(p.Kc, 32 / p.elt);
+    p.gather = false;
+    if (!explicit_im2col && groups == 1 && C_in * p.elt < 32 && p.Kpad <= 256 &&
+        C_out <= (p.f32 ? 128 : 256)) {
+        const int bn = round_up(C_out, 16);
+        const size_t a_stage = static_cast<size_t>(128) * p.Kpad * p.elt * (p.f32 ? 2 : 1);
+        // Halo staging: every 128-pixel tile lies inside one image (Ho*Wo a multiple
+        // of 128) and the rows it reads fit one TMA box, with ME zero columns on the
+        // left covering the padding.
+        p.halo = false;
+        size_t halo_bytes = 0;
+        const int HoWo = p.Ho * p.Wo;
+        if (p.vec_rows && HoWo % 128 == 0 && pad <= per16) {
+            int span = 1;
+            for (int m0 = 0; m0 < HoWo; m0 += 128) {
+                const int s_rows = (m0 + 127) / p.Wo - m0 / p.Wo + 1;
+                span = s_rows > span ? s_rows : span;
+            }
+            const int R = (span - 1) * stride + (Kh - 1) * dilation + 1;
+            const int iw0_max = (p.Wo - 1) * stride - pad;
+            const int BW = round_up(iw0_max + per16 + per16 + 2, per16);
+            const size_t hb = static_cast<size_t>(C_in) * R * BW * p.elt;
+            if (R <= 256 && BW <= 256 && C_in <= 256 && W <= BW &&
+                gather_smem_bytes(p.f32, bn, p.Kpad, 2, hb) <= kSmemBudget) {
+                p.halo = true;
+                p.R = R;
+                p.BW = BW;
+                p.ME = per16;
+                halo_bytes = hb;
+            }
+        }
+        const size_t fixed = gather_smem_bytes(p.f32, bn, p.Kpad, 0, halo_bytes);
+        if (fixed + 2 * a_stage <= kSmemBudget) {
+            size_t st = (kSmemBudget - fixed) / a_stage;
+            p.gather = true;
+            p.BN = bn;
+            p.stages = static_cast<int>(st > 8 ? 8 : st);
+            p.smem = fixed + p.stages * a_stage;
+            p.n_mtiles = static_cast<int>((p.M + 127) / 128);
+            p.n_ntiles = 1;
+            p.splits = 1;
+            p.units = p.n_mtiles;
+            p.xcopy = false;
+            p.off_xcopy = p.off_partial = p.off_xcol = p.ws_total = 0;
+            *P = p;
+            return CONV_OK;
+        }
+    }
     p.xcopy = layout == CONV_NCHW || p.Cpg != p.Cin_g;
     const int row_bytes = p.Cpg * p.elt;
     p.cb = row_bytes % 128 == 0 ? 128 : row_bytes % 64 == 0 ? 64 : row_bytes % 32 == 0 ? 32 : 16;
@@ -284,6 +345,77 @@ int check_launch(cudaError_t e, const char *what) {
     return CONV_OK;
 }
 
+// Records a timing event on `stream`; under stream capture it is recorded as an
+// external event so that it becomes a timing node of the graph.
+int record_event(cudaEvent_t ev, cudaStream_t stream) {
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    cudaError_t e = cudaStreamIsCapturing(stream, &cap);
+    if (e == cudaSuccess)
+        e = cap == cudaStreamCaptureStatusActive
+                ? cudaEventRecordWithFlags(ev, stream, cudaEventRecordExternal)
+                : cudaEventRecord(ev, stream);
+    if (e != cudaSuccess) return fail(CONV_ERR_CUDA, "timing event record: %s", cudaGetErrorString(e));
+    return CONV_OK;
+}
+
+// The software-gather path (few input channels): one kernel, no scratch.
+int gather_impl(const Plan &p, const void *x, const void *w_packed, const void *bias, void *y,
+                DeviceInfo *dev, cudaStream_t stream) {
+    GatherParams g;
+    std::memset(&g, 0, sizeof(g));
+    g.x = x;
+    g.w_packed = w_packed;
+    g.N = p.N; g.C = p.C_in; g.H = p.H; g.W = p.W; g.Kh = p.Kh; g.Kw = p.Kw;
+    g.stride = p.stride; g.pad = p.pad; g.dilation = p.dilation;
+    g.Ho = p.Ho; g.Wo = p.Wo; g.M = static_cast<int>(p.M);
+    g.Cpg = p.Cpg;
+    g.Kc = p.Kc;
+    g.Kpad = p.Kpad;
+    g.BN = p.BN;
+    g.n_mtiles = p.n_mtiles;
+    g.stages = p.stages;
+    g.in_nchw = p.layout == CONV_NCHW ? 1 : 0;
+    g.vec_rows = p.vec_rows ? 1 : 0;
+    g.halo = p.halo ? 1 : 0;
+    if (p.halo) {
+        g.R = p.R;
+        g.BW = p.BW;
+        g.ME = p.ME;
+        cuuint64_t dims[4] = {static_cast<cuuint64_t>(p.W), static_cast<cuuint64_t>(p.H),
+                              static_cast<cuuint64_t>(p.C_in), static_cast<cuuint64_t>(p.N)};
+        cuuint64_t strides[3] = {static_cast<cuuint64_t>(p.W) * p.elt,
+                                 static_cast<cuuint64_t>(p.W) * p.H * p.elt,
+                                 static_cast<cuuint64_t>(p.W) * p.H * p.C_in * p.elt};
+        cuuint32_t box[4] = {static_cast<cuuint32_t>(p.BW), static_cast<cuuint32_t>(p.R),
+                             static_cast<cuuint32_t>(p.C_in), 1};
+        cuuint32_t estr[4] = {1, 1, 1, 1};
+        CUresult r = g_encode_tiled(&g.tmap_x, tma_type(p), 4, const_cast<void *>(x), dims, strides,
+                                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS)
+            return fail(CONV_ERR_CUDA, "cuTensorMapEncodeTiled (input rows) failed (%d)", static_cast<int>(r));
+    }
+    uint32_t cols = 32;
+    while (cols < static_cast<uint32_t>(2 * p.BN)) cols <<= 1;
+    g.tmem_cols = cols;
+    g.y = y;
+    g.bias = bias;
+    g.Cout = p.C_out;
+    g.out_mode = p.layout == CONV_NCHW ? kOutNCHW : kOutNHWC;
+    g.vec_ok = (p.C_out % (16 / p.elt) == 0) ? 1 : 0;
+    g.status = dev->status;
+    g.timeout_ns = g_timeout_ns;
+    g.starve = g_starve;
+    const int grid = p.n_mtiles < dev->sms ? p.n_mtiles : dev->sms;
+    int st;
+    cudaEvent_t ev_start = g_main_start, ev_stop = g_main_stop;
+    if (ev_start && ev_stop && (st = record_event(ev_start, stream)) != CONV_OK) return st;
+    cudaError_t e = launch_gather(g, p.f32, grid, p.smem, stream);
+    if ((st = check_launch(e, "gather tensor-core product")) != CONV_OK) return st;
+    if (ev_start && ev_stop && (st = record_event(ev_stop, stream)) != CONV_OK) return st;
+    return ok();
+}
+
 // Shared body of conv2d_forward and conv2d_forward_im2col_gemm.
 int forward_impl(bool explicit_im2col, const void *x, const void *w_packed, const void *bias, void *y,
                  int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stride, int pad,
@@ -306,6 +438,8 @@ int forward_impl(bool explicit_im2col, const void *x, const void *w_packed, cons
     if (!aligned16(x) || !aligned16(w_packed) || !aligned16(y) || (bias && !aligned16(bias)) ||
         (workspace && !aligned16(workspace)))
         return fail(CONV_ERR_UNSUPPORTED, "device pointers must be 16-byte aligned");
+
+    if (p.gather) return gather_impl(p, x, w_packed, bias, y, dev, stream);
 
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     const void *x_nhwc = p.xcopy ? static_cast<const void *>(ws + p.off_xcopy) : x;
@@ -339,6 +473,8 @@ int forward_impl(bool explicit_im2col, const void *x, const void *w_packed, cons
     kp.splits = p.splits;
     kp.units = p.units;
     kp.stages = p.stages;
+    // fp32: four stages (16 TF32 k-steps, 48 instructions) per tensor-memory chunk.
+    kp.chunk_stages = p.f32 ? 4 : 0;
     uint32_t cols = 32;
     while (cols < static_cast<uint32_t>(2 * p.BN)) cols <<= 1;
     kp.tmem_cols = cols;
@@ -370,10 +506,10 @@ int forward_impl(bool explicit_im2col, const void *x, const void *w_packed, cons
     }
     const int grid = p.units < dev->sms ? p.units : dev->sms;
     cudaEvent_t ev_start = g_main_start, ev_stop = g_main_stop;
-    if (ev_start && ev_stop) cudaEventRecord(ev_start, stream);
+    if (ev_start && ev_stop && (st = record_event(ev_start, stream)) != CONV_OK) return st;
     cudaError_t e = launch_igemm(kp, p.f32, p.cb, !explicit_im2col, grid, p.smem, stream);
     if ((st = check_launch(e, "tensor-core product")) != CONV_OK) return st;
-    if (ev_start && ev_stop) cudaEventRecord(ev_stop, stream);
+    if (ev_start && ev_stop && (st = record_event(ev_stop, stream)) != CONV_OK) return st;
     if (p.splits > 1) {
         e = launch_splitk_reduce(reinterpret_cast<const float *>(ws + p.off_partial), bias, y,
                                  static_cast<int>(p.M), C_out, p.Ho * p.Wo, p.splits,

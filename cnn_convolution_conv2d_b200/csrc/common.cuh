@@ -46,6 +46,8 @@ struct IgemmParams {
     int BN;              // output channels per tile (multiple of 16, <= 256)
     int n_mtiles, n_ntiles, splits, units;
     int stages;          // depth of the shared-memory ring
+    int chunk_stages;    // > 0: restart the tensor-memory accumulator every this many
+                         // stages and sum the chunks in fp32 registers (fp32 path)
     uint32_t tmem_cols;  // tensor-memory columns allocated (two accumulators)
     void *y;
     const void *bias;
@@ -56,10 +58,37 @@ struct IgemmParams {
     int starve;          // test hook: issue no loads
 };
 
-// Launchers (igemm.cu, layout.cu).  All return cudaSuccess or the launch error.
+// One launch of the software-gather kernel (gather.cu) for inputs with few
+// channels: groups = 1, reduction index k = (kh*Kw + kw)*C + c (or the row-vector
+// order), padded to Kpad.
+struct GatherParams {
+    CUtensorMap tmap_x;    // halo mode: 4-D tiled map of x (W, H, C, N)
+    const void *x;
+    const void *w_packed;  // (C_out, Kh, Kw, Cpg) from conv2d_pack_weight
+    int N, C, H, W, Kh, Kw, stride, pad, dilation;
+    int Ho, Wo, M;
+    int Cpg;               // channel pitch of w_packed
+    int Kc, Kpad;          // C*Kh*Kw and its length padded to a 32-byte multiple
+    int BN, n_mtiles, stages;
+    int in_nchw;
+    int vec_rows;          // row-vector gather: k = (c*Kh + kh)*(16/elt) + kw, see gather.cu
+    int halo;              // input rows staged in shared memory by TMA (needs vec_rows)
+    int R, BW, ME;         // halo rows, row width (elements) and left zero margin
+    uint32_t tmem_cols;
+    void *y;
+    const void *bias;
+    int Cout, out_mode, vec_ok;
+    int *status;
+    long long timeout_ns;
+    int starve;
+};
+
+// Launchers (igemm.cu, gather.cu, layout.cu).  All return cudaSuccess or the launch error.
 cudaError_t launch_igemm(const IgemmParams &p, bool f32, int cb_bytes, bool im2col, int grid,
                          size_t smem_bytes, cudaStream_t stream);
 size_t igemm_smem_bytes(bool f32, int BN, int stages);
+cudaError_t launch_gather(const GatherParams &p, bool f32, int grid, size_t smem, cudaStream_t stream);
+size_t gather_smem_bytes(bool f32, int BN, int Kpad, int stages, size_t halo_bytes);
 int igemm_threads(bool f32);
 
 cudaError_t launch_nchw_to_nhwc(const void *src, void *dst, int N, int C, int H, int W,

@@ -24,6 +24,7 @@
 #include <cuda_bf16.h>
 
 #include "common.cuh"
+#include "epilogue.cuh"
 #include "ptx.cuh"
 
 namespace conv2d_b200 {
@@ -41,6 +42,7 @@ constexpr int kProducerWarp = 0;
 constexpr int kMmaWarp = 1;
 constexpr int kEpiWarp0 = 2;
 constexpr int kCvtWarp0 = 6;
+constexpr int kMaxBNf32 = 128;            // widest fp32 tile: its accumulator row lives in registers
 
 template <bool kF32>
 constexpr int threads_for() { return kF32 ? 320 : 192; }
@@ -61,6 +63,19 @@ struct SharedBlock {  // lives at the start of the 1024-aligned dynamic shared m
 };
 static_assert(sizeof(SharedBlock) <= kBarrierBlock, "barrier block too small");
 
+__device__ __forceinline__ OutDesc out_desc(const IgemmParams &p) {
+    OutDesc o;
+    o.y = p.y;
+    o.bias = p.bias;
+    o.M = p.M;
+    o.HoWo = p.HoWo;
+    o.Cout = p.Cout;
+    o.Cout_g = p.Cout_g;
+    o.out_mode = p.out_mode;
+    o.vec_ok = p.vec_ok;
+    return o;
+}
+
 struct Unit {
     int mtile, g, ntile, split, k0, k1;
 };
@@ -78,107 +93,12 @@ __device__ __forceinline__ Unit decode_unit(const IgemmParams &p, int u) {
     return t;
 }
 
-__device__ __forceinline__ float tf32_round(float v) {
-    // round to the nearest value with 10 explicit mantissa bits (ties away from zero)
-    return __uint_as_float((__float_as_uint(v) + 0x1000u) & 0xFFFFE000u);
-}
-
 // Bounded wait that ignores the abort flag: used only while tearing down after an
 // abort, to let copies already in flight land before the CTA exits.
 __device__ __forceinline__ void wait_quiet(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
     const uint64_t start = globaltimer_ns();
     while (!mbar_try_wait(bar, parity)) {
         if (globaltimer_ns() - start > limit_ns) return;
-    }
-}
-
-// --------------------------------------------------------------- epilogue ---
-template <bool kF32>
-__device__ __forceinline__ void store_chunk16(const IgemmParams &p, int m, int g, int col0,
-                                              int split, const uint32_t (&r)[16]) {
-    if (m >= p.M) return;
-    const int nvalid = min(16, p.Cout_g - col0);
-    if (nvalid <= 0) return;
-    const int oc0 = g * p.Cout_g + col0;
-    float v[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
-
-    if (p.out_mode == kOutPartial) {
-        float *dst = static_cast<float *>(p.y) +
-                     (static_cast<size_t>(split) * p.M + m) * p.Cout + oc0;
-        if (nvalid == 16 && p.vec_ok) {
-            float4 *d4 = reinterpret_cast<float4 *>(dst);
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                d4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-        } else {
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-                if (i < nvalid) dst[i] = v[i];
-        }
-        return;
-    }
-    if (p.bias) {
-        if constexpr (kF32) {
-            const float *b = static_cast<const float *>(p.bias) + oc0;
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-                if (i < nvalid) v[i] += __ldg(b + i);
-        } else {
-            const __nv_bfloat16 *b = static_cast<const __nv_bfloat16 *>(p.bias) + oc0;
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-                if (i < nvalid) v[i] += __bfloat162float(b[i]);
-        }
-    }
-    if (p.out_mode == kOutNHWC) {
-        if constexpr (kF32) {
-            float *dst = static_cast<float *>(p.y) + static_cast<size_t>(m) * p.Cout + oc0;
-            if (nvalid == 16 && p.vec_ok) {
-                float4 *d4 = reinterpret_cast<float4 *>(dst);
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    d4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-            } else {
-#pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    if (i < nvalid) dst[i] = v[i];
-            }
-        } else {
-            __nv_bfloat16 *dst =
-                static_cast<__nv_bfloat16 *>(p.y) + static_cast<size_t>(m) * p.Cout + oc0;
-            if (nvalid == 16 && p.vec_ok) {
-                uint32_t packed[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
-                    packed[i] = *reinterpret_cast<uint32_t *>(&h);
-                }
-                uint4 *d4 = reinterpret_cast<uint4 *>(dst);
-                d4[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-                d4[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
-            } else {
-#pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    if (i < nvalid) dst[i] = __float2bfloat16_rn(v[i]);
-            }
-        }
-    } else {  // kOutNCHW: lanes hold consecutive pixels, so each column is a coalesced row
-        const int n = m / p.HoWo;
-        const int pix = m - n * p.HoWo;
-        const size_t base = (static_cast<size_t>(n) * p.Cout + oc0) * p.HoWo + pix;
-        if constexpr (kF32) {
-            float *dst = static_cast<float *>(p.y) + base;
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-                if (i < nvalid) dst[static_cast<size_t>(i) * p.HoWo] = v[i];
-        } else {
-            __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.y) + base;
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-                if (i < nvalid) dst[static_cast<size_t>(i) * p.HoWo] = __float2bfloat16_rn(v[i]);
-        }
     }
 }
 
@@ -365,32 +285,38 @@ __global__ void __launch_bounds__(threads_for<kF32>(), 1)
             bool ok = true;
             for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
                 const Unit t = decode_unit(p, u);
-                if (!mbar_wait(&sb.acc_empty[abuf], aphase ^ 1u, wd, kDevTimeoutAccEmpty)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after_sync();
-                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(abuf * BN);
-                for (int ks = t.k0; ks < t.k1; ++ks) {
-                    uint64_t *ready = kF32 ? &sb.converted[stage] : &sb.full[stage];
-                    if (!mbar_wait(ready, phase, wd, kF32 ? kDevTimeoutConvert : kDevTimeoutFull)) {
+                const int cs = p.chunk_stages > 0 ? p.chunk_stages : t.k1 - t.k0;
+                // Each chunk of the reduction goes into a fresh accumulator; the
+                // epilogue adds the chunks up (see the fp32 epilogue).
+                for (int c0 = t.k0; ok && c0 < t.k1; c0 += cs) {
+                    const int c1 = min(c0 + cs, t.k1);
+                    if (!mbar_wait(&sb.acc_empty[abuf], aphase ^ 1u, wd, kDevTimeoutAccEmpty)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after_sync();
-                    const uint32_t st = smem_addr(ring + static_cast<size_t>(stage) * sbytes);
-                    issue_stage<kF32, kCB>(st, st + b_off, st + alo_off, st + blo_off, BN, d_tmem,
-                                           idesc, ks == t.k0);
-                    mma_commit(&sb.empty[stage]);
-                    if (++stage == p.stages) {
-                        stage = 0;
-                        phase ^= 1u;
+                    const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(abuf * BN);
+                    for (int ks = c0; ks < c1; ++ks) {
+                        uint64_t *ready = kF32 ? &sb.converted[stage] : &sb.full[stage];
+                        if (!mbar_wait(ready, phase, wd, kF32 ? kDevTimeoutConvert : kDevTimeoutFull)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after_sync();
+                        const uint32_t st = smem_addr(ring + static_cast<size_t>(stage) * sbytes);
+                        issue_stage<kF32, kCB>(st, st + b_off, st + alo_off, st + blo_off, BN,
+                                               d_tmem, idesc, ks == c0);
+                        mma_commit(&sb.empty[stage]);
+                        if (++stage == p.stages) {
+                            stage = 0;
+                            phase ^= 1u;
+                        }
                     }
+                    if (!ok) break;
+                    mma_commit(&sb.acc_full[abuf]);
+                    abuf ^= 1;
+                    if (abuf == 0) aphase ^= 1u;
                 }
-                if (!ok) break;
-                mma_commit(&sb.acc_full[abuf]);
-                abuf ^= 1;
-                if (abuf == 0) aphase ^= 1u;
             }
             if (!ok || *wd.abort) {
                 mma_commit(&sb.drain);
@@ -404,25 +330,69 @@ __global__ void __launch_bounds__(threads_for<kF32>(), 1)
         const int row = quarter * 32 + lane;
         int abuf = 0;
         uint32_t aphase = 0;
+        const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+        const OutDesc out = out_desc(p);
         for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
             const Unit t = decode_unit(p, u);
-            const bool ok = mbar_wait(&sb.acc_full[abuf], aphase, wd, kDevTimeoutAccFull);
-            if (!__all_sync(0xffffffffu, ok)) break;
-            tc_fence_after_sync();
             const int m = t.mtile * kBM + row;
-            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                                   static_cast<uint32_t>(abuf * BN);
-            for (int c = 0; c < BN; c += 16) {
-                uint32_t r[16];
-                tmem_ld_x16(taddr + static_cast<uint32_t>(c), r);
-                tmem_ld_wait();
-                store_chunk16<kF32>(p, m, t.g, t.ntile * BN + c, t.split, r);
+            if constexpr (kF32) {
+                // The tensor cores' own accumulation loses accuracy over long
+                // reductions, so each chunk of p.chunk_stages stages is accumulated afresh
+                // in tensor memory and the chunks are summed here with IEEE fp32 adds.
+                const int cs = p.chunk_stages > 0 ? p.chunk_stages : t.k1 - t.k0;
+                const int nch = (t.k1 - t.k0 + cs - 1) / cs;
+                float acc[kMaxBNf32];
+#pragma unroll
+                for (int i = 0; i < kMaxBNf32; ++i) acc[i] = 0.f;
+                bool ok = true;
+                for (int ch = 0; ch < nch; ++ch) {
+                    ok = mbar_wait(&sb.acc_full[abuf], aphase, wd, kDevTimeoutAccFull);
+                    if (!__all_sync(0xffffffffu, ok)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    const uint32_t taddr = tmem_base + lane_base + static_cast<uint32_t>(abuf * BN);
+#pragma unroll
+                    for (int c = 0; c < kMaxBNf32 / 16; ++c) {
+                        if (c * 16 < BN) {
+                            uint32_t r[16];
+                            tmem_ld_x16(taddr + static_cast<uint32_t>(c * 16), r);
+                            tmem_ld_wait();
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) acc[c * 16 + i] += __uint_as_float(r[i]);
+                        }
+                    }
+                    tc_fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sb.acc_empty[abuf]);
+                    abuf ^= 1;
+                    if (abuf == 0) aphase ^= 1u;
+                }
+                if (!ok) break;
+#pragma unroll
+                for (int c = 0; c < kMaxBNf32 / 16; ++c)
+                    if (c * 16 < BN) store16<kF32>(out, m, t.g, t.ntile * BN + c * 16, t.split, &acc[c * 16]);
+            } else {
+                const bool ok = mbar_wait(&sb.acc_full[abuf], aphase, wd, kDevTimeoutAccFull);
+                if (!__all_sync(0xffffffffu, ok)) break;
+                tc_fence_after_sync();
+                const uint32_t taddr = tmem_base + lane_base + static_cast<uint32_t>(abuf * BN);
+                for (int c = 0; c < BN; c += 16) {
+                    uint32_t r[16];
+                    tmem_ld_x16(taddr + static_cast<uint32_t>(c), r);
+                    tmem_ld_wait();
+                    float v[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+                    store16<kF32>(out, m, t.g, t.ntile * BN + c, t.split, v);
+                }
+                tc_fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sb.acc_empty[abuf]);
+                abuf ^= 1;
+                if (abuf == 0) aphase ^= 1u;
             }
-            tc_fence_before_sync();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sb.acc_empty[abuf]);
-            abuf ^= 1;
-            if (abuf == 0) aphase ^= 1u;
         }
     } else if constexpr (kF32) {
         // ------------------------------------------- fp32 -> tf32 hi/lo split ---

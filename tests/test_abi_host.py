@@ -104,8 +104,12 @@ def test_forward_reports_unsupported_limits(lib):
 def test_workspace_size_without_device(lib):
     # channels-last input with C_in a multiple of 8: no scratch at all
     assert cb.conv2d_workspace_size(2, 8, 9, 9, 16, 3, 3, 1, 1, 1, 1, cb.CONV_BF16, "nhwc") == 0
-    # NCHW input: a channels-last copy padded to 8 channels
-    assert cb.conv2d_workspace_size(2, 3, 9, 9, 16, 3, 3, 1, 1, 1, 1, cb.CONV_BF16, "nchw") >= 2 * 9 * 9 * 8 * 2
+    # NCHW input with 16 channels: a channels-last copy
+    assert cb.conv2d_workspace_size(2, 16, 9, 9, 16, 3, 3, 1, 1, 1, 1, cb.CONV_BF16, "nchw") >= 2 * 9 * 9 * 16 * 2
+    # 12 channels in groups of 3: a channels-last copy with each group padded to 8
+    assert cb.conv2d_workspace_size(2, 12, 9, 9, 16, 3, 3, 1, 1, 1, 4, cb.CONV_BF16, "nhwc") >= 2 * 9 * 9 * 32 * 2
+    # 3 channels (first layer): gathered straight from x, no scratch
+    assert cb.conv2d_workspace_size(2, 3, 9, 9, 16, 3, 3, 1, 1, 1, 1, cb.CONV_BF16, "nchw") == 0
     # explicit im2col adds X_col: M rows of Kh*Kw*Cpg elements
     xcol = 2 * 9 * 9 * 9 * 8 * 2
     assert cb.conv2d_im2col_workspace_size(2, 8, 9, 9, 16, 3, 3, 1, 1, 1, 1, cb.CONV_BF16, "nhwc") >= xcol

@@ -78,6 +78,14 @@ EDGE = [  # N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups
     (1, 96, 7, 9, 200, 2, 2, 1, 0, 1, 1),    # even kernel, C_out not a multiple of the tile
     (1, 16, 40, 3, 16, 7, 1, 8, 3, 1, 1),    # stride 8 (the largest supported), thin image
     (5, 8, 6, 6, 16, 3, 3, 1, 1, 1, 1),      # several images inside one 128-row tile
+    (1, 16, 9, 9, 16, 3, 3, 1, 1, 1, 4),     # 4 channels per group: 16-byte rows, hardware im2col
+    (2, 12, 11, 10, 20, 5, 3, 2, 2, 1, 1),   # 12 channels: software gather, reduction 180
+    (2, 3, 16, 32, 24, 7, 7, 2, 3, 1, 1),    # first-layer shape, 16-byte rows: row-vector gather (bf16)
+    (2, 3, 12, 16, 8, 3, 3, 1, 1, 1, 1),     # 16-byte rows, 3x3: row-vector gather (fp32 too)
+    (3, 2, 9, 24, 16, 5, 5, 3, 2, 1, 1),     # row-vector gather with stride 3, two channels
+    (2, 3, 32, 32, 24, 7, 7, 2, 3, 1, 1),    # Ho*Wo = 256: input rows staged by TMA (bf16)
+    (2, 3, 16, 32, 8, 3, 3, 1, 1, 1, 1),     # Ho*Wo = 512: staged rows, 3x3 (fp32 too)
+    (1, 2, 48, 48, 16, 5, 5, 3, 2, 1, 1),    # staged rows with stride 3
 ]
 
 
