@@ -118,6 +118,10 @@ struct Plan {
     bool vec_rows;  // ... with 16-byte row loads (NCHW, aligned rows, unit dilation)
     bool halo;      // ... from input rows staged in shared memory by TMA
     int R, BW, ME;  // halo rows per tile, staged row width, left zero margin (elements)
+    int acols;      // tensor-memory columns per gathered A slot
+    bool tma_out;   // gather epilogue stores each tile with one TMA box store
+    size_t w_image_off;  // offset of the gather kernel's weight image in w_packed
+    int cw;         // output channels per gather epilogue group
     int Kc, Kpad;   // its compact reduction length and padded length
     bool xcopy;     // x goes through the channels-last padding kernel first
     int cb;         // bytes of channels per plane row (16, 32, 64 or 128)
@@ -135,6 +139,37 @@ int out_size(int in, int k, int s, int p, int d, int *out) {
     if (numer < 0) return -1;
     *out = static_cast<int>(numer / s + 1);
     return 0;
+}
+
+// The software-gather kernel reads its weights as ready-made shared-memory images
+// that conv2d_pack_weight writes after the packed OHWI weights: one per reduction
+// order (compact; row-vector) whose padded length fits the kernel's tables.
+struct GatherImages {
+    int bn = 0;              // image rows: C_out rounded up to 16
+    int kpad[2] = {0, 0};    // [0] compact order, [1] row-vector order; 0 = absent
+    size_t off[2] = {0, 0};  // byte offsets in the packed buffer
+    size_t total = 0;        // packed bytes including the images
+};
+
+GatherImages gather_images(int C_out, int C_in, int Kh, int Kw, int groups, int elt) {
+    GatherImages g;
+    const int cpg = round_up(C_in / groups, 16 / elt);
+    size_t off = static_cast<size_t>(C_out) * Kh * Kw * cpg * elt;
+    g.total = off;
+    if (groups != 1 || C_in * elt >= 32 || C_out > (elt == 4 ? 128 : 256)) return g;
+    g.bn = round_up(C_out, 16);
+    const int per16 = 16 / elt;
+    const int kp[2] = {round_up(C_in * Kh * Kw, 32 / elt),
+                       Kw <= per16 ? round_up(C_in * Kh * per16, 32 / elt) : 0};
+    for (int o = 0; o < 2; ++o) {
+        if (kp[o] == 0 || kp[o] > 256) continue;
+        off = align_up(off, 256);
+        g.kpad[o] = kp[o];
+        g.off[o] = off;
+        off += static_cast<size_t>(g.bn) * kp[o] * elt * (elt == 4 ? 2 : 1);
+    }
+    g.total = off;
+    return g;
 }
 
 // Validates a problem and fills the plan.  `explicit_im2col` adds the X_col
@@ -193,7 +228,11 @@ int make_plan(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stri
     if (!explicit_im2col && groups == 1 && C_in * p.elt < 32 && p.Kpad <= 256 &&
         C_out <= (p.f32 ? 128 : 256)) {
         const int bn = round_up(C_out, 16);
-        const size_t a_stage = static_cast<size_t>(128) * p.Kpad * p.elt * (p.f32 ? 2 : 1);
+        // Tensor memory (512 columns): two accumulators of bn columns, then A slots
+        // of Kpad/2 (bf16, two elements per column) or 2*Kpad (fp32 hi + lo) columns.
+        const int acols = p.f32 ? 2 * round_up(p.Kpad, 32) : round_up(p.Kpad / 2, 32);
+        int slots = (512 - 2 * bn) / acols;
+        slots = slots < gather_max_stages() ? slots : gather_max_stages();
         // Halo staging: every 128-pixel tile lies inside one image (Ho*Wo a multiple
         // of 128) and the rows it reads fit one TMA box, with ME zero columns on the
         // left covering the padding.
@@ -211,7 +250,7 @@ int make_plan(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stri
             const int BW = round_up(iw0_max + per16 + per16 + 2, per16);
             const size_t hb = static_cast<size_t>(C_in) * R * BW * p.elt;
             if (R <= 256 && BW <= 256 && C_in <= 256 && W <= BW &&
-                gather_smem_bytes(p.f32, bn, p.Kpad, 2, hb) <= kSmemBudget) {
+                gather_smem_bytes(p.f32, bn, p.Kpad, hb, 0) <= kSmemBudget) {
                 p.halo = true;
                 p.R = R;
                 p.BW = BW;
@@ -219,13 +258,26 @@ int make_plan(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stri
                 halo_bytes = hb;
             }
         }
-        const size_t fixed = gather_smem_bytes(p.f32, bn, p.Kpad, 0, halo_bytes);
-        if (fixed + 2 * a_stage <= kSmemBudget) {
-            size_t st = (kSmemBudget - fixed) / a_stage;
+        // Staged tiles lie inside one image, so a bf16 epilogue can store each tile
+        // with TMA (NCHW output rows of 128 pixels).
+        p.cw = round_up((bn + 1) / 2, 16);
+        p.tma_out = p.halo && !p.f32;
+        size_t smem = gather_smem_bytes(p.f32, bn, p.Kpad, halo_bytes,
+                                        p.tma_out ? static_cast<size_t>(p.cw) * 128 * p.elt : 0);
+        if (p.tma_out && smem > kSmemBudget) {
+            p.tma_out = false;
+            smem = gather_smem_bytes(p.f32, bn, p.Kpad, halo_bytes, 0);
+        }
+        const GatherImages gi = gather_images(C_out, C_in, Kh, Kw, groups, p.elt);
+        const int order = p.vec_rows ? 1 : 0;
+        if (slots >= 2 && smem <= kSmemBudget && gi.kpad[order] == p.Kpad) {
             p.gather = true;
+            p.w_image_off = gi.off[order];
             p.BN = bn;
-            p.stages = static_cast<int>(st > 8 ? 8 : st);
-            p.smem = fixed + p.stages * a_stage;
+            p.stages = slots;
+            p.acols = acols;
+            // at least 120 KB, so that one CTA (holding all tensor memory) runs per SM
+            p.smem = smem > 120 * 1024 ? smem : 120 * 1024;
             p.n_mtiles = static_cast<int>((p.M + 127) / 128);
             p.n_ntiles = 1;
             p.splits = 1;
@@ -365,6 +417,7 @@ int gather_impl(const Plan &p, const void *x, const void *w_packed, const void *
     std::memset(&g, 0, sizeof(g));
     g.x = x;
     g.w_packed = w_packed;
+    g.w_image = static_cast<const uint8_t *>(w_packed) + p.w_image_off;
     g.N = p.N; g.C = p.C_in; g.H = p.H; g.W = p.W; g.Kh = p.Kh; g.Kw = p.Kw;
     g.stride = p.stride; g.pad = p.pad; g.dilation = p.dilation;
     g.Ho = p.Ho; g.Wo = p.Wo; g.M = static_cast<int>(p.M);
@@ -374,6 +427,7 @@ int gather_impl(const Plan &p, const void *x, const void *w_packed, const void *
     g.BN = p.BN;
     g.n_mtiles = p.n_mtiles;
     g.stages = p.stages;
+    g.acols = p.acols;
     g.in_nchw = p.layout == CONV_NCHW ? 1 : 0;
     g.vec_rows = p.vec_rows ? 1 : 0;
     g.halo = p.halo ? 1 : 0;
@@ -395,9 +449,21 @@ int gather_impl(const Plan &p, const void *x, const void *w_packed, const void *
         if (r != CUDA_SUCCESS)
             return fail(CONV_ERR_CUDA, "cuTensorMapEncodeTiled (input rows) failed (%d)", static_cast<int>(r));
     }
-    uint32_t cols = 32;
-    while (cols < static_cast<uint32_t>(2 * p.BN)) cols <<= 1;
-    g.tmem_cols = cols;
+    g.tmem_cols = 512;  // accumulators and A slots
+    g.cw = p.cw;
+    g.tma_out = p.tma_out ? 1 : 0;
+    if (p.tma_out) {
+        const cuuint64_t howo = static_cast<cuuint64_t>(p.Ho) * p.Wo;
+        cuuint64_t dims[3] = {howo, static_cast<cuuint64_t>(p.C_out), static_cast<cuuint64_t>(p.N)};
+        cuuint64_t strides[2] = {howo * p.elt, howo * p.elt * p.C_out};
+        cuuint32_t box[3] = {32, static_cast<cuuint32_t>(p.cw), 1};  // one warp: 32 pixels x cw channels
+        cuuint32_t estr[3] = {1, 1, 1};
+        CUresult r = g_encode_tiled(&g.tmap_y, tma_type(p), 3, y, dims, strides, box, estr,
+                                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                                    CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS)
+            return fail(CONV_ERR_CUDA, "cuTensorMapEncodeTiled (output) failed (%d)", static_cast<int>(r));
+    }
     g.y = y;
     g.bias = bias;
     g.Cout = p.C_out;
@@ -567,8 +633,7 @@ int conv2d_packed_weight_size(int C_out, int C_in, int Kh, int Kw, int groups, c
     if (!bytes || elt == 0 || C_out < 1 || C_in < 1 || Kh < 1 || Kw < 1 || groups < 1 ||
         C_in % groups || C_out % groups)
         return fail(CONV_ERR_INVALID_ARG, "packed weight size: invalid argument");
-    const int cpg = round_up(C_in / groups, 16 / elt);
-    *bytes = static_cast<size_t>(C_out) * Kh * Kw * cpg * elt;
+    *bytes = gather_images(C_out, C_in, Kh, Kw, groups, elt).total;
     return ok();
 }
 
@@ -580,11 +645,19 @@ int conv2d_pack_weight(const void *w_oihw, void *w_packed, int C_out, int C_in, 
     if (!w_oihw || !w_packed) return fail(CONV_ERR_INVALID_ARG, "weight pointers must not be NULL");
     const int elt = elt_of(dtype);
     const int cpg = round_up(C_in / groups, 16 / elt);
-    return check_launch(launch_pack_weight(w_oihw, w_packed, C_out, C_in / groups, Kh, Kw, cpg, elt,
-                                           reinterpret_cast<cudaStream_t>(stream)),
-                        "weight pack") == CONV_OK
-               ? ok()
-               : CONV_ERR_CUDA;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if ((st = check_launch(launch_pack_weight(w_oihw, w_packed, C_out, C_in / groups, Kh, Kw, cpg, elt, s),
+                           "weight pack")) != CONV_OK)
+        return st;
+    const GatherImages gi = gather_images(C_out, C_in, Kh, Kw, groups, elt);
+    for (int o = 0; o < 2; ++o) {
+        if (gi.kpad[o] == 0) continue;
+        if ((st = check_launch(launch_pack_gather_image(w_oihw, static_cast<uint8_t *>(w_packed) + gi.off[o],
+                                                        C_out, C_in, Kh, Kw, gi.bn, gi.kpad[o], o == 1, elt, s),
+                               "weight image")) != CONV_OK)
+            return st;
+    }
+    return ok();
 }
 
 int conv2d_workspace_size(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stride,

@@ -63,17 +63,23 @@ struct IgemmParams {
 // order), padded to Kpad.
 struct GatherParams {
     CUtensorMap tmap_x;    // halo mode: 4-D tiled map of x (W, H, C, N)
+    CUtensorMap tmap_y;    // tma_out mode: 3-D tiled map of y (Ho*Wo, C_out, N)
     const void *x;
     const void *w_packed;  // (C_out, Kh, Kw, Cpg) from conv2d_pack_weight
+    const void *w_image;   // the kernel's shared-memory weight image (written by the pack)
     int N, C, H, W, Kh, Kw, stride, pad, dilation;
     int Ho, Wo, M;
     int Cpg;               // channel pitch of w_packed
     int Kc, Kpad;          // C*Kh*Kw and its length padded to a 32-byte multiple
-    int BN, n_mtiles, stages;
+    int BN, n_mtiles;
+    int stages;            // A slots in tensor memory
+    int acols;             // tensor-memory columns per A slot
     int in_nchw;
     int vec_rows;          // row-vector gather: k = (c*Kh + kh)*(16/elt) + kw, see gather.cu
     int halo;              // input rows staged in shared memory by TMA (needs vec_rows)
     int R, BW, ME;         // halo rows, row width (elements) and left zero margin
+    int tma_out;           // epilogue stages each tile channel-major and stores it by TMA
+    int cw;                // output channels per epilogue group
     uint32_t tmem_cols;
     void *y;
     const void *bias;
@@ -88,7 +94,8 @@ cudaError_t launch_igemm(const IgemmParams &p, bool f32, int cb_bytes, bool im2c
                          size_t smem_bytes, cudaStream_t stream);
 size_t igemm_smem_bytes(bool f32, int BN, int stages);
 cudaError_t launch_gather(const GatherParams &p, bool f32, int grid, size_t smem, cudaStream_t stream);
-size_t gather_smem_bytes(bool f32, int BN, int Kpad, int stages, size_t halo_bytes);
+size_t gather_smem_bytes(bool f32, int BN, int Kpad, size_t halo_bytes, size_t out_stage_bytes);
+int gather_max_stages();
 int igemm_threads(bool f32);
 
 cudaError_t launch_nchw_to_nhwc(const void *src, void *dst, int N, int C, int H, int W,
@@ -99,6 +106,8 @@ cudaError_t launch_nhwc_to_nchw(const void *src, void *dst, int N, int C, int H,
                                 cudaStream_t s);
 cudaError_t launch_pack_weight(const void *w, void *wp, int Cout, int Cin_g, int Kh, int Kw,
                                int Cpg, int elt, cudaStream_t s);
+cudaError_t launch_pack_gather_image(const void *w, void *img, int Cout, int C, int Kh, int Kw,
+                                     int BN, int Kpad, bool rowvec, int elt, cudaStream_t s);
 cudaError_t launch_im2col(const void *x_nhwc, void *xcol, int N, int H, int W, int groups,
                           int Cpg, int Ho, int Wo, int Kh, int Kw, int stride, int pad,
                           int dilation, int elt, cudaStream_t s);

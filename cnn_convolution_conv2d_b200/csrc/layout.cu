@@ -154,6 +154,66 @@ __global__ void pack_weight_kernel(const void *__restrict__ w, void *__restrict_
     }
 }
 
+// --- weight image of the software-gather kernel: OIHW (Cout, C, Kh, Kw) ->
+// the tensor cores' no-swizzle K-major shared-memory layout of a BN x Kpad matrix
+// (8-row groups `nchunks * 128` bytes apart, 16-byte k chunks 128 bytes apart,
+// rows 16 bytes apart), k in the compact order (kh*Kw + kw)*C + c or the row-vector
+// order (c*Kh + kh)*kPer + kw, zero where k or the row is padding.  fp32 weights
+// become two images, tf32 hi then lo.
+template <int kElt>
+__global__ void pack_gather_image_kernel(const void *__restrict__ w, uint8_t *__restrict__ img,
+                                         int Cout, int C, int Kh, int Kw, int BN, int Kpad,
+                                         int rowvec) {
+    constexpr int kPer = 16 / kElt;
+    const int nchunks = Kpad / kPer;
+    const size_t image_bytes = static_cast<size_t>(BN) * Kpad * kElt;
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
+         i < static_cast<long long>(BN) * nchunks; i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const int oc = static_cast<int>(i / nchunks), j = static_cast<int>(i % nchunks);
+        float v[kPer];
+        uint32_t u[kPer];
+        for (int e = 0; e < kPer; ++e) {
+            int c, kh, kw;
+            bool real = oc < Cout;
+            if (rowvec) {
+                c = j / Kh;
+                kh = j % Kh;
+                kw = e;
+                real = real && j < C * Kh && e < Kw;
+            } else {
+                const int k = j * kPer + e;
+                const int tap = k / C;
+                c = k % C;
+                kh = tap / Kw;
+                kw = tap % Kw;
+                real = real && k < C * Kh * Kw;
+            }
+            const size_t src = ((static_cast<size_t>(oc) * C + c) * Kh + kh) * Kw + kw;
+            if (kElt == 4) {
+                v[e] = real ? static_cast<const float *>(w)[src] : 0.f;
+            } else {
+                u[e] = real ? static_cast<const unsigned short *>(w)[src] : 0u;
+            }
+        }
+        const size_t off = static_cast<size_t>(oc >> 3) * nchunks * 128 + static_cast<size_t>(j) * 128 +
+                           static_cast<size_t>(oc & 7) * 16;
+        if (kElt == 4) {
+            float hi[4], lo[4];
+            for (int e = 0; e < 4; ++e) {
+                hi[e] = __uint_as_float((__float_as_uint(v[e]) + 0x1000u) & 0xFFFFE000u);
+                const float r = v[e] - hi[e];
+                lo[e] = __uint_as_float((__float_as_uint(r) + 0x1000u) & 0xFFFFE000u);
+            }
+            *reinterpret_cast<float4 *>(img + off) = make_float4(hi[0], hi[1], hi[2], hi[3]);
+            *reinterpret_cast<float4 *>(img + image_bytes + off) = make_float4(lo[0], lo[1], lo[2], lo[3]);
+        } else {
+            uint32_t wds[4];
+            for (int e = 0; e < 4; ++e) wds[e] = u[2 * e] | (u[2 * e + 1] << 16);
+            *reinterpret_cast<uint4 *>(img + off) = make_uint4(wds[0], wds[1], wds[2], wds[3]);
+        }
+    }
+}
+
 // --- explicit im2col: xcol[m][g*Kp + (kh*Kw + kw)*Cpg + c] = x[n][ih][iw][g*Cpg + c]
 // (0 outside the image), m = (n*Ho + oh)*Wo + ow.  One thread per 16-byte chunk; a
 // chunk never straddles two taps because Cpg*elt is a multiple of 16.
@@ -272,6 +332,18 @@ cudaError_t launch_pack_weight(const void *w, void *wp, int Cout, int Cin_g, int
         pack_weight_kernel<2><<<grid_for(total), kThreads, 0, s>>>(w, wp, Cout, Cin_g, Kh, Kw, Cpg);
     else
         pack_weight_kernel<4><<<grid_for(total), kThreads, 0, s>>>(w, wp, Cout, Cin_g, Kh, Kw, Cpg);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_pack_gather_image(const void *w, void *img, int Cout, int C, int Kh, int Kw,
+                                     int BN, int Kpad, bool rowvec, int elt, cudaStream_t s) {
+    const long long work = static_cast<long long>(BN) * Kpad * elt / 16;
+    if (elt == 2)
+        pack_gather_image_kernel<2><<<grid_for(work), kThreads, 0, s>>>(
+            w, static_cast<uint8_t *>(img), Cout, C, Kh, Kw, BN, Kpad, rowvec ? 1 : 0);
+    else
+        pack_gather_image_kernel<4><<<grid_for(work), kThreads, 0, s>>>(
+            w, static_cast<uint8_t *>(img), Cout, C, Kh, Kw, BN, Kpad, rowvec ? 1 : 0);
     return cudaGetLastError();
 }
 

@@ -71,7 +71,9 @@ int conv2d_output_size(int in, int k, int stride, int pad, int dilation, int *ou
 
 /* Bytes of the packed weight buffer that conv2d_pack_weight writes:
  * C_out * Kh * Kw * Cpg elements of dtype, where Cpg is C_in/groups rounded up
- * to a multiple of 8 (bf16) or 4 (fp32). */
+ * to a multiple of 8 (bf16) or 4 (fp32), followed -- for groups = 1 and fewer
+ * than 32 bytes of input channels per pixel -- by ready-made shared-memory images
+ * of the weight matrix for the few-channel kernel. */
 int conv2d_packed_weight_size(int C_out, int C_in, int Kh, int Kw, int groups,
                               conv_dtype_t dtype, size_t *bytes);
 

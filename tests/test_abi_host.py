@@ -58,9 +58,20 @@ def test_output_size_rejects(lib, args):
 
 
 def test_packed_weight_size(lib):
-    assert cb.conv2d_packed_weight_size(64, 3, 7, 7, 1, cb.CONV_BF16) == 64 * 49 * 8 * 2
-    assert cb.conv2d_packed_weight_size(4, 3, 3, 3, 1, cb.CONV_F32) == 4 * 9 * 4 * 4
+    # many channels or groups: only the (C_out, Kh, Kw, Cpg) weights
     assert cb.conv2d_packed_weight_size(512, 512, 3, 3, 32, cb.CONV_BF16) == 512 * 9 * 16 * 2
+    assert cb.conv2d_packed_weight_size(256, 256, 3, 3, 1, cb.CONV_BF16) == 256 * 9 * 256 * 2
+    # few input channels: followed (256-byte aligned) by the gather kernel's images,
+    # 16-row x Kpad matrices for the compact and row-vector reduction orders
+    main = 64 * 49 * 8 * 2                       # stem: Cpg = 8
+    compact = 64 * 160 * 2                       # 3*7*7 = 147 -> 160
+    rowvec = 64 * 176 * 2                        # 3*7*8 = 168 -> 176
+    assert cb.conv2d_packed_weight_size(64, 3, 7, 7, 1, cb.CONV_BF16) == main + compact + rowvec
+    main32 = 4 * 9 * 4 * 4                       # fp32 tiny: Cpg = 4 -> 576 bytes
+    img_c = 16 * 32 * 4 * 2                      # 27 -> 32, tf32 hi + lo
+    img_r = 16 * 40 * 4 * 2                      # 3*3*4 = 36 -> 40
+    assert main32 == 576
+    assert cb.conv2d_packed_weight_size(4, 3, 3, 3, 1, cb.CONV_F32) == 768 + img_c + img_r
     with pytest.raises(cb.Conv2dError):
         cb.conv2d_packed_weight_size(6, 4, 3, 3, 4, cb.CONV_BF16)   # C_out % groups
 
