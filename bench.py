@@ -44,7 +44,7 @@ if ROOT not in sys.path:
 DEFAULT_WORKLOAD = "stem_bf16"
 L2_BYTES = 126 * 1000 * 1000
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_SOURCES = ["igemm.cu", "ptx.cuh", "common.cuh"]
+KERNEL_SOURCES = ["igemm.cu", "gather.cu", "epilogue.cuh", "ptx.cuh", "common.cuh"]
 
 
 # ------------------------------------------------------------ arithmetic ---
