@@ -42,6 +42,7 @@ SIGNATURES = {
     "conv2d_im2col_workspace_size": (_SHAPE + [_I, _I, ctypes.POINTER(_S)], _I),
     "conv2d_forward_im2col_gemm": ([_P, _P, _P, _P] + _SHAPE + [_I, _I, _P, _S, _P], _I),
     "conv2d_forward_hostio": ([_P, _P, _P, _P, _P, _P] + _SHAPE + [_I, _I, _P, _S, _P], _I),
+    "conv2d_forward_noalloc": ([_P, _P, _P, _P] + _SHAPE + [_I, _I, _P], _I),
     "conv2d_nchw_to_nhwc": ([_P, _P, _I, _I, _I, _I, _I, _I, _I, _P], _I),
     "conv2d_nhwc_to_nchw": ([_P, _P, _I, _I, _I, _I, _I, _P], _I),
     "conv2d_sync_status": ([_P], _I),
@@ -181,6 +182,19 @@ def conv2d_forward_im2col_gemm(x, w_packed, bias, y, N, C_in, H, W, C_out, Kh, K
     _check(load().conv2d_forward_im2col_gemm(_ptr(x), _ptr(w_packed), _ptr(bias), _ptr(y), N, C_in,
                                              H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype,
                                              _layout_code(layout), wp, wb, _stream(stream)))
+    return y
+
+
+NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024  # CONV2D_NOALLOC_SCRATCH_BYTES
+
+
+def conv2d_forward_noalloc(x, w_packed, bias, y, N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation,
+                           groups, dtype, layout, stream=None):
+    """conv2d_forward without a workspace: for callers that cannot allocate device
+    memory; its scratch is the library's built-in NOALLOC_SCRATCH_BYTES array."""
+    _check(load().conv2d_forward_noalloc(_ptr(x), _ptr(w_packed), _ptr(bias), _ptr(y), N, C_in, H, W,
+                                         C_out, Kh, Kw, stride, pad, dilation, groups, dtype,
+                                         _layout_code(layout), _stream(stream)))
     return y
 
 

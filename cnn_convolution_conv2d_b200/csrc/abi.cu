@@ -36,6 +36,12 @@ int ok() {
 // Watchdog status word written by device code when a bounded wait runs out.
 __device__ int g_device_status;
 
+// Scratch of conv2d_forward_noalloc: callers without an allocator get their
+// workspace from here.  Host code passes its device address (looked up once per
+// device), never the name itself.
+constexpr size_t kNoAllocScratchBytes = CONV2D_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
 constexpr int kMaxDevices = 64;
 constexpr size_t kSmemBudget = 227 * 1024;
 constexpr long long kDefaultTimeoutNs = 2000000000LL;
@@ -44,6 +50,7 @@ struct DeviceInfo {
     bool ready = false;
     int sms = 0;
     int *status = nullptr;
+    void *noalloc_scratch = nullptr;  // device address of g_noalloc_scratch
 };
 DeviceInfo g_devices[kMaxDevices];
 std::mutex g_mutex;
@@ -609,6 +616,24 @@ int workspace_impl(bool explicit_im2col, int N, int C_in, int H, int W, int C_ou
 
 int elt_of(conv_dtype_t dtype) { return dtype == CONV_F32 ? 4 : dtype == CONV_BF16 ? 2 : 0; }
 
+// Device address of the built-in scratch on the current device, looked up on the
+// first use per device (with that device current) and cached.
+int noalloc_scratch(void **out) {
+    DeviceInfo *dev = nullptr;
+    int st = device_info(&dev);
+    if (st != CONV_OK) return st;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (!dev->noalloc_scratch) {
+        void *ptr = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+        if (e != cudaSuccess || !ptr)
+            return fail(CONV_ERR_CUDA, "built-in scratch address: %s", cudaGetErrorString(e));
+        dev->noalloc_scratch = ptr;
+    }
+    *out = dev->noalloc_scratch;
+    return CONV_OK;
+}
+
 }  // namespace
 }  // namespace conv2d_b200
 
@@ -690,6 +715,26 @@ int conv2d_forward_im2col_gemm(const void *x, const void *w_packed, const void *
                                conv_stream_t stream) {
     return forward_impl(true, x, w_packed, bias, y, N, C_in, H, W, C_out, Kh, Kw, stride, pad,
                         dilation, groups, dtype, layout, workspace, workspace_bytes,
+                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+int conv2d_forward_noalloc(const void *x, const void *w_packed, const void *bias, void *y, int N,
+                           int C_in, int H, int W, int C_out, int Kh, int Kw, int stride, int pad,
+                           int dilation, int groups, conv_dtype_t dtype, conv_layout_t layout,
+                           conv_stream_t stream) {
+    size_t need = 0;
+    int st = workspace_impl(false, N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype,
+                            layout, &need);
+    if (st != CONV_OK) return st;
+    if (need > kNoAllocScratchBytes)
+        return fail(CONV_ERR_WORKSPACE,
+                    "this problem needs %zu bytes of scratch; the built-in scratch of "
+                    "conv2d_forward_noalloc holds %zu (use conv2d_forward with a workspace)",
+                    need, kNoAllocScratchBytes);
+    void *scratch = nullptr;
+    if (need > 0 && (st = noalloc_scratch(&scratch)) != CONV_OK) return st;
+    return forward_impl(false, x, w_packed, bias, y, N, C_in, H, W, C_out, Kh, Kw, stride, pad,
+                        dilation, groups, dtype, layout, scratch, need > 0 ? kNoAllocScratchBytes : 0,
                         reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -182,6 +182,31 @@ int conv2d_sync_status(conv_stream_t stream);
  * (empty string if none).  The pointer stays valid until the thread's next call. */
 const char *conv2d_last_error(void);
 
+/* Bytes of the device scratch built into the library for conv2d_forward_noalloc. */
+#define CONV2D_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+
+/* conv2d_forward for callers that cannot allocate device memory -- code running
+ * where cudaMalloc is not allowed or not wanted (while a CUDA graph is being
+ * captured, under an allocator that owns all device memory, or in a plugin whose
+ * host gives it only input and output buffers).  The pages describe no such
+ * entry point; it exists for deployment.
+ * Arguments and results are those of conv2d_forward without the workspace: the
+ * scratch it needs (a channels-last copy of x, split partial sums) comes from a
+ * CONV2D_NOALLOC_SCRATCH_BYTES array compiled into the library, which every GPU
+ * that loads the library holds until the process exits.  A problem needing more
+ * scratch than that is rejected with CONV_ERR_WORKSPACE before anything is
+ * enqueued.  Nothing in this call allocates memory.
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture.  All calls share the one array and it keeps the last call's contents
+ * (every byte a call reads it has written first, so nothing needs clearing):
+ * calls whose work overlaps on the GPU -- on different streams without ordering
+ * between them -- race on it and must not be made. */
+int conv2d_forward_noalloc(const void *x, const void *w_packed, const void *bias, void *y,
+                           int N, int C_in, int H, int W, int C_out, int Kh, int Kw,
+                           int stride, int pad, int dilation, int groups,
+                           conv_dtype_t dtype, conv_layout_t layout, conv_stream_t stream);
+
 /* Measurement aid: when `start` and `stop` (cudaEvent_t handles the caller created
  * with timing enabled) are both non-NULL, every later forward call records `start`
  * on its stream immediately before launching its tensor-core kernel and `stop`
