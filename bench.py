@@ -224,6 +224,16 @@ def dist_env():
     return rank, world, local
 
 
+def rank_seed(cfg, rank: int) -> int:
+    """Seed of a rank's batch: each rank draws a different batch of the same workload."""
+    return cfg.seed + 1000 * rank
+
+
+def weak_scaling_value(world: int, flop_per_rank_step: float, steps: int, max_elapsed_ms: float) -> float:
+    """Whole-job TFLOP/s: the work of all ranks over the slowest rank's timed region."""
+    return world * flop_per_rank_step * steps / (max_elapsed_ms * 1e-3) / 1e12
+
+
 def max_over_ranks(value: float, world: int, device) -> float:
     if world == 1:
         return value
@@ -341,7 +351,7 @@ def run_ours(args, cfg):
     barrier(world)
     cb.load()
 
-    inp = workloads.make_inputs(cfg, seed=cfg.seed + 1000 * rank)
+    inp = workloads.make_inputs(cfg, seed=rank_seed(cfg, rank))
     dt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
     x_host = torch.from_numpy(inp["x"]).to(dt)
     if cfg.layout == "nhwc":
@@ -415,7 +425,7 @@ def run_ours(args, cfg):
     kernel_ms = statistics.fmean(a.elapsed_time(c) for a, c in kev)
     kernel_ms = max_over_ranks(kernel_ms, world, device)
     ms_per_step = elapsed_ms / args.steps
-    value = world * flops(cfg) * args.steps / (elapsed_ms * 1e-3) / 1e12
+    value = weak_scaling_value(world, flops(cfg), args.steps, elapsed_ms)
 
     # End to end through the host-buffer entry point: H2D of x, forward, D2H of y.
     x_pin = x_host.pin_memory()
@@ -434,7 +444,7 @@ def run_ours(args, cfg):
     barrier(world)
     cb.conv2d_sync_status()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, device) / e2e_steps
-    e2e_value = world * flops(cfg) / (e2e_ms * 1e-3) / 1e12
+    e2e_value = weak_scaling_value(world, flops(cfg), 1, e2e_ms)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
