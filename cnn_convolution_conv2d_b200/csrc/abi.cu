@@ -126,7 +126,7 @@ struct Plan {
     bool halo;      // ... from input rows staged in shared memory by TMA
     int R, BW, ME;  // halo rows per tile, staged row width, left zero margin (elements)
     int acols;      // tensor-memory columns per gathered A slot
-    bool tma_out;   // gather epilogue stores each tile with one TMA box store
+    bool tma_out;   // epilogue stores through shared memory and TMA (both kernels)
     size_t w_image_off;  // offset of the gather kernel's weight image in w_packed
     int cw;         // output channels per gather epilogue group
     int Kc, Kpad;   // its compact reduction length and padded length
@@ -319,11 +319,16 @@ int make_plan(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stri
         if (s >= 2) p.splits = s;
     }
     p.units = static_cast<int>(base * p.splits);
+    // bf16 channels-last output leaves through shared memory and TMA stores when
+    // every 32-column block of a tile lies inside its group's columns.
+    p.tma_out = !p.f32 && layout == CONV_NHWC && p.splits == 1 &&
+                p.BN % 32 == 0 && p.Cout_g % p.BN == 0 && (C_out * p.elt) % 16 == 0;
     const size_t stage = static_cast<size_t>(128 + p.BN) * 128 * (p.f32 ? 2 : 1);
-    int stages = static_cast<int>((kSmemBudget - 2048) / stage);
+    const size_t ystage = igemm_smem_bytes(p.f32, p.BN, 0, p.tma_out) - igemm_smem_bytes(p.f32, p.BN, 0, false);
+    int stages = static_cast<int>((kSmemBudget - 2048 - ystage) / stage);
     p.stages = stages > 8 ? 8 : stages;
     if (p.stages < 2) return fail(CONV_ERR_UNSUPPORTED, "tile does not fit in shared memory");
-    p.smem = igemm_smem_bytes(p.f32, p.BN, p.stages);
+    p.smem = igemm_smem_bytes(p.f32, p.BN, p.stages, p.tma_out);
 
     size_t off = 0;
     p.off_xcopy = off;
@@ -565,6 +570,18 @@ int forward_impl(bool explicit_im2col, const void *x, const void *w_packed, cons
     kp.status = dev->status;
     kp.timeout_ns = g_timeout_ns;
     kp.starve = g_starve;
+    kp.tma_out = (p.tma_out && p.splits == 1) ? 1 : 0;
+    if (kp.tma_out) {
+        cuuint64_t dims[2] = {static_cast<cuuint64_t>(C_out), static_cast<cuuint64_t>(p.M)};
+        cuuint64_t strides[1] = {static_cast<cuuint64_t>(C_out) * p.elt};
+        cuuint32_t box[2] = {32, 32};
+        cuuint32_t estr[2] = {1, 1};
+        CUresult r = g_encode_tiled(&kp.tmap_y, tma_type(p), 2, y, dims, strides, box, estr,
+                                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                                    CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS)
+            return fail(CONV_ERR_CUDA, "cuTensorMapEncodeTiled (output) failed (%d)", static_cast<int>(r));
+    }
 
     if (p.xcopy) {
         cudaError_t e = layout == CONV_NCHW

@@ -33,6 +33,7 @@ enum DeviceStatus : int {
 struct IgemmParams {
     CUtensorMap tmap_a;  // A operand: im2col-mode map of x (NHWC) or tiled map of X_col
     CUtensorMap tmap_b;  // B operand: tiled map of the packed weights {Kp, Cout_g, groups}
+    CUtensorMap tmap_y;  // tma_out: y as {C_out, M}, 32 x 32 boxes with 64-byte swizzle
     int M;               // N * Ho * Wo
     int HoWo, Wo;
     int stride, pad, dilation;
@@ -53,6 +54,7 @@ struct IgemmParams {
     const void *bias;
     int out_mode;
     int vec_ok;          // 16-byte stores allowed for full chunks in NHWC / partial mode
+    int tma_out;         // bf16 NHWC output staged in shared memory and stored by TMA
     int *status;
     long long timeout_ns;
     int starve;          // test hook: issue no loads
@@ -92,7 +94,7 @@ struct GatherParams {
 // Launchers (igemm.cu, gather.cu, layout.cu).  All return cudaSuccess or the launch error.
 cudaError_t launch_igemm(const IgemmParams &p, bool f32, int cb_bytes, bool im2col, int grid,
                          size_t smem_bytes, cudaStream_t stream);
-size_t igemm_smem_bytes(bool f32, int BN, int stages);
+size_t igemm_smem_bytes(bool f32, int BN, int stages, bool tma_out);
 cudaError_t launch_gather(const GatherParams &p, bool f32, int grid, size_t smem, cudaStream_t stream);
 size_t gather_smem_bytes(bool f32, int BN, int Kpad, size_t halo_bytes, size_t out_stage_bytes);
 int gather_max_stages();

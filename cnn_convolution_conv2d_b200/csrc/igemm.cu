@@ -43,9 +43,15 @@ constexpr int kMmaWarp = 1;
 constexpr int kEpiWarp0 = 2;
 constexpr int kCvtWarp0 = 6;
 constexpr int kMaxBNf32 = 128;            // widest fp32 tile: its accumulator row lives in registers
+constexpr int kStageBufBytes = 32 * 64;   // tma_out: one 32-row x 32-column bf16 block
+constexpr int kYStageBytes = 8 * 2 * kStageBufBytes;  // two buffers per epilogue warp
 
+// bf16: warps 2..9 drain the accumulator (two per tensor-memory lane quarter, each
+// taking half of the columns); fp32: warps 2..5 drain, warps 6..9 split operands.
 template <bool kF32>
-constexpr int threads_for() { return kF32 ? 320 : 192; }
+__host__ __device__ constexpr int epi_warps() { return kF32 ? 4 : 8; }
+template <bool kF32>
+__host__ __device__ constexpr int threads_for() { return 320; }
 
 __host__ __device__ inline uint32_t stage_bytes(bool f32, int BN) {
     return static_cast<uint32_t>((kAStageBytes + BN * kStageRowBytes) * (f32 ? 2 : 1));
@@ -188,7 +194,7 @@ __global__ void __launch_bounds__(threads_for<kF32>(), 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&sb.acc_full[i], 1);
-            mbar_init(&sb.acc_empty[i], 4);
+            mbar_init(&sb.acc_empty[i], epi_warps<kF32>());
         }
         mbar_init(&sb.drain, 1);
         sb.abort = 0;
@@ -324,14 +330,21 @@ __global__ void __launch_bounds__(threads_for<kF32>(), 1)
             }
         }
         __syncwarp();
-    } else if (warp < kEpiWarp0 + 4) {
+    } else if (warp < kEpiWarp0 + epi_warps<kF32>()) {
         // ------------------------------------------------------------ epilogue ---
         const int quarter = warp & 3;  // tensor-memory lanes [32*quarter, 32*quarter + 32)
+        // columns of the tile this warp drains: all (fp32), or one half (bf16), in
+        // multiples of 32 so that TMA-store blocks never straddle two warps
+        const int half = (warp - kEpiWarp0) >> 2;
+        const int cspan = kF32 ? BN : ((BN / 2 + 31) & ~31);
+        const int c_lo = min(BN, half * cspan), c_hi = min(BN, c_lo + cspan);
         const int row = quarter * 32 + lane;
         int abuf = 0;
         uint32_t aphase = 0;
         const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
         const OutDesc out = out_desc(p);
+        uint8_t *ystage = ring + static_cast<size_t>(p.stages) * sbytes;  // tma_out staging
+        int sbi = 0;
         for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
             const Unit t = decode_unit(p, u);
             const int m = t.mtile * kBM + row;
@@ -373,12 +386,82 @@ __global__ void __launch_bounds__(threads_for<kF32>(), 1)
 #pragma unroll
                 for (int c = 0; c < kMaxBNf32 / 16; ++c)
                     if (c * 16 < BN) store16<kF32>(out, m, t.g, t.ntile * BN + c * 16, t.split, &acc[c * 16]);
+            } else if (p.tma_out) {
+                // bf16 channels-last output through shared memory: per block of 32 columns
+                // each thread writes its row's 64 bytes into this warp's staging buffer
+                // (64-byte swizzle: 16-byte chunk q of row r goes to chunk q ^ ((r >> 1) & 3),
+                // conflict-free), then one lane stores the 32 x 32 block with TMA; two
+                // buffers per warp let the next block fill while the previous store reads.
+                const bool ok = mbar_wait(&sb.acc_full[abuf], aphase, wd, kDevTimeoutAccFull);
+                if (!__all_sync(0xffffffffu, ok)) break;
+                tc_fence_after_sync();
+                const uint32_t taddr = tmem_base + lane_base + static_cast<uint32_t>(abuf * BN);
+                const int mrow0 = t.mtile * kBM + quarter * 32;
+                const int col0 = t.g * p.Cout_g + t.ntile * BN;
+                if (c_lo >= c_hi) {  // nothing to drain in this half: release at once
+                    tc_fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sb.acc_empty[abuf]);
+                }
+                for (int c = c_lo; c < c_hi; c += 32) {
+                    uint32_t r[2][16];
+                    tmem_ld_x16(taddr + static_cast<uint32_t>(c), r[0]);
+                    tmem_ld_x16(taddr + static_cast<uint32_t>(c + 16), r[1]);
+                    tmem_ld_wait();
+                    if (c + 32 >= c_hi) {  // this warp's part of the accumulator is read
+                        tc_fence_before_sync();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&sb.acc_empty[abuf]);
+                    }
+                    float bv[32];
+                    if (p.bias) {
+                        const uint4 *b4 = reinterpret_cast<const uint4 *>(
+                            static_cast<const __nv_bfloat16 *>(p.bias) + col0 + c);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const uint4 w = __ldg(b4 + q);
+                            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                            for (int h = 0; h < 4; ++h) {
+                                bv[8 * q + 2 * h] = __uint_as_float(ws[h] << 16);
+                                bv[8 * q + 2 * h + 1] = __uint_as_float(ws[h] & 0xFFFF0000u);
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) bv[i] = 0.f;
+                    }
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const float v0 = __uint_as_float(r[(2 * i) >> 4][(2 * i) & 15]) + bv[2 * i];
+                        const float v1 = __uint_as_float(r[(2 * i + 1) >> 4][(2 * i + 1) & 15]) + bv[2 * i + 1];
+                        __nv_bfloat162 h = __floats2bfloat162_rn(v0, v1);
+                        pk[i] = *reinterpret_cast<uint32_t *>(&h);
+                    }
+                    if (lane == 0) bulk_wait_group_read<1>();  // this buffer's previous store has read it
+                    __syncwarp();
+                    uint8_t *buf = ystage + ((warp - kEpiWarp0) * 2 + sbi) * kStageBufBytes;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        *reinterpret_cast<uint4 *>(buf + lane * 64 + ((q ^ ((lane >> 1) & 3)) * 16)) =
+                            make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0 && mrow0 < p.M) {
+                        tma_store_2d(&p.tmap_y, buf, col0 + c, mrow0);
+                        bulk_commit_group();
+                    }
+                    sbi ^= 1;
+                }
+                abuf ^= 1;
+                if (abuf == 0) aphase ^= 1u;
             } else {
                 const bool ok = mbar_wait(&sb.acc_full[abuf], aphase, wd, kDevTimeoutAccFull);
                 if (!__all_sync(0xffffffffu, ok)) break;
                 tc_fence_after_sync();
                 const uint32_t taddr = tmem_base + lane_base + static_cast<uint32_t>(abuf * BN);
-                for (int c = 0; c < BN; c += 16) {
+                for (int c = c_lo; c < c_hi; c += 16) {
                     uint32_t r[16];
                     tmem_ld_x16(taddr + static_cast<uint32_t>(c), r);
                     tmem_ld_wait();
@@ -394,6 +477,7 @@ __global__ void __launch_bounds__(threads_for<kF32>(), 1)
                 if (abuf == 0) aphase ^= 1u;
             }
         }
+        if (p.tma_out && lane == 0) bulk_wait_group_all();  // stores done before exit
     } else if constexpr (kF32) {
         // ------------------------------------------- fp32 -> tf32 hi/lo split ---
         const int tid = (warp - kCvtWarp0) * 32 + lane;  // 0..127
@@ -474,9 +558,9 @@ cudaError_t launch_cb(const IgemmParams &p, int cb, int grid, size_t smem, cudaS
 
 }  // namespace
 
-size_t igemm_smem_bytes(bool f32, int BN, int stages) {
+size_t igemm_smem_bytes(bool f32, int BN, int stages, bool tma_out) {
     return 1024 /* alignment slack */ + kBarrierBlock +
-           static_cast<size_t>(stages) * stage_bytes(f32, BN);
+           static_cast<size_t>(stages) * stage_bytes(f32, BN) + (tma_out ? kYStageBytes : 0);
 }
 
 int igemm_threads(bool f32) { return f32 ? threads_for<true>() : threads_for<false>(); }
