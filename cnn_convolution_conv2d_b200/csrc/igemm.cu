@@ -87,15 +87,37 @@ struct Unit {
 };
 
 __device__ __forceinline__ Unit decode_unit(const IgemmParams &p, int u) {
+    // 32-bit arithmetic, and no division where a factor is 1: this runs once per
+    // tile on the issuing threads, where a 64-bit division costs about as much as
+    // a stage of MMAs.
     Unit t;
-    t.split = u % p.splits;
-    int r = u / p.splits;
-    t.ntile = r % p.n_ntiles;
-    r /= p.n_ntiles;
-    t.g = r % p.groups;
-    t.mtile = r / p.groups;
-    t.k0 = static_cast<int>((static_cast<long long>(t.split) * p.kstages) / p.splits);
-    t.k1 = static_cast<int>((static_cast<long long>(t.split + 1) * p.kstages) / p.splits);
+    int r = u;
+    t.split = 0;
+    t.ntile = 0;
+    t.g = 0;
+    if (p.splits > 1) {
+        const int q = r / p.splits;
+        t.split = r - q * p.splits;
+        r = q;
+    }
+    if (p.n_ntiles > 1) {
+        const int q = r / p.n_ntiles;
+        t.ntile = r - q * p.n_ntiles;
+        r = q;
+    }
+    if (p.groups > 1) {
+        const int q = r / p.groups;
+        t.g = r - q * p.groups;
+        r = q;
+    }
+    t.mtile = r;
+    if (p.splits > 1) {
+        t.k0 = (t.split * p.kstages) / p.splits;  // kstages * splits < 2^31 (checked by the host)
+        t.k1 = ((t.split + 1) * p.kstages) / p.splits;
+    } else {
+        t.k0 = 0;
+        t.k1 = p.kstages;
+    }
     return t;
 }
 
@@ -235,6 +257,20 @@ __global__ void __launch_bounds__(threads_for<kF32>(), 1)
                     h0 = oh * p.stride - p.pad;
                     w0 = ow * p.stride - p.pad;
                 }
+                // Filter tap (kh, kw) and channel block of the next plane, stepped
+                // along instead of divided out per plane; past the last plane (the
+                // padding of the last stage, whose weights are zero) the tap stays at
+                // the last one so that the load is still well formed.
+                int cblk = 0, kh = 0, kw = 0, tap = 0;
+                if constexpr (kIm2col) {
+                    if (t.k0 > 0) {
+                        const int plane0 = t.k0 * kNP;
+                        tap = plane0 / p.nCB;
+                        cblk = plane0 - tap * p.nCB;
+                        kh = tap / p.Kw;
+                        kw = tap - kh * p.Kw;
+                    }
+                }
                 for (int ks = t.k0; ks < t.k1; ++ks) {
                     if (!mbar_wait(&sb.empty[stage], phase ^ 1u, wd, kDevTimeoutEmpty)) {
                         ok = false;
@@ -248,15 +284,22 @@ __global__ void __launch_bounds__(threads_for<kF32>(), 1)
                             const int plane = ks * kNP + j;
                             const int kelem = plane * kCBe;  // offset in the group's reduction
                             if constexpr (kIm2col) {
-                                const int tap = min(plane / p.nCB, p.taps - 1);
-                                const int cblk = plane - (plane / p.nCB) * p.nCB;
-                                const int kh = tap / p.Kw;
-                                const int kw = tap - kh * p.Kw;
+                                const bool in = tap < p.taps;
+                                const int khc = in ? kh : (p.taps - 1) / p.Kw;
+                                const int kwc = in ? kw : p.Kw - 1;
                                 const int c = t.g * p.Cpg + cblk * kCBe;
                                 tma_load_im2col_4d(st + j * (kBM * kCB), &p.tmap_a, &sb.full[stage],
                                                    c, w0, h0, img,
-                                                   static_cast<uint16_t>(kw * p.dilation),
-                                                   static_cast<uint16_t>(kh * p.dilation));
+                                                   static_cast<uint16_t>(kwc * p.dilation),
+                                                   static_cast<uint16_t>(khc * p.dilation));
+                                if (++cblk == p.nCB) {
+                                    cblk = 0;
+                                    ++tap;
+                                    if (++kw == p.Kw) {
+                                        kw = 0;
+                                        ++kh;
+                                    }
+                                }
                             } else {
                                 tma_load_2d(st + j * (kBM * kCB), &p.tmap_a, &sb.full[stage],
                                             t.g * p.Kp + kelem, m0);

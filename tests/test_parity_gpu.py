@@ -86,6 +86,10 @@ EDGE = [  # N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups
     (2, 3, 32, 32, 24, 7, 7, 2, 3, 1, 1),    # Ho*Wo = 256: input rows staged by TMA (bf16)
     (2, 3, 16, 32, 8, 3, 3, 1, 1, 1, 1),     # Ho*Wo = 512: staged rows, 3x3 (fp32 too)
     (1, 2, 48, 48, 16, 5, 5, 3, 2, 1, 1),    # staged rows with stride 3
+    (2, 48, 7, 9, 40, 1, 1, 1, 0, 1, 1),     # 1x1 stride 1: x read as the im2col matrix, M < one tile
+    (3, 40, 10, 13, 24, 1, 1, 1, 0, 1, 1),   # ... 40 channels (80- or 160-byte rows), ragged last tile
+    (1, 64, 15, 15, 96, 1, 1, 1, 0, 1, 4),   # ... grouped, 16 channels per group
+    (1, 32, 6, 6, 32, 1, 1, 1, 0, 3, 1),     # ... dilation has no effect on a 1x1 filter
 ]
 
 
@@ -103,7 +107,7 @@ def test_edge_shapes(shape, layout, dtype):
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("explicit", [False, True])
 @pytest.mark.parametrize("shape", [(2, 3, 9, 11, 4, 3, 3, 2, 1, 1, 1), (2, 16, 12, 12, 32, 3, 3, 1, 1, 1, 1),
-                                   (1, 32, 10, 10, 64, 3, 3, 1, 1, 2, 4)],
+                                   (1, 32, 10, 10, 64, 3, 3, 1, 1, 2, 4), (2, 64, 11, 12, 48, 1, 1, 1, 0, 1, 1)],
                          ids=lambda s: "x".join(map(str, s)))
 def test_small_integers_bit_exact(shape, explicit, dtype):
     """Integer inputs in [-2, 2]: every partial sum is exact, so outputs match exactly."""
