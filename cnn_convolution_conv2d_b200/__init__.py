@@ -50,6 +50,7 @@ SIGNATURES = {
     "conv2d_set_main_kernel_events": ([_P, _P], _I),
     "conv2d_kernel_launch_count": ([ctypes.POINTER(ctypes.c_ulonglong)], _I),
     "conv2d_debug_set_watchdog": ([_L, _I], _I),
+    "conv2d_debug_set_pair_mode": ([_I], _I),
 }
 
 _lib = None
@@ -244,6 +245,11 @@ def conv2d_kernel_launch_count() -> int:
 
 def conv2d_debug_set_watchdog(timeout_ns: int = 0, starve_loads: bool = False):
     _check(load().conv2d_debug_set_watchdog(int(timeout_ns), 1 if starve_loads else 0))
+
+
+def conv2d_debug_set_pair_mode(mode: int = 0):
+    """0: CTA-pair kernel when it pays, 1: whenever eligible, 2: never (test hook)."""
+    _check(load().conv2d_debug_set_pair_mode(int(mode)))
 
 
 # ------------------------------------------------------------- convenience ---

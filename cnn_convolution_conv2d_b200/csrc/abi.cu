@@ -6,6 +6,7 @@
 #include <cstdio>
 #include <cstring>
 #include <atomic>
+#include <map>
 #include <mutex>
 #include <string>
 
@@ -56,6 +57,8 @@ DeviceInfo g_devices[kMaxDevices];
 std::mutex g_mutex;
 long long g_timeout_ns = kDefaultTimeoutNs;
 int g_starve = 0;
+int g_pair_mode = 0;  // CTA pairs: 0 when they pay, 1 whenever eligible, 2 never
+std::map<long long, int> g_pair_clusters;  // see pair_cluster_limit
 cudaEvent_t g_main_start = nullptr, g_main_stop = nullptr;
 std::atomic<unsigned long long> g_launches{0};
 
@@ -132,6 +135,7 @@ struct Plan {
     int Kc, Kpad;   // its compact reduction length and padded length
     bool xcopy;     // x goes through the channels-last padding kernel first
     bool direct_a;  // 1x1, stride 1, no padding: X_col is x itself, read with tiled loads
+    bool pair;      // CTA-pair kernel: units of 256 rows, M = 256 MMAs over an SM pair
     int cb;         // bytes of channels per plane row (16, 32, 64 or 128)
     int BN, taps, nCB, planes, kstages, Kp;
     int n_mtiles, n_ntiles, splits, units, stages;
@@ -185,7 +189,7 @@ GatherImages gather_images(int C_out, int C_in, int Kh, int Kw, int groups, int 
 // made before a device is known use the device's count when one is current).
 int make_plan(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stride, int pad,
               int dilation, int groups, conv_dtype_t dtype, conv_layout_t layout,
-              bool explicit_im2col, int sms, Plan *P) {
+              bool explicit_im2col, int sms, Plan *P, bool allow_pair = true) {
     if (N < 1 || C_in < 1 || H < 1 || W < 1 || C_out < 1 || Kh < 1 || Kw < 1)
         return fail(CONV_ERR_INVALID_ARG, "sizes must be >= 1 (N=%d C_in=%d H=%d W=%d C_out=%d Kh=%d Kw=%d)",
                     N, C_in, H, W, C_out, Kh, Kw);
@@ -315,7 +319,7 @@ int make_plan(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stri
     p.Kp = p.taps * p.Cpg;
     if (p.kstages > (1 << 26)) return fail(CONV_ERR_UNSUPPORTED, "reduction too long (%d stages)", p.kstages);
     p.n_mtiles = static_cast<int>((p.M + 127) / 128);
-    const long long base = static_cast<long long>(p.n_mtiles) * p.n_ntiles * groups;
+    long long base = static_cast<long long>(p.n_mtiles) * p.n_ntiles * groups;
     if (base >= (1LL << 31)) return fail(CONV_ERR_UNSUPPORTED, "too many tiles");
     p.splits = 1;
     if (sms > 0 && base < sms) {
@@ -324,17 +328,30 @@ int make_plan(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stri
         s = s < 16 ? s : 16;
         if (s >= 2) p.splits = s;
     }
+    // CTA pairs (bf16): each SM stages half of the weight tile and the pair's MMAs
+    // read the other half from the peer, which halves the weight traffic and the
+    // shared-memory bandwidth spent on it.  Used when the 256-row units still give
+    // every SM pair work; the test hook can force or forbid them.
+    const long long pair_units = ((p.M + 255) / 256) * p.n_ntiles * groups;
+    const bool pair_ok = allow_pair && !p.f32 && p.BN % 32 == 0 && g_pair_mode != 2;
+    if (pair_ok && ((p.splits == 1 && sms > 0 && pair_units >= sms / 2) || g_pair_mode == 1)) {
+        p.pair = true;
+        p.splits = 1;
+        p.n_mtiles = static_cast<int>((p.M + 255) / 256);
+        base = pair_units;
+    }
     p.units = static_cast<int>(base * p.splits);
     // bf16 channels-last output leaves through shared memory and TMA stores when
     // every 32-column block of a tile lies inside its group's columns.
     p.tma_out = !p.f32 && layout == CONV_NHWC && p.splits == 1 &&
                 p.BN % 32 == 0 && p.Cout_g % p.BN == 0 && (C_out * p.elt) % 16 == 0;
-    const size_t stage = static_cast<size_t>(128 + p.BN) * 128 * (p.f32 ? 2 : 1);
-    const size_t ystage = igemm_smem_bytes(p.f32, p.BN, 0, p.tma_out) - igemm_smem_bytes(p.f32, p.BN, 0, false);
+    const int bn_local = p.pair ? p.BN / 2 : p.BN;  // B rows staged per CTA
+    const size_t stage = static_cast<size_t>(128 + bn_local) * 128 * (p.f32 ? 2 : 1);
+    const size_t ystage = igemm_smem_bytes(p.f32, bn_local, 0, p.tma_out) - igemm_smem_bytes(p.f32, bn_local, 0, false);
     int stages = static_cast<int>((kSmemBudget - 2048 - ystage) / stage);
     p.stages = stages > 8 ? 8 : stages;
     if (p.stages < 2) return fail(CONV_ERR_UNSUPPORTED, "tile does not fit in shared memory");
-    p.smem = igemm_smem_bytes(p.f32, p.BN, p.stages, p.tma_out);
+    p.smem = igemm_smem_bytes(p.f32, bn_local, p.stages, p.tma_out);
 
     size_t off = 0;
     p.off_xcopy = off;
@@ -400,7 +417,7 @@ int encode_b(const Plan &p, const void *w_packed, CUtensorMap *map) {
                           static_cast<cuuint64_t>(p.groups)};
     cuuint64_t strides[2] = {static_cast<cuuint64_t>(p.Kp) * p.elt,
                              static_cast<cuuint64_t>(p.Kp) * p.elt * p.Cout_g};
-    cuuint32_t box[3] = {static_cast<cuuint32_t>(p.cb / p.elt), static_cast<cuuint32_t>(p.BN), 1};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(p.cb / p.elt), static_cast<cuuint32_t>(p.pair ? p.BN / 2 : p.BN), 1};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = g_encode_tiled(map, tma_type(p), 3, const_cast<void *>(w_packed), dims, strides, box,
                                 estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_for(p.cb),
@@ -500,6 +517,28 @@ int gather_impl(const Plan &p, const void *x, const void *w_packed, const void *
     return ok();
 }
 
+// Resident two-CTA clusters of the pair kernel for one configuration, asked of the
+// runtime once per configuration and device and remembered.
+int pair_cluster_limit(int cb, bool im2col, size_t smem) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    const long long key = ((static_cast<long long>(dev) * 256 + cb) * 2 + (im2col ? 1 : 0)) * 1048576 +
+                          static_cast<long long>(smem);
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        auto it = g_pair_clusters.find(key);
+        if (it != g_pair_clusters.end()) return it->second;
+    }
+    int n = 0;
+    if (igemm_pair_max_clusters(cb, im2col, smem, &n) != cudaSuccess) {
+        (void)cudaGetLastError();
+        n = 0;
+    }
+    std::lock_guard<std::mutex> lock(g_mutex);
+    g_pair_clusters[key] = n;
+    return n;
+}
+
 // Shared body of conv2d_forward and conv2d_forward_im2col_gemm.
 int forward_impl(bool explicit_im2col, const void *x, const void *w_packed, const void *bias, void *y,
                  int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stride, int pad,
@@ -516,6 +555,16 @@ int forward_impl(bool explicit_im2col, const void *x, const void *w_packed, cons
     st = make_plan(N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype, layout,
                    explicit_im2col, dev->sms, &p);
     if (st != CONV_OK) return st;
+    const bool a_im2col = !(explicit_im2col || p.direct_a);
+    int pair_clusters = 0;
+    if (p.pair) {
+        pair_clusters = pair_cluster_limit(p.cb, a_im2col, p.smem);
+        if (pair_clusters < 1) {  // the device cannot co-schedule the pair kernel: single CTAs
+            st = make_plan(N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype, layout,
+                           explicit_im2col, dev->sms, &p, false);
+            if (st != CONV_OK) return st;
+        }
+    }
     if (p.ws_total > 0 && (!workspace || workspace_bytes < p.ws_total))
         return fail(CONV_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", p.ws_total,
                     workspace ? workspace_bytes : static_cast<size_t>(0));
@@ -602,10 +651,12 @@ int forward_impl(bool explicit_im2col, const void *x, const void *w_packed, cons
                                       stride, pad, dilation, p.elt, stream);
         if ((st = check_launch(e, "im2col")) != CONV_OK) return st;
     }
-    const int grid = p.units < dev->sms ? p.units : dev->sms;
+    // one CTA per SM, or one cluster per SM pair, each looping over units of work
+    const int grid = p.pair ? 2 * (p.units < pair_clusters ? p.units : pair_clusters)
+                            : (p.units < dev->sms ? p.units : dev->sms);
     cudaEvent_t ev_start = g_main_start, ev_stop = g_main_stop;
     if (ev_start && ev_stop && (st = record_event(ev_start, stream)) != CONV_OK) return st;
-    cudaError_t e = launch_igemm(kp, p.f32, p.cb, !(explicit_im2col || p.direct_a), grid, p.smem, stream);
+    cudaError_t e = launch_igemm(kp, p.f32, p.cb, a_im2col, p.pair, grid, p.smem, stream);
     if ((st = check_launch(e, "tensor-core product")) != CONV_OK) return st;
     if (ev_start && ev_stop && (st = record_event(ev_stop, stream)) != CONV_OK) return st;
     if (p.splits > 1) {
@@ -854,6 +905,13 @@ int conv2d_debug_set_watchdog(long long timeout_ns, int starve_loads) {
     std::lock_guard<std::mutex> lock(g_mutex);
     g_timeout_ns = timeout_ns > 0 ? timeout_ns : kDefaultTimeoutNs;
     g_starve = starve_loads ? 1 : 0;
+    return ok();
+}
+
+int conv2d_debug_set_pair_mode(int mode) {
+    if (mode < 0 || mode > 2) return fail(CONV_ERR_INVALID_ARG, "pair mode must be 0, 1 or 2");
+    std::lock_guard<std::mutex> lock(g_mutex);
+    g_pair_mode = mode;
     return ok();
 }
 

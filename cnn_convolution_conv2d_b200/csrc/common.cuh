@@ -92,9 +92,14 @@ struct GatherParams {
 };
 
 // Launchers (igemm.cu, gather.cu, layout.cu).  All return cudaSuccess or the launch error.
-cudaError_t launch_igemm(const IgemmParams &p, bool f32, int cb_bytes, bool im2col, int grid,
+// pair: bf16 only, grid even, launched as clusters of two CTAs (p.n_mtiles counts
+// 256-row units, the tensor map of B has boxes of BN/2 rows).
+cudaError_t launch_igemm(const IgemmParams &p, bool f32, int cb_bytes, bool im2col, bool pair, int grid,
                          size_t smem_bytes, cudaStream_t stream);
+// Bytes of dynamic shared memory for `stages` stages holding BN rows of B each.
 size_t igemm_smem_bytes(bool f32, int BN, int stages, bool tma_out);
+// Two-CTA clusters of the pair kernel that can be resident at once.
+cudaError_t igemm_pair_max_clusters(int cb_bytes, bool im2col, size_t smem_bytes, int *clusters);
 cudaError_t launch_gather(const GatherParams &p, bool f32, int grid, size_t smem, cudaStream_t stream);
 size_t gather_smem_bytes(bool f32, int BN, int Kpad, size_t halo_bytes, size_t out_stage_bytes);
 int gather_max_stages();

@@ -133,13 +133,28 @@ __device__ __forceinline__ void wait_quiet(uint64_t *bar, uint32_t parity, uint6
 // ------------------------------------------------------------------ MMAs ---
 // Issues the tensor-core instructions for one staged block of the reduction
 // (128 bytes per operand row: kNP planes of kCB bytes).
-template <bool kF32, int kCB>
+// `BNl` is the number of B rows staged in this CTA (all BN columns, or half of
+// them for a CTA pair, whose MMAs read the other half from the peer CTA).
+template <bool kF32, int kCB, bool kPair>
+__device__ __forceinline__ void mma_one(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                        uint32_t idesc, uint32_t acc) {
+    if constexpr (kPair) {
+        mma_bf16_pair(d_tmem, a_desc, b_desc, idesc, acc);
+    } else if constexpr (kF32) {
+        mma_tf32(d_tmem, a_desc, b_desc, idesc, acc);
+    } else {
+        mma_bf16(d_tmem, a_desc, b_desc, idesc, acc);
+    }
+}
+
+template <bool kF32, int kCB, bool kPair>
 __device__ __forceinline__ void issue_stage(uint32_t a, uint32_t b, uint32_t alo, uint32_t blo,
-                                            int BN, uint32_t d_tmem, uint32_t idesc,
+                                            int BNl, uint32_t d_tmem, uint32_t idesc,
                                             bool first) {
+    static_assert(!(kF32 && kPair), "CTA pairs are bf16 only");
     constexpr int kNP = kStageRowBytes / kCB;
     const uint32_t a_plane = kBM * kCB;
-    const uint32_t b_plane = static_cast<uint32_t>(BN) * kCB;
+    const uint32_t b_plane = static_cast<uint32_t>(BNl) * kCB;
     if constexpr (kCB >= 32) {
         constexpr uint32_t kSw = kCB == 128 ? kSw128 : (kCB == 64 ? kSw64 : kSw32);
         constexpr uint32_t kSbo = 8 * kCB;  // eight rows of one swizzle atom
@@ -158,8 +173,8 @@ __device__ __forceinline__ void issue_stage(uint32_t a, uint32_t b, uint32_t alo
                     mma_tf32(d_tmem, smem_desc(a + ao, 16, kSbo, kSw),
                              smem_desc(b + bo, 16, kSbo, kSw), idesc, 1u);
                 } else {
-                    mma_bf16(d_tmem, smem_desc(a + ao, 16, kSbo, kSw),
-                             smem_desc(b + bo, 16, kSbo, kSw), idesc, acc);
+                    mma_one<false, kCB, kPair>(d_tmem, smem_desc(a + ao, 16, kSbo, kSw),
+                                               smem_desc(b + bo, 16, kSbo, kSw), idesc, acc);
                 }
             }
         }
@@ -178,17 +193,21 @@ __device__ __forceinline__ void issue_stage(uint32_t a, uint32_t b, uint32_t alo
                 mma_tf32(d_tmem, smem_desc(a + ao, a_plane, 128, kSwNone),
                          smem_desc(b + bo, b_plane, 128, kSwNone), idesc, 1u);
             } else {
-                mma_bf16(d_tmem, smem_desc(a + ao, a_plane, 128, kSwNone),
-                         smem_desc(b + bo, b_plane, 128, kSwNone), idesc, acc);
+                mma_one<false, kCB, kPair>(d_tmem, smem_desc(a + ao, a_plane, 128, kSwNone),
+                                           smem_desc(b + bo, b_plane, 128, kSwNone), idesc, acc);
             }
         }
     }
 }
 
 // ---------------------------------------------------------------- kernel ---
-template <bool kF32, int kCB, bool kIm2col>
+// kPair: launched in clusters of two CTAs on an SM pair; each unit of work is 256
+// output pixels (128 per CTA) x BN channels, computed by M = 256 pair MMAs issued from
+// the even CTA, with each CTA staging its own 128 rows of A and BN/2 rows of B.
+template <bool kF32, int kCB, bool kIm2col, bool kPair>
 __global__ void __launch_bounds__(threads_for<kF32>(), 1)
     igemm_kernel(const __grid_constant__ IgemmParams p) {
+    static_assert(!(kF32 && kPair), "CTA pairs are bf16 only");
     constexpr int kElt = kF32 ? 4 : 2;
     constexpr int kCBe = kCB / kElt;              // channels (elements) per plane row
     constexpr int kNP = kStageRowBytes / kCB;     // planes per stage
@@ -202,11 +221,18 @@ __global__ void __launch_bounds__(threads_for<kF32>(), 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int BN = p.BN;
-    const uint32_t sbytes = stage_bytes(kF32, BN);
+    // CTA pairs: rank 0 issues the MMAs and owns the full / acc_empty barriers
+    const uint32_t rank = kPair ? cluster_ctarank() : 0u;
+    const int unit0 = kPair ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+    const int ustep = kPair ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+    constexpr int kUnitRows = kPair ? 2 * kBM : kBM;  // output pixels per unit of work
+    const int row_off = static_cast<int>(rank) * kBM;  // this CTA's rows within a unit
+    const int BNl = kPair ? BN / 2 : BN;               // B rows staged in this CTA
+    const uint32_t sbytes = stage_bytes(kF32, BNl);
     const uint32_t b_off = kAStageBytes;
-    const uint32_t alo_off = kAStageBytes + BN * kStageRowBytes;
+    const uint32_t alo_off = kAStageBytes + BNl * kStageRowBytes;
     const uint32_t blo_off = alo_off + kAStageBytes;
-    const uint32_t tx_bytes = kAStageBytes + BN * kStageRowBytes;
+    const uint32_t tx_bytes = (kAStageBytes + BNl * kStageRowBytes) * (kPair ? 2u : 1u);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.stages; ++s) {
@@ -216,20 +242,29 @@ __global__ void __launch_bounds__(threads_for<kF32>(), 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&sb.acc_full[i], 1);
-            mbar_init(&sb.acc_empty[i], epi_warps<kF32>());
+            mbar_init(&sb.acc_empty[i], epi_warps<kF32>() * (kPair ? 2 : 1));
         }
         mbar_init(&sb.drain, 1);
         sb.abort = 0;
         fence_mbar_init();
     }
     if (warp == kMmaWarp) {
-        tmem_alloc(&sb.tmem_base, p.tmem_cols);
-        tmem_relinquish();
+        if constexpr (kPair) {
+            tmem_alloc_pair(&sb.tmem_base, p.tmem_cols);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(&sb.tmem_base, p.tmem_cols);
+            tmem_relinquish();
+        }
     }
     tc_fence_before_sync();
     __syncthreads();
+    if constexpr (kPair) cluster_sync();  // the peer's barriers exist before anyone signals them
     tc_fence_after_sync();
     const uint32_t tmem_base = sb.tmem_base;
+    // shared::cluster addresses of rank 0's full and acc_empty barriers
+    const uint32_t full0 = kPair ? mapa_shared(smem_addr(&sb.full[0]), 0u) : 0u;
+    const uint32_t acc_empty0 = kPair ? mapa_shared(smem_addr(&sb.acc_empty[0]), 0u) : 0u;
 
     Watchdog wd;
     wd.abort = &sb.abort;
@@ -245,9 +280,12 @@ __global__ void __launch_bounds__(threads_for<kF32>(), 1)
             uint32_t phase = 0;
             long long loads_issued = 0;
             bool ok = true;
-            for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
+            for (int u = unit0; ok && u < p.units; u += ustep) {
                 const Unit t = decode_unit(p, u);
-                const int m0 = t.mtile * kBM;
+                // A rows of this CTA; the odd CTA of a pair past the last row tile
+                // reloads that tile (its results are never stored)
+                const int m0 = kPair ? min(t.mtile * kUnitRows + row_off, ((p.M - 1) / kBM) * kBM)
+                                     : t.mtile * kBM;
                 int img = 0, h0 = 0, w0 = 0;
                 if constexpr (kIm2col) {
                     img = m0 / p.HoWo;
@@ -278,7 +316,9 @@ __global__ void __launch_bounds__(threads_for<kF32>(), 1)
                     }
                     uint8_t *st = ring + static_cast<size_t>(stage) * sbytes;
                     if (!p.starve) {
-                        mbar_arrive_expect_tx(&sb.full[stage], tx_bytes);
+                        // a pair's loads all count on rank 0's barrier, armed once for both
+                        if (!kPair || rank == 0) mbar_arrive_expect_tx(&sb.full[stage], tx_bytes);
+                        const uint32_t fbar = full0 + 8u * static_cast<uint32_t>(stage);
 #pragma unroll
                         for (int j = 0; j < kNP; ++j) {
                             const int plane = ks * kNP + j;
@@ -288,10 +328,15 @@ __global__ void __launch_bounds__(threads_for<kF32>(), 1)
                                 const int khc = in ? kh : (p.taps - 1) / p.Kw;
                                 const int kwc = in ? kw : p.Kw - 1;
                                 const int c = t.g * p.Cpg + cblk * kCBe;
-                                tma_load_im2col_4d(st + j * (kBM * kCB), &p.tmap_a, &sb.full[stage],
-                                                   c, w0, h0, img,
-                                                   static_cast<uint16_t>(kwc * p.dilation),
-                                                   static_cast<uint16_t>(khc * p.dilation));
+                                if constexpr (kPair)
+                                    tma_load_im2col_4d_pair(st + j * (kBM * kCB), &p.tmap_a, fbar, c, w0, h0,
+                                                            img, static_cast<uint16_t>(kwc * p.dilation),
+                                                            static_cast<uint16_t>(khc * p.dilation));
+                                else
+                                    tma_load_im2col_4d(st + j * (kBM * kCB), &p.tmap_a, &sb.full[stage],
+                                                       c, w0, h0, img,
+                                                       static_cast<uint16_t>(kwc * p.dilation),
+                                                       static_cast<uint16_t>(khc * p.dilation));
                                 if (++cblk == p.nCB) {
                                     cblk = 0;
                                     ++tap;
@@ -301,11 +346,18 @@ __global__ void __launch_bounds__(threads_for<kF32>(), 1)
                                     }
                                 }
                             } else {
-                                tma_load_2d(st + j * (kBM * kCB), &p.tmap_a, &sb.full[stage],
-                                            t.g * p.Kp + kelem, m0);
+                                if constexpr (kPair)
+                                    tma_load_2d_pair(st + j * (kBM * kCB), &p.tmap_a, fbar, t.g * p.Kp + kelem, m0);
+                                else
+                                    tma_load_2d(st + j * (kBM * kCB), &p.tmap_a, &sb.full[stage],
+                                                t.g * p.Kp + kelem, m0);
                             }
-                            tma_load_3d(st + b_off + j * (BN * kCB), &p.tmap_b, &sb.full[stage],
-                                        kelem, t.ntile * BN, t.g);
+                            if constexpr (kPair)
+                                tma_load_3d_pair(st + b_off + j * (BNl * kCB), &p.tmap_b, fbar, kelem,
+                                                 t.ntile * BN + static_cast<int>(rank) * BNl, t.g);
+                            else
+                                tma_load_3d(st + b_off + j * (BN * kCB), &p.tmap_b, &sb.full[stage],
+                                            kelem, t.ntile * BN, t.g);
                         }
                         ++loads_issued;
                     }
@@ -315,7 +367,26 @@ __global__ void __launch_bounds__(threads_for<kF32>(), 1)
                     }
                 }
             }
-            if (*wd.abort && loads_issued > 0) {
+            if constexpr (kPair) {
+                if (!*wd.abort) {
+                    // Wait until the MMAs have released every slot, so that no commit
+                    // from rank 0 is still on its way to this CTA's barriers at exit.
+                    for (int i = 0; i < p.stages; ++i) {
+                        if (!mbar_wait(&sb.empty[stage], phase ^ 1u, wd, kDevTimeoutEmpty)) break;
+                        if (++stage == p.stages) {
+                            stage = 0;
+                            phase ^= 1u;
+                        }
+                    }
+                }
+                if (*wd.abort && loads_issued > 0) {
+                    // A pair's loads complete on rank 0's barriers: give the copies
+                    // still in flight a fixed, generous time to land.
+                    const uint64_t t0 = globaltimer_ns();
+                    while (globaltimer_ns() - t0 < 200000u) {
+                    }
+                }
+            } else if (*wd.abort && loads_issued > 0) {
                 // Let the copies still in flight land before the CTA goes away.
                 const long long first = loads_issued > p.stages ? loads_issued - p.stages : 0;
                 for (long long i = first; i < loads_issued; ++i)
@@ -325,14 +396,14 @@ __global__ void __launch_bounds__(threads_for<kF32>(), 1)
         }
     } else if (warp == kMmaWarp) {
         // --------------------------------------------------- tensor-core issue ---
-        if (lane == 0) {
-            const uint32_t idesc = instr_desc(kF32 ? 2u : 1u, kBM, static_cast<uint32_t>(BN));
+        if (lane == 0 && rank == 0) {
+            const uint32_t idesc = instr_desc(kF32 ? 2u : 1u, kUnitRows, static_cast<uint32_t>(BN));
             int stage = 0;
             uint32_t phase = 0;
             int abuf = 0;
             uint32_t aphase = 0;
             bool ok = true;
-            for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
+            for (int u = unit0; ok && u < p.units; u += ustep) {
                 const Unit t = decode_unit(p, u);
                 const int cs = p.chunk_stages > 0 ? p.chunk_stages : t.k1 - t.k0;
                 // Each chunk of the reduction goes into a fresh accumulator; the
@@ -353,22 +424,31 @@ __global__ void __launch_bounds__(threads_for<kF32>(), 1)
                         }
                         tc_fence_after_sync();
                         const uint32_t st = smem_addr(ring + static_cast<size_t>(stage) * sbytes);
-                        issue_stage<kF32, kCB>(st, st + b_off, st + alo_off, st + blo_off, BN,
-                                               d_tmem, idesc, ks == c0);
-                        mma_commit(&sb.empty[stage]);
+                        issue_stage<kF32, kCB, kPair>(st, st + b_off, st + alo_off, st + blo_off, BNl,
+                                                      d_tmem, idesc, ks == c0);
+                        if constexpr (kPair)
+                            mma_commit_pair(&sb.empty[stage], 0x3);  // both CTAs' slots
+                        else
+                            mma_commit(&sb.empty[stage]);
                         if (++stage == p.stages) {
                             stage = 0;
                             phase ^= 1u;
                         }
                     }
                     if (!ok) break;
-                    mma_commit(&sb.acc_full[abuf]);
+                    if constexpr (kPair)
+                        mma_commit_pair(&sb.acc_full[abuf], 0x3);
+                    else
+                        mma_commit(&sb.acc_full[abuf]);
                     abuf ^= 1;
                     if (abuf == 0) aphase ^= 1u;
                 }
             }
             if (!ok || *wd.abort) {
-                mma_commit(&sb.drain);
+                if constexpr (kPair)
+                    mma_commit_pair(&sb.drain, 0x1);
+                else
+                    mma_commit(&sb.drain);
                 wait_quiet(&sb.drain, 0, wd.timeout_ns);
             }
         }
@@ -387,10 +467,17 @@ __global__ void __launch_bounds__(threads_for<kF32>(), 1)
         const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
         const OutDesc out = out_desc(p);
         uint8_t *ystage = ring + static_cast<size_t>(p.stages) * sbytes;  // tma_out staging
+        // hands accumulator `b` back to the MMA issuer (rank 0 of a pair)
+        auto release_acc = [&](int b) {
+            if constexpr (kPair)
+                mbar_arrive_cluster(acc_empty0 + 8u * static_cast<uint32_t>(b));
+            else
+                mbar_arrive(&sb.acc_empty[b]);
+        };
         int sbi = 0;
-        for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
+        for (int u = unit0; u < p.units; u += ustep) {
             const Unit t = decode_unit(p, u);
-            const int m = t.mtile * kBM + row;
+            const int m = t.mtile * kUnitRows + row_off + row;
             if constexpr (kF32) {
                 // The tensor cores' own accumulation loses accuracy over long
                 // reductions, so each chunk of p.chunk_stages stages is accumulated afresh
@@ -421,7 +508,7 @@ __global__ void __launch_bounds__(threads_for<kF32>(), 1)
                     }
                     tc_fence_before_sync();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&sb.acc_empty[abuf]);
+                    if (lane == 0) release_acc(abuf);
                     abuf ^= 1;
                     if (abuf == 0) aphase ^= 1u;
                 }
@@ -439,12 +526,12 @@ __global__ void __launch_bounds__(threads_for<kF32>(), 1)
                 if (!__all_sync(0xffffffffu, ok)) break;
                 tc_fence_after_sync();
                 const uint32_t taddr = tmem_base + lane_base + static_cast<uint32_t>(abuf * BN);
-                const int mrow0 = t.mtile * kBM + quarter * 32;
+                const int mrow0 = t.mtile * kUnitRows + row_off + quarter * 32;
                 const int col0 = t.g * p.Cout_g + t.ntile * BN;
                 if (c_lo >= c_hi) {  // nothing to drain in this half: release at once
                     tc_fence_before_sync();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&sb.acc_empty[abuf]);
+                    if (lane == 0) release_acc(abuf);
                 }
                 for (int c = c_lo; c < c_hi; c += 32) {
                     uint32_t r[2][16];
@@ -454,7 +541,7 @@ __global__ void __launch_bounds__(threads_for<kF32>(), 1)
                     if (c + 32 >= c_hi) {  // this warp's part of the accumulator is read
                         tc_fence_before_sync();
                         __syncwarp();
-                        if (lane == 0) mbar_arrive(&sb.acc_empty[abuf]);
+                        if (lane == 0) release_acc(abuf);
                     }
                     float bv[32];
                     if (p.bias) {
@@ -515,7 +602,7 @@ __global__ void __launch_bounds__(threads_for<kF32>(), 1)
                 }
                 tc_fence_before_sync();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&sb.acc_empty[abuf]);
+                if (lane == 0) release_acc(abuf);
                 abuf ^= 1;
                 if (abuf == 0) aphase ^= 1u;
             }
@@ -527,7 +614,7 @@ __global__ void __launch_bounds__(threads_for<kF32>(), 1)
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
-        for (int u = blockIdx.x; ok && u < p.units; u += gridDim.x) {
+        for (int u = unit0; ok && u < p.units; u += ustep) {
             const Unit t = decode_unit(p, u);
             for (int ks = t.k0; ks < t.k1; ++ks) {
                 if (!mbar_wait(&sb.full[stage], phase, wd, kDevTimeoutFull)) {
@@ -572,29 +659,71 @@ __global__ void __launch_bounds__(threads_for<kF32>(), 1)
 
     tc_fence_before_sync();
     __syncthreads();
+    if constexpr (kPair) cluster_sync();  // neither CTA leaves while the pair still works
     if (warp == kMmaWarp) {
         tc_fence_after_sync();
-        tmem_dealloc(tmem_base, p.tmem_cols);
+        if constexpr (kPair)
+            tmem_dealloc_pair(tmem_base, p.tmem_cols);
+        else
+            tmem_dealloc(tmem_base, p.tmem_cols);
     }
 }
 
-template <bool kF32, int kCB, bool kIm2col>
+template <bool kF32, int kCB, bool kIm2col, bool kPair>
 cudaError_t launch_one(const IgemmParams &p, int grid, size_t smem, cudaStream_t stream) {
-    auto kern = igemm_kernel<kF32, kCB, kIm2col>;
+    auto kern = igemm_kernel<kF32, kCB, kIm2col, kPair>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    kern<<<grid, threads_for<kF32>(), smem, stream>>>(p);
+    if constexpr (kPair) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(grid));
+        cfg.blockDim = dim3(threads_for<kF32>());
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, kern, p);
+        if (e != cudaSuccess) return e;
+    } else {
+        kern<<<grid, threads_for<kF32>(), smem, stream>>>(p);
+    }
     return cudaGetLastError();
 }
 
-template <bool kF32, bool kIm2col>
+// How many two-CTA clusters of the pair kernel fit on the device at once.
+template <int kCB, bool kIm2col>
+cudaError_t pair_clusters_one(size_t smem, int *out) {
+    auto kern = igemm_kernel<false, kCB, kIm2col, true>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2);
+    cfg.blockDim = dim3(threads_for<false>());
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaOccupancyMaxActiveClusters(out, kern, &cfg);
+}
+
+template <bool kF32, bool kIm2col, bool kPair>
 cudaError_t launch_cb(const IgemmParams &p, int cb, int grid, size_t smem, cudaStream_t s) {
     switch (cb) {
-        case 128: return launch_one<kF32, 128, kIm2col>(p, grid, smem, s);
-        case 64: return launch_one<kF32, 64, kIm2col>(p, grid, smem, s);
-        case 32: return launch_one<kF32, 32, kIm2col>(p, grid, smem, s);
-        case 16: return launch_one<kF32, 16, kIm2col>(p, grid, smem, s);
+        case 128: return launch_one<kF32, 128, kIm2col, kPair>(p, grid, smem, s);
+        case 64: return launch_one<kF32, 64, kIm2col, kPair>(p, grid, smem, s);
+        case 32: return launch_one<kF32, 32, kIm2col, kPair>(p, grid, smem, s);
+        case 16: return launch_one<kF32, 16, kIm2col, kPair>(p, grid, smem, s);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -608,15 +737,35 @@ size_t igemm_smem_bytes(bool f32, int BN, int stages, bool tma_out) {
 
 int igemm_threads(bool f32) { return f32 ? threads_for<true>() : threads_for<false>(); }
 
-cudaError_t launch_igemm(const IgemmParams &p, bool f32, int cb_bytes, bool im2col, int grid,
+cudaError_t igemm_pair_max_clusters(int cb_bytes, bool im2col, size_t smem_bytes, int *clusters) {
+    *clusters = 0;
+    switch (cb_bytes) {
+        case 128: return im2col ? pair_clusters_one<128, true>(smem_bytes, clusters)
+                                : pair_clusters_one<128, false>(smem_bytes, clusters);
+        case 64: return im2col ? pair_clusters_one<64, true>(smem_bytes, clusters)
+                               : pair_clusters_one<64, false>(smem_bytes, clusters);
+        case 32: return im2col ? pair_clusters_one<32, true>(smem_bytes, clusters)
+                               : pair_clusters_one<32, false>(smem_bytes, clusters);
+        case 16: return im2col ? pair_clusters_one<16, true>(smem_bytes, clusters)
+                               : pair_clusters_one<16, false>(smem_bytes, clusters);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_igemm(const IgemmParams &p, bool f32, int cb_bytes, bool im2col, bool pair, int grid,
                          size_t smem_bytes, cudaStream_t stream) {
     if (p.stages < 2 || p.stages > kMaxStages) return cudaErrorInvalidValue;
-    if (f32) {
-        return im2col ? launch_cb<true, true>(p, cb_bytes, grid, smem_bytes, stream)
-                      : launch_cb<true, false>(p, cb_bytes, grid, smem_bytes, stream);
+    if (pair) {
+        if (f32 || grid % 2 != 0) return cudaErrorInvalidValue;
+        return im2col ? launch_cb<false, true, true>(p, cb_bytes, grid, smem_bytes, stream)
+                      : launch_cb<false, false, true>(p, cb_bytes, grid, smem_bytes, stream);
     }
-    return im2col ? launch_cb<false, true>(p, cb_bytes, grid, smem_bytes, stream)
-                  : launch_cb<false, false>(p, cb_bytes, grid, smem_bytes, stream);
+    if (f32) {
+        return im2col ? launch_cb<true, true, false>(p, cb_bytes, grid, smem_bytes, stream)
+                      : launch_cb<true, false, false>(p, cb_bytes, grid, smem_bytes, stream);
+    }
+    return im2col ? launch_cb<false, true, false>(p, cb_bytes, grid, smem_bytes, stream)
+                  : launch_cb<false, false, false>(p, cb_bytes, grid, smem_bytes, stream);
 }
 
 }  // namespace conv2d_b200

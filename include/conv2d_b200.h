@@ -226,6 +226,15 @@ int conv2d_kernel_launch_count(unsigned long long *count);
  * instead of hanging. */
 int conv2d_debug_set_watchdog(long long timeout_ns, int starve_loads);
 
+/* Test hook for the choice of kernel on bf16 problems: mode 0 (the default) uses
+ * the CTA-pair tensor-core kernel (clusters of two CTAs on an SM pair, M = 256
+ * products) when its 256-row units still give every SM pair work, 1 uses it
+ * whenever the tile shape allows it (also on problems too small to fill the
+ * device, so that the tests can compare it with the oracle in full), and 2 never
+ * uses it.  Results are the same in every mode up to the order of fp32 additions.
+ * Returns CONV_ERR_INVALID_ARG for any other mode. */
+int conv2d_debug_set_pair_mode(int mode);
+
 #ifdef __cplusplus
 }
 #endif

@@ -131,3 +131,23 @@ def test_workspace_size_without_device(lib):
 def test_watchdog_hook_accepts_settings(lib):
     cb.conv2d_debug_set_watchdog(1000, False)
     cb.conv2d_debug_set_watchdog(0, False)   # back to the default
+
+
+def test_pair_mode_hook_checks_its_argument(lib):
+    for mode in (1, 2, 0):                  # ends on the default
+        cb.conv2d_debug_set_pair_mode(mode)
+    for bad in (-1, 3):
+        with pytest.raises(cb.Conv2dError) as err:
+            cb.conv2d_debug_set_pair_mode(bad)
+        assert err.value.status == cb.CONV_ERR_INVALID_ARG
+
+
+def test_pair_mode_leaves_workspace_of_split_free_problems_unchanged(lib):
+    # the 1x1 layer needs no scratch whichever kernel runs it
+    shape = (64, 256, 56, 56, 1024, 1, 1, 1, 0, 1, 1)
+    try:
+        for mode in (0, 1, 2):
+            cb.conv2d_debug_set_pair_mode(mode)
+            assert cb.conv2d_workspace_size(*shape, cb.CONV_BF16, "nhwc") == 0
+    finally:
+        cb.conv2d_debug_set_pair_mode(0)

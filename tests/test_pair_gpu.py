@@ -1,0 +1,125 @@
+"""The CTA-pair tensor-core kernel against the oracle, through the C ABI (needs a B200).
+
+On bf16 problems large enough to give every SM pair work, the library runs the
+implicit GEMM in clusters of two CTAs: each unit is 256 output pixels, the even
+CTA issues M = 256 tensor-core products that read 128 rows of A and half of the
+weight tile from each CTA's shared memory.  Full-size workloads take that path by
+default (and are sampled in test_parity_gpu.py); here the test hook
+conv2d_debug_set_pair_mode(1) forces it onto problems small enough for the oracle
+to check every output, including ragged last units and a unit whose second half
+lies wholly past the last pixel.
+"""
+import numpy as np
+import pytest
+
+import cnn_convolution_conv2d_b200 as cb
+from cnn_convolution_conv2d_b200 import workloads
+import parity
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def cuda_ready():
+    import torch
+    assert torch.cuda.is_available(), "these tests need a CUDA device (run with -m 'not gpu' on CPU)"
+    from cnn_convolution_conv2d_b200 import build
+    build.build()
+    cb.load()
+    cb.conv2d_debug_set_watchdog(0, False)
+    yield
+    cb.conv2d_debug_set_pair_mode(0)
+    cb.conv2d_sync_status()
+
+
+@pytest.fixture
+def pairs_forced():
+    cb.conv2d_debug_set_pair_mode(1)
+    yield
+    cb.conv2d_debug_set_pair_mode(0)
+
+
+SMALL = {
+    "resnet3x3_bf16_nhwc": dict(N=2, H=20, W=20),   # M = 800: 4 units, the last one ragged
+    "pointwise1x1_bf16": dict(N=2, H=20, W=20),     # four column tiles of 256, tiled A loads
+    "k7_17x17_bf16": dict(N=1, C_in=128, C_out=128),  # long reduction (49 taps), one unit
+}
+
+
+@pytest.mark.parametrize("layout", ["nhwc", "nchw"])
+@pytest.mark.parametrize("name", sorted(SMALL))
+def test_pair_small_workloads(name, layout, pairs_forced):
+    cfg = parity.config(name, **SMALL[name]).scaled(layout=layout)
+    inp = workloads.make_inputs(cfg)
+    parity.assert_close(cfg, parity.run_gpu(cfg, inp), parity.run_oracle(cfg, inp), name + " (pair)")
+
+
+PAIR_EDGE = [  # N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups
+    (3, 64, 10, 13, 64, 3, 3, 1, 1, 1, 1),     # M = 390: second unit ends 122 rows short
+    (1, 32, 9, 9, 96, 1, 1, 1, 0, 1, 1),       # M = 81: the odd CTA's rows all lie past M
+    (2, 128, 12, 12, 256, 3, 3, 2, 1, 1, 1),   # stride 2, BN = 256 (128 weight rows per CTA)
+    (2, 64, 11, 11, 64, 3, 3, 1, 2, 2, 2),     # 2 groups of 32 channels, dilation 2
+    (1, 48, 16, 16, 32, 5, 5, 1, 2, 1, 1),     # 96-byte rows (32-byte planes), BN = 32
+    (1, 40, 8, 8, 64, 1, 1, 1, 0, 1, 1),       # 1x1 direct loads, 80-byte rows (16-byte planes)
+    (2, 96, 9, 9, 160, 2, 3, 1, 0, 1, 1),      # even kernel height, BN = 160
+]
+
+
+@pytest.mark.parametrize("layout", ["nhwc", "nchw"])
+@pytest.mark.parametrize("shape", PAIR_EDGE, ids=lambda s: "x".join(map(str, s)))
+def test_pair_edge_shapes(shape, layout, pairs_forced):
+    N, C_in, H, W, C_out, Kh, Kw, s, p, d, g = shape
+    cfg = workloads.ConvConfig("pair_edge", N, C_in, H, W, C_out, Kh, Kw, s, p, d, g, True, "bf16", layout,
+                               seed=sum(shape) + 11)
+    inp = workloads.make_inputs(cfg)
+    parity.assert_close(cfg, parity.run_gpu(cfg, inp), parity.run_oracle(cfg, inp), str(shape) + " (pair)")
+
+
+@pytest.mark.parametrize("shape", [(2, 32, 10, 10, 64, 3, 3, 1, 1, 1, 1), (3, 64, 9, 7, 96, 1, 1, 1, 0, 1, 1)],
+                         ids=lambda s: "x".join(map(str, s)))
+def test_pair_small_integers_bit_exact(shape, pairs_forced):
+    """Integer inputs in [-2, 2]: every partial sum is exact, so the pair kernel's
+    outputs equal the oracle's exactly."""
+    N, C_in, H, W, C_out, Kh, Kw, s, p, d, g = shape
+    cfg = workloads.ConvConfig("ints", N, C_in, H, W, C_out, Kh, Kw, s, p, d, g, True, "bf16", "nhwc",
+                               ("integers", -2, 2), ("integers", -2, 2), ("integers", -2, 2), seed=5)
+    inp = workloads.make_inputs(cfg)
+    ref = parity.run_oracle(cfg, inp)
+    assert np.abs(ref).max() <= 256
+    assert np.array_equal(parity.run_gpu(cfg, inp), ref)
+
+
+def test_pair_and_single_cta_kernels_agree_on_repeated_calls():
+    """The same layer run with pairs forbidden, forced and back: the three results
+    agree to the bf16 rounding of one output, and repeated pair calls are identical."""
+    cfg = parity.config("resnet3x3_bf16_nhwc", N=3, H=14, W=14)
+    inp = workloads.make_inputs(cfg)
+    outs = []
+    try:
+        for mode in (2, 1, 1, 0):
+            cb.conv2d_debug_set_pair_mode(mode)
+            outs.append(parity.run_gpu(cfg, inp))
+    finally:
+        cb.conv2d_debug_set_pair_mode(0)
+    assert np.array_equal(outs[1], outs[2])
+    for o in (outs[0], outs[3]):
+        assert np.abs(o - outs[1]).max() <= 2 ** -7 * max(1.0, np.abs(o).max())
+
+
+def test_pair_watchdog_returns_timeout_instead_of_hanging(pairs_forced):
+    """With loads withheld the waits of both CTAs of every pair run out; the kernel
+    exits with TIMEOUT and the next normal call works."""
+    cfg = parity.config("resnet3x3_bf16_nhwc", N=1, H=12, W=12)
+    inp = workloads.make_inputs(cfg)
+    layer = parity.make_layer(cfg, inp)
+    x = parity.to_device_x(cfg, inp["x"])
+    try:
+        cb.conv2d_debug_set_watchdog(1_000_000, True)
+        layer(x)
+        with pytest.raises(cb.Conv2dError) as err:
+            cb.conv2d_sync_status()
+        assert err.value.status == cb.CONV_ERR_TIMEOUT
+    finally:
+        cb.conv2d_debug_set_watchdog(0, False)
+    cb.conv2d_sync_status()
+    parity.assert_close(cfg, parity.run_gpu(cfg, inp, layer=layer), parity.run_oracle(cfg, inp), "after timeout")
