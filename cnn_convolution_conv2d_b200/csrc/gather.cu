@@ -224,6 +224,16 @@ __global__ void __launch_bounds__(threads_for<kF32>(), 1) gather_kernel(const __
             // (c*R + kh*d + (oh - oh_first)*stride); chunks j >= C*Kh are padding.
             const uint32_t hstride = align1k(halo_bytes);
             const int nreal = p.C * p.Kh;
+            // bf16: word offsets of this thread's chunks [jb, je) in a staged row, and
+            // whether each is a real one (padding chunks read word 0 and are zeroed)
+            int cwo[16];
+            bool creal[16];
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const int j = jb + u;
+                creal[u] = j < je && j < nreal;
+                cwo[u] = creal[u] ? table[j].x : 0;
+            }
             int stage = 0, li = 0;
             uint32_t phase = 0;
             for (int t = blockIdx.x; t < p.n_mtiles; t += gridDim.x, ++li) {
@@ -240,6 +250,37 @@ __global__ void __launch_bounds__(threads_for<kF32>(), 1) gather_kernel(const __
                 const uint32_t *h32 = reinterpret_cast<const uint32_t *>(halo_buf + b * hstride);
                 const uint32_t *hrow = h32 + (kF32 ? ebase : (ebase >> 1));
                 const uint32_t sh = (ebase & 1) * 16u;  // bf16: half-word start within the word
+                if constexpr (!kF32) {
+                    // At most two batches of eight chunks per thread (nchunks <= 32):
+                    // all forty word loads of a batch are issued before any is used.
+                    const uint32_t slot = lane_addr + a_first + static_cast<uint32_t>(stage) * acols;
+#pragma unroll
+                    for (int bt = 0; bt < 2; ++bt) {
+                        const int j0 = jb + 8 * bt;
+                        if (j0 < je) {
+                            uint32_t w[8][5];
+#pragma unroll
+                            for (int u = 0; u < 8; ++u)
+#pragma unroll
+                                for (int i = 0; i < 5; ++i) w[u][i] = hrow[cwo[8 * bt + u] + i];
+                            uint32_t hw[32];
+#pragma unroll
+                            for (int u = 0; u < 8; ++u)
+#pragma unroll
+                                for (int i = 0; i < 4; ++i)
+                                    hw[4 * u + i] = creal[8 * bt + u] ? __funnelshift_r(w[u][i], w[u][i + 1], sh) : 0u;
+                            const uint32_t col = slot + static_cast<uint32_t>(4 * j0);
+                            if (j0 + 8 <= je && (j0 & 7) == 0) {
+                                tmem_st_x32(col, hw);
+                            } else {  // chunk pairs (every range boundary is even)
+#pragma unroll
+                                for (int q = 0; q < 4; ++q)
+                                    if (j0 + 2 * q < je) tmem_st_x8(col + 8 * q, &hw[8 * q]);
+                            }
+                        }
+                    }
+                    tmem_st_wait();
+                } else
                 build_row(a_first + static_cast<uint32_t>(stage) * acols, [&](int j, uint32_t *h, uint32_t *l) {
                     if (j < nreal) {
                         const int wo = table[j].x;
@@ -411,8 +452,6 @@ __global__ void __launch_bounds__(threads_for<kF32>(), 1) gather_kernel(const __
                     break;
                 }
                 tc_fence_after_sync();
-                const int t2 = t + 2 * static_cast<int>(gridDim.x);
-                if (p.halo && !p.starve && t2 < p.n_mtiles) issue_halo(t2, li & 1);
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(abuf * p.BN);
                 const uint32_t a_hi = tmem_base + a_first + static_cast<uint32_t>(stage) * acols;
                 const uint32_t a_lo = a_hi + lo_off;
@@ -430,6 +469,11 @@ __global__ void __launch_bounds__(threads_for<kF32>(), 1) gather_kernel(const __
                 }
                 mma_commit(&sb.empty[stage]);
                 mma_commit(&sb.acc_full[abuf]);
+                // The gather warps are done with this tile's staged rows (they arrived
+                // on full[stage]), so its buffer takes tile t + 2; issued after the
+                // products so that they are not held up by the address arithmetic.
+                const int t2 = t + 2 * static_cast<int>(gridDim.x);
+                if (p.halo && !p.starve && t2 < p.n_mtiles) issue_halo(t2, li & 1);
                 if (++stage == p.stages) {
                     stage = 0;
                     phase ^= 1u;
