@@ -314,11 +314,12 @@ def run_reference(args, cfg):
         oracle.conv2d_points(x64, w64, b64, idx[i], cfg.stride, cfg.pad, cfg.dilation, cfg.groups)
     wall = time.perf_counter() - t
     value = args.steps * points * per_point / wall / 1e12
-    sample = (f"{points} random output points per step of {cfg.name} "
-              f"({points / (cfg.N * cfg.C_out * cfg.Ho * cfg.Wo):.2e} of one forward pass)")
+    sample = (f"{points} random output points per step of {cfg.name} (drawn with replacement; "
+              f"{points / (cfg.N * cfg.C_out * cfg.Ho * cfg.Wo):.3g} forward passes' worth of outputs), "
+              f"fp64 on the host cores, no GPU")
     line = {
         "impl": "reference", "metric": metric_name(cfg), "value": value, "unit": "TFLOP/s",
-        "n_gpus": 0, "steps": args.steps, "warmup": args.warmup,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": wall / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(cfg, args, world=1),
