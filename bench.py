@@ -44,7 +44,11 @@ if ROOT not in sys.path:
 DEFAULT_WORKLOAD = "stem_bf16"
 L2_BYTES = 126 * 1000 * 1000
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_SOURCES = ["igemm.cu", "gather.cu", "epilogue.cuh", "ptx.cuh", "common.cuh"]
+# sources each measured kernel is built from (a change voids its committed ncu counters)
+KERNEL_SOURCES = {
+    "igemm_kernel": ["igemm.cu", "epilogue.cuh", "ptx.cuh", "common.cuh"],
+    "gather_kernel": ["gather.cu", "epilogue.cuh", "ptx.cuh", "common.cuh"],
+}
 
 
 # ------------------------------------------------------------ arithmetic ---
@@ -105,9 +109,9 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(kernel: str) -> str:
     h = hashlib.sha256()
-    for name in KERNEL_SOURCES:
+    for name in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, "cnn_convolution_conv2d_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -121,7 +125,7 @@ def committed_traffic(workload: str):
             d = json.load(f).get(workload)
     except (OSError, ValueError):
         return None
-    if not d or d.get("kernel_hash") != kernel_source_hash():
+    if not d or d.get("kernel") not in KERNEL_SOURCES or d.get("kernel_hash") != kernel_source_hash(d["kernel"]):
         return None
     return float(d["dram_bytes_per_launch"])
 

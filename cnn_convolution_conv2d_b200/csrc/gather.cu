@@ -533,7 +533,58 @@ __global__ void __launch_bounds__(threads_for<kF32>(), 1) gather_kernel(const __
                 const uint32_t wstride = static_cast<uint32_t>(p.cw) * 32u * kElt;
                 uint8_t *wstage = stage_out + (warp - kMmaWarp - 1) * 2 * wstride;
                 int sbi = 0;
-                for (int t = blockIdx.x; t < p.n_mtiles; t += gridDim.x) {
+                if (cb1 - cb0 == 32) {
+                    // A full 32-channel block (the first-layer shape): its biases stay in
+                    // registers, and lanes swap values in pairs so that each thread writes
+                    // whole 32-bit words (two pixels of one channel) into the
+                    // channel-major staging buffer: half the conversions and stores.
+                    uint32_t bsel[16];  // bf16 biases (exact: they came from bf16), two per word
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        __nv_bfloat162 b2 = __floats2bfloat162_rn(sbias[cb0 + 2 * i], sbias[cb0 + 2 * i + 1]);
+                        bsel[i] = *reinterpret_cast<uint32_t *>(&b2);
+                    }
+                    const bool odd = (lane & 1) != 0;
+                    for (int t = blockIdx.x; t < p.n_mtiles; t += gridDim.x) {
+                        const bool ok = mbar_wait(&sb.acc_full[abuf], aphase, wd, kDevTimeoutAccFull);
+                        if (!__all_sync(0xffffffffu, ok)) break;
+                        tc_fence_after_sync();
+                        const uint32_t taddr = tmem_base + lane_base + static_cast<uint32_t>(abuf * p.BN + cb0);
+                        uint32_t r[2][16];
+                        tmem_ld_x16(taddr, r[0]);
+                        tmem_ld_x16(taddr + 16u, r[1]);
+                        tmem_ld_wait();
+                        tc_fence_before_sync();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&sb.acc_empty[abuf]);
+                        abuf ^= 1;
+                        if (abuf == 0) aphase ^= 1u;
+                        if (lane == 0) bulk_wait_group_read<1>();  // this buffer's previous store has read it
+                        __syncwarp();
+                        uint32_t *stg32 = reinterpret_cast<uint32_t *>(wstage + sbi * wstride);
+#pragma unroll
+                        for (int k = 0; k < 16; ++k) {
+                            const float v0 = __uint_as_float(r[k >> 3][(2 * k) & 15]) + __uint_as_float(bsel[k] << 16);
+                            const float v1 = __uint_as_float(r[k >> 3][(2 * k + 1) & 15]) +
+                                             __uint_as_float(bsel[k] & 0xFFFF0000u);
+                            // even lane (pixel 2w): channel 2k of pixels 2w, 2w+1;
+                            // odd lane (pixel 2w+1): channel 2k+1 of pixels 2w, 2w+1
+                            const float recv = __shfl_xor_sync(0xffffffffu, odd ? v0 : v1, 1);
+                            __nv_bfloat162 h = odd ? __floats2bfloat162_rn(recv, v1) : __floats2bfloat162_rn(v0, recv);
+                            stg32[(2 * k + (odd ? 1 : 0)) * 16 + (lane >> 1)] = *reinterpret_cast<uint32_t *>(&h);
+                        }
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            const int m0 = t * kBM;
+                            const int img = m0 / (p.Ho * p.Wo);
+                            tma_store_3d(&p.tmap_y, stg32, m0 - img * p.Ho * p.Wo + quarter * 32, cb0, img);
+                            bulk_commit_group();
+                        }
+                        sbi ^= 1;
+                    }
+                }
+                for (int t = blockIdx.x; t < p.n_mtiles && cb1 - cb0 != 32; t += gridDim.x) {
                     const bool ok = mbar_wait(&sb.acc_full[abuf], aphase, wd, kDevTimeoutAccFull);
                     if (!__all_sync(0xffffffffu, ok)) break;
                     tc_fence_after_sync();
