@@ -99,6 +99,19 @@ def main_kernel_bytes(cfg) -> float:
     return e * (x_in + w + (cfg.C_out if cfg.bias else 0) + cfg.N * cfg.C_out * cfg.Ho * cfg.Wo)
 
 
+def xcol_bytes(cfg) -> float:
+    """Bytes of the explicit X_col matrix: M rows of groups * Kh*Kw*Cpg elements."""
+    return elt_bytes(cfg) * cfg.N * cfg.Ho * cfg.Wo * cfg.groups * cfg.Kh * cfg.Kw * padded_channels(cfg)
+
+
+def explicit_kernel_bytes(cfg) -> float:
+    """Minimum bytes of the tensor-core GEMM of the explicit path: X_col, packed
+    weights, bias, output."""
+    e = elt_bytes(cfg)
+    w = cfg.C_out * cfg.Kh * cfg.Kw * padded_channels(cfg)
+    return xcol_bytes(cfg) + e * (w + (cfg.C_out if cfg.bias else 0) + cfg.N * cfg.C_out * cfg.Ho * cfg.Wo)
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -130,9 +143,9 @@ def committed_traffic(workload: str):
     return float(d["dram_bytes_per_launch"])
 
 
-def roofline(cfg, kernel_ms: float, peaks, peak_kind: str, workload: str) -> dict:
+def roofline(cfg, kernel_ms: float, peaks, peak_kind: str, workload: str, explicit: bool = False) -> dict:
     f = flops(cfg)
-    b = main_kernel_bytes(cfg)
+    b = explicit_kernel_bytes(cfg) if explicit else main_kernel_bytes(cfg)
     ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
     if f / b >= ridge and cfg.dtype == "bf16":
         achieved = f / (kernel_ms * 1e-3) / 1e12
@@ -151,7 +164,9 @@ def roofline(cfg, kernel_ms: float, peaks, peak_kind: str, workload: str) -> dic
     out["kernel_ms"] = kernel_ms
     out["algorithmic_bytes_per_launch"] = b
     out["algorithmic_flops_per_launch"] = f
-    out["traffic"] = committed_traffic(workload)
+    out["traffic"] = None if explicit else committed_traffic(workload)
+    if explicit:
+        out["kernel"] = "igemm_kernel over the explicit X_col (tiled TMA loads, tcgen05)"
     return out
 
 
@@ -382,11 +397,12 @@ def run_ours(args, cfg):
     nsets = max(2, min(16, math.ceil(2 * L2_BYTES / set_bytes) + 1))
     xs = [x_host.to(device) for _ in range(nsets)]
     ys = [torch.empty(y_shape, dtype=dt, device=device) for _ in range(nsets)]
-    layer.workspace(cfg.N, cfg.H, cfg.W)
+    ex = args.explicit_im2col
+    layer.workspace(cfg.N, cfg.H, cfg.W, ex)
     stream = torch.cuda.current_stream()
 
     for i in range(max(args.warmup, 3)):
-        layer(xs[i % nsets], ys[i % nsets])
+        layer(xs[i % nsets], ys[i % nsets], explicit_im2col=ex)
     cb.conv2d_sync_status()
 
     # Steps per captured graph: a divisor of K, at most 512.
@@ -407,7 +423,7 @@ def run_ours(args, cfg):
         with torch.cuda.graph(graph):
             for i in range(G):
                 cb.conv2d_set_main_kernel_events(*kev[i])
-                layer(xs[i % nsets], ys[i % nsets])
+                layer(xs[i % nsets], ys[i % nsets], explicit_im2col=ex)
         cb.conv2d_set_main_kernel_events(None, None)
         launches_per_rep = cb.conv2d_kernel_launch_count() - launches0
         graph.replay()  # one untimed replay: graph upload
@@ -429,7 +445,7 @@ def run_ours(args, cfg):
         for r in range(reps):
             for i in range(G):
                 cb.conv2d_set_main_kernel_events(*kev[i])
-                layer(xs[i % nsets], ys[i % nsets])
+                layer(xs[i % nsets], ys[i % nsets], explicit_im2col=ex)
         cb.conv2d_set_main_kernel_events(None, None)
     ev1.record(stream)
     torch.cuda.synchronize()
@@ -490,13 +506,16 @@ def run_ours(args, cfg):
         cfgd["l2"] = (f"not resident: steps rotate over {nsets} input/output sets "
                       f"({nsets * set_bytes / 1e6:.0f} MB > 2x the 126 MB L2)")
         cfgd["launch"] = f"CUDA graphs of {G} steps x {reps} replays" if args.graph else "eager"
+        if ex:
+            cfgd["path"] = (f"explicit im2col + GEMM (conv2d_forward_im2col_gemm): X_col of "
+                            f"{xcol_bytes(cfg) / 1e6:.1f} MB written and read back every step")
         line = {
             "metric": metric_name(cfg), "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": cfg.dtype, "data": "synthetic (seeded; x ~ N(0,1), He-scaled weights)",
             "config": cfgd,
-            "roofline": with_write_context(roofline(cfg, kernel_ms, peaks, peak_kind, cfg.name), cfg,
+            "roofline": with_write_context(roofline(cfg, kernel_ms, peaks, peak_kind, cfg.name, ex), cfg,
                                            kernel_ms, fill_gbs),
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "TFLOP/s",
@@ -515,6 +534,51 @@ def run_ours(args, cfg):
         dist.destroy_process_group()
 
 
+def run_transpose(args, cfg):
+    """Bandwidth of the standalone layout kernels on this workload's tensors: x NCHW ->
+    channels-last (channel-padded per group), and y channels-last -> NCHW.  One GPU;
+    buffers rotate over sets larger than 2x L2; CUDA events; bytes = read + write once."""
+    import torch
+    import cnn_convolution_conv2d_b200 as cb
+    from cnn_convolution_conv2d_b200 import build
+
+    build.build()
+    cb.load()
+    device = torch.device("cuda", 0)
+    dt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+    dcode = cb.CONV_BF16 if cfg.dtype == "bf16" else cb.CONV_F32
+    e = elt_bytes(cfg)
+    cpg = padded_channels(cfg)
+    peaks, peak_kind = load_peaks()
+    lines = {}
+    cases = [("nchw_to_nhwc", cfg.N * cfg.C_in * cfg.H * cfg.W, cfg.N * cfg.H * cfg.W * cfg.groups * cpg,
+              lambda s_, d_: cb.conv2d_nchw_to_nhwc(s_, d_, cfg.N, cfg.C_in, cfg.H, cfg.W, cfg.groups, cpg, dcode)),
+             ("nhwc_to_nchw", cfg.N * cfg.C_out * cfg.Ho * cfg.Wo, cfg.N * cfg.C_out * cfg.Ho * cfg.Wo,
+              lambda s_, d_: cb.conv2d_nhwc_to_nchw(s_, d_, cfg.N, cfg.C_out, cfg.Ho, cfg.Wo, dcode))]
+    for name, n_in, n_out, fn in cases:
+        nsets = max(2, min(16, math.ceil(2 * L2_BYTES / ((n_in + n_out) * e)) + 1))
+        srcs = [torch.randn(n_in, device=device).to(dt) for _ in range(nsets)]
+        dsts = [torch.empty(n_out, dtype=dt, device=device) for _ in range(nsets)]
+        for i in range(max(args.warmup, 3)):
+            fn(srcs[i % nsets], dsts[i % nsets])
+        cb.conv2d_sync_status()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        steps = max(1, min(args.steps, 2000))
+        a.record()
+        for i in range(steps):
+            fn(srcs[i % nsets], dsts[i % nsets])
+        b.record()
+        torch.cuda.synchronize()
+        cb.conv2d_sync_status()
+        ms = a.elapsed_time(b) / steps
+        gbs = (n_in + n_out) * e / (ms * 1e-3) / 1e9
+        lines[name] = {"us_per_launch": ms * 1e3, "bytes_per_launch": (n_in + n_out) * e, "achieved_gbs": gbs,
+                       "frac_of_hbm_peak": gbs / peaks["hbm_gbs"], "sets": nsets, "launches": steps}
+    print(json.dumps({"metric": "layout transpose GB/s on 1 B200 and % of HBM copy bandwidth",
+                      "workload": cfg.name, "peak_gbs": peaks["hbm_gbs"], "peak_source": f"{peak_kind} HBM copy bandwidth",
+                      **lines}), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -526,6 +590,10 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--explicit-im2col", action="store_true",
+                    help="time the pages' formulation: explicit X_col in HBM, then the GEMM")
+    ap.add_argument("--transpose", action="store_true",
+                    help="time the standalone NCHW<->NHWC kernels on the workload's x and y instead")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -537,6 +605,11 @@ def main(argv=None):
     if args.impl == "reference":
         if rank == 0:
             run_reference(args, cfg)
+        return
+    if args.transpose:
+        if world != 1:
+            ap.error("--transpose runs on one GPU")
+        run_transpose(args, cfg)
         return
     run_ours(args, cfg)
 
