@@ -22,6 +22,72 @@ inline int grid_for(long long work, int per_block = kThreads) {
     return static_cast<int>(g);
 }
 
+// --- Transpose of the two inner dimensions of a [B][R][S] array of 2-byte elements
+// into [B][S][R] (NCHW -> NHWC with R = C, S = H*W; NHWC -> NCHW with R = H*W, S = C),
+// for R and S multiples of 8.  64 x 64 tiles through shared memory; every global access
+// is a 16-byte vector, and each warp touches four 128-byte rows per instruction.  In
+// shared memory the tile is 64 rows of 32 words (two elements per word); word w of row r
+// sits at column w ^ (r & 31), so that the row-wise stores are conflict-free and the
+// column-wise reads at most two-way.
+__global__ void __launch_bounds__(256) transpose_b16_kernel(const uint16_t *__restrict__ src,
+                                                            uint16_t *__restrict__ dst, int B, int R, int S) {
+    __shared__ uint32_t tile[64][32];
+    const int tiles_r = (R + 63) / 64, tiles_s = (S + 63) / 64;
+    const long long per_b = static_cast<long long>(tiles_r) * tiles_s;
+    const long long ntiles = static_cast<long long>(B) * per_b;
+    const int t = threadIdx.x;
+    for (long long tt = blockIdx.x; tt < ntiles; tt += gridDim.x) {
+        const long long b = tt / per_b;
+        const int rem = static_cast<int>(tt - b * per_b);
+        const int r0 = (rem / tiles_s) * 64, s0 = (rem - (rem / tiles_s) * tiles_s) * 64;
+        const uint16_t *sb = src + b * static_cast<long long>(R) * S;
+        uint16_t *db = dst + b * static_cast<long long>(R) * S;
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {  // 64 source rows x 8 vectors of 8 elements
+            const int row = (t >> 3) + 32 * k, vec = t & 7;
+            const int r = r0 + row, c = s0 + 8 * vec;
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (r < R && c < S) v = __ldg(reinterpret_cast<const uint4 *>(sb + static_cast<long long>(r) * S + c));
+            const int sw = row & 31;
+            tile[row][(4 * vec + 0) ^ sw] = v.x;
+            tile[row][(4 * vec + 1) ^ sw] = v.y;
+            tile[row][(4 * vec + 2) ^ sw] = v.z;
+            tile[row][(4 * vec + 3) ^ sw] = v.w;
+        }
+        __syncthreads();
+        {  // 64 destination rows (pairs per thread) x 8 vectors of 8 elements
+            const int vec = t & 7, wj = t >> 3;  // source rows 8*vec..+7, source word column wj
+            uint32_t w[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int row = 8 * vec + i;
+                w[i] = tile[row][wj ^ (row & 31)];
+            }
+            const int r = r0 + 8 * vec;
+            const int c = s0 + 2 * wj;  // destination rows c and c + 1
+            if (r < R) {
+                if (c < S) {
+                    const uint4 lo = make_uint4(__byte_perm(w[0], w[1], 0x5410), __byte_perm(w[2], w[3], 0x5410),
+                                                __byte_perm(w[4], w[5], 0x5410), __byte_perm(w[6], w[7], 0x5410));
+                    *reinterpret_cast<uint4 *>(db + static_cast<long long>(c) * R + r) = lo;
+                }
+                if (c + 1 < S) {
+                    const uint4 hi = make_uint4(__byte_perm(w[0], w[1], 0x7632), __byte_perm(w[2], w[3], 0x7632),
+                                                __byte_perm(w[4], w[5], 0x7632), __byte_perm(w[6], w[7], 0x7632));
+                    *reinterpret_cast<uint4 *>(db + static_cast<long long>(c + 1) * R + r) = hi;
+                }
+            }
+        }
+        __syncthreads();
+    }
+}
+
+void launch_transpose_b16(const void *src, void *dst, int B, int R, int S, cudaStream_t s) {
+    const long long tiles = static_cast<long long>(B) * ((R + 63) / 64) * ((S + 63) / 64);
+    const int grid = static_cast<int>(tiles < 148LL * 8 ? tiles : 148LL * 8);
+    transpose_b16_kernel<<<grid, 256, 0, s>>>(static_cast<const uint16_t *>(src), static_cast<uint16_t *>(dst), B, R, S);
+}
+
 template <int kElt> struct Word;
 template <> struct Word<2> { using T = uint16_t; };
 template <> struct Word<4> { using T = uint32_t; };
@@ -286,7 +352,9 @@ cudaError_t launch_nchw_to_nhwc(const void *src, void *dst, int N, int C, int H,
     const int HW = H * W;
     const int Ctot = groups * Cpg;
     const long long pixels = static_cast<long long>(N) * HW;
-    if (Ctot * elt <= 64 && (Ctot * elt) % 16 == 0) {
+    if (elt == 2 && Cpg == C / groups && C % 8 == 0 && HW % 8 == 0 && C * elt > 64) {
+        launch_transpose_b16(src, dst, N, C, HW, s);  // no channel padding: a plain transpose
+    } else if (Ctot * elt <= 64 && (Ctot * elt) % 16 == 0) {
         if (elt == 2)
             nchw_to_nhwc_small<2><<<grid_for(pixels), kThreads, 0, s>>>(src, dst, N, C, HW, groups, Cpg);
         else
@@ -316,6 +384,10 @@ cudaError_t launch_nhwc_pad(const void *src, void *dst, int N, int C, int H, int
 cudaError_t launch_nhwc_to_nchw(const void *src, void *dst, int N, int C, int H, int W, int elt,
                                 cudaStream_t s) {
     const int HW = H * W;
+    if (elt == 2 && C % 8 == 0 && HW % 8 == 0) {
+        launch_transpose_b16(src, dst, N, HW, C, s);
+        return cudaGetLastError();
+    }
     const long long tiles = static_cast<long long>(N) * ((C + 31) / 32) * ((HW + 31) / 32);
     const int grid = static_cast<int>(tiles < 148LL * 32 ? tiles : 148LL * 32);
     if (elt == 2)
