@@ -42,8 +42,17 @@ def _shape(layer, cfg):
             layer.dilation, layer.groups)
 
 
+@pytest.fixture(params=[0, 1], ids=["auto", "pairs"])
+def pair_mode(request):
+    """Each case once with the library's own kernel choice and once with the CTA-pair
+    kernel forced wherever the tile shape allows it (bf16 cases)."""
+    cb.conv2d_debug_set_pair_mode(request.param)
+    yield request.param
+    cb.conv2d_debug_set_pair_mode(0)
+
+
 @pytest.mark.parametrize("case", sorted(CASES))
-def test_noalloc_matches_forward_on_two_calls(case):
+def test_noalloc_matches_forward_on_two_calls(case, pair_mode):
     import torch
     name, kw = CASES[case]
     cfg = parity.config(name, **kw)
@@ -52,7 +61,9 @@ def test_noalloc_matches_forward_on_two_calls(case):
     x = parity.to_device_x(cfg, inp["x"])
     shape = _shape(layer, cfg)
     need = cb.conv2d_workspace_size(*shape, layer.dtype, layer.layout)
-    assert 0 < need <= cb.NOALLOC_SCRATCH_BYTES  # the case exercises the built-in scratch
+    assert need <= cb.NOALLOC_SCRATCH_BYTES
+    if pair_mode == 0:
+        assert need > 0  # the case exercises the built-in scratch (pairs need no split sums)
     ref = layer(x)                               # existing entry point, allocated workspace
     cb.conv2d_sync_status()
     want = parity.from_device_y(cfg, ref)
