@@ -82,6 +82,56 @@ __global__ void __launch_bounds__(256) transpose_b16_kernel(const uint16_t *__re
     }
 }
 
+// --- The same for 4-byte elements (R and S multiples of 4): 32 x 32 tiles, one
+// 16-byte vector (4 elements) per thread in each direction; word c of row r sits at
+// column c ^ (r & 31), conflict-free both ways.
+__global__ void __launch_bounds__(256) transpose_b32_kernel(const uint32_t *__restrict__ src,
+                                                            uint32_t *__restrict__ dst, int B, int R, int S) {
+    __shared__ uint32_t tile[32][32];
+    const int tiles_r = (R + 31) / 32, tiles_s = (S + 31) / 32;
+    const long long per_b = static_cast<long long>(tiles_r) * tiles_s;
+    const long long ntiles = static_cast<long long>(B) * per_b;
+    const int t = threadIdx.x;
+    for (long long tt = blockIdx.x; tt < ntiles; tt += gridDim.x) {
+        const long long b = tt / per_b;
+        const int rem = static_cast<int>(tt - b * per_b);
+        const int r0 = (rem / tiles_s) * 32, s0 = (rem - (rem / tiles_s) * tiles_s) * 32;
+        const uint32_t *sb = src + b * static_cast<long long>(R) * S;
+        uint32_t *db = dst + b * static_cast<long long>(R) * S;
+        {  // 32 source rows x 8 vectors of 4 elements
+            const int row = t >> 3, vec = t & 7;
+            const int r = r0 + row, c = s0 + 4 * vec;
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (r < R && c < S) v = __ldg(reinterpret_cast<const uint4 *>(sb + static_cast<long long>(r) * S + c));
+            const int sw = row & 31;
+            tile[row][(4 * vec + 0) ^ sw] = v.x;
+            tile[row][(4 * vec + 1) ^ sw] = v.y;
+            tile[row][(4 * vec + 2) ^ sw] = v.z;
+            tile[row][(4 * vec + 3) ^ sw] = v.w;
+        }
+        __syncthreads();
+        {  // 32 destination rows x 8 vectors of 4 elements
+            const int vec = t & 7, col = t >> 3;  // source rows 4*vec..+3, source column col
+            uint32_t w[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int row = 4 * vec + i;
+                w[i] = tile[row][col ^ (row & 31)];
+            }
+            const int r = r0 + 4 * vec, c = s0 + col;
+            if (r < R && c < S)
+                *reinterpret_cast<uint4 *>(db + static_cast<long long>(c) * R + r) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        __syncthreads();
+    }
+}
+
+void launch_transpose_b32(const void *src, void *dst, int B, int R, int S, cudaStream_t s) {
+    const long long tiles = static_cast<long long>(B) * ((R + 31) / 32) * ((S + 31) / 32);
+    const int grid = static_cast<int>(tiles < 148LL * 8 ? tiles : 148LL * 8);
+    transpose_b32_kernel<<<grid, 256, 0, s>>>(static_cast<const uint32_t *>(src), static_cast<uint32_t *>(dst), B, R, S);
+}
+
 void launch_transpose_b16(const void *src, void *dst, int B, int R, int S, cudaStream_t s) {
     const long long tiles = static_cast<long long>(B) * ((R + 63) / 64) * ((S + 63) / 64);
     const int grid = static_cast<int>(tiles < 148LL * 8 ? tiles : 148LL * 8);
@@ -354,6 +404,8 @@ cudaError_t launch_nchw_to_nhwc(const void *src, void *dst, int N, int C, int H,
     const long long pixels = static_cast<long long>(N) * HW;
     if (elt == 2 && Cpg == C / groups && C % 8 == 0 && HW % 8 == 0 && C * elt > 64) {
         launch_transpose_b16(src, dst, N, C, HW, s);  // no channel padding: a plain transpose
+    } else if (elt == 4 && Cpg == C / groups && C % 4 == 0 && HW % 4 == 0 && C * elt > 64) {
+        launch_transpose_b32(src, dst, N, C, HW, s);
     } else if (Ctot * elt <= 64 && (Ctot * elt) % 16 == 0) {
         if (elt == 2)
             nchw_to_nhwc_small<2><<<grid_for(pixels), kThreads, 0, s>>>(src, dst, N, C, HW, groups, Cpg);
@@ -386,6 +438,10 @@ cudaError_t launch_nhwc_to_nchw(const void *src, void *dst, int N, int C, int H,
     const int HW = H * W;
     if (elt == 2 && C % 8 == 0 && HW % 8 == 0) {
         launch_transpose_b16(src, dst, N, HW, C, s);
+        return cudaGetLastError();
+    }
+    if (elt == 4 && C % 4 == 0 && HW % 4 == 0) {
+        launch_transpose_b32(src, dst, N, HW, C, s);
         return cudaGetLastError();
     }
     const long long tiles = static_cast<long long>(N) * ((C + 31) / 32) * ((HW + 31) / 32);

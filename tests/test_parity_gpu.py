@@ -226,18 +226,21 @@ def test_watchdog_returns_timeout_instead_of_hanging():
     parity.assert_close(cfg, parity.run_gpu(cfg, inp, layer=layer), parity.run_oracle(cfg, inp), "after timeout")
 
 
-@pytest.mark.parametrize("shape", [(2, 64, 8, 8), (1, 72, 17, 8), (3, 200, 5, 24), (1, 256, 56, 56)],
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("shape", [(2, 64, 8, 8), (1, 72, 17, 8), (3, 200, 5, 24), (1, 256, 56, 56), (1, 36, 3, 4)],
                          ids=lambda s: "x".join(map(str, s)))
-def test_bf16_vector_transpose_both_ways(shape):
-    """bf16 without channel padding, C and H*W multiples of 8: the 64x64-tile vector
-    transpose, full and partial tiles, against torch's permute (a pure data movement)."""
+def test_vector_transpose_both_ways(shape, dtype):
+    """No channel padding, C and H*W multiples of the 16-byte vector (8 bf16 / 4 fp32):
+    the vector tile transposes, full and partial tiles, against torch's permute (a pure
+    data movement, so the results must be identical)."""
     import torch
     N, C, H, W = shape
-    x = (torch.randn(N, C, H, W) * 3).to(torch.bfloat16).cuda()
-    nhwc = torch.full((N, H, W, C), 7.0, dtype=torch.bfloat16, device="cuda")
-    cb.conv2d_nchw_to_nhwc(x, nhwc, N, C, H, W, 1, C, cb.CONV_BF16)
+    tdt, code = (torch.bfloat16, cb.CONV_BF16) if dtype == "bf16" else (torch.float32, cb.CONV_F32)
+    x = (torch.randn(N, C, H, W) * 3).to(tdt).cuda()
+    nhwc = torch.full((N, H, W, C), 7.0, dtype=tdt, device="cuda")
+    cb.conv2d_nchw_to_nhwc(x, nhwc, N, C, H, W, 1, C, code)
     back = torch.full_like(x, 7.0)
-    cb.conv2d_nhwc_to_nchw(nhwc, back, N, C, H, W, cb.CONV_BF16)
+    cb.conv2d_nhwc_to_nchw(nhwc, back, N, C, H, W, code)
     cb.conv2d_sync_status()
     assert torch.equal(nhwc, x.permute(0, 2, 3, 1))
     assert torch.equal(back, x)
