@@ -123,3 +123,13 @@ def test_pair_watchdog_returns_timeout_instead_of_hanging(pairs_forced):
         cb.conv2d_debug_set_watchdog(0, False)
     cb.conv2d_sync_status()
     parity.assert_close(cfg, parity.run_gpu(cfg, inp, layer=layer), parity.run_oracle(cfg, inp), "after timeout")
+
+
+@pytest.mark.parametrize("name", ["resnet3x3_bf16_nhwc", "k7_17x17_bf16"])
+def test_pair_explicit_im2col_gemm(name, pairs_forced):
+    """The pages' formulation (X_col in memory, then the GEMM) with the GEMM on CTA
+    pairs reading X_col through tiled loads."""
+    cfg = parity.config(name, **SMALL[name])
+    inp = workloads.make_inputs(cfg)
+    got = parity.run_gpu(cfg, inp, explicit_im2col=True)
+    parity.assert_close(cfg, got, parity.run_oracle(cfg, inp), name + " (pair, explicit im2col)")
