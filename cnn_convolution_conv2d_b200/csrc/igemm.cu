@@ -3,24 +3,35 @@
 //
 // The product is the one of the im2col/GEMM tutorial (zskr.cn/news/1820658) §2.3,
 // Y = W_row @ X_col, computed transposed: rows are output pixels
-// m = (n*Ho + oh)*Wo + ow (tcgen05 M = 128 per tile), columns are the output channels
+// m = (n*Ho + oh)*Wo + ow (tcgen05 M = 128 per CTA), columns are the output channels
 // of one group (tcgen05 N = BN), and the reduction runs over the filter taps
 // (kh, kw) and the input channels of the group -- the "expand per tile, multiply,
 // discard" scheme the "手撕 Conv2D" page (lpnh.cn/news/2493075) §4.1 mentions, with
-// the expansion done by the tensor memory accelerator's im2col mode.
+// the expansion done by the tensor memory accelerator's im2col mode (or, for a 1x1
+// filter at stride 1 without padding, by tiled loads of x, which is then X_col).
 //
-// One persistent CTA per SM, warp-specialised:
+// Persistent and warp-specialised, one CTA per SM:
 //   warp 0      : TMA producer -- per stage, one im2col load of 128 output pixels x
 //                 CB bytes of channels per plane (filter-tap offsets kw*d, kh*d; reads
 //                 outside the image return zero, which is the zero padding) and one
-//                 tiled load of BN weight rows x CB bytes per plane;
+//                 tiled load of the weight rows x CB bytes per plane;
 //   warp 1      : allocates tensor memory and issues tcgen05.mma from one thread,
 //                 releasing each stage with tcgen05.commit;
-//   warps 2..5  : epilogue -- tcgen05.ld of the fp32 accumulator, + bias, round, store;
-//   warps 6..9  : (fp32 only) split every staged fp32 value v into tf32 parts
-//                 hi = tf32(v), lo = tf32(v - hi) for the three-product scheme.
+//   warps 2..9  : (bf16) epilogue -- tcgen05.ld of the fp32 accumulator, + bias, round,
+//                 store (channels-last through shared memory and TMA stores), two
+//                 warps per tensor-memory lane quarter, each draining half the columns;
+//   warps 2..5  : (fp32) epilogue, with warps 6..9 splitting every staged fp32 value v
+//                 into tf32 parts hi = tf32(v), lo = tf32(v - hi) for three products.
 // Two accumulators in tensor memory let the epilogue of one tile overlap the
 // main loop of the next.  Every wait is bounded (see ptx.cuh).
+//
+// CTA pairs (kPair, bf16): the grid is launched in clusters of two CTAs on an SM pair.
+// A unit of work is 256 output pixels; each CTA stages its own 128 rows of A and half
+// of the BN weight rows, all loads count on the even CTA's full barrier, the even CTA
+// issues M = 256 tcgen05.mma.cta_group::2 that read both CTAs' shared memory and write
+// each CTA's 128 accumulator rows into its own tensor memory, and its commits release
+// both CTAs' ring slots and accumulators by multicast arrive.  Both CTAs' epilogue
+// warps hand the accumulator back on the even CTA's barrier.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
