@@ -244,3 +244,30 @@ def test_vector_transpose_both_ways(shape, dtype):
     cb.conv2d_sync_status()
     assert torch.equal(nhwc, x.permute(0, 2, 3, 1))
     assert torch.equal(back, x)
+
+
+def test_forward_rejects_misaligned_pointers_and_small_workspace_without_writing():
+    """Host-side checks that need a device (they follow the device query): a pointer off
+    a 16-byte boundary is UNSUPPORTED, a workspace below conv2d_workspace_size is
+    WORKSPACE, and y is left untouched in both cases."""
+    import torch
+    cfg = parity.config("resnet3x3_bf16_nhwc", N=1, H=8, W=8, layout="nchw")  # NCHW: needs a workspace
+    inp = workloads.make_inputs(cfg)
+    layer = parity.make_layer(cfg, inp)
+    x = parity.to_device_x(cfg, inp["x"])
+    shape = (cfg.N, layer.C_in, cfg.H, cfg.W, layer.C_out, layer.Kh, layer.Kw, layer.stride, layer.pad,
+             layer.dilation, layer.groups)
+    need = cb.conv2d_workspace_size(*shape, layer.dtype, layer.layout)
+    assert need > 0
+    ws = torch.empty(need + 64, dtype=torch.uint8, device="cuda")
+    y = torch.full(layer.out_shape(cfg.N, cfg.H, cfg.W), 3.0, dtype=torch.bfloat16, device="cuda")
+    lib = cb.load()
+    args = [*shape, layer.dtype, layer.layout]
+    odd_x = x.data_ptr() + 2  # still inside x's allocation, 2 bytes off a 16-byte boundary
+    st = lib.conv2d_forward(odd_x, layer.w_packed.data_ptr(), None, y.data_ptr(), *args, ws.data_ptr(), need, None)
+    assert st == cb.CONV_ERR_UNSUPPORTED and "aligned" in cb.conv2d_last_error()
+    st = lib.conv2d_forward(x.data_ptr(), layer.w_packed.data_ptr(), None, y.data_ptr(), *args, ws.data_ptr(),
+                            need - 16, None)
+    assert st == cb.CONV_ERR_WORKSPACE
+    cb.conv2d_sync_status()
+    assert bool((y == 3.0).all())
