@@ -51,6 +51,7 @@ SIGNATURES = {
     "conv2d_kernel_launch_count": ([ctypes.POINTER(ctypes.c_ulonglong)], _I),
     "conv2d_debug_set_watchdog": ([_L, _I], _I),
     "conv2d_debug_set_pair_mode": ([_I], _I),
+    "conv2d_describe_plan": ([_I] * 11 + [_I, _I, _I, _I, ctypes.c_char_p, ctypes.c_size_t], _I),
 }
 
 _lib = None
@@ -245,6 +246,17 @@ def conv2d_kernel_launch_count() -> int:
 
 def conv2d_debug_set_watchdog(timeout_ns: int = 0, starve_loads: bool = False):
     _check(load().conv2d_debug_set_watchdog(int(timeout_ns), 1 if starve_loads else 0))
+
+
+def conv2d_describe_plan(N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype, layout,
+                         explicit_im2col=False, sms=-1) -> dict:
+    """The library's plan for a problem (kernel, tile shape, passes) as a dict."""
+    import json
+    buf = ctypes.create_string_buffer(512)
+    _check(load().conv2d_describe_plan(N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype,
+                                       _layout_code(layout), 1 if explicit_im2col else 0, int(sms), buf,
+                                       ctypes.sizeof(buf)))
+    return json.loads(buf.value.decode())
 
 
 def conv2d_debug_set_pair_mode(mode: int = 0):

@@ -668,6 +668,43 @@ int forward_impl(bool explicit_im2col, const void *x, const void *w_packed, cons
     return ok();
 }
 
+// The plan as a JSON object, for callers and tests that want to know which kernel,
+// tile shape and passes a problem gets.  sms < 0: this process's current device (none:
+// no device-dependent choices); sms >= 0: as if the device had that many SMs.
+int describe_impl(bool explicit_im2col, int N, int C_in, int H, int W, int C_out, int Kh, int Kw,
+                  int stride, int pad, int dilation, int groups, conv_dtype_t dtype,
+                  conv_layout_t layout, int sms, char *buf, size_t buflen) {
+    if (!buf || buflen == 0) return fail(CONV_ERR_INVALID_ARG, "buf must not be NULL");
+    Plan p;
+    int st = make_plan(N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype, layout,
+                       explicit_im2col, 0, &p);
+    if (st != CONV_OK) return st;
+    if (sms < 0) {
+        DeviceInfo *dev = nullptr;
+        int ndev = 0;
+        sms = 0;
+        if (cudaGetDeviceCount(&ndev) == cudaSuccess && ndev > 0 && device_info(&dev) == CONV_OK)
+            sms = dev->sms;
+        else
+            cudaGetLastError();
+    }
+    st = make_plan(N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype, layout,
+                   explicit_im2col, sms, &p);
+    if (st != CONV_OK) return st;
+    const char *a_load = p.gather ? "gather" : explicit_im2col ? "xcol" : p.direct_a ? "tiled_x" : "im2col";
+    const int n = std::snprintf(
+        buf, buflen,
+        "{\"kernel\": \"%s\", \"pair\": %d, \"a_load\": \"%s\", \"BN\": %d, \"cb\": %d, "
+        "\"stages\": %d, \"splits\": %d, \"units\": %d, \"xcopy\": %d, \"halo\": %d, "
+        "\"tma_out\": %d, \"Kpad\": %d, \"smem\": %zu, \"workspace\": %zu, \"sms\": %d}",
+        p.gather ? "gather" : "igemm", p.pair ? 1 : 0, a_load, p.BN, p.gather ? 0 : p.cb,
+        p.stages, p.gather ? 1 : p.splits, p.gather ? p.n_mtiles : p.units, p.xcopy ? 1 : 0,
+        p.halo ? 1 : 0, p.tma_out ? 1 : 0, p.gather ? p.Kpad : 0, p.smem, p.ws_total, sms);
+    if (n < 0 || static_cast<size_t>(n) >= buflen)
+        return fail(CONV_ERR_INVALID_ARG, "buf of %zu bytes is too small (%d needed)", buflen, n + 1);
+    return ok();
+}
+
 int workspace_impl(bool explicit_im2col, int N, int C_in, int H, int W, int C_out, int Kh, int Kw,
                    int stride, int pad, int dilation, int groups, conv_dtype_t dtype,
                    conv_layout_t layout, size_t *bytes) {
@@ -906,6 +943,13 @@ int conv2d_debug_set_watchdog(long long timeout_ns, int starve_loads) {
     g_timeout_ns = timeout_ns > 0 ? timeout_ns : kDefaultTimeoutNs;
     g_starve = starve_loads ? 1 : 0;
     return ok();
+}
+
+int conv2d_describe_plan(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stride,
+                         int pad, int dilation, int groups, conv_dtype_t dtype, conv_layout_t layout,
+                         int explicit_im2col, int sms, char *buf, size_t buflen) {
+    return describe_impl(explicit_im2col != 0, N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation,
+                         groups, dtype, layout, sms, buf, buflen);
 }
 
 int conv2d_debug_set_pair_mode(int mode) {

@@ -235,6 +235,26 @@ int conv2d_debug_set_watchdog(long long timeout_ns, int starve_loads);
  * Returns CONV_ERR_INVALID_ARG for any other mode. */
 int conv2d_debug_set_pair_mode(int mode);
 
+/* The plan the library makes for a problem, written into buf (buflen bytes, owned by
+ * the caller) as one JSON object: "kernel" ("igemm" = the implicit-GEMM tensor-core
+ * kernel, "gather" = the few-channel kernel), "pair" (1: CTA-pair launch), "a_load"
+ * (how the im2col operand is read: "im2col" = TMA im2col mode, "tiled_x" = x itself
+ * through tiled loads, "xcol" = the explicit X_col, "gather" = software gather), "BN"
+ * (output channels per tile), "cb" (bytes of channels per plane), "stages", "splits",
+ * "units", "xcopy" (1: a channels-last copy of x comes first), "halo", "tma_out",
+ * "Kpad", "smem" (bytes of shared memory per CTA), "workspace" (bytes) and "sms".
+ * The tile and launch choices follow the same rules the forward pass applies (zskr
+ * §4.3 implicit GEMM; output size per pwwt §4.2).  sms < 0 plans for this process's
+ * current CUDA device (with no device: as if it had none, so without reduction splits
+ * or CTA pairs); sms >= 0 plans as if the device had that many SMs.  The forward pass
+ * may still fall back from CTA pairs if the device cannot co-schedule them.
+ * explicit_im2col != 0 describes conv2d_forward_im2col_gemm.  Returns
+ * CONV_ERR_INVALID_ARG for invalid shapes (as conv2d_forward) or a NULL / too small
+ * buffer, CONV_ERR_UNSUPPORTED for unsupported problems; nothing runs on a GPU. */
+int conv2d_describe_plan(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stride,
+                         int pad, int dilation, int groups, conv_dtype_t dtype, conv_layout_t layout,
+                         int explicit_im2col, int sms, char *buf, size_t buflen);
+
 #ifdef __cplusplus
 }
 #endif

@@ -151,3 +151,56 @@ def test_pair_mode_leaves_workspace_of_split_free_problems_unchanged(lib):
             assert cb.conv2d_workspace_size(*shape, cb.CONV_BF16, "nhwc") == 0
     finally:
         cb.conv2d_debug_set_pair_mode(0)
+
+
+def _plan(shape, dtype=cb.CONV_BF16, layout="nhwc", **kw):
+    return cb.conv2d_describe_plan(*shape, dtype, layout, **kw)
+
+
+def test_plan_for_the_workloads_on_a_148_sm_device(lib):
+    """The kernel and tile choices the forward pass makes, pinned on the CPU."""
+    p1 = _plan((64, 256, 56, 56, 1024, 1, 1, 1, 0, 1, 1), sms=148)   # 1x1: x is X_col
+    assert (p1["kernel"], p1["pair"], p1["a_load"], p1["BN"], p1["stages"], p1["tma_out"]) == \
+        ("igemm", 1, "tiled_x", 256, 6, 1)
+    assert p1["units"] == (64 * 56 * 56 // 256) * 4 and p1["workspace"] == 0
+    p3 = _plan((64, 256, 56, 56, 256, 3, 3, 1, 1, 1, 1), sms=148)    # 3x3: hardware im2col, pairs
+    assert (p3["kernel"], p3["pair"], p3["a_load"], p3["BN"], p3["units"]) == ("igemm", 1, "im2col", 256, 784)
+    stem = _plan((32, 3, 224, 224, 64, 7, 7, 2, 3, 1, 1), layout="nchw", sms=148)
+    assert (stem["kernel"], stem["halo"], stem["tma_out"], stem["BN"], stem["workspace"]) == ("gather", 1, 1, 64, 0)
+    assert stem["Kpad"] == 176                                         # 3 channels x 7 rows x 8 (7 taps + 1) -> 168 -> 176
+    k7 = _plan((16, 512, 17, 17, 512, 7, 7, 1, 3, 1, 1), sms=148)     # 19 pair units < 74: single CTAs, split
+    assert (k7["pair"], k7["splits"], k7["units"]) == (0, 2, 37 * 2 * 2)
+    assert k7["workspace"] == 2 * 16 * 17 * 17 * 512 * 4               # fp32 partial sums per split
+    g = _plan((16, 512, 28, 28, 512, 3, 3, 2, 2, 2, 32), sms=148)     # 16 channels per group
+    assert (g["pair"], g["BN"], g["cb"]) == (0, 16, 32)
+    ex = _plan((64, 256, 56, 56, 256, 3, 3, 1, 1, 1, 1), explicit_im2col=True, sms=148)
+    assert ex["a_load"] == "xcol" and ex["workspace"] >= 924_844_032   # the 924.8 MB X_col
+    f32 = _plan((16, 512, 17, 17, 512, 7, 7, 1, 3, 1, 1), dtype=cb.CONV_F32, sms=148)
+    assert f32["pair"] == 0 and f32["BN"] == 128                        # CTA pairs are bf16 only
+
+
+def test_plan_without_a_device_count_makes_no_device_choices(lib):
+    p = _plan((64, 256, 56, 56, 256, 3, 3, 1, 1, 1, 1), sms=0)
+    assert p["pair"] == 0 and p["splits"] == 1 and p["units"] == 1568 and p["sms"] == 0
+
+
+def test_pair_mode_hook_changes_the_plan(lib):
+    small = (2, 64, 20, 20, 64, 3, 3, 1, 1, 1, 1)
+    try:
+        assert _plan(small, sms=148)["pair"] == 0        # 4 units of 256 rows: not enough work
+        cb.conv2d_debug_set_pair_mode(1)
+        assert _plan(small, sms=148)["pair"] == 1
+        assert _plan((2, 64, 20, 20, 48, 3, 3, 1, 1, 1, 1), sms=148)["pair"] == 0  # BN = 48: no even split
+        cb.conv2d_debug_set_pair_mode(2)
+        assert _plan((64, 256, 56, 56, 256, 3, 3, 1, 1, 1, 1), sms=148)["pair"] == 0
+    finally:
+        cb.conv2d_debug_set_pair_mode(0)
+
+
+def test_describe_plan_rejects_bad_arguments(lib):
+    with pytest.raises(cb.Conv2dError) as err:
+        _plan((1, 8, 4, 4, 8, 7, 7, 1, 0, 1, 1))          # empty output
+    assert err.value.status == cb.CONV_ERR_INVALID_ARG
+    buf = ctypes.create_string_buffer(8)
+    st = lib.conv2d_describe_plan(1, 8, 4, 4, 8, 3, 3, 1, 1, 1, 1, cb.CONV_BF16, cb.CONV_NHWC, 0, 0, buf, 8)
+    assert st == cb.CONV_ERR_INVALID_ARG                   # buffer too small
