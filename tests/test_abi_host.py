@@ -204,3 +204,15 @@ def test_describe_plan_rejects_bad_arguments(lib):
     buf = ctypes.create_string_buffer(8)
     st = lib.conv2d_describe_plan(1, 8, 4, 4, 8, 3, 3, 1, 1, 1, 1, cb.CONV_BF16, cb.CONV_NHWC, 0, 0, buf, 8)
     assert st == cb.CONV_ERR_INVALID_ARG                   # buffer too small
+
+
+def test_bench_mirror_of_the_gather_choice_agrees_with_the_library(lib):
+    """bench.py labels the kernel and counts its bytes with a Python copy of the
+    library's few-channel rule; keep the two in step for every workload."""
+    import bench
+    from cnn_convolution_conv2d_b200 import workloads
+    for name, c in workloads.CONFIGS.items():
+        plan = cb.conv2d_describe_plan(c.N, c.C_in, c.H, c.W, c.C_out, c.Kh, c.Kw, c.stride, c.pad, c.dilation,
+                                       c.groups, cb.CONV_BF16 if c.dtype == "bf16" else cb.CONV_F32, c.layout,
+                                       sms=148)
+        assert (plan["kernel"] == "gather") == bench.uses_gather(c), name
