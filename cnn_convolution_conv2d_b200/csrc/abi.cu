@@ -55,10 +55,27 @@ struct DeviceInfo {
 };
 DeviceInfo g_devices[kMaxDevices];
 std::mutex g_mutex;
-long long g_timeout_ns = kDefaultTimeoutNs;
-int g_starve = 0;
-int g_pair_mode = 0;  // CTA pairs: 0 when they pay, 1 whenever eligible, 2 never
+// Test-hook settings: written by the conv2d_debug_* setters, read once per call
+// (see Settings) so that one call never mixes two settings.
+std::atomic<long long> g_timeout_ns{kDefaultTimeoutNs};
+std::atomic<int> g_starve{0};
+std::atomic<int> g_pair_mode{0};  // CTA pairs: 0 when they pay, 1 whenever eligible, 2 never
 std::map<long long, int> g_pair_clusters;  // see pair_cluster_limit
+
+// The test-hook settings as one call sees them.
+struct Settings {
+    long long timeout_ns;
+    int starve;
+    int pair_mode;
+};
+
+Settings settings_now() {
+    Settings s;
+    s.timeout_ns = g_timeout_ns.load(std::memory_order_relaxed);
+    s.starve = g_starve.load(std::memory_order_relaxed);
+    s.pair_mode = g_pair_mode.load(std::memory_order_relaxed);
+    return s;
+}
 cudaEvent_t g_main_start = nullptr, g_main_stop = nullptr;
 std::atomic<unsigned long long> g_launches{0};
 
@@ -141,6 +158,7 @@ struct Plan {
     int n_mtiles, n_ntiles, splits, units, stages;
     size_t smem;
     size_t off_xcopy, off_partial, off_xcol, ws_total;
+    int pair_clusters;  // resident two-CTA clusters of the pair kernel (pair plans only)
 };
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -189,7 +207,7 @@ GatherImages gather_images(int C_out, int C_in, int Kh, int Kw, int groups, int 
 // made before a device is known use the device's count when one is current).
 int make_plan(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stride, int pad,
               int dilation, int groups, conv_dtype_t dtype, conv_layout_t layout,
-              bool explicit_im2col, int sms, Plan *P, bool allow_pair = true) {
+              bool explicit_im2col, int sms, Plan *P, int pair_mode, bool allow_pair = true) {
     if (N < 1 || C_in < 1 || H < 1 || W < 1 || C_out < 1 || Kh < 1 || Kw < 1)
         return fail(CONV_ERR_INVALID_ARG, "sizes must be >= 1 (N=%d C_in=%d H=%d W=%d C_out=%d Kh=%d Kw=%d)",
                     N, C_in, H, W, C_out, Kh, Kw);
@@ -333,8 +351,8 @@ int make_plan(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stri
     // shared-memory bandwidth spent on it.  Used when the 256-row units still give
     // every SM pair work; the test hook can force or forbid them.
     const long long pair_units = ((p.M + 255) / 256) * p.n_ntiles * groups;
-    const bool pair_ok = allow_pair && !p.f32 && p.BN % 32 == 0 && g_pair_mode != 2;
-    if (pair_ok && ((p.splits == 1 && sms > 0 && pair_units >= sms / 2) || g_pair_mode == 1)) {
+    const bool pair_ok = allow_pair && !p.f32 && p.BN % 32 == 0 && pair_mode != 2;
+    if (pair_ok && ((p.splits == 1 && sms > 0 && pair_units >= sms / 2) || pair_mode == 1)) {
         p.pair = true;
         p.splits = 1;
         p.n_mtiles = static_cast<int>((p.M + 255) / 256);
@@ -447,7 +465,7 @@ int record_event(cudaEvent_t ev, cudaStream_t stream) {
 
 // The software-gather path (few input channels): one kernel, no scratch.
 int gather_impl(const Plan &p, const void *x, const void *w_packed, const void *bias, void *y,
-                DeviceInfo *dev, cudaStream_t stream) {
+                DeviceInfo *dev, const Settings &cfg, cudaStream_t stream) {
     GatherParams g;
     std::memset(&g, 0, sizeof(g));
     g.x = x;
@@ -505,8 +523,8 @@ int gather_impl(const Plan &p, const void *x, const void *w_packed, const void *
     g.out_mode = p.layout == CONV_NCHW ? kOutNCHW : kOutNHWC;
     g.vec_ok = (p.C_out % (16 / p.elt) == 0) ? 1 : 0;
     g.status = dev->status;
-    g.timeout_ns = g_timeout_ns;
-    g.starve = g_starve;
+    g.timeout_ns = cfg.timeout_ns;
+    g.starve = cfg.starve;
     const int grid = p.n_mtiles < dev->sms ? p.n_mtiles : dev->sms;
     int st;
     cudaEvent_t ev_start = g_main_start, ev_stop = g_main_stop;
@@ -539,32 +557,54 @@ int pair_cluster_limit(int cb, bool im2col, size_t smem) {
     return n;
 }
 
+// The plan a forward call on the current device makes, including the fall-back
+// from CTA pairs to single CTAs when the device cannot co-schedule the pair kernel.
+// Size queries and the forward pass share it, so that they always agree.
+int device_plan(bool explicit_im2col, int N, int C_in, int H, int W, int C_out, int Kh, int Kw,
+                int stride, int pad, int dilation, int groups, conv_dtype_t dtype,
+                conv_layout_t layout, DeviceInfo *dev, const Settings &cfg, Plan *p) {
+    int st = make_plan(N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype, layout,
+                       explicit_im2col, dev ? dev->sms : 0, p, cfg.pair_mode);
+    if (st != CONV_OK) return st;
+    p->pair_clusters = 0;
+    if (p->pair && dev) {
+        const bool a_im2col = !(explicit_im2col || p->direct_a);
+        p->pair_clusters = pair_cluster_limit(p->cb, a_im2col, p->smem);
+        if (p->pair_clusters < 1)  // the device cannot co-schedule the pair kernel: single CTAs
+            return make_plan(N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype, layout,
+                             explicit_im2col, dev->sms, p, cfg.pair_mode, false);
+    }
+    return CONV_OK;
+}
+
+// The current device, or NULL (and no error) when this process has none.
+DeviceInfo *current_device_or_null() {
+    DeviceInfo *dev = nullptr;
+    int ndev = 0;
+    if (cudaGetDeviceCount(&ndev) == cudaSuccess && ndev > 0 && device_info(&dev) == CONV_OK) return dev;
+    cudaGetLastError();
+    return nullptr;
+}
+
 // Shared body of conv2d_forward and conv2d_forward_im2col_gemm.
 int forward_impl(bool explicit_im2col, const void *x, const void *w_packed, const void *bias, void *y,
                  int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stride, int pad,
                  int dilation, int groups, conv_dtype_t dtype, conv_layout_t layout, void *workspace,
                  size_t workspace_bytes, cudaStream_t stream) {
+    const Settings cfg = settings_now();
     DeviceInfo *dev = nullptr;
     Plan p;
     int st = make_plan(N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype, layout,
-                       explicit_im2col, 0, &p);
+                       explicit_im2col, 0, &p, cfg.pair_mode);
     if (st != CONV_OK) return st;
     if (!x || !w_packed || !y) return fail(CONV_ERR_INVALID_ARG, "x, w_packed and y must not be NULL");
     st = device_info(&dev);
     if (st != CONV_OK) return st;
-    st = make_plan(N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype, layout,
-                   explicit_im2col, dev->sms, &p);
+    st = device_plan(explicit_im2col, N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype,
+                     layout, dev, cfg, &p);
     if (st != CONV_OK) return st;
     const bool a_im2col = !(explicit_im2col || p.direct_a);
-    int pair_clusters = 0;
-    if (p.pair) {
-        pair_clusters = pair_cluster_limit(p.cb, a_im2col, p.smem);
-        if (pair_clusters < 1) {  // the device cannot co-schedule the pair kernel: single CTAs
-            st = make_plan(N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype, layout,
-                           explicit_im2col, dev->sms, &p, false);
-            if (st != CONV_OK) return st;
-        }
-    }
+    const int pair_clusters = p.pair_clusters;
     if (p.ws_total > 0 && (!workspace || workspace_bytes < p.ws_total))
         return fail(CONV_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", p.ws_total,
                     workspace ? workspace_bytes : static_cast<size_t>(0));
@@ -572,7 +612,7 @@ int forward_impl(bool explicit_im2col, const void *x, const void *w_packed, cons
         (workspace && !aligned16(workspace)))
         return fail(CONV_ERR_UNSUPPORTED, "device pointers must be 16-byte aligned");
 
-    if (p.gather) return gather_impl(p, x, w_packed, bias, y, dev, stream);
+    if (p.gather) return gather_impl(p, x, w_packed, bias, y, dev, cfg, stream);
 
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     const void *x_nhwc = p.xcopy ? static_cast<const void *>(ws + p.off_xcopy) : x;
@@ -625,8 +665,8 @@ int forward_impl(bool explicit_im2col, const void *x, const void *w_packed, cons
         kp.vec_ok = (C_out % per16 == 0 && p.Cout_g % per16 == 0) ? 1 : 0;
     }
     kp.status = dev->status;
-    kp.timeout_ns = g_timeout_ns;
-    kp.starve = g_starve;
+    kp.timeout_ns = cfg.timeout_ns;
+    kp.starve = cfg.starve;
     kp.tma_out = (p.tma_out && p.splits == 1) ? 1 : 0;
     if (kp.tma_out) {
         cuuint64_t dims[2] = {static_cast<cuuint64_t>(C_out), static_cast<cuuint64_t>(p.M)};
@@ -675,21 +715,20 @@ int describe_impl(bool explicit_im2col, int N, int C_in, int H, int W, int C_out
                   int stride, int pad, int dilation, int groups, conv_dtype_t dtype,
                   conv_layout_t layout, int sms, char *buf, size_t buflen) {
     if (!buf || buflen == 0) return fail(CONV_ERR_INVALID_ARG, "buf must not be NULL");
+    const Settings cfg = settings_now();
     Plan p;
     int st = make_plan(N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype, layout,
-                       explicit_im2col, 0, &p);
+                       explicit_im2col, 0, &p, cfg.pair_mode);
     if (st != CONV_OK) return st;
     if (sms < 0) {
-        DeviceInfo *dev = nullptr;
-        int ndev = 0;
-        sms = 0;
-        if (cudaGetDeviceCount(&ndev) == cudaSuccess && ndev > 0 && device_info(&dev) == CONV_OK)
-            sms = dev->sms;
-        else
-            cudaGetLastError();
+        DeviceInfo *dev = current_device_or_null();
+        sms = dev ? dev->sms : 0;
+        st = device_plan(explicit_im2col, N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups,
+                         dtype, layout, dev, cfg, &p);
+    } else {
+        st = make_plan(N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype, layout,
+                       explicit_im2col, sms, &p, cfg.pair_mode);
     }
-    st = make_plan(N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype, layout,
-                   explicit_im2col, sms, &p);
     if (st != CONV_OK) return st;
     const char *a_load = p.gather ? "gather" : explicit_im2col ? "xcol" : p.direct_a ? "tiled_x" : "im2col";
     const int n = std::snprintf(
@@ -709,19 +748,14 @@ int workspace_impl(bool explicit_im2col, int N, int C_in, int H, int W, int C_ou
                    int stride, int pad, int dilation, int groups, conv_dtype_t dtype,
                    conv_layout_t layout, size_t *bytes) {
     if (!bytes) return fail(CONV_ERR_INVALID_ARG, "bytes must not be NULL");
+    const Settings cfg = settings_now();
     Plan p;
     int st = make_plan(N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype, layout,
-                       explicit_im2col, 0, &p);
+                       explicit_im2col, 0, &p, cfg.pair_mode);
     if (st != CONV_OK) return st;
-    DeviceInfo *dev = nullptr;
-    int sms = 0;
-    int ndev = 0;
-    if (cudaGetDeviceCount(&ndev) == cudaSuccess && ndev > 0 && device_info(&dev) == CONV_OK)
-        sms = dev->sms;
-    else
-        cudaGetLastError();  // no usable device: size without a split
-    st = make_plan(N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype, layout,
-                   explicit_im2col, sms, &p);
+    // with no usable device: sized without reduction splits or CTA pairs
+    st = device_plan(explicit_im2col, N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype,
+                     layout, current_device_or_null(), cfg, &p);
     if (st != CONV_OK) return st;
     *bytes = p.ws_total;
     return ok();
@@ -844,10 +878,11 @@ int conv2d_forward_noalloc(const void *x, const void *w_packed, const void *bias
                     "this problem needs %zu bytes of scratch; the built-in scratch of "
                     "conv2d_forward_noalloc holds %zu (use conv2d_forward with a workspace)",
                     need, kNoAllocScratchBytes);
+    // The whole array goes to the forward pass, which checks its own plan against it.
     void *scratch = nullptr;
-    if (need > 0 && (st = noalloc_scratch(&scratch)) != CONV_OK) return st;
+    if ((st = noalloc_scratch(&scratch)) != CONV_OK) return st;
     return forward_impl(false, x, w_packed, bias, y, N, C_in, H, W, C_out, Kh, Kw, stride, pad,
-                        dilation, groups, dtype, layout, scratch, need > 0 ? kNoAllocScratchBytes : 0,
+                        dilation, groups, dtype, layout, scratch, kNoAllocScratchBytes,
                         reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -858,7 +893,7 @@ int conv2d_forward_hostio(const void *x_host, void *y_host, void *x_dev, void *y
                           size_t workspace_bytes, conv_stream_t stream) {
     Plan p;
     int st = make_plan(N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype, layout,
-                       false, 0, &p);
+                       false, 0, &p, 0);
     if (st != CONV_OK) return st;
     if (!x_host || !y_host || !x_dev || !y_dev)
         return fail(CONV_ERR_INVALID_ARG, "host and device activation buffers must not be NULL");
@@ -939,9 +974,8 @@ int conv2d_kernel_launch_count(unsigned long long *count) {
 }
 
 int conv2d_debug_set_watchdog(long long timeout_ns, int starve_loads) {
-    std::lock_guard<std::mutex> lock(g_mutex);
-    g_timeout_ns = timeout_ns > 0 ? timeout_ns : kDefaultTimeoutNs;
-    g_starve = starve_loads ? 1 : 0;
+    g_timeout_ns.store(timeout_ns > 0 ? timeout_ns : kDefaultTimeoutNs, std::memory_order_relaxed);
+    g_starve.store(starve_loads ? 1 : 0, std::memory_order_relaxed);
     return ok();
 }
 
@@ -954,8 +988,7 @@ int conv2d_describe_plan(int N, int C_in, int H, int W, int C_out, int Kh, int K
 
 int conv2d_debug_set_pair_mode(int mode) {
     if (mode < 0 || mode > 2) return fail(CONV_ERR_INVALID_ARG, "pair mode must be 0, 1 or 2");
-    std::lock_guard<std::mutex> lock(g_mutex);
-    g_pair_mode = mode;
+    g_pair_mode.store(mode, std::memory_order_relaxed);
     return ok();
 }
 

@@ -391,10 +391,23 @@ __global__ void __launch_bounds__(threads_for<kF32>(), 1)
                     }
                 }
                 if (*wd.abort && loads_issued > 0) {
-                    // A pair's loads complete on rank 0's barriers: give the copies
-                    // still in flight a fixed, generous time to land.
-                    const uint64_t t0 = globaltimer_ns();
-                    while (globaltimer_ns() - t0 < 200000u) {
+                    if (rank == 0) {
+                        // Both CTAs' loads of a stage complete on rank 0's full barrier:
+                        // wait (bounded) for every phase this CTA armed and has not seen
+                        // complete, so that no copy of either CTA is still writing into a
+                        // stage of an armed phase.  The odd CTA leaves only after the
+                        // final cluster barrier, i.e. after these waits.
+                        const long long first = loads_issued > p.stages ? loads_issued - p.stages : 0;
+                        for (long long i = first; i < loads_issued; ++i)
+                            wait_quiet(&sb.full[i % p.stages], static_cast<uint32_t>((i / p.stages) & 1),
+                                       wd.timeout_ns);
+                    } else {
+                        // The odd CTA cannot observe its own copies (they count on the even
+                        // CTA's barrier).  Copies it issued for a phase the even CTA never
+                        // armed get a fixed time to land: the one remaining bounded case.
+                        const uint64_t t0 = globaltimer_ns();
+                        while (globaltimer_ns() - t0 < 200000u) {
+                        }
                     }
                 }
             } else if (*wd.abort && loads_issued > 0) {

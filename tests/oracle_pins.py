@@ -160,6 +160,28 @@ def pin_worked_example(lib):
             assert yd[0, 0, 0, 0] == ex["window_c0"][a, bb], (a, bb, yd[0, 0, 0, 0])
 
 
+def read_hand_example():
+    """Rows of hand_example_5x5_pad1.txt: the 5x5 output worked by hand."""
+    rows = []
+    with open(os.path.join(GOLDEN, "hand_example_5x5_pad1.txt"), encoding="utf-8") as f:
+        for line in f:
+            parts = line.split()
+            if parts and parts[0] == "out":
+                rows.append([float(v) for v in parts[1:]])
+    return np.array(rows)
+
+
+def pin_hand_example_5x5(lib):
+    """lpnh §1.1's hand-drawn case: 5x5 arange input, 3x3 ones, stride 1, pad 1 -- the
+    25 window sums worked by hand (tests/golden/hand_example_5x5_pad1.txt)."""
+    want = read_hand_example()
+    assert want.shape == (5, 5)
+    x = np.arange(25, dtype=np.float64).reshape(1, 1, 5, 5)
+    y = oracle.conv2d(x, np.ones((1, 1, 3, 3)), None, 1, 1, 1, 1, lib=lib)
+    assert y.shape == (1, 1, 5, 5)
+    assert np.array_equal(y[0, 0], want), y[0, 0]
+
+
 def pin_box_sum(lib):
     """All-ones kernels equal integral-image box sums (incl. the 3-channel worked example)."""
     rng = np.random.default_rng(11)
@@ -335,6 +357,6 @@ def pin_points_match_full(lib):
     assert np.array_equal(pts, y[tuple(idx.T)])
 
 
-ALL_PINS = [pin_output_size, pin_worked_example, pin_box_sum, pin_brute_force, pin_torch_f64,
+ALL_PINS = [pin_output_size, pin_worked_example, pin_hand_example_5x5, pin_box_sum, pin_brute_force, pin_torch_f64,
             pin_pointwise_matmul, pin_delta_shift, pin_zero_weight, pin_linearity,
             pin_groups_split, pin_exact_integers, pin_single_pixel, pin_points_match_full]

@@ -79,21 +79,37 @@ def test_write_context_is_output_bytes_over_the_fill_rate():
     assert "write_context" not in bench.with_write_context(bench.roofline(r3, 0.2, PEAKS, "m", "x"), r3, 0.2, 1.0)
 
 
+def test_fp32_above_the_tf32_ridge_is_tensor_bound_against_half_the_bf16_peak():
+    k7 = cfg("k7_17x17_f32")                # 3379 FLOP/B, three TF32 products per multiply-add
+    rl = bench.roofline(k7, 1.0, PEAKS, "measured", "none")
+    assert rl["bound"] == "tensor" and rl["peak"] == pytest.approx(1371.8 * 0.5)
+    assert rl["algorithmic_tflops"] == pytest.approx(bench.flops(k7) / 1e-3 / 1e12)
+    assert rl["executed_tf32_tflops"] == pytest.approx(3 * rl["algorithmic_tflops"])
+    assert rl["frac"] == pytest.approx(rl["executed_tf32_tflops"] / (1371.8 * 0.5))
+    g = cfg("grouped_dilated_f32")          # 14 FLOP/B: memory-bound in any precision
+    assert bench.roofline(g, 0.03, PEAKS, "measured", "none")["bound"] == "hbm"
+
+
 def test_committed_traffic_is_void_when_the_kernel_source_changes(tmp_path, monkeypatch):
     prof = tmp_path / "profiles"
     prof.mkdir()
     good = bench.kernel_source_hash("igemm_kernel")
+    entry = {"kernel": "igemm_kernel", "dram_bytes_read": 100.0, "dram_bytes_write": 20.0, "l2_write_bytes": 50.0}
     (prof / "traffic.json").write_text(json.dumps({
-        "a": {"kernel": "igemm_kernel", "kernel_hash": good, "dram_bytes_per_launch": 123.0},
-        "b": {"kernel": "igemm_kernel", "kernel_hash": "0" * 16, "dram_bytes_per_launch": 456.0},
-        "c": {"kernel": "no_such_kernel", "kernel_hash": good, "dram_bytes_per_launch": 789.0},
+        "a": {**entry, "kernel_hash": good},
+        "b": {**entry, "kernel_hash": "0" * 16},
+        "c": {**entry, "kernel": "no_such_kernel", "kernel_hash": good},
+        "d": {"kernel": "igemm_kernel", "kernel_hash": good, "dram_bytes_read": 1.0, "dram_bytes_write": 2.0},
+        "e": {**entry, "kernel_hash": good, "dram_bytes_write": 80.0, "scale_to_full_launch": 2.0},
     }))
     csrc = os.path.join(ROOT, "cnn_convolution_conv2d_b200", "csrc")
     # read profiles from the temporary tree, kernel sources from the real one
     os.symlink(os.path.join(ROOT, "cnn_convolution_conv2d_b200"), tmp_path / "cnn_convolution_conv2d_b200")
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    assert bench.committed_traffic("a") == 123.0
+    assert bench.committed_traffic("a") == 150.0       # reads + the L2-side writes (above DRAM's count)
     assert bench.committed_traffic("b") is None
     assert bench.committed_traffic("c") is None
+    assert bench.committed_traffic("d") is None        # no L2-side write count: not reported
+    assert bench.committed_traffic("e") == 2.0 * 180.0  # DRAM writes above L2's, scaled to a full launch
     assert bench.committed_traffic("missing") is None
     assert os.path.isdir(csrc)
