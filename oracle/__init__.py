@@ -4,11 +4,14 @@ Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 ``bench.py`` may import this package.  The CUDA library and its Python binding
 never import it; the two share no code.
 
-The arithmetic lives in ``conv2d_oracle.c`` (fp64, six nested loops with
-bounds-checked zero padding, after the "手撕 Conv2D" page (lpnh.cn/news/2493075)
-§1.1-§2.1).  This module compiles that file with gcc (no -ffast-math, so IEEE
-double arithmetic is kept) and exposes it through ctypes.  Inputs are widened
-to float64 before the call; widening bf16- or fp32-valued data is exact.
+The arithmetic lives in C files compiled with gcc (no -ffast-math, so IEEE double
+arithmetic is kept) and exposed through ctypes:
+  * ``conv2d_oracle.c``: the forward pass, six nested loops with bounds-checked zero
+    padding, after the "手撕 Conv2D" page (lpnh.cn/news/2493075) §1.1-§2.1;
+  * ``conv2d_backward_oracle.c``: the gradients dx, dW, db, after the same page's
+    §5.1-§5.2 naive backward loops.
+Inputs are widened to float64 before the call; widening bf16- or fp32-valued data
+is exact.
 """
 from __future__ import annotations
 
@@ -21,8 +24,11 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 SOURCE = os.path.join(_HERE, "conv2d_oracle.c")
 LIBRARY = os.path.join(_HERE, "liboracle.so")
+BWD_SOURCE = os.path.join(_HERE, "conv2d_backward_oracle.c")
+BWD_LIBRARY = os.path.join(_HERE, "liboracle_backward.so")
 
 _lib = None
+_bwd = None
 
 
 def build(source: str = SOURCE, output: str = LIBRARY, extra_flags=()) -> str:
@@ -31,6 +37,12 @@ def build(source: str = SOURCE, output: str = LIBRARY, extra_flags=()) -> str:
            "-o", output, source]
     subprocess.run(cmd, check=True)
     return output
+
+
+def build_all() -> None:
+    """Compile every C oracle of this package."""
+    build(SOURCE, LIBRARY)
+    build(BWD_SOURCE, BWD_LIBRARY)
 
 
 def load(path: str | None = None):
@@ -116,3 +128,93 @@ def conv2d_points(x, w, bias, idx, stride=1, pad=0, dilation=1, groups=1, lib=No
 def num_threads(lib=None) -> int:
     """OpenMP threads the oracle's loops use."""
     return int((lib or load()).oracle_num_threads())
+
+
+# ---------------------------------------------------------------- backward ---
+def _bind_backward(lib):
+    L = ctypes.c_long
+    P = ctypes.c_void_p
+    lib.oracle_conv2d_backward.argtypes = [P] * 6 + [L] * 11
+    lib.oracle_conv2d_backward.restype = ctypes.c_int
+    lib.oracle_conv2d_backward_data_points.argtypes = [P, P] + [L] * 11 + [P, L, P]
+    lib.oracle_conv2d_backward_data_points.restype = ctypes.c_int
+    lib.oracle_conv2d_backward_weight_points.argtypes = [P, P] + [L] * 11 + [P, L, P]
+    lib.oracle_conv2d_backward_weight_points.restype = ctypes.c_int
+    lib.oracle_backward_num_threads.argtypes = []
+    lib.oracle_backward_num_threads.restype = ctypes.c_int
+    return lib
+
+
+def load_backward(path: str | None = None):
+    """Load (building first if needed) the backward oracle library."""
+    global _bwd
+    if path is not None:
+        return _bind_backward(ctypes.CDLL(path))
+    if _bwd is None:
+        if (not os.path.exists(BWD_LIBRARY)
+                or os.path.getmtime(BWD_LIBRARY) < os.path.getmtime(BWD_SOURCE)):
+            build(BWD_SOURCE, BWD_LIBRARY)
+        _bwd = _bind_backward(ctypes.CDLL(BWD_LIBRARY))
+    return _bwd
+
+
+def _bwd_shape(dy, x_shape, w):
+    N, C_in, H, W = x_shape
+    C_out, cin_g, Kh, Kw = w.shape
+    if dy.shape[0] != N or dy.shape[1] != C_out:
+        raise ValueError("dy does not match x and w")
+    groups = C_in // cin_g
+    if cin_g * groups != C_in:
+        raise ValueError("weight shape does not match C_in / groups")
+    return N, C_in, H, W, C_out, Kh, Kw, groups
+
+
+def conv2d_backward(dy, x, w, stride=1, pad=0, dilation=1, groups=1, lib=None):
+    """(dx, dW, db) in float64 for y = conv2d(x, w, b): dy (N, C_out, Ho, Wo) NCHW,
+    x NCHW, w OIHW (C_out, C_in/groups, Kh, Kw)."""
+    lib = lib or load_backward()
+    dy, x, w = _f64(dy), _f64(x), _f64(w)
+    N, C_in, H, W, C_out, Kh, Kw, g = _bwd_shape(dy, x.shape, w)
+    if g != groups:
+        raise ValueError("weight shape does not match C_in / groups")
+    Ho = out_size(H, Kh, stride, pad, dilation)
+    Wo = out_size(W, Kw, stride, pad, dilation)
+    if dy.shape != (N, C_out, Ho, Wo):
+        raise ValueError(f"dy must have shape {(N, C_out, Ho, Wo)}")
+    dx = np.empty_like(x)
+    dW = np.empty_like(w)
+    db = np.empty(C_out)
+    rc = lib.oracle_conv2d_backward(_ptr(dy), _ptr(x), _ptr(w), _ptr(dx), _ptr(dW), _ptr(db), N, C_in,
+                                    H, W, C_out, Kh, Kw, stride, pad, dilation, groups)
+    if rc != 0:
+        raise ValueError("oracle rejected the shape")
+    return dx, dW, db
+
+
+def conv2d_backward_data_points(dy, w, x_shape, idx, stride=1, pad=0, dilation=1, groups=1, lib=None):
+    """Selected dx[n, ic, ih, iw] for the rows (n, ic, ih, iw) of ``idx``."""
+    lib = lib or load_backward()
+    dy, w = _f64(dy), _f64(w)
+    N, C_in, H, W, C_out, Kh, Kw, _ = _bwd_shape(dy, x_shape, w)
+    idx = np.ascontiguousarray(idx, dtype=np.int64).reshape(-1, 4)
+    out = np.empty(idx.shape[0])
+    rc = lib.oracle_conv2d_backward_data_points(_ptr(dy), _ptr(w), N, C_in, H, W, C_out, Kh, Kw, stride,
+                                                pad, dilation, groups, _ptr(idx), idx.shape[0], _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle rejected the shape or an index")
+    return out
+
+
+def conv2d_backward_weight_points(dy, x, w_shape, idx, stride=1, pad=0, dilation=1, groups=1, lib=None):
+    """Selected dW[oc, c, kh, kw] for the rows (oc, c, kh, kw) of ``idx``."""
+    lib = lib or load_backward()
+    dy, x = _f64(dy), _f64(x)
+    N, C_in, H, W = x.shape
+    C_out, cin_g, Kh, Kw = w_shape
+    idx = np.ascontiguousarray(idx, dtype=np.int64).reshape(-1, 4)
+    out = np.empty(idx.shape[0])
+    rc = lib.oracle_conv2d_backward_weight_points(_ptr(dy), _ptr(x), N, C_in, H, W, C_out, Kh, Kw, stride,
+                                                  pad, dilation, groups, _ptr(idx), idx.shape[0], _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle rejected the shape or an index")
+    return out
