@@ -55,6 +55,7 @@ TF32_PRODUCTS = 3
 KERNEL_SOURCES = {
     "igemm_kernel": ["igemm.cu", "epilogue.cuh", "ptx.cuh", "common.cuh"],
     "gather_kernel": ["gather.cu", "epilogue.cuh", "ptx.cuh", "common.cuh"],
+    "dw_kernel": ["depthwise.cu", "ptx.cuh", "common.cuh"],
 }
 
 
@@ -94,11 +95,21 @@ def uses_gather(cfg) -> bool:
     return cfg.groups == 1 and cfg.C_in * e < 32 and kpad <= 256 and cfg.C_out <= (256 if e == 2 else 128)
 
 
+def uses_depthwise(cfg) -> bool:
+    """Mirrors the library's choice of the depthwise stencil kernel: groups = C_in = C_out."""
+    return cfg.groups == cfg.C_in == cfg.C_out
+
+
 def main_kernel_bytes(cfg) -> float:
     """Minimum bytes the tensor-core kernel itself moves per launch: its input (x
     itself for the gather kernel, else the channels-last input or its channel-padded
     copy when the step makes one), the packed weights, the bias, and the output."""
     e = elt_bytes(cfg)
+    if uses_depthwise(cfg):  # x (or its channel-padded channels-last copy), one weight per tap and channel
+        cp = -(-cfg.C_in // (16 // e)) * (16 // e)
+        c_in = cp if (cfg.layout == "nchw" or cp != cfg.C_in) else cfg.C_in
+        return e * (cfg.N * cfg.H * cfg.W * c_in + cfg.C_out * cfg.Kh * cfg.Kw + (cfg.C_out if cfg.bias else 0)
+                    + cfg.N * cfg.C_out * cfg.Ho * cfg.Wo)
     cpg = padded_channels(cfg)
     copy = (cfg.layout == "nchw" or cpg != cfg.C_in // cfg.groups) and not uses_gather(cfg)
     x_in = cfg.N * cfg.H * cfg.W * (cfg.groups * cpg if copy else cfg.C_in)
@@ -181,7 +192,9 @@ def roofline(cfg, kernel_ms: float, peaks, peak_kind: str, workload: str, explic
         out = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                "peak_source": f"{peak_kind} HBM copy bandwidth"}
     out["frac"] = achieved / peak
-    out["kernel"] = ("gather_kernel (software-gathered im2col rows, tcgen05)" if uses_gather(cfg)
+    out["kernel"] = ("dw_kernel (depthwise stencil over TMA-staged channels-last tiles, CUDA cores)"
+                     if uses_depthwise(cfg)
+                     else "gather_kernel (software-gathered im2col rows, tcgen05)" if uses_gather(cfg)
                      else "igemm_kernel (implicit GEMM: TMA im2col/tiled loads, tcgen05; "
                           "CTA pairs on large bf16 problems)")
     out["kernel_ms"] = kernel_ms

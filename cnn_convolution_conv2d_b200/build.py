@@ -20,7 +20,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIBRARY = os.path.join(PKG, "libconv2d_b200.so")
-SOURCES = ["abi.cu", "igemm.cu", "gather.cu", "layout.cu"]
+SOURCES = ["abi.cu", "igemm.cu", "gather.cu", "layout.cu", "depthwise.cu"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

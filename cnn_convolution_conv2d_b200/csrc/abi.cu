@@ -140,7 +140,8 @@ struct Plan {
     conv_layout_t layout;
     int Ho, Wo;
     long long M;
-    int Cin_g, Cout_g, Cpg;
+    int Cin_g, Cout_g, Cpg;  // per group the kernels see (merged groups: gm of the caller's)
+    int gm;                  // caller's groups merged into one (see group_merge)
     bool gather;    // few input channels: the software-gather kernel reads x directly
     bool vec_rows;  // ... with 16-byte row loads (NCHW, aligned rows, unit dilation)
     bool halo;      // ... from input rows staged in shared memory by TMA
@@ -159,6 +160,11 @@ struct Plan {
     size_t smem;
     size_t off_xcopy, off_partial, off_xcol, ws_total;
     int pair_clusters;  // resident two-CTA clusters of the pair kernel (pair plans only)
+    // depthwise kernel (groups = C_in = C_out)
+    bool dw;
+    int dw_window;      // 3, 5, 7: register-window form; 0: general form
+    int dw_Cp;          // channels per pixel of the staged tensor (multiple of 16 bytes)
+    int TH, TW, IH, IW, n_th, n_tw, dw_wregion, dw_ctas_per_sm;
 };
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -169,6 +175,23 @@ int out_size(int in, int k, int s, int p, int d, int *out) {
     if (numer < 0) return -1;
     *out = static_cast<int>(numer / s + 1);
     return 0;
+}
+
+// Narrow groups -- fewer than 64 output channels each, 16-byte rows of input channels --
+// are merged gm at a time into one wider group whose packed weights are block-diagonal
+// (zero where an output channel meets another group's input channels).  The product then
+// runs with N = gm * C_out/groups columns instead of a handful, which the tensor cores
+// execute at full rate; the zeros cost tensor-core cycles but no memory traffic beyond the
+// gm-times larger (still small) packed weights.  Depends only on the weight's shape, so
+// that conv2d_pack_weight and the forward pass agree.
+int group_merge(int C_out, int C_in, int groups, int elt) {
+    if (groups <= 1) return 1;
+    const int cin_g = C_in / groups, cout_g = C_out / groups;
+    if (cout_g >= 64 || (cin_g * elt) % 16 != 0) return 1;
+    int best = 1;
+    for (int gm = 2; gm <= groups; ++gm)
+        if (groups % gm == 0 && gm * cout_g <= 128 && gm * cin_g * elt <= 256) best = gm;
+    return best;
 }
 
 // The software-gather kernel reads its weights as ready-made shared-memory images
@@ -183,7 +206,8 @@ struct GatherImages {
 
 GatherImages gather_images(int C_out, int C_in, int Kh, int Kw, int groups, int elt) {
     GatherImages g;
-    const int cpg = round_up(C_in / groups, 16 / elt);
+    const int gm = group_merge(C_out, C_in, groups, elt);
+    const int cpg = round_up(C_in / groups, 16 / elt) * gm;
     size_t off = static_cast<size_t>(C_out) * Kh * Kw * cpg * elt;
     g.total = off;
     if (groups != 1 || C_in * elt >= 32 || C_out > (elt == 4 ? 128 : 256)) return g;
@@ -200,6 +224,58 @@ GatherImages gather_images(int C_out, int C_in, int Kh, int Kw, int groups, int 
     }
     g.total = off;
     return g;
+}
+
+// Depthwise problems (groups = C_in = C_out) go to the direct stencil kernel when its
+// staged input box fits: tiles of TH x 8 output pixels x 128 bytes of channels, one
+// persistent CTA per SM with as many stages as fit.  Returns false (and
+// the problem goes to the general kernels) when no tile shape fits.
+bool plan_depthwise(Plan *pp) {
+    Plan &p = *pp;
+    const int per16 = 16 / p.elt;
+    p.dw_Cp = round_up(p.C_in, per16);
+    p.dw_window = (p.stride == 1 && p.dilation == 1 && p.Kh == p.Kw &&
+                   (p.Kh == 3 || p.Kh == 5 || p.Kh == 7)) ? p.Kh : 0;
+    p.TW = 2 * dw_pixels_per_thread();
+    p.IW = (p.TW - 1) * p.stride + (p.Kw - 1) * p.dilation + 1;
+    if (p.IW > 256) return false;
+    const int taps = p.Kh * p.Kw;
+    const int cc = 128 / p.elt;
+    const size_t wbytes = static_cast<size_t>(taps) * 128 + cc * 4;
+    p.dw_wregion = static_cast<int>(align_up(wbytes * dw_compute_warps(), 1024));
+    const size_t fixed = dw_header_bytes() + p.dw_wregion;
+    // the tallest tile (at most 32 rows) whose staged box fits twice
+    size_t stage = 0;
+    for (p.TH = 32; p.TH >= 1; p.TH /= 2) {
+        p.IH = (p.TH - 1) * p.stride + (p.Kh - 1) * p.dilation + 1;
+        stage = static_cast<size_t>(p.IH) * p.IW * 128;
+        if (p.IH <= 256 && fixed + 2 * stage <= kSmemBudget) break;
+    }
+    if (p.TH < 1) return false;
+    p.dw_ctas_per_sm = 1;
+    int stages = static_cast<int>((kSmemBudget - fixed) / stage);
+    stages = stages > dw_max_stages() ? dw_max_stages() : stages;
+    p.stages = stages;
+    p.smem = fixed + static_cast<size_t>(stages) * stage;
+    p.n_th = (p.Ho + p.TH - 1) / p.TH;
+    p.n_tw = (p.Wo + p.TW - 1) / p.TW;
+    const long long units = static_cast<long long>((p.dw_Cp + cc - 1) / cc) * p.N * p.n_th * p.n_tw;
+    if (units >= (1LL << 31)) return false;
+    p.units = static_cast<int>(units);
+    p.dw = true;
+    p.gather = false;
+    p.pair = false;
+    p.direct_a = false;
+    p.tma_out = false;
+    p.splits = 1;
+    p.BN = 0;
+    p.cb = 128;
+    p.n_mtiles = p.units;
+    p.xcopy = p.layout == CONV_NCHW || p.dw_Cp != p.C_in;
+    p.off_xcopy = 0;
+    p.off_partial = p.off_xcol = 0;
+    p.ws_total = p.xcopy ? align_up(static_cast<size_t>(p.N) * p.H * p.W * p.dw_Cp * p.elt, 256) : 0;
+    return true;
 }
 
 // Validates a problem and fills the plan.  `explicit_im2col` adds the X_col
@@ -245,6 +321,19 @@ int make_plan(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stri
     p.Cout_g = C_out / groups;
     const int align = 16 / p.elt;
     p.Cpg = round_up(p.Cin_g, align);
+    p.dw = false;
+    if (!explicit_im2col && groups == C_in && C_out == C_in && plan_depthwise(&p)) {
+        *P = p;
+        return CONV_OK;
+    }
+    // From here on `p.groups` is the number of (possibly merged) groups the kernels see.
+    p.gm = group_merge(C_out, C_in, groups, p.elt);
+    if (p.gm > 1) {
+        p.groups = groups / p.gm;
+        p.Cin_g *= p.gm;
+        p.Cout_g *= p.gm;
+        p.Cpg = p.Cin_g;
+    }
     // Fewer than 32 bytes of channels per pixel: hardware im2col rows would be too
     // narrow, so the gather kernel builds the rows from x in place (groups = 1, the
     // whole C_out x K weight matrix resident in shared memory).
@@ -337,7 +426,7 @@ int make_plan(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stri
     p.Kp = p.taps * p.Cpg;
     if (p.kstages > (1 << 26)) return fail(CONV_ERR_UNSUPPORTED, "reduction too long (%d stages)", p.kstages);
     p.n_mtiles = static_cast<int>((p.M + 127) / 128);
-    long long base = static_cast<long long>(p.n_mtiles) * p.n_ntiles * groups;
+    long long base = static_cast<long long>(p.n_mtiles) * p.n_ntiles * p.groups;
     if (base >= (1LL << 31)) return fail(CONV_ERR_UNSUPPORTED, "too many tiles");
     p.splits = 1;
     if (sms > 0 && base < sms) {
@@ -350,7 +439,7 @@ int make_plan(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stri
     // read the other half from the peer, which halves the weight traffic and the
     // shared-memory bandwidth spent on it.  Used when the 256-row units still give
     // every SM pair work; the test hook can force or forbid them.
-    const long long pair_units = ((p.M + 255) / 256) * p.n_ntiles * groups;
+    const long long pair_units = ((p.M + 255) / 256) * p.n_ntiles * p.groups;
     const bool pair_ok = allow_pair && !p.f32 && p.BN % 32 == 0 && pair_mode != 2;
     if (pair_ok && ((p.splits == 1 && sms > 0 && pair_units >= sms / 2) || pair_mode == 1)) {
         p.pair = true;
@@ -373,11 +462,11 @@ int make_plan(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stri
 
     size_t off = 0;
     p.off_xcopy = off;
-    if (p.xcopy) off = align_up(off + static_cast<size_t>(N) * H * W * groups * p.Cpg * p.elt, 256);
+    if (p.xcopy) off = align_up(off + static_cast<size_t>(N) * H * W * p.groups * p.Cpg * p.elt, 256);
     p.off_partial = off;
     if (p.splits > 1) off = align_up(off + static_cast<size_t>(p.splits) * p.M * C_out * 4, 256);
     p.off_xcol = off;
-    if (explicit_im2col) off = align_up(off + static_cast<size_t>(p.M) * groups * p.Kp * p.elt, 256);
+    if (explicit_im2col) off = align_up(off + static_cast<size_t>(p.M) * p.groups * p.Kp * p.elt, 256);
     p.ws_total = off;
     *P = p;
     return CONV_OK;
@@ -535,6 +624,57 @@ int gather_impl(const Plan &p, const void *x, const void *w_packed, const void *
     return ok();
 }
 
+// The depthwise path: an optional channels-last (padded) copy of x, then one kernel.
+int dw_impl(const Plan &p, const void *x, const void *w_packed, const void *bias, void *y, void *workspace,
+            DeviceInfo *dev, const Settings &cfg, cudaStream_t stream) {
+    DwParams d;
+    std::memset(&d, 0, sizeof(d));
+    const void *x_nhwc = x;
+    int st;
+    if (p.xcopy) {
+        x_nhwc = workspace;
+        cudaError_t e = p.layout == CONV_NCHW
+                            ? launch_nchw_to_nhwc(x, workspace, p.N, p.C_in, p.H, p.W, 1, p.dw_Cp, p.elt, stream)
+                            : launch_nhwc_pad(x, workspace, p.N, p.C_in, p.H, p.W, 1, p.dw_Cp, p.elt, stream);
+        if ((st = check_launch(e, "channels-last copy")) != CONV_OK) return st;
+    }
+    cuuint64_t dims[4] = {static_cast<cuuint64_t>(p.dw_Cp), static_cast<cuuint64_t>(p.W),
+                          static_cast<cuuint64_t>(p.H), static_cast<cuuint64_t>(p.N)};
+    cuuint64_t strides[3] = {static_cast<cuuint64_t>(p.dw_Cp) * p.elt,
+                             static_cast<cuuint64_t>(p.dw_Cp) * p.elt * p.W,
+                             static_cast<cuuint64_t>(p.dw_Cp) * p.elt * p.W * p.H};
+    cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / p.elt), static_cast<cuuint32_t>(p.IW),
+                         static_cast<cuuint32_t>(p.IH), 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = g_encode_tiled(&d.tmap_x, tma_type(p), 4, const_cast<void *>(x_nhwc), dims, strides, box, estr,
+                                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return fail(CONV_ERR_CUDA, "cuTensorMapEncodeTiled (depthwise input) failed (%d)", static_cast<int>(r));
+    d.w_packed = w_packed;
+    d.bias = bias;
+    d.y = y;
+    d.N = p.N; d.C = p.C_in; d.Ho = p.Ho; d.Wo = p.Wo; d.Kh = p.Kh; d.Kw = p.Kw;
+    d.stride = p.stride; d.pad = p.pad; d.dilation = p.dilation;
+    d.Cpg = p.Cpg;
+    d.TH = p.TH; d.TW = p.TW; d.IH = p.IH; d.IW = p.IW;
+    d.n_th = p.n_th; d.n_tw = p.n_tw; d.units = p.units; d.stages = p.stages;
+    d.wregion = p.dw_wregion;
+    d.out_nchw = p.layout == CONV_NCHW ? 1 : 0;
+    d.vec_ok = (p.C_in % (16 / p.elt)) == 0 ? 1 : 0;
+    d.status = dev->status;
+    d.timeout_ns = cfg.timeout_ns;
+    d.starve = cfg.starve;
+    const long long slots = static_cast<long long>(dev->sms) * p.dw_ctas_per_sm;
+    const int grid = static_cast<int>(p.units < slots ? p.units : slots);
+    cudaEvent_t ev_start = g_main_start, ev_stop = g_main_stop;
+    if (ev_start && ev_stop && (st = record_event(ev_start, stream)) != CONV_OK) return st;
+    cudaError_t e = launch_depthwise(d, p.f32, p.dw_window, grid, p.smem, stream);
+    if ((st = check_launch(e, "depthwise")) != CONV_OK) return st;
+    if (ev_start && ev_stop && (st = record_event(ev_stop, stream)) != CONV_OK) return st;
+    return ok();
+}
+
 // Resident two-CTA clusters of the pair kernel for one configuration, asked of the
 // runtime once per configuration and device and remembered.
 int pair_cluster_limit(int cb, bool im2col, size_t smem) {
@@ -613,6 +753,7 @@ int forward_impl(bool explicit_im2col, const void *x, const void *w_packed, cons
         return fail(CONV_ERR_UNSUPPORTED, "device pointers must be 16-byte aligned");
 
     if (p.gather) return gather_impl(p, x, w_packed, bias, y, dev, cfg, stream);
+    if (p.dw) return dw_impl(p, x, w_packed, bias, y, workspace, dev, cfg, stream);
 
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     const void *x_nhwc = p.xcopy ? static_cast<const void *>(ws + p.off_xcopy) : x;
@@ -639,7 +780,7 @@ int forward_impl(bool explicit_im2col, const void *x, const void *w_packed, cons
     kp.planes = p.planes;
     kp.kstages = p.kstages;
     kp.Kp = p.Kp;
-    kp.groups = groups;
+    kp.groups = p.groups;
     kp.Cout_g = p.Cout_g;
     kp.Cout = C_out;
     kp.BN = p.BN;
@@ -682,12 +823,12 @@ int forward_impl(bool explicit_im2col, const void *x, const void *w_packed, cons
 
     if (p.xcopy) {
         cudaError_t e = layout == CONV_NCHW
-                            ? launch_nchw_to_nhwc(x, ws + p.off_xcopy, N, C_in, H, W, groups, p.Cpg, p.elt, stream)
-                            : launch_nhwc_pad(x, ws + p.off_xcopy, N, C_in, H, W, groups, p.Cpg, p.elt, stream);
+                            ? launch_nchw_to_nhwc(x, ws + p.off_xcopy, N, C_in, H, W, p.groups, p.Cpg, p.elt, stream)
+                            : launch_nhwc_pad(x, ws + p.off_xcopy, N, C_in, H, W, p.groups, p.Cpg, p.elt, stream);
         if ((st = check_launch(e, "channels-last copy")) != CONV_OK) return st;
     }
     if (explicit_im2col) {
-        cudaError_t e = launch_im2col(x_nhwc, xcol, N, H, W, groups, p.Cpg, p.Ho, p.Wo, Kh, Kw,
+        cudaError_t e = launch_im2col(x_nhwc, xcol, N, H, W, p.groups, p.Cpg, p.Ho, p.Wo, Kh, Kw,
                                       stride, pad, dilation, p.elt, stream);
         if ((st = check_launch(e, "im2col")) != CONV_OK) return st;
     }
@@ -730,13 +871,14 @@ int describe_impl(bool explicit_im2col, int N, int C_in, int H, int W, int C_out
                        explicit_im2col, sms, &p, cfg.pair_mode);
     }
     if (st != CONV_OK) return st;
-    const char *a_load = p.gather ? "gather" : explicit_im2col ? "xcol" : p.direct_a ? "tiled_x" : "im2col";
+    const char *a_load = p.dw ? "tile" : p.gather ? "gather" : explicit_im2col ? "xcol" : p.direct_a ? "tiled_x" : "im2col";
+    const char *kernel = p.dw ? "depthwise" : p.gather ? "gather" : "igemm";
     const int n = std::snprintf(
         buf, buflen,
         "{\"kernel\": \"%s\", \"pair\": %d, \"a_load\": \"%s\", \"BN\": %d, \"cb\": %d, "
         "\"stages\": %d, \"splits\": %d, \"units\": %d, \"xcopy\": %d, \"halo\": %d, "
         "\"tma_out\": %d, \"Kpad\": %d, \"smem\": %zu, \"workspace\": %zu, \"sms\": %d}",
-        p.gather ? "gather" : "igemm", p.pair ? 1 : 0, a_load, p.BN, p.gather ? 0 : p.cb,
+        kernel, p.pair ? 1 : 0, a_load, p.BN, p.gather ? 0 : p.cb,
         p.stages, p.gather ? 1 : p.splits, p.gather ? p.n_mtiles : p.units, p.xcopy ? 1 : 0,
         p.halo ? 1 : 0, p.tma_out ? 1 : 0, p.gather ? p.Kpad : 0, p.smem, p.ws_total, sms);
     if (n < 0 || static_cast<size_t>(n) >= buflen)
@@ -816,9 +958,11 @@ int conv2d_pack_weight(const void *w_oihw, void *w_packed, int C_out, int C_in, 
     if (st != CONV_OK) return st;
     if (!w_oihw || !w_packed) return fail(CONV_ERR_INVALID_ARG, "weight pointers must not be NULL");
     const int elt = elt_of(dtype);
-    const int cpg = round_up(C_in / groups, 16 / elt);
+    const int gm = group_merge(C_out, C_in, groups, elt);
+    const int cpg = round_up(C_in / groups, 16 / elt) * gm;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if ((st = check_launch(launch_pack_weight(w_oihw, w_packed, C_out, C_in / groups, Kh, Kw, cpg, elt, s),
+    if ((st = check_launch(launch_pack_weight(w_oihw, w_packed, C_out, C_in / groups, C_out / groups, gm, Kh,
+                                              Kw, cpg, elt, s),
                            "weight pack")) != CONV_OK)
         return st;
     const GatherImages gi = gather_images(C_out, C_in, Kh, Kw, groups, elt);

@@ -91,6 +91,25 @@ struct GatherParams {
     int starve;
 };
 
+// One launch of the depthwise kernel (depthwise.cu): groups = C_in = C_out, x
+// channels-last with Cp >= C channels per pixel (a multiple of 16 bytes).  Tiles are
+// TH x TW output pixels x 128 bytes of channels; tile u = ((chunk*N + n)*n_th + th)*n_tw + tw.
+struct DwParams {
+    CUtensorMap tmap_x;    // x as {Cp, W, H, N}, boxes of {128 bytes, IW, IH, 1}
+    const void *w_packed;  // (C, Kh, Kw, Cpg) from conv2d_pack_weight
+    const void *bias;
+    void *y;
+    int N, C, Ho, Wo, Kh, Kw, stride, pad, dilation;
+    int Cpg;               // channel pitch of w_packed
+    int TH, TW, IH, IW;    // output tile and the staged input box
+    int n_th, n_tw, units, stages;
+    int wregion;           // bytes of the per-warp weight copies ahead of the stage ring
+    int out_nchw, vec_ok;
+    int *status;
+    long long timeout_ns;
+    int starve;
+};
+
 // Launchers (igemm.cu, gather.cu, layout.cu).  All return cudaSuccess or the launch error.
 // pair: bf16 only, grid even, launched as clusters of two CTAs (p.n_mtiles counts
 // 256-row units, the tensor map of B has boxes of BN/2 rows).
@@ -105,14 +124,25 @@ size_t gather_smem_bytes(bool f32, int BN, int Kpad, size_t halo_bytes, size_t o
 int gather_max_stages();
 int igemm_threads(bool f32);
 
+// window_k: 3, 5 or 7 for the register-window form (stride 1, unit dilation, square
+// filter), 0 for the general form.
+cudaError_t launch_depthwise(const DwParams &p, bool f32, int window_k, int grid, size_t smem,
+                             cudaStream_t stream);
+int dw_pixels_per_thread();
+int dw_threads();
+int dw_compute_warps();
+int dw_max_stages();
+size_t dw_header_bytes();
+
 cudaError_t launch_nchw_to_nhwc(const void *src, void *dst, int N, int C, int H, int W,
                                 int groups, int Cpg, int elt, cudaStream_t s);
 cudaError_t launch_nhwc_pad(const void *src, void *dst, int N, int C, int H, int W, int groups,
                             int Cpg, int elt, cudaStream_t s);
 cudaError_t launch_nhwc_to_nchw(const void *src, void *dst, int N, int C, int H, int W, int elt,
                                 cudaStream_t s);
-cudaError_t launch_pack_weight(const void *w, void *wp, int Cout, int Cin_g, int Kh, int Kw,
-                               int Cpg, int elt, cudaStream_t s);
+// gm > 1: groups merged gm at a time, block-diagonal (see group_merge in abi.cu).
+cudaError_t launch_pack_weight(const void *w, void *wp, int Cout, int Cin_g, int Cout_g, int gm, int Kh,
+                               int Kw, int Cpg, int elt, cudaStream_t s);
 cudaError_t launch_pack_gather_image(const void *w, void *img, int Cout, int C, int Kh, int Kw,
                                      int BN, int Kpad, bool rowvec, int elt, cudaStream_t s);
 cudaError_t launch_im2col(const void *x_nhwc, void *xcol, int N, int H, int W, int groups,

@@ -250,10 +250,12 @@ __global__ void nhwc_to_nchw_tiled(const void *__restrict__ src, void *__restric
     }
 }
 
-// --- weights OIHW (Cout, Cin_g, Kh, Kw) -> (Cout, Kh, Kw, Cpg), zero for c >= Cin_g.
+// --- weights OIHW (Cout, Cin_g, Kh, Kw) -> (Cout, Kh, Kw, Cpg), zero for c >= Cin_g.  With
+// groups merged gm at a time (gm > 1), Cpg = gm * Cin_g and output channel oc keeps its
+// weights in block j = (oc / Cout_g) % gm of its row, zeros elsewhere (block-diagonal).
 template <int kElt>
 __global__ void pack_weight_kernel(const void *__restrict__ w, void *__restrict__ wp, int Cout,
-                                   int Cin_g, int Kh, int Kw, int Cpg) {
+                                   int Cin_g, int Cout_g, int gm, int Kh, int Kw, int Cpg) {
     using T = typename Word<kElt>::T;
     const T *s = static_cast<const T *>(w);
     T *d = static_cast<T *>(wp);
@@ -266,7 +268,11 @@ __global__ void pack_weight_kernel(const void *__restrict__ w, void *__restrict_
         r /= Kw;
         const int kh = static_cast<int>(r % Kh);
         const long long oc = r / Kh;
-        d[i] = c < Cin_g ? s[((oc * Cin_g + c) * Kh + kh) * Kw + kw] : T(0);
+        // merged groups: output channel oc belongs to sub-group j of its merged group and
+        // sees only that sub-group's Cin_g channels (block-diagonal)
+        const int j = static_cast<int>((oc / Cout_g) % gm);
+        const int cl = c - j * Cin_g;
+        d[i] = (cl >= 0 && cl < Cin_g) ? s[((oc * Cin_g + cl) * Kh + kh) * Kw + kw] : T(0);
     }
 }
 
@@ -453,13 +459,13 @@ cudaError_t launch_nhwc_to_nchw(const void *src, void *dst, int N, int C, int H,
     return cudaGetLastError();
 }
 
-cudaError_t launch_pack_weight(const void *w, void *wp, int Cout, int Cin_g, int Kh, int Kw,
-                               int Cpg, int elt, cudaStream_t s) {
+cudaError_t launch_pack_weight(const void *w, void *wp, int Cout, int Cin_g, int Cout_g, int gm, int Kh,
+                               int Kw, int Cpg, int elt, cudaStream_t s) {
     const long long total = static_cast<long long>(Cout) * Kh * Kw * Cpg;
     if (elt == 2)
-        pack_weight_kernel<2><<<grid_for(total), kThreads, 0, s>>>(w, wp, Cout, Cin_g, Kh, Kw, Cpg);
+        pack_weight_kernel<2><<<grid_for(total), kThreads, 0, s>>>(w, wp, Cout, Cin_g, Cout_g, gm, Kh, Kw, Cpg);
     else
-        pack_weight_kernel<4><<<grid_for(total), kThreads, 0, s>>>(w, wp, Cout, Cin_g, Kh, Kw, Cpg);
+        pack_weight_kernel<4><<<grid_for(total), kThreads, 0, s>>>(w, wp, Cout, Cin_g, Cout_g, gm, Kh, Kw, Cpg);
     return cudaGetLastError();
 }
 

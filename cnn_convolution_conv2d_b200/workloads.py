@@ -85,6 +85,13 @@ CONFIGS = {
                                 "bf16", "nhwc", ("normal", 1.0), _he(512 * 49), ("normal", 1.0), 5),
     "k7_17x17_f32": ConvConfig("k7_17x17_f32", 16, 512, 17, 17, 512, 7, 7, 1, 3, 1, 1, True,
                                "f32", "nhwc", ("normal", 1.0), _he(512 * 49), ("normal", 1.0), 5),
+    # depthwise 3x3 (groups = C_in = C_out, one filter per channel): the variant the
+    # im2col/GEMM tutorial (zskr.cn/news/1820658) §4.2 and "手撕 Conv2D" §7 single out;
+    # the 3x3 layer's activations, 64x256x56x56, stride 1, pad 1, bias; w ~ N(0, 2/9)
+    "depthwise3x3_bf16": ConvConfig("depthwise3x3_bf16", 64, 256, 56, 56, 256, 3, 3, 1, 1, 1, 256, True,
+                                    "bf16", "nhwc", ("normal", 1.0), _he(9), ("normal", 1.0), 6),
+    "depthwise3x3_f32": ConvConfig("depthwise3x3_f32", 64, 256, 56, 56, 256, 3, 3, 1, 1, 1, 256, True,
+                                   "f32", "nhwc", ("normal", 1.0), _he(9), ("normal", 1.0), 6),
 }
 
 

@@ -73,7 +73,11 @@ int conv2d_output_size(int in, int k, int stride, int pad, int dilation, int *ou
  * C_out * Kh * Kw * Cpg elements of dtype, where Cpg is C_in/groups rounded up
  * to a multiple of 8 (bf16) or 4 (fp32), followed -- for groups = 1 and fewer
  * than 32 bytes of input channels per pixel -- by ready-made shared-memory images
- * of the weight matrix for the few-channel kernel. */
+ * of the weight matrix for the few-channel kernel.  Narrow groups (fewer than 64
+ * output channels each, C_in/groups a multiple of 8 bf16 / 4 fp32) are packed gm at
+ * a time as one block-diagonal group, Cpg = gm * C_in/groups, with gm the largest
+ * divisor of groups that keeps gm * C_out/groups <= 128 and gm * C_in/groups * the
+ * element size <= 256 bytes; the forward pass then computes gm groups per product. */
 int conv2d_packed_weight_size(int C_out, int C_in, int Kh, int Kw, int groups,
                               conv_dtype_t dtype, size_t *bytes);
 
@@ -104,7 +108,10 @@ int conv2d_workspace_size(int N, int C_in, int H, int W, int C_out, int Kh, int 
  * tile by tile into shared memory by the tensor memory accelerator's im2col mode
  * (out-of-image reads return zero: the zero padding), weights by tiled loads,
  * tcgen05 tensor-core instructions accumulate in tensor memory, and the epilogue
- * adds bias and stores y in `layout`.
+ * adds bias and stores y in `layout`.  Depthwise problems (groups = C_in = C_out:
+ * one filter per channel) instead run a direct stencil kernel over channels-last
+ * tiles staged in shared memory -- the case the im2col/GEMM tutorial §4.2 names as
+ * one where im2col only adds traffic -- with the same arguments and results.
  *   x         : input, layout as above, dtype elements
  *   w_packed  : weights from conv2d_pack_weight (same C_out, C_in, Kh, Kw, groups, dtype)
  *   bias      : (C_out,) dtype elements, or NULL for no bias

@@ -59,7 +59,10 @@ def test_output_size_rejects(lib, args):
 
 def test_packed_weight_size(lib):
     # many channels or groups: only the (C_out, Kh, Kw, Cpg) weights
-    assert cb.conv2d_packed_weight_size(512, 512, 3, 3, 32, cb.CONV_BF16) == 512 * 9 * 16 * 2
+    # 32 groups of 16 -> 16 channels: merged 8 at a time, block-diagonal rows of 8 * 16 channels
+    assert cb.conv2d_packed_weight_size(512, 512, 3, 3, 32, cb.CONV_BF16) == 512 * 9 * 16 * 8 * 2
+    assert cb.conv2d_packed_weight_size(512, 512, 3, 3, 32, cb.CONV_F32) == 512 * 9 * 16 * 4 * 4  # 4 at a time
+    assert cb.conv2d_packed_weight_size(24, 24, 3, 3, 4, cb.CONV_BF16) == 24 * 9 * 8 * 2  # 12-byte rows: no merge
     assert cb.conv2d_packed_weight_size(256, 256, 3, 3, 1, cb.CONV_BF16) == 256 * 9 * 256 * 2
     # few input channels: followed (256-byte aligned) by the gather kernel's images,
     # 16-row x Kpad matrices for the compact and row-vector reduction orders
@@ -171,8 +174,8 @@ def test_plan_for_the_workloads_on_a_148_sm_device(lib):
     k7 = _plan((16, 512, 17, 17, 512, 7, 7, 1, 3, 1, 1), sms=148)     # 19 pair units < 74: single CTAs, split
     assert (k7["pair"], k7["splits"], k7["units"]) == (0, 2, 37 * 2 * 2)
     assert k7["workspace"] == 2 * 16 * 17 * 17 * 512 * 4               # fp32 partial sums per split
-    g = _plan((16, 512, 28, 28, 512, 3, 3, 2, 2, 2, 32), sms=148)     # 16 channels per group
-    assert (g["pair"], g["BN"], g["cb"]) == (0, 16, 32)
+    g = _plan((16, 512, 28, 28, 512, 3, 3, 2, 2, 2, 32), sms=148)     # 16 channels per group, merged 8 at a time
+    assert (g["pair"], g["BN"], g["cb"], g["units"]) == (0, 128, 128, 25 * 4)
     ex = _plan((64, 256, 56, 56, 256, 3, 3, 1, 1, 1, 1), explicit_im2col=True, sms=148)
     assert ex["a_load"] == "xcol" and ex["workspace"] >= 924_844_032   # the 924.8 MB X_col
     f32 = _plan((16, 512, 17, 17, 512, 7, 7, 1, 3, 1, 1), dtype=cb.CONV_F32, sms=148)
@@ -216,3 +219,19 @@ def test_bench_mirror_of_the_gather_choice_agrees_with_the_library(lib):
                                        c.groups, cb.CONV_BF16 if c.dtype == "bf16" else cb.CONV_F32, c.layout,
                                        sms=148)
         assert (plan["kernel"] == "gather") == bench.uses_gather(c), name
+        assert (plan["kernel"] == "depthwise") == bench.uses_depthwise(c), name
+
+
+def test_depthwise_plans(lib):
+    """groups = C_in = C_out goes to the depthwise stencil kernel: register-window form for
+    stride-1 square 3/5/7 filters, channel-padded copy when 16-byte rows need it."""
+    d = _plan((64, 256, 56, 56, 256, 3, 3, 1, 1, 1, 256), sms=148)
+    assert (d["kernel"], d["a_load"], d["xcopy"], d["workspace"]) == ("depthwise", "tile", 0, 0)
+    assert d["units"] == 4 * 64 * 2 * 7            # 64-channel chunks x images x 32x8 output tiles
+    odd = _plan((2, 20, 9, 9, 20, 5, 3, 2, 2, 2, 20), sms=148)   # 40-byte rows: padded copy
+    assert odd["kernel"] == "depthwise" and odd["xcopy"] == 1
+    assert odd["workspace"] == 2 * 9 * 9 * 24 * 2 + (256 - (2 * 9 * 9 * 24 * 2) % 256) % 256
+    nchw = _plan((4, 32, 10, 10, 32, 3, 3, 1, 1, 1, 32), dtype=cb.CONV_F32, layout="nchw", sms=148)
+    assert nchw["kernel"] == "depthwise" and nchw["xcopy"] == 1
+    mult = _plan((2, 16, 8, 8, 32, 3, 3, 1, 1, 1, 16), sms=148)  # channel multiplier 2: general kernel
+    assert mult["kernel"] == "igemm"
