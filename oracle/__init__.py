@@ -9,7 +9,9 @@ arithmetic is kept) and exposed through ctypes:
   * ``conv2d_oracle.c``: the forward pass, six nested loops with bounds-checked zero
     padding, after the "手撕 Conv2D" page (lpnh.cn/news/2493075) §1.1-§2.1;
   * ``conv2d_backward_oracle.c``: the gradients dx, dW, db, after the same page's
-    §5.1-§5.2 naive backward loops.
+    §5.1-§5.2 naive backward loops;
+  * ``conv3d_oracle.c``: the 3-D forward pass of "PyTorch高维张量乘法与conv2d/conv3d
+    维度语义解析" §5.1, the same loops with a depth dimension.
 Inputs are widened to float64 before the call; widening bf16- or fp32-valued data
 is exact.
 """
@@ -26,9 +28,12 @@ SOURCE = os.path.join(_HERE, "conv2d_oracle.c")
 LIBRARY = os.path.join(_HERE, "liboracle.so")
 BWD_SOURCE = os.path.join(_HERE, "conv2d_backward_oracle.c")
 BWD_LIBRARY = os.path.join(_HERE, "liboracle_backward.so")
+C3D_SOURCE = os.path.join(_HERE, "conv3d_oracle.c")
+C3D_LIBRARY = os.path.join(_HERE, "liboracle_conv3d.so")
 
 _lib = None
 _bwd = None
+_c3d = None
 
 
 def build(source: str = SOURCE, output: str = LIBRARY, extra_flags=()) -> str:
@@ -43,6 +48,7 @@ def build_all() -> None:
     """Compile every C oracle of this package."""
     build(SOURCE, LIBRARY)
     build(BWD_SOURCE, BWD_LIBRARY)
+    build(C3D_SOURCE, C3D_LIBRARY)
 
 
 def load(path: str | None = None):
@@ -215,6 +221,64 @@ def conv2d_backward_weight_points(dy, x, w_shape, idx, stride=1, pad=0, dilation
     out = np.empty(idx.shape[0])
     rc = lib.oracle_conv2d_backward_weight_points(_ptr(dy), _ptr(x), N, C_in, H, W, C_out, Kh, Kw, stride,
                                                   pad, dilation, groups, _ptr(idx), idx.shape[0], _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle rejected the shape or an index")
+    return out
+
+
+# ------------------------------------------------------------------ conv3d ---
+def _bind_conv3d(lib):
+    L = ctypes.c_long
+    P = ctypes.c_void_p
+    lib.oracle_conv3d.argtypes = [P, P, P, P] + [L] * 13
+    lib.oracle_conv3d.restype = ctypes.c_int
+    lib.oracle_conv3d_points.argtypes = [P, P, P] + [L] * 13 + [P, L, P]
+    lib.oracle_conv3d_points.restype = ctypes.c_int
+    return lib
+
+
+def load_conv3d(path: str | None = None):
+    """Load (building first if needed) the conv3d oracle library."""
+    global _c3d
+    if path is not None:
+        return _bind_conv3d(ctypes.CDLL(path))
+    if _c3d is None:
+        if (not os.path.exists(C3D_LIBRARY)
+                or os.path.getmtime(C3D_LIBRARY) < os.path.getmtime(C3D_SOURCE)):
+            build(C3D_SOURCE, C3D_LIBRARY)
+        _c3d = _bind_conv3d(ctypes.CDLL(C3D_LIBRARY))
+    return _c3d
+
+
+def conv3d(x, w, bias=None, stride=1, pad=0, dilation=1, groups=1, lib=None):
+    """y = conv3d(x, w, bias) in float64; x NCDHW, w OIDHW (C_out, C_in/groups, Kd, Kh, Kw)."""
+    lib = lib or load_conv3d()
+    x, w, bias = _f64(x), _f64(w), _f64(bias)
+    N, C_in, D, H, W = x.shape
+    C_out, cin_g, Kd, Kh, Kw = w.shape
+    if cin_g * groups != C_in:
+        raise ValueError("weight shape does not match C_in / groups")
+    if bias is not None and bias.shape != (C_out,):
+        raise ValueError("bias must have shape (C_out,)")
+    Do, Ho, Wo = (out_size(v, k, stride, pad, dilation) for v, k in ((D, Kd), (H, Kh), (W, Kw)))
+    y = np.empty((N, C_out, Do, Ho, Wo), dtype=np.float64)
+    rc = lib.oracle_conv3d(_ptr(x), _ptr(w), _ptr(bias), _ptr(y), N, C_in, D, H, W, C_out, Kd, Kh, Kw, stride,
+                           pad, dilation, groups)
+    if rc != 0:
+        raise ValueError("oracle rejected the shape")
+    return y
+
+
+def conv3d_points(x, w, bias, idx, stride=1, pad=0, dilation=1, groups=1, lib=None):
+    """Selected outputs y[n, oc, od, oh, ow] for the rows of ``idx``."""
+    lib = lib or load_conv3d()
+    x, w, bias = _f64(x), _f64(w), _f64(bias)
+    idx = np.ascontiguousarray(idx, dtype=np.int64).reshape(-1, 5)
+    N, C_in, D, H, W = x.shape
+    C_out, _, Kd, Kh, Kw = w.shape
+    out = np.empty(idx.shape[0])
+    rc = lib.oracle_conv3d_points(_ptr(x), _ptr(w), _ptr(bias), N, C_in, D, H, W, C_out, Kd, Kh, Kw, stride, pad,
+                                  dilation, groups, _ptr(idx), idx.shape[0], _ptr(out))
     if rc != 0:
         raise ValueError("oracle rejected the shape or an index")
     return out
