@@ -55,6 +55,7 @@ TF32_PRODUCTS = 3
 KERNEL_SOURCES = {
     "igemm_kernel": ["igemm.cu", "epilogue.cuh", "ptx.cuh", "common.cuh"],
     "gather_kernel": ["gather.cu", "epilogue.cuh", "ptx.cuh", "common.cuh"],
+    "gather_t_kernel": ["gather_t.cu", "ptx.cuh", "common.cuh"],
     "dw_kernel": ["depthwise.cu", "ptx.cuh", "common.cuh"],
 }
 
@@ -167,7 +168,16 @@ def committed_traffic(workload: str):
     return scale * (float(d["dram_bytes_read"]) + max(float(d["dram_bytes_write"]), float(d["l2_write_bytes"])))
 
 
-def roofline(cfg, kernel_ms: float, peaks, peak_kind: str, workload: str, explicit: bool = False) -> dict:
+KERNEL_LABELS = {
+    "igemm": "igemm_kernel (implicit GEMM: TMA im2col/tiled loads, tcgen05; CTA pairs on large bf16 problems)",
+    "gather": "gather_kernel (software-gathered im2col rows in tensor memory, tcgen05)",
+    "gather_t": "gather_t_kernel (transposed product: output channels on the lanes, one output row per tile)",
+    "depthwise": "dw_kernel (depthwise stencil over TMA-staged channels-last tiles, CUDA cores)",
+}
+
+
+def roofline(cfg, kernel_ms: float, peaks, peak_kind: str, workload: str, explicit: bool = False,
+             plan_kernel: str | None = None) -> dict:
     f = flops(cfg)
     b = explicit_kernel_bytes(cfg) if explicit else main_kernel_bytes(cfg)
     ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
@@ -192,11 +202,9 @@ def roofline(cfg, kernel_ms: float, peaks, peak_kind: str, workload: str, explic
         out = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                "peak_source": f"{peak_kind} HBM copy bandwidth"}
     out["frac"] = achieved / peak
-    out["kernel"] = ("dw_kernel (depthwise stencil over TMA-staged channels-last tiles, CUDA cores)"
-                     if uses_depthwise(cfg)
-                     else "gather_kernel (software-gathered im2col rows, tcgen05)" if uses_gather(cfg)
-                     else "igemm_kernel (implicit GEMM: TMA im2col/tiled loads, tcgen05; "
-                          "CTA pairs on large bf16 problems)")
+    if plan_kernel is None:
+        plan_kernel = "depthwise" if uses_depthwise(cfg) else "gather" if uses_gather(cfg) else "igemm"
+    out["kernel"] = KERNEL_LABELS.get(plan_kernel, plan_kernel)
     out["kernel_ms"] = kernel_ms
     out["algorithmic_bytes_per_launch"] = b
     out["algorithmic_flops_per_launch"] = f
@@ -538,7 +546,11 @@ def run_ours(args, cfg):
 
     if rank == 0:
         peaks, peak_kind = load_peaks()
+        plan = cb.conv2d_describe_plan(cfg.N, cfg.C_in, cfg.H, cfg.W, cfg.C_out, cfg.Kh, cfg.Kw, cfg.stride, cfg.pad,
+                                       cfg.dilation, cfg.groups, cb.CONV_BF16 if cfg.dtype == "bf16" else cb.CONV_F32,
+                                       cfg.layout, explicit_im2col=ex)
         cfgd = workload_config(cfg, args, world)
+        cfgd["plan"] = plan
         cfgd["l2"] = (f"not resident: steps rotate over {nsets} input/output sets "
                       f"({nsets * set_bytes / 1e6:.0f} MB > 2x the 126 MB L2)")
         cfgd["launch"] = f"CUDA graphs of {G} steps x {reps} replays" if args.graph else "eager"
@@ -551,8 +563,8 @@ def run_ours(args, cfg):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": cfg.dtype, "data": "synthetic (seeded; x ~ N(0,1), He-scaled weights)",
             "config": cfgd,
-            "roofline": with_write_context(roofline(cfg, kernel_ms, peaks, peak_kind, cfg.name, ex), cfg,
-                                           kernel_ms, fill_gbs),
+            "roofline": with_write_context(roofline(cfg, kernel_ms, peaks, peak_kind, cfg.name, ex,
+                                                    plan_kernel=plan["kernel"]), cfg, kernel_ms, fill_gbs),
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
@@ -568,6 +580,339 @@ def run_ours(args, cfg):
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def run_backward(args, cfg):
+    """Throughput of one backward pass on one GPU: --backward data (dx: the transposed
+    convolution on the forward kernels, zero-inserted dy for stride > 1) or weight (dW
+    and db: the pixel-reduction tensor-core product, or the CUDA-core kernel for few
+    channels per group).  Same timing as the forward line: W warm-up steps, K steps in
+    CUDA graphs, inputs rotated over sets larger than 2x L2, CUDA events on the stream
+    and around the main kernel.  FLOPs are the gradient's algorithmic count, equal to
+    the forward pass's (pwwt §3.3's formula)."""
+    import torch
+    import cnn_convolution_conv2d_b200 as cb
+    from cnn_convolution_conv2d_b200 import build, workloads
+
+    build.build()
+    cb.load()
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(0)
+    inp = workloads.make_inputs(cfg)
+    dt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+    x_host = torch.from_numpy(inp["x"]).to(dt)
+    if cfg.layout == "nhwc":
+        x_host = x_host.permute(0, 2, 3, 1).contiguous()
+    w = torch.from_numpy(inp["w"]).to(dt).to(device)
+    b = None if inp["b"] is None else torch.from_numpy(inp["b"]).to(dt).to(device)
+    layer = cb.Conv2dB200(w, b, cfg.stride, cfg.pad, cfg.dilation, cfg.groups, cfg.layout)
+    y_shape = layer.out_shape(cfg.N, cfg.H, cfg.W)
+    g = torch.Generator().manual_seed(cfg.seed + 500)
+    dy_host = torch.randn(y_shape, generator=g).to(dt)
+    set_bytes = (x_host.numel() + dy_host.numel()) * x_host.element_size()
+    nsets = max(2, min(16, math.ceil(2 * L2_BYTES / set_bytes) + 1))
+    dys = [dy_host.to(device) for _ in range(nsets)]
+    if args.backward == "data":
+        outs = [torch.empty(x_host.shape, dtype=dt, device=device) for _ in range(nsets)]
+
+        def step(i):
+            layer.backward_data(dys[i % nsets], cfg.H, cfg.W, dx=outs[i % nsets])
+    else:
+        xs = [x_host.to(device) for _ in range(nsets)]
+        dw = torch.empty(tuple(w.shape), dtype=dt, device=device)
+        db = None if b is None else torch.empty(cfg.C_out, dtype=dt, device=device)
+
+        def step(i):
+            layer.backward_weight(xs[i % nsets], dys[i % nsets], dw=dw, db=db)
+    for i in range(max(args.warmup, 3)):
+        step(i)
+    cb.conv2d_sync_status()
+    G = 1
+    for gsz in range(min(args.steps, 256), 0, -1):
+        if args.steps % gsz == 0:
+            G = gsz
+            break
+    reps = args.steps // G
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(G)]
+    for a, c in kev:
+        a.record()
+        c.record()
+    torch.cuda.synchronize()
+    launches0 = cb.conv2d_kernel_launch_count()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for i in range(G):
+            cb.conv2d_set_main_kernel_events(*kev[i])
+            step(i)
+    cb.conv2d_set_main_kernel_events(None, None)
+    launches_per_rep = cb.conv2d_kernel_launch_count() - launches0
+    graph.replay()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(0)
+    clocks.start()
+    time.sleep(0.05)
+    stream = torch.cuda.current_stream()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    ev0.record(stream)
+    for _ in range(reps):
+        graph.replay()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    t1 = time.perf_counter()
+    clocks.stop()
+    cb.conv2d_sync_status()
+    elapsed = ev0.elapsed_time(ev1)
+    kernel_ms = statistics.fmean(a.elapsed_time(c) for a, c in kev)
+    f = flops(cfg)
+    peaks, peak_kind = load_peaks()
+    plan = cb.conv2d_describe_plan(cfg.N, cfg.C_in, cfg.H, cfg.W, cfg.C_out, cfg.Kh, cfg.Kw, cfg.stride, cfg.pad,
+                                   cfg.dilation, cfg.groups, cb.CONV_BF16 if cfg.dtype == "bf16" else cb.CONV_F32,
+                                   cfg.layout)
+    executed = f * (cfg.stride ** 2 if args.backward == "data" else 1)
+    achieved = executed / (kernel_ms * 1e-3) / 1e12
+    if cfg.dtype == "bf16":
+        peak, ksrc = peaks["bf16_tflops_sustained"], f"{peak_kind} bf16 sustained"
+    else:
+        achieved *= TF32_PRODUCTS
+        peak, ksrc = peaks["bf16_tflops_sustained"] * TF32_PER_BF16, f"{peak_kind} bf16 sustained x {TF32_PER_BF16}"
+    line = {
+        "metric": f"conv2d backward-{args.backward} TFLOP/s on 1 B200 and % of dense tensor roofline",
+        "value": f * args.steps / (elapsed * 1e-3) / 1e12, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": elapsed / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic (seeded; dy ~ N(0,1))",
+        "config": {"workload": workload_config(cfg, args, 1)["workload"], "pass": args.backward,
+                   "l2": f"not resident: steps rotate over {nsets} sets ({nsets * set_bytes / 1e6:.0f} MB)",
+                   "launch": f"CUDA graphs of {G} steps x {reps} replays", "forward_plan": plan},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "peak_source": ksrc, "kernel_ms": kernel_ms, "algorithmic_flops_per_launch": f,
+                     "executed_flops_per_launch": executed, "traffic": None,
+                     "kernel": ("igemm_kernel / dw_kernel on the transposed convolution" if args.backward == "data"
+                                else "wgrad_kernel (pixel-reduction tcgen05 product, MN-major operands)"
+                                if (cfg.C_in // cfg.groups) * elt_bytes(cfg) >= 32
+                                else "wgrad_direct_kernel (CUDA cores)")},
+        "gpu_launches": launches_per_rep * reps,
+        "clocks": clocks.summary(t0, t1),
+    }
+    print(json.dumps(line), flush=True)
+    del graph
+
+
+def run_conv3d(args, cfg):
+    """Throughput of the 3-D forward pass (conv3d_forward) on one GPU, with the forward
+    line's timing: W warm-up steps, K steps in CUDA graphs, inputs rotated over sets
+    larger than 2x L2, CUDA events on the stream and around the tensor-core kernel.
+    FLOPs = 2*N*C_out*Do*Ho*Wo*(C_in/groups)*Kd*Kh*Kw (pwwt §3.3's count, one more
+    spatial factor)."""
+    import torch
+    import cnn_convolution_conv2d_b200 as cb
+    from cnn_convolution_conv2d_b200 import build, workloads
+
+    build.build()
+    cb.load()
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(0)
+    inp = workloads.make_inputs3d(cfg)
+    dt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+    x_host = torch.from_numpy(inp["x"]).to(dt)
+    if cfg.layout == "nhwc":
+        x_host = x_host.permute(0, 2, 3, 4, 1).contiguous()
+    w = torch.from_numpy(inp["w"]).to(dt).to(device)
+    b = None if inp["b"] is None else torch.from_numpy(inp["b"]).to(dt).to(device)
+    layer = cb.Conv3dB200(w, b, cfg.stride, cfg.pad, cfg.dilation, cfg.groups, cfg.layout)
+    y_shape = layer.out_shape(cfg.N, cfg.D, cfg.H, cfg.W)
+    set_bytes = (x_host.numel() + math.prod(y_shape)) * x_host.element_size()
+    nsets = max(2, min(16, math.ceil(2 * L2_BYTES / set_bytes) + 1))
+    xs = [x_host.to(device) for _ in range(nsets)]
+    ys = [torch.empty(y_shape, dtype=dt, device=device) for _ in range(nsets)]
+    for i in range(max(args.warmup, 3)):
+        layer(xs[i % nsets], ys[i % nsets])
+    cb.conv2d_sync_status()
+    G = 1
+    for gsz in range(min(args.steps, 256), 0, -1):
+        if args.steps % gsz == 0:
+            G = gsz
+            break
+    reps = args.steps // G
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(G)]
+    for a, c in kev:
+        a.record()
+        c.record()
+    torch.cuda.synchronize()
+    launches0 = cb.conv2d_kernel_launch_count()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for i in range(G):
+            cb.conv2d_set_main_kernel_events(*kev[i])
+            layer(xs[i % nsets], ys[i % nsets])
+    cb.conv2d_set_main_kernel_events(None, None)
+    launches_per_rep = cb.conv2d_kernel_launch_count() - launches0
+    graph.replay()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(0)
+    clocks.start()
+    time.sleep(0.05)
+    stream = torch.cuda.current_stream()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    ev0.record(stream)
+    for _ in range(reps):
+        graph.replay()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    t1 = time.perf_counter()
+    clocks.stop()
+    cb.conv2d_sync_status()
+    elapsed = ev0.elapsed_time(ev1)
+    kernel_ms = statistics.fmean(a.elapsed_time(c) for a, c in kev)
+    e = elt_bytes(cfg)
+    f = 2.0 * cfg.N * cfg.C_out * cfg.Do * cfg.Ho * cfg.Wo * (cfg.C_in // cfg.groups) * cfg.Kd * cfg.Kh * cfg.Kw
+    nbytes = e * (cfg.N * cfg.C_in * cfg.D * cfg.H * cfg.W + cfg.C_out * (cfg.C_in // cfg.groups) * cfg.Kd * cfg.Kh
+                  * cfg.Kw + (cfg.C_out if cfg.bias else 0) + cfg.N * cfg.C_out * cfg.Do * cfg.Ho * cfg.Wo)
+    peaks, peak_kind = load_peaks()
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    mult = 1 if cfg.dtype == "bf16" else TF32_PRODUCTS
+    tpeak = peaks["bf16_tflops_sustained"] * (1 if cfg.dtype == "bf16" else TF32_PER_BF16)
+    if mult * f / nbytes >= ridge * tpeak / peaks["bf16_tflops_sustained"]:
+        achieved = mult * f / (kernel_ms * 1e-3) / 1e12
+        rl = {"bound": "tensor", "achieved": achieved, "peak": tpeak, "unit": "TFLOP/s", "frac": achieved / tpeak,
+              "peak_source": f"{peak_kind} bf16 sustained" + ("" if mult == 1 else f" x {TF32_PER_BF16}, x3 products")}
+    else:
+        achieved = nbytes / (kernel_ms * 1e-3) / 1e9
+        rl = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+              "frac": achieved / peaks["hbm_gbs"], "peak_source": f"{peak_kind} HBM copy bandwidth"}
+    rl.update({"kernel": "igemm_kernel (5-D TMA im2col, tcgen05)", "kernel_ms": kernel_ms,
+               "algorithmic_flops_per_launch": f, "algorithmic_bytes_per_launch": nbytes, "traffic": None})
+    desc = (f"{cfg.name}: N={cfg.N} C_in={cfg.C_in} {cfg.D}x{cfg.H}x{cfg.W} -> C_out={cfg.C_out}, "
+            f"{cfg.Kd}x{cfg.Kh}x{cfg.Kw} s{cfg.stride} p{cfg.pad} d{cfg.dilation} g{cfg.groups}, {cfg.dtype}, "
+            f"{'NDHWC' if cfg.layout == 'nhwc' else 'NCDHW'} in/out")
+    line = {
+        "metric": "conv3d fwd TFLOP/s on 1 B200 and % of dense tensor (or HBM) roofline",
+        "value": f * args.steps / (elapsed * 1e-3) / 1e12, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": elapsed / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic (seeded; x ~ N(0,1), He-scaled weights)",
+        "config": {"workload": desc, "l2": f"not resident: steps rotate over {nsets} sets",
+                   "launch": f"CUDA graphs of {G} steps x {reps} replays"},
+        "roofline": rl, "gpu_launches": launches_per_rep * reps, "clocks": clocks.summary(t0, t1),
+    }
+    print(json.dumps(line), flush=True)
+    del graph
+
+
+def run_winograd(args, cfg):
+    """Throughput of the Winograd forward pass F(m x m, 3 x 3) (conv2d_forward_winograd)
+    on one GPU for a 3x3 stride-1 workload, with the forward line's timing.  `value` counts
+    the convolution's algorithmic FLOPs (as every forward line); the roofline is the
+    transformed-domain product (the (m+2)^2 channel GEMMs on the tensor cores) against the
+    tensor peak, and the step's bytes (x, V and M written and read, y) against HBM."""
+    import numpy as np
+    import torch
+    import cnn_convolution_conv2d_b200 as cb
+    from cnn_convolution_conv2d_b200 import build, workloads
+    import oracle
+
+    m = args.winograd
+    if (cfg.Kh, cfg.Kw, cfg.stride, cfg.dilation, cfg.groups) != (3, 3, 1, 1, 1):
+        raise SystemExit("--winograd needs a 3x3, stride-1, unit-dilation, ungrouped workload")
+    build.build()
+    cb.load()
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(0)
+    inp = workloads.make_inputs(cfg)
+    dt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+    x_host = torch.from_numpy(inp["x"]).to(dt)
+    if cfg.layout == "nhwc":
+        x_host = x_host.permute(0, 2, 3, 1).contiguous()
+    w = torch.from_numpy(inp["w"]).to(dt).to(device)
+    b = None if inp["b"] is None else torch.from_numpy(inp["b"]).to(dt).to(device)
+    layer = cb.WinogradConv2dB200(w, b, cfg.pad, m, cfg.layout)
+    y_shape = (cfg.N, cfg.Ho, cfg.Wo, cfg.C_out) if cfg.layout == "nhwc" else (cfg.N, cfg.C_out, cfg.Ho, cfg.Wo)
+    set_bytes = (x_host.numel() + math.prod(y_shape)) * x_host.element_size()
+    nsets = max(2, min(16, math.ceil(2 * L2_BYTES / set_bytes) + 1))
+    xs = [x_host.to(device) for _ in range(nsets)]
+    ys = [torch.empty(y_shape, dtype=dt, device=device) for _ in range(nsets)]
+    for i in range(max(args.warmup, 3)):
+        layer(xs[i % nsets], ys[i % nsets])
+    cb.conv2d_sync_status()
+    # accuracy of this run against the oracle on sampled outputs (the transforms' rounding)
+    idx = np.stack([np.random.default_rng(5).integers(0, n, 2048) for n in (cfg.N, cfg.C_out, cfg.Ho, cfg.Wo)], 1)
+    yy = ys[0].float()
+    got = (yy[tuple(torch.from_numpy(idx[:, i]).to(device) for i in (0, 2, 3, 1))] if cfg.layout == "nhwc"
+           else yy[tuple(torch.from_numpy(idx[:, i]).to(device) for i in range(4))]).cpu().numpy()
+    ref = oracle.conv2d_points(inp["x"], inp["w"], inp["b"], idx, 1, cfg.pad, 1, 1)
+    err = {"max_abs_over_max_ref": float(np.abs(got - ref).max() / np.abs(ref).max()),
+           "normwise_sampled": float(np.linalg.norm(got - ref) / np.linalg.norm(ref)), "points": 2048}
+    G = 1
+    for gsz in range(min(args.steps, 256), 0, -1):
+        if args.steps % gsz == 0:
+            G = gsz
+            break
+    reps = args.steps // G
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(G)]
+    for a, c in kev:
+        a.record()
+        c.record()
+    torch.cuda.synchronize()
+    launches0 = cb.conv2d_kernel_launch_count()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for i in range(G):
+            cb.conv2d_set_main_kernel_events(*kev[i])
+            layer(xs[i % nsets], ys[i % nsets])
+    cb.conv2d_set_main_kernel_events(None, None)
+    launches_per_rep = cb.conv2d_kernel_launch_count() - launches0
+    graph.replay()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(0)
+    clocks.start()
+    time.sleep(0.05)
+    stream = torch.cuda.current_stream()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    ev0.record(stream)
+    for _ in range(reps):
+        graph.replay()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    t1 = time.perf_counter()
+    clocks.stop()
+    cb.conv2d_sync_status()
+    elapsed = ev0.elapsed_time(ev1)
+    kernel_ms = statistics.fmean(a.elapsed_time(c) for a, c in kev)
+    a2 = (m + 2) ** 2
+    tiles = cfg.N * (-(-cfg.Ho // m)) * (-(-cfg.Wo // m))
+    e = elt_bytes(cfg)
+    cpg = -(-cfg.C_in // (16 // e)) * (16 // e)
+    gemm_flops = 2.0 * a2 * tiles * cpg * cfg.C_out
+    mult = 1 if cfg.dtype == "bf16" else TF32_PRODUCTS
+    peaks, peak_kind = load_peaks()
+    tpeak = peaks["bf16_tflops_sustained"] * (1 if cfg.dtype == "bf16" else TF32_PER_BF16)
+    v_bytes = tiles * a2 * cpg * e
+    m_bytes = tiles * a2 * cfg.C_out * 4
+    step_b = step_bytes(cfg) + 2 * v_bytes + 2 * m_bytes
+    line = {
+        "metric": "conv2d fwd TFLOP/s on 1 B200 and % of dense tensor (or HBM) roofline",
+        "value": flops(cfg) * args.steps / (elapsed * 1e-3) / 1e12, "unit": "TFLOP/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": elapsed / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic (seeded)",
+        "config": {"workload": workload_config(cfg, args, 1)["workload"], "path": f"Winograd F({m}x{m},3x3)",
+                   "l2": f"not resident: steps rotate over {nsets} sets",
+                   "launch": f"CUDA graphs of {G} steps x {reps} replays"},
+        "roofline": {"bound": "tensor", "achieved": mult * gemm_flops / (kernel_ms * 1e-3) / 1e12, "peak": tpeak,
+                     "unit": "TFLOP/s", "frac": mult * gemm_flops / (kernel_ms * 1e-3) / 1e12 / tpeak,
+                     "peak_source": f"{peak_kind} bf16 sustained" + ("" if mult == 1 else " x 0.5"),
+                     "kernel": "igemm_kernel on the transformed tiles ((m+2)^2 groups of 1x1)",
+                     "kernel_ms": kernel_ms, "gemm_flops_per_launch": gemm_flops, "traffic": None,
+                     "multiplies_vs_direct": a2 / (m * m * 9.0),
+                     "step_bytes": step_b, "step_hbm_frac": step_b / (elapsed / args.steps * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+        "accuracy_vs_oracle": err,
+        "gpu_launches": launches_per_rep * reps, "clocks": clocks.summary(t0, t1),
+    }
+    print(json.dumps(line), flush=True)
+    del graph
 
 
 def run_transpose(args, cfg):
@@ -630,10 +975,19 @@ def main(argv=None):
                     help="time the pages' formulation: explicit X_col in HBM, then the GEMM")
     ap.add_argument("--transpose", action="store_true",
                     help="time the standalone NCHW<->NHWC kernels on the workload's x and y instead")
+    ap.add_argument("--backward", choices=["data", "weight"],
+                    help="time one backward pass (input or weight gradient) of the workload instead")
+    ap.add_argument("--winograd", type=int, choices=[2, 4],
+                    help="time the Winograd F(m x m, 3 x 3) forward pass of a 3x3 stride-1 workload instead")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     from cnn_convolution_conv2d_b200 import workloads
+    if args.workload in workloads.CONFIGS3D:
+        if args.impl != "ours" or args.gpus != 1:
+            ap.error("3-D workloads run on one GPU through this library")
+        run_conv3d(args, workloads.CONFIGS3D[args.workload])
+        return
     cfg = workloads.CONFIGS[args.workload]
     rank, world, _ = dist_env()
     if world != args.gpus:
@@ -646,6 +1000,16 @@ def main(argv=None):
         if world != 1:
             ap.error("--transpose runs on one GPU")
         run_transpose(args, cfg)
+        return
+    if args.backward:
+        if world != 1:
+            ap.error("--backward runs on one GPU")
+        run_backward(args, cfg)
+        return
+    if args.winograd:
+        if world != 1:
+            ap.error("--winograd runs on one GPU")
+        run_winograd(args, cfg)
         return
     run_ours(args, cfg)
 

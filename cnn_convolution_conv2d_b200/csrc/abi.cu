@@ -135,6 +135,9 @@ int device_info(DeviceInfo **out) {
 // ------------------------------------------------------------------- plan ---
 struct Plan {
     int N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups;
+    int pad_w;      // column padding (= pad, the row padding, for every caller-facing entry)
+    bool vol;       // 3-D convolution: input depth D, filter depth Kd, output depth Do
+    int D, Kd, Do;
     bool f32;
     int elt;
     conv_layout_t layout;
@@ -143,6 +146,8 @@ struct Plan {
     int Cin_g, Cout_g, Cpg;  // per group the kernels see (merged groups: gm of the caller's)
     int gm;                  // caller's groups merged into one (see group_merge)
     bool gather;    // few input channels: the software-gather kernel reads x directly
+    bool gather_t;  // ... in its transposed form (gather_t.cu): bf16 NCHW, one output row per tile
+    int tpix;       // its pixels per tile (Wo rounded up to 16)
     bool vec_rows;  // ... with 16-byte row loads (NCHW, aligned rows, unit dilation)
     bool halo;      // ... from input rows staged in shared memory by TMA
     int R, BW, ME;  // halo rows per tile, staged row width, left zero margin (elements)
@@ -278,16 +283,35 @@ bool plan_depthwise(Plan *pp) {
     return true;
 }
 
+// A convolution the backward entry points run internally: its column padding may differ
+// from its row padding (the transposed convolution of a non-square filter) and either may
+// be negative (the window starts inside the image).  Internal convolutions never take the
+// few-channel gather kernel, whose weight images exist only for caller-packed weights.
+struct PadW {
+    int pad_w;
+    // when set: the product's fp32 results [split][M][C_out] go here (no bias, no
+    // split reduction) for a later pass to finish -- the Winograd path's output transform
+    float *partial_out = nullptr;
+};
+
+// The depth of a 3-D convolution: input depth D and filter depth Kd (stride, padding and
+// dilation are shared with the other two directions).
+struct Vol {
+    int D, Kd;
+};
+
 // Validates a problem and fills the plan.  `explicit_im2col` adds the X_col
 // buffer to the scratch layout.  `sms` = 0 plans without split (size queries
 // made before a device is known use the device's count when one is current).
 int make_plan(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stride, int pad,
               int dilation, int groups, conv_dtype_t dtype, conv_layout_t layout,
-              bool explicit_im2col, int sms, Plan *P, int pair_mode, bool allow_pair = true) {
+              bool explicit_im2col, int sms, Plan *P, int pair_mode, bool allow_pair = true,
+              const PadW *padw = nullptr, const Vol *vol = nullptr) {
+    const int pad_w = padw ? padw->pad_w : pad;
     if (N < 1 || C_in < 1 || H < 1 || W < 1 || C_out < 1 || Kh < 1 || Kw < 1)
         return fail(CONV_ERR_INVALID_ARG, "sizes must be >= 1 (N=%d C_in=%d H=%d W=%d C_out=%d Kh=%d Kw=%d)",
                     N, C_in, H, W, C_out, Kh, Kw);
-    if (stride < 1 || dilation < 1 || pad < 0 || groups < 1)
+    if (stride < 1 || dilation < 1 || (!padw && pad < 0) || groups < 1)
         return fail(CONV_ERR_INVALID_ARG, "need stride >= 1, dilation >= 1, pad >= 0, groups >= 1");
     if (C_in % groups != 0 || C_out % groups != 0)
         return fail(CONV_ERR_INVALID_ARG, "C_in (%d) and C_out (%d) must be divisible by groups (%d)",
@@ -298,23 +322,37 @@ int make_plan(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stri
         return fail(CONV_ERR_INVALID_ARG, "unknown layout %d", static_cast<int>(layout));
     Plan p{};
     p.N = N; p.C_in = C_in; p.H = H; p.W = W; p.C_out = C_out; p.Kh = Kh; p.Kw = Kw;
-    p.stride = stride; p.pad = pad; p.dilation = dilation; p.groups = groups;
+    p.stride = stride; p.pad = pad; p.pad_w = pad_w; p.dilation = dilation; p.groups = groups;
+    p.vol = vol != nullptr;
+    p.D = vol ? vol->D : 1;
+    p.Kd = vol ? vol->Kd : 1;
+    p.Do = 1;
+    if (vol && (p.D < 1 || p.Kd < 1)) return fail(CONV_ERR_INVALID_ARG, "D and Kd must be >= 1");
+    if (vol && explicit_im2col) return fail(CONV_ERR_UNSUPPORTED, "no explicit im2col for volumes");
+    if (vol && out_size(p.D, p.Kd, stride, pad, dilation, &p.Do))
+        return fail(CONV_ERR_INVALID_ARG, "empty output: the dilated kernel is deeper than the padded input");
     p.f32 = dtype == CONV_F32;
     p.elt = p.f32 ? 4 : 2;
     p.layout = layout;
-    if (out_size(H, Kh, stride, pad, dilation, &p.Ho) || out_size(W, Kw, stride, pad, dilation, &p.Wo))
+    if (out_size(H, Kh, stride, pad, dilation, &p.Ho) || out_size(W, Kw, stride, pad_w, dilation, &p.Wo))
         return fail(CONV_ERR_INVALID_ARG, "empty output: the dilated kernel is larger than the padded input");
-    p.M = static_cast<long long>(N) * p.Ho * p.Wo;
+    p.M = static_cast<long long>(N) * p.Do * p.Ho * p.Wo;
     // Limits of the hardware im2col addressing (traversal stride <= 8, bounding-box
     // corners in [-128, 127] for a 4-D tensor) and of 32-bit indexing.
     if (stride > 8) return fail(CONV_ERR_UNSUPPORTED, "stride %d > 8", stride);
-    if (pad > 127) return fail(CONV_ERR_UNSUPPORTED, "pad %d > 127", pad);
+    if (pad > 127 || pad_w > 127 || pad < -127 || pad_w < -127)
+        return fail(CONV_ERR_UNSUPPORTED, "pad %d > 127", pad > pad_w ? pad : pad_w);
     const long long up_h = pad - static_cast<long long>(Kh - 1) * dilation;
-    const long long up_w = pad - static_cast<long long>(Kw - 1) * dilation;
+    const long long up_w = pad_w - static_cast<long long>(Kw - 1) * dilation;
     if (up_h < -128 || up_w < -128)
         return fail(CONV_ERR_UNSUPPORTED, "dilation*(K-1) - pad exceeds 128");
+    if (vol) {  // corners of a 5-D im2col bounding box lie in [-16, 15]
+        const long long up_d = pad - static_cast<long long>(p.Kd - 1) * dilation;
+        if (pad > 16 || up_h < -16 || up_w < -16 || up_d < -16 || up_h > 15 || up_w > 15 || up_d > 15)
+            return fail(CONV_ERR_UNSUPPORTED, "3-D: pad and pad - dilation*(K-1) must lie in [-16, 15]");
+    }
     if (p.M >= (1LL << 31) - 256) return fail(CONV_ERR_UNSUPPORTED, "N*Ho*Wo too large");
-    if (static_cast<long long>(N) * H * W * C_in >= (1LL << 40))
+    if (static_cast<long long>(N) * p.D * H * W * C_in >= (1LL << 40))
         return fail(CONV_ERR_UNSUPPORTED, "input too large");
 
     p.Cin_g = C_in / groups;
@@ -322,7 +360,7 @@ int make_plan(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stri
     const int align = 16 / p.elt;
     p.Cpg = round_up(p.Cin_g, align);
     p.dw = false;
-    if (!explicit_im2col && groups == C_in && C_out == C_in && plan_depthwise(&p)) {
+    if (!vol && !explicit_im2col && groups == C_in && C_out == C_in && plan_depthwise(&p)) {
         *P = p;
         return CONV_OK;
     }
@@ -344,7 +382,7 @@ int make_plan(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stri
     p.Kc = p.vec_rows ? C_in * Kh * per16 : C_in * Kh * Kw;
     p.Kpad = round_up(p.Kc, 32 / p.elt);
     p.gather = false;
-    if (!explicit_im2col && groups == 1 && C_in * p.elt < 32 && p.Kpad <= 256 &&
+    if (!padw && !vol && !explicit_im2col && groups == 1 && C_in * p.elt < 32 && p.Kpad <= 256 &&
         C_out <= (p.f32 ? 128 : 256)) {
         const int bn = round_up(C_out, 16);
         // Tensor memory (512 columns): two accumulators of bn columns, then A slots
@@ -391,13 +429,35 @@ int make_plan(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stri
         const int order = p.vec_rows ? 1 : 0;
         if (slots >= 2 && smem <= kSmemBudget && gi.kpad[order] == p.Kpad) {
             p.gather = true;
+            // Transposed form: output channels on the lanes, one output row per tile,
+            // channel rows stored straight into NCHW y.  Needs the row-vector order,
+            // whole 16-byte stores per row (Wo % 8 == 0) and the row's staged input box.
+            p.gather_t = false;
+            if (!p.f32 && p.vec_rows && p.Wo % 8 == 0 && p.Wo <= 256 && C_out <= 128 && pad <= per16 &&
+                C_in * Kh <= 32) {
+                const int iw0_max = (p.Wo - 1) * stride - pad;
+                const int BW = round_up(iw0_max + per16 + per16 + 2, per16);
+                const int tpix = round_up(p.Wo, 16);
+                const size_t hb = static_cast<size_t>(C_in) * Kh * BW * p.elt;
+                const size_t tsmem = gather_t_smem_bytes(p.Kpad, tpix, hb);
+                if (BW <= 256 && W <= BW && Kh <= 256 && tsmem <= kSmemBudget) {
+                    p.gather_t = true;
+                    p.halo = true;
+                    p.R = Kh;
+                    p.BW = BW;
+                    p.ME = per16;
+                    p.tpix = tpix;
+                    p.tma_out = false;
+                    smem = tsmem;
+                }
+            }
             p.w_image_off = gi.off[order];
             p.BN = bn;
             p.stages = slots;
             p.acols = acols;
             // at least 120 KB, so that one CTA (holding all tensor memory) runs per SM
             p.smem = smem > 120 * 1024 ? smem : 120 * 1024;
-            p.n_mtiles = static_cast<int>((p.M + 127) / 128);
+            p.n_mtiles = p.gather_t ? N * p.Ho : static_cast<int>((p.M + 127) / 128);
             p.n_ntiles = 1;
             p.splits = 1;
             p.units = p.n_mtiles;
@@ -411,14 +471,14 @@ int make_plan(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stri
     // A 1x1 filter at stride 1 without padding makes the im2col matrix the
     // channels-last input itself (one row per pixel), so the tensor-core kernel reads
     // it with plain tiled loads, which stream far faster than im2col-mode loads.
-    p.direct_a = !explicit_im2col && Kh == 1 && Kw == 1 && stride == 1 && pad == 0;
+    p.direct_a = !explicit_im2col && p.Kd == 1 && Kh == 1 && Kw == 1 && stride == 1 && pad == 0 && pad_w == 0;
     const int row_bytes = p.Cpg * p.elt;
     p.cb = row_bytes % 128 == 0 ? 128 : row_bytes % 64 == 0 ? 64 : row_bytes % 32 == 0 ? 32 : 16;
     const int cap = p.f32 ? 128 : 256;
     const int nt = (p.Cout_g + cap - 1) / cap;
     p.BN = round_up((p.Cout_g + nt - 1) / nt, 16);
     p.n_ntiles = (p.Cout_g + p.BN - 1) / p.BN;
-    p.taps = Kh * Kw;
+    p.taps = p.Kd * Kh * Kw;
     p.nCB = row_bytes / p.cb;
     p.planes = p.taps * p.nCB;
     const int np = 128 / p.cb;
@@ -450,7 +510,7 @@ int make_plan(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stri
     p.units = static_cast<int>(base * p.splits);
     // bf16 channels-last output leaves through shared memory and TMA stores when
     // every 32-column block of a tile lies inside its group's columns.
-    p.tma_out = !p.f32 && layout == CONV_NHWC && p.splits == 1 &&
+    p.tma_out = !p.f32 && layout == CONV_NHWC && p.splits == 1 && !(padw && padw->partial_out) &&
                 p.BN % 32 == 0 && p.Cout_g % p.BN == 0 && (C_out * p.elt) % 16 == 0;
     const int bn_local = p.pair ? p.BN / 2 : p.BN;  // B rows staged per CTA
     const size_t stage = static_cast<size_t>(128 + bn_local) * 128 * (p.f32 ? 2 : 1);
@@ -462,7 +522,7 @@ int make_plan(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stri
 
     size_t off = 0;
     p.off_xcopy = off;
-    if (p.xcopy) off = align_up(off + static_cast<size_t>(N) * H * W * p.groups * p.Cpg * p.elt, 256);
+    if (p.xcopy) off = align_up(off + static_cast<size_t>(N) * p.D * H * W * p.groups * p.Cpg * p.elt, 256);
     p.off_partial = off;
     if (p.splits > 1) off = align_up(off + static_cast<size_t>(p.splits) * p.M * C_out * 4, 256);
     p.off_xcol = off;
@@ -493,14 +553,34 @@ int encode_a_im2col(const Plan &p, const void *x_nhwc, CUtensorMap *map) {
     cuuint64_t dims[4] = {ctot, static_cast<cuuint64_t>(p.W), static_cast<cuuint64_t>(p.H),
                           static_cast<cuuint64_t>(p.N)};
     cuuint64_t strides[3] = {ctot * p.elt, ctot * p.elt * p.W, ctot * p.elt * p.W * p.H};
-    int lower[2] = {-p.pad, -p.pad};  // (w, h)
-    int upper[2] = {p.pad - (p.Kw - 1) * p.dilation, p.pad - (p.Kh - 1) * p.dilation};
+    int lower[2] = {-p.pad_w, -p.pad};  // (w, h)
+    int upper[2] = {p.pad_w - (p.Kw - 1) * p.dilation, p.pad - (p.Kh - 1) * p.dilation};
     cuuint32_t estr[4] = {1, static_cast<cuuint32_t>(p.stride), static_cast<cuuint32_t>(p.stride), 1};
     CUresult r = g_encode_im2col(map, tma_type(p), 4, const_cast<void *>(x_nhwc), dims, strides, lower,
                                  upper, static_cast<cuuint32_t>(p.cb / p.elt), 128, estr,
                                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_for(p.cb),
                                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(CONV_ERR_CUDA, "cuTensorMapEncodeIm2col failed (%d)", static_cast<int>(r));
+    return CONV_OK;
+}
+
+// A operand, implicit, volumes: 5-D im2col view of the channels-last input (c, w, h, d, n).
+int encode_a_im2col_5d(const Plan &p, const void *x_ndhwc, CUtensorMap *map) {
+    const cuuint64_t ctot = static_cast<cuuint64_t>(p.groups) * p.Cpg;
+    cuuint64_t dims[5] = {ctot, static_cast<cuuint64_t>(p.W), static_cast<cuuint64_t>(p.H),
+                          static_cast<cuuint64_t>(p.D), static_cast<cuuint64_t>(p.N)};
+    cuuint64_t strides[4] = {ctot * p.elt, ctot * p.elt * p.W, ctot * p.elt * p.W * p.H,
+                             ctot * p.elt * p.W * p.H * p.D};
+    int lower[3] = {-p.pad_w, -p.pad, -p.pad};  // (w, h, d)
+    int upper[3] = {p.pad_w - (p.Kw - 1) * p.dilation, p.pad - (p.Kh - 1) * p.dilation,
+                    p.pad - (p.Kd - 1) * p.dilation};
+    cuuint32_t estr[5] = {1, static_cast<cuuint32_t>(p.stride), static_cast<cuuint32_t>(p.stride),
+                          static_cast<cuuint32_t>(p.stride), 1};
+    CUresult r = g_encode_im2col(map, tma_type(p), 5, const_cast<void *>(x_ndhwc), dims, strides, lower, upper,
+                                 static_cast<cuuint32_t>(p.cb / p.elt), 128, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                 swizzle_for(p.cb), CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(CONV_ERR_CUDA, "cuTensorMapEncodeIm2col (5-D) failed (%d)", static_cast<int>(r));
     return CONV_OK;
 }
 
@@ -592,6 +672,11 @@ int gather_impl(const Plan &p, const void *x, const void *w_packed, const void *
             return fail(CONV_ERR_CUDA, "cuTensorMapEncodeTiled (input rows) failed (%d)", static_cast<int>(r));
     }
     g.tmem_cols = 512;  // accumulators and A slots
+    if (p.gather_t) {
+        g.tpix = p.tpix;
+        g.tmem_cols = 32;
+        while (g.tmem_cols < static_cast<uint32_t>(2 * p.tpix)) g.tmem_cols <<= 1;
+    }
     g.cw = p.cw;
     g.tma_out = p.tma_out ? 1 : 0;
     if (p.tma_out) {
@@ -618,7 +703,7 @@ int gather_impl(const Plan &p, const void *x, const void *w_packed, const void *
     int st;
     cudaEvent_t ev_start = g_main_start, ev_stop = g_main_stop;
     if (ev_start && ev_stop && (st = record_event(ev_start, stream)) != CONV_OK) return st;
-    cudaError_t e = launch_gather(g, p.f32, grid, p.smem, stream);
+    cudaError_t e = p.gather_t ? launch_gather_t(g, grid, p.smem, stream) : launch_gather(g, p.f32, grid, p.smem, stream);
     if ((st = check_launch(e, "gather tensor-core product")) != CONV_OK) return st;
     if (ev_start && ev_stop && (st = record_event(ev_stop, stream)) != CONV_OK) return st;
     return ok();
@@ -655,7 +740,7 @@ int dw_impl(const Plan &p, const void *x, const void *w_packed, const void *bias
     d.bias = bias;
     d.y = y;
     d.N = p.N; d.C = p.C_in; d.Ho = p.Ho; d.Wo = p.Wo; d.Kh = p.Kh; d.Kw = p.Kw;
-    d.stride = p.stride; d.pad = p.pad; d.dilation = p.dilation;
+    d.stride = p.stride; d.pad = p.pad; d.pad_w = p.pad_w; d.dilation = p.dilation;
     d.Cpg = p.Cpg;
     d.TH = p.TH; d.TW = p.TW; d.IH = p.IH; d.IW = p.IW;
     d.n_th = p.n_th; d.n_tw = p.n_tw; d.units = p.units; d.stages = p.stages;
@@ -677,18 +762,18 @@ int dw_impl(const Plan &p, const void *x, const void *w_packed, const void *bias
 
 // Resident two-CTA clusters of the pair kernel for one configuration, asked of the
 // runtime once per configuration and device and remembered.
-int pair_cluster_limit(int cb, bool im2col, size_t smem) {
+int pair_cluster_limit(int cb, bool im2col, size_t smem, bool vol = false) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-    const long long key = ((static_cast<long long>(dev) * 256 + cb) * 2 + (im2col ? 1 : 0)) * 1048576 +
-                          static_cast<long long>(smem);
+    const long long key = (((static_cast<long long>(dev) * 256 + cb) * 2 + (im2col ? 1 : 0)) * 2 + (vol ? 1 : 0)) *
+                              1048576 + static_cast<long long>(smem);
     {
         std::lock_guard<std::mutex> lock(g_mutex);
         auto it = g_pair_clusters.find(key);
         if (it != g_pair_clusters.end()) return it->second;
     }
     int n = 0;
-    if (igemm_pair_max_clusters(cb, im2col, smem, &n) != cudaSuccess) {
+    if (igemm_pair_max_clusters(cb, im2col, smem, &n, vol) != cudaSuccess) {
         (void)cudaGetLastError();
         n = 0;
     }
@@ -702,17 +787,18 @@ int pair_cluster_limit(int cb, bool im2col, size_t smem) {
 // Size queries and the forward pass share it, so that they always agree.
 int device_plan(bool explicit_im2col, int N, int C_in, int H, int W, int C_out, int Kh, int Kw,
                 int stride, int pad, int dilation, int groups, conv_dtype_t dtype,
-                conv_layout_t layout, DeviceInfo *dev, const Settings &cfg, Plan *p) {
+                conv_layout_t layout, DeviceInfo *dev, const Settings &cfg, Plan *p,
+                const PadW *padw = nullptr, const Vol *vol = nullptr) {
     int st = make_plan(N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype, layout,
-                       explicit_im2col, dev ? dev->sms : 0, p, cfg.pair_mode);
+                       explicit_im2col, dev ? dev->sms : 0, p, cfg.pair_mode, true, padw, vol);
     if (st != CONV_OK) return st;
     p->pair_clusters = 0;
     if (p->pair && dev) {
         const bool a_im2col = !(explicit_im2col || p->direct_a);
-        p->pair_clusters = pair_cluster_limit(p->cb, a_im2col, p->smem);
+        p->pair_clusters = pair_cluster_limit(p->cb, a_im2col, p->smem, p->vol);
         if (p->pair_clusters < 1)  // the device cannot co-schedule the pair kernel: single CTAs
             return make_plan(N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype, layout,
-                             explicit_im2col, dev->sms, p, cfg.pair_mode, false);
+                             explicit_im2col, dev->sms, p, cfg.pair_mode, false, padw, vol);
     }
     return CONV_OK;
 }
@@ -730,18 +816,19 @@ DeviceInfo *current_device_or_null() {
 int forward_impl(bool explicit_im2col, const void *x, const void *w_packed, const void *bias, void *y,
                  int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stride, int pad,
                  int dilation, int groups, conv_dtype_t dtype, conv_layout_t layout, void *workspace,
-                 size_t workspace_bytes, cudaStream_t stream) {
+                 size_t workspace_bytes, cudaStream_t stream, const PadW *padw = nullptr,
+                 const Vol *vol = nullptr) {
     const Settings cfg = settings_now();
     DeviceInfo *dev = nullptr;
     Plan p;
     int st = make_plan(N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype, layout,
-                       explicit_im2col, 0, &p, cfg.pair_mode);
+                       explicit_im2col, 0, &p, cfg.pair_mode, true, padw, vol);
     if (st != CONV_OK) return st;
     if (!x || !w_packed || !y) return fail(CONV_ERR_INVALID_ARG, "x, w_packed and y must not be NULL");
     st = device_info(&dev);
     if (st != CONV_OK) return st;
     st = device_plan(explicit_im2col, N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype,
-                     layout, dev, cfg, &p);
+                     layout, dev, cfg, &p, padw, vol);
     if (st != CONV_OK) return st;
     const bool a_im2col = !(explicit_im2col || p.direct_a);
     const int pair_clusters = p.pair_clusters;
@@ -763,15 +850,19 @@ int forward_impl(bool explicit_im2col, const void *x, const void *w_packed, cons
     std::memset(&kp, 0, sizeof(kp));
     st = explicit_im2col ? encode_a_xcol(p, xcol, &kp.tmap_a)
          : p.direct_a    ? encode_a_xcol(p, x_nhwc, &kp.tmap_a)
+         : p.vol         ? encode_a_im2col_5d(p, x_nhwc, &kp.tmap_a)
                          : encode_a_im2col(p, x_nhwc, &kp.tmap_a);
     if (st != CONV_OK) return st;
     st = encode_b(p, w_packed, &kp.tmap_b);
     if (st != CONV_OK) return st;
     kp.M = static_cast<int>(p.M);
-    kp.HoWo = p.Ho * p.Wo;
+    kp.HoWo = p.Do * p.Ho * p.Wo;
+    kp.HoWo2 = p.Ho * p.Wo;
+    kp.Kh = Kh;
     kp.Wo = p.Wo;
     kp.stride = stride;
-    kp.pad = pad;
+    kp.pad = p.pad;
+    kp.pad_w = p.pad_w;
     kp.dilation = dilation;
     kp.Kw = Kw;
     kp.taps = p.taps;
@@ -795,8 +886,9 @@ int forward_impl(bool explicit_im2col, const void *x, const void *w_packed, cons
     while (cols < static_cast<uint32_t>(2 * p.BN)) cols <<= 1;
     kp.tmem_cols = cols;
     kp.bias = bias;
-    if (p.splits > 1) {
-        kp.y = ws + p.off_partial;
+    const bool external_partial = padw && padw->partial_out;
+    if (p.splits > 1 || external_partial) {
+        kp.y = external_partial ? static_cast<void *>(padw->partial_out) : static_cast<void *>(ws + p.off_partial);
         kp.out_mode = kOutPartial;
         kp.vec_ok = (C_out % 4 == 0 && p.Cout_g % 4 == 0) ? 1 : 0;
     } else {
@@ -823,8 +915,9 @@ int forward_impl(bool explicit_im2col, const void *x, const void *w_packed, cons
 
     if (p.xcopy) {
         cudaError_t e = layout == CONV_NCHW
-                            ? launch_nchw_to_nhwc(x, ws + p.off_xcopy, N, C_in, H, W, p.groups, p.Cpg, p.elt, stream)
-                            : launch_nhwc_pad(x, ws + p.off_xcopy, N, C_in, H, W, p.groups, p.Cpg, p.elt, stream);
+                            ? launch_nchw_to_nhwc(x, ws + p.off_xcopy, N, C_in, p.D * H, W, p.groups, p.Cpg, p.elt,
+                                                  stream)
+                            : launch_nhwc_pad(x, ws + p.off_xcopy, N, C_in, p.D * H, W, p.groups, p.Cpg, p.elt, stream);
         if ((st = check_launch(e, "channels-last copy")) != CONV_OK) return st;
     }
     if (explicit_im2col) {
@@ -837,12 +930,12 @@ int forward_impl(bool explicit_im2col, const void *x, const void *w_packed, cons
                             : (p.units < dev->sms ? p.units : dev->sms);
     cudaEvent_t ev_start = g_main_start, ev_stop = g_main_stop;
     if (ev_start && ev_stop && (st = record_event(ev_start, stream)) != CONV_OK) return st;
-    cudaError_t e = launch_igemm(kp, p.f32, p.cb, a_im2col, p.pair, grid, p.smem, stream);
+    cudaError_t e = launch_igemm(kp, p.f32, p.cb, a_im2col, p.pair, grid, p.smem, stream, p.vol);
     if ((st = check_launch(e, "tensor-core product")) != CONV_OK) return st;
     if (ev_start && ev_stop && (st = record_event(ev_stop, stream)) != CONV_OK) return st;
-    if (p.splits > 1) {
+    if (p.splits > 1 && !external_partial) {
         e = launch_splitk_reduce(reinterpret_cast<const float *>(ws + p.off_partial), bias, y,
-                                 static_cast<int>(p.M), C_out, p.Ho * p.Wo, p.splits,
+                                 static_cast<int>(p.M), C_out, p.Do * p.Ho * p.Wo, p.splits,
                                  layout == CONV_NCHW ? kOutNCHW : kOutNHWC, p.f32, stream);
         if ((st = check_launch(e, "split reduction")) != CONV_OK) return st;
     }
@@ -872,7 +965,7 @@ int describe_impl(bool explicit_im2col, int N, int C_in, int H, int W, int C_out
     }
     if (st != CONV_OK) return st;
     const char *a_load = p.dw ? "tile" : p.gather ? "gather" : explicit_im2col ? "xcol" : p.direct_a ? "tiled_x" : "im2col";
-    const char *kernel = p.dw ? "depthwise" : p.gather ? "gather" : "igemm";
+    const char *kernel = p.dw ? "depthwise" : p.gather_t ? "gather_t" : p.gather ? "gather" : "igemm";
     const int n = std::snprintf(
         buf, buflen,
         "{\"kernel\": \"%s\", \"pair\": %d, \"a_load\": \"%s\", \"BN\": %d, \"cb\": %d, "
@@ -888,16 +981,16 @@ int describe_impl(bool explicit_im2col, int N, int C_in, int H, int W, int C_out
 
 int workspace_impl(bool explicit_im2col, int N, int C_in, int H, int W, int C_out, int Kh, int Kw,
                    int stride, int pad, int dilation, int groups, conv_dtype_t dtype,
-                   conv_layout_t layout, size_t *bytes) {
+                   conv_layout_t layout, size_t *bytes, const PadW *padw = nullptr, const Vol *vol = nullptr) {
     if (!bytes) return fail(CONV_ERR_INVALID_ARG, "bytes must not be NULL");
     const Settings cfg = settings_now();
     Plan p;
     int st = make_plan(N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype, layout,
-                       explicit_im2col, 0, &p, cfg.pair_mode);
+                       explicit_im2col, 0, &p, cfg.pair_mode, true, padw, vol);
     if (st != CONV_OK) return st;
     // with no usable device: sized without reduction splits or CTA pairs
     st = device_plan(explicit_im2col, N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype,
-                     layout, current_device_or_null(), cfg, &p);
+                     layout, current_device_or_null(), cfg, &p, padw, vol);
     if (st != CONV_OK) return st;
     *bytes = p.ws_total;
     return ok();
@@ -923,6 +1016,378 @@ int noalloc_scratch(void **out) {
     return CONV_OK;
 }
 
+
+// ----------------------------------------------------------------- backward ---
+// Weight gradient plan: the tensor-core kernel (wgrad.cu) when a group has at least 32
+// bytes of input channels, else the CUDA-core kernel (depthwise and other few-channel
+// groups).  Scratch: [x copy][dy copy][fp32 partial sums][bias-gradient partials].
+struct WgPlan {
+    Plan f;                       // the forward problem: validation, Ho, Wo, M
+    bool tc;                      // tensor-core kernel
+    int Cin_g, Cout_g, Cpg, dy_cpg, BN, n_ctiles, n_otiles, taps, kstages, splits, units, stages;
+    bool xcopy, dycopy;
+    size_t smem, off_xcopy, off_dycopy, off_ws, off_db, ws_total;
+    int db_partials;
+};
+
+int wgrad_plan(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stride, int pad, int dilation,
+               int groups, conv_dtype_t dtype, conv_layout_t layout, bool want_db, int sms, WgPlan *out) {
+    WgPlan w{};
+    int st = make_plan(N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype, layout, false, 0,
+                       &w.f, 2);
+    if (st != CONV_OK) return st;
+    const Plan &f = w.f;
+    const int elt = f.elt;
+    w.Cin_g = C_in / groups;
+    w.Cout_g = C_out / groups;
+    w.taps = Kh * Kw;
+    w.tc = w.Cin_g * elt >= 32;
+    const int align = 16 / elt;
+    size_t off = 0;
+    if (w.tc) {
+        const int cc = 128 / elt;
+        w.Cpg = round_up(w.Cin_g, cc);
+        w.dy_cpg = round_up(w.Cout_g, align);
+        w.xcopy = layout == CONV_NCHW || w.Cpg != w.Cin_g;
+        w.dycopy = layout == CONV_NCHW || w.dy_cpg != w.Cout_g;
+        const int cap = f.f32 ? 128 : 256;
+        for (w.BN = cap; w.BN > cc && w.Cpg % w.BN != 0; w.BN -= cc) {
+        }
+        w.n_ctiles = w.Cpg / w.BN;
+        w.n_otiles = (w.Cout_g + 127) / 128;
+        const int pk = wgrad_pixels_per_stage(f.f32);
+        const long long kst = (f.M + pk - 1) / pk;
+        const long long base = static_cast<long long>(w.n_otiles) * groups * w.taps * w.n_ctiles;
+        if (base * 64 >= (1LL << 31) || kst >= (1LL << 30)) return fail(CONV_ERR_UNSUPPORTED, "too many tiles");
+        w.kstages = static_cast<int>(kst);
+        w.splits = 1;
+        if (sms > 0 && base < sms) {
+            long long sp = sms / base;
+            sp = sp < w.kstages / 4 ? sp : w.kstages / 4;
+            sp = sp < 64 ? sp : 64;
+            w.splits = sp > 1 ? static_cast<int>(sp) : 1;
+        }
+        w.units = static_cast<int>(base * w.splits);
+        const size_t fixed = wgrad_smem_bytes(f.f32, w.BN, 0);
+        const size_t stage = wgrad_smem_bytes(f.f32, w.BN, 1) - fixed;
+        int stages = static_cast<int>((kSmemBudget - fixed) / stage);
+        w.stages = stages > wgrad_max_stages() ? wgrad_max_stages() : stages;
+        if (w.stages < 2) return fail(CONV_ERR_UNSUPPORTED, "weight-gradient tile does not fit in shared memory");
+        w.smem = wgrad_smem_bytes(f.f32, w.BN, w.stages);
+    } else {
+        // CUDA cores: channels-last copies without padding, splits over rows of pixels
+        w.Cpg = w.Cin_g;
+        w.dy_cpg = w.Cout_g;
+        w.xcopy = w.dycopy = layout == CONV_NCHW;
+        const long long elems = static_cast<long long>(C_out) * w.taps * w.Cin_g;
+        const long long rows = static_cast<long long>(N) * f.Ho;
+        long long sp = (148LL * 1024 + elems - 1) / elems;
+        sp = sp < rows ? sp : rows;
+        sp = sp < 256 ? sp : 256;
+        w.splits = sp > 1 ? static_cast<int>(sp) : 1;
+    }
+    w.off_xcopy = off;
+    if (w.xcopy) off = align_up(off + static_cast<size_t>(N) * H * W * groups * w.Cpg * elt, 256);
+    w.off_dycopy = off;
+    if (w.dycopy) off = align_up(off + static_cast<size_t>(f.M) * groups * w.dy_cpg * elt, 256);
+    w.off_ws = off;
+    off = align_up(off + static_cast<size_t>(w.splits) * C_out * w.taps * w.Cpg * 4, 256);
+    w.off_db = off;
+    w.db_partials = want_db ? bias_grad_partials(f.M, C_out, N, layout == CONV_NCHW) : 0;
+    if (want_db) off = align_up(off + static_cast<size_t>(w.db_partials) * C_out * 4, 256);
+    w.ws_total = off;
+    *out = w;
+    return CONV_OK;
+}
+
+// Copies x or dy into channels-last with `cpg` channels per group (zero padding) when the
+// plan asks for it; returns the tensor the kernels read.
+int to_channels_last(bool copy, const void *src, uint8_t *dst, int N, int C, int H, int W, int groups, int cpg,
+                     const Plan &f, cudaStream_t stream, const void **out) {
+    *out = src;
+    if (!copy) return CONV_OK;
+    cudaError_t e = f.layout == CONV_NCHW ? launch_nchw_to_nhwc(src, dst, N, C, H, W, groups, cpg, f.elt, stream)
+                                          : launch_nhwc_pad(src, dst, N, C, H, W, groups, cpg, f.elt, stream);
+    int st = check_launch(e, "channels-last copy");
+    if (st != CONV_OK) return st;
+    *out = dst;
+    return CONV_OK;
+}
+
+int bias_grad_impl(const Plan &f, const void *dy, void *db, float *partials, cudaStream_t stream) {
+    return check_launch(launch_bias_grad(dy, partials, db, f.N, f.C_out, static_cast<long long>(f.Ho) * f.Wo,
+                                         f.layout == CONV_NCHW, f.f32, stream),
+                        "bias gradient");
+}
+
+int backward_weight_impl(const void *x, const void *dy, void *dw, void *db, int N, int C_in, int H, int W,
+                         int C_out, int Kh, int Kw, int stride, int pad, int dilation, int groups,
+                         conv_dtype_t dtype, conv_layout_t layout, void *workspace, size_t workspace_bytes,
+                         cudaStream_t stream) {
+    const Settings cfg = settings_now();
+    WgPlan w;
+    int st = wgrad_plan(N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype, layout, db != nullptr,
+                        0, &w);
+    if (st != CONV_OK) return st;
+    if (!x || !dy || !dw) return fail(CONV_ERR_INVALID_ARG, "x, dy and dw must not be NULL");
+    DeviceInfo *dev = nullptr;
+    if ((st = device_info(&dev)) != CONV_OK) return st;
+    st = wgrad_plan(N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype, layout, db != nullptr,
+                    dev->sms, &w);
+    if (st != CONV_OK) return st;
+    if (!workspace || workspace_bytes < w.ws_total)
+        return fail(CONV_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", w.ws_total,
+                    workspace ? workspace_bytes : static_cast<size_t>(0));
+    if (!aligned16(x) || !aligned16(dy) || !aligned16(dw) || (db && !aligned16(db)) || !aligned16(workspace))
+        return fail(CONV_ERR_UNSUPPORTED, "device pointers must be 16-byte aligned");
+    const Plan &f = w.f;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    float *partial = reinterpret_cast<float *>(ws + w.off_ws);
+    if (db && (st = bias_grad_impl(f, dy, db, reinterpret_cast<float *>(ws + w.off_db), stream)) != CONV_OK)
+        return st;
+    const void *xl = nullptr, *dyl = nullptr;
+    if ((st = to_channels_last(w.xcopy, x, ws + w.off_xcopy, N, C_in, H, W, w.tc ? groups : 1,
+                               w.tc ? w.Cpg : C_in, f, stream, &xl)) != CONV_OK)
+        return st;
+    if ((st = to_channels_last(w.dycopy, dy, ws + w.off_dycopy, N, C_out, f.Ho, f.Wo, w.tc ? groups : 1,
+                               w.tc ? w.dy_cpg : C_out, f, stream, &dyl)) != CONV_OK)
+        return st;
+    cudaEvent_t ev_start = g_main_start, ev_stop = g_main_stop;
+    if (!w.tc) {
+        if (ev_start && ev_stop && (st = record_event(ev_start, stream)) != CONV_OK) return st;
+        if ((st = check_launch(launch_wgrad_direct(xl, dyl, partial, N, C_in, H, W, C_out, f.Ho, f.Wo, Kh, Kw, stride,
+                                                   pad, dilation, groups, w.splits, f.f32, stream),
+                               "weight gradient (CUDA cores)")) != CONV_OK)
+            return st;
+        if (ev_start && ev_stop && (st = record_event(ev_stop, stream)) != CONV_OK) return st;
+    } else {
+        WgradParams k;
+        std::memset(&k, 0, sizeof(k));
+        const int elt = f.elt, cc = 128 / elt, pk = wgrad_pixels_per_stage(f.f32);
+        {
+            cuuint64_t dims[2] = {static_cast<cuuint64_t>(groups) * w.dy_cpg, static_cast<cuuint64_t>(f.M)};
+            cuuint64_t strides[1] = {static_cast<cuuint64_t>(groups) * w.dy_cpg * elt};
+            cuuint32_t box[2] = {static_cast<cuuint32_t>(cc), static_cast<cuuint32_t>(pk)};
+            cuuint32_t estr[2] = {1, 1};
+            CUresult r = g_encode_tiled(&k.tmap_dy, tma_type(f), 2, const_cast<void *>(dyl), dims, strides, box, estr,
+                                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+            if (r != CUDA_SUCCESS)
+                return fail(CONV_ERR_CUDA, "cuTensorMapEncodeTiled (output gradient) failed (%d)", static_cast<int>(r));
+        }
+        {
+            const cuuint64_t ctot = static_cast<cuuint64_t>(groups) * w.Cpg;
+            cuuint64_t dims[4] = {ctot, static_cast<cuuint64_t>(W), static_cast<cuuint64_t>(H),
+                                  static_cast<cuuint64_t>(N)};
+            cuuint64_t strides[3] = {ctot * elt, ctot * elt * W, ctot * elt * W * H};
+            int lower[2] = {-pad, -pad};
+            int upper[2] = {pad - (Kw - 1) * dilation, pad - (Kh - 1) * dilation};
+            cuuint32_t estr[4] = {1, static_cast<cuuint32_t>(stride), static_cast<cuuint32_t>(stride), 1};
+            CUresult r = g_encode_im2col(&k.tmap_x, tma_type(f), 4, const_cast<void *>(xl), dims, strides, lower, upper,
+                                         static_cast<cuuint32_t>(cc), static_cast<cuuint32_t>(pk), estr,
+                                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+            if (r != CUDA_SUCCESS)
+                return fail(CONV_ERR_CUDA, "cuTensorMapEncodeIm2col (input) failed (%d)", static_cast<int>(r));
+        }
+        k.ws = partial;
+        k.M = static_cast<int>(f.M);
+        k.HoWo = f.Ho * f.Wo;
+        k.Wo = f.Wo;
+        k.stride = stride;
+        k.pad = pad;
+        k.dilation = dilation;
+        k.Kw = Kw;
+        k.taps = w.taps;
+        k.Cpg = w.Cpg;
+        k.dy_cpg = w.dy_cpg;
+        k.Cout = C_out;
+        k.Cout_g = w.Cout_g;
+        k.groups = groups;
+        k.BN = w.BN;
+        k.n_ctiles = w.n_ctiles;
+        k.n_otiles = w.n_otiles;
+        k.kstages = w.kstages;
+        k.splits = w.splits;
+        k.units = w.units;
+        k.stages = w.stages;
+        k.chunk_stages = f.f32 ? 4 : 0;
+        k.tmem_cols = 2 * w.BN <= 256 ? (2 * w.BN <= 128 ? 128 : 256) : 512;
+        k.status = dev->status;
+        k.timeout_ns = cfg.timeout_ns;
+        k.starve = cfg.starve;
+        const int grid = w.units < dev->sms ? w.units : dev->sms;
+        if (ev_start && ev_stop && (st = record_event(ev_start, stream)) != CONV_OK) return st;
+        if ((st = check_launch(launch_wgrad(k, f.f32, grid, w.smem, stream), "weight gradient")) != CONV_OK) return st;
+        if (ev_start && ev_stop && (st = record_event(ev_stop, stream)) != CONV_OK) return st;
+    }
+    if ((st = check_launch(launch_wgrad_reduce(partial, dw, C_out, w.Cin_g, w.taps, w.Cpg, w.splits, f.f32, stream),
+                           "weight-gradient reduction")) != CONV_OK)
+        return st;
+    return ok();
+}
+
+// Input gradient: the transposed convolution, run as a forward convolution of dy (or of
+// dy with s-1 zeros inserted between its rows and columns when stride s > 1) with the
+// spatially flipped, channel-exchanged kernel, stride 1 and padding d*(K-1) - pad.
+struct DgradShape {
+    int Hi, Wi;          // extent of the tensor the inner convolution reads
+    int pad_h, pad_w;    // its padding
+    bool zeros;          // dy goes through zero insertion first
+    size_t zbytes;       // bytes of the zero-inserted dy
+};
+
+int dgrad_shape(const Plan &f, DgradShape *d) {
+    d->pad_h = f.dilation * (f.Kh - 1) - f.pad;
+    d->pad_w = f.dilation * (f.Kw - 1) - f.pad;
+    d->zeros = f.stride > 1;
+    if (d->zeros) {
+        d->Hi = f.H - f.dilation * (f.Kh - 1) + 2 * f.pad;
+        d->Wi = f.W - f.dilation * (f.Kw - 1) + 2 * f.pad;
+    } else {
+        d->Hi = f.Ho;
+        d->Wi = f.Wo;
+    }
+    d->zbytes = d->zeros ? align_up(static_cast<size_t>(f.N) * d->Hi * d->Wi * f.C_out * f.elt, 256) : 0;
+    return CONV_OK;
+}
+
+int backward_data_impl(const void *dy, const void *w_packed_t, void *dx, int N, int C_in, int H, int W, int C_out,
+                       int Kh, int Kw, int stride, int pad, int dilation, int groups, conv_dtype_t dtype,
+                       conv_layout_t layout, void *workspace, size_t workspace_bytes, cudaStream_t stream,
+                       size_t *bytes_only) {
+    Plan f;
+    int st = make_plan(N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype, layout, false, 0, &f, 2);
+    if (st != CONV_OK) return st;
+    DgradShape d;
+    dgrad_shape(f, &d);
+    const PadW pw{d.pad_w};
+    if (bytes_only) {
+        size_t inner = 0;
+        st = workspace_impl(false, N, C_out, d.Hi, d.Wi, C_in, Kh, Kw, 1, d.pad_h, dilation, groups, dtype, layout,
+                            &inner, &pw);
+        if (st != CONV_OK) return st;
+        *bytes_only = d.zbytes + inner;
+        return ok();
+    }
+    if (!dy || !w_packed_t || !dx) return fail(CONV_ERR_INVALID_ARG, "dy, w_packed_t and dx must not be NULL");
+    if (d.zbytes > 0 && (!workspace || workspace_bytes < d.zbytes))
+        return fail(CONV_ERR_WORKSPACE, "workspace of at least %zu bytes needed, %zu given", d.zbytes,
+                    workspace ? workspace_bytes : static_cast<size_t>(0));
+    if (!aligned16(dy) || !aligned16(w_packed_t) || !aligned16(dx) || (workspace && !aligned16(workspace)))
+        return fail(CONV_ERR_UNSUPPORTED, "device pointers must be 16-byte aligned");
+    const void *src = dy;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    if (d.zeros) {
+        // validate the inner convolution before anything is enqueued
+        size_t inner = 0;
+        st = workspace_impl(false, N, C_out, d.Hi, d.Wi, C_in, Kh, Kw, 1, d.pad_h, dilation, groups, dtype, layout,
+                            &inner, &pw);
+        if (st != CONV_OK) return st;
+        if (workspace_bytes < d.zbytes + inner)
+            return fail(CONV_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", d.zbytes + inner,
+                        workspace_bytes);
+        if ((st = check_launch(launch_zero_insert(dy, ws, N, C_out, f.Ho, f.Wo, d.Hi, d.Wi, stride,
+                                                  layout == CONV_NCHW, f.elt, stream),
+                               "zero insertion")) != CONV_OK)
+            return st;
+        src = ws;
+    }
+    return forward_impl(false, src, w_packed_t, nullptr, dx, N, C_out, d.Hi, d.Wi, C_in, Kh, Kw, 1, d.pad_h,
+                        dilation, groups, dtype, layout, ws ? ws + d.zbytes : nullptr,
+                        workspace_bytes > d.zbytes ? workspace_bytes - d.zbytes : 0, stream, &pw);
+}
+
+// ------------------------------------------------------------------ Winograd ---
+// F(m x m, 3 x 3), m = 2 or 4 (winograd.cu): input transform -> the tensor-core product
+// as a grouped 1x1 convolution with alpha^2 groups over the transformed tiles, fp32
+// results -> output transform.  Scratch: [V][M partial sums][the product's own scratch].
+struct WinoPlan {
+    Plan f;          // the 3x3 problem: validation, Ho, Wo
+    Plan g;          // the product
+    int m, a, Cpg, TH, TW, T;
+    size_t off_v, off_m, off_inner, ws_total;
+};
+
+int wino_plan(int N, int C_in, int H, int W, int C_out, int pad, int m, conv_dtype_t dtype, conv_layout_t layout,
+              DeviceInfo *dev, const Settings &cfg, WinoPlan *out) {
+    WinoPlan w{};
+    if (m != 2 && m != 4) return fail(CONV_ERR_INVALID_ARG, "Winograd tile m must be 2 or 4 (F(2x2,3x3), F(4x4,3x3))");
+    int st = make_plan(N, C_in, H, W, C_out, 3, 3, 1, pad, 1, 1, dtype, layout, false, 0, &w.f, 2);
+    if (st != CONV_OK) return st;
+    w.m = m;
+    w.a = m + 2;
+    w.Cpg = round_up(C_in, 16 / w.f.elt);
+    w.TH = (w.f.Ho + m - 1) / m;
+    w.TW = (w.f.Wo + m - 1) / m;
+    const long long T = static_cast<long long>(N) * w.TH * w.TW;
+    if (T >= (1LL << 31) - 256) return fail(CONV_ERR_UNSUPPORTED, "too many Winograd tiles");
+    w.T = static_cast<int>(T);
+    const int a2 = w.a * w.a;
+    const PadW pw{0, reinterpret_cast<float *>(16)};  // placeholder address: plans the external-partial form
+    st = device_plan(false, 1, a2 * w.Cpg, 1, w.T, a2 * C_out, 1, 1, 1, 0, 1, a2, dtype, CONV_NHWC, dev, cfg, &w.g,
+                     &pw);
+    if (st != CONV_OK) return st;
+    size_t off = 0;
+    w.off_v = off;
+    off = align_up(off + static_cast<size_t>(T) * a2 * w.Cpg * w.f.elt, 256);
+    w.off_m = off;
+    off = align_up(off + static_cast<size_t>(w.g.splits) * T * a2 * C_out * 4, 256);
+    w.off_inner = off;
+    w.ws_total = off + w.g.ws_total;
+    *out = w;
+    return CONV_OK;
+}
+
+int winograd_impl(const void *x, const void *u_packed, const void *bias, void *y, int N, int C_in, int H, int W,
+                  int C_out, int pad, int m, conv_dtype_t dtype, conv_layout_t layout, void *workspace,
+                  size_t workspace_bytes, cudaStream_t stream, size_t *bytes_only) {
+    const Settings cfg = settings_now();
+    WinoPlan w;
+    int st;
+    if (bytes_only) {
+        if ((st = wino_plan(N, C_in, H, W, C_out, pad, m, dtype, layout, current_device_or_null(), cfg, &w)) != CONV_OK)
+            return st;
+        *bytes_only = w.ws_total;
+        return ok();
+    }
+    if ((st = wino_plan(N, C_in, H, W, C_out, pad, m, dtype, layout, nullptr, cfg, &w)) != CONV_OK) return st;
+    if (!x || !u_packed || !y) return fail(CONV_ERR_INVALID_ARG, "x, u_packed and y must not be NULL");
+    DeviceInfo *dev = nullptr;
+    if ((st = device_info(&dev)) != CONV_OK) return st;
+    if ((st = wino_plan(N, C_in, H, W, C_out, pad, m, dtype, layout, dev, cfg, &w)) != CONV_OK) return st;
+    if (!workspace || workspace_bytes < w.ws_total)
+        return fail(CONV_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", w.ws_total,
+                    workspace ? workspace_bytes : static_cast<size_t>(0));
+    if (!aligned16(x) || !aligned16(u_packed) || !aligned16(y) || (bias && !aligned16(bias)) || !aligned16(workspace))
+        return fail(CONV_ERR_UNSUPPORTED, "device pointers must be 16-byte aligned");
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    float *mp = reinterpret_cast<float *>(ws + w.off_m);
+    const bool nchw = layout == CONV_NCHW;
+    if ((st = check_launch(launch_wino_input(x, ws + w.off_v, N, C_in, H, W, w.Cpg, w.TH, w.TW, pad, m, nchw,
+                                             w.f.f32, stream),
+                           "Winograd input transform")) != CONV_OK)
+        return st;
+    const int a2 = w.a * w.a;
+    const PadW pw{0, mp};
+    if ((st = forward_impl(false, ws + w.off_v, u_packed, nullptr, mp, 1, a2 * w.Cpg, 1, w.T, a2 * C_out, 1, 1, 1, 0,
+                           1, a2, dtype, CONV_NHWC, ws + w.off_inner, workspace_bytes - w.off_inner, stream, &pw)) !=
+        CONV_OK)
+        return st;
+    return check_launch(launch_wino_output(mp, bias, y, N, C_out, w.f.Ho, w.f.Wo, w.TH, w.TW, w.g.splits, m, nchw,
+                                           w.f.f32, stream),
+                        "Winograd output transform") == CONV_OK
+               ? ok()
+               : CONV_ERR_CUDA;
+}
+
+// Packed size of the transposed convolution's kernel: C_in output channels of
+// C_out/groups reduction channels per group (merged like any narrow group).
+int packed_weight_t_bytes(int C_out, int C_in, int Kh, int Kw, int groups, int elt, int *cpg, int *gm) {
+    *gm = group_merge(C_in, C_out, groups, elt);
+    *cpg = round_up(C_out / groups, 16 / elt) * *gm;
+    return 0;
+}
 }  // namespace
 }  // namespace conv2d_b200
 
@@ -1134,6 +1599,193 @@ int conv2d_debug_set_pair_mode(int mode) {
     if (mode < 0 || mode > 2) return fail(CONV_ERR_INVALID_ARG, "pair mode must be 0, 1 or 2");
     g_pair_mode.store(mode, std::memory_order_relaxed);
     return ok();
+}
+
+
+int conv2d_packed_weight_backward_data_size(int C_out, int C_in, int Kh, int Kw, int groups, conv_dtype_t dtype,
+                                            size_t *bytes) {
+    const int elt = elt_of(dtype);
+    if (!bytes || elt == 0 || C_out < 1 || C_in < 1 || Kh < 1 || Kw < 1 || groups < 1 || C_in % groups ||
+        C_out % groups)
+        return fail(CONV_ERR_INVALID_ARG, "packed weight size: invalid argument");
+    int cpg = 0, gm = 1;
+    packed_weight_t_bytes(C_out, C_in, Kh, Kw, groups, elt, &cpg, &gm);
+    *bytes = static_cast<size_t>(C_in) * Kh * Kw * cpg * elt;
+    return ok();
+}
+
+int conv2d_pack_weight_backward_data(const void *w_oihw, void *w_packed_t, int C_out, int C_in, int Kh, int Kw,
+                                     int groups, conv_dtype_t dtype, conv_stream_t stream) {
+    size_t bytes = 0;
+    int st = conv2d_packed_weight_backward_data_size(C_out, C_in, Kh, Kw, groups, dtype, &bytes);
+    if (st != CONV_OK) return st;
+    if (!w_oihw || !w_packed_t) return fail(CONV_ERR_INVALID_ARG, "weight pointers must not be NULL");
+    const int elt = elt_of(dtype);
+    int cpg = 0, gm = 1;
+    packed_weight_t_bytes(C_out, C_in, Kh, Kw, groups, elt, &cpg, &gm);
+    if ((st = check_launch(launch_pack_weight_t(w_oihw, w_packed_t, C_in, C_out / groups, C_in / groups, gm, Kh, Kw,
+                                                cpg, elt, reinterpret_cast<cudaStream_t>(stream)),
+                           "transposed weight pack")) != CONV_OK)
+        return st;
+    return ok();
+}
+
+int conv2d_backward_data_workspace_size(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stride,
+                                        int pad, int dilation, int groups, conv_dtype_t dtype,
+                                        conv_layout_t layout, size_t *bytes) {
+    if (!bytes) return fail(CONV_ERR_INVALID_ARG, "bytes must not be NULL");
+    return backward_data_impl(nullptr, nullptr, nullptr, N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation,
+                              groups, dtype, layout, nullptr, 0, nullptr, bytes);
+}
+
+int conv2d_backward_data(const void *dy, const void *w_packed_t, void *dx, int N, int C_in, int H, int W,
+                         int C_out, int Kh, int Kw, int stride, int pad, int dilation, int groups,
+                         conv_dtype_t dtype, conv_layout_t layout, void *workspace, size_t workspace_bytes,
+                         conv_stream_t stream) {
+    return backward_data_impl(dy, w_packed_t, dx, N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups,
+                              dtype, layout, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream),
+                              nullptr);
+}
+
+int conv2d_backward_weight_workspace_size(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stride,
+                                          int pad, int dilation, int groups, conv_dtype_t dtype,
+                                          conv_layout_t layout, int with_bias, size_t *bytes) {
+    if (!bytes) return fail(CONV_ERR_INVALID_ARG, "bytes must not be NULL");
+    WgPlan w;
+    DeviceInfo *dev = current_device_or_null();
+    int st = wgrad_plan(N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype, layout, with_bias != 0,
+                        dev ? dev->sms : 0, &w);
+    if (st != CONV_OK) return st;
+    *bytes = w.ws_total;
+    return ok();
+}
+
+int conv2d_backward_weight(const void *x, const void *dy, void *dw, void *db, int N, int C_in, int H, int W,
+                           int C_out, int Kh, int Kw, int stride, int pad, int dilation, int groups,
+                           conv_dtype_t dtype, conv_layout_t layout, void *workspace, size_t workspace_bytes,
+                           conv_stream_t stream) {
+    return backward_weight_impl(x, dy, dw, db, N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype,
+                                layout, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int conv2d_backward_bias_workspace_size(int N, int C_out, int Ho, int Wo, conv_layout_t layout, size_t *bytes) {
+    if (!bytes || N < 1 || C_out < 1 || Ho < 1 || Wo < 1 || (layout != CONV_NHWC && layout != CONV_NCHW))
+        return fail(CONV_ERR_INVALID_ARG, "bias gradient size: invalid argument");
+    const long long rows = static_cast<long long>(N) * Ho * Wo;
+    *bytes = static_cast<size_t>(bias_grad_partials(rows, C_out, N, layout == CONV_NCHW)) * C_out * 4;
+    return ok();
+}
+
+int conv2d_backward_bias(const void *dy, void *db, int N, int C_out, int Ho, int Wo, conv_dtype_t dtype,
+                         conv_layout_t layout, void *workspace, size_t workspace_bytes, conv_stream_t stream) {
+    size_t need = 0;
+    int st = conv2d_backward_bias_workspace_size(N, C_out, Ho, Wo, layout, &need);
+    if (st != CONV_OK) return st;
+    const int elt = elt_of(dtype);
+    if (!dy || !db || elt == 0) return fail(CONV_ERR_INVALID_ARG, "dy and db must not be NULL; dtype must be valid");
+    if (!workspace || workspace_bytes < need)
+        return fail(CONV_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need,
+                    workspace ? workspace_bytes : static_cast<size_t>(0));
+    if (!aligned16(workspace)) return fail(CONV_ERR_UNSUPPORTED, "device pointers must be 16-byte aligned");
+    return check_launch(launch_bias_grad(dy, static_cast<float *>(workspace), db, N, C_out,
+                                         static_cast<long long>(Ho) * Wo, layout == CONV_NCHW, dtype == CONV_F32,
+                                         reinterpret_cast<cudaStream_t>(stream)),
+                        "bias gradient") == CONV_OK
+               ? ok()
+               : CONV_ERR_CUDA;
+}
+
+
+// ------------------------------------------------------------------ conv3d ---
+int conv3d_packed_weight_size(int C_out, int C_in, int Kd, int Kh, int Kw, int groups, conv_dtype_t dtype,
+                              size_t *bytes) {
+    const int elt = elt_of(dtype);
+    if (!bytes || elt == 0 || C_out < 1 || C_in < 1 || Kd < 1 || Kh < 1 || Kw < 1 || groups < 1 ||
+        C_in % groups || C_out % groups)
+        return fail(CONV_ERR_INVALID_ARG, "packed weight size: invalid argument");
+    const int gm = group_merge(C_out, C_in, groups, elt);
+    const int cpg = round_up(C_in / groups, 16 / elt) * gm;
+    *bytes = static_cast<size_t>(C_out) * Kd * Kh * Kw * cpg * elt;
+    return ok();
+}
+
+int conv3d_pack_weight(const void *w_oidhw, void *w_packed, int C_out, int C_in, int Kd, int Kh, int Kw,
+                       int groups, conv_dtype_t dtype, conv_stream_t stream) {
+    size_t bytes = 0;
+    int st = conv3d_packed_weight_size(C_out, C_in, Kd, Kh, Kw, groups, dtype, &bytes);
+    if (st != CONV_OK) return st;
+    if (!w_oidhw || !w_packed) return fail(CONV_ERR_INVALID_ARG, "weight pointers must not be NULL");
+    const int elt = elt_of(dtype);
+    const int gm = group_merge(C_out, C_in, groups, elt);
+    const int cpg = round_up(C_in / groups, 16 / elt) * gm;
+    // (kd, kh) flattened: the OIDHW weight is an OIHW weight of filter height Kd*Kh
+    if ((st = check_launch(launch_pack_weight(w_oidhw, w_packed, C_out, C_in / groups, C_out / groups, gm, Kd * Kh,
+                                              Kw, cpg, elt, reinterpret_cast<cudaStream_t>(stream)),
+                           "weight pack")) != CONV_OK)
+        return st;
+    return ok();
+}
+
+int conv3d_workspace_size(int N, int C_in, int D, int H, int W, int C_out, int Kd, int Kh, int Kw, int stride,
+                          int pad, int dilation, int groups, conv_dtype_t dtype, conv_layout_t layout,
+                          size_t *bytes) {
+    const Vol vol{D, Kd};
+    return workspace_impl(false, N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype, layout, bytes,
+                          nullptr, &vol);
+}
+
+int conv3d_forward(const void *x, const void *w_packed, const void *bias, void *y, int N, int C_in, int D, int H,
+                   int W, int C_out, int Kd, int Kh, int Kw, int stride, int pad, int dilation, int groups,
+                   conv_dtype_t dtype, conv_layout_t layout, void *workspace, size_t workspace_bytes,
+                   conv_stream_t stream) {
+    const Vol vol{D, Kd};
+    return forward_impl(false, x, w_packed, bias, y, N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups,
+                        dtype, layout, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream), nullptr,
+                        &vol);
+}
+
+
+// ---------------------------------------------------------------- Winograd ---
+int conv2d_winograd_packed_weight_size(int C_out, int C_in, int m, conv_dtype_t dtype, size_t *bytes) {
+    const int elt = elt_of(dtype);
+    if (!bytes || elt == 0 || C_out < 1 || C_in < 1 || (m != 2 && m != 4))
+        return fail(CONV_ERR_INVALID_ARG, "Winograd packed weight size: invalid argument");
+    const int a2 = (m + 2) * (m + 2);
+    const int cpg = round_up(C_in, 16 / elt);
+    const int gm = group_merge(a2 * C_out, a2 * cpg, a2, elt);
+    *bytes = static_cast<size_t>(a2) * C_out * cpg * gm * elt;
+    return ok();
+}
+
+int conv2d_pack_weight_winograd(const void *w_oihw, void *u_packed, int C_out, int C_in, int m, conv_dtype_t dtype,
+                                conv_stream_t stream) {
+    size_t bytes = 0;
+    int st = conv2d_winograd_packed_weight_size(C_out, C_in, m, dtype, &bytes);
+    if (st != CONV_OK) return st;
+    if (!w_oihw || !u_packed) return fail(CONV_ERR_INVALID_ARG, "weight pointers must not be NULL");
+    const int elt = elt_of(dtype);
+    const int a2 = (m + 2) * (m + 2);
+    const int cpg = round_up(C_in, 16 / elt);
+    const int gm = group_merge(a2 * C_out, a2 * cpg, a2, elt);
+    return check_launch(launch_wino_weight(w_oihw, u_packed, C_out, C_in, cpg, gm, m, dtype == CONV_F32,
+                                           reinterpret_cast<cudaStream_t>(stream)),
+                        "Winograd weight transform") == CONV_OK
+               ? ok()
+               : CONV_ERR_CUDA;
+}
+
+int conv2d_winograd_workspace_size(int N, int C_in, int H, int W, int C_out, int pad, int m, conv_dtype_t dtype,
+                                   conv_layout_t layout, size_t *bytes) {
+    if (!bytes) return fail(CONV_ERR_INVALID_ARG, "bytes must not be NULL");
+    return winograd_impl(nullptr, nullptr, nullptr, nullptr, N, C_in, H, W, C_out, pad, m, dtype, layout, nullptr, 0,
+                         nullptr, bytes);
+}
+
+int conv2d_forward_winograd(const void *x, const void *u_packed, const void *bias, void *y, int N, int C_in, int H,
+                            int W, int C_out, int pad, int m, conv_dtype_t dtype, conv_layout_t layout,
+                            void *workspace, size_t workspace_bytes, conv_stream_t stream) {
+    return winograd_impl(x, u_packed, bias, y, N, C_in, H, W, C_out, pad, m, dtype, layout, workspace,
+                         workspace_bytes, reinterpret_cast<cudaStream_t>(stream), nullptr);
 }
 
 }  // extern "C"

@@ -34,9 +34,11 @@ struct IgemmParams {
     CUtensorMap tmap_a;  // A operand: im2col-mode map of x (NHWC) or tiled map of X_col
     CUtensorMap tmap_b;  // B operand: tiled map of the packed weights {Kp, Cout_g, groups}
     CUtensorMap tmap_y;  // tma_out: y as {C_out, M}, 32 x 32 boxes with 64-byte swizzle
-    int M;               // N * Ho * Wo
-    int HoWo, Wo;
+    int M;               // N * Ho * Wo (volumes: N * Do * Ho * Wo)
+    int HoWo, Wo;        // HoWo: output pixels per image (volumes: Do * Ho * Wo)
+    int HoWo2, Kh;       // volumes: Ho * Wo per output depth slice, and the filter height
     int stride, pad, dilation;
+    int pad_w;           // column padding (pad: row padding)
     int Kw, taps;        // taps = Kh * Kw
     int Cpg;             // padded input channels per group (elements)
     int nCB;             // channel blocks per tap
@@ -82,6 +84,7 @@ struct GatherParams {
     int R, BW, ME;         // halo rows, row width (elements) and left zero margin
     int tma_out;           // epilogue stages each tile channel-major and stores it by TMA
     int cw;                // output channels per epilogue group
+    int tpix;              // transposed kernel (gather_t.cu): pixels per tile, Wo rounded up to 16
     uint32_t tmem_cols;
     void *y;
     const void *bias;
@@ -100,6 +103,7 @@ struct DwParams {
     const void *bias;
     void *y;
     int N, C, Ho, Wo, Kh, Kw, stride, pad, dilation;
+    int pad_w;             // column padding (pad: row padding)
     int Cpg;               // channel pitch of w_packed
     int TH, TW, IH, IW;    // output tile and the staged input box
     int n_th, n_tw, units, stages;
@@ -110,17 +114,42 @@ struct DwParams {
     int starve;
 };
 
+// One launch of the weight-gradient kernel (wgrad.cu): per group, dW_row = dout_col X_col^T
+// with the reduction over output pixels in stages of PK (64 bf16 / 32 fp32), written as
+// fp32 partial sums ws[split][C_out][taps][Cpg].  Unit u = (((split*n_otiles + otile)*groups
+// + g)*taps + tap)*n_ctiles + ctile.
+struct WgradParams {
+    CUtensorMap tmap_dy;   // dy channels-last as {groups*dy_cpg, M}, boxes of {128 bytes, PK}, 128-byte swizzle
+    CUtensorMap tmap_x;    // im2col map of channels-last x ({groups*Cpg, W, H, N}), PK pixels x 128 bytes
+    float *ws;
+    int M, HoWo, Wo, stride, pad, dilation, Kw, taps;
+    int Cpg;               // channels per group of the x tensor read (multiple of 128 bytes)
+    int dy_cpg;            // channels per group of the dy tensor read (multiple of 16 bytes)
+    int Cout, Cout_g, groups;
+    int BN;                // channels per tile (multiple of 128 bytes; <= 256 bf16, <= 128 fp32)
+    int n_ctiles, n_otiles, kstages, splits, units, stages, chunk_stages;
+    uint32_t tmem_cols;
+    int *status;
+    long long timeout_ns;
+    int starve;
+};
+
 // Launchers (igemm.cu, gather.cu, layout.cu).  All return cudaSuccess or the launch error.
 // pair: bf16 only, grid even, launched as clusters of two CTAs (p.n_mtiles counts
-// 256-row units, the tensor map of B has boxes of BN/2 rows).
+// 256-row units, the tensor map of B has boxes of BN/2 rows).  vol: 5-D (volumetric)
+// im2col map, filter taps stepped over (kd, kh, kw); needs im2col.
 cudaError_t launch_igemm(const IgemmParams &p, bool f32, int cb_bytes, bool im2col, bool pair, int grid,
-                         size_t smem_bytes, cudaStream_t stream);
+                         size_t smem_bytes, cudaStream_t stream, bool vol = false);
 // Bytes of dynamic shared memory for `stages` stages holding BN rows of B each.
 size_t igemm_smem_bytes(bool f32, int BN, int stages, bool tma_out);
 // Two-CTA clusters of the pair kernel that can be resident at once.
-cudaError_t igemm_pair_max_clusters(int cb_bytes, bool im2col, size_t smem_bytes, int *clusters);
+cudaError_t igemm_pair_max_clusters(int cb_bytes, bool im2col, size_t smem_bytes, int *clusters, bool vol = false);
 cudaError_t launch_gather(const GatherParams &p, bool f32, int grid, size_t smem, cudaStream_t stream);
 size_t gather_smem_bytes(bool f32, int BN, int Kpad, size_t halo_bytes, size_t out_stage_bytes);
+// The transposed few-channel kernel (gather_t.cu): bf16, NCHW in and out, one output row
+// per tile, output channels on the tensor-memory lanes.
+cudaError_t launch_gather_t(const GatherParams &p, int grid, size_t smem, cudaStream_t stream);
+size_t gather_t_smem_bytes(int Kpad, int tpix, size_t halo_bytes);
 int gather_max_stages();
 int igemm_threads(bool f32);
 
@@ -133,6 +162,35 @@ int dw_threads();
 int dw_compute_warps();
 int dw_max_stages();
 size_t dw_header_bytes();
+
+cudaError_t launch_wgrad(const WgradParams &p, bool f32, int grid, size_t smem, cudaStream_t stream);
+size_t wgrad_smem_bytes(bool f32, int BN, int stages);
+int wgrad_pixels_per_stage(bool f32);
+int wgrad_max_stages();
+// Weight gradient on the CUDA cores for few channels per group: partial sums
+// ws[split][C_out][Kh*Kw][C_in/groups] from channels-last x and dy.
+cudaError_t launch_wgrad_direct(const void *x, const void *dy, float *ws, int N, int C_in, int H, int W, int C_out,
+                                int Ho, int Wo, int Kh, int Kw, int stride, int pad, int dilation, int groups,
+                                int splits, bool f32, cudaStream_t s);
+cudaError_t launch_wgrad_reduce(const float *ws, void *dw, int Cout, int Cin_g, int taps, int Cpg, int splits,
+                                bool f32, cudaStream_t s);
+// Bias gradient db[c] = sum of dy over images and output positions: partials (count from
+// bias_grad_partials, times C floats of scratch), then their sum in the bias type.
+int bias_grad_partials(long long rows, int C, int N, bool nchw);
+cudaError_t launch_bias_grad(const void *dy, float *partial, void *db, int N, int C, long long plane, bool nchw,
+                             bool f32, cudaStream_t s);
+cudaError_t launch_zero_insert(const void *dy, void *dyz, int N, int C, int Ho, int Wo, int Hz, int Wz, int stride,
+                               bool nchw, int elt, cudaStream_t s);
+cudaError_t launch_pack_weight_t(const void *w, void *wp, int O, int R, int Cin_g, int gm, int Kh, int Kw, int Cpg,
+                                 int elt, cudaStream_t s);
+
+// Winograd F(m x m, 3 x 3) transforms (winograd.cu), m = 2 or 4.
+cudaError_t launch_wino_input(const void *x, void *v, int N, int C, int H, int W, int Cpg, int TH, int TW, int pad,
+                              int m, bool nchw, bool f32, cudaStream_t s);
+cudaError_t launch_wino_weight(const void *w, void *u, int C_out, int C, int Cpg, int gm, int m, bool f32,
+                               cudaStream_t s);
+cudaError_t launch_wino_output(const float *mp, const void *bias, void *y, int N, int C_out, int Ho, int Wo, int TH,
+                               int TW, int splits, int m, bool nchw, bool f32, cudaStream_t s);
 
 cudaError_t launch_nchw_to_nhwc(const void *src, void *dst, int N, int C, int H, int W,
                                 int groups, int Cpg, int elt, cudaStream_t s);

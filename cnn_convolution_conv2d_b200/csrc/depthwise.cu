@@ -136,7 +136,7 @@ __global__ void __launch_bounds__(kDwThreads, 1) dw_kernel(const __grid_constant
                 if (!p.starve) {
                     mbar_arrive_expect_tx(&sb.full[stage], sbytes);
                     tma_load_4d(ring + static_cast<size_t>(stage) * sbytes, &p.tmap_x, &sb.full[stage],
-                                t.chunk * kCC, t.tw * p.TW * p.stride - p.pad,
+                                t.chunk * kCC, t.tw * p.TW * p.stride - p.pad_w,
                                 t.th * p.TH * p.stride - p.pad, t.n);
                     ++issued;
                 }

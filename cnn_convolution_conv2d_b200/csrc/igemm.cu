@@ -215,9 +215,12 @@ __device__ __forceinline__ void issue_stage(uint32_t a, uint32_t b, uint32_t alo
 // kPair: launched in clusters of two CTAs on an SM pair; each unit of work is 256
 // output pixels (128 per CTA) x BN channels, computed by M = 256 pair MMAs issued from
 // the even CTA, with each CTA staging its own 128 rows of A and BN/2 rows of B.
-template <bool kF32, int kCB, bool kIm2col, bool kPair>
+// kVol (with kIm2col): the input is a 5-D channels-last volume (c, w, h, d, n), rows
+// are output voxels and the filter taps run over (kd, kh, kw) -- the 3-D convolution.
+template <bool kF32, int kCB, bool kIm2col, bool kPair, bool kVol = false>
 __global__ void __launch_bounds__(threads_for<kF32>(), 1)
     igemm_kernel(const __grid_constant__ IgemmParams p) {
+    static_assert(kIm2col || !kVol, "volumes are read through im2col-mode loads");
     static_assert(!(kF32 && kPair), "CTA pairs are bf16 only");
     constexpr int kElt = kF32 ? 4 : 2;
     constexpr int kCBe = kCB / kElt;              // channels (elements) per plane row
@@ -297,27 +300,37 @@ __global__ void __launch_bounds__(threads_for<kF32>(), 1)
                 // reloads that tile (its results are never stored)
                 const int m0 = kPair ? min(t.mtile * kUnitRows + row_off, ((p.M - 1) / kBM) * kBM)
                                      : t.mtile * kBM;
-                int img = 0, h0 = 0, w0 = 0;
+                int img = 0, d0 = 0, h0 = 0, w0 = 0;
                 if constexpr (kIm2col) {
                     img = m0 / p.HoWo;
-                    const int rem = m0 - img * p.HoWo;
+                    int rem = m0 - img * p.HoWo;
+                    if constexpr (kVol) {
+                        const int od = rem / p.HoWo2;
+                        rem -= od * p.HoWo2;
+                        d0 = od * p.stride - p.pad;
+                    }
                     const int oh = rem / p.Wo;
                     const int ow = rem - oh * p.Wo;
                     h0 = oh * p.stride - p.pad;
-                    w0 = ow * p.stride - p.pad;
+                    w0 = ow * p.stride - p.pad_w;
                 }
                 // Filter tap (kh, kw) and channel block of the next plane, stepped
                 // along instead of divided out per plane; past the last plane (the
                 // padding of the last stage, whose weights are zero) the tap stays at
                 // the last one so that the load is still well formed.
-                int cblk = 0, kh = 0, kw = 0, tap = 0;
+                int cblk = 0, kd = 0, kh = 0, kw = 0, tap = 0;
                 if constexpr (kIm2col) {
                     if (t.k0 > 0) {
                         const int plane0 = t.k0 * kNP;
                         tap = plane0 / p.nCB;
                         cblk = plane0 - tap * p.nCB;
-                        kh = tap / p.Kw;
-                        kw = tap - kh * p.Kw;
+                        int r = tap;
+                        if constexpr (kVol) {
+                            kd = r / (p.Kh * p.Kw);
+                            r -= kd * p.Kh * p.Kw;
+                        }
+                        kh = r / p.Kw;
+                        kw = r - kh * p.Kw;
                     }
                 }
                 for (int ks = t.k0; ks < t.k1; ++ks) {
@@ -336,24 +349,37 @@ __global__ void __launch_bounds__(threads_for<kF32>(), 1)
                             const int kelem = plane * kCBe;  // offset in the group's reduction
                             if constexpr (kIm2col) {
                                 const bool in = tap < p.taps;
-                                const int khc = in ? kh : (p.taps - 1) / p.Kw;
+                                // past the last plane: the last tap, so the load stays well formed
+                                const int kdc = in ? kd : (kVol ? (p.taps - 1) / (p.Kh * p.Kw) : 0);
+                                const int khc = in ? kh : (kVol ? p.Kh - 1 : (p.taps - 1) / p.Kw);
                                 const int kwc = in ? kw : p.Kw - 1;
                                 const int c = t.g * p.Cpg + cblk * kCBe;
-                                if constexpr (kPair)
+                                const uint16_t ow_ = static_cast<uint16_t>(kwc * p.dilation);
+                                const uint16_t oh_ = static_cast<uint16_t>(khc * p.dilation);
+                                if constexpr (kVol) {
+                                    const uint16_t od_ = static_cast<uint16_t>(kdc * p.dilation);
+                                    if constexpr (kPair)
+                                        tma_load_im2col_5d_pair(st + j * (kBM * kCB), &p.tmap_a, fbar, c, w0, h0, d0,
+                                                                img, ow_, oh_, od_);
+                                    else
+                                        tma_load_im2col_5d(st + j * (kBM * kCB), &p.tmap_a, &sb.full[stage], c, w0,
+                                                           h0, d0, img, ow_, oh_, od_);
+                                } else if constexpr (kPair) {
                                     tma_load_im2col_4d_pair(st + j * (kBM * kCB), &p.tmap_a, fbar, c, w0, h0,
-                                                            img, static_cast<uint16_t>(kwc * p.dilation),
-                                                            static_cast<uint16_t>(khc * p.dilation));
-                                else
+                                                            img, ow_, oh_);
+                                } else {
                                     tma_load_im2col_4d(st + j * (kBM * kCB), &p.tmap_a, &sb.full[stage],
-                                                       c, w0, h0, img,
-                                                       static_cast<uint16_t>(kwc * p.dilation),
-                                                       static_cast<uint16_t>(khc * p.dilation));
+                                                       c, w0, h0, img, ow_, oh_);
+                                }
                                 if (++cblk == p.nCB) {
                                     cblk = 0;
                                     ++tap;
                                     if (++kw == p.Kw) {
                                         kw = 0;
-                                        ++kh;
+                                        if (++kh == p.Kh && kVol) {
+                                            kh = 0;
+                                            ++kd;
+                                        }
                                     }
                                 }
                             } else {
@@ -693,9 +719,9 @@ __global__ void __launch_bounds__(threads_for<kF32>(), 1)
     }
 }
 
-template <bool kF32, int kCB, bool kIm2col, bool kPair>
+template <bool kF32, int kCB, bool kIm2col, bool kPair, bool kVol = false>
 cudaError_t launch_one(const IgemmParams &p, int grid, size_t smem, cudaStream_t stream) {
-    auto kern = igemm_kernel<kF32, kCB, kIm2col, kPair>;
+    auto kern = igemm_kernel<kF32, kCB, kIm2col, kPair, kVol>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
@@ -721,9 +747,9 @@ cudaError_t launch_one(const IgemmParams &p, int grid, size_t smem, cudaStream_t
 }
 
 // How many two-CTA clusters of the pair kernel fit on the device at once.
-template <int kCB, bool kIm2col>
+template <int kCB, bool kIm2col, bool kVol = false>
 cudaError_t pair_clusters_one(size_t smem, int *out) {
-    auto kern = igemm_kernel<false, kCB, kIm2col, true>;
+    auto kern = igemm_kernel<false, kCB, kIm2col, true, kVol>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
@@ -741,13 +767,13 @@ cudaError_t pair_clusters_one(size_t smem, int *out) {
     return cudaOccupancyMaxActiveClusters(out, kern, &cfg);
 }
 
-template <bool kF32, bool kIm2col, bool kPair>
+template <bool kF32, bool kIm2col, bool kPair, bool kVol = false>
 cudaError_t launch_cb(const IgemmParams &p, int cb, int grid, size_t smem, cudaStream_t s) {
     switch (cb) {
-        case 128: return launch_one<kF32, 128, kIm2col, kPair>(p, grid, smem, s);
-        case 64: return launch_one<kF32, 64, kIm2col, kPair>(p, grid, smem, s);
-        case 32: return launch_one<kF32, 32, kIm2col, kPair>(p, grid, smem, s);
-        case 16: return launch_one<kF32, 16, kIm2col, kPair>(p, grid, smem, s);
+        case 128: return launch_one<kF32, 128, kIm2col, kPair, kVol>(p, grid, smem, s);
+        case 64: return launch_one<kF32, 64, kIm2col, kPair, kVol>(p, grid, smem, s);
+        case 32: return launch_one<kF32, 32, kIm2col, kPair, kVol>(p, grid, smem, s);
+        case 16: return launch_one<kF32, 16, kIm2col, kPair, kVol>(p, grid, smem, s);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -761,8 +787,17 @@ size_t igemm_smem_bytes(bool f32, int BN, int stages, bool tma_out) {
 
 int igemm_threads(bool f32) { return f32 ? threads_for<true>() : threads_for<false>(); }
 
-cudaError_t igemm_pair_max_clusters(int cb_bytes, bool im2col, size_t smem_bytes, int *clusters) {
+cudaError_t igemm_pair_max_clusters(int cb_bytes, bool im2col, size_t smem_bytes, int *clusters, bool vol) {
     *clusters = 0;
+    if (vol) {
+        switch (cb_bytes) {
+            case 128: return pair_clusters_one<128, true, true>(smem_bytes, clusters);
+            case 64: return pair_clusters_one<64, true, true>(smem_bytes, clusters);
+            case 32: return pair_clusters_one<32, true, true>(smem_bytes, clusters);
+            case 16: return pair_clusters_one<16, true, true>(smem_bytes, clusters);
+            default: return cudaErrorInvalidValue;
+        }
+    }
     switch (cb_bytes) {
         case 128: return im2col ? pair_clusters_one<128, true>(smem_bytes, clusters)
                                 : pair_clusters_one<128, false>(smem_bytes, clusters);
@@ -777,8 +812,17 @@ cudaError_t igemm_pair_max_clusters(int cb_bytes, bool im2col, size_t smem_bytes
 }
 
 cudaError_t launch_igemm(const IgemmParams &p, bool f32, int cb_bytes, bool im2col, bool pair, int grid,
-                         size_t smem_bytes, cudaStream_t stream) {
+                         size_t smem_bytes, cudaStream_t stream, bool vol) {
     if (p.stages < 2 || p.stages > kMaxStages) return cudaErrorInvalidValue;
+    if (vol) {
+        if (!im2col) return cudaErrorInvalidValue;
+        if (pair) {
+            if (f32 || grid % 2 != 0) return cudaErrorInvalidValue;
+            return launch_cb<false, true, true, true>(p, cb_bytes, grid, smem_bytes, stream);
+        }
+        return f32 ? launch_cb<true, true, false, true>(p, cb_bytes, grid, smem_bytes, stream)
+                   : launch_cb<false, true, false, true>(p, cb_bytes, grid, smem_bytes, stream);
+    }
     if (pair) {
         if (f32 || grid % 2 != 0) return cudaErrorInvalidValue;
         return im2col ? launch_cb<false, true, true>(p, cb_bytes, grid, smem_bytes, stream)

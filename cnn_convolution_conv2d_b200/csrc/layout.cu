@@ -14,6 +14,7 @@ namespace conv2d_b200 {
 namespace {
 
 constexpr int kThreads = 256;
+constexpr int kBiasRows = 512;  // rows of channels-last dy summed per block of the bias gradient
 
 inline int grid_for(long long work, int per_block = kThreads) {
     long long g = (work + per_block - 1) / per_block;
@@ -401,6 +402,192 @@ __global__ void splitk_reduce_kernel(const float *__restrict__ ws, const void *_
     }
 }
 
+
+// --- weight gradient: dW[oc][c][kh][kw] = sum_s ws[s][oc][tap][c] (the splits of the
+// tensor-core kernel's reduction over pixels), c < Cin_g, written OIHW in the weight type.
+template <bool kF32>
+__global__ void wgrad_reduce_kernel(const float *__restrict__ ws, void *__restrict__ dw, int Cout, int Cin_g,
+                                    int taps, int Cpg, int splits) {
+    const long long total = static_cast<long long>(Cout) * Cin_g * taps;
+    const long long slice = static_cast<long long>(Cout) * taps * Cpg;
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const int tap = static_cast<int>(i % taps);
+        const long long r = i / taps;
+        const int c = static_cast<int>(r % Cin_g);
+        const long long oc = r / Cin_g;
+        const float *src = ws + (oc * taps + tap) * Cpg + c;
+        float acc = 0.f;
+        for (int s = 0; s < splits; ++s) acc += src[s * slice];
+        if (kF32)
+            static_cast<float *>(dw)[i] = acc;
+        else
+            static_cast<__nv_bfloat16 *>(dw)[i] = __float2bfloat16_rn(acc);
+    }
+}
+
+// --- bias gradient, first pass: partial[b][c] = sum over a block of rows of dy.
+// Channels-last dy is [rows][C]; each block sums `rows_per_block` rows, one thread per
+// channel (consecutive threads read consecutive channels: coalesced).
+template <bool kF32>
+__global__ void bias_grad_rows_kernel(const void *__restrict__ dy, float *__restrict__ partial, long long rows,
+                                      int C, int rows_per_block) {
+    const long long r0 = static_cast<long long>(blockIdx.x) * rows_per_block;
+    const long long r1 = r0 + rows_per_block < rows ? r0 + rows_per_block : rows;
+    for (int c = threadIdx.x; c < C; c += blockDim.x) {
+        float acc = 0.f;
+        for (long long r = r0; r < r1; ++r) {
+            const long long at = r * C + c;
+            acc += kF32 ? static_cast<const float *>(dy)[at]
+                        : __bfloat162float(static_cast<const __nv_bfloat16 *>(dy)[at]);
+        }
+        partial[static_cast<long long>(blockIdx.x) * C + c] = acc;
+    }
+}
+
+// NCHW dy is [N][C][plane]: one warp sums one (n, c) plane; partial[n][c].
+template <bool kF32>
+__global__ void bias_grad_planes_kernel(const void *__restrict__ dy, float *__restrict__ partial, int N, int C,
+                                        long long plane) {
+    const int lane = threadIdx.x & 31;
+    const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x / 32);
+    for (long long wi = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) / 32;
+         wi < static_cast<long long>(N) * C; wi += warps) {
+        float acc = 0.f;
+        for (long long k = lane; k < plane; k += 32) {
+            const long long at = wi * plane + k;
+            acc += kF32 ? static_cast<const float *>(dy)[at]
+                        : __bfloat162float(static_cast<const __nv_bfloat16 *>(dy)[at]);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0) partial[wi] = acc;
+    }
+}
+
+// Second pass: db[c] = sum_b partial[b][c], in the bias type.
+template <bool kF32>
+__global__ void bias_grad_final_kernel(const float *__restrict__ partial, void *__restrict__ db, int blocks, int C) {
+    for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < C; c += gridDim.x * blockDim.x) {
+        float acc = 0.f;
+        for (int b = 0; b < blocks; ++b) acc += partial[static_cast<long long>(b) * C + c];
+        if (kF32)
+            static_cast<float *>(db)[c] = acc;
+        else
+            static_cast<__nv_bfloat16 *>(db)[c] = __float2bfloat16_rn(acc);
+    }
+}
+
+// --- zero insertion for the input gradient of a strided convolution: dyz (Hz x Wz) has
+// dy[n][c][oh][ow] at (oh*s, ow*s) and zeros elsewhere, in dy's layout.
+template <int kElt>
+__global__ void zero_insert_kernel(const void *__restrict__ dy, void *__restrict__ dyz, int N, int C, int Ho, int Wo,
+                                   int Hz, int Wz, int s, int nchw) {
+    using T = typename Word<kElt>::T;
+    const T *src = static_cast<const T *>(dy);
+    T *dst = static_cast<T *>(dyz);
+    const long long total = static_cast<long long>(N) * C * Hz * Wz;
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        long long n, c, j, k;
+        if (nchw) {
+            k = i % Wz;
+            long long r = i / Wz;
+            j = r % Hz;
+            r /= Hz;
+            c = r % C;
+            n = r / C;
+        } else {
+            c = i % C;
+            long long r = i / C;
+            k = r % Wz;
+            r /= Wz;
+            j = r % Hz;
+            n = r / Hz;
+        }
+        T v = T(0);
+        if (j % s == 0 && k % s == 0 && j / s < Ho && k / s < Wo) {
+            const long long oh = j / s, ow = k / s;
+            v = nchw ? src[((n * C + c) * Ho + oh) * Wo + ow] : src[((n * Ho + oh) * Wo + ow) * C + c];
+        }
+        dst[i] = v;
+    }
+}
+
+// --- weights of the input gradient: the kernel of the transposed convolution, packed
+// like pack_weight_kernel's output for a convolution with O = C_in output channels and
+// R = C_out/groups reduction channels per group: entry (o, kh, kw, c) holds
+// w[g*R + cl][o % Cin_g][Kh-1-kh][Kw-1-kw] with g = o / Cin_g (spatially flipped,
+// input and output channels exchanged within each group), zero for padding channels
+// and, with groups merged gm at a time, outside the diagonal block.
+template <int kElt>
+__global__ void pack_weight_t_kernel(const void *__restrict__ w, void *__restrict__ wp, int O, int R, int Cin_g,
+                                     int gm, int Kh, int Kw, int Cpg) {
+    using T = typename Word<kElt>::T;
+    const T *s = static_cast<const T *>(w);
+    T *d = static_cast<T *>(wp);
+    const long long total = static_cast<long long>(O) * Kh * Kw * Cpg;
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const int c = static_cast<int>(i % Cpg);
+        long long r = i / Cpg;
+        const int kw = static_cast<int>(r % Kw);
+        r /= Kw;
+        const int kh = static_cast<int>(r % Kh);
+        const long long o = r / Kh;
+        const long long g = o / Cin_g;
+        const int j = static_cast<int>(g % gm);
+        const int cl = c - j * R;
+        T v = T(0);
+        if (cl >= 0 && cl < R)
+            v = s[(((g * R + cl) * Cin_g + (o - g * Cin_g)) * Kh + (Kh - 1 - kh)) * Kw + (Kw - 1 - kw)];
+        d[i] = v;
+    }
+}
+
+// --- weight gradient for few channels per group (depthwise and the like), on the CUDA
+// cores: one thread per (split, oc, tap, c), c fastest, summing dy * x over the split's
+// rows of output pixels (lpnh §5.1's formula); x and dy channels-last.  Partial sums go to
+// ws[split][oc][tap][c] (Cpg = Cin_g), reduced by wgrad_reduce_kernel.
+template <bool kF32>
+__global__ void wgrad_direct_kernel(const void *__restrict__ x, const void *__restrict__ dy, float *__restrict__ ws,
+                                    int N, int C_in, int H, int W, int C_out, int Ho, int Wo, int Kh, int Kw,
+                                    int stride, int pad, int dilation, int groups, int splits) {
+    const int cin_g = C_in / groups, cout_g = C_out / groups, taps = Kh * Kw;
+    const long long per_split = static_cast<long long>(C_out) * taps * cin_g;
+    const long long total = per_split * splits;
+    const long long rows = static_cast<long long>(N) * Ho;
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const int split = static_cast<int>(i / per_split);
+        long long r = i - split * per_split;
+        const int c = static_cast<int>(r % cin_g);
+        r /= cin_g;
+        const int tap = static_cast<int>(r % taps);
+        const int oc = static_cast<int>(r / taps);
+        const int kh = tap / Kw, kw = tap - (tap / Kw) * Kw;
+        const int ic = (oc / cout_g) * cin_g + c;
+        const long long r0 = rows * split / splits, r1 = rows * (split + 1) / splits;
+        float acc = 0.f;
+        for (long long row = r0; row < r1; ++row) {
+            const int n = static_cast<int>(row / Ho), oh = static_cast<int>(row - static_cast<long long>(n) * Ho);
+            const int ih = oh * stride + kh * dilation - pad;
+            if (ih < 0 || ih >= H) continue;
+            for (int ow = 0; ow < Wo; ++ow) {
+                const int iw = ow * stride + kw * dilation - pad;
+                if (iw < 0 || iw >= W) continue;
+                const long long dyi = (row * Wo + ow) * C_out + oc;
+                const long long xi = ((static_cast<long long>(n) * H + ih) * W + iw) * C_in + ic;
+                if (kF32)
+                    acc = fmaf(static_cast<const float *>(dy)[dyi], static_cast<const float *>(x)[xi], acc);
+                else
+                    acc = fmaf(__bfloat162float(static_cast<const __nv_bfloat16 *>(dy)[dyi]),
+                               __bfloat162float(static_cast<const __nv_bfloat16 *>(x)[xi]), acc);
+            }
+        }
+        ws[((static_cast<long long>(split) * C_out + oc) * taps + tap) * cin_g + c] = acc;
+    }
+}
 }  // namespace
 
 cudaError_t launch_nchw_to_nhwc(const void *src, void *dst, int N, int C, int H, int W,
@@ -504,6 +691,81 @@ cudaError_t launch_splitk_reduce(const float *ws, const void *bias, void *y, int
     else
         splitk_reduce_kernel<false><<<grid_for(total), kThreads, 0, s>>>(ws, bias, y, M, Cout, HoWo,
                                                                          splits, nchw);
+    return cudaGetLastError();
+}
+
+
+cudaError_t launch_wgrad_reduce(const float *ws, void *dw, int Cout, int Cin_g, int taps, int Cpg, int splits,
+                                bool f32, cudaStream_t s) {
+    const long long total = static_cast<long long>(Cout) * Cin_g * taps;
+    if (f32)
+        wgrad_reduce_kernel<true><<<grid_for(total), kThreads, 0, s>>>(ws, dw, Cout, Cin_g, taps, Cpg, splits);
+    else
+        wgrad_reduce_kernel<false><<<grid_for(total), kThreads, 0, s>>>(ws, dw, Cout, Cin_g, taps, Cpg, splits);
+    return cudaGetLastError();
+}
+
+int bias_grad_partials(long long rows, int C, int N, bool nchw) {
+    return nchw ? N : static_cast<int>((rows + kBiasRows - 1) / kBiasRows);
+}
+
+cudaError_t launch_bias_grad(const void *dy, float *partial, void *db, int N, int C, long long plane, bool nchw,
+                             bool f32, cudaStream_t s) {
+    const long long rows = static_cast<long long>(N) * plane;
+    const int blocks = bias_grad_partials(rows, C, N, nchw);
+    if (nchw) {
+        const int grid = grid_for(static_cast<long long>(N) * C * 32);
+        if (f32)
+            bias_grad_planes_kernel<true><<<grid, kThreads, 0, s>>>(dy, partial, N, C, plane);
+        else
+            bias_grad_planes_kernel<false><<<grid, kThreads, 0, s>>>(dy, partial, N, C, plane);
+    } else {
+        if (f32)
+            bias_grad_rows_kernel<true><<<blocks, kThreads, 0, s>>>(dy, partial, rows, C, kBiasRows);
+        else
+            bias_grad_rows_kernel<false><<<blocks, kThreads, 0, s>>>(dy, partial, rows, C, kBiasRows);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    if (f32)
+        bias_grad_final_kernel<true><<<grid_for(C), kThreads, 0, s>>>(partial, db, blocks, C);
+    else
+        bias_grad_final_kernel<false><<<grid_for(C), kThreads, 0, s>>>(partial, db, blocks, C);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_zero_insert(const void *dy, void *dyz, int N, int C, int Ho, int Wo, int Hz, int Wz, int stride,
+                               bool nchw, int elt, cudaStream_t s) {
+    const long long total = static_cast<long long>(N) * C * Hz * Wz;
+    if (elt == 2)
+        zero_insert_kernel<2><<<grid_for(total), kThreads, 0, s>>>(dy, dyz, N, C, Ho, Wo, Hz, Wz, stride, nchw ? 1 : 0);
+    else
+        zero_insert_kernel<4><<<grid_for(total), kThreads, 0, s>>>(dy, dyz, N, C, Ho, Wo, Hz, Wz, stride, nchw ? 1 : 0);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_pack_weight_t(const void *w, void *wp, int O, int R, int Cin_g, int gm, int Kh, int Kw, int Cpg,
+                                 int elt, cudaStream_t s) {
+    const long long total = static_cast<long long>(O) * Kh * Kw * Cpg;
+    if (elt == 2)
+        pack_weight_t_kernel<2><<<grid_for(total), kThreads, 0, s>>>(w, wp, O, R, Cin_g, gm, Kh, Kw, Cpg);
+    else
+        pack_weight_t_kernel<4><<<grid_for(total), kThreads, 0, s>>>(w, wp, O, R, Cin_g, gm, Kh, Kw, Cpg);
+    return cudaGetLastError();
+}
+
+
+cudaError_t launch_wgrad_direct(const void *x, const void *dy, float *ws, int N, int C_in, int H, int W, int C_out,
+                                int Ho, int Wo, int Kh, int Kw, int stride, int pad, int dilation, int groups,
+                                int splits, bool f32, cudaStream_t s) {
+    const long long total = static_cast<long long>(C_out) * Kh * Kw * (C_in / groups) * splits;
+    const int grid = grid_for(total, 128);
+    if (f32)
+        wgrad_direct_kernel<true><<<grid, 128, 0, s>>>(x, dy, ws, N, C_in, H, W, C_out, Ho, Wo, Kh, Kw, stride, pad,
+                                                      dilation, groups, splits);
+    else
+        wgrad_direct_kernel<false><<<grid, 128, 0, s>>>(x, dy, ws, N, C_in, H, W, C_out, Ho, Wo, Kh, Kw, stride,
+                                                       pad, dilation, groups, splits);
     return cudaGetLastError();
 }
 

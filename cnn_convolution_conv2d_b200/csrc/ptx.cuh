@@ -147,6 +147,19 @@ __device__ __forceinline__ void tma_load_im2col_4d(void *dst, const CUtensorMap 
         : "memory");
 }
 
+// im2col-mode load of a 5-D channels-last tensor (c, w, h, d, n): the volumetric form,
+// with filter-tap offsets (off_w, off_h, off_d).
+__device__ __forceinline__ void tma_load_im2col_5d(void *dst, const CUtensorMap *map, uint64_t *bar, int c,
+                                                   int w, int h, int d, int n, uint16_t off_w, uint16_t off_h,
+                                                   uint16_t off_d) {
+    asm volatile(
+        "cp.async.bulk.tensor.5d.shared::cluster.global.im2col.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2], {%8, %9, %10};" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(c), "r"(w), "r"(h), "r"(d), "r"(n),
+        "h"(off_w), "h"(off_h), "h"(off_d)
+        : "memory");
+}
+
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar,
                                             int x, int y) {
     asm volatile(
@@ -185,6 +198,17 @@ __device__ __forceinline__ void tma_load_im2col_4d_pair(void *dst, const CUtenso
         " [%0], [%1, {%3, %4, %5, %6}], [%2], {%7, %8};" ::"r"(smem_addr(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c), "r"(w), "r"(h), "r"(n),
         "h"(off_w), "h"(off_h)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_load_im2col_5d_pair(void *dst, const CUtensorMap *map, uint32_t bar_cluster,
+                                                        int c, int w, int h, int d, int n, uint16_t off_w,
+                                                        uint16_t off_h, uint16_t off_d) {
+    asm volatile(
+        "cp.async.bulk.tensor.5d.shared::cluster.global.im2col.mbarrier::complete_tx::bytes.cta_group::2"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2], {%8, %9, %10};" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c), "r"(w), "r"(h), "r"(d), "r"(n),
+        "h"(off_w), "h"(off_h), "h"(off_d)
         : "memory");
 }
 
@@ -393,6 +417,14 @@ __device__ __forceinline__ void tmem_ld_x16(uint32_t taddr, uint32_t (&r)[16]) {
           "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
           "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
         : "r"(taddr));
+}
+
+// 32 lanes x 32 bits, 8 consecutive columns: thread i of the warp receives row
+// (lane base + i), columns [col, col + 8).
+__device__ __forceinline__ void tmem_ld_x8(uint32_t taddr, uint32_t (&r)[8]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr));
 }
 
 // 32 lanes x 32 bits, 8 / 32 consecutive columns: thread i of the warp writes row

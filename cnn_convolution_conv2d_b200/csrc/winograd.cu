@@ -1,0 +1,337 @@
+// winograd.cu -- the minimal-filtering (Winograd) form of the 3x3, stride-1, unit-
+// dilation convolution: F(2x2, 3x3) and F(4x4, 3x3).
+//
+// The im2col/GEMM tutorial (zskr.cn/news/1820658) §5.1 describes it: an m x m block of
+// outputs of an r x r filter needs m^2 r^2 multiplications directly but only (m+r-1)^2
+// after linear transforms of the input tile and the filter (36 -> 16 for F(2x2,3x3),
+// 2.25x), and it applies only to small filters with stride 1 and dilation 1, with larger
+// rounding error from the transforms; the "手撕 Conv2D" page (lpnh.cn/news/2493075) §7
+// names F(2,3) and F(4,3).  The transforms are the published ones of Lavin & Gray,
+// "Fast Algorithms for Convolutional Neural Networks" (2016):
+//     Y = A^T [ (G g G^T) o (B^T d B) ] A
+// with d an alpha x alpha input tile (alpha = m + 2), g the 3 x 3 filter and o the
+// elementwise product.  Summed over input channels, the elementwise product becomes,
+// for each of the alpha^2 tile positions xi, one matrix product
+//     M[xi][tile][oc] = sum_c V[xi][tile][c] * U[xi][oc][c],
+// which runs here on the same tensor-core kernel as the forward pass (a grouped 1x1
+// convolution with alpha^2 groups over the transformed tiles).  The three steps:
+//   1. input transform (this file): V = B^T d B per tile and channel vector, written
+//      channels-last as [tile][xi][Cpg] (Cpg: channels padded to 16 bytes), in the
+//      input dtype -- one rounding for bf16;
+//   2. the product on the tensor cores, fp32 results [tile][xi][oc];
+//   3. output transform (this file): Y = A^T M A + bias per tile and output channel
+//      vector, one rounding to the output dtype, written NHWC or NCHW.
+// U = G g G^T is computed once when the weights are packed.  All three kernels are
+// memory-bound CUDA-core loops; the transformed tensors (V, M) are alpha^2/m^2 times
+// the size of x and y, which is the cost of not fusing the transforms into the product.
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+
+namespace conv2d_b200 {
+namespace {
+
+constexpr int kWgThreads256 = 256;
+
+inline int wino_grid(long long work) {
+    long long g = (work + kWgThreads256 - 1) / kWgThreads256;
+    if (g < 1) g = 1;
+    if (g > 148LL * 32) g = 148LL * 32;
+    return static_cast<int>(g);
+}
+
+// B^T rows (alpha x alpha), G (alpha x 3) and A^T (m x alpha) of F(m x m, 3 x 3).
+template <int kM>
+struct WinoMats;
+
+template <>
+struct WinoMats<2> {
+    static constexpr int kA = 4;
+    __device__ static float bt(int i, int j) {
+        constexpr float t[4][4] = {{1, 0, -1, 0}, {0, 1, 1, 0}, {0, -1, 1, 0}, {0, 1, 0, -1}};
+        return t[i][j];
+    }
+    __device__ static float g(int i, int j) {
+        constexpr float t[4][3] = {{1, 0, 0}, {0.5f, 0.5f, 0.5f}, {0.5f, -0.5f, 0.5f}, {0, 0, 1}};
+        return t[i][j];
+    }
+    __device__ static float at(int i, int j) {
+        constexpr float t[2][4] = {{1, 1, 1, 0}, {0, 1, -1, -1}};
+        return t[i][j];
+    }
+};
+
+template <>
+struct WinoMats<4> {
+    static constexpr int kA = 6;
+    __device__ static float bt(int i, int j) {
+        constexpr float t[6][6] = {{4, 0, -5, 0, 1, 0},  {0, -4, -4, 1, 1, 0}, {0, 4, -4, -1, 1, 0},
+                                   {0, -2, -1, 2, 1, 0}, {0, 2, -1, -2, 1, 0}, {0, 4, 0, -5, 0, 1}};
+        return t[i][j];
+    }
+    __device__ static float g(int i, int j) {
+        constexpr float t[6][3] = {{1.f / 4, 0, 0},
+                                   {-1.f / 6, -1.f / 6, -1.f / 6},
+                                   {-1.f / 6, 1.f / 6, -1.f / 6},
+                                   {1.f / 24, 1.f / 12, 1.f / 6},
+                                   {1.f / 24, -1.f / 12, 1.f / 6},
+                                   {0, 0, 1}};
+        return t[i][j];
+    }
+    __device__ static float at(int i, int j) {
+        constexpr float t[4][6] = {{1, 1, 1, 1, 1, 0}, {0, 1, -1, 2, -2, 0}, {0, 1, 1, 4, 4, 0}, {0, 1, -1, 8, -8, 1}};
+        return t[i][j];
+    }
+};
+
+template <bool kF32>
+__device__ __forceinline__ float ld1(const void *p, long long i) {
+    if constexpr (kF32)
+        return static_cast<const float *>(p)[i];
+    else
+        return __bfloat162float(static_cast<const __nv_bfloat16 *>(p)[i]);
+}
+
+template <bool kF32>
+__device__ __forceinline__ void st1(void *p, long long i, float v) {
+    if constexpr (kF32)
+        static_cast<float *>(p)[i] = v;
+    else
+        static_cast<__nv_bfloat16 *>(p)[i] = __float2bfloat16_rn(v);
+}
+
+// 1. V[tile][xi][c] = (B^T d B)[xi] for each tile (n, th, tw) and channel c < Cpg (zero
+// for c >= C): d[a][b] = x[n][th*m - pad + a][tw*m - pad + b][c], zero outside the image.
+// One thread per (tile, group of kV consecutive channels).
+template <bool kF32, int kM, int kV>
+__global__ void __launch_bounds__(kWgThreads256) wino_input_kernel(const void *__restrict__ x, void *__restrict__ v,
+                                                                 int N, int C, int H, int W, int Cpg, int TH, int TW,
+                                                                 int pad, int nchw) {
+    using Mt = WinoMats<kM>;
+    constexpr int kA = Mt::kA;
+    const int cgroups = Cpg / kV;
+    const long long total = static_cast<long long>(N) * TH * TW * cgroups;
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const int cg = static_cast<int>(i % cgroups);
+        const long long tile = i / cgroups;
+        const int tw = static_cast<int>(tile % TW);
+        const long long r = tile / TW;
+        const int th = static_cast<int>(r % TH);
+        const int n = static_cast<int>(r / TH);
+        const int c0 = cg * kV;
+        const int h0 = th * kM - pad, w0 = tw * kM - pad;
+        // t = B^T d, one input column at a time
+        float t[kA][kA][kV];
+#pragma unroll
+        for (int b = 0; b < kA; ++b) {
+            float d[kA][kV];
+            const int iw = w0 + b;
+#pragma unroll
+            for (int k = 0; k < kA; ++k) {
+                const int ih = h0 + k;
+                const bool in = ih >= 0 && ih < H && iw >= 0 && iw < W;
+#pragma unroll
+                for (int e = 0; e < kV; ++e) {
+                    const int c = c0 + e;
+                    float val = 0.f;
+                    if (in && c < C) {
+                        const long long at = nchw ? ((static_cast<long long>(n) * C + c) * H + ih) * W + iw
+                                                  : ((static_cast<long long>(n) * H + ih) * W + iw) * C + c;
+                        val = ld1<kF32>(x, at);
+                    }
+                    d[k][e] = val;
+                }
+            }
+#pragma unroll
+            for (int a = 0; a < kA; ++a)
+#pragma unroll
+                for (int e = 0; e < kV; ++e) {
+                    float sum = 0.f;
+#pragma unroll
+                    for (int k = 0; k < kA; ++k) sum += Mt::bt(a, k) * d[k][e];
+                    t[a][b][e] = sum;
+                }
+        }
+        // V = t B
+        const long long base = tile * kA * kA * Cpg + c0;
+#pragma unroll
+        for (int a = 0; a < kA; ++a)
+#pragma unroll
+            for (int b = 0; b < kA; ++b)
+#pragma unroll
+                for (int e = 0; e < kV; ++e) {
+                    float s = 0.f;
+#pragma unroll
+                    for (int k = 0; k < kA; ++k) s += t[a][k][e] * Mt::bt(b, k);
+                    st1<kF32>(v, base + static_cast<long long>(a * kA + b) * Cpg + e, s);
+                }
+    }
+}
+
+// U packed for the product: rows o = xi * C_out + oc (alpha^2 groups of C_out), each
+// row Cpgw entries; entry c of row o holds (G g[oc][c] G^T)[xi] for c < C, zero for the
+// padding channels and -- with groups merged gm at a time -- outside the diagonal block.
+template <bool kF32, int kM>
+__global__ void __launch_bounds__(kWgThreads256) wino_weight_kernel(const void *__restrict__ w, void *__restrict__ u,
+                                                                  int C_out, int C, int Cpg, int gm, int Cpgw) {
+    using Mt = WinoMats<kM>;
+    constexpr int kA = Mt::kA;
+    const long long total = static_cast<long long>(kA) * kA * C_out * Cpgw;
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const int cw = static_cast<int>(i % Cpgw);
+        const long long o = i / Cpgw;
+        const int xi = static_cast<int>(o / C_out);
+        const int oc = static_cast<int>(o - static_cast<long long>(xi) * C_out);
+        const int j = xi % gm;
+        const int c = cw - j * Cpg;
+        float val = 0.f;
+        if (c >= 0 && c < C) {
+            const int a = xi / kA, b = xi - (xi / kA) * kA;
+            const long long g0 = (static_cast<long long>(oc) * C + c) * 9;
+#pragma unroll
+            for (int p = 0; p < 3; ++p)
+#pragma unroll
+                for (int q = 0; q < 3; ++q) val += Mt::g(a, p) * ld1<kF32>(w, g0 + p * 3 + q) * Mt::g(b, q);
+        }
+        st1<kF32>(u, i, val);
+    }
+}
+
+// 3. y[n][th*m + i][tw*m + j][oc] = bias[oc] + (A^T M A)[i][j], M[xi] summed over the
+// product's splits (fp32 partial sums [split][tile][alpha^2 * C_out]).
+template <bool kF32, int kM, int kV>
+__global__ void __launch_bounds__(kWgThreads256) wino_output_kernel(const float *__restrict__ mp,
+                                                                  const void *__restrict__ bias, void *__restrict__ y,
+                                                                  int N, int C_out, int Ho, int Wo, int TH, int TW,
+                                                                  int splits, int nchw) {
+    using Mt = WinoMats<kM>;
+    constexpr int kA = Mt::kA;
+    const int cgroups = (C_out + kV - 1) / kV;
+    const long long tiles = static_cast<long long>(N) * TH * TW;
+    const long long total = tiles * cgroups;
+    const long long row = static_cast<long long>(kA) * kA * C_out;
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const int cg = static_cast<int>(i % cgroups);
+        const long long tile = i / cgroups;
+        const int tw = static_cast<int>(tile % TW);
+        const long long r = tile / TW;
+        const int th = static_cast<int>(r % TH);
+        const int n = static_cast<int>(r / TH);
+        const int c0 = cg * kV;
+        // t = A^T M, one column of M (summed over the splits) at a time
+        float t[kM][kA][kV];
+#pragma unroll
+        for (int b = 0; b < kA; ++b) {
+            float m[kA][kV];
+#pragma unroll
+            for (int k = 0; k < kA; ++k)
+#pragma unroll
+                for (int e = 0; e < kV; ++e) {
+                    float sum = 0.f;
+                    if (c0 + e < C_out)
+                        for (int sp = 0; sp < splits; ++sp)
+                            sum += mp[(sp * tiles + tile) * row + static_cast<long long>(k * kA + b) * C_out + c0 + e];
+                    m[k][e] = sum;
+                }
+#pragma unroll
+            for (int a = 0; a < kM; ++a)
+#pragma unroll
+                for (int e = 0; e < kV; ++e) {
+                    float sum = 0.f;
+#pragma unroll
+                    for (int k = 0; k < kA; ++k) sum += Mt::at(a, k) * m[k][e];
+                    t[a][b][e] = sum;
+                }
+        }
+        float bv[kV];
+#pragma unroll
+        for (int e = 0; e < kV; ++e) bv[e] = (bias && c0 + e < C_out) ? ld1<kF32>(bias, c0 + e) : 0.f;
+#pragma unroll
+        for (int a = 0; a < kM; ++a) {
+            const int oh = th * kM + a;
+            if (oh >= Ho) break;
+#pragma unroll
+            for (int b = 0; b < kM; ++b) {
+                const int ow = tw * kM + b;
+                if (ow >= Wo) break;
+#pragma unroll
+                for (int e = 0; e < kV; ++e) {
+                    const int oc = c0 + e;
+                    if (oc >= C_out) break;
+                    float s = bv[e];
+#pragma unroll
+                    for (int k = 0; k < kA; ++k) s += t[a][k][e] * Mt::at(b, k);
+                    const long long at = nchw ? ((static_cast<long long>(n) * C_out + oc) * Ho + oh) * Wo + ow
+                                              : ((static_cast<long long>(n) * Ho + oh) * Wo + ow) * C_out + oc;
+                    st1<kF32>(y, at, s);
+                }
+            }
+        }
+    }
+}
+
+template <bool kF32, int kM>
+cudaError_t input_t(const void *x, void *v, int N, int C, int H, int W, int Cpg, int TH, int TW, int pad, bool nchw,
+                    cudaStream_t s) {
+    constexpr int kV = kM == 2 ? 4 : 2;  // channels per thread
+    const long long work = static_cast<long long>(N) * TH * TW * (Cpg / kV);
+    wino_input_kernel<kF32, kM, kV><<<wino_grid(work), kWgThreads256, 0, s>>>(x, v, N, C, H, W, Cpg, TH, TW, pad,
+                                                                            nchw ? 1 : 0);
+    return cudaGetLastError();
+}
+
+template <bool kF32, int kM>
+cudaError_t output_t(const float *mp, const void *bias, void *y, int N, int C_out, int Ho, int Wo, int TH, int TW,
+                     int splits, bool nchw, cudaStream_t s) {
+    constexpr int kV = kM == 2 ? 4 : 2;
+    const long long work = static_cast<long long>(N) * TH * TW * ((C_out + kV - 1) / kV);
+    wino_output_kernel<kF32, kM, kV><<<wino_grid(work), kWgThreads256, 0, s>>>(mp, bias, y, N, C_out, Ho, Wo, TH, TW,
+                                                                             splits, nchw ? 1 : 0);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_wino_input(const void *x, void *v, int N, int C, int H, int W, int Cpg, int TH, int TW, int pad,
+                              int m, bool nchw, bool f32, cudaStream_t s) {
+    if (Cpg % 4 != 0) return cudaErrorInvalidValue;  // a multiple of both vector widths
+    if (m == 2) return f32 ? input_t<true, 2>(x, v, N, C, H, W, Cpg, TH, TW, pad, nchw, s)
+                           : input_t<false, 2>(x, v, N, C, H, W, Cpg, TH, TW, pad, nchw, s);
+    if (m == 4) return f32 ? input_t<true, 4>(x, v, N, C, H, W, Cpg, TH, TW, pad, nchw, s)
+                           : input_t<false, 4>(x, v, N, C, H, W, Cpg, TH, TW, pad, nchw, s);
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_wino_weight(const void *w, void *u, int C_out, int C, int Cpg, int gm, int m, bool f32,
+                               cudaStream_t s) {
+    const int a = m + 2;
+    const long long work = static_cast<long long>(a) * a * C_out * Cpg * gm;
+    if (m == 2) {
+        if (f32)
+            wino_weight_kernel<true, 2><<<wino_grid(work), kWgThreads256, 0, s>>>(w, u, C_out, C, Cpg, gm, Cpg * gm);
+        else
+            wino_weight_kernel<false, 2><<<wino_grid(work), kWgThreads256, 0, s>>>(w, u, C_out, C, Cpg, gm, Cpg * gm);
+    } else if (m == 4) {
+        if (f32)
+            wino_weight_kernel<true, 4><<<wino_grid(work), kWgThreads256, 0, s>>>(w, u, C_out, C, Cpg, gm, Cpg * gm);
+        else
+            wino_weight_kernel<false, 4><<<wino_grid(work), kWgThreads256, 0, s>>>(w, u, C_out, C, Cpg, gm, Cpg * gm);
+    } else {
+        return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_wino_output(const float *mp, const void *bias, void *y, int N, int C_out, int Ho, int Wo, int TH,
+                               int TW, int splits, int m, bool nchw, bool f32, cudaStream_t s) {
+    if (m == 2) return f32 ? output_t<true, 2>(mp, bias, y, N, C_out, Ho, Wo, TH, TW, splits, nchw, s)
+                           : output_t<false, 2>(mp, bias, y, N, C_out, Ho, Wo, TH, TW, splits, nchw, s);
+    if (m == 4) return f32 ? output_t<true, 4>(mp, bias, y, N, C_out, Ho, Wo, TH, TW, splits, nchw, s)
+                           : output_t<false, 4>(mp, bias, y, N, C_out, Ho, Wo, TH, TW, splits, nchw, s);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace conv2d_b200

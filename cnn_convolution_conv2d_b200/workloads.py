@@ -129,3 +129,77 @@ def make_inputs(cfg: ConvConfig, seed: int | None = None) -> dict:
         x, w = bf16_round(x), bf16_round(w)
         b = None if b is None else bf16_round(b)
     return {"x": x, "w": w, "b": b}
+
+
+@dataclasses.dataclass(frozen=True)
+class Conv3dConfig:
+    """A 3-D convolution workload: x (N, C_in, D, H, W), w (C_out, C_in/groups, Kd, Kh, Kw)
+    ("PyTorch高维张量乘法与conv2d/conv3d维度语义解析" §5.1).  ``layout`` "nchw" means NCDHW,
+    "nhwc" NDHWC."""
+    name: str
+    N: int
+    C_in: int
+    D: int
+    H: int
+    W: int
+    C_out: int
+    Kd: int
+    Kh: int
+    Kw: int
+    stride: int = 1
+    pad: int = 0
+    dilation: int = 1
+    groups: int = 1
+    bias: bool = True
+    dtype: str = "bf16"
+    layout: str = "nhwc"
+    x_dist: tuple = ("normal", 1.0)
+    w_dist: tuple = ("normal", 1.0)
+    b_dist: tuple = ("normal", 1.0)
+    seed: int = 0
+
+    def _o(self, v, k):
+        return (v + 2 * self.pad - self.dilation * (k - 1) - 1) // self.stride + 1
+
+    @property
+    def Do(self) -> int:
+        return self._o(self.D, self.Kd)
+
+    @property
+    def Ho(self) -> int:
+        return self._o(self.H, self.Kh)
+
+    @property
+    def Wo(self) -> int:
+        return self._o(self.W, self.Kw)
+
+    def scaled(self, **kw) -> "Conv3dConfig":
+        return dataclasses.replace(self, **kw)
+
+
+CONFIGS3D = {
+    # the two layers of the network "PyTorch高维张量乘法与conv2d/conv3d维度语义解析" §6.2 runs:
+    # x (4, 3, 16, 64, 64) -> 16 channels, 3x3x3, stride 1, pad 1 -> 32 channels, stride 2
+    "conv3d_l1_bf16": Conv3dConfig("conv3d_l1_bf16", 4, 3, 16, 64, 64, 16, 3, 3, 3, 1, 1, 1, 1, True, "bf16",
+                                   "nchw", ("normal", 1.0), ("normal", 2.0 / 81), ("normal", 1.0), 7),
+    "conv3d_l2_bf16": Conv3dConfig("conv3d_l2_bf16", 4, 16, 16, 64, 64, 32, 3, 3, 3, 2, 1, 1, 1, True, "bf16",
+                                   "nhwc", ("normal", 1.0), ("normal", 2.0 / 432), ("normal", 1.0), 8),
+    # a wider video block of the same kind (64 channels, 16 frames of 56x56): the
+    # throughput workload of the 3-D path
+    "conv3d_video_bf16": Conv3dConfig("conv3d_video_bf16", 8, 64, 16, 56, 56, 64, 3, 3, 3, 1, 1, 1, 1, True, "bf16",
+                                      "nhwc", ("normal", 1.0), ("normal", 2.0 / 1728), ("normal", 1.0), 9),
+    "conv3d_video_f32": Conv3dConfig("conv3d_video_f32", 8, 64, 16, 56, 56, 64, 3, 3, 3, 1, 1, 1, 1, True, "f32",
+                                     "nhwc", ("normal", 1.0), ("normal", 2.0 / 1728), ("normal", 1.0), 9),
+}
+
+
+def make_inputs3d(cfg: Conv3dConfig, seed: int | None = None) -> dict:
+    """Seeded x (NCDHW), w (OIDHW) and bias as float32 (bf16-rounded for bf16 workloads)."""
+    rng = np.random.default_rng(cfg.seed if seed is None else seed)
+    x = _draw(rng, cfg.x_dist, (cfg.N, cfg.C_in, cfg.D, cfg.H, cfg.W))
+    w = _draw(rng, cfg.w_dist, (cfg.C_out, cfg.C_in // cfg.groups, cfg.Kd, cfg.Kh, cfg.Kw))
+    b = _draw(rng, cfg.b_dist, (cfg.C_out,)) if cfg.bias else None
+    if cfg.dtype == "bf16":
+        x, w = bf16_round(x), bf16_round(w)
+        b = None if b is None else bf16_round(b)
+    return {"x": x, "w": w, "b": b}

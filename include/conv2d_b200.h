@@ -214,6 +214,157 @@ int conv2d_forward_noalloc(const void *x, const void *w_packed, const void *bias
                            int stride, int pad, int dilation, int groups,
                            conv_dtype_t dtype, conv_layout_t layout, conv_stream_t stream);
 
+/* ------------------------------------------------------------ backward pass ---
+ * The gradients of a loss L with respect to the input, the weights and the bias of
+ * y = conv2d(x, w) + bias, given dy = dL/dy: the three formulas of the "手撕 Conv2D"
+ * page (lpnh.cn/news/2493075) §5.1 -- db[oc] = sum over n, oh, ow of dy;
+ * dW[oc][c][kh][kw] = sum over n, oh, ow of dy[n][oc][oh][ow] * x[n][c][oh*s + kh*d - p][ow*s + kw*d - p];
+ * dx = every dy scattered back, times its weight, onto the input positions of its
+ * window -- which the im2col/GEMM tutorial (zskr.cn/news/1820658) §3.3 writes as
+ * dW_row = dout_col X_col^T, db = sum of dout, dx = col2im(W_row^T dout_col).
+ * Shapes, dtypes, layouts and the shape arguments are those of conv2d_forward for the
+ * same convolution: dy has y's shape and layout, dx has x's.  Gradients are
+ * accumulated in fp32 (fp32: three TF32 products per multiply-add, as the forward
+ * pass) and rounded once to the dtype. */
+
+/* Bytes of the kernel conv2d_pack_weight_backward_data writes: C_in * Kh * Kw * Cpg
+ * elements of dtype with Cpg = C_out/groups rounded up to a multiple of 8 (bf16) / 4
+ * (fp32), times the group merge factor described at conv2d_packed_weight_size for a
+ * convolution of C_in output and C_out input channels. */
+int conv2d_packed_weight_backward_data_size(int C_out, int C_in, int Kh, int Kw, int groups,
+                                            conv_dtype_t dtype, size_t *bytes);
+
+/* Packs w_oihw (C_out, C_in/groups, Kh, Kw) for conv2d_backward_data: the kernel of the
+ * transposed convolution, w_t[ic][kh][kw][oc] = w[oc][ic][Kh-1-kh][Kw-1-kw] within each
+ * group (spatially flipped, input and output channels exchanged), in the packed
+ * channels-last layout.  Done once per weight; w_packed_t holds
+ * conv2d_packed_weight_backward_data_size() bytes and must not overlap w_oihw. */
+int conv2d_pack_weight_backward_data(const void *w_oihw, void *w_packed_t, int C_out, int C_in,
+                                     int Kh, int Kw, int groups, conv_dtype_t dtype,
+                                     conv_stream_t stream);
+
+/* Device scratch bytes conv2d_backward_data needs (0 when none). */
+int conv2d_backward_data_workspace_size(int N, int C_in, int H, int W, int C_out, int Kh, int Kw,
+                                        int stride, int pad, int dilation, int groups,
+                                        conv_dtype_t dtype, conv_layout_t layout, size_t *bytes);
+
+/* Input gradient dx (x's shape and layout) from dy (y's shape and layout): the
+ * transposed convolution, computed as a forward convolution of dy with the packed
+ * kernel of conv2d_pack_weight_backward_data, stride 1 and padding
+ * dilation*(K-1) - pad in each dimension, on the same tensor-core kernels as
+ * conv2d_forward (or the depthwise kernel).  For stride s > 1, dy is first expanded
+ * in the workspace with s-1 zero rows and columns between its rows and columns (so
+ * the product does s*s times the multiply-adds of the gradient's own count).
+ * Errors as conv2d_forward, plus CONV_ERR_UNSUPPORTED when the transposed
+ * convolution falls outside the kernels' addressing limits (padding beyond +-127). */
+int conv2d_backward_data(const void *dy, const void *w_packed_t, void *dx,
+                         int N, int C_in, int H, int W, int C_out, int Kh, int Kw,
+                         int stride, int pad, int dilation, int groups,
+                         conv_dtype_t dtype, conv_layout_t layout,
+                         void *workspace, size_t workspace_bytes, conv_stream_t stream);
+
+/* Device scratch bytes conv2d_backward_weight needs; with_bias != 0 includes the bias
+ * gradient's partial sums. */
+int conv2d_backward_weight_workspace_size(int N, int C_in, int H, int W, int C_out, int Kh,
+                                          int Kw, int stride, int pad, int dilation, int groups,
+                                          conv_dtype_t dtype, conv_layout_t layout, int with_bias,
+                                          size_t *bytes);
+
+/* Weight gradient dw (C_out, C_in/groups, Kh, Kw) -- the pages' OIHW layout -- and,
+ * when db is not NULL, the bias gradient db (C_out,), from x and dy.  With at least 32
+ * bytes of input channels per group the product dW_row = dout_col X_col^T runs on the
+ * tensor cores with its reduction over output pixels split across SMs (input patches
+ * staged by the tensor memory accelerator's im2col mode, never formed in memory);
+ * fewer channels per group (depthwise and the like) run on the CUDA cores.  Errors as
+ * conv2d_forward; the workspace must hold conv2d_backward_weight_workspace_size() bytes
+ * (with_bias = db != NULL). */
+int conv2d_backward_weight(const void *x, const void *dy, void *dw, void *db,
+                           int N, int C_in, int H, int W, int C_out, int Kh, int Kw,
+                           int stride, int pad, int dilation, int groups,
+                           conv_dtype_t dtype, conv_layout_t layout,
+                           void *workspace, size_t workspace_bytes, conv_stream_t stream);
+
+/* Device scratch bytes conv2d_backward_bias needs (partial sums). */
+int conv2d_backward_bias_workspace_size(int N, int C_out, int Ho, int Wo, conv_layout_t layout,
+                                        size_t *bytes);
+
+/* Bias gradient alone: db[oc] = sum of dy[n][oc][oh][ow] over n, oh, ow (lpnh §5.1),
+ * summed in fp32 and rounded once to dtype.  dy is (N, C_out, Ho, Wo) in `layout`. */
+int conv2d_backward_bias(const void *dy, void *db, int N, int C_out, int Ho, int Wo,
+                         conv_dtype_t dtype, conv_layout_t layout, void *workspace,
+                         size_t workspace_bytes, conv_stream_t stream);
+
+/* ------------------------------------------------------------------- conv3d ---
+ * The 3-D convolution forward pass of "PyTorch高维张量乘法与conv2d/conv3d维度语义解析"
+ * (pwwt.cn/news/6111401) §5.1: x (N, C_in, D, H, W), w (C_out, C_in/groups, Kd, Kh, Kw),
+ * y (N, C_out, Do, Ho, Wo); the kernel slides over depth, height and width alike, each
+ * output extent given by conv2d_output_size's formula (§6.2 applies it to D, H and W):
+ *     y[n][oc][od][oh][ow] = bias[oc] + sum_{c, kd, kh, kw}
+ *         x[n][g*C_in/groups + c][od*s + kd*d - p][oh*s + kh*d - p][ow*s + kw*d - p] * w[oc][c][kd][kh][kw],
+ * terms outside the volume dropped.  Stride, pad and dilation apply to all three
+ * directions.  layout CONV_NCHW means NCDHW tensors, CONV_NHWC means NDHWC.  The same
+ * implicit matrix product as conv2d_forward runs over output voxels, its input patches
+ * staged by the tensor memory accelerator's 5-D im2col mode.  Beyond conv2d_forward's
+ * errors: CONV_ERR_UNSUPPORTED when pad or pad - dilation*(K-1) lies outside
+ * [-16, 15] in any direction (the 5-D im2col addressing range). */
+
+/* Bytes of conv3d_pack_weight's output: C_out * Kd * Kh * Kw * Cpg elements of dtype, Cpg
+ * as for conv2d_packed_weight_size (group merging included, no few-channel images). */
+int conv3d_packed_weight_size(int C_out, int C_in, int Kd, int Kh, int Kw, int groups,
+                              conv_dtype_t dtype, size_t *bytes);
+
+/* Packs w_oidhw (C_out, C_in/groups, Kd, Kh, Kw) into (C_out, Kd, Kh, Kw, Cpg), each tap's
+ * input channels contiguous and zero-padded (the channels-last filter order). */
+int conv3d_pack_weight(const void *w_oidhw, void *w_packed, int C_out, int C_in, int Kd, int Kh,
+                       int Kw, int groups, conv_dtype_t dtype, conv_stream_t stream);
+
+/* Device scratch bytes conv3d_forward needs (channels-last copy of an NCDHW or
+ * channel-unaligned x, split partial sums). */
+int conv3d_workspace_size(int N, int C_in, int D, int H, int W, int C_out, int Kd, int Kh,
+                          int Kw, int stride, int pad, int dilation, int groups,
+                          conv_dtype_t dtype, conv_layout_t layout, size_t *bytes);
+
+/* The 3-D forward pass; arguments as conv2d_forward with the depth extents added. */
+int conv3d_forward(const void *x, const void *w_packed, const void *bias, void *y,
+                   int N, int C_in, int D, int H, int W, int C_out, int Kd, int Kh, int Kw,
+                   int stride, int pad, int dilation, int groups,
+                   conv_dtype_t dtype, conv_layout_t layout,
+                   void *workspace, size_t workspace_bytes, conv_stream_t stream);
+
+/* ----------------------------------------------------------------- Winograd ---
+ * The minimal-filtering form of a 3x3, stride-1, unit-dilation, ungrouped convolution
+ * that the im2col/GEMM tutorial (zskr.cn/news/1820658) §5.1 sets beside im2col + GEMM:
+ * F(m x m, 3 x 3) with m = 2 (16 multiplications per 2x2 output block instead of 36) or
+ * m = 4 (36 instead of 144), using the published transforms of Lavin & Gray (2016),
+ * Y = A^T [ (G g G^T) o (B^T d B) ] A over (m+2) x (m+2) input tiles.  The input
+ * transform, the (m+2)^2 channel products (on the tensor cores, fp32 results) and the
+ * output transform (+ bias, one rounding) run as three steps through the workspace.
+ * Results equal conv2d_forward's up to rounding; the transforms enlarge the rounding
+ * error, more for m = 4 (§5.1's numerical caveat).  Arguments as conv2d_forward for a
+ * 3x3 filter with stride 1, dilation 1 and groups 1; CONV_ERR_INVALID_ARG for m other
+ * than 2 or 4. */
+
+/* Bytes of conv2d_pack_weight_winograd's output: (m+2)^2 * C_out rows of C_in channels
+ * padded to 16 bytes (times the group merge factor of conv2d_packed_weight_size for
+ * C_out < 64), dtype elements. */
+int conv2d_winograd_packed_weight_size(int C_out, int C_in, int m, conv_dtype_t dtype, size_t *bytes);
+
+/* The transformed filters U = G g G^T of w_oihw (C_out, C_in, 3, 3), packed for the
+ * product.  Done once per weight. */
+int conv2d_pack_weight_winograd(const void *w_oihw, void *u_packed, int C_out, int C_in, int m,
+                                conv_dtype_t dtype, conv_stream_t stream);
+
+/* Device scratch bytes conv2d_forward_winograd needs: the transformed input, the fp32
+ * products and the product's own scratch. */
+int conv2d_winograd_workspace_size(int N, int C_in, int H, int W, int C_out, int pad, int m,
+                                   conv_dtype_t dtype, conv_layout_t layout, size_t *bytes);
+
+/* The forward pass of a 3x3 stride-1 convolution by F(m x m, 3 x 3). */
+int conv2d_forward_winograd(const void *x, const void *u_packed, const void *bias, void *y,
+                            int N, int C_in, int H, int W, int C_out, int pad, int m,
+                            conv_dtype_t dtype, conv_layout_t layout, void *workspace,
+                            size_t workspace_bytes, conv_stream_t stream);
+
 /* Measurement aid: when `start` and `stop` (cudaEvent_t handles the caller created
  * with timing enabled) are both non-NULL, every later forward call records `start`
  * on its stream immediately before launching its tensor-core kernel and `stop`

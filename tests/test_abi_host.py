@@ -16,7 +16,7 @@ HEADER = os.path.join(ROOT, "include", "conv2d_b200.h")
 def declared_functions():
     text = open(HEADER, encoding="utf-8").read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(conv2d_\w+)\s*\(", text, flags=re.M)))
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(conv[23]d_\w+)\s*\(", text, flags=re.M)))
 
 
 @pytest.fixture(scope="module")
@@ -169,7 +169,11 @@ def test_plan_for_the_workloads_on_a_148_sm_device(lib):
     p3 = _plan((64, 256, 56, 56, 256, 3, 3, 1, 1, 1, 1), sms=148)    # 3x3: hardware im2col, pairs
     assert (p3["kernel"], p3["pair"], p3["a_load"], p3["BN"], p3["units"]) == ("igemm", 1, "im2col", 256, 784)
     stem = _plan((32, 3, 224, 224, 64, 7, 7, 2, 3, 1, 1), layout="nchw", sms=148)
-    assert (stem["kernel"], stem["halo"], stem["tma_out"], stem["BN"], stem["workspace"]) == ("gather", 1, 1, 64, 0)
+    # the transposed few-channel kernel: one output row (112 pixels) per tile
+    assert (stem["kernel"], stem["halo"], stem["BN"], stem["workspace"], stem["units"]) == \
+        ("gather_t", 1, 64, 0, 32 * 112)
+    nhwc_out = _plan((32, 3, 224, 224, 64, 7, 7, 2, 3, 1, 1), layout="nhwc", sms=148)
+    assert nhwc_out["kernel"] == "gather"                              # channels-last: the lane-per-pixel form
     assert stem["Kpad"] == 176                                         # 3 channels x 7 rows x 8 (7 taps + 1) -> 168 -> 176
     k7 = _plan((16, 512, 17, 17, 512, 7, 7, 1, 3, 1, 1), sms=148)     # 19 pair units < 74: single CTAs, split
     assert (k7["pair"], k7["splits"], k7["units"]) == (0, 2, 37 * 2 * 2)
@@ -218,7 +222,7 @@ def test_bench_mirror_of_the_gather_choice_agrees_with_the_library(lib):
         plan = cb.conv2d_describe_plan(c.N, c.C_in, c.H, c.W, c.C_out, c.Kh, c.Kw, c.stride, c.pad, c.dilation,
                                        c.groups, cb.CONV_BF16 if c.dtype == "bf16" else cb.CONV_F32, c.layout,
                                        sms=148)
-        assert (plan["kernel"] == "gather") == bench.uses_gather(c), name
+        assert (plan["kernel"] in ("gather", "gather_t")) == bench.uses_gather(c), name
         assert (plan["kernel"] == "depthwise") == bench.uses_depthwise(c), name
 
 
@@ -235,3 +239,57 @@ def test_depthwise_plans(lib):
     assert nchw["kernel"] == "depthwise" and nchw["xcopy"] == 1
     mult = _plan((2, 16, 8, 8, 32, 3, 3, 1, 1, 1, 16), sms=148)  # channel multiplier 2: general kernel
     assert mult["kernel"] == "igemm"
+
+
+def test_backward_sizes_on_the_host(lib):
+    """Sizes of the backward entry points, without a device."""
+    # transposed kernel: C_in output channels of C_out/groups (padded) reduction channels
+    assert cb.conv2d_packed_weight_backward_data_size(64, 32, 3, 3, 1, cb.CONV_BF16) == 32 * 9 * 64 * 2
+    assert cb.conv2d_packed_weight_backward_data_size(6, 3, 3, 3, 1, cb.CONV_BF16) == 3 * 9 * 8 * 2  # 6 -> 8
+    assert cb.conv2d_packed_weight_backward_data_size(12, 12, 3, 3, 12, cb.CONV_F32) == 12 * 9 * 4 * 4  # depthwise
+    # stride 2: the zero-inserted dy (Hz = H - d(K-1) + 2p = 9 - 2 + 2 = 9, same for W) comes first
+    base = cb.conv2d_backward_data_workspace_size(2, 16, 9, 9, 32, 3, 3, 1, 1, 1, 1, cb.CONV_BF16, "nhwc")
+    assert base == 0
+    s2 = cb.conv2d_backward_data_workspace_size(2, 16, 9, 9, 32, 3, 3, 2, 1, 1, 1, cb.CONV_BF16, "nhwc")
+    assert s2 >= 2 * 9 * 9 * 32 * 2
+    # weight gradient: padded channels-last copies and one split of fp32 partials without a device
+    wg = cb.conv2d_backward_weight_workspace_size(2, 16, 9, 9, 32, 3, 3, 1, 1, 1, 1, cb.CONV_BF16, "nhwc")
+    assert wg >= 2 * 9 * 9 * 64 * 2 + 32 * 9 * 64 * 4     # x padded to 64 channels; partials [C_out][taps][64]
+    assert cb.conv2d_backward_weight_workspace_size(2, 16, 9, 9, 32, 3, 3, 1, 1, 1, 1, cb.CONV_BF16, "nhwc",
+                                                    with_bias=True) > wg
+    assert cb.conv2d_backward_bias_workspace_size(2, 32, 9, 9, "nchw") == 2 * 32 * 4
+
+
+def test_backward_rejects_bad_arguments(lib):
+    with pytest.raises(cb.Conv2dError) as err:
+        cb.conv2d_backward_data_workspace_size(2, 16, 9, 9, 32, 3, 3, 1, 1, 1, 3, cb.CONV_BF16, "nhwc")
+    assert err.value.status == cb.CONV_ERR_INVALID_ARG        # groups must divide both channel counts
+    st = lib.conv2d_backward_weight(None, None, None, None, 2, 16, 9, 9, 32, 3, 3, 1, 1, 1, 1, cb.CONV_BF16,
+                                    cb.CONV_NHWC, None, 0, None)
+    assert st == cb.CONV_ERR_INVALID_ARG
+
+
+def test_conv3d_sizes_and_limits_on_the_host(lib):
+    assert cb.conv3d_packed_weight_size(16, 3, 3, 3, 3, 1, cb.CONV_BF16) == 16 * 27 * 8 * 2
+    # NCDHW input: the channels-last copy, 3 channels padded to 8
+    assert cb.conv3d_workspace_size(4, 3, 16, 64, 64, 16, 3, 3, 3, 1, 1, 1, 1, cb.CONV_BF16, "nchw") == \
+        4 * 16 * 64 * 64 * 8 * 2
+    # the 5-D im2col addressing range: pad 17 is out of it
+    st = lib.conv3d_forward(16, 16, None, 16, 1, 8, 40, 40, 40, 8, 3, 3, 3, 1, 17, 1, 1, cb.CONV_BF16,
+                            cb.CONV_NHWC, None, 0, None)
+    assert st == cb.CONV_ERR_UNSUPPORTED
+    st = lib.conv3d_forward(16, 16, None, 16, 1, 8, 2, 8, 8, 8, 5, 3, 3, 1, 0, 1, 1, cb.CONV_BF16,
+                            cb.CONV_NHWC, None, 0, None)
+    assert st == cb.CONV_ERR_INVALID_ARG                       # filter deeper than the input
+
+
+def test_winograd_sizes_on_the_host(lib):
+    # F(2x2,3x3): 16 transformed filters per (oc, c); 64 channels each way, no group merge
+    assert cb.conv2d_winograd_packed_weight_size(64, 64, 2, cb.CONV_BF16) == 16 * 64 * 64 * 2
+    assert cb.conv2d_winograd_packed_weight_size(64, 64, 4, cb.CONV_F32) == 36 * 64 * 64 * 4
+    for m in (3, 6):
+        with pytest.raises(cb.Conv2dError):
+            cb.conv2d_winograd_packed_weight_size(8, 8, m, cb.CONV_BF16)
+    ws = cb.conv2d_winograd_workspace_size(2, 64, 12, 12, 64, 1, 2, cb.CONV_BF16, "nhwc")
+    tiles = 2 * 6 * 6
+    assert ws >= tiles * 16 * 64 * 2 + tiles * 16 * 64 * 4  # V (bf16) and the fp32 products

@@ -1,0 +1,106 @@
+"""The 3-D convolution forward pass through the C ABI against the fp64 conv3d oracle
+(needs a B200).
+
+The oracle is pinned on the CPU (tests/oracle_pins_conv3d.py).  Cases span several
+128-row tiles with ragged ends, non-cubic filters, strides, dilation and groups; the
+workloads of "PyTorch高维张量乘法与conv2d/conv3d维度语义解析" §6.2 and the wider video
+block are compared element by element over the whole output."""
+import numpy as np
+import pytest
+
+import cnn_convolution_conv2d_b200 as cb
+from cnn_convolution_conv2d_b200 import workloads
+import oracle
+import parity
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def cuda_ready():
+    import torch
+    assert torch.cuda.is_available(), "these tests need a CUDA device (run with -m 'not gpu' on CPU)"
+    from cnn_convolution_conv2d_b200 import build
+    build.build()
+    cb.load()
+    cb.conv2d_debug_set_watchdog(0, False)
+    yield
+    cb.conv2d_sync_status()
+
+
+def run_gpu3d(cfg, inp):
+    import torch
+    dt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+    w = torch.from_numpy(inp["w"]).to(dt).cuda()
+    b = None if inp["b"] is None else torch.from_numpy(inp["b"]).to(dt).cuda()
+    layer = cb.Conv3dB200(w, b, cfg.stride, cfg.pad, cfg.dilation, cfg.groups, cfg.layout)
+    x = torch.from_numpy(inp["x"]).to(dt)
+    if cfg.layout == "nhwc":
+        x = x.permute(0, 2, 3, 4, 1)
+    y = layer(x.contiguous().cuda())
+    cb.conv2d_sync_status()
+    y = y.float().cpu()
+    if cfg.layout == "nhwc":
+        y = y.permute(0, 4, 1, 2, 3)
+    return y.contiguous().numpy().astype(np.float64)
+
+
+def run_oracle3d(cfg, inp):
+    return oracle.conv3d(inp["x"], inp["w"], inp["b"], cfg.stride, cfg.pad, cfg.dilation, cfg.groups)
+
+
+EDGE3D = [  # N, C_in, D, H, W, C_out, Kd, Kh, Kw, stride, pad, dilation, groups
+    (2, 16, 6, 9, 8, 32, 3, 3, 3, 1, 1, 1, 1),      # ragged last tile (864 voxels)
+    (1, 64, 7, 10, 11, 48, 3, 3, 3, 2, 1, 1, 1),    # stride 2, 128-byte channel rows, C_out 48
+    (2, 3, 5, 12, 12, 8, 3, 3, 3, 1, 1, 1, 1),      # three input channels: padded channels-last copy
+    (1, 32, 8, 8, 8, 16, 2, 3, 5, 1, 2, 2, 1),      # non-cubic filter, dilation 2
+    (1, 64, 4, 9, 9, 64, 1, 3, 3, 1, 1, 1, 4),      # (1, 3, 3) filter, groups of 16
+    (2, 24, 9, 6, 7, 40, 3, 1, 3, 3, 2, 1, 1),      # stride 3, filter of height 1
+    (1, 32, 5, 5, 5, 32, 1, 1, 1, 1, 0, 1, 1),      # 1x1x1: the input read as the im2col matrix
+    (3, 8, 1, 7, 7, 16, 1, 3, 3, 1, 1, 1, 1),       # a single frame
+]
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("layout", ["nhwc", "nchw"])
+@pytest.mark.parametrize("shape", EDGE3D, ids=lambda s: "x".join(map(str, s)))
+def test_conv3d_edge_shapes(shape, layout, dtype):
+    cfg = workloads.Conv3dConfig("edge3d", *shape, True, dtype, layout, seed=sum(shape))
+    inp = workloads.make_inputs3d(cfg)
+    parity.assert_close(cfg, run_gpu3d(cfg, inp), run_oracle3d(cfg, inp), str(shape))
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_conv3d_small_integers_bit_exact(dtype):
+    ints = ("integers", -2, 2)
+    cfg = workloads.Conv3dConfig("ints3d", 2, 16, 5, 6, 7, 16, 3, 3, 3, 1, 1, 1, 1, True, dtype, "nhwc",
+                                 ints, ints, ints, seed=3)
+    inp = workloads.make_inputs3d(cfg)
+    ref = run_oracle3d(cfg, inp)
+    assert np.abs(ref).max() <= 256
+    assert np.array_equal(run_gpu3d(cfg, inp), ref)
+
+
+def test_conv3d_one_frame_filter_is_per_frame_conv2d():
+    """pwwt §5.3 on the GPU: a (1, 3, 3) filter gives, frame by frame, what the 2-D
+    forward pass gives on that frame (with depth padding 1 the real frames are 1..D)."""
+    import torch
+    cfg = workloads.Conv3dConfig("frames", 2, 32, 4, 10, 9, 16, 1, 3, 3, 1, 1, 1, 1, True, "bf16", "nchw", seed=4)
+    inp = workloads.make_inputs3d(cfg)
+    got = run_gpu3d(cfg, inp)                      # pad 1 in depth too: frames 1..D are the real ones
+    w2 = torch.from_numpy(inp["w"][:, :, 0]).to(torch.bfloat16).cuda()
+    b2 = torch.from_numpy(inp["b"]).to(torch.bfloat16).cuda()
+    layer2 = cb.Conv2dB200(w2, b2, 1, 1, 1, 1, "nchw")
+    for f in range(cfg.D):
+        x2 = torch.from_numpy(np.ascontiguousarray(inp["x"][:, :, f])).to(torch.bfloat16).cuda()
+        y2 = layer2(x2).float().cpu().numpy().astype(np.float64)
+        # the two paths may tile and split the reduction differently: equal up to the
+        # order of fp32 additions, i.e. within the bf16 bar
+        assert np.abs(got[:, :, f + 1] - y2).max() <= parity.BF16_MAXABS * np.abs(y2).max(), f
+
+
+@pytest.mark.parametrize("name", sorted(workloads.CONFIGS3D))
+def test_conv3d_workloads_whole_output(name):
+    cfg = workloads.CONFIGS3D[name]
+    inp = workloads.make_inputs3d(cfg)
+    parity.assert_close(cfg, run_gpu3d(cfg, inp), run_oracle3d(cfg, inp), name)
