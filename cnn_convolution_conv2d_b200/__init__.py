@@ -61,7 +61,7 @@ SIGNATURES = {
     "conv2d_backward_bias_workspace_size": ([_I, _I, _I, _I, _I, ctypes.POINTER(_S)], _I),
     "conv2d_backward_bias": ([_P, _P, _I, _I, _I, _I, _I, _I, _P, _S, _P], _I),
     "conv3d_packed_weight_size": ([_I] * 7 + [ctypes.POINTER(_S)], _I),
-    "conv3d_pack_weight": ([_P, _P] + [_I] * 7 + [_I, _P], _I),
+    "conv3d_pack_weight": ([_P, _P] + [_I] * 7 + [_P], _I),
     "conv3d_workspace_size": ([_I] * 13 + [_I, _I, ctypes.POINTER(_S)], _I),
     "conv3d_forward": ([_P, _P, _P, _P] + [_I] * 13 + [_I, _I, _P, _S, _P], _I),
     "conv2d_winograd_packed_weight_size": ([_I, _I, _I, _I, ctypes.POINTER(_S)], _I),
@@ -362,8 +362,8 @@ def conv2d_pack_weight_winograd(w_oihw, m: int = 2, u_packed=None, stream=None):
         raise ValueError("Winograd F(m x m, 3 x 3) needs a 3x3 filter")
     code = _dtype_code(w_oihw.dtype)
     nbytes = conv2d_winograd_packed_weight_size(C_out, C_in, m, code)
-    if u_packed is None:
-        u_packed = torch.empty(nbytes // w_oihw.element_size(), dtype=w_oihw.dtype, device=w_oihw.device)
+    if u_packed is None:  # raw bytes: the transform type can differ from the weight's
+        u_packed = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=w_oihw.device)
     _check(load().conv2d_pack_weight_winograd(_ptr(w_oihw), _ptr(u_packed), C_out, C_in, m, code, _stream(stream)))
     return u_packed
 

@@ -190,7 +190,10 @@ int out_size(int in, int k, int s, int p, int d, int *out) {
 // gm-times larger (still small) packed weights.  Depends only on the weight's shape, so
 // that conv2d_pack_weight and the forward pass agree.
 int group_merge(int C_out, int C_in, int groups, int elt) {
-    if (groups <= 1) return 1;
+    // fp32 runs three products per multiply-add and splits every staged weight into tf32
+    // hi and lo parts: there the block-diagonal zeros cost more than the wider N saves
+    // (measured on the grouped layer: 34 -> 46 us), so only bf16 groups are merged.
+    if (groups <= 1 || elt != 2) return 1;
     const int cin_g = C_in / groups, cout_g = C_out / groups;
     if (cout_g >= 64 || (cin_g * elt) % 16 != 0) return 1;
     int best = 1;
@@ -232,7 +235,7 @@ GatherImages gather_images(int C_out, int C_in, int Kh, int Kw, int groups, int 
 }
 
 // Depthwise problems (groups = C_in = C_out) go to the direct stencil kernel when its
-// staged input box fits: tiles of TH x 8 output pixels x 128 bytes of channels, one
+// staged input box fits: tiles of TH (<= 30) x 8 output pixels x 128 bytes of channels, one
 // persistent CTA per SM with as many stages as fit.  Returns false (and
 // the problem goes to the general kernels) when no tile shape fits.
 bool plan_depthwise(Plan *pp) {
@@ -249,12 +252,18 @@ bool plan_depthwise(Plan *pp) {
     const size_t wbytes = static_cast<size_t>(taps) * 128 + cc * 4;
     p.dw_wregion = static_cast<int>(align_up(wbytes * dw_compute_warps(), 1024));
     const size_t fixed = dw_header_bytes() + p.dw_wregion;
-    // the tallest tile (at most 32 rows) whose staged box fits twice
+    // the tallest tile (30 rows: one item per compute thread) whose staged box fits twice
     size_t stage = 0;
-    for (p.TH = 32; p.TH >= 1; p.TH /= 2) {
-        p.IH = (p.TH - 1) * p.stride + (p.Kh - 1) * p.dilation + 1;
-        stage = static_cast<size_t>(p.IH) * p.IW * 128;
-        if (p.IH <= 256 && fixed + 2 * stage <= kSmemBudget) break;
+    const int th_choices[6] = {30, 15, 8, 4, 2, 1};
+    p.TH = 0;
+    for (int th : th_choices) {
+        const int ih = (th - 1) * p.stride + (p.Kh - 1) * p.dilation + 1;
+        stage = static_cast<size_t>(ih) * p.IW * 128;
+        if (ih <= 256 && fixed + 2 * stage <= kSmemBudget) {
+            p.TH = th;
+            p.IH = ih;
+            break;
+        }
     }
     if (p.TH < 1) return false;
     p.dw_ctas_per_sm = 1;
@@ -795,7 +804,7 @@ int device_plan(bool explicit_im2col, int N, int C_in, int H, int W, int C_out, 
     p->pair_clusters = 0;
     if (p->pair && dev) {
         const bool a_im2col = !(explicit_im2col || p->direct_a);
-        p->pair_clusters = pair_cluster_limit(p->cb, a_im2col, p->smem, p->vol);
+        p->pair_clusters = pair_cluster_limit(p->cb, a_im2col, p->smem, p->vol && a_im2col);
         if (p->pair_clusters < 1)  // the device cannot co-schedule the pair kernel: single CTAs
             return make_plan(N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype, layout,
                              explicit_im2col, dev->sms, p, cfg.pair_mode, false, padw, vol);
@@ -930,7 +939,8 @@ int forward_impl(bool explicit_im2col, const void *x, const void *w_packed, cons
                             : (p.units < dev->sms ? p.units : dev->sms);
     cudaEvent_t ev_start = g_main_start, ev_stop = g_main_stop;
     if (ev_start && ev_stop && (st = record_event(ev_start, stream)) != CONV_OK) return st;
-    cudaError_t e = launch_igemm(kp, p.f32, p.cb, a_im2col, p.pair, grid, p.smem, stream, p.vol);
+    // a 1x1x1 stride-1 unpadded volume reads x itself as X_col (tiled loads), like 2-D
+    cudaError_t e = launch_igemm(kp, p.f32, p.cb, a_im2col, p.pair, grid, p.smem, stream, p.vol && a_im2col);
     if ((st = check_launch(e, "tensor-core product")) != CONV_OK) return st;
     if (ev_start && ev_stop && (st = record_event(ev_stop, stream)) != CONV_OK) return st;
     if (p.splits > 1 && !external_partial) {
@@ -1050,7 +1060,7 @@ int wgrad_plan(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int str
         w.dy_cpg = round_up(w.Cout_g, align);
         w.xcopy = layout == CONV_NCHW || w.Cpg != w.Cin_g;
         w.dycopy = layout == CONV_NCHW || w.dy_cpg != w.Cout_g;
-        const int cap = f.f32 ? 128 : 256;
+        const int cap = f.f32 ? 64 : 256;  // fp32 stages hold raw, hi and lo copies
         for (w.BN = cap; w.BN > cc && w.Cpg % w.BN != 0; w.BN -= cc) {
         }
         w.n_ctiles = w.Cpg / w.BN;
@@ -1305,9 +1315,14 @@ int backward_data_impl(const void *dy, const void *w_packed_t, void *dx, int N, 
 struct WinoPlan {
     Plan f;          // the 3x3 problem: validation, Ho, Wo
     Plan g;          // the product
+    conv_dtype_t tdt;  // transform and product type (see wino_tdt)
     int m, a, Cpg, TH, TW, T;
     size_t off_v, off_m, off_inner, ws_total;
 };
+
+// Type of the transformed tiles and filters and of their product: the data's own for
+// F(2x2,3x3), fp32 for F(4x4,3x3) (its bf16 transforms miss the bf16 tolerance).
+conv_dtype_t wino_tdt(conv_dtype_t dtype, int m) { return m == 4 ? CONV_F32 : dtype; }
 
 int wino_plan(int N, int C_in, int H, int W, int C_out, int pad, int m, conv_dtype_t dtype, conv_layout_t layout,
               DeviceInfo *dev, const Settings &cfg, WinoPlan *out) {
@@ -1317,7 +1332,9 @@ int wino_plan(int N, int C_in, int H, int W, int C_out, int pad, int m, conv_dty
     if (st != CONV_OK) return st;
     w.m = m;
     w.a = m + 2;
-    w.Cpg = round_up(C_in, 16 / w.f.elt);
+    w.tdt = wino_tdt(dtype, m);
+    const int telt = w.tdt == CONV_F32 ? 4 : 2;
+    w.Cpg = round_up(C_in, 16 / telt);
     w.TH = (w.f.Ho + m - 1) / m;
     w.TW = (w.f.Wo + m - 1) / m;
     const long long T = static_cast<long long>(N) * w.TH * w.TW;
@@ -1325,12 +1342,12 @@ int wino_plan(int N, int C_in, int H, int W, int C_out, int pad, int m, conv_dty
     w.T = static_cast<int>(T);
     const int a2 = w.a * w.a;
     const PadW pw{0, reinterpret_cast<float *>(16)};  // placeholder address: plans the external-partial form
-    st = device_plan(false, 1, a2 * w.Cpg, 1, w.T, a2 * C_out, 1, 1, 1, 0, 1, a2, dtype, CONV_NHWC, dev, cfg, &w.g,
+    st = device_plan(false, 1, a2 * w.Cpg, 1, w.T, a2 * C_out, 1, 1, 1, 0, 1, a2, w.tdt, CONV_NHWC, dev, cfg, &w.g,
                      &pw);
     if (st != CONV_OK) return st;
     size_t off = 0;
     w.off_v = off;
-    off = align_up(off + static_cast<size_t>(T) * a2 * w.Cpg * w.f.elt, 256);
+    off = align_up(off + static_cast<size_t>(T) * a2 * w.Cpg * telt, 256);
     w.off_m = off;
     off = align_up(off + static_cast<size_t>(w.g.splits) * T * a2 * C_out * 4, 256);
     w.off_inner = off;
@@ -1365,13 +1382,13 @@ int winograd_impl(const void *x, const void *u_packed, const void *bias, void *y
     float *mp = reinterpret_cast<float *>(ws + w.off_m);
     const bool nchw = layout == CONV_NCHW;
     if ((st = check_launch(launch_wino_input(x, ws + w.off_v, N, C_in, H, W, w.Cpg, w.TH, w.TW, pad, m, nchw,
-                                             w.f.f32, stream),
+                                             w.f.f32, w.tdt == CONV_F32, stream),
                            "Winograd input transform")) != CONV_OK)
         return st;
     const int a2 = w.a * w.a;
     const PadW pw{0, mp};
     if ((st = forward_impl(false, ws + w.off_v, u_packed, nullptr, mp, 1, a2 * w.Cpg, 1, w.T, a2 * C_out, 1, 1, 1, 0,
-                           1, a2, dtype, CONV_NHWC, ws + w.off_inner, workspace_bytes - w.off_inner, stream, &pw)) !=
+                           1, a2, w.tdt, CONV_NHWC, ws + w.off_inner, workspace_bytes - w.off_inner, stream, &pw)) !=
         CONV_OK)
         return st;
     return check_launch(launch_wino_output(mp, bias, y, N, C_out, w.f.Ho, w.f.Wo, w.TH, w.TW, w.g.splits, m, nchw,
@@ -1751,9 +1768,10 @@ int conv2d_winograd_packed_weight_size(int C_out, int C_in, int m, conv_dtype_t 
     if (!bytes || elt == 0 || C_out < 1 || C_in < 1 || (m != 2 && m != 4))
         return fail(CONV_ERR_INVALID_ARG, "Winograd packed weight size: invalid argument");
     const int a2 = (m + 2) * (m + 2);
-    const int cpg = round_up(C_in, 16 / elt);
-    const int gm = group_merge(a2 * C_out, a2 * cpg, a2, elt);
-    *bytes = static_cast<size_t>(a2) * C_out * cpg * gm * elt;
+    const int telt = wino_tdt(dtype, m) == CONV_F32 ? 4 : 2;
+    const int cpg = round_up(C_in, 16 / telt);
+    const int gm = group_merge(a2 * C_out, a2 * cpg, a2, telt);
+    *bytes = static_cast<size_t>(a2) * C_out * cpg * gm * telt;
     return ok();
 }
 
@@ -1763,11 +1781,12 @@ int conv2d_pack_weight_winograd(const void *w_oihw, void *u_packed, int C_out, i
     int st = conv2d_winograd_packed_weight_size(C_out, C_in, m, dtype, &bytes);
     if (st != CONV_OK) return st;
     if (!w_oihw || !u_packed) return fail(CONV_ERR_INVALID_ARG, "weight pointers must not be NULL");
-    const int elt = elt_of(dtype);
     const int a2 = (m + 2) * (m + 2);
-    const int cpg = round_up(C_in, 16 / elt);
-    const int gm = group_merge(a2 * C_out, a2 * cpg, a2, elt);
-    return check_launch(launch_wino_weight(w_oihw, u_packed, C_out, C_in, cpg, gm, m, dtype == CONV_F32,
+    const bool u_f32 = wino_tdt(dtype, m) == CONV_F32;
+    const int telt = u_f32 ? 4 : 2;
+    const int cpg = round_up(C_in, 16 / telt);
+    const int gm = group_merge(a2 * C_out, a2 * cpg, a2, telt);
+    return check_launch(launch_wino_weight(w_oihw, u_packed, C_out, C_in, cpg, gm, m, dtype == CONV_F32, u_f32,
                                            reinterpret_cast<cudaStream_t>(stream)),
                         "Winograd weight transform") == CONV_OK
                ? ok()

@@ -185,9 +185,10 @@ cudaError_t launch_pack_weight_t(const void *w, void *wp, int O, int R, int Cin_
                                  int elt, cudaStream_t s);
 
 // Winograd F(m x m, 3 x 3) transforms (winograd.cu), m = 2 or 4.
+// f32: the data type; v_f32 / u_f32: the transform type (fp32 whenever the data is fp32).
 cudaError_t launch_wino_input(const void *x, void *v, int N, int C, int H, int W, int Cpg, int TH, int TW, int pad,
-                              int m, bool nchw, bool f32, cudaStream_t s);
-cudaError_t launch_wino_weight(const void *w, void *u, int C_out, int C, int Cpg, int gm, int m, bool f32,
+                              int m, bool nchw, bool f32, bool v_f32, cudaStream_t s);
+cudaError_t launch_wino_weight(const void *w, void *u, int C_out, int C, int Cpg, int gm, int m, bool f32, bool u_f32,
                                cudaStream_t s);
 cudaError_t launch_wino_output(const float *mp, const void *bias, void *y, int N, int C_out, int Ho, int Wo, int TH,
                                int TW, int splits, int m, bool nchw, bool f32, cudaStream_t s);

@@ -17,7 +17,7 @@
 //                pixels x 128 bytes of channels, starting at (oh0*s - p, ow0*s - p); the
 //                part of the box outside the image is filled with zeros by the copy engine,
 //                which is the zero padding -- into a ring of shared-memory stages;
-//   warps 1..16: compute.  Each thread owns R consecutive output pixels of one row and 16
+//   warps 1..15: compute.  Each thread owns R consecutive output pixels of one row and 16
 //                bytes of channels; for stride 1 and unit dilation it reads each input row
 //                once into a register window of R + Kw - 1 pixels and reuses it for every
 //                filter column.  Weights of the tile's channels are kept per warp in shared
@@ -35,7 +35,9 @@ namespace {
 using namespace ptx;
 
 constexpr int kDwRowBytes = 128;  // bytes of channels per staged pixel
-constexpr int kDwComputeWarps = 16;
+// 16 warps in all: four per SM sub-partition, so each thread may use 128 registers
+// (a 17th warp would put five on one sub-partition and cap every thread at 96)
+constexpr int kDwComputeWarps = 15;
 constexpr int kDwThreads = 32 * (1 + kDwComputeWarps);
 constexpr int kDwMaxStages = 6;
 constexpr int kDwHeader = 1024;   // barriers, ahead of the weights and the stage ring
@@ -63,6 +65,17 @@ __device__ __forceinline__ void unpack16(const uint4 &u, float *f) {
             f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
         }
     }
+}
+
+// acc[0..1] += x[0..1] * w[0..1] as one paired fp32 FMA (fma.rn.f32x2, two lanes per
+// instruction), each lane rounded as fmaf would round it.
+__device__ __forceinline__ void ffma2(float *acc, const float *x, const float *w) {
+    uint64_t a, xx, ww;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "f"(acc[0]), "f"(acc[1]));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(xx) : "f"(x[0]), "f"(x[1]));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(ww) : "f"(w[0]), "f"(w[1]));
+    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(a) : "l"(xx), "l"(ww));
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(acc[0]), "=f"(acc[1]) : "l"(a));
 }
 
 struct DwTile {
@@ -233,7 +246,7 @@ __global__ void __launch_bounds__(kDwThreads, 1) dw_kernel(const __grid_constant
 #pragma unroll
                             for (int r = 0; r < kR; ++r)
 #pragma unroll
-                                for (int v = 0; v < kV; ++v) acc[r][v] = fmaf(win[r + kw][v], wv[v], acc[r][v]);
+                                for (int v = 0; v < kV; v += 2) ffma2(&acc[r][v], &win[r + kw][v], &wv[v]);
                         }
                     } else {
                         for (int kw = 0; kw < p.Kw; ++kw) {
@@ -245,7 +258,7 @@ __global__ void __launch_bounds__(kDwThreads, 1) dw_kernel(const __grid_constant
                                 float xv[kV];
                                 unpack16<kF32>(*reinterpret_cast<const uint4 *>(rp + col * kDwRowBytes), xv);
 #pragma unroll
-                                for (int v = 0; v < kV; ++v) acc[r][v] = fmaf(xv[v], wv[v], acc[r][v]);
+                                for (int v = 0; v < kV; v += 2) ffma2(&acc[r][v], &xv[v], &wv[v]);
                             }
                         }
                     }

@@ -23,10 +23,12 @@
 //
 // Persistent and warp-specialised like the forward kernel (igemm.cu): warp 0 issues the
 // TMA loads, warp 1 allocates tensor memory and issues the MMAs from one thread, warps
-// 2..9 (bf16) or 2..5 (fp32) drain the double-buffered accumulator; for fp32 warps 6..9
-// split every staged value into tf32 hi and lo parts for three products per
-// multiply-add, and the accumulator restarts every few stages with the chunks summed in
-// fp32 registers (as in the forward fp32 path).  Every wait is bounded (see ptx.cuh).
+// 2..9 (bf16) or 2..5 (fp32) drain the double-buffered accumulator.  fp32: the tensor
+// cores read tf32 operands MN-major only in a 32-byte-atom swizzle that these loads do not
+// produce, so warps 6..9 rewrite every staged block K-major (pixels contiguous, the
+// forward kernel's 128-byte swizzle), split into tf32 hi and lo parts for three products
+// per multiply-add, and the accumulator restarts every few stages with the chunks summed
+// in fp32 registers (as in the forward fp32 path).  Every wait is bounded (see ptx.cuh).
 #include "common.cuh"
 #include "epilogue.cuh"
 #include "ptx.cuh"
@@ -109,7 +111,8 @@ __global__ void __launch_bounds__(kWgThreads, 1) wgrad_kernel(const __grid_const
     const int b_blocks = BN / kCC;
     const uint32_t a_bytes = a_blocks * kBlk, b_bytes = b_blocks * kBlk;
     const uint32_t tx_bytes = a_bytes + b_bytes;
-    const uint32_t sbytes = tx_bytes * (kF32 ? 2u : 1u);  // fp32: hi in place, lo behind
+    // fp32: the raw (MN-major) blocks, then K-major hi and lo copies of both operands
+    const uint32_t sbytes = tx_bytes * (kF32 ? 3u : 1u);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.stages; ++s) {
@@ -190,8 +193,10 @@ __global__ void __launch_bounds__(kWgThreads, 1) wgrad_kernel(const __grid_const
     } else if (warp == 1) {
         // --------------------------------------------------- tensor-core issue ---
         if (lane == 0) {
-            // MN-major A (output channels contiguous) and B (input channels contiguous)
-            const uint32_t idesc = instr_desc(kF32 ? 2u : 1u, 128, static_cast<uint32_t>(BN)) | (1u << 15) | (1u << 16);
+            // bf16: MN-major A (output channels contiguous) and B (input channels
+            // contiguous); fp32: the converted K-major copies
+            const uint32_t idesc = kF32 ? instr_desc(2u, 128, static_cast<uint32_t>(BN))
+                                        : (instr_desc(1u, 128, static_cast<uint32_t>(BN)) | (1u << 15) | (1u << 16));
             int stage = 0;
             uint32_t phase = 0;
             int abuf = 0;
@@ -217,18 +222,21 @@ __global__ void __launch_bounds__(kWgThreads, 1) wgrad_kernel(const __grid_const
                         tc_fence_after_sync();
                         const uint32_t a = smem_addr(ring + static_cast<size_t>(stage) * sbytes);
                         const uint32_t b = a + a_bytes;
-                        const uint32_t alo = a + tx_bytes, blo = b + tx_bytes;
 #pragma unroll
                         for (int ks = 0; ks < kPK / kKS; ++ks) {
                             const uint32_t off = static_cast<uint32_t>(ks * kKS * 128);
                             const uint32_t acc = (kb == c0 && ks == 0) ? 0u : 1u;
                             if constexpr (kF32) {
-                                mma_tf32(d_tmem, smem_desc(alo + off, kBlk, 1024, kSw128),
-                                         smem_desc(b + off, kBlk, 1024, kSw128), idesc, acc);
-                                mma_tf32(d_tmem, smem_desc(a + off, kBlk, 1024, kSw128),
-                                         smem_desc(blo + off, kBlk, 1024, kSw128), idesc, 1u);
-                                mma_tf32(d_tmem, smem_desc(a + off, kBlk, 1024, kSw128),
-                                         smem_desc(b + off, kBlk, 1024, kSw128), idesc, 1u);
+                                // K-major copies: rows of 32 pixels (128 bytes), 32 bytes of k per MMA
+                                const uint32_t ah = a + tx_bytes, bh = ah + a_bytes;
+                                const uint32_t al = a + 2 * tx_bytes, bl = al + a_bytes;
+                                const uint32_t ko = static_cast<uint32_t>(ks * 32);
+                                mma_tf32(d_tmem, smem_desc(al + ko, 16, 1024, kSw128),
+                                         smem_desc(bh + ko, 16, 1024, kSw128), idesc, acc);
+                                mma_tf32(d_tmem, smem_desc(ah + ko, 16, 1024, kSw128),
+                                         smem_desc(bl + ko, 16, 1024, kSw128), idesc, 1u);
+                                mma_tf32(d_tmem, smem_desc(ah + ko, 16, 1024, kSw128),
+                                         smem_desc(bh + ko, 16, 1024, kSw128), idesc, 1u);
                             } else {
                                 mma_bf16(d_tmem, smem_desc(a + off, kBlk, 1024, kSw128),
                                          smem_desc(b + off, kBlk, 1024, kSw128), idesc, acc);
@@ -344,18 +352,36 @@ __global__ void __launch_bounds__(kWgThreads, 1) wgrad_kernel(const __grid_const
                     ok = false;
                     break;
                 }
-                uint8_t *st = ring + static_cast<size_t>(stage) * sbytes;
-                float4 *hi = reinterpret_cast<float4 *>(st);
-                float4 *lo = reinterpret_cast<float4 *>(st + tx_bytes);
-                for (uint32_t i = tid; i < tx_bytes / 16; i += 128) {
-                    const float4 v = hi[i];
-                    float4 h, l;
-                    h.x = tf32_round(v.x); l.x = tf32_round(v.x - h.x);
-                    h.y = tf32_round(v.y); l.y = tf32_round(v.y - h.y);
-                    h.z = tf32_round(v.z); l.z = tf32_round(v.z - h.z);
-                    h.w = tf32_round(v.w); l.w = tf32_round(v.w - h.w);
-                    hi[i] = h;
-                    lo[i] = l;
+                // Raw block j of an operand: PK pixel rows of 128 bytes (32 MN elements),
+                // 16-byte chunk q of row p at chunk q ^ (p & 7).  K-major copy: MN element
+                // r of the operand is row r (128 bytes = 32 pixels), 16-byte chunk q of row r
+                // at q ^ (r & 7), 8-row groups 1024 bytes apart.  Each thread moves one
+                // 16-byte raw chunk (four MN elements of one pixel) per step.
+                const uint8_t *raw = ring + static_cast<size_t>(stage) * sbytes;
+                uint8_t *hi = const_cast<uint8_t *>(raw) + tx_bytes;
+                uint8_t *lo = const_cast<uint8_t *>(raw) + 2 * tx_bytes;
+                const int chunks = static_cast<int>(tx_bytes / 16);
+                for (int i = tid; i < chunks; i += 128) {
+                    const int blk = i / (kPK * 8);          // 8 chunks per 128-byte row
+                    const int rem = i - blk * (kPK * 8);
+                    const int px = rem >> 3, q = rem & 7;
+                    const float4 v = *reinterpret_cast<const float4 *>(raw + blk * kBlk + px * 128 +
+                                                                       ((q ^ (px & 7)) << 4));
+                    const float vv[4] = {v.x, v.y, v.z, v.w};
+                    // operand row of MN element (blk*32 + 4q + e); B follows A's 128 rows
+                    const uint32_t region = blk < a_blocks ? 0u : a_bytes;
+                    const int r0 = (blk < a_blocks ? blk : blk - a_blocks) * 32 + 4 * q;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int r = r0 + e;
+                        const uint32_t off = region + static_cast<uint32_t>(r >> 3) * 1024u +
+                                             static_cast<uint32_t>(r & 7) * 128u +
+                                             static_cast<uint32_t>(((px >> 2) ^ (r & 7)) << 4) +
+                                             static_cast<uint32_t>(px & 3) * 4u;
+                        const float h = tf32_round(vv[e]);
+                        *reinterpret_cast<float *>(hi + off) = h;
+                        *reinterpret_cast<float *>(lo + off) = tf32_round(vv[e] - h);
+                    }
                 }
                 fence_proxy_async_smem();
                 mbar_arrive(&sb.converted[stage]);
@@ -393,7 +419,7 @@ int wgrad_max_stages() { return kWgMaxStages; }
 size_t wgrad_smem_bytes(bool f32, int BN, int stages) {
     const size_t blk = f32 ? wg_block_bytes<true>() : wg_block_bytes<false>();
     const int cc = f32 ? 32 : 64;
-    const size_t stage = (128 / cc + BN / cc) * blk * (f32 ? 2 : 1);
+    const size_t stage = (128 / cc + BN / cc) * blk * (f32 ? 3 : 1);
     return 1024 /* alignment slack */ + kWgHeader + static_cast<size_t>(stages) * stage;
 }
 

@@ -17,7 +17,9 @@
 // convolution with alpha^2 groups over the transformed tiles).  The three steps:
 //   1. input transform (this file): V = B^T d B per tile and channel vector, written
 //      channels-last as [tile][xi][Cpg] (Cpg: channels padded to 16 bytes), in the
-//      input dtype -- one rounding for bf16;
+//      transform type: bf16 for F(2x2,3x3) on bf16 data (one more rounding), fp32
+//      otherwise -- F(4x4,3x3)'s larger transform entries make bf16 V and U miss the bf16
+//      tolerance (measured), so its transforms and product stay in fp32 (3xTF32);
 //   2. the product on the tensor cores, fp32 results [tile][xi][oc];
 //   3. output transform (this file): Y = A^T M A + bias per tile and output channel
 //      vector, one rounding to the output dtype, written NHWC or NCHW.
@@ -100,10 +102,57 @@ __device__ __forceinline__ void st1(void *p, long long i, float v) {
         static_cast<__nv_bfloat16 *>(p)[i] = __float2bfloat16_rn(v);
 }
 
+// kV consecutive elements at element index i (i a multiple of kV, the base aligned):
+// one 4-, 8- or 16-byte access instead of kV scalar ones.
+template <bool kF32, int kV>
+__device__ __forceinline__ void ldv(const void *p, long long i, float *f) {
+    if constexpr (kF32) {
+        if constexpr (kV == 4) {
+            const float4 v = *reinterpret_cast<const float4 *>(static_cast<const float *>(p) + i);
+            f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
+        } else {
+            const float2 v = *reinterpret_cast<const float2 *>(static_cast<const float *>(p) + i);
+            f[0] = v.x; f[1] = v.y;
+        }
+    } else {
+        const unsigned short *q = static_cast<const unsigned short *>(p) + i;
+        if constexpr (kV == 4) {
+            const uint2 v = *reinterpret_cast<const uint2 *>(q);
+            f[0] = __uint_as_float(v.x << 16); f[1] = __uint_as_float(v.x & 0xFFFF0000u);
+            f[2] = __uint_as_float(v.y << 16); f[3] = __uint_as_float(v.y & 0xFFFF0000u);
+        } else {
+            const uint32_t v = *reinterpret_cast<const uint32_t *>(q);
+            f[0] = __uint_as_float(v << 16); f[1] = __uint_as_float(v & 0xFFFF0000u);
+        }
+    }
+}
+
+template <bool kF32, int kV>
+__device__ __forceinline__ void stv(void *p, long long i, const float *f) {
+    if constexpr (kF32) {
+        if constexpr (kV == 4)
+            *reinterpret_cast<float4 *>(static_cast<float *>(p) + i) = make_float4(f[0], f[1], f[2], f[3]);
+        else
+            *reinterpret_cast<float2 *>(static_cast<float *>(p) + i) = make_float2(f[0], f[1]);
+    } else {
+        uint32_t w[kV / 2];
+#pragma unroll
+        for (int k = 0; k < kV / 2; ++k) {
+            __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * k], f[2 * k + 1]);
+            w[k] = *reinterpret_cast<uint32_t *>(&h);
+        }
+        unsigned short *q = static_cast<unsigned short *>(p) + i;
+        if constexpr (kV == 4)
+            *reinterpret_cast<uint2 *>(q) = make_uint2(w[0], w[1]);
+        else
+            *reinterpret_cast<uint32_t *>(q) = w[0];
+    }
+}
+
 // 1. V[tile][xi][c] = (B^T d B)[xi] for each tile (n, th, tw) and channel c < Cpg (zero
 // for c >= C): d[a][b] = x[n][th*m - pad + a][tw*m - pad + b][c], zero outside the image.
 // One thread per (tile, group of kV consecutive channels).
-template <bool kF32, int kM, int kV>
+template <bool kF32, bool kVF32, int kM, int kV>
 __global__ void __launch_bounds__(kWgThreads256) wino_input_kernel(const void *__restrict__ x, void *__restrict__ v,
                                                                  int N, int C, int H, int W, int Cpg, int TH, int TW,
                                                                  int pad, int nchw) {
@@ -111,6 +160,7 @@ __global__ void __launch_bounds__(kWgThreads256) wino_input_kernel(const void *_
     constexpr int kA = Mt::kA;
     const int cgroups = Cpg / kV;
     const long long total = static_cast<long long>(N) * TH * TW * cgroups;
+    const bool vec = !nchw && C % kV == 0;
     for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
          i += static_cast<long long>(gridDim.x) * blockDim.x) {
         const int cg = static_cast<int>(i % cgroups);
@@ -131,6 +181,15 @@ __global__ void __launch_bounds__(kWgThreads256) wino_input_kernel(const void *_
             for (int k = 0; k < kA; ++k) {
                 const int ih = h0 + k;
                 const bool in = ih >= 0 && ih < H && iw >= 0 && iw < W;
+                if (vec) {  // channels-last, C a multiple of kV: one vector access
+                    if (in && c0 < C) {
+                        ldv<kF32, kV>(x, ((static_cast<long long>(n) * H + ih) * W + iw) * C + c0, d[k]);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < kV; ++e) d[k][e] = 0.f;
+                    }
+                    continue;
+                }
 #pragma unroll
                 for (int e = 0; e < kV; ++e) {
                     const int c = c0 + e;
@@ -158,21 +217,24 @@ __global__ void __launch_bounds__(kWgThreads256) wino_input_kernel(const void *_
 #pragma unroll
         for (int a = 0; a < kA; ++a)
 #pragma unroll
-            for (int b = 0; b < kA; ++b)
+            for (int b = 0; b < kA; ++b) {
+                float o[kV];
 #pragma unroll
                 for (int e = 0; e < kV; ++e) {
                     float s = 0.f;
 #pragma unroll
                     for (int k = 0; k < kA; ++k) s += t[a][k][e] * Mt::bt(b, k);
-                    st1<kF32>(v, base + static_cast<long long>(a * kA + b) * Cpg + e, s);
+                    o[e] = s;
                 }
+                stv<kVF32, kV>(v, base + static_cast<long long>(a * kA + b) * Cpg, o);  // Cpg % kV == 0
+            }
     }
 }
 
 // U packed for the product: rows o = xi * C_out + oc (alpha^2 groups of C_out), each
 // row Cpgw entries; entry c of row o holds (G g[oc][c] G^T)[xi] for c < C, zero for the
 // padding channels and -- with groups merged gm at a time -- outside the diagonal block.
-template <bool kF32, int kM>
+template <bool kF32, bool kUF32, int kM>
 __global__ void __launch_bounds__(kWgThreads256) wino_weight_kernel(const void *__restrict__ w, void *__restrict__ u,
                                                                   int C_out, int C, int Cpg, int gm, int Cpgw) {
     using Mt = WinoMats<kM>;
@@ -195,7 +257,7 @@ __global__ void __launch_bounds__(kWgThreads256) wino_weight_kernel(const void *
 #pragma unroll
                 for (int q = 0; q < 3; ++q) val += Mt::g(a, p) * ld1<kF32>(w, g0 + p * 3 + q) * Mt::g(b, q);
         }
-        st1<kF32>(u, i, val);
+        st1<kUF32>(u, i, val);
     }
 }
 
@@ -212,6 +274,7 @@ __global__ void __launch_bounds__(kWgThreads256) wino_output_kernel(const float 
     const long long tiles = static_cast<long long>(N) * TH * TW;
     const long long total = tiles * cgroups;
     const long long row = static_cast<long long>(kA) * kA * C_out;
+    const bool vec = C_out % kV == 0;
     for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
          i += static_cast<long long>(gridDim.x) * blockDim.x) {
         const int cg = static_cast<int>(i % cgroups);
@@ -227,15 +290,24 @@ __global__ void __launch_bounds__(kWgThreads256) wino_output_kernel(const float 
         for (int b = 0; b < kA; ++b) {
             float m[kA][kV];
 #pragma unroll
-            for (int k = 0; k < kA; ++k)
+            for (int k = 0; k < kA; ++k) {
 #pragma unroll
-                for (int e = 0; e < kV; ++e) {
-                    float sum = 0.f;
-                    if (c0 + e < C_out)
-                        for (int sp = 0; sp < splits; ++sp)
-                            sum += mp[(sp * tiles + tile) * row + static_cast<long long>(k * kA + b) * C_out + c0 + e];
-                    m[k][e] = sum;
+                for (int e = 0; e < kV; ++e) m[k][e] = 0.f;
+                if (vec) {
+                    for (int sp = 0; sp < splits; ++sp) {
+                        float f[kV];
+                        ldv<true, kV>(mp, (sp * tiles + tile) * row + static_cast<long long>(k * kA + b) * C_out + c0, f);
+#pragma unroll
+                        for (int e = 0; e < kV; ++e) m[k][e] += f[e];
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < kV; ++e)
+                        if (c0 + e < C_out)
+                            for (int sp = 0; sp < splits; ++sp)
+                                m[k][e] += mp[(sp * tiles + tile) * row + static_cast<long long>(k * kA + b) * C_out + c0 + e];
                 }
+            }
 #pragma unroll
             for (int a = 0; a < kM; ++a)
 #pragma unroll
@@ -257,29 +329,38 @@ __global__ void __launch_bounds__(kWgThreads256) wino_output_kernel(const float 
             for (int b = 0; b < kM; ++b) {
                 const int ow = tw * kM + b;
                 if (ow >= Wo) break;
+                float o[kV];
 #pragma unroll
                 for (int e = 0; e < kV; ++e) {
-                    const int oc = c0 + e;
-                    if (oc >= C_out) break;
                     float s = bv[e];
 #pragma unroll
                     for (int k = 0; k < kA; ++k) s += t[a][k][e] * Mt::at(b, k);
-                    const long long at = nchw ? ((static_cast<long long>(n) * C_out + oc) * Ho + oh) * Wo + ow
-                                              : ((static_cast<long long>(n) * Ho + oh) * Wo + ow) * C_out + oc;
-                    st1<kF32>(y, at, s);
+                    o[e] = s;
+                }
+                if (vec && !nchw) {
+                    stv<kF32, kV>(y, ((static_cast<long long>(n) * Ho + oh) * Wo + ow) * C_out + c0, o);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < kV; ++e) {
+                        const int oc = c0 + e;
+                        if (oc >= C_out) break;
+                        const long long at = nchw ? ((static_cast<long long>(n) * C_out + oc) * Ho + oh) * Wo + ow
+                                                  : ((static_cast<long long>(n) * Ho + oh) * Wo + ow) * C_out + oc;
+                        st1<kF32>(y, at, o[e]);
+                    }
                 }
             }
         }
     }
 }
 
-template <bool kF32, int kM>
+template <bool kF32, bool kVF32, int kM>
 cudaError_t input_t(const void *x, void *v, int N, int C, int H, int W, int Cpg, int TH, int TW, int pad, bool nchw,
                     cudaStream_t s) {
     constexpr int kV = kM == 2 ? 4 : 2;  // channels per thread
     const long long work = static_cast<long long>(N) * TH * TW * (Cpg / kV);
-    wino_input_kernel<kF32, kM, kV><<<wino_grid(work), kWgThreads256, 0, s>>>(x, v, N, C, H, W, Cpg, TH, TW, pad,
-                                                                            nchw ? 1 : 0);
+    wino_input_kernel<kF32, kVF32, kM, kV><<<wino_grid(work), kWgThreads256, 0, s>>>(x, v, N, C, H, W, Cpg, TH, TW,
+                                                                                   pad, nchw ? 1 : 0);
     return cudaGetLastError();
 }
 
@@ -296,33 +377,35 @@ cudaError_t output_t(const float *mp, const void *bias, void *y, int N, int C_ou
 }  // namespace
 
 cudaError_t launch_wino_input(const void *x, void *v, int N, int C, int H, int W, int Cpg, int TH, int TW, int pad,
-                              int m, bool nchw, bool f32, cudaStream_t s) {
+                              int m, bool nchw, bool f32, bool v_f32, cudaStream_t s) {
     if (Cpg % 4 != 0) return cudaErrorInvalidValue;  // a multiple of both vector widths
-    if (m == 2) return f32 ? input_t<true, 2>(x, v, N, C, H, W, Cpg, TH, TW, pad, nchw, s)
-                           : input_t<false, 2>(x, v, N, C, H, W, Cpg, TH, TW, pad, nchw, s);
-    if (m == 4) return f32 ? input_t<true, 4>(x, v, N, C, H, W, Cpg, TH, TW, pad, nchw, s)
-                           : input_t<false, 4>(x, v, N, C, H, W, Cpg, TH, TW, pad, nchw, s);
+    if (f32 && !v_f32) return cudaErrorInvalidValue;
+    if (m == 2) return f32 ? input_t<true, true, 2>(x, v, N, C, H, W, Cpg, TH, TW, pad, nchw, s)
+                           : v_f32 ? input_t<false, true, 2>(x, v, N, C, H, W, Cpg, TH, TW, pad, nchw, s)
+                                   : input_t<false, false, 2>(x, v, N, C, H, W, Cpg, TH, TW, pad, nchw, s);
+    if (m == 4) return f32 ? input_t<true, true, 4>(x, v, N, C, H, W, Cpg, TH, TW, pad, nchw, s)
+                           : v_f32 ? input_t<false, true, 4>(x, v, N, C, H, W, Cpg, TH, TW, pad, nchw, s)
+                                   : input_t<false, false, 4>(x, v, N, C, H, W, Cpg, TH, TW, pad, nchw, s);
     return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_wino_weight(const void *w, void *u, int C_out, int C, int Cpg, int gm, int m, bool f32,
-                               cudaStream_t s) {
-    const int a = m + 2;
-    const long long work = static_cast<long long>(a) * a * C_out * Cpg * gm;
-    if (m == 2) {
-        if (f32)
-            wino_weight_kernel<true, 2><<<wino_grid(work), kWgThreads256, 0, s>>>(w, u, C_out, C, Cpg, gm, Cpg * gm);
-        else
-            wino_weight_kernel<false, 2><<<wino_grid(work), kWgThreads256, 0, s>>>(w, u, C_out, C, Cpg, gm, Cpg * gm);
-    } else if (m == 4) {
-        if (f32)
-            wino_weight_kernel<true, 4><<<wino_grid(work), kWgThreads256, 0, s>>>(w, u, C_out, C, Cpg, gm, Cpg * gm);
-        else
-            wino_weight_kernel<false, 4><<<wino_grid(work), kWgThreads256, 0, s>>>(w, u, C_out, C, Cpg, gm, Cpg * gm);
-    } else {
-        return cudaErrorInvalidValue;
-    }
+template <bool kF32, bool kUF32, int kM>
+cudaError_t weight_t(const void *w, void *u, int C_out, int C, int Cpg, int gm, cudaStream_t s) {
+    const long long work = static_cast<long long>(kM + 2) * (kM + 2) * C_out * Cpg * gm;
+    wino_weight_kernel<kF32, kUF32, kM><<<wino_grid(work), kWgThreads256, 0, s>>>(w, u, C_out, C, Cpg, gm, Cpg * gm);
     return cudaGetLastError();
+}
+
+cudaError_t launch_wino_weight(const void *w, void *u, int C_out, int C, int Cpg, int gm, int m, bool f32, bool u_f32,
+                               cudaStream_t s) {
+    if (f32 && !u_f32) return cudaErrorInvalidValue;
+    if (m == 2) return f32 ? weight_t<true, true, 2>(w, u, C_out, C, Cpg, gm, s)
+                           : u_f32 ? weight_t<false, true, 2>(w, u, C_out, C, Cpg, gm, s)
+                                   : weight_t<false, false, 2>(w, u, C_out, C, Cpg, gm, s);
+    if (m == 4) return f32 ? weight_t<true, true, 4>(w, u, C_out, C, Cpg, gm, s)
+                           : u_f32 ? weight_t<false, true, 4>(w, u, C_out, C, Cpg, gm, s)
+                                   : weight_t<false, false, 4>(w, u, C_out, C, Cpg, gm, s);
+    return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_wino_output(const float *mp, const void *bias, void *y, int N, int C_out, int Ho, int Wo, int TH,

@@ -73,8 +73,8 @@ int conv2d_output_size(int in, int k, int stride, int pad, int dilation, int *ou
  * C_out * Kh * Kw * Cpg elements of dtype, where Cpg is C_in/groups rounded up
  * to a multiple of 8 (bf16) or 4 (fp32), followed -- for groups = 1 and fewer
  * than 32 bytes of input channels per pixel -- by ready-made shared-memory images
- * of the weight matrix for the few-channel kernel.  Narrow groups (fewer than 64
- * output channels each, C_in/groups a multiple of 8 bf16 / 4 fp32) are packed gm at
+ * of the weight matrix for the few-channel kernel.  Narrow bf16 groups (fewer than 64
+ * output channels each, C_in/groups a multiple of 8) are packed gm at
  * a time as one block-diagonal group, Cpg = gm * C_in/groups, with gm the largest
  * divisor of groups that keeps gm * C_out/groups <= 128 and gm * C_in/groups * the
  * element size <= 256 bytes; the forward pass then computes gm groups per product. */
@@ -340,13 +340,16 @@ int conv3d_forward(const void *x, const void *w_packed, const void *bias, void *
  * transform, the (m+2)^2 channel products (on the tensor cores, fp32 results) and the
  * output transform (+ bias, one rounding) run as three steps through the workspace.
  * Results equal conv2d_forward's up to rounding; the transforms enlarge the rounding
- * error, more for m = 4 (§5.1's numerical caveat).  Arguments as conv2d_forward for a
+ * error, more for m = 4 (§5.1's numerical caveat): with bf16 data, m = 2 keeps its
+ * transformed tiles and filters in bf16, while m = 4 keeps them, and runs their product,
+ * in fp32 (three TF32 products), since in bf16 its error exceeds the bf16 tolerance of
+ * this library (measured 6% of max |y| against 2%).  Arguments as conv2d_forward for a
  * 3x3 filter with stride 1, dilation 1 and groups 1; CONV_ERR_INVALID_ARG for m other
  * than 2 or 4. */
 
 /* Bytes of conv2d_pack_weight_winograd's output: (m+2)^2 * C_out rows of C_in channels
  * padded to 16 bytes (times the group merge factor of conv2d_packed_weight_size for
- * C_out < 64), dtype elements. */
+ * C_out < 64), elements of the transform type (dtype for m = 2, fp32 for m = 4). */
 int conv2d_winograd_packed_weight_size(int C_out, int C_in, int m, conv_dtype_t dtype, size_t *bytes);
 
 /* The transformed filters U = G g G^T of w_oihw (C_out, C_in, 3, 3), packed for the

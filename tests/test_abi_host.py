@@ -61,7 +61,7 @@ def test_packed_weight_size(lib):
     # many channels or groups: only the (C_out, Kh, Kw, Cpg) weights
     # 32 groups of 16 -> 16 channels: merged 8 at a time, block-diagonal rows of 8 * 16 channels
     assert cb.conv2d_packed_weight_size(512, 512, 3, 3, 32, cb.CONV_BF16) == 512 * 9 * 16 * 8 * 2
-    assert cb.conv2d_packed_weight_size(512, 512, 3, 3, 32, cb.CONV_F32) == 512 * 9 * 16 * 4 * 4  # 4 at a time
+    assert cb.conv2d_packed_weight_size(512, 512, 3, 3, 32, cb.CONV_F32) == 512 * 9 * 16 * 4  # fp32: no merge
     assert cb.conv2d_packed_weight_size(24, 24, 3, 3, 4, cb.CONV_BF16) == 24 * 9 * 8 * 2  # 12-byte rows: no merge
     assert cb.conv2d_packed_weight_size(256, 256, 3, 3, 1, cb.CONV_BF16) == 256 * 9 * 256 * 2
     # few input channels: followed (256-byte aligned) by the gather kernel's images,
@@ -231,7 +231,7 @@ def test_depthwise_plans(lib):
     stride-1 square 3/5/7 filters, channel-padded copy when 16-byte rows need it."""
     d = _plan((64, 256, 56, 56, 256, 3, 3, 1, 1, 1, 256), sms=148)
     assert (d["kernel"], d["a_load"], d["xcopy"], d["workspace"]) == ("depthwise", "tile", 0, 0)
-    assert d["units"] == 4 * 64 * 2 * 7            # 64-channel chunks x images x 32x8 output tiles
+    assert d["units"] == 4 * 64 * 2 * 7            # 64-channel chunks x images x 30x8 output tiles
     odd = _plan((2, 20, 9, 9, 20, 5, 3, 2, 2, 2, 20), sms=148)   # 40-byte rows: padded copy
     assert odd["kernel"] == "depthwise" and odd["xcopy"] == 1
     assert odd["workspace"] == 2 * 9 * 9 * 24 * 2 + (256 - (2 * 9 * 9 * 24 * 2) % 256) % 256
@@ -287,9 +287,23 @@ def test_winograd_sizes_on_the_host(lib):
     # F(2x2,3x3): 16 transformed filters per (oc, c); 64 channels each way, no group merge
     assert cb.conv2d_winograd_packed_weight_size(64, 64, 2, cb.CONV_BF16) == 16 * 64 * 64 * 2
     assert cb.conv2d_winograd_packed_weight_size(64, 64, 4, cb.CONV_F32) == 36 * 64 * 64 * 4
+    assert cb.conv2d_winograd_packed_weight_size(64, 64, 4, cb.CONV_BF16) == 36 * 64 * 64 * 4  # fp32 transforms
     for m in (3, 6):
         with pytest.raises(cb.Conv2dError):
             cb.conv2d_winograd_packed_weight_size(8, 8, m, cb.CONV_BF16)
     ws = cb.conv2d_winograd_workspace_size(2, 64, 12, 12, 64, 1, 2, cb.CONV_BF16, "nhwc")
     tiles = 2 * 6 * 6
     assert ws >= tiles * 16 * 64 * 2 + tiles * 16 * 64 * 4  # V (bf16) and the fp32 products
+
+
+def test_binding_signatures_match_the_header_argument_counts():
+    """Every ctypes signature of the binding has as many arguments as the header's
+    declaration (a missing or extra argument would shift every later one)."""
+    text = open(HEADER, encoding="utf-8").read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    decls = re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(conv[23]d_\w+)\s*\(([^)]*)\)\s*;", text, flags=re.M)
+    assert decls
+    for name, params in decls:
+        params = params.strip()
+        count = 0 if params in ("", "void") else len([p for p in params.split(",") if p.strip()])
+        assert len(cb.SIGNATURES[name][0]) == count, (name, count, len(cb.SIGNATURES[name][0]))
