@@ -67,15 +67,37 @@ __device__ __forceinline__ void unpack16(const uint4 &u, float *f) {
     }
 }
 
-// acc[0..1] += x[0..1] * w[0..1] as one paired fp32 FMA (fma.rn.f32x2, two lanes per
-// instruction), each lane rounded as fmaf would round it.
-__device__ __forceinline__ void ffma2(float *acc, const float *x, const float *w) {
-    uint64_t a, xx, ww;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "f"(acc[0]), "f"(acc[1]));
-    asm("mov.b64 %0, {%1, %2};" : "=l"(xx) : "f"(x[0]), "f"(x[1]));
-    asm("mov.b64 %0, {%1, %2};" : "=l"(ww) : "f"(w[0]), "f"(w[1]));
-    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(a) : "l"(xx), "l"(ww));
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(acc[0]), "=f"(acc[1]) : "l"(a));
+// Paired fp32 arithmetic: a 64-bit register holds two fp32 lanes (channels 2i, 2i+1).
+// fma2 is one fma.rn.f32x2 -- two fused multiply-adds per instruction, each lane rounded
+// as fmaf rounds it.
+__device__ __forceinline__ uint64_t pair(uint32_t lo, uint32_t hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+    return r;
+}
+
+__device__ __forceinline__ void fma2(uint64_t &acc, uint64_t x, uint64_t w) {
+    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(x), "l"(w));
+}
+
+__device__ __forceinline__ void unpair(uint64_t v, float &lo, float &hi) {
+    uint32_t a, b;
+    asm("mov.b64 {%0, %1}, %2;" : "=r"(a), "=r"(b) : "l"(v));
+    lo = __uint_as_float(a);
+    hi = __uint_as_float(b);
+}
+
+// 16 bytes of channels as kV/2 fp32 pairs (bf16: each 32-bit word holds channels 2i, 2i+1).
+template <bool kF32>
+__device__ __forceinline__ void unpack16_pairs(const uint4 &u, uint64_t *p) {
+    if constexpr (kF32) {
+        p[0] = pair(u.x, u.y);
+        p[1] = pair(u.z, u.w);
+    } else {
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) p[i] = pair(w[i] << 16, w[i] & 0xFFFF0000u);
+    }
 }
 
 struct DwTile {
@@ -226,29 +248,46 @@ __global__ void __launch_bounds__(kDwThreads, 1) dw_kernel(const __grid_constant
                 const int ow0 = t.tw * p.TW + px0;
                 if (oh >= p.Ho || ow0 >= p.Wo) continue;
                 float acc[kR][kV];
+                if constexpr (kKW > 0) {
+                    // stride 1, unit dilation, kKW x kKW: every filter row reads a window of
+                    // kR + kKW - 1 input pixels once; products in fp32 pairs
+                    constexpr int kP = kV / 2;
+                    uint64_t accp[kR][kP];
 #pragma unroll
-                for (int r = 0; r < kR; ++r)
+                    for (int r = 0; r < kR; ++r)
 #pragma unroll
-                    for (int v = 0; v < kV; ++v) acc[r][v] = 0.f;
-                for (int kh = 0; kh < p.Kh; ++kh) {
-                    const int row = py * p.stride + kh * p.dilation;
-                    const uint8_t *rp = stg + static_cast<size_t>(row) * p.IW * kDwRowBytes + cg * 16;
-                    const uint8_t *wp = wsm + kh * p.Kw * kDwRowBytes + cg * 16;
-                    if constexpr (kKW > 0) {
-                        float win[kR + kKW - 1][kV];
+                        for (int v = 0; v < kP; ++v) accp[r][v] = 0ull;
+#pragma unroll
+                    for (int kh = 0; kh < kKW; ++kh) {
+                        const uint8_t *rp = stg + static_cast<size_t>(py + kh) * p.IW * kDwRowBytes + cg * 16;
+                        const uint8_t *wp = wsm + kh * kKW * kDwRowBytes + cg * 16;
+                        uint64_t win[kR + kKW - 1][kP];
 #pragma unroll
                         for (int j = 0; j < kR + kKW - 1; ++j)
-                            unpack16<kF32>(*reinterpret_cast<const uint4 *>(rp + (px0 + j) * kDwRowBytes), win[j]);
+                            unpack16_pairs<kF32>(*reinterpret_cast<const uint4 *>(rp + (px0 + j) * kDwRowBytes), win[j]);
 #pragma unroll
                         for (int kw = 0; kw < kKW; ++kw) {
-                            float wv[kV];
-                            unpack16<kF32>(*reinterpret_cast<const uint4 *>(wp + kw * kDwRowBytes), wv);
+                            uint64_t wv[kP];
+                            unpack16_pairs<kF32>(*reinterpret_cast<const uint4 *>(wp + kw * kDwRowBytes), wv);
 #pragma unroll
                             for (int r = 0; r < kR; ++r)
 #pragma unroll
-                                for (int v = 0; v < kV; v += 2) ffma2(&acc[r][v], &win[r + kw][v], &wv[v]);
+                                for (int v = 0; v < kP; ++v) fma2(accp[r][v], win[r + kw][v], wv[v]);
                         }
-                    } else {
+                    }
+#pragma unroll
+                    for (int r = 0; r < kR; ++r)
+#pragma unroll
+                        for (int v = 0; v < kP; ++v) unpair(accp[r][v], acc[r][2 * v], acc[r][2 * v + 1]);
+                } else {
+#pragma unroll
+                    for (int r = 0; r < kR; ++r)
+#pragma unroll
+                        for (int v = 0; v < kV; ++v) acc[r][v] = 0.f;
+                    for (int kh = 0; kh < p.Kh; ++kh) {
+                        const int row = py * p.stride + kh * p.dilation;
+                        const uint8_t *rp = stg + static_cast<size_t>(row) * p.IW * kDwRowBytes + cg * 16;
+                        const uint8_t *wp = wsm + kh * p.Kw * kDwRowBytes + cg * 16;
                         for (int kw = 0; kw < p.Kw; ++kw) {
                             float wv[kV];
                             unpack16<kF32>(*reinterpret_cast<const uint4 *>(wp + kw * kDwRowBytes), wv);
@@ -258,7 +297,7 @@ __global__ void __launch_bounds__(kDwThreads, 1) dw_kernel(const __grid_constant
                                 float xv[kV];
                                 unpack16<kF32>(*reinterpret_cast<const uint4 *>(rp + col * kDwRowBytes), xv);
 #pragma unroll
-                                for (int v = 0; v < kV; v += 2) ffma2(&acc[r][v], &xv[v], &wv[v]);
+                                for (int v = 0; v < kV; ++v) acc[r][v] = fmaf(xv[v], wv[v], acc[r][v]);
                             }
                         }
                     }
