@@ -148,6 +148,12 @@ struct Plan {
     bool gather;    // few input channels: the software-gather kernel reads x directly
     bool gather_t;  // ... in its transposed form (gather_t.cu): bf16 NCHW, one output row per tile
     int tpix;       // its pixels per tile (Wo rounded up to 16)
+    int nhalo;      // its staged-row buffers
+    int nacc;       // its accumulators
+    int nout;       // its output images
+    int rt;         // its output rows per tile
+    int kt;         // its reduction length per tile
+    bool a_tmem;    // its A operand resident in tensor memory
     bool vec_rows;  // ... with 16-byte row loads (NCHW, aligned rows, unit dilation)
     bool halo;      // ... from input rows staged in shared memory by TMA
     int R, BW, ME;  // halo rows per tile, staged row width, left zero margin (elements)
@@ -438,26 +444,59 @@ int make_plan(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stri
         const int order = p.vec_rows ? 1 : 0;
         if (slots >= 2 && smem <= kSmemBudget && gi.kpad[order] == p.Kpad) {
             p.gather = true;
-            // Transposed form: output channels on the lanes, one output row per tile,
-            // channel rows stored straight into NCHW y.  Needs the row-vector order,
-            // whole 16-byte stores per row (Wo % 8 == 0) and the row's staged input box.
+            // Transposed form: output channels on the lanes, one or two output rows per
+            // tile, channel rows stored into NCHW y without transposition.  Needs the
+            // row-vector order, whole 16-byte pieces per row (Wo % 8 == 0) and the tile's
+            // staged input box.
             p.gather_t = false;
-            if (!p.f32 && p.vec_rows && p.Wo % 8 == 0 && p.Wo <= 256 && C_out <= 128 && pad <= per16 &&
-                C_in * Kh <= 32) {
+            if (!p.f32 && p.vec_rows && p.Wo % 8 == 0 && p.Wo <= 256 && C_out <= 128 && pad <= per16) {
                 const int iw0_max = (p.Wo - 1) * stride - pad;
                 const int BW = round_up(iw0_max + per16 + per16 + 2, per16);
                 const int tpix = round_up(p.Wo, 16);
-                const size_t hb = static_cast<size_t>(C_in) * Kh * BW * p.elt;
-                const size_t tsmem = gather_t_smem_bytes(p.Kpad, tpix, hb);
-                if (BW <= 256 && W <= BW && Kh <= 256 && tsmem <= kSmemBudget) {
-                    p.gather_t = true;
-                    p.halo = true;
-                    p.R = Kh;
-                    p.BW = BW;
-                    p.ME = per16;
-                    p.tpix = tpix;
-                    p.tma_out = false;
-                    smem = tsmem;
+                // Two output rows per tile when the channels fill half the lanes, else one.
+                // The output block of a tile goes out by TMA stores from double-buffered
+                // output images when they fit beside at least three staged-row buffers,
+                // else from one image, else straight from the registers; then as many
+                // staged-row buffers as fit (up to the kernel's limit): one tile's work is
+                // shorter than the latency of its rows' load.
+                for (int rt = C_out <= 64 ? 2 : 1; rt >= 1 && !p.gather_t; --rt) {
+                    const int R = Kh + (rt - 1) * stride;
+                    if (C_in * R > gather_t_max_chunks() || BW > 256 || W > BW || R > 256) continue;
+                    const int kt = rt == 1 ? p.Kpad : round_up(C_in * R * per16, 32 / p.elt);
+                    const size_t hb = static_cast<size_t>(C_in) * R * BW * p.elt;
+                    const size_t ob = static_cast<size_t>(bn) * rt * p.Wo * p.elt;
+                    // A in tensor memory when at least two accumulators fit beside it (its
+                    // kt/2 columns), else in shared memory
+                    const int acc_tm = (512 - kt / 2) / tpix;
+                    for (int a_tm = (tpix >= 64 && acc_tm >= 2) ? 1 : 0; a_tm >= 0 && !p.gather_t; --a_tm) {
+                        const int opts[3][3] = {{1, 2, 3}, {1, 1, 2}, {0, 1, 2}};  // tma_out, images, fewest row buffers
+                        for (const auto &o : opts) {
+                            const size_t obytes = o[0] ? ob : 0;
+                            int nhalo = gather_t_max_halo();
+                            while (nhalo > o[2] &&
+                                   gather_t_smem_bytes(kt, tpix, hb, nhalo, obytes, o[1], a_tm != 0) > kSmemBudget)
+                                --nhalo;
+                            const size_t tsmem = gather_t_smem_bytes(kt, tpix, hb, nhalo, obytes, o[1], a_tm != 0);
+                            if (tsmem > kSmemBudget) continue;
+                            p.gather_t = true;
+                            p.rt = rt;
+                            p.kt = kt;
+                            p.a_tmem = a_tm != 0;
+                            p.nhalo = nhalo;
+                            p.nout = o[1];
+                            p.tma_out = o[0] != 0;
+                            // as many accumulators as the 512 tensor-memory columns hold
+                            const int acc = a_tm ? acc_tm : 512 / tpix;
+                            p.nacc = acc < gather_t_max_acc() ? acc : gather_t_max_acc();
+                            p.halo = true;
+                            p.R = R;
+                            p.BW = BW;
+                            p.ME = per16;
+                            p.tpix = tpix;
+                            smem = tsmem;
+                            break;
+                        }
+                    }
                 }
             }
             p.w_image_off = gi.off[order];
@@ -466,7 +505,7 @@ int make_plan(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stri
             p.acols = acols;
             // at least 120 KB, so that one CTA (holding all tensor memory) runs per SM
             p.smem = smem > 120 * 1024 ? smem : 120 * 1024;
-            p.n_mtiles = p.gather_t ? N * p.Ho : static_cast<int>((p.M + 127) / 128);
+            p.n_mtiles = p.gather_t ? N * ((p.Ho + p.rt - 1) / p.rt) : static_cast<int>((p.M + 127) / 128);
             p.n_ntiles = 1;
             p.splits = 1;
             p.units = p.n_mtiles;
@@ -683,12 +722,31 @@ int gather_impl(const Plan &p, const void *x, const void *w_packed, const void *
     g.tmem_cols = 512;  // accumulators and A slots
     if (p.gather_t) {
         g.tpix = p.tpix;
+        g.nhalo = p.nhalo;
+        g.nacc = p.nacc;
+        g.nout = p.nout;
+        g.rt = p.rt;
+        g.kt = p.kt;
+        g.a_tmem = p.a_tmem ? 1 : 0;
         g.tmem_cols = 32;
-        while (g.tmem_cols < static_cast<uint32_t>(2 * p.tpix)) g.tmem_cols <<= 1;
+        while (g.tmem_cols < static_cast<uint32_t>(p.nacc * p.tpix + (p.a_tmem ? p.kt / 2 : 0))) g.tmem_cols <<= 1;
     }
     g.cw = p.cw;
     g.tma_out = p.tma_out ? 1 : 0;
-    if (p.tma_out) {
+    if (p.tma_out && p.gather_t) {
+        // y as (Wo, Ho, C_out, N); one box per tile: the tile's output rows of every channel
+        const cuuint64_t wo = static_cast<cuuint64_t>(p.Wo), ho = static_cast<cuuint64_t>(p.Ho);
+        cuuint64_t dims[4] = {wo, ho, static_cast<cuuint64_t>(p.C_out), static_cast<cuuint64_t>(p.N)};
+        cuuint64_t strides[3] = {wo * p.elt, wo * ho * p.elt, wo * ho * p.elt * p.C_out};
+        cuuint32_t box[4] = {static_cast<cuuint32_t>(p.Wo), static_cast<cuuint32_t>(p.rt),
+                             static_cast<cuuint32_t>(p.BN), 1};
+        cuuint32_t estr[4] = {1, 1, 1, 1};
+        CUresult r = g_encode_tiled(&g.tmap_y, tma_type(p), 4, y, dims, strides, box, estr,
+                                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                                    CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS)
+            return fail(CONV_ERR_CUDA, "cuTensorMapEncodeTiled (output rows) failed (%d)", static_cast<int>(r));
+    } else if (p.tma_out) {
         const cuuint64_t howo = static_cast<cuuint64_t>(p.Ho) * p.Wo;
         cuuint64_t dims[3] = {howo, static_cast<cuuint64_t>(p.C_out), static_cast<cuuint64_t>(p.N)};
         cuuint64_t strides[2] = {howo * p.elt, howo * p.elt * p.C_out};
@@ -980,10 +1038,12 @@ int describe_impl(bool explicit_im2col, int N, int C_in, int H, int W, int C_out
         buf, buflen,
         "{\"kernel\": \"%s\", \"pair\": %d, \"a_load\": \"%s\", \"BN\": %d, \"cb\": %d, "
         "\"stages\": %d, \"splits\": %d, \"units\": %d, \"xcopy\": %d, \"halo\": %d, "
-        "\"tma_out\": %d, \"Kpad\": %d, \"smem\": %zu, \"workspace\": %zu, \"sms\": %d}",
+        "\"tma_out\": %d, \"Kpad\": %d, \"smem\": %zu, \"workspace\": %zu, \"sms\": %d, "
+        "\"rows\": %d, \"out_images\": %d, \"a_tmem\": %d}",
         kernel, p.pair ? 1 : 0, a_load, p.BN, p.gather ? 0 : p.cb,
         p.stages, p.gather ? 1 : p.splits, p.gather ? p.n_mtiles : p.units, p.xcopy ? 1 : 0,
-        p.halo ? 1 : 0, p.tma_out ? 1 : 0, p.gather ? p.Kpad : 0, p.smem, p.ws_total, sms);
+        p.halo ? 1 : 0, p.tma_out ? 1 : 0, p.gather ? p.Kpad : 0, p.smem, p.ws_total, sms,
+        p.gather_t ? p.rt : 0, p.gather_t && p.tma_out ? p.nout : 0, p.gather_t && p.a_tmem ? 1 : 0);
     if (n < 0 || static_cast<size_t>(n) >= buflen)
         return fail(CONV_ERR_INVALID_ARG, "buf of %zu bytes is too small (%d needed)", buflen, n + 1);
     return ok();

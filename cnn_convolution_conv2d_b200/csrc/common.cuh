@@ -67,7 +67,7 @@ struct IgemmParams {
 // order), padded to Kpad.
 struct GatherParams {
     CUtensorMap tmap_x;    // halo mode: 4-D tiled map of x (W, H, C, N)
-    CUtensorMap tmap_y;    // tma_out mode: 3-D tiled map of y (Ho*Wo, C_out, N)
+    CUtensorMap tmap_y;    // tma_out mode: 3-D tiled map of y (Ho*Wo, C_out, N); gather_t: 4-D (Wo, Ho, C_out, N)
     const void *x;
     const void *w_packed;  // (C_out, Kh, Kw, Cpg) from conv2d_pack_weight
     const void *w_image;   // the kernel's shared-memory weight image (written by the pack)
@@ -85,6 +85,12 @@ struct GatherParams {
     int tma_out;           // epilogue stages each tile channel-major and stores it by TMA
     int cw;                // output channels per epilogue group
     int tpix;              // transposed kernel (gather_t.cu): pixels per tile, Wo rounded up to 16
+    int nhalo;             // ... its staged-row buffers (loads run this many tiles ahead)
+    int nacc;              // ... its accumulators in tensor memory
+    int nout;              // ... its output images (tma_out)
+    int rt;                // ... output rows per tile (1, or 2 when C_out <= 64)
+    int kt;                // ... the reduction length of a tile's product (padded)
+    int a_tmem;            // ... and whether A is resident in tensor memory
     uint32_t tmem_cols;
     void *y;
     const void *bias;
@@ -149,7 +155,10 @@ size_t gather_smem_bytes(bool f32, int BN, int Kpad, size_t halo_bytes, size_t o
 // The transposed few-channel kernel (gather_t.cu): bf16, NCHW in and out, one output row
 // per tile, output channels on the tensor-memory lanes.
 cudaError_t launch_gather_t(const GatherParams &p, int grid, size_t smem, cudaStream_t stream);
-size_t gather_t_smem_bytes(int Kpad, int tpix, size_t halo_bytes);
+size_t gather_t_smem_bytes(int kt, int tpix, size_t halo_bytes, int nhalo, size_t out_bytes, int nout, bool a_tmem);
+int gather_t_max_halo();
+int gather_t_max_acc();
+int gather_t_max_chunks();
 int gather_max_stages();
 int igemm_threads(bool f32);
 

@@ -169,9 +169,11 @@ def test_plan_for_the_workloads_on_a_148_sm_device(lib):
     p3 = _plan((64, 256, 56, 56, 256, 3, 3, 1, 1, 1, 1), sms=148)    # 3x3: hardware im2col, pairs
     assert (p3["kernel"], p3["pair"], p3["a_load"], p3["BN"], p3["units"]) == ("igemm", 1, "im2col", 256, 784)
     stem = _plan((32, 3, 224, 224, 64, 7, 7, 2, 3, 1, 1), layout="nchw", sms=148)
-    # the transposed few-channel kernel: one output row (112 pixels) per tile
-    assert (stem["kernel"], stem["halo"], stem["BN"], stem["workspace"], stem["units"]) == \
-        ("gather_t", 1, 64, 0, 32 * 112)
+    # the transposed few-channel kernel: 64 channels fill half the lanes, so a tile is two
+    # output rows (2 x 112 pixels), stored from double-buffered output images by TMA; the
+    # weights stay in tensor memory
+    assert (stem["kernel"], stem["halo"], stem["BN"], stem["workspace"], stem["units"], stem["rows"],
+            stem["out_images"], stem["a_tmem"]) == ("gather_t", 1, 64, 0, 32 * 56, 2, 2, 1)
     nhwc_out = _plan((32, 3, 224, 224, 64, 7, 7, 2, 3, 1, 1), layout="nhwc", sms=148)
     assert nhwc_out["kernel"] == "gather"                              # channels-last: the lane-per-pixel form
     assert stem["Kpad"] == 176                                         # 3 channels x 7 rows x 8 (7 taps + 1) -> 168 -> 176

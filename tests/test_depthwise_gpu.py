@@ -55,6 +55,8 @@ DW_EDGE = [  # N, C, H, W, Kh, Kw, stride, pad, dilation
     (1, 200, 5, 70, 3, 3, 1, 1, 1),     # 200 channels: partial last chunk; wide image
     (2, 64, 40, 12, 3, 3, 3, 4, 1),     # stride 3, pad larger than the filter's reach
     (1, 8, 300, 9, 3, 1, 1, 1, 1),      # tall image: ten 32-row tiles, 3x1 filter
+    (1, 6, 7, 9, 3, 3, 1, 1, 1),        # 6 channels (not a multiple of 4), odd output rows
+    (2, 12, 11, 13, 5, 5, 1, 2, 1),     # 5x5 window, odd output rows, ragged columns
 ]
 
 

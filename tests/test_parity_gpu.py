@@ -104,6 +104,31 @@ def test_edge_shapes(shape, layout, dtype):
     parity.assert_close(cfg, parity.run_gpu(cfg, inp), parity.run_oracle(cfg, inp), str(shape))
 
 
+TRANSPOSED_FIRST_LAYER = [  # bf16 NCHW, few channels, Wo % 8 == 0: the transposed kernel
+    # shape, (output rows per tile, output images (0: stored straight from the registers),
+    #         A in tensor memory)
+    ((12, 3, 128, 128, 64, 7, 7, 2, 3, 1, 1), (2, 2, 1)),   # 384 row-pair tiles: each CTA wraps its rings
+    ((3, 3, 64, 80, 40, 5, 5, 1, 2, 1, 1), (2, 2, 1)),      # stride 1; C_out 40: image rows 40..47 clipped
+    ((2, 3, 40, 96, 24, 3, 3, 2, 1, 1, 1), (2, 2, 0)),      # 3x3 stride 2, C_out 24, 48 pixels: A in shared memory
+    ((2, 3, 30, 64, 32, 7, 7, 2, 3, 1, 1), (2, 2, 0)),      # Ho = 15: the last pair's second row clipped
+    ((2, 3, 40, 96, 96, 3, 3, 2, 1, 1, 1), (1, 2, 0)),      # C_out 96: one row per tile, A in shared memory
+    ((2, 4, 64, 128, 128, 7, 7, 1, 3, 1, 1), (1, 2, 1)),    # C_out 128, reduction 224
+    ((1, 4, 17, 160, 128, 8, 7, 1, 3, 1, 1), (1, 1, 1)),    # reduction 256, 160 pixels: room for one image
+    ((1, 4, 17, 192, 128, 8, 7, 1, 3, 1, 1), (1, 0, 1)),    # 192 pixels: no room for an image
+]
+
+
+@pytest.mark.parametrize("shape,form", TRANSPOSED_FIRST_LAYER, ids=lambda s: "x".join(map(str, s)))
+def test_transposed_first_layer(shape, form):
+    N, C_in, H, W, C_out, Kh, Kw, s, p, d, g = shape
+    plan = cb.conv2d_describe_plan(*shape, cb.CONV_BF16, "nchw")
+    assert (plan["kernel"], plan["rows"], plan["out_images"], plan["a_tmem"]) == ("gather_t",) + form, plan
+    cfg = workloads.ConvConfig("first", N, C_in, H, W, C_out, Kh, Kw, s, p, d, g, True, "bf16", "nchw",
+                               seed=sum(shape))
+    inp = workloads.make_inputs(cfg)
+    parity.assert_close(cfg, parity.run_gpu(cfg, inp), parity.run_oracle(cfg, inp), str(shape))
+
+
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("explicit", [False, True])
 @pytest.mark.parametrize("shape", [(2, 3, 9, 11, 4, 3, 3, 2, 1, 1, 1), (2, 16, 12, 12, 32, 3, 3, 1, 1, 1, 1),
