@@ -64,6 +64,7 @@ SIGNATURES = {
     "conv3d_pack_weight": ([_P, _P] + [_I] * 7 + [_P], _I),
     "conv3d_workspace_size": ([_I] * 13 + [_I, _I, ctypes.POINTER(_S)], _I),
     "conv3d_forward": ([_P, _P, _P, _P] + [_I] * 13 + [_I, _I, _P, _S, _P], _I),
+    "conv3d_describe_plan": ([_I] * 13 + [_I, _I, _I, ctypes.c_char_p, ctypes.c_size_t], _I),
     "conv2d_winograd_packed_weight_size": ([_I, _I, _I, _I, ctypes.POINTER(_S)], _I),
     "conv2d_pack_weight_winograd": ([_P, _P, _I, _I, _I, _I, _P], _I),
     "conv2d_winograd_workspace_size": ([_I] * 7 + [_I, _I, ctypes.POINTER(_S)], _I),
@@ -272,6 +273,16 @@ def conv2d_describe_plan(N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, gr
     _check(load().conv2d_describe_plan(N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype,
                                        _layout_code(layout), 1 if explicit_im2col else 0, int(sms), buf,
                                        ctypes.sizeof(buf)))
+    return json.loads(buf.value.decode())
+
+
+def conv3d_describe_plan(N, C_in, D, H, W, C_out, Kd, Kh, Kw, stride, pad, dilation, groups, dtype, layout,
+                         sms=-1) -> dict:
+    """conv3d_forward's plan for a problem (kernel, tile shape, passes) as a dict."""
+    import json
+    buf = ctypes.create_string_buffer(512)
+    _check(load().conv3d_describe_plan(N, C_in, D, H, W, C_out, Kd, Kh, Kw, stride, pad, dilation, groups, dtype,
+                                       _layout_code(layout), int(sms), buf, ctypes.sizeof(buf)))
     return json.loads(buf.value.decode())
 
 

@@ -137,6 +137,8 @@ struct Plan {
     int N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups;
     int pad_w;      // column padding (= pad, the row padding, for every caller-facing entry)
     bool vol;       // 3-D convolution: input depth D, filter depth Kd, output depth Do
+    bool vreuse;    // ... on the input-slice-reuse kernel (vol.cu)
+    int vJ, vn_k, vn_odb;  // its output slices per unit, tiles per slice, slice blocks
     int D, Kd, Do;
     bool f32;
     int elt;
@@ -556,6 +558,37 @@ int make_plan(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stri
         base = pair_units;
     }
     p.units = static_cast<int>(base * p.splits);
+    // 3-D, stride 1, unit dilation, 64 input channels, at most 128 output channels: the
+    // kernel that loads each input depth slice once for all the depth taps that read it
+    // (vol.cu), with two accumulator sets of J slices in tensor memory and at least three
+    // stages beside the weights of two (kh, kw).
+    p.vreuse = false;
+    if (vol && !p.f32 && !padw && !explicit_im2col && groups == 1 && layout == CONV_NHWC && stride == 1 &&
+        dilation == 1 && C_in == 64 && C_out % 32 == 0 && C_out <= 128 && (p.Ho * p.Wo) % 32 == 0 &&
+        p.Ho * p.Wo >= 128) {
+        int J = 256 / C_out < vol_reuse_max_j() ? 256 / C_out : vol_reuse_max_j();
+        J = J < p.Do ? J : p.Do;
+        int vst = vol_reuse_max_stages();
+        while (vst > 3 && vol_reuse_smem_bytes(p.Kd, C_out, vst) > kSmemBudget) --vst;
+        if (vol_reuse_smem_bytes(p.Kd, C_out, vst) <= kSmemBudget) {
+            p.vreuse = true;
+            p.vJ = J;
+            p.vn_k = (p.Ho * p.Wo + 127) / 128;
+            p.vn_odb = (p.Do + J - 1) / J;
+            p.pair = false;
+            p.splits = 1;
+            p.BN = C_out;
+            p.n_ntiles = 1;
+            p.units = N * p.vn_odb * p.vn_k;
+            p.stages = vst;
+            p.tma_out = true;
+            p.smem = vol_reuse_smem_bytes(p.Kd, C_out, vst);
+            p.ws_total = 0;
+            p.xcopy = false;
+            *P = p;
+            return CONV_OK;
+        }
+    }
     // bf16 channels-last output leaves through shared memory and TMA stores when
     // every 32-column block of a tile lies inside its group's columns.
     p.tma_out = !p.f32 && layout == CONV_NHWC && p.splits == 1 && !(padw && padw->partial_out) &&
@@ -860,6 +893,7 @@ int device_plan(bool explicit_im2col, int N, int C_in, int H, int W, int C_out, 
                        explicit_im2col, dev ? dev->sms : 0, p, cfg.pair_mode, true, padw, vol);
     if (st != CONV_OK) return st;
     p->pair_clusters = 0;
+    if (p->vreuse) return CONV_OK;
     if (p->pair && dev) {
         const bool a_im2col = !(explicit_im2col || p->direct_a);
         p->pair_clusters = pair_cluster_limit(p->cb, a_im2col, p->smem, p->vol && a_im2col);
@@ -877,6 +911,58 @@ DeviceInfo *current_device_or_null() {
     if (cudaGetDeviceCount(&ndev) == cudaSuccess && ndev > 0 && device_info(&dev) == CONV_OK) return dev;
     cudaGetLastError();
     return nullptr;
+}
+
+// The 3-D path with input-slice reuse (vol.cu): one kernel, no scratch.
+int vol_impl(const Plan &p, const void *x, const void *w_packed, const void *bias, void *y, DeviceInfo *dev,
+             const Settings &cfg, cudaStream_t stream) {
+    VolParams v;
+    std::memset(&v, 0, sizeof(v));
+    int st = encode_a_im2col_5d(p, x, &v.tmap_a);
+    if (st != CONV_OK) return st;
+    st = encode_b(p, w_packed, &v.tmap_b);
+    if (st != CONV_OK) return st;
+    {
+        cuuint64_t dims[2] = {static_cast<cuuint64_t>(p.C_out), static_cast<cuuint64_t>(p.M)};
+        cuuint64_t strides[1] = {static_cast<cuuint64_t>(p.C_out) * p.elt};
+        cuuint32_t box[2] = {32, 32};
+        cuuint32_t estr[2] = {1, 1};
+        CUresult r = g_encode_tiled(&v.tmap_y, tma_type(p), 2, y, dims, strides, box, estr,
+                                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                                    CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS)
+            return fail(CONV_ERR_CUDA, "cuTensorMapEncodeTiled (output) failed (%d)", static_cast<int>(r));
+    }
+    v.M = static_cast<int>(p.M);
+    v.Do = p.Do;
+    v.HoWo2 = p.Ho * p.Wo;
+    v.Wo = p.Wo;
+    v.Kd = p.Kd;
+    v.Kh = p.Kh;
+    v.Kw = p.Kw;
+    v.taps = p.Kd * p.Kh * p.Kw;
+    v.pad = p.pad;
+    v.pad_w = p.pad_w;
+    v.BN = p.BN;
+    v.J = p.vJ;
+    v.n_k = p.vn_k;
+    v.n_odb = p.vn_odb;
+    v.units = p.units;
+    v.stages = p.stages;
+    uint32_t cols = 32;
+    while (cols < static_cast<uint32_t>(2 * p.vJ * p.BN)) cols <<= 1;
+    v.tmem_cols = cols;
+    v.bias = bias;
+    v.status = dev->status;
+    v.timeout_ns = cfg.timeout_ns;
+    v.starve = cfg.starve;
+    const int grid = p.units < dev->sms ? p.units : dev->sms;
+    cudaEvent_t ev_start = g_main_start, ev_stop = g_main_stop;
+    if (ev_start && ev_stop && (st = record_event(ev_start, stream)) != CONV_OK) return st;
+    cudaError_t e = launch_vol_reuse(v, grid, p.smem, stream);
+    if ((st = check_launch(e, "3-D product with input-slice reuse")) != CONV_OK) return st;
+    if (ev_start && ev_stop && (st = record_event(ev_stop, stream)) != CONV_OK) return st;
+    return ok();
 }
 
 // Shared body of conv2d_forward and conv2d_forward_im2col_gemm.
@@ -908,6 +994,7 @@ int forward_impl(bool explicit_im2col, const void *x, const void *w_packed, cons
 
     if (p.gather) return gather_impl(p, x, w_packed, bias, y, dev, cfg, stream);
     if (p.dw) return dw_impl(p, x, w_packed, bias, y, workspace, dev, cfg, stream);
+    if (p.vreuse) return vol_impl(p, x, w_packed, bias, y, dev, cfg, stream);
 
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     const void *x_nhwc = p.xcopy ? static_cast<const void *>(ws + p.off_xcopy) : x;
@@ -1015,25 +1102,25 @@ int forward_impl(bool explicit_im2col, const void *x, const void *w_packed, cons
 // no device-dependent choices); sms >= 0: as if the device had that many SMs.
 int describe_impl(bool explicit_im2col, int N, int C_in, int H, int W, int C_out, int Kh, int Kw,
                   int stride, int pad, int dilation, int groups, conv_dtype_t dtype,
-                  conv_layout_t layout, int sms, char *buf, size_t buflen) {
+                  conv_layout_t layout, int sms, char *buf, size_t buflen, const Vol *vol = nullptr) {
     if (!buf || buflen == 0) return fail(CONV_ERR_INVALID_ARG, "buf must not be NULL");
     const Settings cfg = settings_now();
     Plan p;
     int st = make_plan(N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype, layout,
-                       explicit_im2col, 0, &p, cfg.pair_mode);
+                       explicit_im2col, 0, &p, cfg.pair_mode, true, nullptr, vol);
     if (st != CONV_OK) return st;
     if (sms < 0) {
         DeviceInfo *dev = current_device_or_null();
         sms = dev ? dev->sms : 0;
         st = device_plan(explicit_im2col, N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups,
-                         dtype, layout, dev, cfg, &p);
+                         dtype, layout, dev, cfg, &p, nullptr, vol);
     } else {
         st = make_plan(N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype, layout,
-                       explicit_im2col, sms, &p, cfg.pair_mode);
+                       explicit_im2col, sms, &p, cfg.pair_mode, true, nullptr, vol);
     }
     if (st != CONV_OK) return st;
     const char *a_load = p.dw ? "tile" : p.gather ? "gather" : explicit_im2col ? "xcol" : p.direct_a ? "tiled_x" : "im2col";
-    const char *kernel = p.dw ? "depthwise" : p.gather_t ? "gather_t" : p.gather ? "gather" : "igemm";
+    const char *kernel = p.dw ? "depthwise" : p.vreuse ? "vol_reuse" : p.gather_t ? "gather_t" : p.gather ? "gather" : "igemm";
     const int n = std::snprintf(
         buf, buflen,
         "{\"kernel\": \"%s\", \"pair\": %d, \"a_load\": \"%s\", \"BN\": %d, \"cb\": %d, "
@@ -1670,6 +1757,14 @@ int conv2d_describe_plan(int N, int C_in, int H, int W, int C_out, int Kh, int K
                          int explicit_im2col, int sms, char *buf, size_t buflen) {
     return describe_impl(explicit_im2col != 0, N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation,
                          groups, dtype, layout, sms, buf, buflen);
+}
+
+int conv3d_describe_plan(int N, int C_in, int D, int H, int W, int C_out, int Kd, int Kh, int Kw, int stride,
+                         int pad, int dilation, int groups, conv_dtype_t dtype, conv_layout_t layout, int sms,
+                         char *buf, size_t buflen) {
+    const Vol vol{D, Kd};
+    return describe_impl(false, N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype, layout, sms, buf,
+                         buflen, &vol);
 }
 
 int conv2d_debug_set_pair_mode(int mode) {

@@ -62,6 +62,25 @@ struct IgemmParams {
     int starve;          // test hook: issue no loads
 };
 
+// One launch of the volume kernel with input-slice reuse (vol.cu): 3-D, bf16, stride 1,
+// unit dilation, C_in = 64, groups = 1, channels-last.  A unit is J output depth slices
+// of one 128-voxel tile of a depth slice; u = (n*n_odb + b)*n_k + k.
+struct VolParams {
+    CUtensorMap tmap_a;  // 5-D im2col map of x (c, w, h, d, n), boxes of 128 voxels x 64 channels
+    CUtensorMap tmap_b;  // packed weights {taps*64, C_out, 1}, boxes of 64 x C_out
+    CUtensorMap tmap_y;  // y as {C_out, M}, 32 x 32 boxes with 64-byte swizzle
+    int M, Do, HoWo2, Wo;
+    int Kd, Kh, Kw, taps, pad, pad_w;
+    int BN;              // = C_out (a multiple of 32, <= 128)
+    int J;               // output depth slices per unit (accumulators: 2*J*BN columns)
+    int n_k, n_odb, units, stages;
+    uint32_t tmem_cols;
+    const void *bias;
+    int *status;
+    long long timeout_ns;
+    int starve;
+};
+
 // One launch of the software-gather kernel (gather.cu) for inputs with few
 // channels: groups = 1, reduction index k = (kh*Kw + kw)*C + c (or the row-vector
 // order), padded to Kpad.
@@ -155,6 +174,10 @@ size_t gather_smem_bytes(bool f32, int BN, int Kpad, size_t halo_bytes, size_t o
 // The transposed few-channel kernel (gather_t.cu): bf16, NCHW in and out, one output row
 // per tile, output channels on the tensor-memory lanes.
 cudaError_t launch_gather_t(const GatherParams &p, int grid, size_t smem, cudaStream_t stream);
+cudaError_t launch_vol_reuse(const VolParams &p, int grid, size_t smem, cudaStream_t stream);
+size_t vol_reuse_smem_bytes(int Kd, int BN, int stages);
+int vol_reuse_max_stages();
+int vol_reuse_max_j();
 size_t gather_t_smem_bytes(int kt, int tpix, size_t halo_bytes, int nhalo, size_t out_bytes, int nout, bool a_tmem);
 int gather_t_max_halo();
 int gather_t_max_acc();

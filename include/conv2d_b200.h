@@ -304,7 +304,12 @@ int conv2d_backward_bias(const void *dy, void *db, int N, int C_out, int Ho, int
  * terms outside the volume dropped.  Stride, pad and dilation apply to all three
  * directions.  layout CONV_NCHW means NCDHW tensors, CONV_NHWC means NDHWC.  The same
  * implicit matrix product as conv2d_forward runs over output voxels, its input patches
- * staged by the tensor memory accelerator's 5-D im2col mode.  Beyond conv2d_forward's
+ * staged by the tensor memory accelerator's 5-D im2col mode.  bf16 NDHWC problems with
+ * stride 1, unit dilation, 64 input channels, groups 1 and at most 128 output channels
+ * (a multiple of 32; Ho*Wo a multiple of 32 and >= 128)
+ * run on a kernel that loads each input depth slice once for all the depth taps that read
+ * it (J output slices per unit of work; the sums are the same, their fp32 rounding order
+ * is per tap as elsewhere).  Beyond conv2d_forward's
  * errors: CONV_ERR_UNSUPPORTED when pad or pad - dilation*(K-1) lies outside
  * [-16, 15] in any direction (the 5-D im2col addressing range). */
 
@@ -330,6 +335,15 @@ int conv3d_forward(const void *x, const void *w_packed, const void *bias, void *
                    int stride, int pad, int dilation, int groups,
                    conv_dtype_t dtype, conv_layout_t layout,
                    void *workspace, size_t workspace_bytes, conv_stream_t stream);
+
+/* The plan conv3d_forward makes for a problem (conv2d_describe_plan's JSON object, with
+ * "kernel": "vol_reuse" for the kernel that loads each input depth slice once for all
+ * the depth taps that read it, "igemm" for the implicit GEMM over output voxels).
+ * Arguments as conv3d_forward; sms and buf as conv2d_describe_plan.  Nothing runs on
+ * a GPU. */
+int conv3d_describe_plan(int N, int C_in, int D, int H, int W, int C_out, int Kd, int Kh, int Kw,
+                         int stride, int pad, int dilation, int groups, conv_dtype_t dtype,
+                         conv_layout_t layout, int sms, char *buf, size_t buflen);
 
 /* ----------------------------------------------------------------- Winograd ---
  * The minimal-filtering form of a 3x3, stride-1, unit-dilation, ungrouped convolution

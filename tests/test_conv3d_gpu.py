@@ -70,6 +70,47 @@ def test_conv3d_edge_shapes(shape, layout, dtype):
     parity.assert_close(cfg, run_gpu3d(cfg, inp), run_oracle3d(cfg, inp), str(shape))
 
 
+VOL_REUSE = [  # N, C_in, D, H, W, C_out, Kd, Kh, Kw, stride, pad, dilation, groups; bias
+    ((2, 64, 7, 16, 16, 64, 3, 3, 3, 1, 1, 1, 1), True),    # Do = 7: the last unit has 3 of 4 slices
+    ((2, 64, 7, 16, 16, 64, 3, 3, 3, 1, 1, 1, 1), False),   # ... without bias
+    ((1, 64, 5, 12, 24, 32, 3, 3, 3, 1, 1, 1, 1), True),    # 288 voxels a slice: a 32-voxel tile; C_out 32
+    ((1, 64, 6, 16, 20, 96, 1, 3, 3, 1, 1, 1, 1), True),    # one depth tap, C_out 96 (2 slices per unit)
+    ((1, 64, 8, 18, 34, 64, 3, 3, 3, 1, 0, 1, 1), True),    # no padding, 512 voxels a slice
+    ((1, 64, 6, 16, 16, 128, 3, 1, 1, 1, 0, 1, 1), True),   # C_out 128, a (3, 1, 1) filter
+    ((1, 64, 4, 16, 16, 128, 3, 3, 3, 1, 1, 1, 1), True),   # C_out 128: products one depth tap wide
+    ((2, 64, 3, 18, 18, 64, 3, 3, 3, 1, 0, 1, 1), True),    # one output slice per image (J = 1)
+]
+
+
+@pytest.mark.parametrize("shape,bias", VOL_REUSE, ids=lambda s: "x".join(map(str, s)) if isinstance(s, tuple) else str(s))
+def test_conv3d_input_slice_reuse(shape, bias):
+    """bf16 NDHWC, stride 1, 64 input channels: the kernel that loads each input depth
+    slice once for every depth tap that reads it, over the whole output."""
+    plan = cb.conv3d_describe_plan(*shape, cb.CONV_BF16, "nhwc")
+    assert plan["kernel"] == "vol_reuse", plan
+    cfg = workloads.Conv3dConfig("reuse3d", *shape, bias, "bf16", "nhwc", seed=sum(shape))
+    inp = workloads.make_inputs3d(cfg)
+    parity.assert_close(cfg, run_gpu3d(cfg, inp), run_oracle3d(cfg, inp), str(shape))
+
+
+def test_conv3d_input_slice_reuse_integers_bit_exact():
+    ints = ("integers", -1, 1)
+    cfg = workloads.Conv3dConfig("ints3d", 1, 64, 6, 16, 16, 64, 3, 3, 3, 1, 1, 1, 1, True, "bf16", "nhwc",
+                                 ints, ints, ints, seed=5)
+    assert cb.conv3d_describe_plan(1, 64, 6, 16, 16, 64, 3, 3, 3, 1, 1, 1, 1, cb.CONV_BF16, "nhwc")["kernel"] == "vol_reuse"
+    inp = workloads.make_inputs3d(cfg)
+    ref = run_oracle3d(cfg, inp)
+    assert np.abs(ref).max() <= 256
+    assert np.array_equal(run_gpu3d(cfg, inp), ref)
+
+
+def test_conv3d_video_layer_takes_input_slice_reuse():
+    cfg = workloads.CONFIGS3D["conv3d_video_bf16"]
+    plan = cb.conv3d_describe_plan(cfg.N, cfg.C_in, cfg.D, cfg.H, cfg.W, cfg.C_out, cfg.Kd, cfg.Kh, cfg.Kw,
+                                   cfg.stride, cfg.pad, cfg.dilation, cfg.groups, cb.CONV_BF16, cfg.layout)
+    assert plan["kernel"] == "vol_reuse", plan
+
+
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_conv3d_small_integers_bit_exact(dtype):
     ints = ("integers", -2, 2)
