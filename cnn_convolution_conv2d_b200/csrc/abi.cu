@@ -204,9 +204,12 @@ int group_merge(int C_out, int C_in, int groups, int elt) {
     if (groups <= 1 || elt != 2) return 1;
     const int cin_g = C_in / groups, cout_g = C_out / groups;
     if (cout_g >= 64 || (cin_g * elt) % 16 != 0) return 1;
+    // At most one 128-byte channel row per pixel and tap: a second plane would double the
+    // rows the TMA engines load per output (their row rate bounds these layers) and the
+    // block-diagonal zeros the weight tiles carry.
     int best = 1;
     for (int gm = 2; gm <= groups; ++gm)
-        if (groups % gm == 0 && gm * cout_g <= 128 && gm * cin_g * elt <= 256) best = gm;
+        if (groups % gm == 0 && gm * cout_g <= 128 && gm * cin_g * elt <= 128) best = gm;
     return best;
 }
 
@@ -548,10 +551,13 @@ int make_plan(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stri
     // CTA pairs (bf16): each SM stages half of the weight tile and the pair's MMAs
     // read the other half from the peer, which halves the weight traffic and the
     // shared-memory bandwidth spent on it.  Used when the 256-row units still give
-    // every SM pair work; the test hook can force or forbid them.
+    // every SM pair work and the tile has at least 128 columns: narrower pair products
+    // (M = 256, N = 64) issue no faster than single-CTA ones and gain nothing (measured:
+    // the grouped layer 10.8 against 10.2 us, the 3-D video layer 218 against 213 us); the
+    // test hook can force or forbid them.
     const long long pair_units = ((p.M + 255) / 256) * p.n_ntiles * p.groups;
     const bool pair_ok = allow_pair && !p.f32 && p.BN % 32 == 0 && pair_mode != 2;
-    if (pair_ok && ((p.splits == 1 && sms > 0 && pair_units >= sms / 2) || pair_mode == 1)) {
+    if (pair_ok && ((p.splits == 1 && sms > 0 && pair_units >= sms / 2 && p.BN >= 128) || pair_mode == 1)) {
         p.pair = true;
         p.splits = 1;
         p.n_mtiles = static_cast<int>((p.M + 255) / 256);

@@ -59,8 +59,9 @@ def test_output_size_rejects(lib, args):
 
 def test_packed_weight_size(lib):
     # many channels or groups: only the (C_out, Kh, Kw, Cpg) weights
-    # 32 groups of 16 -> 16 channels: merged 8 at a time, block-diagonal rows of 8 * 16 channels
-    assert cb.conv2d_packed_weight_size(512, 512, 3, 3, 32, cb.CONV_BF16) == 512 * 9 * 16 * 8 * 2
+    # 32 groups of 16 -> 16 channels: merged 4 at a time (one 128-byte channel row),
+    # block-diagonal rows of 4 * 16 channels
+    assert cb.conv2d_packed_weight_size(512, 512, 3, 3, 32, cb.CONV_BF16) == 512 * 9 * 16 * 4 * 2
     assert cb.conv2d_packed_weight_size(512, 512, 3, 3, 32, cb.CONV_F32) == 512 * 9 * 16 * 4  # fp32: no merge
     assert cb.conv2d_packed_weight_size(24, 24, 3, 3, 4, cb.CONV_BF16) == 24 * 9 * 8 * 2  # 12-byte rows: no merge
     assert cb.conv2d_packed_weight_size(256, 256, 3, 3, 1, cb.CONV_BF16) == 256 * 9 * 256 * 2
@@ -180,8 +181,8 @@ def test_plan_for_the_workloads_on_a_148_sm_device(lib):
     k7 = _plan((16, 512, 17, 17, 512, 7, 7, 1, 3, 1, 1), sms=148)     # 19 pair units < 74: single CTAs, split
     assert (k7["pair"], k7["splits"], k7["units"]) == (0, 2, 37 * 2 * 2)
     assert k7["workspace"] == 2 * 16 * 17 * 17 * 512 * 4               # fp32 partial sums per split
-    g = _plan((16, 512, 28, 28, 512, 3, 3, 2, 2, 2, 32), sms=148)     # 16 channels per group, merged 8 at a time
-    assert (g["pair"], g["BN"], g["cb"], g["units"]) == (0, 128, 128, 25 * 4)
+    g = _plan((16, 512, 28, 28, 512, 3, 3, 2, 2, 2, 32), sms=148)     # 16 channels per group, merged 4 at a time
+    assert (g["pair"], g["BN"], g["cb"], g["units"]) == (0, 64, 128, 25 * 8)
     ex = _plan((64, 256, 56, 56, 256, 3, 3, 1, 1, 1, 1), explicit_im2col=True, sms=148)
     assert ex["a_load"] == "xcol" and ex["workspace"] >= 924_844_032   # the 924.8 MB X_col
     f32 = _plan((16, 512, 17, 17, 512, 7, 7, 1, 3, 1, 1), dtype=cb.CONV_F32, sms=148)
