@@ -1188,6 +1188,7 @@ struct WgPlan {
     Plan f;                       // the forward problem: validation, Ho, Wo, M
     bool tc;                      // tensor-core kernel
     int Cin_g, Cout_g, Cpg, dy_cpg, BN, n_ctiles, n_otiles, taps, kstages, splits, units, stages;
+    int om;                       // 128-row output-channel tiles per unit (n_otiles counts units' worth)
     bool xcopy, dycopy;
     size_t smem, off_xcopy, off_dycopy, off_ws, off_db, ws_total;
     int db_partials;
@@ -1218,6 +1219,10 @@ int wgrad_plan(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int str
         }
         w.n_ctiles = w.Cpg / w.BN;
         w.n_otiles = (w.Cout_g + 127) / 128;
+        // bf16 with an even number of 128-row tiles: two per unit (one staged block of x
+        // feeds both), when both accumulators fit in tensor memory
+        w.om = (!f.f32 && w.n_otiles % 2 == 0 && 2 * w.BN <= 512) ? 2 : 1;
+        w.n_otiles /= w.om;
         const int pk = wgrad_pixels_per_stage(f.f32);
         const long long kst = (f.M + pk - 1) / pk;
         const long long base = static_cast<long long>(w.n_otiles) * groups * w.taps * w.n_ctiles;
@@ -1231,12 +1236,12 @@ int wgrad_plan(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int str
             w.splits = sp > 1 ? static_cast<int>(sp) : 1;
         }
         w.units = static_cast<int>(base * w.splits);
-        const size_t fixed = wgrad_smem_bytes(f.f32, w.BN, 0);
-        const size_t stage = wgrad_smem_bytes(f.f32, w.BN, 1) - fixed;
+        const size_t fixed = wgrad_smem_bytes(f.f32, w.BN, 0, w.om);
+        const size_t stage = wgrad_smem_bytes(f.f32, w.BN, 1, w.om) - fixed;
         int stages = static_cast<int>((kSmemBudget - fixed) / stage);
         w.stages = stages > wgrad_max_stages() ? wgrad_max_stages() : stages;
         if (w.stages < 2) return fail(CONV_ERR_UNSUPPORTED, "weight-gradient tile does not fit in shared memory");
-        w.smem = wgrad_smem_bytes(f.f32, w.BN, w.stages);
+        w.smem = wgrad_smem_bytes(f.f32, w.BN, w.stages, w.om);
     } else {
         // CUDA cores: channels-last copies without padding, splits over rows of pixels
         w.Cpg = w.Cin_g;
@@ -1370,12 +1375,13 @@ int backward_weight_impl(const void *x, const void *dy, void *dw, void *db, int 
         k.BN = w.BN;
         k.n_ctiles = w.n_ctiles;
         k.n_otiles = w.n_otiles;
+        k.om = w.om;
         k.kstages = w.kstages;
         k.splits = w.splits;
         k.units = w.units;
         k.stages = w.stages;
         k.chunk_stages = f.f32 ? 4 : 0;
-        k.tmem_cols = 2 * w.BN <= 256 ? (2 * w.BN <= 128 ? 128 : 256) : 512;
+        k.tmem_cols = 2 * w.BN <= 256 ? (2 * w.BN <= 128 ? 128 : 256) : 512;  // two sets, or two tiles
         k.status = dev->status;
         k.timeout_ns = cfg.timeout_ns;
         k.starve = cfg.starve;

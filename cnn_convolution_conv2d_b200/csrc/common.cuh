@@ -153,6 +153,7 @@ struct WgradParams {
     int Cout, Cout_g, groups;
     int BN;                // channels per tile (multiple of 128 bytes; <= 256 bf16, <= 128 fp32)
     int n_ctiles, n_otiles, kstages, splits, units, stages, chunk_stages;
+    int om;                // 128-row output-channel tiles per unit (1, or 2 in bf16); n_otiles counts units' worth
     uint32_t tmem_cols;
     int *status;
     long long timeout_ns;
@@ -196,7 +197,7 @@ int dw_max_stages();
 size_t dw_header_bytes();
 
 cudaError_t launch_wgrad(const WgradParams &p, bool f32, int grid, size_t smem, cudaStream_t stream);
-size_t wgrad_smem_bytes(bool f32, int BN, int stages);
+size_t wgrad_smem_bytes(bool f32, int BN, int stages, int om);
 int wgrad_pixels_per_stage(bool f32);
 int wgrad_max_stages();
 // Weight gradient on the CUDA cores for few channels per group: partial sums

@@ -81,6 +81,9 @@ BWD = [  # N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups
     (1, 16, 12, 12, 16, 3, 3, 1, 3, 1, 1),     # pad 3 > K-1: the transposed convolution starts inside dy
     (2, 24, 15, 13, 16, 5, 5, 3, 2, 1, 1),     # stride 3, rows the windows never reach (zero gradient)
     (1, 256, 6, 6, 320, 3, 3, 1, 1, 1, 1),     # two 256-channel tiles of C_in, three 128-row tiles of C_out
+    (2, 64, 10, 10, 256, 3, 3, 1, 1, 1, 1),    # bf16: both 128-row tiles of C_out in one unit
+    (1, 64, 9, 9, 200, 3, 3, 1, 1, 1, 1),      # ... the second of them partial (200 channels)
+    (1, 128, 6, 6, 512, 3, 3, 1, 1, 1, 2),     # ... per group of 256 output channels
 ]
 
 
@@ -102,7 +105,7 @@ def test_backward_matches_oracle(shape, layout, dtype):
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("shape", [(1, 64, 6, 6, 64, 3, 3, 1, 1, 1, 1), (2, 32, 7, 7, 16, 3, 3, 2, 1, 1, 1),
-                                   (1, 16, 6, 6, 16, 3, 3, 1, 1, 1, 16)],
+                                   (1, 16, 6, 6, 16, 3, 3, 1, 1, 1, 16), (1, 64, 6, 6, 256, 3, 3, 1, 1, 1, 1)],
                          ids=lambda s: "x".join(map(str, s)))
 def test_backward_small_integers_bit_exact(shape, dtype):
     """Integer inputs in [-1, 1] and a short pixel reduction: every sum is an integer of
