@@ -21,7 +21,7 @@ CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIBRARY = os.path.join(PKG, "libconv2d_b200.so")
 SOURCES = ["abi.cu", "igemm.cu", "gather.cu", "gather_t.cu", "layout.cu", "depthwise.cu", "wgrad.cu",
-           "winograd.cu", "vol.cu"]
+           "winograd.cu", "vol.cu", "pw.cu"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -138,6 +138,7 @@ struct Plan {
     int pad_w;      // column padding (= pad, the row padding, for every caller-facing entry)
     bool vol;       // 3-D convolution: input depth D, filter depth Kd, output depth Do
     bool vreuse;    // ... on the input-slice-reuse kernel (vol.cu)
+    bool pw;        // 1x1 on the kernel with resident weights (pw.cu)
     int vJ, vn_k, vn_odb;  // its output slices per unit, tiles per slice, slice blocks
     int D, Kd, Do;
     bool f32;
@@ -606,6 +607,19 @@ int make_plan(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stri
     p.stages = stages > 8 ? 8 : stages;
     if (p.stages < 2) return fail(CONV_ERR_UNSUPPORTED, "tile does not fit in shared memory");
     p.smem = igemm_smem_bytes(p.f32, bn_local, p.stages, p.tma_out);
+    // A pointwise layer with a short reduction on CTA pairs: the kernel that keeps each
+    // cluster's 256-column weight tile resident and streams only the input rows (pw.cu).
+    p.pw = false;
+    if (p.pair && p.direct_a && p.tma_out && !p.f32 && groups == 1 && layout == CONV_NHWC && C_in % 64 == 0 &&
+        C_in == p.Cpg && C_in / 64 <= pw_max_planes() && C_out % 256 == 0 && p.BN == 256) {
+        int pst = pw_max_stages();
+        while (pst > 3 && pw_smem_bytes(C_in / 64, 256, pst) > kSmemBudget) --pst;
+        if (pw_smem_bytes(C_in / 64, 256, pst) <= kSmemBudget) {
+            p.pw = true;
+            p.stages = pst;
+            p.smem = pw_smem_bytes(C_in / 64, 256, pst);
+        }
+    }
 
     size_t off = 0;
     p.off_xcopy = off;
@@ -888,6 +902,27 @@ int pair_cluster_limit(int cb, bool im2col, size_t smem, bool vol = false) {
     return n;
 }
 
+// Resident two-CTA clusters of the pointwise kernel (pw.cu) at this shared-memory size,
+// asked of the runtime once per device and size and remembered.
+int pw_cluster_limit(size_t smem) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    const long long key = -((static_cast<long long>(dev) + 1) * 1048576 + static_cast<long long>(smem));
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        auto it = g_pair_clusters.find(key);
+        if (it != g_pair_clusters.end()) return it->second;
+    }
+    int n = 0;
+    if (pw_max_clusters(smem, &n) != cudaSuccess) {
+        (void)cudaGetLastError();
+        n = 0;
+    }
+    std::lock_guard<std::mutex> lock(g_mutex);
+    g_pair_clusters[key] = n;
+    return n;
+}
+
 // The plan a forward call on the current device makes, including the fall-back
 // from CTA pairs to single CTAs when the device cannot co-schedule the pair kernel.
 // Size queries and the forward pass share it, so that they always agree.
@@ -900,6 +935,14 @@ int device_plan(bool explicit_im2col, int N, int C_in, int H, int W, int C_out, 
     if (st != CONV_OK) return st;
     p->pair_clusters = 0;
     if (p->vreuse) return CONV_OK;
+    if (p->pw && dev) {
+        // clusters split evenly over the column tiles
+        const int n = pw_cluster_limit(p->smem);
+        p->pair_clusters = (n / p->n_ntiles) * p->n_ntiles;
+        if (p->pair_clusters >= p->n_ntiles) return CONV_OK;
+        return make_plan(N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype, layout,
+                         explicit_im2col, dev->sms, p, cfg.pair_mode, false, padw, vol);
+    }
     if (p->pair && dev) {
         const bool a_im2col = !(explicit_im2col || p->direct_a);
         p->pair_clusters = pair_cluster_limit(p->cb, a_im2col, p->smem, p->vol && a_im2col);
@@ -971,6 +1014,46 @@ int vol_impl(const Plan &p, const void *x, const void *w_packed, const void *bia
     return ok();
 }
 
+// The pointwise path with resident weights (pw.cu): one kernel, no scratch.
+int pw_impl(const Plan &p, const void *x, const void *w_packed, const void *bias, void *y, DeviceInfo *dev,
+            const Settings &cfg, cudaStream_t stream) {
+    PwParams k;
+    std::memset(&k, 0, sizeof(k));
+    int st = encode_a_xcol(p, x, &k.tmap_a);
+    if (st != CONV_OK) return st;
+    st = encode_b(p, w_packed, &k.tmap_b);
+    if (st != CONV_OK) return st;
+    {
+        cuuint64_t dims[2] = {static_cast<cuuint64_t>(p.C_out), static_cast<cuuint64_t>(p.M)};
+        cuuint64_t strides[1] = {static_cast<cuuint64_t>(p.C_out) * p.elt};
+        cuuint32_t box[2] = {32, 32};
+        cuuint32_t estr[2] = {1, 1};
+        CUresult r = g_encode_tiled(&k.tmap_y, tma_type(p), 2, y, dims, strides, box, estr,
+                                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                                    CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS)
+            return fail(CONV_ERR_CUDA, "cuTensorMapEncodeTiled (output) failed (%d)", static_cast<int>(r));
+    }
+    k.M = static_cast<int>(p.M);
+    k.nk = p.C_in / 64;
+    k.BN = p.BN;
+    k.n_ntiles = p.n_ntiles;
+    k.m_tiles = static_cast<int>((p.M + 255) / 256);
+    k.cpn = p.pair_clusters / p.n_ntiles;
+    k.stages = p.stages;
+    k.tmem_cols = 512;
+    k.bias = bias;
+    k.status = dev->status;
+    k.timeout_ns = cfg.timeout_ns;
+    k.starve = cfg.starve;
+    cudaEvent_t ev_start = g_main_start, ev_stop = g_main_stop;
+    if (ev_start && ev_stop && (st = record_event(ev_start, stream)) != CONV_OK) return st;
+    cudaError_t e = launch_pw(k, p.smem, stream);
+    if ((st = check_launch(e, "pointwise product with resident weights")) != CONV_OK) return st;
+    if (ev_start && ev_stop && (st = record_event(ev_stop, stream)) != CONV_OK) return st;
+    return ok();
+}
+
 // Shared body of conv2d_forward and conv2d_forward_im2col_gemm.
 int forward_impl(bool explicit_im2col, const void *x, const void *w_packed, const void *bias, void *y,
                  int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stride, int pad,
@@ -1001,6 +1084,7 @@ int forward_impl(bool explicit_im2col, const void *x, const void *w_packed, cons
     if (p.gather) return gather_impl(p, x, w_packed, bias, y, dev, cfg, stream);
     if (p.dw) return dw_impl(p, x, w_packed, bias, y, workspace, dev, cfg, stream);
     if (p.vreuse) return vol_impl(p, x, w_packed, bias, y, dev, cfg, stream);
+    if (p.pw) return pw_impl(p, x, w_packed, bias, y, dev, cfg, stream);
 
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     const void *x_nhwc = p.xcopy ? static_cast<const void *>(ws + p.off_xcopy) : x;
@@ -1126,7 +1210,7 @@ int describe_impl(bool explicit_im2col, int N, int C_in, int H, int W, int C_out
     }
     if (st != CONV_OK) return st;
     const char *a_load = p.dw ? "tile" : p.gather ? "gather" : explicit_im2col ? "xcol" : p.direct_a ? "tiled_x" : "im2col";
-    const char *kernel = p.dw ? "depthwise" : p.vreuse ? "vol_reuse" : p.gather_t ? "gather_t" : p.gather ? "gather" : "igemm";
+    const char *kernel = p.dw ? "depthwise" : p.vreuse ? "vol_reuse" : p.pw ? "pointwise" : p.gather_t ? "gather_t" : p.gather ? "gather" : "igemm";
     const int n = std::snprintf(
         buf, buflen,
         "{\"kernel\": \"%s\", \"pair\": %d, \"a_load\": \"%s\", \"BN\": %d, \"cb\": %d, "

@@ -81,6 +81,21 @@ struct VolParams {
     int starve;
 };
 
+// One launch of the pointwise kernel (pw.cu): 1x1, stride 1, no padding, bf16, groups 1,
+// channels-last, C_in = 64*nk (nk <= 4), C_out a multiple of BN = 256, CTA pairs.  Cluster c
+// keeps column tile c % n_ntiles resident and takes row tiles c / n_ntiles + i*cpn.
+struct PwParams {
+    CUtensorMap tmap_a;  // x as X_col {C_in, M}, boxes of {64, 128}, 128-byte swizzle
+    CUtensorMap tmap_b;  // packed weights {C_in, C_out, 1}, boxes of {64, BN/2}, 128-byte swizzle
+    CUtensorMap tmap_y;  // y as {C_out, M}, 32 x 32 boxes with 64-byte swizzle
+    int M, nk, BN, n_ntiles, m_tiles, cpn, stages;
+    uint32_t tmem_cols;
+    const void *bias;
+    int *status;
+    long long timeout_ns;
+    int starve;
+};
+
 // One launch of the software-gather kernel (gather.cu) for inputs with few
 // channels: groups = 1, reduction index k = (kh*Kw + kw)*C + c (or the row-vector
 // order), padded to Kpad.
@@ -176,6 +191,11 @@ size_t gather_smem_bytes(bool f32, int BN, int Kpad, size_t halo_bytes, size_t o
 // per tile, output channels on the tensor-memory lanes.
 cudaError_t launch_gather_t(const GatherParams &p, int grid, size_t smem, cudaStream_t stream);
 cudaError_t launch_vol_reuse(const VolParams &p, int grid, size_t smem, cudaStream_t stream);
+cudaError_t launch_pw(const PwParams &p, size_t smem, cudaStream_t stream);
+cudaError_t pw_max_clusters(size_t smem, int *clusters);
+size_t pw_smem_bytes(int nk, int BN, int stages);
+int pw_max_stages();
+int pw_max_planes();
 size_t vol_reuse_smem_bytes(int Kd, int BN, int stages);
 int vol_reuse_max_stages();
 int vol_reuse_max_j();

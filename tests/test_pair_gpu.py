@@ -133,3 +133,40 @@ def test_pair_explicit_im2col_gemm(name, pairs_forced):
     inp = workloads.make_inputs(cfg)
     got = parity.run_gpu(cfg, inp, explicit_im2col=True)
     parity.assert_close(cfg, got, parity.run_oracle(cfg, inp), name + " (pair, explicit im2col)")
+
+
+PW_SHAPES = [  # 1x1, stride 1, no padding: the kernel with each cluster's weight tile resident
+    ((2, 64, 9, 9, 256, 1, 1, 1, 0, 1, 1), True),     # M = 162: one row tile, the odd CTA's rows partly past M
+    ((3, 128, 10, 11, 512, 1, 1, 1, 0, 1, 1), True),  # two column tiles, M = 330: a ragged second row tile
+    ((1, 256, 12, 12, 768, 1, 1, 1, 0, 1, 1), False), # reduction 256 (four planes), three column tiles, no bias
+    ((2, 192, 8, 8, 256, 1, 1, 1, 0, 1, 1), True),    # three planes
+]
+
+
+@pytest.mark.parametrize("shape,bias", PW_SHAPES, ids=lambda s: "x".join(map(str, s)) if isinstance(s, tuple) else str(s))
+def test_pointwise_resident_weights(shape, bias, pairs_forced):
+    N, C_in, H, W, C_out, Kh, Kw, s, p, d, g = shape
+    plan = cb.conv2d_describe_plan(*shape, cb.CONV_BF16, "nhwc")
+    assert plan["kernel"] == "pointwise", plan
+    cfg = workloads.ConvConfig("pw", N, C_in, H, W, C_out, Kh, Kw, s, p, d, g, bias, "bf16", "nhwc",
+                               seed=sum(shape) + 21)
+    inp = workloads.make_inputs(cfg)
+    parity.assert_close(cfg, parity.run_gpu(cfg, inp), parity.run_oracle(cfg, inp), str(shape) + " (pointwise)")
+
+
+def test_pointwise_resident_weights_integers_bit_exact(pairs_forced):
+    shape = (3, 128, 9, 7, 512, 1, 1, 1, 0, 1, 1)
+    assert cb.conv2d_describe_plan(*shape, cb.CONV_BF16, "nhwc")["kernel"] == "pointwise"
+    ints = ("integers", -2, 2)
+    cfg = workloads.ConvConfig("pw_ints", *shape, True, "bf16", "nhwc", ints, ints, ints, seed=9)
+    inp = workloads.make_inputs(cfg)
+    ref = parity.run_oracle(cfg, inp)
+    assert np.abs(ref).max() <= 256
+    assert np.array_equal(parity.run_gpu(cfg, inp), ref)
+
+
+def test_pointwise_workload_takes_resident_weights():
+    cfg = workloads.CONFIGS["pointwise1x1_bf16"]
+    plan = cb.conv2d_describe_plan(cfg.N, cfg.C_in, cfg.H, cfg.W, cfg.C_out, cfg.Kh, cfg.Kw, cfg.stride, cfg.pad,
+                                   cfg.dilation, cfg.groups, cb.CONV_BF16, cfg.layout)
+    assert plan["kernel"] == "pointwise", plan
