@@ -151,7 +151,9 @@ __device__ __forceinline__ void stv(void *p, long long i, const float *f) {
 
 // 1. V[tile][xi][c] = (B^T d B)[xi] for each tile (n, th, tw) and channel c < Cpg (zero
 // for c >= C): d[a][b] = x[n][th*m - pad + a][tw*m - pad + b][c], zero outside the image.
-// One thread per (tile, group of kV consecutive channels).
+// One thread per (tile, group of kV consecutive channels).  All alpha^2 loads of a tile are
+// issued before any arithmetic (they are independent, and so in flight together), then
+// B^T is applied to the columns in place and B to the rows on the way out.
 template <bool kF32, bool kVF32, int kM, int kV>
 __global__ void __launch_bounds__(kWgThreads256) wino_input_kernel(const void *__restrict__ x, void *__restrict__ v,
                                                                  int N, int C, int H, int W, int Cpg, int TH, int TW,
@@ -171,48 +173,55 @@ __global__ void __launch_bounds__(kWgThreads256) wino_input_kernel(const void *_
         const int n = static_cast<int>(r / TH);
         const int c0 = cg * kV;
         const int h0 = th * kM - pad, w0 = tw * kM - pad;
-        // t = B^T d, one input column at a time
-        float t[kA][kA][kV];
+        float d[kA][kA][kV];
 #pragma unroll
-        for (int b = 0; b < kA; ++b) {
-            float d[kA][kV];
-            const int iw = w0 + b;
+        for (int k = 0; k < kA; ++k) {
+            const int ih = h0 + k;
 #pragma unroll
-            for (int k = 0; k < kA; ++k) {
-                const int ih = h0 + k;
+            for (int b = 0; b < kA; ++b) {
+                const int iw = w0 + b;
                 const bool in = ih >= 0 && ih < H && iw >= 0 && iw < W;
                 if (vec) {  // channels-last, C a multiple of kV: one vector access
                     if (in && c0 < C) {
-                        ldv<kF32, kV>(x, ((static_cast<long long>(n) * H + ih) * W + iw) * C + c0, d[k]);
+                        ldv<kF32, kV>(x, ((static_cast<long long>(n) * H + ih) * W + iw) * C + c0, d[k][b]);
                     } else {
 #pragma unroll
-                        for (int e = 0; e < kV; ++e) d[k][e] = 0.f;
+                        for (int e = 0; e < kV; ++e) d[k][b][e] = 0.f;
                     }
-                    continue;
-                }
+                } else {
 #pragma unroll
-                for (int e = 0; e < kV; ++e) {
-                    const int c = c0 + e;
-                    float val = 0.f;
-                    if (in && c < C) {
-                        const long long at = nchw ? ((static_cast<long long>(n) * C + c) * H + ih) * W + iw
-                                                  : ((static_cast<long long>(n) * H + ih) * W + iw) * C + c;
-                        val = ld1<kF32>(x, at);
+                    for (int e = 0; e < kV; ++e) {
+                        const int c = c0 + e;
+                        float val = 0.f;
+                        if (in && c < C) {
+                            const long long at = nchw ? ((static_cast<long long>(n) * C + c) * H + ih) * W + iw
+                                                      : ((static_cast<long long>(n) * H + ih) * W + iw) * C + c;
+                            val = ld1<kF32>(x, at);
+                        }
+                        d[k][b][e] = val;
                     }
-                    d[k][e] = val;
                 }
             }
+        }
+        // columns: d[.][b] <- B^T d[.][b]
+#pragma unroll
+        for (int b = 0; b < kA; ++b) {
+            float t[kA][kV];
 #pragma unroll
             for (int a = 0; a < kA; ++a)
 #pragma unroll
                 for (int e = 0; e < kV; ++e) {
                     float sum = 0.f;
 #pragma unroll
-                    for (int k = 0; k < kA; ++k) sum += Mt::bt(a, k) * d[k][e];
-                    t[a][b][e] = sum;
+                    for (int k = 0; k < kA; ++k) sum += Mt::bt(a, k) * d[k][b][e];
+                    t[a][e] = sum;
                 }
+#pragma unroll
+            for (int a = 0; a < kA; ++a)
+#pragma unroll
+                for (int e = 0; e < kV; ++e) d[a][b][e] = t[a][e];
         }
-        // V = t B
+        // rows: V[a][b] = sum_k (B^T d)[a][k] B[k][b]
         const long long base = tile * kA * kA * Cpg + c0;
 #pragma unroll
         for (int a = 0; a < kA; ++a)
@@ -221,10 +230,10 @@ __global__ void __launch_bounds__(kWgThreads256) wino_input_kernel(const void *_
                 float o[kV];
 #pragma unroll
                 for (int e = 0; e < kV; ++e) {
-                    float s = 0.f;
+                    float sum = 0.f;
 #pragma unroll
-                    for (int k = 0; k < kA; ++k) s += t[a][k][e] * Mt::bt(b, k);
-                    o[e] = s;
+                    for (int k = 0; k < kA; ++k) sum += d[a][k][e] * Mt::bt(b, k);
+                    o[e] = sum;
                 }
                 stv<kVF32, kV>(v, base + static_cast<long long>(a * kA + b) * Cpg, o);  // Cpg % kV == 0
             }
@@ -262,7 +271,8 @@ __global__ void __launch_bounds__(kWgThreads256) wino_weight_kernel(const void *
 }
 
 // 3. y[n][th*m + i][tw*m + j][oc] = bias[oc] + (A^T M A)[i][j], M[xi] summed over the
-// product's splits (fp32 partial sums [split][tile][alpha^2 * C_out]).
+// product's splits (fp32 partial sums [split][tile][alpha^2 * C_out]).  As in the input
+// transform, all alpha^2 loads of a tile (per split) are issued before any arithmetic.
 template <bool kF32, int kM, int kV>
 __global__ void __launch_bounds__(kWgThreads256) wino_output_kernel(const float *__restrict__ mp,
                                                                   const void *__restrict__ bias, void *__restrict__ y,
@@ -284,39 +294,44 @@ __global__ void __launch_bounds__(kWgThreads256) wino_output_kernel(const float 
         const int th = static_cast<int>(r % TH);
         const int n = static_cast<int>(r / TH);
         const int c0 = cg * kV;
-        // t = A^T M, one column of M (summed over the splits) at a time
-        float t[kM][kA][kV];
+        // the first split straight into m, all loads in flight together; later splits
+        // (rare) added one vector at a time
+        float m[kA][kA][kV];
+        for (int sp = 0; sp < splits; ++sp) {
+            const float *src = mp + (sp * tiles + tile) * row + c0;
+#pragma unroll
+            for (int k = 0; k < kA; ++k)
+#pragma unroll
+                for (int b = 0; b < kA; ++b) {
+                    const long long at = static_cast<long long>(k * kA + b) * C_out;
+                    float f[kV];
+                    if (vec) {
+                        ldv<true, kV>(src, at, f);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < kV; ++e) f[e] = c0 + e < C_out ? src[at + e] : 0.f;
+                    }
+#pragma unroll
+                    for (int e = 0; e < kV; ++e) m[k][b][e] = sp == 0 ? f[e] : m[k][b][e] + f[e];
+                }
+        }
+        // columns: m[a][b] <- (A^T M)[a][b] for a < m
 #pragma unroll
         for (int b = 0; b < kA; ++b) {
-            float m[kA][kV];
-#pragma unroll
-            for (int k = 0; k < kA; ++k) {
-#pragma unroll
-                for (int e = 0; e < kV; ++e) m[k][e] = 0.f;
-                if (vec) {
-                    for (int sp = 0; sp < splits; ++sp) {
-                        float f[kV];
-                        ldv<true, kV>(mp, (sp * tiles + tile) * row + static_cast<long long>(k * kA + b) * C_out + c0, f);
-#pragma unroll
-                        for (int e = 0; e < kV; ++e) m[k][e] += f[e];
-                    }
-                } else {
-#pragma unroll
-                    for (int e = 0; e < kV; ++e)
-                        if (c0 + e < C_out)
-                            for (int sp = 0; sp < splits; ++sp)
-                                m[k][e] += mp[(sp * tiles + tile) * row + static_cast<long long>(k * kA + b) * C_out + c0 + e];
-                }
-            }
+            float t[kM][kV];
 #pragma unroll
             for (int a = 0; a < kM; ++a)
 #pragma unroll
                 for (int e = 0; e < kV; ++e) {
                     float sum = 0.f;
 #pragma unroll
-                    for (int k = 0; k < kA; ++k) sum += Mt::at(a, k) * m[k][e];
-                    t[a][b][e] = sum;
+                    for (int k = 0; k < kA; ++k) sum += Mt::at(a, k) * m[k][b][e];
+                    t[a][e] = sum;
                 }
+#pragma unroll
+            for (int a = 0; a < kM; ++a)
+#pragma unroll
+                for (int e = 0; e < kV; ++e) m[a][b][e] = t[a][e];
         }
         float bv[kV];
 #pragma unroll
@@ -334,7 +349,7 @@ __global__ void __launch_bounds__(kWgThreads256) wino_output_kernel(const float 
                 for (int e = 0; e < kV; ++e) {
                     float s = bv[e];
 #pragma unroll
-                    for (int k = 0; k < kA; ++k) s += t[a][k][e] * Mt::at(b, k);
+                    for (int k = 0; k < kA; ++k) s += m[a][k][e] * Mt::at(b, k);
                     o[e] = s;
                 }
                 if (vec && !nchw) {
