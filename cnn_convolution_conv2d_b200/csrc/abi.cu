@@ -470,7 +470,7 @@ int make_plan(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stri
                     if (C_in * R > gather_t_max_chunks() || BW > 256 || W > BW || R > 256) continue;
                     const int kt = rt == 1 ? p.Kpad : round_up(C_in * R * per16, 32 / p.elt);
                     const size_t hb = static_cast<size_t>(C_in) * R * BW * p.elt;
-                    const size_t ob = static_cast<size_t>(bn) * rt * p.Wo * p.elt;
+                    const size_t ob = static_cast<size_t>((p.Wo + 63) / 64) * bn * rt * 128;  // 64-pixel parts
                     // A in tensor memory when at least two accumulators fit beside it (its
                     // kt/2 columns), else in shared memory
                     const int acc_tm = (512 - kt / 2) / tpix;
@@ -787,15 +787,15 @@ int gather_impl(const Plan &p, const void *x, const void *w_packed, const void *
     g.cw = p.cw;
     g.tma_out = p.tma_out ? 1 : 0;
     if (p.tma_out && p.gather_t) {
-        // y as (Wo, Ho, C_out, N); one box per tile: the tile's output rows of every channel
+        // y as (Wo, C_out, Ho, N); boxes of 64 pixels x every channel x the tile's output
+        // rows, 128-byte swizzled (rows of the box: row-of-tile-major, then channel)
         const cuuint64_t wo = static_cast<cuuint64_t>(p.Wo), ho = static_cast<cuuint64_t>(p.Ho);
-        cuuint64_t dims[4] = {wo, ho, static_cast<cuuint64_t>(p.C_out), static_cast<cuuint64_t>(p.N)};
-        cuuint64_t strides[3] = {wo * p.elt, wo * ho * p.elt, wo * ho * p.elt * p.C_out};
-        cuuint32_t box[4] = {static_cast<cuuint32_t>(p.Wo), static_cast<cuuint32_t>(p.rt),
-                             static_cast<cuuint32_t>(p.BN), 1};
+        cuuint64_t dims[4] = {wo, static_cast<cuuint64_t>(p.C_out), ho, static_cast<cuuint64_t>(p.N)};
+        cuuint64_t strides[3] = {wo * ho * p.elt, wo * p.elt, wo * ho * p.elt * p.C_out};
+        cuuint32_t box[4] = {64, static_cast<cuuint32_t>(p.BN), static_cast<cuuint32_t>(p.rt), 1};
         cuuint32_t estr[4] = {1, 1, 1, 1};
         CUresult r = g_encode_tiled(&g.tmap_y, tma_type(p), 4, y, dims, strides, box, estr,
-                                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                                     CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS)
             return fail(CONV_ERR_CUDA, "cuTensorMapEncodeTiled (output rows) failed (%d)", static_cast<int>(r));

@@ -42,7 +42,8 @@
 //                       tcgen05.mma from one thread;
 //   warps 9..16       : epilogue, two warps per lane quarter (each half of the columns):
 //                       tcgen05.ld, + bias, one rounding to bf16, 16-byte writes into
-//                       the output image, then one TMA store.
+//                       the output image (64-pixel parts, 128-byte swizzled), then one TMA
+//                       store per part.
 // Every wait is bounded (ptx.cuh).
 #include <cuda_bf16.h>
 
@@ -110,7 +111,11 @@ __global__ void __launch_bounds__(kGtThreads, 1) gather_t_kernel(const __grid_co
     const uint32_t halo_bytes = static_cast<uint32_t>(p.C) * p.R * p.BW * 2u;
     const uint32_t halo_stride = gt_align1k(halo_bytes);
     uint8_t *out_sm = halo_sm + p.nhalo * halo_stride;            // output images (tma_out)
-    const uint32_t out_stride = gt_align1k(static_cast<uint32_t>(p.BN) * rt * p.Wo * 2u);
+    // an output image: ceil(Wo / 64) parts of (rt x BN) 128-byte rows (64 pixels), each the
+    // 128-byte-swizzled box of one TMA store
+    const int oparts = (p.Wo + 63) / 64;
+    const uint32_t opart_bytes = static_cast<uint32_t>(rt * p.BN) * 128u;
+    const uint32_t out_stride = gt_align1k(static_cast<uint32_t>(oparts) * opart_bytes);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -376,9 +381,11 @@ __global__ void __launch_bounds__(kGtThreads, 1) gather_t_kernel(const __grid_co
             const int oh0 = (t - img * tiles_per_img) * rt;
             const bool valid = ch_ok && oh0 + r < p.Ho;
             if (__any_sync(0xffffffffu, valid) && c_lo < c_hi) {
-                // image layout [channel][row of the tile][Wo], the TMA box's order
-                uint8_t *orow = out_sm + ob * out_stride +
-                                (static_cast<uint32_t>(valid ? oc : 0) * rt + r) * p.Wo * 2u;
+                // image row (r*BN + oc) of each part; 16-byte chunk k of a row sits at chunk
+                // k ^ (row & 7) (the store's 128-byte swizzle): the eight rows a quarter-warp
+                // writes at once land in eight different bank groups
+                const uint32_t irow = static_cast<uint32_t>(r * p.BN + (valid ? oc : 0));
+                uint8_t *orow = out_sm + ob * out_stride + irow * 128u;
                 __nv_bfloat16 *yrow = static_cast<__nv_bfloat16 *>(p.y) +
                                       ((static_cast<size_t>(img) * p.Cout + (valid ? oc : 0)) * p.Ho +
                                        (valid ? oh0 + r : 0)) * p.Wo;
@@ -404,9 +411,12 @@ __global__ void __launch_bounds__(kGtThreads, 1) gather_t_kernel(const __grid_co
                                     pk[i] = *reinterpret_cast<uint32_t *>(&h);
                                 }
                                 const uint4 v4 = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                                if (staged)
-                                    *reinterpret_cast<uint4 *>(orow + (cb + 8 * q) * 2) = v4;
-                                else
+                                if (staged) {
+                                    const int col = cb + 8 * q;
+                                    const uint32_t k = static_cast<uint32_t>((col & 63) >> 3);
+                                    *reinterpret_cast<uint4 *>(orow + static_cast<uint32_t>(col >> 6) * opart_bytes +
+                                                               ((k ^ (irow & 7u)) << 4)) = v4;
+                                } else
                                     *reinterpret_cast<uint4 *>(yrow + cb + 8 * q) = v4;
                             }
                         }
@@ -421,7 +431,8 @@ __global__ void __launch_bounds__(kGtThreads, 1) gather_t_kernel(const __grid_co
                 fence_proxy_async_smem();
                 named_barrier(2, kGtEpi * 32);
                 if (issuer) {
-                    tma_store_4d(&p.tmap_y, out_sm + ob * out_stride, 0, oh0, 0, img);
+                    for (int part = 0; part < oparts; ++part)
+                        tma_store_4d(&p.tmap_y, out_sm + ob * out_stride + part * opart_bytes, part * 64, 0, oh0, img);
                     bulk_commit_group();
                 }
             }

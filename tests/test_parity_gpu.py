@@ -113,8 +113,9 @@ TRANSPOSED_FIRST_LAYER = [  # bf16 NCHW, few channels, Wo % 8 == 0: the transpos
     ((2, 3, 30, 64, 32, 7, 7, 2, 3, 1, 1), (2, 2, 0)),      # Ho = 15: the last pair's second row clipped
     ((2, 3, 40, 96, 96, 3, 3, 2, 1, 1, 1), (1, 2, 0)),      # C_out 96: one row per tile, A in shared memory
     ((2, 4, 64, 128, 128, 7, 7, 1, 3, 1, 1), (1, 2, 1)),    # C_out 128, reduction 224
-    ((1, 4, 17, 160, 128, 8, 7, 1, 3, 1, 1), (1, 1, 1)),    # reduction 256, 160 pixels: room for one image
-    ((1, 4, 17, 192, 128, 8, 7, 1, 3, 1, 1), (1, 0, 1)),    # 192 pixels: no room for an image
+    ((1, 4, 17, 160, 128, 7, 7, 1, 3, 1, 1), (1, 1, 1)),    # 160 pixels (three 64-pixel parts): room for one image
+    ((1, 3, 17, 160, 64, 7, 7, 1, 3, 1, 1), (2, 1, 1)),     # ... two rows per tile, one image
+    ((1, 4, 17, 192, 128, 8, 7, 1, 3, 1, 1), (1, 0, 1)),    # reduction 256, 192 pixels: no room for an image
 ]
 
 
