@@ -100,6 +100,51 @@ __device__ __forceinline__ void unpack16_pairs(const uint4 &u, uint64_t *p) {
     }
 }
 
+// Stores kV consecutive channels (c ..) of output pixel pix (= (n*Ho + oh)*Wo + ow), rounded
+// once to the output type; vector stores for whole groups in channels-last output.
+template <bool kF32, int kV>
+__device__ __forceinline__ void dw_store(const DwParams &p, size_t pix, size_t n, int oh, int ow, int c,
+                                         const float *o, bool whole) {
+    if (!p.out_nchw) {
+        if constexpr (kF32) {
+            float *dst = static_cast<float *>(p.y) + pix * p.C + c;
+            if (whole) {
+                *reinterpret_cast<float4 *>(dst) = make_float4(o[0], o[1], o[2], o[3]);
+            } else {
+#pragma unroll
+                for (int v = 0; v < kV; ++v)
+                    if (c + v < p.C) dst[v] = o[v];
+            }
+        } else {
+            __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.y) + pix * p.C + c;
+            if (whole) {
+                uint32_t pk[kV / 2];
+#pragma unroll
+                for (int i = 0; i < kV / 2; ++i) {
+                    __nv_bfloat162 h = __floats2bfloat162_rn(o[2 * i], o[2 * i + 1]);
+                    pk[i] = *reinterpret_cast<uint32_t *>(&h);
+                }
+                *reinterpret_cast<uint4 *>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            } else {
+#pragma unroll
+                for (int v = 0; v < kV; ++v)
+                    if (c + v < p.C) dst[v] = __float2bfloat16_rn(o[v]);
+            }
+        }
+    } else {  // NCHW: y[n][c][oh][ow]
+        const size_t plane = static_cast<size_t>(p.Ho) * p.Wo;
+        const size_t at = (n * p.C + c) * plane + static_cast<size_t>(oh) * p.Wo + ow;
+#pragma unroll
+        for (int v = 0; v < kV; ++v) {
+            if (c + v >= p.C) break;
+            if constexpr (kF32)
+                static_cast<float *>(p.y)[at + v * plane] = o[v];
+            else
+                static_cast<__nv_bfloat16 *>(p.y)[at + v * plane] = __float2bfloat16_rn(o[v]);
+        }
+    }
+}
+
 struct DwTile {
     int chunk, n, th, tw;
 };
@@ -240,31 +285,129 @@ __global__ void __launch_bounds__(kDwThreads, 1) dw_kernel(const __grid_constant
             const bool ok = mbar_wait(&sb.full[stage], phase, wd, kDevTimeoutFull);
             if (!__all_sync(0xffffffffu, ok)) break;
             const uint8_t *stg = ring + static_cast<size_t>(stage) * sbytes;
-            for (int it = tid; it < items; it += 32 * kDwComputeWarps) {
-                const int cg = it & 7, pg = it >> 3;
-                const int py = pg / groups_per_row;
-                const int px0 = (pg - py * groups_per_row) * kR;
-                const int oh = t.th * p.TH + py;
-                const int ow0 = t.tw * p.TW + px0;
-                if (oh >= p.Ho || ow0 >= p.Wo) continue;
-                float acc[kR][kV];
-                if constexpr (kKW > 0) {
-                    // stride 1, unit dilation, kKW x kKW: every filter row reads a window of
-                    // kR + kKW - 1 input pixels once; products in fp32 pairs
-                    constexpr int kP = kV / 2;
+            if constexpr (kKW == 0) {
+                // general form: 16 bytes of channels of kR pixels of one output row per item
+                for (int it = tid; it < items; it += 32 * kDwComputeWarps) {
+                    const int cg = it & 7, pg = it >> 3;
+                    const int py = pg / groups_per_row;
+                    const int px0 = (pg - py * groups_per_row) * kR;
+                    const int oh = t.th * p.TH + py;
+                    const int ow0 = t.tw * p.TW + px0;
+                    if (oh >= p.Ho || ow0 >= p.Wo) continue;
+                    float acc[kR][kV];
+                    {
+    #pragma unroll
+                        for (int r = 0; r < kR; ++r)
+    #pragma unroll
+                            for (int v = 0; v < kV; ++v) acc[r][v] = 0.f;
+                        for (int kh = 0; kh < p.Kh; ++kh) {
+                            const int row = py * p.stride + kh * p.dilation;
+                            const uint8_t *rp = stg + static_cast<size_t>(row) * p.IW * kDwRowBytes + cg * 16;
+                            const uint8_t *wp = wsm + kh * p.Kw * kDwRowBytes + cg * 16;
+                            for (int kw = 0; kw < p.Kw; ++kw) {
+                                float wv[kV];
+                                unpack16<kF32>(*reinterpret_cast<const uint4 *>(wp + kw * kDwRowBytes), wv);
+    #pragma unroll
+                                for (int r = 0; r < kR; ++r) {
+                                    const int col = (px0 + r) * p.stride + kw * p.dilation;
+                                    float xv[kV];
+                                    unpack16<kF32>(*reinterpret_cast<const uint4 *>(rp + col * kDwRowBytes), xv);
+    #pragma unroll
+                                    for (int v = 0; v < kV; ++v) acc[r][v] = fmaf(xv[v], wv[v], acc[r][v]);
+                                }
+                            }
+                        }
+                    }
+                    // epilogue: + bias, one rounding, store
+                    const int c = t.chunk * kCC + cg * kV;
+                    if (c >= p.C) continue;
+                    float bv[kV];
+    #pragma unroll
+                    for (int v = 0; v < kV; ++v) bv[v] = bsm[cg * kV + v];
+                    const bool whole = c + kV <= p.C && p.vec_ok;
+    #pragma unroll
+                    for (int r = 0; r < kR; ++r) {
+                        const int ow = ow0 + r;
+                        if (ow >= p.Wo) break;
+                        float o[kV];
+    #pragma unroll
+                        for (int v = 0; v < kV; ++v) o[v] = acc[r][v] + bv[v];
+                        const size_t pix = (static_cast<size_t>(t.n) * p.Ho + oh) * p.Wo + ow;
+                        if (!p.out_nchw) {
+                            if constexpr (kF32) {
+                                float *dst = static_cast<float *>(p.y) + pix * p.C + c;
+                                if (whole) {
+                                    *reinterpret_cast<float4 *>(dst) = make_float4(o[0], o[1], o[2], o[3]);
+                                } else {
+    #pragma unroll
+                                    for (int v = 0; v < kV; ++v)
+                                        if (c + v < p.C) dst[v] = o[v];
+                                }
+                            } else {
+                                __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.y) + pix * p.C + c;
+                                if (whole) {
+                                    uint32_t pk[4];
+    #pragma unroll
+                                    for (int i = 0; i < 4; ++i) {
+                                        __nv_bfloat162 h = __floats2bfloat162_rn(o[2 * i], o[2 * i + 1]);
+                                        pk[i] = *reinterpret_cast<uint32_t *>(&h);
+                                    }
+                                    *reinterpret_cast<uint4 *>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                                } else {
+    #pragma unroll
+                                    for (int v = 0; v < kV; ++v)
+                                        if (c + v < p.C) dst[v] = __float2bfloat16_rn(o[v]);
+                                }
+                            }
+                        } else {  // NCHW: y[n][c][oh][ow]
+                            const size_t plane = static_cast<size_t>(p.Ho) * p.Wo;
+                            const size_t at = (static_cast<size_t>(t.n) * p.C + c) * plane +
+                                              static_cast<size_t>(oh) * p.Wo + ow;
+    #pragma unroll
+                            for (int v = 0; v < kV; ++v) {
+                                if (c + v >= p.C) break;
+                                if constexpr (kF32)
+                                    static_cast<float *>(p.y)[at + v * plane] = o[v];
+                                else
+                                    static_cast<__nv_bfloat16 *>(p.y)[at + v * plane] = __float2bfloat16_rn(o[v]);
+                            }
+                        }
+                    }
+                }
+            }
+            if constexpr (kKW > 0) {
+                // Stride 1, unit dilation, kKW x kKW: every filter row reads a window of
+                // kR + kKW - 1 input pixels once; products in fp32 pairs started from the
+                // bias.  A tile row holds two groups of kR pixels (TW = 2*kR).
+                constexpr int kP = kV / 2;
+                for (int it = tid; it < items; it += 32 * kDwComputeWarps) {
+                    const int cg = it & 7, pg = it >> 3;
+                    const int py = pg >> 1, px0 = (pg & 1) * kR;
+                    const int oh = t.th * p.TH + py;
+                    const int ow0 = t.tw * p.TW + px0;
+                    const int c = t.chunk * kCC + cg * kV;
+                    if (oh >= p.Ho || ow0 >= p.Wo || c >= p.C) continue;
                     uint64_t accp[kR][kP];
+                    {
+                        const float *bq = bsm + cg * kV;
+                        uint64_t b2[kP];
 #pragma unroll
-                    for (int r = 0; r < kR; ++r)
+                        for (int v = 0; v < kP; ++v) b2[v] = pair(__float_as_uint(bq[2 * v]), __float_as_uint(bq[2 * v + 1]));
 #pragma unroll
-                        for (int v = 0; v < kP; ++v) accp[r][v] = 0ull;
+                        for (int r = 0; r < kR; ++r)
+#pragma unroll
+                            for (int v = 0; v < kP; ++v) accp[r][v] = b2[v];
+                    }
+                    const uint8_t *rp0 = stg + (static_cast<uint32_t>(py) * p.IW + px0) * kDwRowBytes + cg * 16;
+                    const uint8_t *wp0 = wsm + cg * 16;
 #pragma unroll
                     for (int kh = 0; kh < kKW; ++kh) {
-                        const uint8_t *rp = stg + static_cast<size_t>(py + kh) * p.IW * kDwRowBytes + cg * 16;
-                        const uint8_t *wp = wsm + kh * kKW * kDwRowBytes + cg * 16;
+                        const uint8_t *rp = rp0 + static_cast<uint32_t>(kh) * p.IW * kDwRowBytes;
+                        const uint8_t *wp = wp0 + kh * kKW * kDwRowBytes;
                         uint64_t win[kR + kKW - 1][kP];
 #pragma unroll
                         for (int j = 0; j < kR + kKW - 1; ++j)
-                            unpack16_pairs<kF32>(*reinterpret_cast<const uint4 *>(rp + (px0 + j) * kDwRowBytes), win[j]);
+                            unpack16_pairs<kF32>(*reinterpret_cast<const uint4 *>(rp + j * kDwRowBytes), win[j]);
 #pragma unroll
                         for (int kw = 0; kw < kKW; ++kw) {
                             uint64_t wv[kP];
@@ -275,86 +418,16 @@ __global__ void __launch_bounds__(kDwThreads, 1) dw_kernel(const __grid_constant
                                 for (int v = 0; v < kP; ++v) fma2(accp[r][v], win[r + kw][v], wv[v]);
                         }
                     }
+                    // epilogue: one rounding, store (the bias is already in)
+                    const bool whole = c + kV <= p.C && p.vec_ok;
+                    const size_t pix0 = (static_cast<size_t>(t.n) * p.Ho + oh) * p.Wo + ow0;
 #pragma unroll
-                    for (int r = 0; r < kR; ++r)
+                    for (int r = 0; r < kR; ++r) {
+                        if (ow0 + r >= p.Wo) break;
+                        float o[kV];
 #pragma unroll
-                        for (int v = 0; v < kP; ++v) unpair(accp[r][v], acc[r][2 * v], acc[r][2 * v + 1]);
-                } else {
-#pragma unroll
-                    for (int r = 0; r < kR; ++r)
-#pragma unroll
-                        for (int v = 0; v < kV; ++v) acc[r][v] = 0.f;
-                    for (int kh = 0; kh < p.Kh; ++kh) {
-                        const int row = py * p.stride + kh * p.dilation;
-                        const uint8_t *rp = stg + static_cast<size_t>(row) * p.IW * kDwRowBytes + cg * 16;
-                        const uint8_t *wp = wsm + kh * p.Kw * kDwRowBytes + cg * 16;
-                        for (int kw = 0; kw < p.Kw; ++kw) {
-                            float wv[kV];
-                            unpack16<kF32>(*reinterpret_cast<const uint4 *>(wp + kw * kDwRowBytes), wv);
-#pragma unroll
-                            for (int r = 0; r < kR; ++r) {
-                                const int col = (px0 + r) * p.stride + kw * p.dilation;
-                                float xv[kV];
-                                unpack16<kF32>(*reinterpret_cast<const uint4 *>(rp + col * kDwRowBytes), xv);
-#pragma unroll
-                                for (int v = 0; v < kV; ++v) acc[r][v] = fmaf(xv[v], wv[v], acc[r][v]);
-                            }
-                        }
-                    }
-                }
-                // epilogue: + bias, one rounding, store
-                const int c = t.chunk * kCC + cg * kV;
-                if (c >= p.C) continue;
-                float bv[kV];
-#pragma unroll
-                for (int v = 0; v < kV; ++v) bv[v] = bsm[cg * kV + v];
-                const bool whole = c + kV <= p.C && p.vec_ok;
-#pragma unroll
-                for (int r = 0; r < kR; ++r) {
-                    const int ow = ow0 + r;
-                    if (ow >= p.Wo) break;
-                    float o[kV];
-#pragma unroll
-                    for (int v = 0; v < kV; ++v) o[v] = acc[r][v] + bv[v];
-                    const size_t pix = (static_cast<size_t>(t.n) * p.Ho + oh) * p.Wo + ow;
-                    if (!p.out_nchw) {
-                        if constexpr (kF32) {
-                            float *dst = static_cast<float *>(p.y) + pix * p.C + c;
-                            if (whole) {
-                                *reinterpret_cast<float4 *>(dst) = make_float4(o[0], o[1], o[2], o[3]);
-                            } else {
-#pragma unroll
-                                for (int v = 0; v < kV; ++v)
-                                    if (c + v < p.C) dst[v] = o[v];
-                            }
-                        } else {
-                            __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.y) + pix * p.C + c;
-                            if (whole) {
-                                uint32_t pk[4];
-#pragma unroll
-                                for (int i = 0; i < 4; ++i) {
-                                    __nv_bfloat162 h = __floats2bfloat162_rn(o[2 * i], o[2 * i + 1]);
-                                    pk[i] = *reinterpret_cast<uint32_t *>(&h);
-                                }
-                                *reinterpret_cast<uint4 *>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                            } else {
-#pragma unroll
-                                for (int v = 0; v < kV; ++v)
-                                    if (c + v < p.C) dst[v] = __float2bfloat16_rn(o[v]);
-                            }
-                        }
-                    } else {  // NCHW: y[n][c][oh][ow]
-                        const size_t plane = static_cast<size_t>(p.Ho) * p.Wo;
-                        const size_t at = (static_cast<size_t>(t.n) * p.C + c) * plane +
-                                          static_cast<size_t>(oh) * p.Wo + ow;
-#pragma unroll
-                        for (int v = 0; v < kV; ++v) {
-                            if (c + v >= p.C) break;
-                            if constexpr (kF32)
-                                static_cast<float *>(p.y)[at + v * plane] = o[v];
-                            else
-                                static_cast<__nv_bfloat16 *>(p.y)[at + v * plane] = __float2bfloat16_rn(o[v]);
-                        }
+                        for (int v = 0; v < kP; ++v) unpair(accp[r][v], o[2 * v], o[2 * v + 1]);
+                        dw_store<kF32, kV>(p, pix0 + r, static_cast<size_t>(t.n), oh, ow0 + r, c, o, whole);
                     }
                 }
             }
