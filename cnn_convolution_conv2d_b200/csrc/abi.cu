@@ -139,6 +139,7 @@ struct Plan {
     bool vol;       // 3-D convolution: input depth D, filter depth Kd, output depth Do
     bool vreuse;    // ... on the input-slice-reuse kernel (vol.cu)
     bool pw;        // 1x1 on the kernel with resident weights (pw.cu)
+    int pw_ybufs;   // its output staging blocks per epilogue warp
     int vJ, vn_k, vn_odb;  // its output slices per unit, tiles per slice, slice blocks
     int D, Kd, Do;
     bool f32;
@@ -608,19 +609,28 @@ int make_plan(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stri
     if (p.stages < 2) return fail(CONV_ERR_UNSUPPORTED, "tile does not fit in shared memory");
     p.smem = igemm_smem_bytes(p.f32, bn_local, p.stages, p.tma_out);
     // A pointwise layer with a short reduction on CTA pairs: the kernel that keeps each
-    // cluster's 256-column weight tile resident and streams only the input rows (pw.cu).
+    // cluster's 256-column weight tile resident and streams only the input rows (pw.cu);
+    // bf16 channels-last output, or the raw fp32 sums a later pass finishes (Winograd).
     p.pw = false;
-    if (p.pair && p.direct_a && p.tma_out && !p.f32 && groups == 1 && layout == CONV_NHWC && C_in % 64 == 0 &&
-        C_in == p.Cpg && C_in / 64 <= pw_max_planes() && C_out % 256 == 0 && p.BN == 256) {
-        int pst = pw_max_stages();
-        while (pst > 3 && pw_smem_bytes(C_in / 64, 256, pst) > kSmemBudget) --pst;
-        if (pw_smem_bytes(C_in / 64, 256, pst) <= kSmemBudget) {
-            p.pw = true;
-            p.stages = pst;
-            p.smem = pw_smem_bytes(C_in / 64, 256, pst);
+    p.pw_ybufs = 2;
+    const bool partial_ext = padw && padw->partial_out;
+    const int pw_nk = p.Cin_g / 64;
+    if (p.pair && p.direct_a && !p.f32 && p.splits == 1 && p.gm == 1 && layout == CONV_NHWC &&
+        (partial_ext || p.tma_out) && p.Cin_g % 64 == 0 && p.Cin_g == p.Cpg && pw_nk <= pw_max_planes() &&
+        p.Cout_g % 256 == 0 && p.BN == 256) {
+        // two staging blocks per epilogue warp while that leaves four input stages, else one
+        for (int yb = 2; yb >= 1 && !p.pw; --yb) {
+            int pst = pw_max_stages();
+            while (pst > 4 && pw_smem_bytes(pw_nk, 256, pst, partial_ext, yb) > kSmemBudget) --pst;
+            if (pw_smem_bytes(pw_nk, 256, pst, partial_ext, yb) <= kSmemBudget) {
+                p.pw = true;
+                p.pw_ybufs = yb;
+                p.stages = pst;
+                p.smem = pw_smem_bytes(pw_nk, 256, pst, partial_ext, yb);
+            }
         }
+        if (p.pw) p.tma_out = true;
     }
-
     size_t off = 0;
     p.off_xcopy = off;
     if (p.xcopy) off = align_up(off + static_cast<size_t>(N) * p.D * H * W * p.groups * p.Cpg * p.elt, 256);
@@ -904,17 +914,17 @@ int pair_cluster_limit(int cb, bool im2col, size_t smem, bool vol = false) {
 
 // Resident two-CTA clusters of the pointwise kernel (pw.cu) at this shared-memory size,
 // asked of the runtime once per device and size and remembered.
-int pw_cluster_limit(size_t smem) {
+int pw_cluster_limit(size_t smem, bool out_f32) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-    const long long key = -((static_cast<long long>(dev) + 1) * 1048576 + static_cast<long long>(smem));
+    const long long key = -(((static_cast<long long>(dev) + 1) * 2 + (out_f32 ? 1 : 0)) * 1048576 + static_cast<long long>(smem));
     {
         std::lock_guard<std::mutex> lock(g_mutex);
         auto it = g_pair_clusters.find(key);
         if (it != g_pair_clusters.end()) return it->second;
     }
     int n = 0;
-    if (pw_max_clusters(smem, &n) != cudaSuccess) {
+    if (pw_max_clusters(smem, out_f32, &n) != cudaSuccess) {
         (void)cudaGetLastError();
         n = 0;
     }
@@ -937,9 +947,10 @@ int device_plan(bool explicit_im2col, int N, int C_in, int H, int W, int C_out, 
     if (p->vreuse) return CONV_OK;
     if (p->pw && dev) {
         // clusters split evenly over the column tiles
-        const int n = pw_cluster_limit(p->smem);
-        p->pair_clusters = (n / p->n_ntiles) * p->n_ntiles;
-        if (p->pair_clusters >= p->n_ntiles) return CONV_OK;
+        const int per = p->n_ntiles * p->groups;  // (group, column tile) pairs
+        const int n = pw_cluster_limit(p->smem, padw && padw->partial_out);
+        p->pair_clusters = (n / per) * per;
+        if (p->pair_clusters >= per) return CONV_OK;
         return make_plan(N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype, layout,
                          explicit_im2col, dev->sms, p, cfg.pair_mode, false, padw, vol);
     }
@@ -1016,7 +1027,9 @@ int vol_impl(const Plan &p, const void *x, const void *w_packed, const void *bia
 
 // The pointwise path with resident weights (pw.cu): one kernel, no scratch.
 int pw_impl(const Plan &p, const void *x, const void *w_packed, const void *bias, void *y, DeviceInfo *dev,
-            const Settings &cfg, cudaStream_t stream) {
+            const Settings &cfg, cudaStream_t stream, float *partial_out) {
+    const bool out_f32 = partial_out != nullptr;
+    void *dst = out_f32 ? static_cast<void *>(partial_out) : y;
     PwParams k;
     std::memset(&k, 0, sizeof(k));
     int st = encode_a_xcol(p, x, &k.tmap_a);
@@ -1024,25 +1037,32 @@ int pw_impl(const Plan &p, const void *x, const void *w_packed, const void *bias
     st = encode_b(p, w_packed, &k.tmap_b);
     if (st != CONV_OK) return st;
     {
+        const int oelt = out_f32 ? 4 : p.elt;
         cuuint64_t dims[2] = {static_cast<cuuint64_t>(p.C_out), static_cast<cuuint64_t>(p.M)};
-        cuuint64_t strides[1] = {static_cast<cuuint64_t>(p.C_out) * p.elt};
+        cuuint64_t strides[1] = {static_cast<cuuint64_t>(p.C_out) * oelt};
         cuuint32_t box[2] = {32, 32};
         cuuint32_t estr[2] = {1, 1};
-        CUresult r = g_encode_tiled(&k.tmap_y, tma_type(p), 2, y, dims, strides, box, estr,
-                                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+        CUresult r = g_encode_tiled(&k.tmap_y, out_f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : tma_type(p), 2, dst, dims,
+                                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                    out_f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
                                     CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS)
             return fail(CONV_ERR_CUDA, "cuTensorMapEncodeTiled (output) failed (%d)", static_cast<int>(r));
     }
     k.M = static_cast<int>(p.M);
-    k.nk = p.C_in / 64;
+    k.nk = p.Cin_g / 64;
+    k.groups = p.groups;
+    k.Kp = p.Kp;
+    k.Cout_g = p.Cout_g;
+    k.out_f32 = out_f32 ? 1 : 0;
+    k.ybufs = p.pw_ybufs;
     k.BN = p.BN;
     k.n_ntiles = p.n_ntiles;
     k.m_tiles = static_cast<int>((p.M + 255) / 256);
-    k.cpn = p.pair_clusters / p.n_ntiles;
+    k.cpn = p.pair_clusters / (p.n_ntiles * p.groups);
     k.stages = p.stages;
     k.tmem_cols = 512;
-    k.bias = bias;
+    k.bias = out_f32 ? nullptr : bias;
     k.status = dev->status;
     k.timeout_ns = cfg.timeout_ns;
     k.starve = cfg.starve;
@@ -1084,7 +1104,7 @@ int forward_impl(bool explicit_im2col, const void *x, const void *w_packed, cons
     if (p.gather) return gather_impl(p, x, w_packed, bias, y, dev, cfg, stream);
     if (p.dw) return dw_impl(p, x, w_packed, bias, y, workspace, dev, cfg, stream);
     if (p.vreuse) return vol_impl(p, x, w_packed, bias, y, dev, cfg, stream);
-    if (p.pw) return pw_impl(p, x, w_packed, bias, y, dev, cfg, stream);
+    if (p.pw) return pw_impl(p, x, w_packed, bias, y, dev, cfg, stream, padw ? padw->partial_out : nullptr);
 
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     const void *x_nhwc = p.xcopy ? static_cast<const void *>(ws + p.off_xcopy) : x;

@@ -81,14 +81,18 @@ struct VolParams {
     int starve;
 };
 
-// One launch of the pointwise kernel (pw.cu): 1x1, stride 1, no padding, bf16, groups 1,
-// channels-last, C_in = 64*nk (nk <= 4), C_out a multiple of BN = 256, CTA pairs.  Cluster c
-// keeps column tile c % n_ntiles resident and takes row tiles c / n_ntiles + i*cpn.
+// One launch of the pointwise kernel (pw.cu): 1x1, stride 1, no padding, bf16 operands,
+// channels-last, per group C_in = 64*nk (nk <= 4) and C_out a multiple of BN = 256, CTA
+// pairs.  Cluster c keeps (group, column tile) c % (groups*n_ntiles) resident and takes row
+// tiles c / (groups*n_ntiles) + i*cpn.
 struct PwParams {
-    CUtensorMap tmap_a;  // x as X_col {C_in, M}, boxes of {64, 128}, 128-byte swizzle
-    CUtensorMap tmap_b;  // packed weights {C_in, C_out, 1}, boxes of {64, BN/2}, 128-byte swizzle
-    CUtensorMap tmap_y;  // y as {C_out, M}, 32 x 32 boxes with 64-byte swizzle
+    CUtensorMap tmap_a;  // x as X_col {groups*Kp, M}, boxes of {64, 128}, 128-byte swizzle
+    CUtensorMap tmap_b;  // packed weights {Kp, Cout_g, groups}, boxes of {64, BN/2, 1}, 128-byte swizzle
+    CUtensorMap tmap_y;  // y as {C_out, M}, 32 x 32 boxes: bf16 with 64-byte, fp32 with 128-byte swizzle
     int M, nk, BN, n_ntiles, m_tiles, cpn, stages;
+    int groups, Kp, Cout_g;
+    int out_f32;         // the raw fp32 sums (no bias) instead of bf16 + bias
+    int ybufs;           // output staging blocks per epilogue warp (1 or 2)
     uint32_t tmem_cols;
     const void *bias;
     int *status;
@@ -192,8 +196,8 @@ size_t gather_smem_bytes(bool f32, int BN, int Kpad, size_t halo_bytes, size_t o
 cudaError_t launch_gather_t(const GatherParams &p, int grid, size_t smem, cudaStream_t stream);
 cudaError_t launch_vol_reuse(const VolParams &p, int grid, size_t smem, cudaStream_t stream);
 cudaError_t launch_pw(const PwParams &p, size_t smem, cudaStream_t stream);
-cudaError_t pw_max_clusters(size_t smem, int *clusters);
-size_t pw_smem_bytes(int nk, int BN, int stages);
+cudaError_t pw_max_clusters(size_t smem, bool out_f32, int *clusters);
+size_t pw_smem_bytes(int nk, int BN, int stages, bool out_f32, int ybufs);
 int pw_max_stages();
 int pw_max_planes();
 size_t vol_reuse_smem_bytes(int Kd, int BN, int stages);

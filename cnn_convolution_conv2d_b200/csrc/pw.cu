@@ -11,9 +11,13 @@
 // tile of W^T resident (each CTA its 128 columns, loaded once) and streams only the A rows
 // of the row tiles it owns; the clusters are split evenly over the column tiles.
 //
-// CTA pairs on SM pairs (cta_group::2, M = 256 rows, N = 256 columns), bf16, C_in a multiple
-// of 64 up to 256, C_out a multiple of 256, channels-last output stored through
-// 64-byte-swizzled shared-memory blocks by TMA, bias added in fp32.
+// CTA pairs on SM pairs (cta_group::2, M = 256 rows, N = 256 columns), bf16 operands, per
+// group C_in a multiple of 64 up to 256 and C_out a multiple of 256; the clusters are split
+// evenly over (group, column tile).  Output through swizzled shared-memory blocks and TMA
+// stores: bf16 channels-last with the bias added in fp32, or the raw fp32 sums (the
+// Winograd path's channel products, finished by its output transform).  fp32 layers stay on
+// the general kernel: their three-product tf32 split needs the weights' low parts resident
+// too, which does not fit beside the input ring.
 //   warp 0     : loads: the resident weight planes once, then one A plane per stage;
 //   warp 1     : tensor-memory allocation; the even CTA issues the products;
 //   warps 2..9 : epilogue, two warps per tensor-memory lane quarter (halves of the columns).
@@ -32,13 +36,13 @@ constexpr int kPRows = 128;                 // A rows per CTA per tile
 constexpr int kPPlane = 128;                // bytes of one 64-channel plane row
 constexpr int kPAStage = kPRows * kPPlane;
 constexpr int kPMaxStages = 8;
-constexpr int kPMaxPlanes = 4;              // C_in <= 256
+constexpr int kPMaxPlanes = 4;              // 128-byte planes: C_in <= 256
 constexpr int kPHeader = 1024;
 constexpr int kPThreads = 320;
 constexpr int kPEpiWarp0 = 2;
 constexpr int kPEpiWarps = 8;
-constexpr int kPStageBuf = 32 * 64;         // one 32 x 32 bf16 output block
-constexpr int kPYStage = kPEpiWarps * 2 * kPStageBuf;
+// one 32 x 32 output block: 64-byte rows (bf16) or 128-byte rows (fp32); one or two per warp
+__host__ __device__ constexpr int pw_stage_buf(bool out_f32) { return 32 * (out_f32 ? 128 : 64); }
 
 struct PwShared {
     uint64_t full[kPMaxStages];
@@ -59,7 +63,10 @@ __device__ __forceinline__ void pw_wait_quiet(uint64_t *bar, uint32_t parity, ui
     }
 }
 
+template <bool kOutF32>
 __global__ void __launch_bounds__(kPThreads, 1) pw_kernel(const __grid_constant__ PwParams p) {
+    constexpr int kPStageBuf = pw_stage_buf(kOutF32);
+    constexpr int kPlaneElems = 64;  // channels in one 128-byte plane row
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_addr(smem_raw);
     uint8_t *base = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
@@ -69,15 +76,17 @@ __global__ void __launch_bounds__(kPThreads, 1) pw_kernel(const __grid_constant_
     const uint32_t plane_bytes = static_cast<uint32_t>(BNl) * kPPlane;
     uint8_t *bres = base + kPHeader;                          // resident weights: [plane][BNl][128 B]
     uint8_t *ring = bres + static_cast<uint32_t>(p.nk) * plane_bytes;
-    uint8_t *ystage = ring + p.stages * kPAStage;
+    uint8_t *ystage = ring + p.stages * kPAStage;                  // 1024-aligned: swizzled blocks
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();
-    // cluster c owns column tile c % n_ntiles and row tiles c / n_ntiles + i * cpn
+    // cluster c owns (group, column tile) c % (groups * n_ntiles) and row tiles
+    // c / (groups * n_ntiles) + i * cpn
     const int cl = static_cast<int>(blockIdx.x >> 1);
-    const int ntile = cl % p.n_ntiles;
-    const int mt0 = cl / p.n_ntiles;
+    const int gn = cl % (p.groups * p.n_ntiles);
+    const int g = gn / p.n_ntiles, ntile = gn - (gn / p.n_ntiles) * p.n_ntiles;
+    const int mt0 = cl / (p.groups * p.n_ntiles);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.stages; ++s) {
@@ -122,8 +131,8 @@ __global__ void __launch_bounds__(kPThreads, 1) pw_kernel(const __grid_constant_
                 // both CTAs' copies count on the even CTA's barrier (armed there for both)
                 if (rank == 0) mbar_arrive_expect_tx(&sb.b_ready, 2u * static_cast<uint32_t>(p.nk) * plane_bytes);
                 for (int kp = 0; kp < p.nk; ++kp)
-                    tma_load_3d_pair(bres + kp * plane_bytes, &p.tmap_b, bready0, kp * 64,
-                                     ntile * BN + static_cast<int>(rank) * BNl, 0);
+                    tma_load_3d_pair(bres + kp * plane_bytes, &p.tmap_b, bready0, kp * kPlaneElems,
+                                     ntile * BN + static_cast<int>(rank) * BNl, g);
                 b_issued = true;
             }
             int stage = 0;
@@ -143,7 +152,7 @@ __global__ void __launch_bounds__(kPThreads, 1) pw_kernel(const __grid_constant_
                     if (!p.starve) {
                         if (rank == 0) mbar_arrive_expect_tx(&sb.full[stage], 2u * kPAStage);
                         tma_load_2d_pair(ring + stage * kPAStage, &p.tmap_a, full0 + 8u * static_cast<uint32_t>(stage),
-                                         kp * 64, m0);
+                                         g * p.Kp + kp * kPlaneElems, m0);
                         ++loads_issued;
                     }
                     if (++stage == p.stages) {
@@ -236,7 +245,7 @@ __global__ void __launch_bounds__(kPThreads, 1) pw_kernel(const __grid_constant_
         const int cspan = ((BN / 2 + 31) & ~31);
         const int c_lo = min(BN, (e >> 2) * cspan), c_hi = min(BN, c_lo + cspan);
         const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-        const int col0 = ntile * BN;
+        const int col0 = g * p.Cout_g + ntile * BN;
         int abuf = 0;
         uint32_t aphase = 0;
         int sbi = 0;
@@ -257,46 +266,60 @@ __global__ void __launch_bounds__(kPThreads, 1) pw_kernel(const __grid_constant_
                     if (lane == 0) mbar_arrive_cluster(acc_empty0 + 8u * static_cast<uint32_t>(abuf));
                 }
                 if (mrow0 >= p.M) continue;
-                float bv[32];
-                if (p.bias) {
-                    const uint4 *b4 = reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(p.bias) + col0 + c);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const uint4 w = __ldg(b4 + q);
-                        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                        for (int h = 0; h < 4; ++h) {
-                            bv[8 * q + 2 * h] = __uint_as_float(ws[h] << 16);
-                            bv[8 * q + 2 * h + 1] = __uint_as_float(ws[h] & 0xFFFF0000u);
-                        }
-                    }
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) bv[i] = 0.f;
+                if (lane == 0) {  // this buffer's previous store has read it
+                    if (p.ybufs == 2)
+                        bulk_wait_group_read<1>();
+                    else
+                        bulk_wait_group_read<0>();
                 }
-                uint32_t pk[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float v0 = __uint_as_float(r[(2 * i) >> 4][(2 * i) & 15]) + bv[2 * i];
-                    const float v1 = __uint_as_float(r[(2 * i + 1) >> 4][(2 * i + 1) & 15]) + bv[2 * i + 1];
-                    __nv_bfloat162 h = __floats2bfloat162_rn(v0, v1);
-                    pk[i] = *reinterpret_cast<uint32_t *>(&h);
-                }
-                if (lane == 0) bulk_wait_group_read<1>();  // this buffer's previous store has read it
                 __syncwarp();
-                // 64-byte swizzle: 16-byte chunk q of row r goes to chunk q ^ ((r >> 1) & 3)
-                uint8_t *buf = ystage + (e * 2 + sbi) * kPStageBuf;
+                uint8_t *buf = ystage + (e * p.ybufs + sbi) * kPStageBuf;
+                if constexpr (kOutF32) {
+                    // 128-byte swizzle: 16-byte chunk q of row r goes to chunk q ^ (r & 7)
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    *reinterpret_cast<uint4 *>(buf + lane * 64 + ((q ^ ((lane >> 1) & 3)) * 16)) =
-                        make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+                    for (int q = 0; q < 8; ++q)
+                        *reinterpret_cast<uint4 *>(buf + lane * 128 + ((q ^ (lane & 7)) * 16)) =
+                            make_uint4(r[q >> 2][4 * (q & 3)], r[q >> 2][4 * (q & 3) + 1], r[q >> 2][4 * (q & 3) + 2],
+                                       r[q >> 2][4 * (q & 3) + 3]);
+                } else {
+                    float bv[32];
+                    if (p.bias) {
+                        const uint4 *b4 = reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(p.bias) + col0 + c);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const uint4 w = __ldg(b4 + q);
+                            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                            for (int h = 0; h < 4; ++h) {
+                                bv[8 * q + 2 * h] = __uint_as_float(ws[h] << 16);
+                                bv[8 * q + 2 * h + 1] = __uint_as_float(ws[h] & 0xFFFF0000u);
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) bv[i] = 0.f;
+                    }
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const float v0 = __uint_as_float(r[(2 * i) >> 4][(2 * i) & 15]) + bv[2 * i];
+                        const float v1 = __uint_as_float(r[(2 * i + 1) >> 4][(2 * i + 1) & 15]) + bv[2 * i + 1];
+                        __nv_bfloat162 h = __floats2bfloat162_rn(v0, v1);
+                        pk[i] = *reinterpret_cast<uint32_t *>(&h);
+                    }
+                    // 64-byte swizzle: 16-byte chunk q of row r goes to chunk q ^ ((r >> 1) & 3)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        *reinterpret_cast<uint4 *>(buf + lane * 64 + ((q ^ ((lane >> 1) & 3)) * 16)) =
+                            make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+                }
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {
                     tma_store_2d(&p.tmap_y, buf, col0 + c, mrow0);
                     bulk_commit_group();
                 }
-                sbi ^= 1;
+                sbi ^= p.ybufs - 1;
             }
             if (c_lo >= c_hi) {  // nothing to drain in this half: release at once
                 tc_fence_before_sync();
@@ -320,17 +343,23 @@ __global__ void __launch_bounds__(kPThreads, 1) pw_kernel(const __grid_constant_
 
 }  // namespace
 
-size_t pw_smem_bytes(int nk, int BN, int stages) {
+size_t pw_smem_bytes(int nk, int BN, int stages, bool out_f32, int ybufs) {
     return 1024 /* alignment slack */ + kPHeader + static_cast<size_t>(nk) * (BN / 2) * kPPlane +
-           static_cast<size_t>(stages) * kPAStage + kPYStage;
+           static_cast<size_t>(stages) * kPAStage + static_cast<size_t>(kPEpiWarps) * ybufs * pw_stage_buf(out_f32);
 }
+
+namespace {
+using PwKernel = void (*)(PwParams);
+PwKernel pw_kernel_for(bool out_f32) { return out_f32 ? pw_kernel<true> : pw_kernel<false>; }
+}  // namespace
 
 int pw_max_stages() { return kPMaxStages; }
 int pw_max_planes() { return kPMaxPlanes; }
 
-cudaError_t pw_max_clusters(size_t smem, int *out) {
+cudaError_t pw_max_clusters(size_t smem, bool out_f32, int *out) {
     *out = 0;
-    cudaError_t e = cudaFuncSetAttribute(pw_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    const PwKernel kern = pw_kernel_for(out_f32);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2);
@@ -343,17 +372,20 @@ cudaError_t pw_max_clusters(size_t smem, int *out) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaOccupancyMaxActiveClusters(out, pw_kernel, &cfg);
+    return cudaOccupancyMaxActiveClusters(out, kern, &cfg);
 }
 
 cudaError_t launch_pw(const PwParams &p, size_t smem, cudaStream_t stream) {
     if (p.stages < 2 || p.stages > kPMaxStages || p.nk < 1 || p.nk > kPMaxPlanes || p.BN != 256 ||
-        p.n_ntiles < 1 || p.cpn < 1 || p.m_tiles < 1 || 2 * p.BN > static_cast<int>(p.tmem_cols))
+        p.n_ntiles < 1 || p.groups < 1 || p.cpn < 1 || p.m_tiles < 1 || 2 * p.BN > static_cast<int>(p.tmem_cols) ||
+        p.Kp < 64 * p.nk || p.Cout_g < p.BN * p.n_ntiles || (p.ybufs != 1 && p.ybufs != 2) ||
+        (p.bias && p.out_f32))
         return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(pw_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    const PwKernel kern = pw_kernel_for(p.out_f32 != 0);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(2 * p.cpn * p.n_ntiles));
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * p.cpn * p.n_ntiles * p.groups));
     cfg.blockDim = dim3(kPThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
@@ -364,7 +396,7 @@ cudaError_t launch_pw(const PwParams &p, size_t smem, cudaStream_t stream) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, pw_kernel, p);
+    e = cudaLaunchKernelEx(&cfg, kern, p);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

@@ -135,20 +135,22 @@ def test_pair_explicit_im2col_gemm(name, pairs_forced):
     parity.assert_close(cfg, got, parity.run_oracle(cfg, inp), name + " (pair, explicit im2col)")
 
 
-PW_SHAPES = [  # 1x1, stride 1, no padding: the kernel with each cluster's weight tile resident
-    ((2, 64, 9, 9, 256, 1, 1, 1, 0, 1, 1), True),     # M = 162: one row tile, the odd CTA's rows partly past M
-    ((3, 128, 10, 11, 512, 1, 1, 1, 0, 1, 1), True),  # two column tiles, M = 330: a ragged second row tile
-    ((1, 256, 12, 12, 768, 1, 1, 1, 0, 1, 1), False), # reduction 256 (four planes), three column tiles, no bias
-    ((2, 192, 8, 8, 256, 1, 1, 1, 0, 1, 1), True),    # three planes
+PW_SHAPES = [  # 1x1, stride 1, no padding: the kernel with each cluster's weight tile resident (bf16)
+    ((2, 64, 9, 9, 256, 1, 1, 1, 0, 1, 1), True, "bf16"),     # M = 162: one row tile, the odd CTA's rows partly past M
+    ((3, 128, 10, 11, 512, 1, 1, 1, 0, 1, 1), True, "bf16"),  # two column tiles, M = 330: a ragged second row tile
+    ((1, 256, 12, 12, 768, 1, 1, 1, 0, 1, 1), False, "bf16"), # reduction 256 (four planes), three column tiles, no bias
+    ((2, 192, 8, 8, 256, 1, 1, 1, 0, 1, 1), True, "bf16"),    # three planes
+    ((2, 128, 8, 9, 512, 1, 1, 1, 0, 1, 2), True, "bf16"),    # two groups of 64 -> 256: clusters over (group, tile)
 ]
 
 
-@pytest.mark.parametrize("shape,bias", PW_SHAPES, ids=lambda s: "x".join(map(str, s)) if isinstance(s, tuple) else str(s))
-def test_pointwise_resident_weights(shape, bias, pairs_forced):
+@pytest.mark.parametrize("shape,bias,dtype", PW_SHAPES,
+                         ids=lambda s: "x".join(map(str, s)) if isinstance(s, tuple) else str(s))
+def test_pointwise_resident_weights(shape, bias, dtype, pairs_forced):
     N, C_in, H, W, C_out, Kh, Kw, s, p, d, g = shape
-    plan = cb.conv2d_describe_plan(*shape, cb.CONV_BF16, "nhwc")
+    plan = cb.conv2d_describe_plan(*shape, cb.CONV_BF16 if dtype == "bf16" else cb.CONV_F32, "nhwc")
     assert plan["kernel"] == "pointwise", plan
-    cfg = workloads.ConvConfig("pw", N, C_in, H, W, C_out, Kh, Kw, s, p, d, g, bias, "bf16", "nhwc",
+    cfg = workloads.ConvConfig("pw", N, C_in, H, W, C_out, Kh, Kw, s, p, d, g, bias, dtype, "nhwc",
                                seed=sum(shape) + 21)
     inp = workloads.make_inputs(cfg)
     parity.assert_close(cfg, parity.run_gpu(cfg, inp), parity.run_oracle(cfg, inp), str(shape) + " (pointwise)")

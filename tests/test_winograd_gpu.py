@@ -45,6 +45,7 @@ WINO = [  # N, C_in, H, W, C_out, pad
     (1, 64, 8, 8, 16, 0),        # no padding: 6x6 outputs
     (1, 16, 7, 7, 200, 2),       # pad 2, 200 output channels
     (1, 256, 14, 14, 256, 1),    # 256 channels each way
+    (1, 96, 9, 9, 512, 1),       # 96 input channels, two 256-column tiles per transformed channel
 ]
 
 
