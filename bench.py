@@ -893,6 +893,18 @@ def run_winograd(args, cfg):
     v_bytes = tiles * a2 * cpg * e
     m_bytes = tiles * a2 * cfg.C_out * 4
     step_b = step_bytes(cfg) + 2 * v_bytes + 2 * m_bytes
+    # the product reads V and the transformed filters once and writes M once: bound by
+    # whichever of its FLOPs and bytes takes longer at the measured peaks
+    prod_bytes = v_bytes + m_bytes + a2 * cfg.C_out * cpg * e
+    prod_plan = cb.conv2d_winograd_describe_plan(cfg.N, cfg.C_in, cfg.H, cfg.W, cfg.C_out, cfg.pad, m,
+                                                 cb.CONV_BF16 if cfg.dtype == "bf16" else cb.CONV_F32, cfg.layout)
+    hbm_bound = prod_bytes / (peaks["hbm_gbs"] * 1e9) > mult * gemm_flops / (tpeak * 1e12)
+    if hbm_bound:
+        ach, pk, unit = prod_bytes / (kernel_ms * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s"
+        psrc = f"{peak_kind} HBM copy bandwidth"
+    else:
+        ach, pk, unit = mult * gemm_flops / (kernel_ms * 1e-3) / 1e12, tpeak, "TFLOP/s"
+        psrc = f"{peak_kind} bf16 sustained" + ("" if mult == 1 else " x 0.5")
     line = {
         "metric": "conv2d fwd TFLOP/s on 1 B200 and % of dense tensor (or HBM) roofline",
         "value": flops(cfg) * args.steps / (elapsed * 1e-3) / 1e12, "unit": "TFLOP/s", "n_gpus": 1,
@@ -901,11 +913,13 @@ def run_winograd(args, cfg):
         "config": {"workload": workload_config(cfg, args, 1)["workload"], "path": f"Winograd F({m}x{m},3x3)",
                    "l2": f"not resident: steps rotate over {nsets} sets",
                    "launch": f"CUDA graphs of {G} steps x {reps} replays"},
-        "roofline": {"bound": "tensor", "achieved": mult * gemm_flops / (kernel_ms * 1e-3) / 1e12, "peak": tpeak,
-                     "unit": "TFLOP/s", "frac": mult * gemm_flops / (kernel_ms * 1e-3) / 1e12 / tpeak,
-                     "peak_source": f"{peak_kind} bf16 sustained" + ("" if mult == 1 else " x 0.5"),
-                     "kernel": "igemm_kernel on the transformed tiles ((m+2)^2 groups of 1x1)",
-                     "kernel_ms": kernel_ms, "gemm_flops_per_launch": gemm_flops, "traffic": None,
+        "roofline": {"bound": "hbm" if hbm_bound else "tensor", "achieved": ach, "peak": pk, "unit": unit,
+                     "frac": ach / pk, "peak_source": psrc,
+                     "kernel": ("pw_kernel" if prod_plan["kernel"] == "pointwise" else "igemm_kernel")
+                     + " on the transformed tiles ((m+2)^2 groups of 1x1)",
+                     "kernel_ms": kernel_ms, "gemm_flops_per_launch": gemm_flops,
+                     "product_bytes_per_launch": prod_bytes,
+                     "tensor_frac": mult * gemm_flops / (kernel_ms * 1e-3) / 1e12 / tpeak, "traffic": None,
                      "multiplies_vs_direct": a2 / (m * m * 9.0),
                      "step_bytes": step_b, "step_hbm_frac": step_b / (elapsed / args.steps * 1e-3) / 1e9 / peaks["hbm_gbs"]},
         "accuracy_vs_oracle": err,

@@ -69,6 +69,7 @@ SIGNATURES = {
     "conv2d_pack_weight_winograd": ([_P, _P, _I, _I, _I, _I, _P], _I),
     "conv2d_winograd_workspace_size": ([_I] * 7 + [_I, _I, ctypes.POINTER(_S)], _I),
     "conv2d_forward_winograd": ([_P, _P, _P, _P] + [_I] * 7 + [_I, _I, _P, _S, _P], _I),
+    "conv2d_winograd_describe_plan": ([_I] * 7 + [_I, _I, _I, ctypes.c_char_p, ctypes.c_size_t], _I),
 }
 
 _lib = None
@@ -283,6 +284,15 @@ def conv3d_describe_plan(N, C_in, D, H, W, C_out, Kd, Kh, Kw, stride, pad, dilat
     buf = ctypes.create_string_buffer(512)
     _check(load().conv3d_describe_plan(N, C_in, D, H, W, C_out, Kd, Kh, Kw, stride, pad, dilation, groups, dtype,
                                        _layout_code(layout), int(sms), buf, ctypes.sizeof(buf)))
+    return json.loads(buf.value.decode())
+
+
+def conv2d_winograd_describe_plan(N, C_in, H, W, C_out, pad, m, dtype, layout, sms=-1) -> dict:
+    """The plan of conv2d_forward_winograd's channel product as a dict."""
+    import json
+    buf = ctypes.create_string_buffer(512)
+    _check(load().conv2d_winograd_describe_plan(N, C_in, H, W, C_out, pad, m, dtype, _layout_code(layout), int(sms),
+                                                buf, ctypes.sizeof(buf)))
     return json.loads(buf.value.decode())
 
 

@@ -1212,21 +1212,22 @@ int forward_impl(bool explicit_im2col, const void *x, const void *w_packed, cons
 // no device-dependent choices); sms >= 0: as if the device had that many SMs.
 int describe_impl(bool explicit_im2col, int N, int C_in, int H, int W, int C_out, int Kh, int Kw,
                   int stride, int pad, int dilation, int groups, conv_dtype_t dtype,
-                  conv_layout_t layout, int sms, char *buf, size_t buflen, const Vol *vol = nullptr) {
+                  conv_layout_t layout, int sms, char *buf, size_t buflen, const Vol *vol = nullptr,
+                  const PadW *padw = nullptr) {
     if (!buf || buflen == 0) return fail(CONV_ERR_INVALID_ARG, "buf must not be NULL");
     const Settings cfg = settings_now();
     Plan p;
     int st = make_plan(N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype, layout,
-                       explicit_im2col, 0, &p, cfg.pair_mode, true, nullptr, vol);
+                       explicit_im2col, 0, &p, cfg.pair_mode, true, padw, vol);
     if (st != CONV_OK) return st;
     if (sms < 0) {
         DeviceInfo *dev = current_device_or_null();
         sms = dev ? dev->sms : 0;
         st = device_plan(explicit_im2col, N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups,
-                         dtype, layout, dev, cfg, &p, nullptr, vol);
+                         dtype, layout, dev, cfg, &p, padw, vol);
     } else {
         st = make_plan(N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype, layout,
-                       explicit_im2col, sms, &p, cfg.pair_mode, true, nullptr, vol);
+                       explicit_im2col, sms, &p, cfg.pair_mode, true, padw, vol);
     }
     if (st != CONV_OK) return st;
     const char *a_load = p.dw ? "tile" : p.gather ? "gather" : explicit_im2col ? "xcol" : p.direct_a ? "tiled_x" : "im2col";
@@ -1881,6 +1882,17 @@ int conv3d_describe_plan(int N, int C_in, int D, int H, int W, int C_out, int Kd
     const Vol vol{D, Kd};
     return describe_impl(false, N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype, layout, sms, buf,
                          buflen, &vol);
+}
+
+int conv2d_winograd_describe_plan(int N, int C_in, int H, int W, int C_out, int pad, int m, conv_dtype_t dtype,
+                                  conv_layout_t layout, int sms, char *buf, size_t buflen) {
+    WinoPlan w;
+    int st = wino_plan(N, C_in, H, W, C_out, pad, m, dtype, layout, nullptr, settings_now(), &w);
+    if (st != CONV_OK) return st;
+    const int a2 = w.a * w.a;
+    const PadW pw{0, reinterpret_cast<float *>(16)};  // placeholder address: plans the external-partial form
+    return describe_impl(false, 1, a2 * w.Cpg, 1, w.T, a2 * C_out, 1, 1, 1, 0, 1, a2, w.tdt, CONV_NHWC, sms, buf,
+                         buflen, nullptr, &pw);
 }
 
 int conv2d_debug_set_pair_mode(int mode) {

@@ -382,6 +382,15 @@ int conv2d_forward_winograd(const void *x, const void *u_packed, const void *bia
                             conv_dtype_t dtype, conv_layout_t layout, void *workspace,
                             size_t workspace_bytes, conv_stream_t stream);
 
+/* The plan of conv2d_forward_winograd's channel product (the (m+2)^2-group 1x1 product of
+ * the transformed tiles), as conv2d_describe_plan's JSON object: "pointwise" where the
+ * product runs on the kernel with resident weights (bf16 transforms, C_in a multiple of 64
+ * up to 256, C_out a multiple of 256), else "igemm".  Arguments as conv2d_forward_winograd;
+ * sms and buf as conv2d_describe_plan.  Nothing runs on the device. */
+int conv2d_winograd_describe_plan(int N, int C_in, int H, int W, int C_out, int pad, int m,
+                                  conv_dtype_t dtype, conv_layout_t layout, int sms, char *buf,
+                                  size_t buflen);
+
 /* Measurement aid: when `start` and `stop` (cudaEvent_t handles the caller created
  * with timing enabled) are both non-NULL, every later forward call records `start`
  * on its stream immediately before launching its tensor-core kernel and `stop`

@@ -189,6 +189,20 @@ def test_plan_for_the_workloads_on_a_148_sm_device(lib):
     assert f32["pair"] == 0 and f32["BN"] == 128                        # CTA pairs are bf16 only
 
 
+def test_winograd_product_plans(lib):
+    """The Winograd channel product on the 3x3 layer: F(2x2,3x3) (bf16 transforms) on the
+    resident-weight pair kernel, 16 groups of 256 -> 256 over 64 x 28 x 28 tiles; F(4x4,3x3)
+    (fp32 transforms, three tf32 products) on the general kernel."""
+    p2 = cb.conv2d_winograd_describe_plan(64, 256, 56, 56, 256, 1, 2, cb.CONV_BF16, "nhwc", sms=148)
+    assert (p2["kernel"], p2["pair"], p2["BN"], p2["units"]) == ("pointwise", 1, 256, 16 * (64 * 28 * 28 // 256))
+    p4 = cb.conv2d_winograd_describe_plan(64, 256, 56, 56, 256, 1, 4, cb.CONV_BF16, "nhwc", sms=148)
+    assert (p4["kernel"], p4["pair"]) == ("igemm", 0)
+    p2n = cb.conv2d_winograd_describe_plan(1, 96, 9, 9, 512, 1, 2, cb.CONV_BF16, "nchw", sms=148)
+    assert p2n["kernel"] == "igemm"                      # 96 channels: not whole 64-channel planes
+    with pytest.raises(cb.Conv2dError):
+        cb.conv2d_winograd_describe_plan(1, 8, 8, 8, 8, 1, 3, cb.CONV_BF16, "nhwc")
+
+
 def test_plan_without_a_device_count_makes_no_device_choices(lib):
     p = _plan((64, 256, 56, 56, 256, 3, 3, 1, 1, 1, 1), sms=0)
     assert p["pair"] == 0 and p["splits"] == 1 and p["units"] == 1568 and p["sms"] == 0

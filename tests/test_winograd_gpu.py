@@ -78,6 +78,18 @@ def test_winograd_full_size_3x3_sampled(m):
     assert np.abs(got - ref).max() <= parity.BF16_MAXABS * np.abs(ref).max()
 
 
+def test_winograd_product_on_the_resident_weight_kernel():
+    """bf16 F(2x2,3x3) with 256 channels each way and 2048 tiles (enough 256-row pair units for
+    every SM pair): the product runs on the pair kernel with resident weights, writing the fp32
+    M blocks by TMA stores; the whole output is checked against the oracle."""
+    shape = (2, 256, 64, 64, 256, 1)
+    assert cb.conv2d_winograd_describe_plan(*shape, 2, cb.CONV_BF16, "nhwc")["kernel"] == "pointwise"
+    N, C_in, H, W, C_out, pad = shape
+    cfg = workloads.ConvConfig("wino_pw", N, C_in, H, W, C_out, 3, 3, 1, pad, 1, 1, False, "bf16", "nhwc", seed=77)
+    inp = workloads.make_inputs(cfg)
+    parity.assert_close(cfg, run_wino(cfg, inp, 2), parity.run_oracle(cfg, inp), "F(2x2,3x3) on the pointwise kernel")
+
+
 def test_winograd_rejects_other_tiles():
     with pytest.raises(cb.Conv2dError) as err:
         cb.conv2d_winograd_packed_weight_size(8, 8, 3, cb.CONV_BF16)
