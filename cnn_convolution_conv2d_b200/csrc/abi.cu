@@ -1040,11 +1040,10 @@ int pw_impl(const Plan &p, const void *x, const void *w_packed, const void *bias
         const int oelt = out_f32 ? 4 : p.elt;
         cuuint64_t dims[2] = {static_cast<cuuint64_t>(p.C_out), static_cast<cuuint64_t>(p.M)};
         cuuint64_t strides[1] = {static_cast<cuuint64_t>(p.C_out) * oelt};
-        cuuint32_t box[2] = {32, 32};
+        cuuint32_t box[2] = {out_f32 ? 32u : 64u, 32};  // 32 rows x 128 bytes
         cuuint32_t estr[2] = {1, 1};
         CUresult r = g_encode_tiled(&k.tmap_y, out_f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : tma_type(p), 2, dst, dims,
-                                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                                    out_f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                                     CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS)
             return fail(CONV_ERR_CUDA, "cuTensorMapEncodeTiled (output) failed (%d)", static_cast<int>(r));

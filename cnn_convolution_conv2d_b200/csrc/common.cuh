@@ -88,7 +88,7 @@ struct VolParams {
 struct PwParams {
     CUtensorMap tmap_a;  // x as X_col {groups*Kp, M}, boxes of {64, 128}, 128-byte swizzle
     CUtensorMap tmap_b;  // packed weights {Kp, Cout_g, groups}, boxes of {64, BN/2, 1}, 128-byte swizzle
-    CUtensorMap tmap_y;  // y as {C_out, M}, 32 x 32 boxes: bf16 with 64-byte, fp32 with 128-byte swizzle
+    CUtensorMap tmap_y;  // y as {C_out, M}, boxes of 32 rows x 128 bytes, 128-byte swizzle
     int M, nk, BN, n_ntiles, m_tiles, cpn, stages;
     int groups, Kp, Cout_g;
     int out_f32;         // the raw fp32 sums (no bias) instead of bf16 + bias

@@ -41,8 +41,9 @@ constexpr int kPHeader = 1024;
 constexpr int kPThreads = 320;
 constexpr int kPEpiWarp0 = 2;
 constexpr int kPEpiWarps = 8;
-// one 32 x 32 output block: 64-byte rows (bf16) or 128-byte rows (fp32); one or two per warp
-__host__ __device__ constexpr int pw_stage_buf(bool out_f32) { return 32 * (out_f32 ? 128 : 64); }
+// one output block of 32 rows x 128 bytes (64 bf16 or 32 fp32 columns): whole 128-byte
+// lines of y per row; one or two staging buffers per epilogue warp
+constexpr int kPStageBuf = 32 * 128;
 
 struct PwShared {
     uint64_t full[kPMaxStages];
@@ -65,7 +66,7 @@ __device__ __forceinline__ void pw_wait_quiet(uint64_t *bar, uint32_t parity, ui
 
 template <bool kOutF32>
 __global__ void __launch_bounds__(kPThreads, 1) pw_kernel(const __grid_constant__ PwParams p) {
-    constexpr int kPStageBuf = pw_stage_buf(kOutF32);
+    constexpr int kBW = kOutF32 ? 32 : 64;  // columns per output block
     constexpr int kPlaneElems = 64;  // channels in one 128-byte plane row
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_addr(smem_raw);
@@ -239,7 +240,7 @@ __global__ void __launch_bounds__(kPThreads, 1) pw_kernel(const __grid_constant_
     } else {
         // ------------------------------------------------------------ epilogue ---
         // Warp e drains lane quarter (warp % 4) and columns [128*(e/4), + 128) of the
-        // accumulator; every 32 x 32 block goes out by one TMA store.
+        // accumulator; every 32-row x 128-byte block goes out by one TMA store.
         const int e = warp - kPEpiWarp0;
         const int quarter = warp & 3;
         const int cspan = ((BN / 2 + 31) & ~31);
@@ -255,12 +256,12 @@ __global__ void __launch_bounds__(kPThreads, 1) pw_kernel(const __grid_constant_
             tc_fence_after_sync();
             const int mrow0 = mt * 2 * kPRows + static_cast<int>(rank) * kPRows + quarter * 32;
             const uint32_t taddr = tmem_base + lane_base + static_cast<uint32_t>(abuf * BN);
-            for (int c = c_lo; c < c_hi; c += 32) {
-                uint32_t r[2][16];
-                tmem_ld_x16(taddr + static_cast<uint32_t>(c), r[0]);
-                tmem_ld_x16(taddr + static_cast<uint32_t>(c + 16), r[1]);
+            for (int c = c_lo; c < c_hi; c += kBW) {
+                uint32_t r[kBW / 16][16];
+#pragma unroll
+                for (int h = 0; h < kBW / 16; ++h) tmem_ld_x16(taddr + static_cast<uint32_t>(c + 16 * h), r[h]);
                 tmem_ld_wait();
-                if (c + 32 >= c_hi) {  // this warp's part of the accumulator is read
+                if (c + kBW >= c_hi) {  // this warp's part of the accumulator is read
                     tc_fence_before_sync();
                     __syncwarp();
                     if (lane == 0) mbar_arrive_cluster(acc_empty0 + 8u * static_cast<uint32_t>(abuf));
@@ -274,44 +275,40 @@ __global__ void __launch_bounds__(kPThreads, 1) pw_kernel(const __grid_constant_
                 }
                 __syncwarp();
                 uint8_t *buf = ystage + (e * p.ybufs + sbi) * kPStageBuf;
+                // 128-byte swizzle: 16-byte chunk q of row r goes to chunk q ^ (r & 7)
                 if constexpr (kOutF32) {
-                    // 128-byte swizzle: 16-byte chunk q of row r goes to chunk q ^ (r & 7)
 #pragma unroll
                     for (int q = 0; q < 8; ++q)
                         *reinterpret_cast<uint4 *>(buf + lane * 128 + ((q ^ (lane & 7)) * 16)) =
                             make_uint4(r[q >> 2][4 * (q & 3)], r[q >> 2][4 * (q & 3) + 1], r[q >> 2][4 * (q & 3) + 2],
                                        r[q >> 2][4 * (q & 3) + 3]);
                 } else {
-                    float bv[32];
-                    if (p.bias) {
-                        const uint4 *b4 = reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(p.bias) + col0 + c);
+                    // chunk q holds columns [8q, 8q + 8): + bias, one rounding to bf16
+                    const uint4 *b4 = p.bias ? reinterpret_cast<const uint4 *>(
+                                                   static_cast<const __nv_bfloat16 *>(p.bias) + col0 + c)
+                                             : nullptr;
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
+                    for (int q = 0; q < 8; ++q) {
+                        uint32_t ws[4] = {0u, 0u, 0u, 0u};
+                        if (b4) {
                             const uint4 w = __ldg(b4 + q);
-                            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                            for (int h = 0; h < 4; ++h) {
-                                bv[8 * q + 2 * h] = __uint_as_float(ws[h] << 16);
-                                bv[8 * q + 2 * h + 1] = __uint_as_float(ws[h] & 0xFFFF0000u);
-                            }
+                            ws[0] = w.x;
+                            ws[1] = w.y;
+                            ws[2] = w.z;
+                            ws[3] = w.w;
                         }
-                    } else {
+                        uint32_t pk[4];
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) bv[i] = 0.f;
+                        for (int i = 0; i < 4; ++i) {
+                            const float v0 = __uint_as_float(r[q >> 1][(q & 1) * 8 + 2 * i]) + __uint_as_float(ws[i] << 16);
+                            const float v1 = __uint_as_float(r[q >> 1][(q & 1) * 8 + 2 * i + 1]) +
+                                             __uint_as_float(ws[i] & 0xFFFF0000u);
+                            __nv_bfloat162 h = __floats2bfloat162_rn(v0, v1);
+                            pk[i] = *reinterpret_cast<uint32_t *>(&h);
+                        }
+                        *reinterpret_cast<uint4 *>(buf + lane * 128 + ((q ^ (lane & 7)) * 16)) =
+                            make_uint4(pk[0], pk[1], pk[2], pk[3]);
                     }
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const float v0 = __uint_as_float(r[(2 * i) >> 4][(2 * i) & 15]) + bv[2 * i];
-                        const float v1 = __uint_as_float(r[(2 * i + 1) >> 4][(2 * i + 1) & 15]) + bv[2 * i + 1];
-                        __nv_bfloat162 h = __floats2bfloat162_rn(v0, v1);
-                        pk[i] = *reinterpret_cast<uint32_t *>(&h);
-                    }
-                    // 64-byte swizzle: 16-byte chunk q of row r goes to chunk q ^ ((r >> 1) & 3)
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        *reinterpret_cast<uint4 *>(buf + lane * 64 + ((q ^ ((lane >> 1) & 3)) * 16)) =
-                            make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
@@ -345,7 +342,7 @@ __global__ void __launch_bounds__(kPThreads, 1) pw_kernel(const __grid_constant_
 
 size_t pw_smem_bytes(int nk, int BN, int stages, bool out_f32, int ybufs) {
     return 1024 /* alignment slack */ + kPHeader + static_cast<size_t>(nk) * (BN / 2) * kPPlane +
-           static_cast<size_t>(stages) * kPAStage + static_cast<size_t>(kPEpiWarps) * ybufs * pw_stage_buf(out_f32);
+           static_cast<size_t>(stages) * kPAStage + static_cast<size_t>(kPEpiWarps) * ybufs * kPStageBuf;
 }
 
 namespace {
