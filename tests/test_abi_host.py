@@ -165,7 +165,7 @@ def test_plan_for_the_workloads_on_a_148_sm_device(lib):
     """The kernel and tile choices the forward pass makes, pinned on the CPU."""
     p1 = _plan((64, 256, 56, 56, 1024, 1, 1, 1, 0, 1, 1), sms=148)   # 1x1: x is X_col, weights resident
     assert (p1["kernel"], p1["pair"], p1["a_load"], p1["BN"], p1["stages"], p1["tma_out"]) == \
-        ("pointwise", 1, "tiled_x", 256, 8, 1)
+        ("pointwise", 1, "tiled_x", 256, 6, 1)
     assert p1["units"] == (64 * 56 * 56 // 256) * 4 and p1["workspace"] == 0
     p3 = _plan((64, 256, 56, 56, 256, 3, 3, 1, 1, 1, 1), sms=148)    # 3x3: hardware im2col, pairs
     assert (p3["kernel"], p3["pair"], p3["a_load"], p3["BN"], p3["units"]) == ("igemm", 1, "im2col", 256, 784)
