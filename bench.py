@@ -783,8 +783,19 @@ def run_conv3d(args, cfg):
         achieved = nbytes / (kernel_ms * 1e-3) / 1e9
         rl = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
               "frac": achieved / peaks["hbm_gbs"], "peak_source": f"{peak_kind} HBM copy bandwidth"}
-    rl.update({"kernel": "igemm_kernel (5-D TMA im2col, tcgen05)", "kernel_ms": kernel_ms,
-               "algorithmic_flops_per_launch": f, "algorithmic_bytes_per_launch": nbytes, "traffic": None})
+    plan = cb.conv3d_describe_plan(cfg.N, cfg.C_in, cfg.D, cfg.H, cfg.W, cfg.C_out, cfg.Kd, cfg.Kh, cfg.Kw,
+                                   cfg.stride, cfg.pad, cfg.dilation, cfg.groups,
+                                   cb.CONV_BF16 if cfg.dtype == "bf16" else cb.CONV_F32, cfg.layout)
+    if plan["fold"]:
+        kname = ("igemm_kernel on the (kd, kh)-folded input (2-D TMA im2col of 1 x Kw, tcgen05); the fold and "
+                 "weight passes are outside kernel_ms, inside ms_per_step")
+    elif plan["kernel"] == "vol_reuse":
+        kname = "vol_reuse_kernel (5-D TMA im2col, each input slice loaded once for all depth taps, tcgen05)"
+    else:
+        kname = "igemm_kernel (5-D TMA im2col, tcgen05)"
+    rl.update({"kernel": kname, "kernel_ms": kernel_ms, "plan": plan,
+               "algorithmic_flops_per_launch": f, "algorithmic_bytes_per_launch": nbytes, "traffic": None,
+               "step_frac": (rl["achieved"] * kernel_ms / (elapsed / args.steps)) / rl["peak"]})
     desc = (f"{cfg.name}: N={cfg.N} C_in={cfg.C_in} {cfg.D}x{cfg.H}x{cfg.W} -> C_out={cfg.C_out}, "
             f"{cfg.Kd}x{cfg.Kh}x{cfg.Kw} s{cfg.stride} p{cfg.pad} d{cfg.dilation} g{cfg.groups}, {cfg.dtype}, "
             f"{'NDHWC' if cfg.layout == 'nhwc' else 'NCDHW'} in/out")

@@ -314,6 +314,9 @@ struct PadW {
     // when set: the product's fp32 results [split][M][C_out] go here (no bias, no
     // split reduction) for a later pass to finish -- the Winograd path's output transform
     float *partial_out = nullptr;
+    // x is channels-last with Cpg channels per group whatever `layout` says (which then
+    // names y's layout only) -- the folded 3-D input
+    bool x_nhwc = false;
 };
 
 // The depth of a 3-D convolution: input depth D and filter depth Kd (stride, padding and
@@ -522,7 +525,9 @@ int make_plan(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stri
             return CONV_OK;
         }
     }
-    p.xcopy = layout == CONV_NCHW || p.Cpg != p.Cin_g;
+    p.xcopy = (layout == CONV_NCHW && !(padw && padw->x_nhwc)) || p.Cpg != p.Cin_g;
+    if (p.xcopy && padw && padw->x_nhwc)
+        return fail(CONV_ERR_UNSUPPORTED, "channels-last input without its channel padding");
     // A 1x1 filter at stride 1 without padding makes the im2col matrix the
     // channels-last input itself (one row per pixel), so the tensor-core kernel reads
     // it with plain tiled loads, which stream far faster than im2col-mode loads.
@@ -1212,7 +1217,7 @@ int forward_impl(bool explicit_im2col, const void *x, const void *w_packed, cons
 int describe_impl(bool explicit_im2col, int N, int C_in, int H, int W, int C_out, int Kh, int Kw,
                   int stride, int pad, int dilation, int groups, conv_dtype_t dtype,
                   conv_layout_t layout, int sms, char *buf, size_t buflen, const Vol *vol = nullptr,
-                  const PadW *padw = nullptr) {
+                  const PadW *padw = nullptr, int fold = 0, size_t ws_extra = 0) {
     if (!buf || buflen == 0) return fail(CONV_ERR_INVALID_ARG, "buf must not be NULL");
     const Settings cfg = settings_now();
     Plan p;
@@ -1236,11 +1241,11 @@ int describe_impl(bool explicit_im2col, int N, int C_in, int H, int W, int C_out
         "{\"kernel\": \"%s\", \"pair\": %d, \"a_load\": \"%s\", \"BN\": %d, \"cb\": %d, "
         "\"stages\": %d, \"splits\": %d, \"units\": %d, \"xcopy\": %d, \"halo\": %d, "
         "\"tma_out\": %d, \"Kpad\": %d, \"smem\": %zu, \"workspace\": %zu, \"sms\": %d, "
-        "\"rows\": %d, \"out_images\": %d, \"a_tmem\": %d}",
+        "\"rows\": %d, \"out_images\": %d, \"a_tmem\": %d, \"fold\": %d}",
         kernel, p.pair ? 1 : 0, a_load, p.BN, p.gather ? 0 : p.cb,
         p.stages, p.gather ? 1 : p.splits, p.gather ? p.n_mtiles : p.units, p.xcopy ? 1 : 0,
-        p.halo ? 1 : 0, p.tma_out ? 1 : 0, p.gather ? p.Kpad : 0, p.smem, p.ws_total, sms,
-        p.gather_t ? p.rt : 0, p.gather_t && p.tma_out ? p.nout : 0, p.gather_t && p.a_tmem ? 1 : 0);
+        p.halo ? 1 : 0, p.tma_out ? 1 : 0, p.gather ? p.Kpad : 0, p.smem, p.ws_total + ws_extra, sms,
+        p.gather_t ? p.rt : 0, p.gather_t && p.tma_out ? p.nout : 0, p.gather_t && p.a_tmem ? 1 : 0, fold);
     if (n < 0 || static_cast<size_t>(n) >= buflen)
         return fail(CONV_ERR_INVALID_ARG, "buf of %zu bytes is too small (%d needed)", buflen, n + 1);
     return ok();
@@ -1575,6 +1580,75 @@ int backward_data_impl(const void *dy, const void *w_packed_t, void *dx, int N, 
 // F(m x m, 3 x 3), m = 2 or 4 (winograd.cu): input transform -> the tensor-core product
 // as a grouped 1x1 convolution with alpha^2 groups over the transformed tiles, fp32
 // results -> output transform.  Scratch: [V][M partial sums][the product's own scratch].
+// A few-channel 3-D layer at stride 1 as a 2-D one over its (kd, kh)-folded input
+// (layout.cu's fold3d): hardware im2col would move one narrow row (C_in channels, at most
+// 16 bytes) per voxel and tap, Kd*Kh*Kw of them; folded, each voxel row holds the Kd*Kh
+// taps' channels (Cf, padded to 64 bytes) and a 1 x Kw convolution over an image of
+// Do*Ho rows gives the same sums (the volume's im2col, pwwt §5, done in two steps).
+struct Fold3d {
+    int Cf, Do, Ho;
+    PadW pw;                       // columns padded by `pad`, x channels-last
+    size_t off_x, off_w, off_inner, ws_total;
+};
+
+bool fold3d_applies(int C_in, int Kd, int Kh, int stride, int groups, conv_dtype_t dtype) {
+    const int elt = dtype == CONV_F32 ? 4 : 2;
+    return groups == 1 && stride == 1 && C_in * elt <= 16 && Kd * Kh > 1;
+}
+
+int fold3d_plan(int N, int C_in, int D, int H, int W, int C_out, int Kd, int Kh, int Kw, int pad, int dilation,
+                conv_dtype_t dtype, conv_layout_t layout, DeviceInfo *dev, const Settings &cfg, Fold3d *f,
+                Plan *inner) {
+    const int elt = dtype == CONV_F32 ? 4 : 2;
+    if (out_size(D, Kd, 1, pad, dilation, &f->Do) != 0 || out_size(H, Kh, 1, pad, dilation, &f->Ho) != 0)
+        return fail(CONV_ERR_INVALID_ARG, "the dilated kernel is larger than the padded input");
+    f->Cf = round_up(Kd * Kh * C_in, 64 / elt);
+    f->pw = PadW{pad, nullptr, true};
+    if (static_cast<long long>(f->Do) * f->Ho >= (1LL << 31) / (W > 0 ? W : 1))
+        return fail(CONV_ERR_UNSUPPORTED, "folded volume too large");
+    int st = device_plan(false, N, f->Cf, f->Do * f->Ho, W, C_out, 1, Kw, 1, 0, dilation, 1, dtype, layout, dev,
+                         cfg, inner, &f->pw);
+    if (st != CONV_OK) return st;
+    f->off_x = 0;
+    size_t off = align_up(static_cast<size_t>(N) * f->Do * f->Ho * W * f->Cf * elt, 256);
+    f->off_w = off;
+    off = align_up(off + static_cast<size_t>(C_out) * Kw * f->Cf * elt, 256);
+    f->off_inner = off;
+    f->ws_total = off + inner->ws_total;
+    return CONV_OK;
+}
+
+int fold3d_forward(const void *x, const void *w_packed, const void *bias, void *y, int N, int C_in, int D, int H,
+                   int W, int C_out, int Kd, int Kh, int Kw, int pad, int dilation, conv_dtype_t dtype,
+                   conv_layout_t layout, void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+    const Settings cfg = settings_now();
+    Fold3d f;
+    Plan inner;
+    // argument errors first, then the device's plan
+    int st = fold3d_plan(N, C_in, D, H, W, C_out, Kd, Kh, Kw, pad, dilation, dtype, layout, nullptr, cfg, &f, &inner);
+    if (st != CONV_OK) return st;
+    DeviceInfo *dev = nullptr;
+    if ((st = device_info(&dev)) != CONV_OK) return st;
+    if ((st = fold3d_plan(N, C_in, D, H, W, C_out, Kd, Kh, Kw, pad, dilation, dtype, layout, dev, cfg, &f,
+                          &inner)) != CONV_OK)
+        return st;
+    if (!x || !w_packed || !y) return fail(CONV_ERR_INVALID_ARG, "x, w_packed and y must not be NULL");
+    if (!workspace || workspace_bytes < f.ws_total)
+        return fail(CONV_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", f.ws_total,
+                    workspace ? workspace_bytes : static_cast<size_t>(0));
+    if (!aligned16(x) || !aligned16(w_packed) || !aligned16(y) || (bias && !aligned16(bias)) || !aligned16(workspace))
+        return fail(CONV_ERR_UNSUPPORTED, "device pointers must be 16-byte aligned");
+    const int elt = elt_of(dtype);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    if ((st = check_launch(launch_fold3d(x, ws + f.off_x, w_packed, ws + f.off_w, N, C_in, D, H, W, f.Do, f.Ho, C_out,
+                                         Kd, Kh, Kw, round_up(C_in, 16 / elt), pad, dilation, f.Cf, elt,
+                                         layout == CONV_NCHW, stream),
+                           "depth-and-row fold")) != CONV_OK)
+        return st;
+    return forward_impl(false, ws + f.off_x, ws + f.off_w, bias, y, N, f.Cf, f.Do * f.Ho, W, C_out, 1, Kw, 1, 0,
+                        dilation, 1, dtype, layout, ws + f.off_inner, workspace_bytes - f.off_inner, stream, &f.pw);
+}
+
 struct WinoPlan {
     Plan f;          // the 3x3 problem: validation, Ho, Wo
     Plan g;          // the product
@@ -1878,6 +1952,16 @@ int conv2d_describe_plan(int N, int C_in, int H, int W, int C_out, int Kh, int K
 int conv3d_describe_plan(int N, int C_in, int D, int H, int W, int C_out, int Kd, int Kh, int Kw, int stride,
                          int pad, int dilation, int groups, conv_dtype_t dtype, conv_layout_t layout, int sms,
                          char *buf, size_t buflen) {
+    if (fold3d_applies(C_in, Kd, Kh, stride, groups, dtype)) {
+        // the 2-D plan of the folded problem, with the fold's buffers in its workspace
+        Plan inner;
+        Fold3d f;
+        int st = fold3d_plan(N, C_in, D, H, W, C_out, Kd, Kh, Kw, pad, dilation, dtype, layout, nullptr,
+                             settings_now(), &f, &inner);
+        if (st != CONV_OK) return st;
+        return describe_impl(false, N, f.Cf, f.Do * f.Ho, W, C_out, 1, Kw, 1, 0, dilation, 1, dtype, layout, sms, buf,
+                             buflen, nullptr, &f.pw, 1, f.off_inner);
+    }
     const Vol vol{D, Kd};
     return describe_impl(false, N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype, layout, sms, buf,
                          buflen, &vol);
@@ -2028,6 +2112,16 @@ int conv3d_pack_weight(const void *w_oidhw, void *w_packed, int C_out, int C_in,
 int conv3d_workspace_size(int N, int C_in, int D, int H, int W, int C_out, int Kd, int Kh, int Kw, int stride,
                           int pad, int dilation, int groups, conv_dtype_t dtype, conv_layout_t layout,
                           size_t *bytes) {
+    if (fold3d_applies(C_in, Kd, Kh, stride, groups, dtype)) {
+        if (!bytes) return fail(CONV_ERR_INVALID_ARG, "bytes must not be NULL");
+        Plan inner;
+        Fold3d f;
+        int st = fold3d_plan(N, C_in, D, H, W, C_out, Kd, Kh, Kw, pad, dilation, dtype, layout,
+                             current_device_or_null(), settings_now(), &f, &inner);
+        if (st != CONV_OK) return st;
+        *bytes = f.ws_total;
+        return ok();
+    }
     const Vol vol{D, Kd};
     return workspace_impl(false, N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype, layout, bytes,
                           nullptr, &vol);
@@ -2037,6 +2131,9 @@ int conv3d_forward(const void *x, const void *w_packed, const void *bias, void *
                    int W, int C_out, int Kd, int Kh, int Kw, int stride, int pad, int dilation, int groups,
                    conv_dtype_t dtype, conv_layout_t layout, void *workspace, size_t workspace_bytes,
                    conv_stream_t stream) {
+    if (fold3d_applies(C_in, Kd, Kh, stride, groups, dtype))
+        return fold3d_forward(x, w_packed, bias, y, N, C_in, D, H, W, C_out, Kd, Kh, Kw, pad, dilation, dtype, layout,
+                              workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
     const Vol vol{D, Kd};
     return forward_impl(false, x, w_packed, bias, y, N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups,
                         dtype, layout, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream), nullptr,

@@ -190,6 +190,12 @@ size_t igemm_smem_bytes(bool f32, int BN, int stages, bool tma_out);
 // Two-CTA clusters of the pair kernel that can be resident at once.
 cudaError_t igemm_pair_max_clusters(int cb_bytes, bool im2col, size_t smem_bytes, int *clusters, bool vol = false);
 cudaError_t launch_gather(const GatherParams &p, bool f32, int grid, size_t smem, cudaStream_t stream);
+// The (kd, kh)-fold of a few-channel 3-D input into xf [N][Do*Ho][W][Cf] (channels-last),
+// and of its packed weights wp [Cout][Kd*Kh*Kw][cpg] into the 2-D packed layout
+// wf [Cout][Kw][Cf], in one launch (layout.cu).
+cudaError_t launch_fold3d(const void *x, void *xf, const void *wp, void *wf, int N, int C, int D, int H, int W,
+                          int Do, int Ho, int Cout, int Kd, int Kh, int Kw, int cpg, int pad, int dilation, int Cf,
+                          int elt, bool nchw, cudaStream_t s);
 size_t gather_smem_bytes(bool f32, int BN, int Kpad, size_t halo_bytes, size_t out_stage_bytes);
 // The transposed few-channel kernel (gather_t.cu): bf16, NCHW in and out, one output row
 // per tile, output channels on the tensor-memory lanes.

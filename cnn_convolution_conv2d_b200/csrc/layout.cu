@@ -3,6 +3,7 @@
 //   * channels-last -> NCHW ("layout out", zskr §3.2 step 5);
 //   * weight packing OIHW -> (oc, kh, kw, c) with zero channel padding;
 //   * explicit im2col (the pages' X_col, one row per output pixel);
+//   * the depth-and-row fold of a few-channel 3-D input (partial im2col) and its weights;
 //   * the fp32 reduction of split partial sums, + bias, in the output layout.
 // All are plain coalesced CUDA-core kernels with grid-stride loops; none reads or
 // writes outside the extents passed in.
@@ -371,6 +372,79 @@ __global__ void im2col_kernel(const void *__restrict__ x, void *__restrict__ xco
     }
 }
 
+// --- depth-and-row fold of a few-channel 3-D input: the (kd, kh) part of the volume's
+// im2col moved into the channels, so that a 1 x Kw convolution over the folded image
+// gives the 3-D result (stride 1):
+//   xf[n][od*Ho + oh][w][(kd*Kh + kh)*C + c] = x[n][c][od - pad + kd*dil][oh - pad + kh*dil][w]
+// (0 outside the volume and for the channel padding up to Cf).  x is NCDHW, or NDHWC with
+// C channels per voxel.  One thread per folded voxel (neighbouring threads read
+// neighbouring w of each tap and channel); each block first tabulates, per folded channel,
+// its offset in x and its depth and row shifts.
+template <typename T>
+__global__ void fold3d_kernel(const T *__restrict__ x, T *__restrict__ xf, const T *__restrict__ wp,
+                              T *__restrict__ wf, int N, int C, int D, int H, int W, int Do, int Ho, int Cout, int Kd,
+                              int Kh, int Kw, int cpg, int pad, int dilation, int Cf, bool nchw) {
+    constexpr int kPer = 16 / sizeof(T);
+    extern __shared__ int4 tab[];  // per folded channel k < Kd*Kh*C: {offset in x, kd*dil, kh*dil, 0}
+    const int kc = Kd * Kh * C;
+    // the folded weights (a few thousand elements) ride along on the first threads:
+    // wf[oc][kw][(kd*Kh + kh)*C + c] = wp[oc][(kd*Kh + kh)*Kw + kw][c], zero past Kd*Kh*C
+    const long long wtotal = static_cast<long long>(Cout) * Kw * Cf;
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < wtotal;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const int k = static_cast<int>(i % Cf);
+        const long long r = i / Cf;
+        const int kw = static_cast<int>(r % Kw);
+        const int oc = static_cast<int>(r / Kw);
+        T e = T(0.f);
+        if (k < kc) {
+            const int t = k / C, c = k - (k / C) * C;
+            e = wp[(static_cast<long long>(oc) * Kd * Kh * Kw + static_cast<long long>(t) * Kw + kw) * cpg + c];
+        }
+        wf[i] = e;
+    }
+    const long long HW = static_cast<long long>(H) * W;
+    for (int k = threadIdx.x; k < kc; k += blockDim.x) {
+        const int t = k / C, c = k - (k / C) * C;
+        const int kd = t / Kh, kh = t - (t / Kh) * Kh;
+        const long long off = nchw ? (static_cast<long long>(c) * D + kd * dilation) * HW + static_cast<long long>(kh) * dilation * W
+                                   : (static_cast<long long>(kd) * dilation * HW + static_cast<long long>(kh) * dilation * W) * C + c;
+        tab[k] = make_int4(static_cast<int>(off), kd * dilation, kh * dilation, 0);
+    }
+    __syncthreads();
+    const long long total = static_cast<long long>(N) * Do * Ho * W;
+    for (long long vox = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; vox < total;
+         vox += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const int w = static_cast<int>(vox % W);
+        const long long r = vox / W;                   // n * (Do*Ho) + od*Ho + oh
+        const int oh = static_cast<int>(r % Ho);
+        const long long r2 = r / Ho;
+        const int od = static_cast<int>(r2 % Do);
+        const int n = static_cast<int>(r2 / Do);
+        const int d0 = od - pad, h0 = oh - pad;        // the window's first depth and row
+        // x offset of (n, c = 0, d0, h0, w), possibly outside x: only in-range taps read it
+        const long long base = nchw ? ((static_cast<long long>(n) * C * D + d0) * H + h0) * W + w
+                                    : (((static_cast<long long>(n) * D + d0) * H + h0) * W + w) * C;
+        uint4 *dst = reinterpret_cast<uint4 *>(xf + vox * Cf);
+        for (int k0 = 0; k0 < Cf; k0 += kPer) {
+            alignas(16) T v[kPer];
+#pragma unroll
+            for (int j = 0; j < kPer; ++j) {
+                const int k = k0 + j;
+                T e = T(0.f);
+                if (k < kc) {
+                    const int4 tk = tab[k];
+                    if (static_cast<unsigned>(d0 + tk.y) < static_cast<unsigned>(D) &&
+                        static_cast<unsigned>(h0 + tk.z) < static_cast<unsigned>(H))
+                        e = x[base + tk.x];
+                }
+                v[j] = e;
+            }
+            dst[k0 / kPer] = *reinterpret_cast<const uint4 *>(v);
+        }
+    }
+}
+
 // --- split reduction: y = bias + sum_s ws[s][m][oc], in the output layout.
 template <bool kF32>
 __global__ void splitk_reduce_kernel(const float *__restrict__ ws, const void *__restrict__ bias,
@@ -678,6 +752,28 @@ cudaError_t launch_im2col(const void *x_nhwc, void *xcol, int N, int H, int W, i
     else
         im2col_kernel<4><<<grid_for(chunks), kThreads, 0, s>>>(x_nhwc, xcol, N, H, W, groups, Cpg,
                                                               Ho, Wo, Kh, Kw, stride, pad, dilation);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_fold3d(const void *x, void *xf, const void *wp, void *wf, int N, int C, int D, int H, int W,
+                          int Do, int Ho, int Cout, int Kd, int Kh, int Kw, int cpg, int pad, int dilation, int Cf,
+                          int elt, bool nchw, cudaStream_t s) {
+    const int kc = Kd * Kh * C;
+    // the per-channel offsets are 32-bit: one image's C*D*H*W elements stay below 2^31
+    if (Cf % (16 / elt) != 0 || Cf < kc || kc > 4096 || cpg < C ||
+        static_cast<long long>(C) * D * H * W >= (1LL << 31))
+        return cudaErrorInvalidValue;
+    const long long voxels = static_cast<long long>(N) * Do * Ho * W;
+    const size_t tab = static_cast<size_t>(kc) * sizeof(int4);
+    if (elt == 2)
+        fold3d_kernel<__nv_bfloat16><<<grid_for(voxels), kThreads, tab, s>>>(
+            static_cast<const __nv_bfloat16 *>(x), static_cast<__nv_bfloat16 *>(xf),
+            static_cast<const __nv_bfloat16 *>(wp), static_cast<__nv_bfloat16 *>(wf), N, C, D, H, W, Do, Ho, Cout, Kd,
+            Kh, Kw, cpg, pad, dilation, Cf, nchw);
+    else
+        fold3d_kernel<float><<<grid_for(voxels), kThreads, tab, s>>>(
+            static_cast<const float *>(x), static_cast<float *>(xf), static_cast<const float *>(wp),
+            static_cast<float *>(wf), N, C, D, H, W, Do, Ho, Cout, Kd, Kh, Kw, cpg, pad, dilation, Cf, nchw);
     return cudaGetLastError();
 }
 

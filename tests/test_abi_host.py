@@ -288,11 +288,20 @@ def test_backward_rejects_bad_arguments(lib):
 
 def test_conv3d_sizes_and_limits_on_the_host(lib):
     assert cb.conv3d_packed_weight_size(16, 3, 3, 3, 3, 1, cb.CONV_BF16) == 16 * 27 * 8 * 2
-    # NCDHW input: the channels-last copy, 3 channels padded to 8
+    # three channels at stride 1: the (kd, kh)-folded input (27 channels padded to 32) and
+    # its 16 x 3 x 32 weights are the workspace; the 2-D product of the fold needs none
     assert cb.conv3d_workspace_size(4, 3, 16, 64, 64, 16, 3, 3, 3, 1, 1, 1, 1, cb.CONV_BF16, "nchw") == \
+        4 * 16 * 64 * 64 * 32 * 2 + 16 * 3 * 32 * 2
+    p = cb.conv3d_describe_plan(4, 3, 16, 64, 64, 16, 3, 3, 3, 1, 1, 1, 1, cb.CONV_BF16, "nchw", sms=148)
+    assert (p["fold"], p["kernel"], p["a_load"], p["cb"], p["BN"], p["units"]) == (1, "igemm", "im2col", 64, 16, 2048)
+    # stride 2 or 16 channels: no fold; NCDHW input then goes through the channels-last copy
+    p2 = cb.conv3d_describe_plan(4, 3, 16, 64, 64, 16, 3, 3, 3, 2, 1, 1, 1, cb.CONV_BF16, "nchw", sms=148)
+    assert (p2["fold"], p2["xcopy"]) == (0, 1)
+    assert cb.conv3d_workspace_size(4, 3, 16, 64, 64, 16, 3, 3, 3, 2, 1, 1, 1, cb.CONV_BF16, "nchw") == \
         4 * 16 * 64 * 64 * 8 * 2
+    assert cb.conv3d_describe_plan(4, 16, 16, 64, 64, 32, 3, 3, 3, 1, 1, 1, 1, cb.CONV_BF16, "nhwc", sms=148)["fold"] == 0
     # the 5-D im2col addressing range: pad 17 is out of it
-    st = lib.conv3d_forward(16, 16, None, 16, 1, 8, 40, 40, 40, 8, 3, 3, 3, 1, 17, 1, 1, cb.CONV_BF16,
+    st = lib.conv3d_forward(16, 16, None, 16, 1, 16, 40, 40, 40, 8, 3, 3, 3, 1, 17, 1, 1, cb.CONV_BF16,
                             cb.CONV_NHWC, None, 0, None)
     assert st == cb.CONV_ERR_UNSUPPORTED
     st = lib.conv3d_forward(16, 16, None, 16, 1, 8, 2, 8, 8, 8, 5, 3, 3, 1, 0, 1, 1, cb.CONV_BF16,

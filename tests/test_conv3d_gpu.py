@@ -52,7 +52,8 @@ def run_oracle3d(cfg, inp):
 EDGE3D = [  # N, C_in, D, H, W, C_out, Kd, Kh, Kw, stride, pad, dilation, groups
     (2, 16, 6, 9, 8, 32, 3, 3, 3, 1, 1, 1, 1),      # ragged last tile (864 voxels)
     (1, 64, 7, 10, 11, 48, 3, 3, 3, 2, 1, 1, 1),    # stride 2, 128-byte channel rows, C_out 48
-    (2, 3, 5, 12, 12, 8, 3, 3, 3, 1, 1, 1, 1),      # three input channels: padded channels-last copy
+    (2, 3, 5, 12, 12, 8, 3, 3, 3, 1, 1, 1, 1),      # three input channels: the (kd, kh)-folded 2-D form
+    (1, 3, 6, 10, 10, 16, 3, 3, 3, 2, 1, 1, 1),     # three input channels at stride 2: hardware im2col
     (1, 32, 8, 8, 8, 16, 2, 3, 5, 1, 2, 2, 1),      # non-cubic filter, dilation 2
     (1, 64, 4, 9, 9, 64, 1, 3, 3, 1, 1, 1, 4),      # (1, 3, 3) filter, groups of 16
     (2, 24, 9, 6, 7, 40, 3, 1, 3, 3, 2, 1, 1),      # stride 3, filter of height 1
@@ -68,6 +69,36 @@ def test_conv3d_edge_shapes(shape, layout, dtype):
     cfg = workloads.Conv3dConfig("edge3d", *shape, True, dtype, layout, seed=sum(shape))
     inp = workloads.make_inputs3d(cfg)
     parity.assert_close(cfg, run_gpu3d(cfg, inp), run_oracle3d(cfg, inp), str(shape))
+
+
+FOLDED = [  # few-channel inputs at stride 1: (kd, kh) folded into the channels, then a 1 x Kw product
+    ((2, 3, 7, 13, 11, 16, 3, 3, 3, 1, 1, 1, 1), "nchw", "bf16"),   # the first 3-D layer's form, ragged tiles
+    ((1, 3, 6, 9, 10, 16, 3, 3, 3, 1, 1, 1, 1), "nhwc", "f32"),     # fp32 (three tf32 products), channels-last
+    ((1, 1, 8, 9, 9, 8, 3, 5, 3, 1, 2, 2, 1), "nchw", "bf16"),      # one channel, non-cubic filter, dilation 2
+    ((2, 8, 5, 6, 7, 32, 2, 2, 3, 1, 0, 1, 1), "nhwc", "bf16"),     # eight channels (16-byte rows), no padding
+    ((1, 4, 5, 7, 8, 24, 3, 3, 1, 1, 1, 1, 1), "nchw", "f32"),      # Kw = 1: the folded product is 1x1
+    ((1, 2, 4, 8, 8, 16, 1, 3, 3, 1, 1, 1, 1), "nhwc", "bf16"),     # Kd = 1: only the rows fold
+]
+
+
+@pytest.mark.parametrize("shape,layout,dtype", FOLDED, ids=lambda s: "x".join(map(str, s)) if isinstance(s, tuple) else s)
+def test_conv3d_folded_few_channels(shape, layout, dtype):
+    plan = cb.conv3d_describe_plan(*shape, cb.CONV_BF16 if dtype == "bf16" else cb.CONV_F32, layout)
+    assert plan["fold"] == 1 and plan["xcopy"] == 0, plan
+    cfg = workloads.Conv3dConfig("fold", *shape, True, dtype, layout, seed=sum(shape) + 5)
+    inp = workloads.make_inputs3d(cfg)
+    parity.assert_close(cfg, run_gpu3d(cfg, inp), run_oracle3d(cfg, inp), str(shape) + " (folded)")
+
+
+def test_conv3d_folded_integers_bit_exact():
+    shape = (2, 3, 6, 10, 9, 16, 3, 3, 3, 1, 1, 1, 1)
+    assert cb.conv3d_describe_plan(*shape, cb.CONV_BF16, "nchw")["fold"] == 1
+    ints = ("integers", -2, 2)
+    cfg = workloads.Conv3dConfig("fold_ints", *shape, True, "bf16", "nchw", ints, ints, ints, seed=11)
+    inp = workloads.make_inputs3d(cfg)
+    ref = run_oracle3d(cfg, inp)
+    assert np.abs(ref).max() <= 256
+    assert np.array_equal(run_gpu3d(cfg, inp), ref)
 
 
 VOL_REUSE = [  # N, C_in, D, H, W, C_out, Kd, Kh, Kw, stride, pad, dilation, groups; bias
