@@ -5,6 +5,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <algorithm>
 #include <atomic>
 #include <map>
 #include <mutex>
@@ -47,11 +48,23 @@ constexpr int kMaxDevices = 64;
 constexpr size_t kSmemBudget = 227 * 1024;
 constexpr long long kDefaultTimeoutNs = 2000000000LL;
 
+constexpr int kHostioChunks = 16;  // most batch chunks one host-buffer call pipelines
+
+// Streams and events of the host-buffer entry point's copy pipeline, made on first use.
+struct HostioPipe {
+    std::mutex m;  // one call's enqueue at a time per device: the events below are shared
+    bool ready = false;
+    cudaStream_t in = nullptr, out = nullptr;  // host -> device, device -> host copies
+    cudaEvent_t start = nullptr, done = nullptr;
+    cudaEvent_t ev_in[kHostioChunks] = {}, ev_comp[kHostioChunks] = {};
+};
+
 struct DeviceInfo {
     bool ready = false;
     int sms = 0;
     int *status = nullptr;
     void *noalloc_scratch = nullptr;  // device address of g_noalloc_scratch
+    HostioPipe hio;
 };
 DeviceInfo g_devices[kMaxDevices];
 std::mutex g_mutex;
@@ -1860,16 +1873,91 @@ int conv2d_forward_hostio(const void *x_host, void *y_host, void *x_dev, void *y
     if (st != CONV_OK) return st;
     if (!x_host || !y_host || !x_dev || !y_dev)
         return fail(CONV_ERR_INVALID_ARG, "host and device activation buffers must not be NULL");
-    const size_t xb = static_cast<size_t>(N) * C_in * H * W * p.elt;
-    const size_t yb = static_cast<size_t>(p.M) * C_out * p.elt;
+    const size_t xi = static_cast<size_t>(C_in) * H * W * p.elt;             // bytes per image
+    const size_t yi = static_cast<size_t>(p.Ho) * p.Wo * C_out * p.elt;
+    const size_t xb = xi * N, yb = yi * N;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    cudaError_t e = cudaMemcpyAsync(x_dev, x_host, xb, cudaMemcpyHostToDevice, s);
-    if (e != cudaSuccess) return fail(CONV_ERR_CUDA, "input copy: %s", cudaGetErrorString(e));
-    st = forward_impl(false, x_dev, w_packed, bias, y_dev, N, C_in, H, W, C_out, Kh, Kw, stride,
-                      pad, dilation, groups, dtype, layout, workspace, workspace_bytes, s);
+    // Batch chunks of at least 8 MB of input, so that the input copy of one chunk, the
+    // product of the one before and the output copy of the one before that run at once
+    // (the two copy directions on their own engines).  Chunks start on 16-byte
+    // boundaries and must fit the caller's workspace; otherwise one chunk.
+    const Settings cfg = settings_now();
+    DeviceInfo *dev = nullptr;
+    if ((st = device_info(&dev)) != CONV_OK) return st;
+    int nch = static_cast<int>(std::min<size_t>(std::min<size_t>(xb / (8u << 20), kHostioChunks), N));
+    if (xi % 16 != 0 || yi % 16 != 0) nch = 1;
+    while (nch > 1) {
+        bool fits = true;
+        for (int nc : {N / nch, (N + nch - 1) / nch}) {
+            Plan q;
+            if (device_plan(false, nc, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups, dtype, layout, dev,
+                            cfg, &q) != CONV_OK ||
+                q.ws_total > (workspace ? workspace_bytes : 0))
+                fits = false;
+        }
+        if (fits) break;
+        nch /= 2;
+    }
+    if (nch <= 1) {
+        cudaError_t e = cudaMemcpyAsync(x_dev, x_host, xb, cudaMemcpyHostToDevice, s);
+        if (e != cudaSuccess) return fail(CONV_ERR_CUDA, "input copy: %s", cudaGetErrorString(e));
+        st = forward_impl(false, x_dev, w_packed, bias, y_dev, N, C_in, H, W, C_out, Kh, Kw, stride,
+                          pad, dilation, groups, dtype, layout, workspace, workspace_bytes, s);
+        if (st != CONV_OK) return st;
+        e = cudaMemcpyAsync(y_host, y_dev, yb, cudaMemcpyDeviceToHost, s);
+        if (e != cudaSuccess) return fail(CONV_ERR_CUDA, "output copy: %s", cudaGetErrorString(e));
+        return ok();
+    }
+    HostioPipe &hp = dev->hio;
+    std::lock_guard<std::mutex> pipe_lock(hp.m);
+    {
+        if (!hp.ready) {
+            cudaError_t e = cudaStreamCreateWithFlags(&hp.in, cudaStreamNonBlocking);
+            if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&hp.out, cudaStreamNonBlocking);
+            if (e == cudaSuccess) e = cudaEventCreateWithFlags(&hp.start, cudaEventDisableTiming);
+            if (e == cudaSuccess) e = cudaEventCreateWithFlags(&hp.done, cudaEventDisableTiming);
+            for (int i = 0; e == cudaSuccess && i < kHostioChunks; ++i) {
+                e = cudaEventCreateWithFlags(&hp.ev_in[i], cudaEventDisableTiming);
+                if (e == cudaSuccess) e = cudaEventCreateWithFlags(&hp.ev_comp[i], cudaEventDisableTiming);
+            }
+            if (e != cudaSuccess) return fail(CONV_ERR_CUDA, "copy pipeline streams: %s", cudaGetErrorString(e));
+            hp.ready = true;
+        }
+    }
+    // fork: both copy streams start after the work already on the caller's stream
+    cudaError_t e = cudaEventRecord(hp.start, s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(hp.in, hp.start, 0);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(hp.out, hp.start, 0);
+    if (e != cudaSuccess) return fail(CONV_ERR_CUDA, "copy pipeline fork: %s", cudaGetErrorString(e));
+    const uint8_t *xh = static_cast<const uint8_t *>(x_host);
+    uint8_t *yh = static_cast<uint8_t *>(y_host);
+    uint8_t *xd = static_cast<uint8_t *>(x_dev);
+    uint8_t *yd = static_cast<uint8_t *>(y_dev);
+    int n0 = 0;
+    for (int c = 0; c < nch && st == CONV_OK && e == cudaSuccess; ++c) {
+        const int nc = N / nch + (c < N % nch ? 1 : 0);
+        const size_t xo = static_cast<size_t>(n0) * xi, yo = static_cast<size_t>(n0) * yi;
+        e = cudaMemcpyAsync(xd + xo, xh + xo, nc * xi, cudaMemcpyHostToDevice, hp.in);
+        if (e == cudaSuccess) e = cudaEventRecord(hp.ev_in[c], hp.in);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(s, hp.ev_in[c], 0);
+        if (e != cudaSuccess) break;
+        st = forward_impl(false, xd + xo, w_packed, bias, yd + yo, nc, C_in, H, W, C_out, Kh, Kw, stride, pad,
+                          dilation, groups, dtype, layout, workspace, workspace_bytes, s);
+        if (st != CONV_OK) break;
+        e = cudaEventRecord(hp.ev_comp[c], s);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(hp.out, hp.ev_comp[c], 0);
+        if (e == cudaSuccess) e = cudaMemcpyAsync(yh + yo, yd + yo, nc * yi, cudaMemcpyDeviceToHost, hp.out);
+        n0 += nc;
+    }
+    // join: the caller's stream continues after the last output copy (also on failure,
+    // so that no copy stream is left behind a capture or ahead of later work)
+    cudaError_t ej = cudaEventRecord(hp.done, hp.out);
+    if (ej == cudaSuccess) ej = cudaStreamWaitEvent(s, hp.done, 0);
+    if (ej == cudaSuccess) ej = cudaEventRecord(hp.done, hp.in);
+    if (ej == cudaSuccess) ej = cudaStreamWaitEvent(s, hp.done, 0);
     if (st != CONV_OK) return st;
-    e = cudaMemcpyAsync(y_host, y_dev, yb, cudaMemcpyDeviceToHost, s);
-    if (e != cudaSuccess) return fail(CONV_ERR_CUDA, "output copy: %s", cudaGetErrorString(e));
+    if (e != cudaSuccess) return fail(CONV_ERR_CUDA, "pipelined copies: %s", cudaGetErrorString(e));
+    if (ej != cudaSuccess) return fail(CONV_ERR_CUDA, "copy pipeline join: %s", cudaGetErrorString(ej));
     return ok();
 }
 

@@ -151,13 +151,18 @@ int conv2d_forward_im2col_gemm(const void *x, const void *w_packed, const void *
                                void *workspace, size_t workspace_bytes,
                                conv_stream_t stream);
 
-/* End-to-end call for host-resident activations: enqueues on `stream` the copy
- * of x_host into x_dev, conv2d_forward(x_dev, ...) into y_dev, and the copy of
- * y_dev back into y_host.  x_host/y_host are host buffers of the x and y sizes
- * (pinned for asynchronous copies); x_dev/y_dev are caller-owned device buffers
- * of the same sizes.  Weights and bias stay resident on the device.  Returns
- * after enqueuing; y_host is valid once the stream is synchronised.  Errors as
- * conv2d_forward. */
+/* End-to-end call for host-resident activations: enqueues the copy of x_host into
+ * x_dev, conv2d_forward(x_dev, ...) into y_dev, and the copy of y_dev back into
+ * y_host, ordered after the work already on `stream` and before the work enqueued on it
+ * later.  x_host/y_host are host buffers of the x and y sizes (pinned for asynchronous
+ * copies); x_dev/y_dev are caller-owned device buffers of the same sizes.  Weights and
+ * bias stay resident on the device.  With at least 16 MB of input (and images of whole
+ * 16-byte multiples) the batch is cut into up to 16 chunks of >= 8 MB along N, each
+ * chunk's input copy, product and output copy chained through two internal copy streams
+ * of the device, so that the two copy directions and the products overlap (only chunk
+ * sizes whose plans fit workspace_bytes are used; otherwise one chunk).  The products run
+ * on `stream`.  Returns after enqueuing; y_host is valid once the stream is
+ * synchronised.  Errors as conv2d_forward. */
 int conv2d_forward_hostio(const void *x_host, void *y_host, void *x_dev, void *y_dev,
                           const void *w_packed, const void *bias,
                           int N, int C_in, int H, int W, int C_out, int Kh, int Kw,

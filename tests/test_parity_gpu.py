@@ -233,6 +233,36 @@ def test_hostio_matches_device_call():
     assert torch.equal(y_host, y_dev_ref.cpu())
 
 
+
+@pytest.mark.parametrize("shape,layout", [
+    ((35, 64, 64, 64, 64, 3, 3, 1, 1, 1, 1), "nhwc"),     # 18.4 MB of input: two chunks of 18 and 17 images
+    ((100, 64, 48, 48, 32, 3, 3, 2, 1, 1, 1), "nchw"),    # 29.5 MB, NCHW, stride 2: three chunks (34, 33, 33)
+])
+def test_hostio_pipelined_chunks_bit_exact(shape, layout):
+    """The host-buffer call cuts large batches into chunks whose copies and products
+    overlap; with integer inputs every order of summation is exact, so the result equals
+    the oracle's whatever the chunks' plans."""
+    import torch
+    N, C_in, H, W, C_out, Kh, Kw, s_, p_, d_, g_ = shape
+    ints = ("integers", -2, 2)
+    cfg = workloads.ConvConfig("hostio", *shape, True, "bf16", layout, ints, ints, ints, seed=23)
+    inp = workloads.make_inputs(cfg)
+    layer = parity.make_layer(cfg, inp)
+    x_dev = parity.to_device_x(cfg, inp["x"])
+    y_dev = layer(x_dev)
+    x_host = x_dev.cpu().pin_memory()
+    y_host = torch.empty(y_dev.shape, dtype=y_dev.dtype).pin_memory()
+    x2 = torch.empty_like(x_dev)
+    y2 = torch.full_like(y_dev, float("nan"))
+    layer.forward_hostio(x_host, y_host, x2, y2)
+    cb.conv2d_sync_status()
+    ref = parity.run_oracle(cfg, inp)
+    assert np.abs(ref).max() <= 256
+    got = y_host.float().numpy().astype(np.float64)
+    if layout == "nhwc":
+        got = got.transpose(0, 3, 1, 2)
+    assert np.array_equal(got, ref)
+
 def test_repeated_calls_are_identical():
     import torch
     cfg = parity.config("k7_17x17_bf16", N=1, C_in=128, C_out=128)
