@@ -147,6 +147,7 @@ int device_info(DeviceInfo **out) {
 
 // ------------------------------------------------------------------- plan ---
 struct Plan {
+    int stride_w;   // column stride (the row stride is `stride`)
     int N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups;
     int pad_w;      // column padding (= pad, the row padding, for every caller-facing entry)
     bool vol;       // 3-D convolution: input depth D, filter depth Kd, output depth Do
@@ -330,6 +331,9 @@ struct PadW {
     // x is channels-last with Cpg channels per group whatever `layout` says (which then
     // names y's layout only) -- the folded 3-D input
     bool x_nhwc = false;
+    // > 0: the column stride, `stride` then being the row stride (the folded 3-D input,
+    // whose rows are already strided)
+    int stride_w = 0;
 };
 
 // The depth of a 3-D convolution: input depth D and filter depth Kd (stride, padding and
@@ -361,6 +365,7 @@ int make_plan(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stri
     Plan p{};
     p.N = N; p.C_in = C_in; p.H = H; p.W = W; p.C_out = C_out; p.Kh = Kh; p.Kw = Kw;
     p.stride = stride; p.pad = pad; p.pad_w = pad_w; p.dilation = dilation; p.groups = groups;
+    p.stride_w = (padw && padw->stride_w > 0) ? padw->stride_w : stride;
     p.vol = vol != nullptr;
     p.D = vol ? vol->D : 1;
     p.Kd = vol ? vol->Kd : 1;
@@ -372,12 +377,14 @@ int make_plan(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stri
     p.f32 = dtype == CONV_F32;
     p.elt = p.f32 ? 4 : 2;
     p.layout = layout;
-    if (out_size(H, Kh, stride, pad, dilation, &p.Ho) || out_size(W, Kw, stride, pad_w, dilation, &p.Wo))
+    if (out_size(H, Kh, stride, pad, dilation, &p.Ho) || out_size(W, Kw, p.stride_w, pad_w, dilation, &p.Wo))
         return fail(CONV_ERR_INVALID_ARG, "empty output: the dilated kernel is larger than the padded input");
     p.M = static_cast<long long>(N) * p.Do * p.Ho * p.Wo;
     // Limits of the hardware im2col addressing (traversal stride <= 8, bounding-box
     // corners in [-128, 127] for a 4-D tensor) and of 32-bit indexing.
-    if (stride > 8) return fail(CONV_ERR_UNSUPPORTED, "stride %d > 8", stride);
+    if (stride > 8 || p.stride_w > 8) return fail(CONV_ERR_UNSUPPORTED, "stride %d > 8", std::max(stride, p.stride_w));
+    if (p.stride_w != stride && (vol || explicit_im2col))
+        return fail(CONV_ERR_UNSUPPORTED, "a separate column stride needs the 2-D implicit form");
     if (pad > 127 || pad_w > 127 || pad < -127 || pad_w < -127)
         return fail(CONV_ERR_UNSUPPORTED, "pad %d > 127", pad > pad_w ? pad : pad_w);
     const long long up_h = pad - static_cast<long long>(Kh - 1) * dilation;
@@ -544,7 +551,8 @@ int make_plan(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stri
     // A 1x1 filter at stride 1 without padding makes the im2col matrix the
     // channels-last input itself (one row per pixel), so the tensor-core kernel reads
     // it with plain tiled loads, which stream far faster than im2col-mode loads.
-    p.direct_a = !explicit_im2col && p.Kd == 1 && Kh == 1 && Kw == 1 && stride == 1 && pad == 0 && pad_w == 0;
+    p.direct_a = !explicit_im2col && p.Kd == 1 && Kh == 1 && Kw == 1 && stride == 1 && p.stride_w == 1 && pad == 0 &&
+                 pad_w == 0;
     const int row_bytes = p.Cpg * p.elt;
     p.cb = row_bytes % 128 == 0 ? 128 : row_bytes % 64 == 0 ? 64 : row_bytes % 32 == 0 ? 32 : 16;
     const int cap = p.f32 ? 128 : 256;
@@ -684,7 +692,7 @@ int encode_a_im2col(const Plan &p, const void *x_nhwc, CUtensorMap *map) {
     cuuint64_t strides[3] = {ctot * p.elt, ctot * p.elt * p.W, ctot * p.elt * p.W * p.H};
     int lower[2] = {-p.pad_w, -p.pad};  // (w, h)
     int upper[2] = {p.pad_w - (p.Kw - 1) * p.dilation, p.pad - (p.Kh - 1) * p.dilation};
-    cuuint32_t estr[4] = {1, static_cast<cuuint32_t>(p.stride), static_cast<cuuint32_t>(p.stride), 1};
+    cuuint32_t estr[4] = {1, static_cast<cuuint32_t>(p.stride_w), static_cast<cuuint32_t>(p.stride), 1};
     CUresult r = g_encode_im2col(map, tma_type(p), 4, const_cast<void *>(x_nhwc), dims, strides, lower,
                                  upper, static_cast<cuuint32_t>(p.cb / p.elt), 128, estr,
                                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_for(p.cb),
@@ -1142,6 +1150,7 @@ int forward_impl(bool explicit_im2col, const void *x, const void *w_packed, cons
     kp.Kh = Kh;
     kp.Wo = p.Wo;
     kp.stride = stride;
+    kp.stride_w = p.stride_w;
     kp.pad = p.pad;
     kp.pad_w = p.pad_w;
     kp.dilation = dilation;
@@ -1589,34 +1598,33 @@ int backward_data_impl(const void *dy, const void *w_packed_t, void *dx, int N, 
                         workspace_bytes > d.zbytes ? workspace_bytes - d.zbytes : 0, stream, &pw);
 }
 
-// ------------------------------------------------------------------ Winograd ---
-// F(m x m, 3 x 3), m = 2 or 4 (winograd.cu): input transform -> the tensor-core product
-// as a grouped 1x1 convolution with alpha^2 groups over the transformed tiles, fp32
-// results -> output transform.  Scratch: [V][M partial sums][the product's own scratch].
-// A few-channel 3-D layer at stride 1 as a 2-D one over its (kd, kh)-folded input
-// (layout.cu's fold3d): hardware im2col would move one narrow row (C_in channels, at most
-// 16 bytes) per voxel and tap, Kd*Kh*Kw of them; folded, each voxel row holds the Kd*Kh
-// taps' channels (Cf, padded to 64 bytes) and a 1 x Kw convolution over an image of
-// Do*Ho rows gives the same sums (the volume's im2col, pwwt §5, done in two steps).
+// A few-channel 3-D layer as a 2-D one over its (kd, kh)-folded input (layout.cu's
+// fold3d): hardware im2col would move one narrow row (C_in channels, at most 16 bytes) per
+// voxel and tap, Kd*Kh*Kw of them; folded, each voxel row holds the Kd*Kh taps' channels
+// (Cf, padded to 64 bytes) and a 1 x Kw convolution with column stride s over an image of
+// Do*Ho rows gives the same sums (the volume's im2col, pwwt §5, done in two steps; the
+// depth and row strides are taken by the fold).
 struct Fold3d {
     int Cf, Do, Ho;
-    PadW pw;                       // columns padded by `pad`, x channels-last
+    PadW pw;                       // columns padded by `pad` and strided by s, x channels-last
     size_t off_x, off_w, off_inner, ws_total;
 };
 
 bool fold3d_applies(int C_in, int Kd, int Kh, int stride, int groups, conv_dtype_t dtype) {
     const int elt = dtype == CONV_F32 ? 4 : 2;
-    return groups == 1 && stride == 1 && C_in * elt <= 16 && Kd * Kh > 1;
+    // (at 32 bytes per voxel -- the stride-2 layer of 16 channels -- the fold's writes cost
+    // more than the rows it saves: 32.6 against 22.6 us per step, so only narrower rows fold)
+    return groups == 1 && stride <= 8 && C_in * elt <= 16 && Kd * Kh > 1;
 }
 
-int fold3d_plan(int N, int C_in, int D, int H, int W, int C_out, int Kd, int Kh, int Kw, int pad, int dilation,
-                conv_dtype_t dtype, conv_layout_t layout, DeviceInfo *dev, const Settings &cfg, Fold3d *f,
-                Plan *inner) {
+int fold3d_plan(int N, int C_in, int D, int H, int W, int C_out, int Kd, int Kh, int Kw, int stride, int pad,
+                int dilation, conv_dtype_t dtype, conv_layout_t layout, DeviceInfo *dev, const Settings &cfg,
+                Fold3d *f, Plan *inner) {
     const int elt = dtype == CONV_F32 ? 4 : 2;
-    if (out_size(D, Kd, 1, pad, dilation, &f->Do) != 0 || out_size(H, Kh, 1, pad, dilation, &f->Ho) != 0)
+    if (out_size(D, Kd, stride, pad, dilation, &f->Do) != 0 || out_size(H, Kh, stride, pad, dilation, &f->Ho) != 0)
         return fail(CONV_ERR_INVALID_ARG, "the dilated kernel is larger than the padded input");
     f->Cf = round_up(Kd * Kh * C_in, 64 / elt);
-    f->pw = PadW{pad, nullptr, true};
+    f->pw = PadW{pad, nullptr, true, stride};
     if (static_cast<long long>(f->Do) * f->Ho >= (1LL << 31) / (W > 0 ? W : 1))
         return fail(CONV_ERR_UNSUPPORTED, "folded volume too large");
     int st = device_plan(false, N, f->Cf, f->Do * f->Ho, W, C_out, 1, Kw, 1, 0, dilation, 1, dtype, layout, dev,
@@ -1632,17 +1640,18 @@ int fold3d_plan(int N, int C_in, int D, int H, int W, int C_out, int Kd, int Kh,
 }
 
 int fold3d_forward(const void *x, const void *w_packed, const void *bias, void *y, int N, int C_in, int D, int H,
-                   int W, int C_out, int Kd, int Kh, int Kw, int pad, int dilation, conv_dtype_t dtype,
+                   int W, int C_out, int Kd, int Kh, int Kw, int stride, int pad, int dilation, conv_dtype_t dtype,
                    conv_layout_t layout, void *workspace, size_t workspace_bytes, cudaStream_t stream) {
     const Settings cfg = settings_now();
     Fold3d f;
     Plan inner;
     // argument errors first, then the device's plan
-    int st = fold3d_plan(N, C_in, D, H, W, C_out, Kd, Kh, Kw, pad, dilation, dtype, layout, nullptr, cfg, &f, &inner);
+    int st = fold3d_plan(N, C_in, D, H, W, C_out, Kd, Kh, Kw, stride, pad, dilation, dtype, layout, nullptr, cfg, &f,
+                         &inner);
     if (st != CONV_OK) return st;
     DeviceInfo *dev = nullptr;
     if ((st = device_info(&dev)) != CONV_OK) return st;
-    if ((st = fold3d_plan(N, C_in, D, H, W, C_out, Kd, Kh, Kw, pad, dilation, dtype, layout, dev, cfg, &f,
+    if ((st = fold3d_plan(N, C_in, D, H, W, C_out, Kd, Kh, Kw, stride, pad, dilation, dtype, layout, dev, cfg, &f,
                           &inner)) != CONV_OK)
         return st;
     if (!x || !w_packed || !y) return fail(CONV_ERR_INVALID_ARG, "x, w_packed and y must not be NULL");
@@ -1654,7 +1663,7 @@ int fold3d_forward(const void *x, const void *w_packed, const void *bias, void *
     const int elt = elt_of(dtype);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     if ((st = check_launch(launch_fold3d(x, ws + f.off_x, w_packed, ws + f.off_w, N, C_in, D, H, W, f.Do, f.Ho, C_out,
-                                         Kd, Kh, Kw, round_up(C_in, 16 / elt), pad, dilation, f.Cf, elt,
+                                         Kd, Kh, Kw, round_up(C_in, 16 / elt), stride, pad, dilation, f.Cf, elt,
                                          layout == CONV_NCHW, stream),
                            "depth-and-row fold")) != CONV_OK)
         return st;
@@ -1662,6 +1671,10 @@ int fold3d_forward(const void *x, const void *w_packed, const void *bias, void *
                         dilation, 1, dtype, layout, ws + f.off_inner, workspace_bytes - f.off_inner, stream, &f.pw);
 }
 
+// ------------------------------------------------------------------ Winograd ---
+// F(m x m, 3 x 3), m = 2 or 4 (winograd.cu): input transform -> the tensor-core product
+// as a grouped 1x1 convolution with alpha^2 groups over the transformed tiles, fp32
+// results -> output transform.  Scratch: [V][M partial sums][the product's own scratch].
 struct WinoPlan {
     Plan f;          // the 3x3 problem: validation, Ho, Wo
     Plan g;          // the product
@@ -2044,7 +2057,7 @@ int conv3d_describe_plan(int N, int C_in, int D, int H, int W, int C_out, int Kd
         // the 2-D plan of the folded problem, with the fold's buffers in its workspace
         Plan inner;
         Fold3d f;
-        int st = fold3d_plan(N, C_in, D, H, W, C_out, Kd, Kh, Kw, pad, dilation, dtype, layout, nullptr,
+        int st = fold3d_plan(N, C_in, D, H, W, C_out, Kd, Kh, Kw, stride, pad, dilation, dtype, layout, nullptr,
                              settings_now(), &f, &inner);
         if (st != CONV_OK) return st;
         return describe_impl(false, N, f.Cf, f.Do * f.Ho, W, C_out, 1, Kw, 1, 0, dilation, 1, dtype, layout, sms, buf,
@@ -2204,7 +2217,7 @@ int conv3d_workspace_size(int N, int C_in, int D, int H, int W, int C_out, int K
         if (!bytes) return fail(CONV_ERR_INVALID_ARG, "bytes must not be NULL");
         Plan inner;
         Fold3d f;
-        int st = fold3d_plan(N, C_in, D, H, W, C_out, Kd, Kh, Kw, pad, dilation, dtype, layout,
+        int st = fold3d_plan(N, C_in, D, H, W, C_out, Kd, Kh, Kw, stride, pad, dilation, dtype, layout,
                              current_device_or_null(), settings_now(), &f, &inner);
         if (st != CONV_OK) return st;
         *bytes = f.ws_total;
@@ -2220,8 +2233,8 @@ int conv3d_forward(const void *x, const void *w_packed, const void *bias, void *
                    conv_dtype_t dtype, conv_layout_t layout, void *workspace, size_t workspace_bytes,
                    conv_stream_t stream) {
     if (fold3d_applies(C_in, Kd, Kh, stride, groups, dtype))
-        return fold3d_forward(x, w_packed, bias, y, N, C_in, D, H, W, C_out, Kd, Kh, Kw, pad, dilation, dtype, layout,
-                              workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+        return fold3d_forward(x, w_packed, bias, y, N, C_in, D, H, W, C_out, Kd, Kh, Kw, stride, pad, dilation, dtype,
+                              layout, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
     const Vol vol{D, Kd};
     return forward_impl(false, x, w_packed, bias, y, N, C_in, H, W, C_out, Kh, Kw, stride, pad, dilation, groups,
                         dtype, layout, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream), nullptr,

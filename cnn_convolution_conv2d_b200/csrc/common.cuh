@@ -37,7 +37,8 @@ struct IgemmParams {
     int M;               // N * Ho * Wo (volumes: N * Do * Ho * Wo)
     int HoWo, Wo;        // HoWo: output pixels per image (volumes: Do * Ho * Wo)
     int HoWo2, Kh;       // volumes: Ho * Wo per output depth slice, and the filter height
-    int stride, pad, dilation;
+    int stride, pad, dilation;  // stride: rows (and depth); columns: stride_w
+    int stride_w;
     int pad_w;           // column padding (pad: row padding)
     int Kw, taps;        // taps = Kh * Kw
     int Cpg;             // padded input channels per group (elements)
@@ -194,8 +195,8 @@ cudaError_t launch_gather(const GatherParams &p, bool f32, int grid, size_t smem
 // and of its packed weights wp [Cout][Kd*Kh*Kw][cpg] into the 2-D packed layout
 // wf [Cout][Kw][Cf], in one launch (layout.cu).
 cudaError_t launch_fold3d(const void *x, void *xf, const void *wp, void *wf, int N, int C, int D, int H, int W,
-                          int Do, int Ho, int Cout, int Kd, int Kh, int Kw, int cpg, int pad, int dilation, int Cf,
-                          int elt, bool nchw, cudaStream_t s);
+                          int Do, int Ho, int Cout, int Kd, int Kh, int Kw, int cpg, int stride, int pad, int dilation,
+                          int Cf, int elt, bool nchw, cudaStream_t s);
 size_t gather_smem_bytes(bool f32, int BN, int Kpad, size_t halo_bytes, size_t out_stage_bytes);
 // The transposed few-channel kernel (gather_t.cu): bf16, NCHW in and out, one output row
 // per tile, output channels on the tensor-memory lanes.

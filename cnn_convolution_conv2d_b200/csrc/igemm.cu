@@ -312,7 +312,7 @@ __global__ void __launch_bounds__(threads_for<kF32>(), 1)
                     const int oh = rem / p.Wo;
                     const int ow = rem - oh * p.Wo;
                     h0 = oh * p.stride - p.pad;
-                    w0 = ow * p.stride - p.pad_w;
+                    w0 = ow * p.stride_w - p.pad_w;
                 }
                 // Filter tap (kh, kw) and channel block of the next plane, stepped
                 // along instead of divided out per plane; past the last plane (the

@@ -373,9 +373,9 @@ __global__ void im2col_kernel(const void *__restrict__ x, void *__restrict__ xco
 }
 
 // --- depth-and-row fold of a few-channel 3-D input: the (kd, kh) part of the volume's
-// im2col moved into the channels, so that a 1 x Kw convolution over the folded image
-// gives the 3-D result (stride 1):
-//   xf[n][od*Ho + oh][w][(kd*Kh + kh)*C + c] = x[n][c][od - pad + kd*dil][oh - pad + kh*dil][w]
+// im2col moved into the channels, so that a 1 x Kw convolution with column stride s over
+// the folded image gives the 3-D result:
+//   xf[n][od*Ho + oh][w][(kd*Kh + kh)*C + c] = x[n][c][od*s - pad + kd*dil][oh*s - pad + kh*dil][w]
 // (0 outside the volume and for the channel padding up to Cf).  x is NCDHW, or NDHWC with
 // C channels per voxel.  One thread per folded voxel (neighbouring threads read
 // neighbouring w of each tap and channel); each block first tabulates, per folded channel,
@@ -383,7 +383,7 @@ __global__ void im2col_kernel(const void *__restrict__ x, void *__restrict__ xco
 template <typename T>
 __global__ void fold3d_kernel(const T *__restrict__ x, T *__restrict__ xf, const T *__restrict__ wp,
                               T *__restrict__ wf, int N, int C, int D, int H, int W, int Do, int Ho, int Cout, int Kd,
-                              int Kh, int Kw, int cpg, int pad, int dilation, int Cf, bool nchw) {
+                              int Kh, int Kw, int cpg, int stride, int pad, int dilation, int Cf, bool nchw) {
     constexpr int kPer = 16 / sizeof(T);
     extern __shared__ int4 tab[];  // per folded channel k < Kd*Kh*C: {offset in x, kd*dil, kh*dil, 0}
     const int kc = Kd * Kh * C;
@@ -412,6 +412,35 @@ __global__ void fold3d_kernel(const T *__restrict__ x, T *__restrict__ xf, const
         tab[k] = make_int4(static_cast<int>(off), kd * dilation, kh * dilation, 0);
     }
     __syncthreads();
+    if (!nchw && (C * static_cast<int>(sizeof(T))) % 16 == 0) {
+        // channels-last, whole 16-byte pieces per voxel: one thread per (voxel, tap slot)
+        // copies the slot's C channels as 16-byte vectors (slots past Kd*Kh are the zero
+        // channel padding; Cf is a multiple of C here)
+        // 32-bit indices: the host keeps voxels x slots below 2^31
+        const unsigned slots = static_cast<unsigned>(Cf / C), q = C * static_cast<unsigned>(sizeof(T)) / 16;
+        const unsigned total = static_cast<unsigned>(N * Do * Ho * W) * slots;
+        for (unsigned i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
+            const unsigned vox = i / slots;
+            const int slot = static_cast<int>(i - vox * slots);
+            const unsigned r = vox / static_cast<unsigned>(W);
+            const int w = static_cast<int>(vox - r * static_cast<unsigned>(W));
+            const unsigned r2 = r / static_cast<unsigned>(Ho);
+            const int oh = static_cast<int>(r - r2 * static_cast<unsigned>(Ho));
+            const int n = static_cast<int>(r2 / static_cast<unsigned>(Do));
+            const int od = static_cast<int>(r2 - static_cast<unsigned>(n) * static_cast<unsigned>(Do));
+            uint4 *dst = reinterpret_cast<uint4 *>(xf + static_cast<size_t>(vox) * Cf + static_cast<size_t>(slot) * C);
+            const int kd = slot / Kh, kh = slot - (slot / Kh) * Kh;
+            const int id = od * stride - pad + kd * dilation, ih = oh * stride - pad + kh * dilation;
+            if (slot < Kd * Kh && id >= 0 && id < D && ih >= 0 && ih < H) {
+                const uint4 *src = reinterpret_cast<const uint4 *>(
+                    x + (((static_cast<long long>(n) * D + id) * H + ih) * W + w) * C);
+                for (unsigned j = 0; j < q; ++j) dst[j] = __ldg(src + j);
+            } else {
+                for (unsigned j = 0; j < q; ++j) dst[j] = make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
+        return;
+    }
     const long long total = static_cast<long long>(N) * Do * Ho * W;
     for (long long vox = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; vox < total;
          vox += static_cast<long long>(gridDim.x) * blockDim.x) {
@@ -421,7 +450,7 @@ __global__ void fold3d_kernel(const T *__restrict__ x, T *__restrict__ xf, const
         const long long r2 = r / Ho;
         const int od = static_cast<int>(r2 % Do);
         const int n = static_cast<int>(r2 / Do);
-        const int d0 = od - pad, h0 = oh - pad;        // the window's first depth and row
+        const int d0 = od * stride - pad, h0 = oh * stride - pad;  // the window's first depth and row
         // x offset of (n, c = 0, d0, h0, w), possibly outside x: only in-range taps read it
         const long long base = nchw ? ((static_cast<long long>(n) * C * D + d0) * H + h0) * W + w
                                     : (((static_cast<long long>(n) * D + d0) * H + h0) * W + w) * C;
@@ -756,24 +785,27 @@ cudaError_t launch_im2col(const void *x_nhwc, void *xcol, int N, int H, int W, i
 }
 
 cudaError_t launch_fold3d(const void *x, void *xf, const void *wp, void *wf, int N, int C, int D, int H, int W,
-                          int Do, int Ho, int Cout, int Kd, int Kh, int Kw, int cpg, int pad, int dilation, int Cf,
-                          int elt, bool nchw, cudaStream_t s) {
+                          int Do, int Ho, int Cout, int Kd, int Kh, int Kw, int cpg, int stride, int pad, int dilation,
+                          int Cf, int elt, bool nchw, cudaStream_t s) {
     const int kc = Kd * Kh * C;
     // the per-channel offsets are 32-bit: one image's C*D*H*W elements stay below 2^31
     if (Cf % (16 / elt) != 0 || Cf < kc || kc > 4096 || cpg < C ||
         static_cast<long long>(C) * D * H * W >= (1LL << 31))
         return cudaErrorInvalidValue;
     const long long voxels = static_cast<long long>(N) * Do * Ho * W;
+    const bool vec = !nchw && (C * elt) % 16 == 0;  // the kernel's 16-byte copy path
+    if (vec && (Cf % C != 0 || voxels * (Cf / C) >= (1LL << 31))) return cudaErrorInvalidValue;
+    const long long work = vec ? voxels * (Cf / C) : voxels;
     const size_t tab = static_cast<size_t>(kc) * sizeof(int4);
     if (elt == 2)
-        fold3d_kernel<__nv_bfloat16><<<grid_for(voxels), kThreads, tab, s>>>(
+        fold3d_kernel<__nv_bfloat16><<<grid_for(work), kThreads, tab, s>>>(
             static_cast<const __nv_bfloat16 *>(x), static_cast<__nv_bfloat16 *>(xf),
             static_cast<const __nv_bfloat16 *>(wp), static_cast<__nv_bfloat16 *>(wf), N, C, D, H, W, Do, Ho, Cout, Kd,
-            Kh, Kw, cpg, pad, dilation, Cf, nchw);
+            Kh, Kw, cpg, stride, pad, dilation, Cf, nchw);
     else
-        fold3d_kernel<float><<<grid_for(voxels), kThreads, tab, s>>>(
+        fold3d_kernel<float><<<grid_for(work), kThreads, tab, s>>>(
             static_cast<const float *>(x), static_cast<float *>(xf), static_cast<const float *>(wp),
-            static_cast<float *>(wf), N, C, D, H, W, Do, Ho, Cout, Kd, Kh, Kw, cpg, pad, dilation, Cf, nchw);
+            static_cast<float *>(wf), N, C, D, H, W, Do, Ho, Cout, Kd, Kh, Kw, cpg, stride, pad, dilation, Cf, nchw);
     return cudaGetLastError();
 }
 

@@ -294,14 +294,19 @@ def test_conv3d_sizes_and_limits_on_the_host(lib):
         4 * 16 * 64 * 64 * 32 * 2 + 16 * 3 * 32 * 2
     p = cb.conv3d_describe_plan(4, 3, 16, 64, 64, 16, 3, 3, 3, 1, 1, 1, 1, cb.CONV_BF16, "nchw", sms=148)
     assert (p["fold"], p["kernel"], p["a_load"], p["cb"], p["BN"], p["units"]) == (1, "igemm", "im2col", 64, 16, 2048)
-    # stride 2 or 16 channels: no fold; NCDHW input then goes through the channels-last copy
-    p2 = cb.conv3d_describe_plan(4, 3, 16, 64, 64, 16, 3, 3, 3, 2, 1, 1, 1, cb.CONV_BF16, "nchw", sms=148)
-    assert (p2["fold"], p2["xcopy"]) == (0, 1)
-    assert cb.conv3d_workspace_size(4, 3, 16, 64, 64, 16, 3, 3, 3, 2, 1, 1, 1, cb.CONV_BF16, "nchw") == \
-        4 * 16 * 64 * 64 * 8 * 2
-    assert cb.conv3d_describe_plan(4, 16, 16, 64, 64, 32, 3, 3, 3, 1, 1, 1, 1, cb.CONV_BF16, "nhwc", sms=148)["fold"] == 0
+    # eight channels (16-byte rows) at stride 2 fold as well: 72 -> 96 channels over the
+    # strided rows, full input width (the product takes the column stride)
+    p2 = cb.conv3d_describe_plan(4, 8, 16, 64, 64, 32, 3, 3, 3, 2, 1, 1, 1, cb.CONV_BF16, "nhwc", sms=148)
+    assert (p2["fold"], p2["cb"], p2["BN"], p2["units"]) == (1, 64, 32, 4 * 8 * 32 * 32 // 128)
+    assert cb.conv3d_workspace_size(4, 8, 16, 64, 64, 32, 3, 3, 3, 2, 1, 1, 1, cb.CONV_BF16, "nhwc") == \
+        4 * 8 * 32 * 64 * 96 * 2 + 32 * 3 * 96 * 2
+    # 16 channels (32-byte rows; the stride-2 3-D layer), or groups: no fold; NCDHW input then
+    # goes through the channels-last copy
+    p3 = cb.conv3d_describe_plan(4, 16, 16, 64, 64, 32, 3, 3, 3, 2, 1, 1, 1, cb.CONV_BF16, "nchw", sms=148)
+    assert (p3["fold"], p3["xcopy"]) == (0, 1)
+    assert cb.conv3d_describe_plan(2, 8, 8, 16, 16, 32, 3, 3, 3, 1, 1, 1, 2, cb.CONV_BF16, "nhwc", sms=148)["fold"] == 0
     # the 5-D im2col addressing range: pad 17 is out of it
-    st = lib.conv3d_forward(16, 16, None, 16, 1, 16, 40, 40, 40, 8, 3, 3, 3, 1, 17, 1, 1, cb.CONV_BF16,
+    st = lib.conv3d_forward(16, 16, None, 16, 1, 32, 40, 40, 40, 8, 3, 3, 3, 1, 17, 1, 1, cb.CONV_BF16,
                             cb.CONV_NHWC, None, 0, None)
     assert st == cb.CONV_ERR_UNSUPPORTED
     st = lib.conv3d_forward(16, 16, None, 16, 1, 8, 2, 8, 8, 8, 5, 3, 3, 1, 0, 1, 1, cb.CONV_BF16,

@@ -53,7 +53,7 @@ EDGE3D = [  # N, C_in, D, H, W, C_out, Kd, Kh, Kw, stride, pad, dilation, groups
     (2, 16, 6, 9, 8, 32, 3, 3, 3, 1, 1, 1, 1),      # ragged last tile (864 voxels)
     (1, 64, 7, 10, 11, 48, 3, 3, 3, 2, 1, 1, 1),    # stride 2, 128-byte channel rows, C_out 48
     (2, 3, 5, 12, 12, 8, 3, 3, 3, 1, 1, 1, 1),      # three input channels: the (kd, kh)-folded 2-D form
-    (1, 3, 6, 10, 10, 16, 3, 3, 3, 2, 1, 1, 1),     # three input channels at stride 2: hardware im2col
+    (1, 3, 6, 10, 10, 16, 3, 3, 3, 2, 1, 1, 1),     # three input channels at stride 2 (folded, column stride 2)
     (1, 32, 8, 8, 8, 16, 2, 3, 5, 1, 2, 2, 1),      # non-cubic filter, dilation 2
     (1, 64, 4, 9, 9, 64, 1, 3, 3, 1, 1, 1, 4),      # (1, 3, 3) filter, groups of 16
     (2, 24, 9, 6, 7, 40, 3, 1, 3, 3, 2, 1, 1),      # stride 3, filter of height 1
@@ -78,6 +78,9 @@ FOLDED = [  # few-channel inputs at stride 1: (kd, kh) folded into the channels,
     ((2, 8, 5, 6, 7, 32, 2, 2, 3, 1, 0, 1, 1), "nhwc", "bf16"),     # eight channels (16-byte rows), no padding
     ((1, 4, 5, 7, 8, 24, 3, 3, 1, 1, 1, 1, 1), "nchw", "f32"),      # Kw = 1: the folded product is 1x1
     ((1, 2, 4, 8, 8, 16, 1, 3, 3, 1, 1, 1, 1), "nhwc", "bf16"),     # Kd = 1: only the rows fold
+    ((2, 8, 9, 12, 13, 32, 3, 3, 3, 2, 1, 1, 1), "nhwc", "bf16"),   # eight channels, stride 2 (16-byte copy path)
+    ((1, 3, 7, 11, 12, 16, 3, 3, 3, 3, 2, 1, 1), "nchw", "bf16"),   # stride 3, pad 2
+    ((1, 4, 6, 9, 10, 24, 3, 3, 3, 2, 1, 2, 1), "nhwc", "f32"),     # fp32 four channels, stride 2, dilation 2
 ]
 
 
