@@ -474,6 +474,85 @@ __global__ void fold3d_kernel(const T *__restrict__ x, T *__restrict__ xf, const
     }
 }
 
+// --- the same fold for a fixed channel count kC and kT = Kd*Kh folded taps (3x3 depth
+// and row taps of an RGB-like input): every index of the folded row is a compile-time
+// constant, the taps' shifts and offsets are computed once per thread, and each thread
+// issues all kT*kC loads of its voxel before its 16-byte stores.
+template <typename T, int kC, int kT>
+__global__ void __launch_bounds__(kThreads) fold3d_fixed_kernel(
+    const T *__restrict__ x, T *__restrict__ xf, const T *__restrict__ wp, T *__restrict__ wf, int N, int D, int H,
+    int W, int Do, int Ho, int Cout, int Kh, int Kw, int cpg, int stride, int pad, int dilation, bool nchw) {
+    constexpr int kPer = 16 / sizeof(T);
+    constexpr int kc = kT * kC;
+    constexpr int kAlign = 64 / sizeof(T);
+    constexpr int kCf = (kc + kAlign - 1) / kAlign * kAlign;
+    const long long wtotal = static_cast<long long>(Cout) * Kw * kCf;
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < wtotal;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const int k = static_cast<int>(i % kCf);
+        const long long r = i / kCf;
+        const int kw = static_cast<int>(r % Kw);
+        const int oc = static_cast<int>(r / Kw);
+        T e = T(0.f);
+        if (k < kc)
+            e = wp[(static_cast<long long>(oc) * kT * Kw + static_cast<long long>(k / kC) * Kw + kw) * cpg + k % kC];
+        wf[i] = e;
+    }
+    const int HW = H * W;          // one image's C*D*H*W < 2^31 (host)
+    const int cstep = nchw ? D * HW : 1;
+    int dd[kT], hh[kT], off[kT];
+#pragma unroll
+    for (int t = 0; t < kT; ++t) {
+        const int kd = t / Kh, kh = t - (t / Kh) * Kh;
+        dd[t] = kd * dilation;
+        hh[t] = kh * dilation;
+        off[t] = (kd * dilation * HW + kh * dilation * W) * (nchw ? 1 : kC);
+    }
+    const unsigned total = static_cast<unsigned>(N * Do * Ho * W);  // < 2^31 (host)
+    for (unsigned vox = blockIdx.x * blockDim.x + threadIdx.x; vox < total; vox += gridDim.x * blockDim.x) {
+        const unsigned r = vox / static_cast<unsigned>(W);
+        const int w = static_cast<int>(vox - r * static_cast<unsigned>(W));
+        const unsigned r2 = r / static_cast<unsigned>(Ho);
+        const int oh = static_cast<int>(r - r2 * static_cast<unsigned>(Ho));
+        const int n = static_cast<int>(r2 / static_cast<unsigned>(Do));
+        const int od = static_cast<int>(r2 - static_cast<unsigned>(n) * static_cast<unsigned>(Do));
+        const int d0 = od * stride - pad, h0 = oh * stride - pad;
+        const long long base = nchw ? ((static_cast<long long>(n) * kC * D + d0) * H + h0) * W + w
+                                    : (((static_cast<long long>(n) * D + d0) * H + h0) * W + w) * kC;
+        alignas(16) T v[kCf];
+#pragma unroll
+        for (int t = 0; t < kT; ++t) {
+            const bool in = static_cast<unsigned>(d0 + dd[t]) < static_cast<unsigned>(D) &&
+                            static_cast<unsigned>(h0 + hh[t]) < static_cast<unsigned>(H);
+#pragma unroll
+            for (int c = 0; c < kC; ++c) v[t * kC + c] = in ? x[base + off[t] + c * cstep] : T(0.f);
+        }
+#pragma unroll
+        for (int k = kc; k < kCf; ++k) v[k] = T(0.f);
+        uint4 *dst = reinterpret_cast<uint4 *>(xf + static_cast<size_t>(vox) * kCf);
+#pragma unroll
+        for (int q = 0; q < kCf / kPer; ++q) dst[q] = reinterpret_cast<const uint4 *>(v)[q];
+    }
+}
+
+template <typename T>
+cudaError_t launch_fold3d_fixed(int C, const void *x, void *xf, const void *wp, void *wf, int N, int D, int H, int W,
+                                int Do, int Ho, int Cout, int Kh, int Kw, int cpg, int stride, int pad, int dilation,
+                                bool nchw, int grid, cudaStream_t s) {
+    const T *xt = static_cast<const T *>(x);
+    const T *wt = static_cast<const T *>(wp);
+    T *xo = static_cast<T *>(xf);
+    T *wo = static_cast<T *>(wf);
+    switch (C) {
+        case 1: fold3d_fixed_kernel<T, 1, 9><<<grid, kThreads, 0, s>>>(xt, xo, wt, wo, N, D, H, W, Do, Ho, Cout, Kh, Kw, cpg, stride, pad, dilation, nchw); break;
+        case 2: fold3d_fixed_kernel<T, 2, 9><<<grid, kThreads, 0, s>>>(xt, xo, wt, wo, N, D, H, W, Do, Ho, Cout, Kh, Kw, cpg, stride, pad, dilation, nchw); break;
+        case 3: fold3d_fixed_kernel<T, 3, 9><<<grid, kThreads, 0, s>>>(xt, xo, wt, wo, N, D, H, W, Do, Ho, Cout, Kh, Kw, cpg, stride, pad, dilation, nchw); break;
+        case 4: fold3d_fixed_kernel<T, 4, 9><<<grid, kThreads, 0, s>>>(xt, xo, wt, wo, N, D, H, W, Do, Ho, Cout, Kh, Kw, cpg, stride, pad, dilation, nchw); break;
+        default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
 // --- split reduction: y = bias + sum_s ws[s][m][oc], in the output layout.
 template <bool kF32>
 __global__ void splitk_reduce_kernel(const float *__restrict__ ws, const void *__restrict__ bias,
@@ -796,6 +875,13 @@ cudaError_t launch_fold3d(const void *x, void *xf, const void *wp, void *wf, int
     const bool vec = !nchw && (C * elt) % 16 == 0;  // the kernel's 16-byte copy path
     if (vec && (Cf % C != 0 || voxels * (Cf / C) >= (1LL << 31))) return cudaErrorInvalidValue;
     const long long work = vec ? voxels * (Cf / C) : voxels;
+    // three-by-three depth and row taps of one to four channels (an RGB-like input): the
+    // kernel with every folded index fixed at compile time (same Cf formula)
+    if (!vec && Kd * Kh == 9 && C >= 1 && C <= 4 && voxels < (1LL << 31))
+        return elt == 2 ? launch_fold3d_fixed<__nv_bfloat16>(C, x, xf, wp, wf, N, D, H, W, Do, Ho, Cout, Kh, Kw, cpg,
+                                                              stride, pad, dilation, nchw, grid_for(voxels), s)
+                        : launch_fold3d_fixed<float>(C, x, xf, wp, wf, N, D, H, W, Do, Ho, Cout, Kh, Kw, cpg, stride,
+                                                      pad, dilation, nchw, grid_for(voxels), s);
     const size_t tab = static_cast<size_t>(kc) * sizeof(int4);
     if (elt == 2)
         fold3d_kernel<__nv_bfloat16><<<grid_for(work), kThreads, tab, s>>>(
