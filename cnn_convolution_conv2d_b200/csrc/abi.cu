@@ -155,6 +155,7 @@ struct Plan {
     bool pw;        // 1x1 on the kernel with resident weights (pw.cu)
     int pw_ybufs;   // its output staging blocks per epilogue warp
     int vJ, vn_k, vn_odb;  // its output slices per unit, tiles per slice, slice blocks
+    int vnacc;             // its accumulator sets (tensor memory: vnacc * vJ * C_out columns)
     int D, Kd, Do;
     bool f32;
     int elt;
@@ -594,19 +595,23 @@ int make_plan(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stri
     p.units = static_cast<int>(base * p.splits);
     // 3-D, stride 1, unit dilation, 64 input channels, at most 128 output channels: the
     // kernel that loads each input depth slice once for all the depth taps that read it
-    // (vol.cu), with two accumulator sets of J slices in tensor memory and at least three
+    // (vol.cu), with accumulator sets of J slices in tensor memory and at least three
     // stages beside the weights of two (kh, kw).
     p.vreuse = false;
     if (vol && !p.f32 && !padw && !explicit_im2col && groups == 1 && layout == CONV_NHWC && stride == 1 &&
         dilation == 1 && C_in == 64 && C_out % 32 == 0 && C_out <= 128 && (p.Ho * p.Wo) % 32 == 0 &&
         p.Ho * p.Wo >= 128) {
-        int J = 256 / C_out < vol_reuse_max_j() ? 256 / C_out : vol_reuse_max_j();
+        // As many output slices per unit as tensor memory holds (each input slice then serves
+        // more of them: (J + Kd - 1) boxes per J slices); two accumulator sets when they fit.
+        int J = 512 / C_out < vol_reuse_max_j() ? 512 / C_out : vol_reuse_max_j();
         J = J < p.Do ? J : p.Do;
+        const int nacc = 2 * J * C_out <= 512 ? 2 : 1;
         int vst = vol_reuse_max_stages();
         while (vst > 3 && vol_reuse_smem_bytes(p.Kd, C_out, vst) > kSmemBudget) --vst;
         if (vol_reuse_smem_bytes(p.Kd, C_out, vst) <= kSmemBudget) {
             p.vreuse = true;
             p.vJ = J;
+            p.vnacc = nacc;
             p.vn_k = (p.Ho * p.Wo + 127) / 128;
             p.vn_odb = (p.Do + J - 1) / J;
             p.pair = false;
@@ -1031,12 +1036,13 @@ int vol_impl(const Plan &p, const void *x, const void *w_packed, const void *bia
     v.pad_w = p.pad_w;
     v.BN = p.BN;
     v.J = p.vJ;
+    v.nacc = p.vnacc;
     v.n_k = p.vn_k;
     v.n_odb = p.vn_odb;
     v.units = p.units;
     v.stages = p.stages;
     uint32_t cols = 32;
-    while (cols < static_cast<uint32_t>(2 * p.vJ * p.BN)) cols <<= 1;
+    while (cols < static_cast<uint32_t>(p.vnacc * p.vJ * p.BN)) cols <<= 1;
     v.tmem_cols = cols;
     v.bias = bias;
     v.status = dev->status;

@@ -73,7 +73,8 @@ struct VolParams {
     int M, Do, HoWo2, Wo;
     int Kd, Kh, Kw, taps, pad, pad_w;
     int BN;              // = C_out (a multiple of 32, <= 128)
-    int J;               // output depth slices per unit (accumulators: 2*J*BN columns)
+    int J;               // output depth slices per unit (accumulators: nacc*J*BN columns)
+    int nacc;            // accumulator sets: 2 (the epilogue of one unit overlaps the next) or 1
     int n_k, n_odb, units, stages;
     uint32_t tmem_cols;
     const void *bias;

@@ -42,7 +42,7 @@ constexpr int kVRows = 128;                 // voxels per tile (M)
 constexpr int kVRowBytes = 128;             // one voxel's 64 bf16 channels
 constexpr int kVAStage = kVRows * kVRowBytes;
 constexpr int kVMaxStages = 8;
-constexpr int kVMaxJ = 4;
+constexpr int kVMaxJ = 8;
 constexpr int kVHeader = 1024;
 constexpr int kVThreads = 320;
 constexpr int kVEpiWarp0 = 2;
@@ -266,8 +266,10 @@ __global__ void __launch_bounds__(kVThreads, 1) vol_reuse_kernel(const __grid_co
                 }
                 if (!ok) break;
                 mma_commit(&sb.acc_full[abuf]);
-                abuf ^= 1;
-                if (abuf == 0) aphase ^= 1u;
+                if (++abuf == p.nacc) {  // one or two accumulator sets
+                    abuf = 0;
+                    aphase ^= 1u;
+                }
             }
             if (!ok || *wd.abort) {
                 mma_commit(&sb.drain);
@@ -350,8 +352,10 @@ __global__ void __launch_bounds__(kVThreads, 1) vol_reuse_kernel(const __grid_co
             tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sb.acc_empty[abuf]);
-            abuf ^= 1;
-            if (abuf == 0) aphase ^= 1u;
+            if (++abuf == p.nacc) {
+                abuf = 0;
+                aphase ^= 1u;
+            }
         }
         if (lane == 0) bulk_wait_group_all();  // stores done before exit
     }
@@ -376,7 +380,8 @@ int vol_reuse_max_j() { return kVMaxJ; }
 
 cudaError_t launch_vol_reuse(const VolParams &p, int grid, size_t smem, cudaStream_t stream) {
     if (p.stages < 2 || p.stages > kVMaxStages || p.J < 1 || p.J > kVMaxJ || p.BN % 32 != 0 || p.BN > 256 ||
-        p.HoWo2 % 32 != 0 || p.HoWo2 < kVRows || 2 * p.J * p.BN > static_cast<int>(p.tmem_cols) ||
+        p.HoWo2 % 32 != 0 || p.HoWo2 < kVRows || (p.nacc != 1 && p.nacc != 2) ||
+        p.nacc * p.J * p.BN > static_cast<int>(p.tmem_cols) ||
         p.Kd < 1 || p.Kh < 1 || p.Kw < 1 || p.taps != p.Kd * p.Kh * p.Kw)
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(vol_reuse_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
