@@ -128,7 +128,8 @@ __global__ void __launch_bounds__(kGtThreads, 1) gather_t_kernel(const __grid_co
         }
         for (int i = 0; i < p.nacc; ++i) {
             mbar_init(&sb.acc_full[i], 1);
-            mbar_init(&sb.acc_empty[i], kGtEpi);
+            // every epilogue warp of the tile's group hands the accumulator back
+            mbar_init(&sb.acc_empty[i], (p.tma_out && p.nout == 2) ? kGtEpi / 2 : kGtEpi);
         }
         mbar_init(&sb.a_ready, 1);
         mbar_init(&sb.drain, 1);
@@ -348,31 +349,45 @@ __global__ void __launch_bounds__(kGtThreads, 1) gather_t_kernel(const __grid_co
         // lane quarter -> (output row of the tile, output channel)
         const int r = rt == 2 ? quarter >> 1 : 0;
         const int oc = (rt == 2 ? (quarter & 1) * 32 : quarter * 32) + lane;
-        const int cspan = ((p.Wo + 15) / 16) * 8;   // columns per half, a multiple of 8
-        const int c_lo = (e >> 2) * cspan, c_hi = min(p.Wo, c_lo + cspan);
-        const bool ch_ok = oc < p.Cout;
         const bool staged = p.tma_out != 0;
-        const bool issuer = e == 0 && lane == 0;    // issues the output image's TMA store
+        // With two output images the epilogue runs as two groups of four warps on alternate
+        // tiles (each group its own image, barriers and store), so that one tile's waits
+        // overlap the other's work; each warp then drains all columns of its lane quarter.
+        // Otherwise all eight warps take every tile, each half of the columns.
+        const int ngroups = (staged && p.nout == 2) ? 2 : 1;
+        const int gsize = kGtEpi / ngroups;         // warps per group
+        const int group = e / gsize;
+        int c_lo = 0, c_hi = p.Wo;
+        if (ngroups == 1) {
+            const int cspan = ((p.Wo + 15) / 16) * 8;   // columns per half, a multiple of 8
+            c_lo = (e >> 2) * cspan;
+            c_hi = min(p.Wo, c_lo + cspan);
+        }
+        const bool ch_ok = oc < p.Cout;
+        const bool issuer = e % gsize == 0 && lane == 0;    // issues the group's TMA stores
+        const int bar_a = 1 + 2 * group, bar_b = 2 + 2 * group;
         const float bv = (ch_ok && p.bias)
                              ? __uint_as_float(static_cast<uint32_t>(static_cast<const unsigned short *>(p.bias)[oc]) << 16)
                              : 0.f;
         const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-        int li = 0;
-        for (int t = blockIdx.x; t < p.n_mtiles; t += gridDim.x, ++li) {
+        int li = group;                             // this CTA's tile count (li-th tile: t)
+        for (int t = blockIdx.x + group * static_cast<int>(gridDim.x); t < p.n_mtiles;
+             t += ngroups * static_cast<int>(gridDim.x), li += ngroups) {
             const int ab = li % p.nacc;
             const uint32_t aph = static_cast<uint32_t>(li / p.nacc) & 1u;
-            const int ob = li % p.nout;             // output image of this tile
+            const int ob = li % p.nout;             // output image of this tile (the group's own with two)
             bool ok = mbar_wait(&sb.acc_full[ab], aph, wd, kDevTimeoutAccFull);
             if (staged) {
                 // this tile's output image was last read by the TMA store of nout tiles
-                // back; all epilogue warps leave together when any wait gave up
+                // back (with two groups: the group's previous store); the group's warps
+                // leave together when any wait gave up
                 if (issuer) {
-                    if (p.nout == 1)
+                    if (p.nout == 1 || ngroups == 2)
                         bulk_wait_group_read<0>();
                     else
                         bulk_wait_group_read<1>();
                 }
-                if (!named_barrier_all(1, kGtEpi * 32, ok)) break;
+                if (!named_barrier_all(bar_a, gsize * 32, ok)) break;
             } else if (!__all_sync(0xffffffffu, ok)) {
                 break;
             }
@@ -429,7 +444,7 @@ __global__ void __launch_bounds__(kGtThreads, 1) gather_t_kernel(const __grid_co
             if (staged) {
                 // rows past C_out or Ho of the image are never written: the store clips them
                 fence_proxy_async_smem();
-                named_barrier(2, kGtEpi * 32);
+                named_barrier(bar_b, gsize * 32);
                 if (issuer) {
                     for (int part = 0; part < oparts; ++part)
                         tma_store_4d(&p.tmap_y, out_sm + ob * out_stride + part * opart_bytes, part * 64, 0, oh0, img);
