@@ -51,12 +51,14 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 TF32_PER_BF16 = 0.5
 # Tensor-core products per multiply-add of the fp32 path (a_hi*b_hi + a_hi*b_lo + a_lo*b_hi).
 TF32_PRODUCTS = 3
-# sources each measured kernel is built from (a change voids its committed ncu counters)
+# sources each measured kernel is built from (a change voids its committed ncu counters);
+# "file:Struct" stands for that struct's definition alone (the kernel's parameter block in
+# the shared header, whose other structs belong to other kernels)
 KERNEL_SOURCES = {
-    "igemm_kernel": ["igemm.cu", "epilogue.cuh", "ptx.cuh", "common.cuh"],
-    "gather_kernel": ["gather.cu", "epilogue.cuh", "ptx.cuh", "common.cuh"],
-    "gather_t_kernel": ["gather_t.cu", "ptx.cuh", "common.cuh"],
-    "dw_kernel": ["depthwise.cu", "ptx.cuh", "common.cuh"],
+    "igemm_kernel": ["igemm.cu", "epilogue.cuh", "ptx.cuh", "common.cuh:IgemmParams"],
+    "gather_kernel": ["gather.cu", "epilogue.cuh", "ptx.cuh", "common.cuh:GatherParams"],
+    "gather_t_kernel": ["gather_t.cu", "ptx.cuh", "common.cuh:GatherParams"],
+    "dw_kernel": ["depthwise.cu", "ptx.cuh", "common.cuh:DwParams"],
 }
 
 
@@ -143,9 +145,14 @@ def load_peaks():
 
 def kernel_source_hash(kernel: str) -> str:
     h = hashlib.sha256()
-    for name in KERNEL_SOURCES[kernel]:
+    for entry in KERNEL_SOURCES[kernel]:
+        name, _, struct = entry.partition(":")
         with open(os.path.join(ROOT, "cnn_convolution_conv2d_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+            data = f.read()
+        if struct:
+            start = data.index(b"struct " + struct.encode() + b" {")
+            data = data[start:data.index(b"\n};", start) + 3]
+        h.update(data)
     return h.hexdigest()[:16]
 
 
