@@ -867,9 +867,10 @@ cudaError_t launch_fold3d(const void *x, void *xf, const void *wp, void *wf, int
                           int Do, int Ho, int Cout, int Kd, int Kh, int Kw, int cpg, int stride, int pad, int dilation,
                           int Cf, int elt, bool nchw, cudaStream_t s) {
     const int kc = Kd * Kh * C;
-    // the per-channel offsets are 32-bit: one image's C*D*H*W elements stay below 2^31
+    // the per-channel offsets are 32-bit: one image's C*D*H*W elements, and the largest tap
+    // shift, stay below 2^31
     if (Cf % (16 / elt) != 0 || Cf < kc || kc > 4096 || cpg < C ||
-        static_cast<long long>(C) * D * H * W >= (1LL << 31))
+        static_cast<long long>(C) * (D + Kd * dilation) * (H + Kh * dilation) * W >= (1LL << 31))
         return cudaErrorInvalidValue;
     const long long voxels = static_cast<long long>(N) * Do * Ho * W;
     const bool vec = !nchw && (C * elt) % 16 == 0;  // the kernel's 16-byte copy path

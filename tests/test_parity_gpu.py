@@ -263,6 +263,35 @@ def test_hostio_pipelined_chunks_bit_exact(shape, layout):
         got = got.transpose(0, 3, 1, 2)
     assert np.array_equal(got, ref)
 
+
+
+def test_hostio_pipelined_under_graph_capture():
+    """The pipelined host-buffer call forks its copies onto two internal streams and joins
+    them back; captured into a CUDA graph and replayed, it gives the eager result."""
+    import torch
+    shape = (35, 64, 64, 64, 64, 3, 3, 1, 1, 1, 1)
+    ints = ("integers", -2, 2)
+    cfg = workloads.ConvConfig("hostio_graph", *shape, True, "bf16", "nhwc", ints, ints, ints, seed=29)
+    inp = workloads.make_inputs(cfg)
+    layer = parity.make_layer(cfg, inp)
+    x_dev = parity.to_device_x(cfg, inp["x"])
+    y_ref = layer(x_dev).cpu()
+    x_host = x_dev.cpu().pin_memory()
+    y_host = torch.zeros(y_ref.shape, dtype=y_ref.dtype).pin_memory()
+    x2 = torch.empty_like(x_dev)
+    y2 = torch.empty(y_ref.shape, dtype=y_ref.dtype, device="cuda")
+    layer.forward_hostio(x_host, y_host, x2, y2)   # sizes the layer's scratch before capture
+    torch.cuda.synchronize()
+    y_host.zero_()
+    stream = torch.cuda.Stream()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        layer.forward_hostio(x_host, y_host, x2, y2, stream=stream)
+    graph.replay()
+    torch.cuda.synchronize()
+    cb.conv2d_sync_status()
+    assert torch.equal(y_host, y_ref)
+
 def test_repeated_calls_are_identical():
     import torch
     cfg = parity.config("k7_17x17_bf16", N=1, C_in=128, C_out=128)
