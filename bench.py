@@ -361,6 +361,38 @@ def oracle_rate_sample(cfg, inp, seconds: float, seed: int = 1234, max_points=No
     return points * per_point / wall, points, wall, oracle.num_threads()
 
 
+def capture_steps(cb, G, step, kev=None):
+    """A CUDA graph of G steps (step(i) for i < G) and the library launches it holds; with
+    kev, the library records kev[i] around step i's main kernel."""
+    import torch
+    launches0 = cb.conv2d_kernel_launch_count()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for i in range(G):
+            if kev is not None:
+                cb.conv2d_set_main_kernel_events(*kev[i])
+            step(i)
+    cb.conv2d_set_main_kernel_events(None, None)
+    launches = cb.conv2d_kernel_launch_count() - launches0
+    graph.replay()  # one untimed replay: graph upload
+    torch.cuda.synchronize()
+    return graph, launches
+
+
+def kernel_time_ms(step_ms, launches_per_step, graph_k, kev):
+    """The main kernel's average launch time.  A step that is one library launch is timed by
+    the events around the whole timed region (step_ms); otherwise the events the library
+    records around the main kernel, in a separate replay of a graph holding them (each event
+    pair adds a few microseconds, so this errs long)."""
+    import torch
+    if launches_per_step == 1:
+        return step_ms, "one launch per step: events over the timed region / steps"
+    graph_k.replay()
+    torch.cuda.synchronize()
+    return (statistics.fmean(a.elapsed_time(c) for a, c in kev),
+            "events around the main kernel in a separate graph replay (each pair adds a few us)")
+
+
 def run_reference(args, cfg):
     """The comparison arm: the oracle as it stands on this machine's host cores."""
     import numpy as np
@@ -468,17 +500,12 @@ def run_ours(args, cfg):
         a.record()
         c.record()
     torch.cuda.synchronize()
-    launches0 = cb.conv2d_kernel_launch_count()
     if args.graph:
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
-            for i in range(G):
-                cb.conv2d_set_main_kernel_events(*kev[i])
-                layer(xs[i % nsets], ys[i % nsets], explicit_im2col=ex)
-        cb.conv2d_set_main_kernel_events(None, None)
-        launches_per_rep = cb.conv2d_kernel_launch_count() - launches0
-        graph.replay()  # one untimed replay: graph upload
-        torch.cuda.synchronize()
+        # the timed graph holds no timing events (a pair per step would add a few us to each)
+        def fstep(i):
+            layer(xs[i % nsets], ys[i % nsets], explicit_im2col=ex)
+        graph, launches_per_rep = capture_steps(cb, G, fstep)
+        graph_k, _ = capture_steps(cb, G, fstep, kev)
 
     clocks = ClockSampler(local)
     clocks.start()
@@ -507,7 +534,11 @@ def run_ours(args, cfg):
     launches = (launches_per_rep * reps if args.graph
                 else cb.conv2d_kernel_launch_count() - launches_before)
     elapsed_ms = max_over_ranks(ev0.elapsed_time(ev1), world, device)
-    kernel_ms = statistics.fmean(a.elapsed_time(c) for a, c in kev)
+    if args.graph:
+        kernel_ms, ktiming = kernel_time_ms(ev0.elapsed_time(ev1) / args.steps, launches_per_rep / G, graph_k, kev)
+    else:
+        kernel_ms = statistics.fmean(a.elapsed_time(c) for a, c in kev)
+        ktiming = "events around the main kernel, eager launches"
     kernel_ms = max_over_ranks(kernel_ms, world, device)
     ms_per_step = elapsed_ms / args.steps
     value = weak_scaling_value(world, flops(cfg), args.steps, elapsed_ms)
@@ -570,8 +601,8 @@ def run_ours(args, cfg):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": cfg.dtype, "data": "synthetic (seeded; x ~ N(0,1), He-scaled weights)",
             "config": cfgd,
-            "roofline": with_write_context(roofline(cfg, kernel_ms, peaks, peak_kind, cfg.name, ex,
-                                                    plan_kernel=plan["kernel"]), cfg, kernel_ms, fill_gbs),
+            "roofline": dict(with_write_context(roofline(cfg, kernel_ms, peaks, peak_kind, cfg.name, ex,
+                                                    plan_kernel=plan["kernel"]), cfg, kernel_ms, fill_gbs), kernel_timing=ktiming),
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
@@ -645,16 +676,9 @@ def run_backward(args, cfg):
         a.record()
         c.record()
     torch.cuda.synchronize()
-    launches0 = cb.conv2d_kernel_launch_count()
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
-        for i in range(G):
-            cb.conv2d_set_main_kernel_events(*kev[i])
-            step(i)
-    cb.conv2d_set_main_kernel_events(None, None)
-    launches_per_rep = cb.conv2d_kernel_launch_count() - launches0
-    graph.replay()
-    torch.cuda.synchronize()
+    # the timed graph holds no timing events (a pair per step would add a few us to each)
+    graph, launches_per_rep = capture_steps(cb, G, step)
+    graph_k, _ = capture_steps(cb, G, step, kev)
     clocks = ClockSampler(0)
     clocks.start()
     time.sleep(0.05)
@@ -671,7 +695,7 @@ def run_backward(args, cfg):
     clocks.stop()
     cb.conv2d_sync_status()
     elapsed = ev0.elapsed_time(ev1)
-    kernel_ms = statistics.fmean(a.elapsed_time(c) for a, c in kev)
+    kernel_ms, ktiming = kernel_time_ms(elapsed / args.steps, launches_per_rep / G, graph_k, kev)
     f = flops(cfg)
     peaks, peak_kind = load_peaks()
     plan = cb.conv2d_describe_plan(cfg.N, cfg.C_in, cfg.H, cfg.W, cfg.C_out, cfg.Kh, cfg.Kw, cfg.stride, cfg.pad,
@@ -693,7 +717,8 @@ def run_backward(args, cfg):
                    "l2": f"not resident: steps rotate over {nsets} sets ({nsets * set_bytes / 1e6:.0f} MB)",
                    "launch": f"CUDA graphs of {G} steps x {reps} replays", "forward_plan": plan},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                     "peak_source": ksrc, "kernel_ms": kernel_ms, "algorithmic_flops_per_launch": f,
+                     "peak_source": ksrc, "kernel_ms": kernel_ms, "kernel_timing": ktiming,
+                     "algorithmic_flops_per_launch": f,
                      "executed_flops_per_launch": executed, "traffic": None,
                      "kernel": ("igemm_kernel / dw_kernel on the transposed convolution" if args.backward == "data"
                                 else "wgrad_kernel (pixel-reduction tcgen05 product, MN-major operands)"
@@ -747,16 +772,11 @@ def run_conv3d(args, cfg):
         a.record()
         c.record()
     torch.cuda.synchronize()
-    launches0 = cb.conv2d_kernel_launch_count()
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
-        for i in range(G):
-            cb.conv2d_set_main_kernel_events(*kev[i])
-            layer(xs[i % nsets], ys[i % nsets])
-    cb.conv2d_set_main_kernel_events(None, None)
-    launches_per_rep = cb.conv2d_kernel_launch_count() - launches0
-    graph.replay()
-    torch.cuda.synchronize()
+    # the timed graph holds no timing events (a pair per step would add a few us to each)
+    def lstep(i):
+        layer(xs[i % nsets], ys[i % nsets])
+    graph, launches_per_rep = capture_steps(cb, G, lstep)
+    graph_k, _ = capture_steps(cb, G, lstep, kev)
     clocks = ClockSampler(0)
     clocks.start()
     time.sleep(0.05)
@@ -773,7 +793,7 @@ def run_conv3d(args, cfg):
     clocks.stop()
     cb.conv2d_sync_status()
     elapsed = ev0.elapsed_time(ev1)
-    kernel_ms = statistics.fmean(a.elapsed_time(c) for a, c in kev)
+    kernel_ms, ktiming = kernel_time_ms(elapsed / args.steps, launches_per_rep / G, graph_k, kev)
     e = elt_bytes(cfg)
     f = 2.0 * cfg.N * cfg.C_out * cfg.Do * cfg.Ho * cfg.Wo * (cfg.C_in // cfg.groups) * cfg.Kd * cfg.Kh * cfg.Kw
     nbytes = e * (cfg.N * cfg.C_in * cfg.D * cfg.H * cfg.W + cfg.C_out * (cfg.C_in // cfg.groups) * cfg.Kd * cfg.Kh
@@ -800,7 +820,7 @@ def run_conv3d(args, cfg):
         kname = "vol_reuse_kernel (5-D TMA im2col, each input slice loaded once for all depth taps, tcgen05)"
     else:
         kname = "igemm_kernel (5-D TMA im2col, tcgen05)"
-    rl.update({"kernel": kname, "kernel_ms": kernel_ms, "plan": plan,
+    rl.update({"kernel": kname, "kernel_ms": kernel_ms, "kernel_timing": ktiming, "plan": plan,
                "algorithmic_flops_per_launch": f, "algorithmic_bytes_per_launch": nbytes, "traffic": None,
                "step_frac": (rl["achieved"] * kernel_ms / (elapsed / args.steps)) / rl["peak"]})
     desc = (f"{cfg.name}: N={cfg.N} C_in={cfg.C_in} {cfg.D}x{cfg.H}x{cfg.W} -> C_out={cfg.C_out}, "
@@ -873,16 +893,11 @@ def run_winograd(args, cfg):
         a.record()
         c.record()
     torch.cuda.synchronize()
-    launches0 = cb.conv2d_kernel_launch_count()
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
-        for i in range(G):
-            cb.conv2d_set_main_kernel_events(*kev[i])
-            layer(xs[i % nsets], ys[i % nsets])
-    cb.conv2d_set_main_kernel_events(None, None)
-    launches_per_rep = cb.conv2d_kernel_launch_count() - launches0
-    graph.replay()
-    torch.cuda.synchronize()
+    # the timed graph holds no timing events (a pair per step would add a few us to each)
+    def lstep(i):
+        layer(xs[i % nsets], ys[i % nsets])
+    graph, launches_per_rep = capture_steps(cb, G, lstep)
+    graph_k, _ = capture_steps(cb, G, lstep, kev)
     clocks = ClockSampler(0)
     clocks.start()
     time.sleep(0.05)
@@ -899,7 +914,7 @@ def run_winograd(args, cfg):
     clocks.stop()
     cb.conv2d_sync_status()
     elapsed = ev0.elapsed_time(ev1)
-    kernel_ms = statistics.fmean(a.elapsed_time(c) for a, c in kev)
+    kernel_ms, ktiming = kernel_time_ms(elapsed / args.steps, launches_per_rep / G, graph_k, kev)
     a2 = (m + 2) ** 2
     tiles = cfg.N * (-(-cfg.Ho // m)) * (-(-cfg.Wo // m))
     e = elt_bytes(cfg)
@@ -935,7 +950,7 @@ def run_winograd(args, cfg):
                      "frac": ach / pk, "peak_source": psrc,
                      "kernel": ("pw_kernel" if prod_plan["kernel"] == "pointwise" else "igemm_kernel")
                      + " on the transformed tiles ((m+2)^2 groups of 1x1)",
-                     "kernel_ms": kernel_ms, "gemm_flops_per_launch": gemm_flops,
+                     "kernel_ms": kernel_ms, "kernel_timing": ktiming, "gemm_flops_per_launch": gemm_flops,
                      "product_bytes_per_launch": prod_bytes,
                      "tensor_frac": mult * gemm_flops / (kernel_ms * 1e-3) / 1e12 / tpeak, "traffic": None,
                      "multiplies_vs_direct": a2 / (m * m * 9.0),
