@@ -123,7 +123,7 @@ __global__ void __launch_bounds__(kGtThreads, 1) gather_t_kernel(const __grid_co
     if (threadIdx.x == 0) {
         for (int i = 0; i < p.nhalo; ++i) mbar_init(&sb.halo_full[i], 1);
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&sb.b_full[i], kGtProd);
+            mbar_init(&sb.b_full[i], kGtProd / 2);  // the gather group of the tile (four warps)
             mbar_init(&sb.b_empty[i], 1);
         }
         for (int i = 0; i < p.nacc; ++i) {
@@ -221,18 +221,20 @@ __global__ void __launch_bounds__(kGtThreads, 1) gather_t_kernel(const __grid_co
 
     if (warp < kGtProd) {
         // ------------------------------------------------------------- gather ---
+        // Two groups of four warps on alternate tiles, each with its own B buffer, so that one
+        // tile's waits overlap the other's gather; a thread builds all chunks of its rows.
+        const int grp = warp / (kGtProd / 2);
         const int row0 = threadIdx.x & 127;         // first pixel (B row) of this thread; then +128
-        const int part = threadIdx.x >> 7;          // which half of the chunks
-        const int half = ((nchunks + 1) / 2 + 1) & ~1;
-        const int jb = part == 0 ? 0 : half, je = part == 0 ? min(half, nchunks) : nchunks;
+        const int jb = 0, je = nchunks;
         // rows past Wo feed columns that are never stored
         // chunk j = c*R + r reads staged row j (unit dilation); chunks past C*R are the
         // reduction's zero padding
         const int crow = p.C * p.R;
         const int bww = p.BW / 2;                   // 32-bit words per staged row (BW is even)
-        int li = 0;
-        for (int t = blockIdx.x; t < p.n_mtiles; t += gridDim.x, ++li) {
-            const int b = li & 1;
+        int li = grp;
+        for (int t = blockIdx.x + grp * static_cast<int>(gridDim.x); t < p.n_mtiles;
+             t += 2 * static_cast<int>(gridDim.x), li += 2) {
+            const int b = li & 1;                   // = grp
             const uint32_t ph = static_cast<uint32_t>(li >> 1) & 1u;
             const int hb = li % p.nhalo;
             const uint32_t hph = static_cast<uint32_t>(li / p.nhalo) & 1u;
@@ -245,11 +247,11 @@ __global__ void __launch_bounds__(kGtThreads, 1) gather_t_kernel(const __grid_co
                 const uint32_t *hrow = h32 + (e0 >> 1);
                 const uint32_t sh = (e0 & 1) * 16u;
                 uint8_t *dst = b_sm + b * b_stride + gt_core(row, 0, sbo);
-                // at most kGtMaxChunks / 2 chunks per thread, in batches of 8: all of a
+                // at most kGtMaxChunks chunks per thread, in batches of 8: all of a
                 // batch's loads are issued before any of its stores (a store could alias a
                 // later load as far as the compiler knows, which would serialise them)
 #pragma unroll
-                for (int g0 = 0; g0 < kGtMaxChunks / 2; g0 += 8) {
+                for (int g0 = 0; g0 < kGtMaxChunks; g0 += 8) {
                     if (jb + g0 >= je) break;
                     uint32_t w[8][5];
 #pragma unroll
