@@ -143,12 +143,40 @@ __global__ void __launch_bounds__(kGtThreads, 1) gather_t_kernel(const __grid_co
         mbar_arrive_expect_tx(&sb.halo_full[hb], halo_bytes);
         tma_load_4d(halo_sm + hb * halo_stride, &p.tmap_x, &sb.halo_full[hb], -p.ME, oh0 * p.stride - p.pad, 0, img);
     };
+    // Two rows per tile build A from the weight image.  Every CTA reads the same image at the
+    // same moment: it comes into shared memory (beside where A is built, else in the output
+    // images, both free until the first tile) by one bulk copy, issued ahead of the staged
+    // input rows so that it does not queue behind them, rather than by a global load per
+    // 16-byte piece (a per-role clock record put that form at ~6.5 K cycles of the launch's
+    // start).
+    const int ichunks = p.Kpad / 8;                                // the image's chunks
+    const uint32_t isbo = static_cast<uint32_t>(ichunks) * 128u;
+    uint8_t *stage = nullptr;
+    if (rt == 2) {
+        const uint32_t img_bytes = static_cast<uint32_t>(p.BN / 8) * isbo;
+        const uint32_t b_space = 2 * b_stride;
+        if (!a_tmem) {
+            if (b_space >= img_bytes) stage = b_sm;
+        } else if (b_space >= gt_align1k(a_bytes) + img_bytes) {
+            stage = b_sm + gt_align1k(a_bytes);                    // A is built at b_sm
+        }
+        if (stage == nullptr && static_cast<uint32_t>(p.nout) * out_stride >= img_bytes) stage = out_sm;
+        if (stage != nullptr && threadIdx.x == 0 && !p.starve) {
+            mbar_arrive_expect_tx(&sb.a_ready, img_bytes);
+            bulk_load(stage, p.w_image, img_bytes, &sb.a_ready);
+        }
+    }
+    const bool a_staged = stage != nullptr;
     if (threadIdx.x == 0 && !p.starve) {
         // the first tiles' input rows are on their way while A is being set up
         prefetch_tensormap(&p.tmap_x);
         for (int k = 0; k < p.nhalo; ++k)
             if (blockIdx.x + k * static_cast<int>(gridDim.x) < p.n_mtiles) issue_halo(blockIdx.x + k * gridDim.x, k);
     }
+    Watchdog wd;
+    wd.abort = &sb.abort;
+    wd.status = p.status;
+    wd.timeout_ns = static_cast<uint64_t>(p.timeout_ns);
     if (rt == 1) {
         // weight rows past the image's (C_out rounded up to 16) are zero: output channels
         // that do not exist come out as zeros and are not stored
@@ -161,14 +189,15 @@ __global__ void __launch_bounds__(kGtThreads, 1) gather_t_kernel(const __grid_co
         uint4 *z = reinterpret_cast<uint4 *>(a_sm);
         for (uint32_t i = threadIdx.x; i < a_bytes / 16u; i += blockDim.x) z[i] = make_uint4(0, 0, 0, 0);
         __syncthreads();
-        const int ichunks = p.Kpad / 8;                            // the image's chunks
-        const uint32_t isbo = static_cast<uint32_t>(ichunks) * 128u;
+        // a copy that never lands leaves A zero and the watchdog's status set
+        const bool img_ok = !a_staged || mbar_wait(&sb.a_ready, 0, wd, kDevTimeoutFull);
         const int real = p.C * p.Kh;
-        const uint8_t *img = static_cast<const uint8_t *>(p.w_image);
-        for (int i = threadIdx.x; i < p.BN * real; i += blockDim.x) {
+        const uint8_t *img = a_staged ? stage : static_cast<const uint8_t *>(p.w_image);
+        for (int i = threadIdx.x; img_ok && i < p.BN * real; i += blockDim.x) {
             const int oc = i / real, j = i - (i / real) * real;
             const int c = j / p.Kh, kh = j - (j / p.Kh) * p.Kh;
-            const uint4 v = __ldg(reinterpret_cast<const uint4 *>(img + gt_core(oc, j, isbo)));
+            const uint4 *q = reinterpret_cast<const uint4 *>(img + gt_core(oc, j, isbo));
+            const uint4 v = a_staged ? *q : __ldg(q);
             const int j0 = c * p.R + kh;
             *reinterpret_cast<uint4 *>(a_sm + gt_core(oc, j0, sbo)) = v;
             *reinterpret_cast<uint4 *>(a_sm + gt_core(64 + oc, j0 + p.stride, sbo)) = v;
@@ -189,11 +218,6 @@ __global__ void __launch_bounds__(kGtThreads, 1) gather_t_kernel(const __grid_co
     tc_fence_after_sync();
     const uint32_t tmem_base = sb.tmem_base;
     const uint32_t a_col = static_cast<uint32_t>(p.nacc * tpix);   // A's first tensor-memory column
-
-    Watchdog wd;
-    wd.abort = &sb.abort;
-    wd.status = p.status;
-    wd.timeout_ns = static_cast<uint64_t>(p.timeout_ns);
 
     if (a_tmem) {
         // A (128 rows x nchunks 16-byte chunks) from shared memory into tensor memory: one
@@ -337,7 +361,7 @@ __global__ void __launch_bounds__(kGtThreads, 1) gather_t_kernel(const __grid_co
             if (!ok || *wd.abort) {
                 mma_commit(&sb.drain);
                 gt_wait_quiet(&sb.drain, 0, wd.timeout_ns);
-                if (!p.starve && rt == 1 && !a_tmem) gt_wait_quiet(&sb.a_ready, 0, wd.timeout_ns);
+                if (!p.starve && ((rt == 1 && !a_tmem) || a_staged)) gt_wait_quiet(&sb.a_ready, 0, wd.timeout_ns);
                 for (int hb = 0; hb < p.nhalo; ++hb)  // let the staged-row loads still in flight land
                     if (issued[hb] > 0)
                         gt_wait_quiet(&sb.halo_full[hb], static_cast<uint32_t>(issued[hb] - 1) & 1u, wd.timeout_ns);

@@ -130,6 +130,31 @@ def test_transposed_first_layer(shape, form):
     parity.assert_close(cfg, parity.run_gpu(cfg, inp), parity.run_oracle(cfg, inp), str(shape))
 
 
+def test_transposed_first_layer_watchdog_returns_timeout():
+    """The transposed first-layer kernel with loads withheld: its first wait (the bulk copy
+    of the weight image that two-row tiles build A from) runs out after 1 ms, every later
+    wait gives up at once, the status reads TIMEOUT, and the next normal call is right."""
+    shape = (2, 3, 30, 64, 32, 7, 7, 2, 3, 1, 1)
+    plan = cb.conv2d_describe_plan(*shape, cb.CONV_BF16, "nchw")
+    assert (plan["kernel"], plan["rows"]) == ("gather_t", 2), plan
+    N, C_in, H, W, C_out, Kh, Kw, s, p, d, g = shape
+    cfg = workloads.ConvConfig("first", N, C_in, H, W, C_out, Kh, Kw, s, p, d, g, True, "bf16", "nchw",
+                               seed=sum(shape))
+    inp = workloads.make_inputs(cfg)
+    layer = parity.make_layer(cfg, inp)
+    x = parity.to_device_x(cfg, inp["x"])
+    try:
+        cb.conv2d_debug_set_watchdog(1_000_000, True)
+        layer(x)
+        with pytest.raises(cb.Conv2dError) as err:
+            cb.conv2d_sync_status()
+        assert err.value.status == cb.CONV_ERR_TIMEOUT
+    finally:
+        cb.conv2d_debug_set_watchdog(0, False)
+    cb.conv2d_sync_status()  # status was cleared
+    parity.assert_close(cfg, parity.run_gpu(cfg, inp, layer=layer), parity.run_oracle(cfg, inp), "after timeout")
+
+
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("explicit", [False, True])
 @pytest.mark.parametrize("shape", [(2, 3, 9, 11, 4, 3, 3, 2, 1, 1, 1), (2, 16, 12, 12, 32, 3, 3, 1, 1, 1, 1),
