@@ -71,6 +71,7 @@ struct GtShared {
     uint64_t acc_full[kGtMaxAcc];
     uint64_t acc_empty[kGtMaxAcc];
     uint64_t a_ready;
+    uint64_t a_tm_ready;   // A is in tensor memory (four epilogue warps)
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
@@ -132,6 +133,7 @@ __global__ void __launch_bounds__(kGtThreads, 1) gather_t_kernel(const __grid_co
             mbar_init(&sb.acc_empty[i], (p.tma_out && p.nout == 2) ? kGtEpi / 2 : kGtEpi);
         }
         mbar_init(&sb.a_ready, 1);
+        mbar_init(&sb.a_tm_ready, 4);
         mbar_init(&sb.drain, 1);
         sb.abort = 0;
         fence_mbar_init();
@@ -143,28 +145,28 @@ __global__ void __launch_bounds__(kGtThreads, 1) gather_t_kernel(const __grid_co
         mbar_arrive_expect_tx(&sb.halo_full[hb], halo_bytes);
         tma_load_4d(halo_sm + hb * halo_stride, &p.tmap_x, &sb.halo_full[hb], -p.ME, oh0 * p.stride - p.pad, 0, img);
     };
-    // Two rows per tile build A from the weight image.  Every CTA reads the same image at the
-    // same moment: it comes into shared memory (beside where A is built, else in the output
-    // images, both free until the first tile) by one bulk copy, issued ahead of the staged
-    // input rows so that it does not queue behind them, rather than by a global load per
-    // 16-byte piece (a per-role clock record put that form at ~6.5 K cycles of the launch's
-    // start).
+    // A from the weight image.  Every CTA reads the same image at the same moment: it comes
+    // into shared memory by one bulk copy, issued ahead of the staged input rows so that it
+    // does not queue behind them, rather than by a global load per 16-byte piece (a per-role
+    // clock record put that form at ~6.5 K cycles of the launch's start).  With A in tensor
+    // memory the image lands in the output images (free until the first tile's accumulator,
+    // which needs A) and four epilogue warps write A's rows from it straight into tensor
+    // memory while the gather warps start on the first tiles; otherwise A is built in
+    // shared memory before the roles split (two rows per tile: from the image staged beside
+    // it; one row: the image is A, loaded by the product warp).
     const int ichunks = p.Kpad / 8;                                // the image's chunks
     const uint32_t isbo = static_cast<uint32_t>(ichunks) * 128u;
+    const uint32_t img_bytes = static_cast<uint32_t>(p.BN / 8) * isbo;
     uint8_t *stage = nullptr;
-    if (rt == 2) {
-        const uint32_t img_bytes = static_cast<uint32_t>(p.BN / 8) * isbo;
-        const uint32_t b_space = 2 * b_stride;
-        if (!a_tmem) {
-            if (b_space >= img_bytes) stage = b_sm;
-        } else if (b_space >= gt_align1k(a_bytes) + img_bytes) {
-            stage = b_sm + gt_align1k(a_bytes);                    // A is built at b_sm
-        }
-        if (stage == nullptr && static_cast<uint32_t>(p.nout) * out_stride >= img_bytes) stage = out_sm;
-        if (stage != nullptr && threadIdx.x == 0 && !p.starve) {
-            mbar_arrive_expect_tx(&sb.a_ready, img_bytes);
-            bulk_load(stage, p.w_image, img_bytes, &sb.a_ready);
-        }
+    if (a_tmem) {
+        if (static_cast<uint32_t>(p.nout) * out_stride >= img_bytes) stage = out_sm;
+    } else if (rt == 2) {
+        if (2 * b_stride >= img_bytes) stage = b_sm;
+        else if (static_cast<uint32_t>(p.nout) * out_stride >= img_bytes) stage = out_sm;
+    }
+    if (stage != nullptr && threadIdx.x == 0 && !p.starve) {
+        mbar_arrive_expect_tx(&sb.a_ready, img_bytes);
+        bulk_load(stage, p.w_image, img_bytes, &sb.a_ready);
     }
     const bool a_staged = stage != nullptr;
     if (threadIdx.x == 0 && !p.starve) {
@@ -177,13 +179,12 @@ __global__ void __launch_bounds__(kGtThreads, 1) gather_t_kernel(const __grid_co
     wd.abort = &sb.abort;
     wd.status = p.status;
     wd.timeout_ns = static_cast<uint64_t>(p.timeout_ns);
-    if (rt == 1) {
+    if (!a_tmem && rt == 1) {
         // weight rows past the image's (C_out rounded up to 16) are zero: output channels
         // that do not exist come out as zeros and are not stored
-        const uint32_t img_bytes = static_cast<uint32_t>(p.BN / 8) * sbo;
         uint4 *z = reinterpret_cast<uint4 *>(a_sm + img_bytes);
         for (uint32_t i = threadIdx.x; i < (a_bytes - img_bytes) / 16u; i += blockDim.x) z[i] = make_uint4(0, 0, 0, 0);
-    } else {
+    } else if (!a_tmem) {
         // Two rows per tile: row r*64 + oc of A, chunk c*R + kh + r*stride, holds the
         // image's row oc, chunk c*Kh + kh (R = Kh + stride staged rows); all else is zero.
         uint4 *z = reinterpret_cast<uint4 *>(a_sm);
@@ -208,40 +209,11 @@ __global__ void __launch_bounds__(kGtThreads, 1) gather_t_kernel(const __grid_co
         tmem_alloc(&sb.tmem_base, p.tmem_cols);
         tmem_relinquish();
     }
-    if (a_tmem && rt == 1 && threadIdx.x == 0 && !p.starve) {
-        const uint32_t img_bytes = static_cast<uint32_t>(p.BN / 8) * sbo;
-        mbar_arrive_expect_tx(&sb.a_ready, img_bytes);
-        bulk_load(a_sm, p.w_image, img_bytes, &sb.a_ready);
-    }
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem_base = sb.tmem_base;
     const uint32_t a_col = static_cast<uint32_t>(p.nacc * tpix);   // A's first tensor-memory column
-
-    if (a_tmem) {
-        // A (128 rows x nchunks 16-byte chunks) from shared memory into tensor memory: one
-        // warp per lane quarter, thread = row, two chunks (8 columns) per store
-        bool ok = true;
-        if (rt == 1) ok = p.starve ? false : mbar_wait(&sb.a_ready, 0, wd, kDevTimeoutFull);
-        const int e = warp - kGtMma - 1;
-        if (ok && e >= 0 && e < 4) {
-            const int quarter = warp & 3;
-            const int m = quarter * 32 + lane;
-            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + a_col;
-            for (int j = 0; j < nchunks; j += 2) {
-                const uint4 c0 = *reinterpret_cast<const uint4 *>(a_sm + gt_core(m, j, sbo));
-                const uint4 c1 = *reinterpret_cast<const uint4 *>(a_sm + gt_core(m, j + 1, sbo));
-                const uint32_t w8[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-                tmem_st_x8(taddr + static_cast<uint32_t>(j * 4), w8);
-            }
-            tmem_st_wait();
-        }
-        // A's shared-memory copy is B's space from here on
-        tc_fence_before_sync();
-        __syncthreads();
-        tc_fence_after_sync();
-    }
 
     if (warp < kGtProd) {
         // ------------------------------------------------------------- gather ---
@@ -316,6 +288,8 @@ __global__ void __launch_bounds__(kGtThreads, 1) gather_t_kernel(const __grid_co
                 for (int k = 0; k < p.nhalo; ++k)
                     issued[k] = blockIdx.x + k * static_cast<int>(gridDim.x) < p.n_mtiles ? 1 : 0;
             bool ok = !*wd.abort;
+            if (a_tmem && !mbar_wait(&sb.a_tm_ready, 0, wd, kDevTimeoutFull)) ok = false;
+            tc_fence_after_sync();
             if (!a_tmem && rt == 1 && !p.starve) {
                 const uint32_t img_bytes = static_cast<uint32_t>(p.BN / 8) * sbo;
                 mbar_arrive_expect_tx(&sb.a_ready, img_bytes);
@@ -372,6 +346,45 @@ __global__ void __launch_bounds__(kGtThreads, 1) gather_t_kernel(const __grid_co
         // ----------------------------------------------------------- epilogue ---
         const int e = warp - kGtMma - 1;            // 0..7
         const int quarter = warp & 3;               // tensor-memory lanes of this warp
+        if (a_tmem && e < 4) {
+            // A's rows into tensor memory, thread = row of this warp's lane quarter: chunk jj
+            // of row r*64 + oc (or oc) is the image's piece (oc, c*Kh + kh) when jj =
+            // c*R + kh + r*stride names one, else zero; two chunks (8 columns) per store
+            const bool img_ok = !a_staged || mbar_wait(&sb.a_ready, 0, wd, kDevTimeoutFull);
+            const int m = quarter * 32 + lane;
+            const int ar = rt == 2 ? m >> 6 : 0;
+            const int aoc = rt == 2 ? m & 63 : m;
+            const uint8_t *img = a_staged ? stage : static_cast<const uint8_t *>(p.w_image);
+            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + a_col;
+            if (img_ok) {
+                int c = 0, khp = 0;                 // chunk jj = c*R + khp
+                for (int j = 0; j < nchunks; j += 2) {
+                    uint32_t w8[8];
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int kh = khp - ar * p.stride;
+                        uint4 v = make_uint4(0, 0, 0, 0);
+                        if (aoc < p.BN && c < p.C && kh >= 0 && kh < p.Kh) {
+                            const uint4 *q = reinterpret_cast<const uint4 *>(img + gt_core(aoc, c * p.Kh + kh, isbo));
+                            v = a_staged ? *q : __ldg(q);
+                        }
+                        w8[4 * h] = v.x;
+                        w8[4 * h + 1] = v.y;
+                        w8[4 * h + 2] = v.z;
+                        w8[4 * h + 3] = v.w;
+                        if (++khp == p.R) {
+                            khp = 0;
+                            ++c;
+                        }
+                    }
+                    tmem_st_x8(taddr + static_cast<uint32_t>(j * 4), w8);
+                }
+                tmem_st_wait();
+            }
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sb.a_tm_ready);
+        }
         // lane quarter -> (output row of the tile, output channel)
         const int r = rt == 2 ? quarter >> 1 : 0;
         const int oc = (rt == 2 ? (quarter & 1) * 32 : quarter * 32) + lane;
