@@ -486,9 +486,10 @@ int make_plan(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stri
                 const int tpix = round_up(p.Wo, 16);
                 // Two output rows per tile when the channels fill half the lanes, else one.
                 // The output block of a tile goes out by TMA stores from double-buffered
-                // output images when they fit beside at least three staged-row buffers,
+                // output images when they fit beside at least four staged-row buffers,
                 // else from one image, else straight from the registers; then as many
-                // staged-row buffers as fit (up to the kernel's limit): one tile's work is
+                // staged-row buffers as fit (up to the kernel's limit), an even number (a
+                // buffer serves one of the kernel's two gather groups): one tile's work is
                 // shorter than the latency of its rows' load.
                 for (int rt = C_out <= 64 ? 2 : 1; rt >= 1 && !p.gather_t; --rt) {
                     const int R = Kh + (rt - 1) * stride;
@@ -500,13 +501,14 @@ int make_plan(int N, int C_in, int H, int W, int C_out, int Kh, int Kw, int stri
                     // kt/2 columns), else in shared memory
                     const int acc_tm = (512 - kt / 2) / tpix;
                     for (int a_tm = (tpix >= 64 && acc_tm >= 2) ? 1 : 0; a_tm >= 0 && !p.gather_t; --a_tm) {
-                        const int opts[3][3] = {{1, 2, 3}, {1, 1, 2}, {0, 1, 2}};  // tma_out, images, fewest row buffers
+                        const int opts[3][3] = {{1, 2, 4}, {1, 1, 2}, {0, 1, 2}};  // tma_out, images, fewest row buffers
                         for (const auto &o : opts) {
                             const size_t obytes = o[0] ? ob : 0;
                             int nhalo = gather_t_max_halo();
                             while (nhalo > o[2] &&
                                    gather_t_smem_bytes(kt, tpix, hb, nhalo, obytes, o[1], a_tm != 0) > kSmemBudget)
                                 --nhalo;
+                            nhalo &= ~1;
                             const size_t tsmem = gather_t_smem_bytes(kt, tpix, hb, nhalo, obytes, o[1], a_tm != 0);
                             if (tsmem > kSmemBudget) continue;
                             p.gather_t = true;

@@ -35,11 +35,12 @@
 //   D (tensor memory, fp32): lanes = (output row, output channel), columns = pixels, a ring
 //      of up to four accumulators (as many as 512 columns hold beside A).
 //
-//   gather warps 0..7 : thread t builds pixel rows t % 128 (+ 128), chunks of half t / 128;
-//   warp 8            : tensor-memory allocation, TMA loads of the staged input rows (up
-//                       to eight tiles ahead: a tile's own work is shorter than the
-//                       latency of its load; the first round is issued at the start),
-//                       tcgen05.mma from one thread;
+//   gather warps 0..7 : two groups of four on alternate tiles, thread t of a group builds
+//                       pixel rows t (+ 128); a group's first thread reloads each staged-row
+//                       buffer it has read with the rows of its tile nhalo ahead (up to
+//                       eight: a tile's own work is shorter than the latency of its load;
+//                       the first round is issued at the start);
+//   warp 8            : tensor-memory allocation, tcgen05.mma from one thread;
 //   warps 9..16       : epilogue, two warps per lane quarter (each half of the columns):
 //                       tcgen05.ld, + bias, one rounding to bf16, 16-byte writes into
 //                       the output image (64-pixel parts, 128-byte swizzled), then one TMA
@@ -227,6 +228,14 @@ __global__ void __launch_bounds__(kGtThreads, 1) gather_t_kernel(const __grid_co
         // reduction's zero padding
         const int crow = p.C * p.R;
         const int bww = p.BW / 2;                   // 32-bit words per staged row (BW is even)
+        // Once the group has read a staged-row buffer, its first thread reloads it with the
+        // rows of the group's tile nhalo ahead (nhalo is even, so a buffer serves one group
+        // and has one issuer).  last[k]: the tile count of the last load into buffer k.
+        const bool lead_warp = warp % (kGtProd / 2) == 0;
+        int last[kGtMaxHalo];
+        for (int k = 0; k < kGtMaxHalo; ++k)
+            last[k] = (k < p.nhalo && k % 2 == grp && !p.starve &&
+                       blockIdx.x + k * static_cast<int>(gridDim.x) < p.n_mtiles) ? k : -1;
         int li = grp;
         for (int t = blockIdx.x + grp * static_cast<int>(gridDim.x); t < p.n_mtiles;
              t += 2 * static_cast<int>(gridDim.x), li += 2) {
@@ -236,7 +245,8 @@ __global__ void __launch_bounds__(kGtThreads, 1) gather_t_kernel(const __grid_co
             const uint32_t hph = static_cast<uint32_t>(li / p.nhalo) & 1u;
             const bool ok = mbar_wait(&sb.b_empty[b], ph ^ 1u, wd, kDevTimeoutEmpty) &&
                             mbar_wait(&sb.halo_full[hb], hph, wd, kDevTimeoutFull);
-            if (!__all_sync(0xffffffffu, ok)) break;
+            // the group's four warps leave together (they meet at the reload below)
+            if (!named_barrier_all(7 + grp, (kGtProd / 2) * 32, ok)) break;
             for (int row = row0; row < p.Wo; row += 128) {
                 const uint32_t *h32 = reinterpret_cast<const uint32_t *>(halo_sm + hb * halo_stride);
                 const int e0 = row * p.stride - p.pad + p.ME;   // staged column of kw = 0
@@ -275,18 +285,32 @@ __global__ void __launch_bounds__(kGtThreads, 1) gather_t_kernel(const __grid_co
             fence_proxy_async_smem();   // the tensor cores read these rows
             __syncwarp();
             if (lane == 0 && !p.starve) mbar_arrive(&sb.b_full[b]);
+            const int t2 = t + p.nhalo * static_cast<int>(gridDim.x);
+            if (!p.starve && t2 < p.n_mtiles) {
+                if (lead_warp) {
+                    named_barrier(5 + grp, (kGtProd / 2) * 32);
+                    if (lane == 0) {
+                        issue_halo(t2, hb);
+                        last[hb] = li + p.nhalo;
+                    }
+                } else {
+                    named_barrier_arrive(5 + grp, (kGtProd / 2) * 32);
+                }
+            }
         }
+        if (lead_warp && lane == 0 && *wd.abort)   // let this group's loads still in flight land
+            for (int k = 0; k < p.nhalo; ++k)
+                if (last[k] >= 0)
+                    gt_wait_quiet(&sb.halo_full[k], static_cast<uint32_t>(last[k] / p.nhalo) & 1u, wd.timeout_ns);
     } else if (warp == kGtMma) {
         // ------------------------------------------- loads and tensor-core issue ---
         if (lane == 0) {
             const uint32_t idesc = instr_desc(1u, 128, static_cast<uint32_t>(tpix));
             const uint32_t a_addr = smem_addr(a_sm);
             const int ksteps = nchunks / 2;       // 32 bytes of k per instruction
-            // loads issued so far per staged-row buffer (the first round at the start)
-            int issued[kGtMaxHalo] = {};
-            if (!p.starve)
-                for (int k = 0; k < p.nhalo; ++k)
-                    issued[k] = blockIdx.x + k * static_cast<int>(gridDim.x) < p.n_mtiles ? 1 : 0;
+            // descriptors' fields but the start address, set once (the issue of a tile's
+            // products is on its critical path)
+            const uint64_t bd0 = smem_desc(0u, 128, sbo, kSwNone);
             bool ok = !*wd.abort;
             if (a_tmem && !mbar_wait(&sb.a_tm_ready, 0, wd, kDevTimeoutFull)) ok = false;
             tc_fence_after_sync();
@@ -296,49 +320,42 @@ __global__ void __launch_bounds__(kGtThreads, 1) gather_t_kernel(const __grid_co
                 bulk_load(a_sm, p.w_image, img_bytes, &sb.a_ready);
             }
             if (!a_tmem && rt == 1 && !mbar_wait(&sb.a_ready, 0, wd, kDevTimeoutFull)) ok = false;
-            int li = 0;
+            int li = 0, ab = 0;
+            uint32_t aph = 0;                     // accumulator ab's phase
             for (int t = blockIdx.x; ok && t < p.n_mtiles; t += gridDim.x, ++li) {
                 const int b = li & 1;
                 const uint32_t ph = static_cast<uint32_t>(li >> 1) & 1u;
-                const int ab = li % p.nacc;
-                const uint32_t aph = static_cast<uint32_t>(li / p.nacc) & 1u;
                 if (!mbar_wait(&sb.acc_empty[ab], aph ^ 1u, wd, kDevTimeoutAccEmpty) ||
                     !mbar_wait(&sb.b_full[b], ph, wd, kDevTimeoutFull)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after_sync();
-                // the gather warps are done with this tile's staged rows: their buffer takes
-                // the tile nhalo ahead
-                const int t2 = t + p.nhalo * static_cast<int>(gridDim.x);
-                if (!p.starve && t2 < p.n_mtiles) {
-                    issue_halo(t2, li % p.nhalo);
-                    ++issued[li % p.nhalo];
-                }
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(ab * tpix);
                 const uint32_t b_addr = smem_addr(b_sm + b * b_stride);
                 if (a_tmem) {
                     for (int ks = 0; ks < ksteps; ++ks)   // 16 k = 8 columns of A per instruction
                         mma_bf16_tmem_a(d_tmem, tmem_base + a_col + static_cast<uint32_t>(ks) * 8u,
-                                        smem_desc(b_addr + static_cast<uint32_t>(ks) * 256u, 128, sbo, kSwNone),
-                                        idesc, ks > 0 ? 1u : 0u);
+                                        bd0 | ((b_addr + static_cast<uint32_t>(ks) * 256u) >> 4), idesc,
+                                        ks > 0 ? 1u : 0u);
                 } else {
                     for (int ks = 0; ks < ksteps; ++ks) {
                         const uint32_t off = static_cast<uint32_t>(ks) * 256u;  // two 16-byte k chunks
-                        mma_bf16(d_tmem, smem_desc(a_addr + off, 128, sbo, kSwNone),
-                                 smem_desc(b_addr + off, 128, sbo, kSwNone), idesc, ks > 0 ? 1u : 0u);
+                        mma_bf16(d_tmem, bd0 | ((a_addr + off) >> 4), bd0 | ((b_addr + off) >> 4), idesc,
+                                 ks > 0 ? 1u : 0u);
                     }
                 }
                 mma_commit(&sb.b_empty[b]);
                 mma_commit(&sb.acc_full[ab]);
+                if (++ab == p.nacc) {
+                    ab = 0;
+                    aph ^= 1u;
+                }
             }
             if (!ok || *wd.abort) {
                 mma_commit(&sb.drain);
                 gt_wait_quiet(&sb.drain, 0, wd.timeout_ns);
                 if (!p.starve && ((rt == 1 && !a_tmem) || a_staged)) gt_wait_quiet(&sb.a_ready, 0, wd.timeout_ns);
-                for (int hb = 0; hb < p.nhalo; ++hb)  // let the staged-row loads still in flight land
-                    if (issued[hb] > 0)
-                        gt_wait_quiet(&sb.halo_full[hb], static_cast<uint32_t>(issued[hb] - 1) & 1u, wd.timeout_ns);
             }
         }
         __syncwarp();
@@ -524,7 +541,7 @@ cudaError_t launch_gather_t(const GatherParams &p, int grid, size_t smem, cudaSt
     if (!rt_ok || p.Kpad > 8 * kGtMaxChunks || p.Kpad % 16 != 0 || p.kt > 8 * kGtMaxChunks || p.kt % 16 != 0 ||
         p.tpix % 16 != 0 || p.tpix > 256 || p.Wo > 256 || p.Wo % 8 != 0 || p.Cout > p.BN ||
         p.C * p.R > kGtMaxChunks || 2 * p.tpix > static_cast<int>(p.tmem_cols) || p.dilation != 1 ||
-        p.nhalo < 2 || p.nhalo > kGtMaxHalo || p.nacc < 2 || p.nacc > kGtMaxAcc ||
+        p.nhalo < 2 || p.nhalo > kGtMaxHalo || p.nhalo % 2 != 0 || p.nacc < 2 || p.nacc > kGtMaxAcc ||
         p.nacc * p.tpix + (p.a_tmem ? p.kt / 2 : 0) > static_cast<int>(p.tmem_cols) ||
         (p.a_tmem && p.tpix < 64) || (p.tma_out && (p.nout < 1 || p.nout > 2)) ||
         (!p.tma_out && p.nout != 1))
