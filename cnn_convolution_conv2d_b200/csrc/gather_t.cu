@@ -87,6 +87,12 @@ __device__ __forceinline__ uint32_t gt_core(int m, int j, uint32_t sbo) {
     return static_cast<uint32_t>(m >> 3) * sbo + static_cast<uint32_t>(j) * 128u + static_cast<uint32_t>(m & 7) * 16u;
 }
 
+// Arrival on hardware barrier `id` without waiting: the other side of a named_barrier that
+// one warp waits on while the rest of its group go on.
+__device__ __forceinline__ void gt_barrier_arrive(int id, int count) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 __device__ __forceinline__ void gt_wait_quiet(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
     const uint64_t start = globaltimer_ns();
     while (!mbar_try_wait(bar, parity)) {
@@ -294,7 +300,7 @@ __global__ void __launch_bounds__(kGtThreads, 1) gather_t_kernel(const __grid_co
                         last[hb] = li + p.nhalo;
                     }
                 } else {
-                    named_barrier_arrive(5 + grp, (kGtProd / 2) * 32);
+                    gt_barrier_arrive(5 + grp, (kGtProd / 2) * 32);
                 }
             }
         }

@@ -286,12 +286,6 @@ __device__ __forceinline__ void named_barrier(int id, int count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
-// Arrival on hardware barrier `id` without waiting: the other side of a named_barrier
-// that one warp waits on while the rest of its group go on.
-__device__ __forceinline__ void named_barrier_arrive(int id, int count) {
-    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-
 // Barrier over `count` threads on hardware barrier `id` that also returns whether
 // `pred` held in every one of them: threads that must leave a loop together take the
 // decision from it.
