@@ -21,8 +21,10 @@
 //                bytes of channels; for stride 1 and unit dilation it reads each input row
 //                once into a register window of R + Kw - 1 pixels and reuses it for every
 //                filter column.  Weights of the tile's channels are kept per warp in shared
-//                memory; accumulation is fp32, bias is added in fp32 and the result is
-//                rounded once to the output type and stored with 16-byte stores (NHWC).
+//                memory; accumulation is fp32 (bf16 inputs by mixed-precision FMAs straight
+//                from their packed words, fp32 by paired FMAs), bias is added in fp32 and
+//                the result is rounded once to the output type and stored with 16-byte
+//                stores (NHWC).
 // Every wait is bounded (see ptx.cuh).
 #include <cuda_bf16.h>
 
@@ -85,6 +87,19 @@ __device__ __forceinline__ void unpair(uint64_t v, float &lo, float &hi) {
     asm("mov.b64 {%0, %1}, %2;" : "=r"(a), "=r"(b) : "l"(v));
     lo = __uint_as_float(a);
     hi = __uint_as_float(b);
+}
+
+// acc0 += lo(x) * lo(w), acc1 += hi(x) * hi(w) on the bf16 halves of two 32-bit words:
+// sm_100's mixed-precision fma (bf16 operands, fp32 addend and result; the product of two
+// bf16 values is exact in fp32, so each is one rounding, as after converting them).
+__device__ __forceinline__ void fma_bf16x2_f32(float &acc0, float &acc1, uint32_t x, uint32_t w) {
+    asm("{\n\t.reg .b16 x0, x1, w0, w1;\n\t"
+        "mov.b32 {x0, x1}, %2;\n\t"
+        "mov.b32 {w0, w1}, %3;\n\t"
+        "fma.rn.f32.bf16 %0, x0, w0, %0;\n\t"
+        "fma.rn.f32.bf16 %1, x1, w1, %1;\n\t}"
+        : "+f"(acc0), "+f"(acc1)
+        : "r"(x), "r"(w));
 }
 
 // 16 bytes of channels as kV/2 fp32 pairs (bf16: each 32-bit word holds channels 2i, 2i+1).
@@ -377,8 +392,9 @@ __global__ void __launch_bounds__(kDwThreads, 1) dw_kernel(const __grid_constant
             }
             if constexpr (kKW > 0) {
                 // Stride 1, unit dilation, kKW x kKW: every filter row reads a window of
-                // kR + kKW - 1 input pixels once; products in fp32 pairs started from the
-                // bias.  A tile row holds two groups of kR pixels (TW = 2*kR).
+                // kR + kKW - 1 input pixels once; products accumulate in fp32 started from
+                // the bias (bf16: mixed-precision FMAs on the raw words; fp32: paired FMAs).
+                // A tile row holds two groups of kR pixels (TW = 2*kR).
                 constexpr int kP = kV / 2;
                 for (int it = tid; it < items; it += 32 * kDwComputeWarps) {
                     const int cg = it & 7, pg = it >> 3;
@@ -387,36 +403,72 @@ __global__ void __launch_bounds__(kDwThreads, 1) dw_kernel(const __grid_constant
                     const int ow0 = t.tw * p.TW + px0;
                     const int c = t.chunk * kCC + cg * kV;
                     if (oh >= p.Ho || ow0 >= p.Wo || c >= p.C) continue;
-                    uint64_t accp[kR][kP];
-                    {
+                    const uint8_t *rp0 = stg + (static_cast<uint32_t>(py) * p.IW + px0) * kDwRowBytes + cg * 16;
+                    const uint8_t *wp0 = wsm + cg * 16;
+                    float o_all[kR][kV];
+                    if constexpr (!kF32) {
+                        // bf16: the window's words as they are, mixed-precision FMAs into
+                        // fp32 accumulators started from the bias (no unpacking)
                         const float *bq = bsm + cg * kV;
-                        uint64_t b2[kP];
-#pragma unroll
-                        for (int v = 0; v < kP; ++v) b2[v] = pair(__float_as_uint(bq[2 * v]), __float_as_uint(bq[2 * v + 1]));
 #pragma unroll
                         for (int r = 0; r < kR; ++r)
 #pragma unroll
-                            for (int v = 0; v < kP; ++v) accp[r][v] = b2[v];
-                    }
-                    const uint8_t *rp0 = stg + (static_cast<uint32_t>(py) * p.IW + px0) * kDwRowBytes + cg * 16;
-                    const uint8_t *wp0 = wsm + cg * 16;
+                            for (int v = 0; v < kV; ++v) o_all[r][v] = bq[v];
 #pragma unroll
-                    for (int kh = 0; kh < kKW; ++kh) {
-                        const uint8_t *rp = rp0 + static_cast<uint32_t>(kh) * p.IW * kDwRowBytes;
-                        const uint8_t *wp = wp0 + kh * kKW * kDwRowBytes;
-                        uint64_t win[kR + kKW - 1][kP];
+                        for (int kh = 0; kh < kKW; ++kh) {
+                            const uint8_t *rp = rp0 + static_cast<uint32_t>(kh) * p.IW * kDwRowBytes;
+                            const uint8_t *wp = wp0 + kh * kKW * kDwRowBytes;
+                            uint4 win[kR + kKW - 1];
 #pragma unroll
-                        for (int j = 0; j < kR + kKW - 1; ++j)
-                            unpack16_pairs<kF32>(*reinterpret_cast<const uint4 *>(rp + j * kDwRowBytes), win[j]);
+                            for (int j = 0; j < kR + kKW - 1; ++j)
+                                win[j] = *reinterpret_cast<const uint4 *>(rp + j * kDwRowBytes);
 #pragma unroll
-                        for (int kw = 0; kw < kKW; ++kw) {
-                            uint64_t wv[kP];
-                            unpack16_pairs<kF32>(*reinterpret_cast<const uint4 *>(wp + kw * kDwRowBytes), wv);
+                            for (int kw = 0; kw < kKW; ++kw) {
+                                const uint4 wv = *reinterpret_cast<const uint4 *>(wp + kw * kDwRowBytes);
+#pragma unroll
+                                for (int r = 0; r < kR; ++r) {
+                                    const uint4 xv = win[r + kw];
+                                    fma_bf16x2_f32(o_all[r][0], o_all[r][1], xv.x, wv.x);
+                                    fma_bf16x2_f32(o_all[r][2], o_all[r][3], xv.y, wv.y);
+                                    fma_bf16x2_f32(o_all[r][4], o_all[r][5], xv.z, wv.z);
+                                    fma_bf16x2_f32(o_all[r][6], o_all[r][7], xv.w, wv.w);
+                                }
+                            }
+                        }
+                    } else {
+                        uint64_t accp[kR][kP];
+                        {
+                            const float *bq = bsm + cg * kV;
+                            uint64_t b2[kP];
+#pragma unroll
+                            for (int v = 0; v < kP; ++v) b2[v] = pair(__float_as_uint(bq[2 * v]), __float_as_uint(bq[2 * v + 1]));
 #pragma unroll
                             for (int r = 0; r < kR; ++r)
 #pragma unroll
-                                for (int v = 0; v < kP; ++v) fma2(accp[r][v], win[r + kw][v], wv[v]);
+                                for (int v = 0; v < kP; ++v) accp[r][v] = b2[v];
                         }
+#pragma unroll
+                        for (int kh = 0; kh < kKW; ++kh) {
+                            const uint8_t *rp = rp0 + static_cast<uint32_t>(kh) * p.IW * kDwRowBytes;
+                            const uint8_t *wp = wp0 + kh * kKW * kDwRowBytes;
+                            uint64_t win[kR + kKW - 1][kP];
+#pragma unroll
+                            for (int j = 0; j < kR + kKW - 1; ++j)
+                                unpack16_pairs<kF32>(*reinterpret_cast<const uint4 *>(rp + j * kDwRowBytes), win[j]);
+#pragma unroll
+                            for (int kw = 0; kw < kKW; ++kw) {
+                                uint64_t wv[kP];
+                                unpack16_pairs<kF32>(*reinterpret_cast<const uint4 *>(wp + kw * kDwRowBytes), wv);
+#pragma unroll
+                                for (int r = 0; r < kR; ++r)
+#pragma unroll
+                                    for (int v = 0; v < kP; ++v) fma2(accp[r][v], win[r + kw][v], wv[v]);
+                            }
+                        }
+#pragma unroll
+                        for (int r = 0; r < kR; ++r)
+#pragma unroll
+                            for (int v = 0; v < kP; ++v) unpair(accp[r][v], o_all[r][2 * v], o_all[r][2 * v + 1]);
                     }
                     // epilogue: one rounding, store (the bias is already in)
                     const bool whole = c + kV <= p.C && p.vec_ok;
@@ -424,10 +476,7 @@ __global__ void __launch_bounds__(kDwThreads, 1) dw_kernel(const __grid_constant
 #pragma unroll
                     for (int r = 0; r < kR; ++r) {
                         if (ow0 + r >= p.Wo) break;
-                        float o[kV];
-#pragma unroll
-                        for (int v = 0; v < kP; ++v) unpair(accp[r][v], o[2 * v], o[2 * v + 1]);
-                        dw_store<kF32, kV>(p, pix0 + r, static_cast<size_t>(t.n), oh, ow0 + r, c, o, whole);
+                        dw_store<kF32, kV>(p, pix0 + r, static_cast<size_t>(t.n), oh, ow0 + r, c, o_all[r], whole);
                     }
                 }
             }
