@@ -320,15 +320,30 @@ __global__ void __launch_bounds__(kDwThreads, 1) dw_kernel(const __grid_constant
                             const uint8_t *rp = stg + static_cast<size_t>(row) * p.IW * kDwRowBytes + cg * 16;
                             const uint8_t *wp = wsm + kh * p.Kw * kDwRowBytes + cg * 16;
                             for (int kw = 0; kw < p.Kw; ++kw) {
-                                float wv[kV];
-                                unpack16<kF32>(*reinterpret_cast<const uint4 *>(wp + kw * kDwRowBytes), wv);
+                                if constexpr (kF32) {
+                                    float wv[kV];
+                                    unpack16<kF32>(*reinterpret_cast<const uint4 *>(wp + kw * kDwRowBytes), wv);
     #pragma unroll
-                                for (int r = 0; r < kR; ++r) {
-                                    const int col = (px0 + r) * p.stride + kw * p.dilation;
-                                    float xv[kV];
-                                    unpack16<kF32>(*reinterpret_cast<const uint4 *>(rp + col * kDwRowBytes), xv);
+                                    for (int r = 0; r < kR; ++r) {
+                                        const int col = (px0 + r) * p.stride + kw * p.dilation;
+                                        float xv[kV];
+                                        unpack16<kF32>(*reinterpret_cast<const uint4 *>(rp + col * kDwRowBytes), xv);
     #pragma unroll
-                                    for (int v = 0; v < kV; ++v) acc[r][v] = fmaf(xv[v], wv[v], acc[r][v]);
+                                        for (int v = 0; v < kV; ++v) acc[r][v] = fmaf(xv[v], wv[v], acc[r][v]);
+                                    }
+                                } else {
+                                    // bf16: mixed-precision FMAs on the packed words (the same
+                                    // exact products and roundings as converting them first)
+                                    const uint4 wq = *reinterpret_cast<const uint4 *>(wp + kw * kDwRowBytes);
+    #pragma unroll
+                                    for (int r = 0; r < kR; ++r) {
+                                        const int col = (px0 + r) * p.stride + kw * p.dilation;
+                                        const uint4 xq = *reinterpret_cast<const uint4 *>(rp + col * kDwRowBytes);
+                                        fma_bf16x2_f32(acc[r][0], acc[r][1], xq.x, wq.x);
+                                        fma_bf16x2_f32(acc[r][2], acc[r][3], xq.y, wq.y);
+                                        fma_bf16x2_f32(acc[r][4], acc[r][5], xq.z, wq.z);
+                                        fma_bf16x2_f32(acc[r][6], acc[r][7], xq.w, wq.w);
+                                    }
                                 }
                             }
                         }
